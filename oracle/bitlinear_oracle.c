@@ -1,0 +1,233 @@
+/*
+ * bitlinear_oracle.c -- plain CPU statement of the BitNet b1.58 BitLinear
+ * W1.58A8 matmul.
+ *
+ * TEST INFRASTRUCTURE. Only the tests, the smoke check and the CPU-baseline
+ * leg of the benchmark may load or run this code. It shares nothing with the
+ * CUDA library (no headers, no helpers, no tables) and the library never
+ * calls it. It is written to be read against the pages, not to be fast:
+ * single-threaded loops, fp32 where the pages' PyTorch listing computes in
+ * fp32, a double accumulator for the weight mean.
+ *
+ * What it follows (page "BitNet b1.58 2B4T Guide: Scaling Native 1-Bit LLMs"):
+ *   - section "Ternary Weight Quantization: absmean Scaling": gamma is the mean
+ *     of |W| over the whole d_out x d_in matrix, and each weight becomes
+ *     Clip(Round(W / gamma), -1, 1);
+ *   - section "8-Bit Activation Quantization: absmax Scaling": per token,
+ *     beta = max_j |x_j| and x~ = Clip(Round(x * Q_b / beta)), Q_b = 127;
+ *   - section "Matrix Multiplication as Pure Integer Addition":
+ *     y = (x~ W~^T) * beta * gamma / Q_b, the product being an integer sum;
+ *   - the page's PyTorch listing (WeightQuantFunction.forward,
+ *     quantize_activations_int8, BitLinear.forward), which fixes what the
+ *     formulas leave open: the epsilon is a clamp(min=1e-5) of gamma and beta,
+ *     Round is torch.round (ties to even), the activation scale is applied as
+ *     x * (127 / beta), the activation clip range is [-128, 127] and the
+ *     output scale is (beta * gamma) / 127.
+ * Readings taken where the pages are silent (all listed in the design notes):
+ *   - arithmetic is IEEE fp32 with round-to-nearest-even, bf16 inputs are
+ *     widened to fp32 exactly, and the output is rounded once to bf16 (RNE);
+ *   - the |W| sum is accumulated in double and divided once, then cast to fp32;
+ *   - one gamma per weight matrix (the formula's double sum over i and j).
+ *
+ * The packed 2-bit layout (oracle_pack_codes) is the storage format the
+ * library's packer must produce; it is written here from its specification
+ * (see the layout comment above oracle_pack_codes), not from the library.
+ *
+ * Build: gcc -O2 -std=c11 -fPIC -shared -ffp-contract=off -fno-fast-math
+ */
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+
+/* clamp(min=1e-5) applied to gamma and beta in the page's listing */
+static const float ORACLE_EPS = 1e-5f;
+/* Q_b = 2^(b-1) with b = 8 bits, used as 127 by the page */
+static const float ORACLE_QB = 127.0f;
+
+/* ---------------------------------------------------------------- weights */
+
+/* gamma = max(mean_{i,j} |W_ij|, 1e-5) over a row-major [N][K] fp32 matrix.
+ * Section "Ternary Weight Quantization: absmean Scaling" (the double sum over
+ * d_out and d_in divided by d_out * d_in); the clamp is the listing's. */
+float oracle_absmean_gamma(const float *W, int64_t N, int64_t K)
+{
+    const int64_t count = N * K;
+    if (count <= 0)
+        return ORACLE_EPS;
+    double sum = 0.0;
+    for (int64_t i = 0; i < count; ++i)
+        sum += fabs((double)W[i]);
+    float gamma = (float)(sum / (double)count);
+    if (gamma < ORACLE_EPS)
+        gamma = ORACLE_EPS;
+    return gamma;
+}
+
+/* W~ = Clip(Round(W / gamma), -1, 1) elementwise, Round = ties-to-even.
+ * Same section; the fp32 division is the listing's weight / gamma. */
+void oracle_ternarize(const float *W, int64_t N, int64_t K, float gamma,
+                      int8_t *Wq)
+{
+    const int64_t count = N * K;
+    for (int64_t i = 0; i < count; ++i) {
+        float q = rintf(W[i] / gamma);
+        if (q > 1.0f)
+            q = 1.0f;
+        if (q < -1.0f)
+            q = -1.0f;
+        Wq[i] = (int8_t)q;
+    }
+}
+
+/* ------------------------------------------------------------ activations */
+
+/* Exact widening of bf16 bit patterns to fp32 (bf16 is the top half of an
+ * IEEE single). */
+void oracle_bf16_to_f32(const uint16_t *in, int64_t n, float *out)
+{
+    for (int64_t i = 0; i < n; ++i) {
+        uint32_t bits = (uint32_t)in[i] << 16;
+        memcpy(&out[i], &bits, sizeof(float));
+    }
+}
+
+/* Per-token absmax int8 quantisation of a row-major [M][K] fp32 matrix.
+ * beta_m = max(max_k |x_mk|, 1e-5); x~_mk = Clip(Round(x_mk * (127 / beta_m)),
+ * -128, 127). Section "8-Bit Activation Quantization: absmax Scaling" and the
+ * listing's quantize_activations_int8. */
+void oracle_quant_act(const float *x, int64_t M, int64_t K, int8_t *xq,
+                      float *beta)
+{
+    for (int64_t m = 0; m < M; ++m) {
+        const float *row = x + m * K;
+        float b = 0.0f;
+        for (int64_t k = 0; k < K; ++k) {
+            float a = fabsf(row[k]);
+            if (a > b)
+                b = a;
+        }
+        if (b < ORACLE_EPS)
+            b = ORACLE_EPS;
+        const float scale = ORACLE_QB / b;
+        for (int64_t k = 0; k < K; ++k) {
+            float q = rintf(row[k] * scale);
+            if (q > 127.0f)
+                q = 127.0f;
+            if (q < -128.0f)
+                q = -128.0f;
+            xq[m * K + k] = (int8_t)q;
+        }
+        beta[m] = b;
+    }
+}
+
+/* ------------------------------------------------------- integer product */
+
+/* acc_mn = sum_k x~_mk * W~_nk with x~ [M][K] and W~ [N][K], both row-major.
+ * Section "Matrix Multiplication as Pure Integer Addition": the contraction
+ * over d_in with W stored d_out x d_in, i.e. y = x W^T. */
+void oracle_matmul_i32(const int8_t *xq, const int8_t *Wq, int64_t M,
+                       int64_t N, int64_t K, int32_t *acc)
+{
+    for (int64_t m = 0; m < M; ++m) {
+        for (int64_t n = 0; n < N; ++n) {
+            int64_t s = 0;
+            for (int64_t k = 0; k < K; ++k)
+                s += (int64_t)xq[m * K + k] * (int64_t)Wq[n * K + k];
+            acc[m * N + n] = (int32_t)s;
+        }
+    }
+}
+
+/* The same sum for a list of (m, n) pairs only, so that large shapes can be
+ * checked on sampled outputs. */
+void oracle_matmul_i32_pairs(const int8_t *xq, const int8_t *Wq, int64_t K,
+                             const int64_t *ms, const int64_t *ns,
+                             int64_t count, int32_t *acc)
+{
+    for (int64_t i = 0; i < count; ++i) {
+        const int8_t *a = xq + ms[i] * K;
+        const int8_t *w = Wq + ns[i] * K;
+        int64_t s = 0;
+        for (int64_t k = 0; k < K; ++k)
+            s += (int64_t)a[k] * (int64_t)w[k];
+        acc[i] = (int32_t)s;
+    }
+}
+
+/* ----------------------------------------------------------------- rescale */
+
+/* fp32 -> bf16 with round-to-nearest, ties to even, on the bit pattern:
+ * keep the upper 16 bits and look at the 16 discarded ones. More than half an
+ * ulp rounds up, exactly half rounds to the even kept value. A carry out of
+ * the mantissa bumps the exponent, which is the correct rounded result and
+ * turns the largest finite values into infinity when they round past it.
+ * NaN stays NaN (quiet bit forced). */
+uint16_t oracle_f32_to_bf16(float f)
+{
+    uint32_t u;
+    memcpy(&u, &f, sizeof(u));
+    if ((u & 0x7f800000u) == 0x7f800000u && (u & 0x007fffffu) != 0u)
+        return (uint16_t)((u >> 16) | 0x0040u);
+    uint32_t kept = u >> 16;
+    uint32_t dropped = u & 0xffffu;
+    if (dropped > 0x8000u || (dropped == 0x8000u && (kept & 1u)))
+        kept += 1u;
+    return (uint16_t)kept;
+}
+
+void oracle_f32_to_bf16_array(const float *in, int64_t n, uint16_t *out)
+{
+    for (int64_t i = 0; i < n; ++i)
+        out[i] = oracle_f32_to_bf16(in[i]);
+}
+
+/* y_mn = bf16( float(acc_mn) * ((beta_m * gamma) / 127) ), fp32 arithmetic.
+ * Section "Matrix Multiplication as Pure Integer Addition" (rescale by
+ * beta * gamma / Q_b) and the listing's BitLinear.forward step 5. */
+void oracle_rescale_bf16(const int32_t *acc, const float *beta, float gamma,
+                         int64_t M, int64_t N, uint16_t *y)
+{
+    for (int64_t m = 0; m < M; ++m) {
+        const float s = (beta[m] * gamma) / ORACLE_QB;
+        for (int64_t n = 0; n < N; ++n)
+            y[m * N + n] = oracle_f32_to_bf16((float)acc[m * N + n] * s);
+    }
+}
+
+/* ------------------------------------------------------------ 2-bit layout */
+
+/* Packed ternary storage (the "2-bit nibbles" of the bitnet.xin guide, section
+ * "Core Architecture"; the layout itself is this library's own):
+ *   - the matrix is N rows of K/4 bytes, row n starting at byte n * K / 4;
+ *   - the 32-bit little-endian word w of a row holds the 16 weights with
+ *     k in [16w, 16w + 16);
+ *   - weight k = 16w + 4j + b (j, b in 0..3) sits in bits 8b + 2j and
+ *     8b + 2j + 1 of that word, as the code W~ + 1 (0, 1 or 2).
+ * Returns 0, or -1 when K is not a multiple of 16 or a weight is not ternary. */
+int oracle_pack_codes(const int8_t *Wq, int64_t N, int64_t K, uint8_t *packed)
+{
+    if (K % 16 != 0)
+        return -1;
+    const int64_t words_per_row = K / 16;
+    for (int64_t n = 0; n < N; ++n) {
+        for (int64_t w = 0; w < words_per_row; ++w) {
+            uint32_t word = 0;
+            for (int j = 0; j < 4; ++j) {
+                for (int b = 0; b < 4; ++b) {
+                    const int64_t k = 16 * w + 4 * j + b;
+                    const int v = Wq[n * K + k];
+                    if (v < -1 || v > 1)
+                        return -1;
+                    word |= (uint32_t)(v + 1) << (8 * b + 2 * j);
+                }
+            }
+            uint8_t *dst = packed + n * (K / 4) + 4 * w;
+            dst[0] = (uint8_t)(word & 0xffu);
+            dst[1] = (uint8_t)((word >> 8) & 0xffu);
+            dst[2] = (uint8_t)((word >> 16) & 0xffu);
+            dst[3] = (uint8_t)((word >> 24) & 0xffu);
+        }
+    }
+    return 0;
+}

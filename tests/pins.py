@@ -1,0 +1,362 @@
+"""Pins for the CPU oracle: checks against facts fixed by the pages and by
+mathematics, independent of the oracle's own code.
+
+Each ``pin_*`` function takes an ``oracle.Oracle`` and raises AssertionError
+when the oracle disagrees with the pinned fact. ``tests/test_oracle_pins.py``
+runs them on the oracle; ``tests/test_oracle_mutants.py`` runs them on copies
+of the oracle with a planted mistake and expects at least one to fail.
+
+What pins what (pages: "BitNet b1.58 2B4T Guide: Scaling Native 1-Bit LLMs"
+unless stated):
+  * hand-worked examples under tests/golden/ (sections "Ternary Weight
+    Quantization", "8-Bit Activation Quantization", "Matrix Multiplication as
+    Pure Integer Addition");
+  * brute force of the add/ignore/subtract form of the product (same section,
+    the sum over W~ = +1 minus the sum over W~ = -1), written as Python loops;
+  * library routines: torch.nn.functional.linear in float64 (exact for these
+    integer sums), torch's fp32 -> bf16 conversion, numpy's float64 mean;
+  * closed forms and invariants: constant and zero inputs, identity weights,
+    +-a weights, the Gaussian zero fraction (about 31%, which the bitnet.xin
+    guide's "Core Architecture" section quotes as about 32% zero entries),
+    |x~| <= 127 with the per-token maximum reaching 127, the rounding bound
+    |x~ - x*127/beta| <= 1/2, invariance under power-of-two scaling, and the
+    bf16 rounding bound of the output.
+"""
+from __future__ import annotations
+
+import math
+import os
+
+import numpy as np
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+
+
+# ------------------------------------------------------------------ fixtures
+
+def _parse_values(text: str):
+    rows = [r.split() for r in text.split(";")]
+    return [[float(v) for v in r] for r in rows if r]
+
+
+def load_golden(name: str) -> dict:
+    out = {}
+    with open(os.path.join(GOLDEN, name)) as f:
+        for line in f:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            key, _, val = line.partition("=")
+            out[key.strip()] = _parse_values(val)
+    return out
+
+
+def load_pack_cases() -> list:
+    cases = []
+    with open(os.path.join(GOLDEN, "pack_words.txt")) as f:
+        for line in f:
+            line = line.strip()
+            if not line.startswith("case"):
+                continue
+            head, _, rest = line.partition(":")
+            wq_part, bytes_part = rest.split(";")
+            wq = [int(v) for v in wq_part.split("=")[1].split()]
+            by = [int(v, 16) for v in bytes_part.split("=")[1].split()]
+            cases.append((head.split()[1], wq, by))
+    return cases
+
+
+def _f32(v):
+    return np.asarray(v, dtype=np.float32)
+
+
+def _bf16_value(bits: np.ndarray) -> np.ndarray:
+    return (bits.astype(np.uint32) << 16).view(np.float32)
+
+
+# ---------------------------------------------------------------- the pins
+
+def pin_hand_example(orc):
+    g = load_golden("hand_example.txt")
+    W = _f32(g["W"])
+    x = _f32(g["x"])
+    r = orc.forward(x, W)
+    gamma_ref = np.float32(g["gamma"][0][0])
+    assert abs(float(r["gamma"]) - float(gamma_ref)) <= 2 * np.spacing(gamma_ref), r["gamma"]
+    np.testing.assert_array_equal(r["Wq"], np.array(g["Wq"], dtype=np.int8))
+    assert float(r["beta"][0]) == g["beta"][0][0]
+    np.testing.assert_array_equal(r["xq"], np.array(g["xq"], dtype=np.int8))
+    np.testing.assert_array_equal(r["acc"], np.array(g["acc"], dtype=np.int32))
+    np.testing.assert_array_equal(_bf16_value(r["y"]), _f32(g["y"]))
+
+
+def pin_weight_ties_even(orc):
+    g = load_golden("weight_ties.txt")
+    W = _f32(g["W"])
+    gamma = orc.absmean_gamma(W)
+    assert float(gamma) == g["gamma"][0][0]
+    np.testing.assert_array_equal(orc.ternarize(W, gamma),
+                                  np.array(g["Wq"], dtype=np.int8))
+
+
+def pin_activation_ties_even(orc):
+    g = load_golden("activation_ties.txt")
+    xq, beta = orc.quant_act(_f32(g["x"]))
+    assert float(beta[0]) == g["beta"][0][0]
+    np.testing.assert_array_equal(xq, np.array(g["xq"], dtype=np.int8))
+
+
+def pin_pack_words(orc):
+    for name, wq, by in load_pack_cases():
+        got = orc.pack_codes(np.array([wq], dtype=np.int8))
+        assert got.tolist() == [by], (name, got.tolist(), by)
+
+
+def decode_packed_spec(packed: np.ndarray, K: int) -> np.ndarray:
+    """Independent decoder of the 2-bit layout, bit by bit from its spec:
+    byte 4w + q of a row is bits 8q..8q+7 of word w; weight k = 16w + 4j + b
+    is the 2-bit field at bit 8b + 2j of that word, minus one."""
+    N = packed.shape[0]
+    out = np.zeros((N, K), dtype=np.int8)
+    for n in range(N):
+        for w in range(K // 16):
+            word = 0
+            for q in range(4):
+                word |= int(packed[n, 4 * w + q]) << (8 * q)
+            for j in range(4):
+                for b in range(4):
+                    code = (word >> (8 * b + 2 * j)) & 3
+                    assert code != 3
+                    out[n, 16 * w + 4 * j + b] = code - 1
+    return out
+
+
+def pin_pack_roundtrip(orc):
+    r = np.random.Generator(np.random.PCG64(7))
+    Wq = r.integers(-1, 2, size=(5, 64), dtype=np.int8)
+    packed = orc.pack_codes(Wq)
+    assert packed.shape == (5, 16)
+    np.testing.assert_array_equal(decode_packed_spec(packed, 64), Wq)
+
+
+def pin_constant_token(orc):
+    for c in (0.75, -3.0, 1e-3):
+        x = np.full((1, 40), c, dtype=np.float32)
+        xq, beta = orc.quant_act(x)
+        assert float(beta[0]) == abs(np.float32(c))
+        assert np.all(xq == (127 if c > 0 else -127))
+
+
+def pin_zero_inputs(orc):
+    xq, beta = orc.quant_act(np.zeros((2, 32), dtype=np.float32))
+    assert np.all(beta == np.float32(1e-5)) and np.all(xq == 0)
+    W = np.zeros((8, 32), dtype=np.float32)
+    gamma = orc.absmean_gamma(W)
+    assert gamma == np.float32(1e-5)
+    assert np.all(orc.ternarize(W, gamma) == 0)
+    r = orc.forward(np.ones((2, 32), dtype=np.float32), W)
+    assert np.all(r["acc"] == 0) and np.all(r["y"] == 0)
+
+
+def pin_tiny_scale_epsilon(orc):
+    # |x| below the epsilon: beta is clamped to 1e-5, so x~ = x * 127 / 1e-5.
+    # 4e-6 * 127 / 1e-5 = 50.8, -2.6e-6 -> -33.02, 1e-6 -> 12.7 (no ties nearby)
+    x = _f32([[4e-6, -2.6e-6, 0.0, 1e-6]])
+    xq, beta = orc.quant_act(x)
+    assert beta[0] == np.float32(1e-5)
+    np.testing.assert_array_equal(xq[0], np.array([51, -33, 0, 13], np.int8))
+
+
+def pin_identity_weights(orc):
+    K = 48
+    W = np.eye(K, dtype=np.float32)          # mean |W| = 1/K, diagonal -> K -> clip 1
+    x = np.random.Generator(np.random.PCG64(3)).standard_normal((3, K)).astype(np.float32)
+    r = orc.forward(x, W)
+    np.testing.assert_array_equal(r["Wq"], np.eye(K, dtype=np.int8))
+    np.testing.assert_array_equal(r["acc"], r["xq"].astype(np.int32))
+
+
+def pin_plus_minus_a(orc):
+    r = np.random.Generator(np.random.PCG64(11))
+    W = np.where(r.random((16, 64)) < 0.5, -0.25, 0.25).astype(np.float32)
+    gamma = orc.absmean_gamma(W)
+    assert gamma == np.float32(0.25)
+    np.testing.assert_array_equal(orc.ternarize(W, gamma), np.sign(W).astype(np.int8))
+    Wc = np.full((3, 16), -0.125, dtype=np.float32)
+    assert orc.absmean_gamma(Wc) == np.float32(0.125)
+    assert np.all(orc.ternarize(Wc, np.float32(0.125)) == -1)
+
+
+def pin_gamma_vs_numpy_mean(orc):
+    W = np.random.Generator(np.random.PCG64(5)).standard_normal((64, 96)).astype(np.float32) * np.float32(0.02)
+    ref = np.float32(np.mean(np.abs(W.astype(np.float64))))
+    got = orc.absmean_gamma(W)
+    assert abs(float(got) - float(ref)) <= np.spacing(ref), (got, ref)
+
+
+def pin_zero_fraction(orc):
+    # Gaussian latent: zero iff |W| < gamma/2 with gamma = sigma*sqrt(2/pi), so
+    # P(0) = P(|Z| < sqrt(2/pi)/2) = erf(sqrt(2/pi)/2/sqrt(2)) ~ 0.310 and
+    # P(+1) = P(-1) ~ 0.345.
+    W = np.random.Generator(np.random.PCG64(0)).standard_normal((256, 256)).astype(np.float32) * np.float32(0.02)
+    Wq = orc.ternarize(W, orc.absmean_gamma(W))
+    p0 = math.erf(math.sqrt(2 / math.pi) / 2 / math.sqrt(2))
+    frac0 = float(np.mean(Wq == 0))
+    assert abs(frac0 - p0) < 0.01, (frac0, p0)
+    assert abs(float(np.mean(Wq == 1)) - (1 - p0) / 2) < 0.01
+    assert abs(float(np.mean(Wq == -1)) - (1 - p0) / 2) < 0.01
+    assert set(np.unique(Wq).tolist()) <= {-1, 0, 1}
+
+
+def pin_bruteforce_add_subtract(orc):
+    r = np.random.Generator(np.random.PCG64(21))
+    for (M, K, N) in ((1, 4, 1), (2, 7, 3), (4, 64, 16), (3, 33, 5)):
+        xq = r.integers(-127, 128, size=(M, K), dtype=np.int8)
+        Wq = r.integers(-1, 2, size=(N, K), dtype=np.int8)
+        acc = orc.matmul_i32(xq, Wq)
+        for m in range(M):
+            for n in range(N):
+                plus = sum(int(xq[m, k]) for k in range(K) if Wq[n, k] == 1)
+                minus = sum(int(xq[m, k]) for k in range(K) if Wq[n, k] == -1)
+                assert int(acc[m, n]) == plus - minus, (M, K, N, m, n)
+
+
+def pin_exhaustive_single_term(orc):
+    xq = np.arange(-128, 128, dtype=np.int8).reshape(256, 1)
+    Wq = np.array([[-1], [0], [1]], dtype=np.int8)
+    acc = orc.matmul_i32(xq, Wq)
+    for i, v in enumerate(range(-128, 128)):
+        assert acc[i].tolist() == [-v, 0, v]
+
+
+def pin_matmul_vs_linear(orc):
+    import torch
+    r = np.random.Generator(np.random.PCG64(31))
+    xq = r.integers(-127, 128, size=(6, 512), dtype=np.int8)
+    Wq = r.integers(-1, 2, size=(40, 512), dtype=np.int8)
+    acc = orc.matmul_i32(xq, Wq)
+    ref = torch.nn.functional.linear(torch.from_numpy(xq.astype(np.float64)),
+                                     torch.from_numpy(Wq.astype(np.float64)))
+    np.testing.assert_array_equal(acc.astype(np.float64), ref.numpy())
+    # sampled pairs agree with the full product
+    ms = np.array([0, 5, 3, 2]); ns = np.array([0, 39, 17, 3])
+    np.testing.assert_array_equal(orc.matmul_i32_pairs(xq, Wq, ms, ns), acc[ms, ns])
+
+
+def pin_quant_act_invariants(orc):
+    r = np.random.Generator(np.random.PCG64(41))
+    x = r.standard_normal((16, 300)).astype(np.float32)
+    x[:, r.choice(300, 3, replace=False)] *= 50
+    x[3] *= 1e-3
+    xq, beta = orc.quant_act(x)
+    np.testing.assert_array_equal(beta, np.max(np.abs(x), axis=1))
+    assert np.all(np.abs(xq.astype(np.int32)) <= 127)
+    assert np.all(np.max(np.abs(xq.astype(np.int32)), axis=1) == 127)
+    exact = x.astype(np.float64) * 127.0 / beta.astype(np.float64)[:, None]
+    assert np.max(np.abs(xq - exact)) <= 0.5 + 1e-4
+    assert np.all(np.sign(xq) * np.sign(x) >= 0)
+    for m in range(x.shape[0]):
+        order = np.argsort(x[m], kind="stable")
+        assert np.all(np.diff(xq[m][order].astype(np.int32)) >= 0)
+
+
+def pin_quant_act_pow2_invariance(orc):
+    r = np.random.Generator(np.random.PCG64(43))
+    x = r.standard_normal((4, 128)).astype(np.float32)
+    base, _ = orc.quant_act(x)
+    for e in (-7, -1, 3, 12):
+        xq, _ = orc.quant_act(x * np.float32(2.0 ** e))
+        np.testing.assert_array_equal(xq, base)
+
+
+def pin_bf16_rounding_vs_torch(orc):
+    import torch
+    r = np.random.Generator(np.random.PCG64(51))
+    f = (r.standard_normal(20000) * np.exp(r.uniform(-60, 60, 20000))).astype(np.float32)
+    base = (r.integers(0, 2 ** 31, 4000, dtype=np.int64).astype(np.uint32) & np.uint32(0x7fff0000))
+    ties = (base | np.uint32(0x8000)).view(np.float32)          # exact halfway cases
+    near = (base | np.uint32(0x7fff)).view(np.float32)
+    specials = np.array([0.0, -0.0, np.inf, -np.inf, 3.3895314e38, -3.3895314e38,
+                         1e-40, -1e-45, 1.0, 2.359375], dtype=np.float32)
+    allf = np.concatenate([f, ties, -ties, near, specials]).astype(np.float32)
+    allf = allf[np.isfinite(allf) | np.isinf(allf)]
+    got = orc.f32_to_bf16(allf)
+    ref = torch.from_numpy(allf).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    np.testing.assert_array_equal(got, ref)
+    nan_bits = orc.f32_to_bf16(np.array([np.nan], dtype=np.float32))
+    assert np.isnan(_bf16_value(nan_bits))[0]
+
+
+def pin_rescale_bound(orc):
+    r = np.random.Generator(np.random.PCG64(61))
+    acc = r.integers(-3_000_000, 3_000_000, size=(5, 70)).astype(np.int32)
+    beta = np.abs(r.standard_normal(5)).astype(np.float32) * 40 + np.float32(0.1)
+    gamma = np.float32(0.0159)
+    y = _bf16_value(orc.rescale_bf16(acc, beta, gamma)).astype(np.float64)
+    exact = acc.astype(np.float64) * beta.astype(np.float64)[:, None] * float(gamma) / 127.0
+    rel = np.abs(y - exact) / np.maximum(np.abs(exact), 1e-30)
+    assert np.all(rel <= 2.0 ** -8 + 1e-6), float(rel.max())
+    assert np.all(np.sign(y) == np.sign(exact))
+
+
+def pin_listing_semantics_torch(orc):
+    """The page's PyTorch listing, restated with torch CPU primitives
+    (mean/abs/clamp/round/linear) on fp32 tensors, gives the same integer
+    stages and the same bf16 output as the oracle on small random cases."""
+    import torch
+    r = np.random.Generator(np.random.PCG64(71))
+    for (M, K, N) in ((4, 256, 256), (3, 96, 40)):
+        W = (r.standard_normal((N, K)) * 0.02).astype(np.float32)
+        x = r.standard_normal((M, K)).astype(np.float32)
+        res = orc.forward(x, W)
+        Wt = torch.from_numpy(W)
+        g = Wt.abs().mean().clamp(min=1e-5)
+        assert abs(float(g) - float(res["gamma"])) <= 2 * np.spacing(res["gamma"])
+        g = torch.tensor(float(res["gamma"]), dtype=torch.float32)
+        wq = (Wt / g).round().clamp(-1.0, 1.0)
+        xt = torch.from_numpy(x)
+        b = xt.abs().amax(dim=-1, keepdim=True).clamp(min=1e-5)
+        xq = (xt * (127.0 / b)).round().clamp(-128.0, 127.0)
+        acc = torch.nn.functional.linear(xq.double(), wq.double())
+        y = (acc.float() * ((b * g) / 127.0)).to(torch.bfloat16)
+        np.testing.assert_array_equal(res["Wq"], wq.numpy().astype(np.int8))
+        np.testing.assert_array_equal(res["xq"], xq.numpy().astype(np.int8))
+        np.testing.assert_array_equal(res["beta"], b.numpy()[:, 0])
+        np.testing.assert_array_equal(res["acc"], acc.numpy().astype(np.int32))
+        np.testing.assert_array_equal(
+            res["y"], y.view(torch.int16).numpy().view(np.uint16))
+
+
+ALL_PINS = [
+    pin_hand_example,
+    pin_weight_ties_even,
+    pin_activation_ties_even,
+    pin_pack_words,
+    pin_pack_roundtrip,
+    pin_constant_token,
+    pin_zero_inputs,
+    pin_tiny_scale_epsilon,
+    pin_identity_weights,
+    pin_plus_minus_a,
+    pin_gamma_vs_numpy_mean,
+    pin_zero_fraction,
+    pin_bruteforce_add_subtract,
+    pin_exhaustive_single_term,
+    pin_matmul_vs_linear,
+    pin_quant_act_invariants,
+    pin_quant_act_pow2_invariance,
+    pin_bf16_rounding_vs_torch,
+    pin_rescale_bound,
+    pin_listing_semantics_torch,
+]
+
+
+def failing_pins(orc) -> list:
+    """Names of the pins the given oracle fails (an exception counts)."""
+    failed = []
+    for pin in ALL_PINS:
+        try:
+            pin(orc)
+        except Exception:  # noqa: BLE001 - any failure is a caught mistake
+            failed.append(pin.__name__)
+    return failed
