@@ -1,0 +1,518 @@
+"""Benchmark of the BitLinear W1.58A8 matmul on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Workload (one step): one decode token through the up (2560 -> 6912) and the
+down (6912 -> 2560) BitLinear projections of the 2B decoder, each with its own
+bf16 token (x ~ N(0,1), 1% outlier channels x50) and absmean-ternarised
+N(0, 0.02) latents packed 2 bits per weight. The packed weights rotate over
+32 device copies (283 MB, more than twice the 126 MB L2), so every step
+streams its weights from HBM. The headline is the GEMV's HBM throughput on
+packed-weight bytes. The same line carries the prefill GEMM (M = 2048 tokens,
+int8 tensor cores) in ``prefill_gemm``.
+
+With ``--gpus N`` (launched by torchrun, one process per GPU) every rank runs
+the same independent workload (weak scaling: the path has no data-path
+collective); the time is the max over ranks and ``value`` counts all ranks'
+bytes.
+
+``--impl reference`` times the CPU oracle (test infrastructure, plain C,
+one thread) on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads  # noqa: E402
+
+METRIC = "BitLinear GEMV HBM GB/s (% of peak); prefill GEMM int8 TOPS (% of peak)"
+UNIT = "GB/s"
+ROTATE = 32                # packed weight copies per matrix (> 2 x L2 in total)
+PREFILL_COPIES = 8
+MEASURED_PEAKS = os.path.join(ROOT, "MEASURED_PEAKS.json")
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+INT8_PER_BF16 = 2.0        # nominal dense int8 / bf16 tensor ratio (4.5 / 2.25 P)
+
+# DRAM traffic per launch of the dominant kernels, from an ncu capture
+# (dram__bytes_read.sum + dram__bytes_write.sum), keyed by the sha256 of the
+# kernel source it was taken on; reported only while that source is unchanged.
+TRAFFIC = {}
+
+
+def kernel_source_hash(name: str) -> str:
+    path = os.path.join(ROOT, "ternary_weight_w1_b200", "csrc", name)
+    with open(path, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def load_peaks():
+    try:
+        with open(MEASURED_PEAKS) as f:
+            d = json.load(f)
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                "source": "measured"}
+    except (OSError, KeyError, ValueError):
+        return {"hbm_gbs": FALLBACK_HBM_GBS, "bf16_tflops": FALLBACK_BF16_TFLOPS,
+                "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+# ------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons in the background."""
+
+    FIELDS = ("timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str, interval_ms: int = 50):
+        self.gpu_id = gpu_id
+        self.interval_ms = interval_ms
+        self.proc = None
+        self.lines = []
+        self.t0 = self.t1 = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-i", self.gpu_id, "-lms", str(self.interval_ms)],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        self.reader = threading.Thread(target=self._read, daemon=True)
+        self.reader.start()
+        time.sleep(0.3)
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append((time.time(), line.strip()))
+
+    def mark(self, start: bool):
+        if start:
+            self.t0 = time.time()
+        else:
+            self.t1 = time.time()
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.2)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        for t, line in self.lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append((t, float(parts[1]), float(parts[2]), parts[4:9]))
+            except ValueError:
+                continue
+        inside = [r for r in rows if self.t0 is not None and self.t0 - 0.06 <= r[0] <= (self.t1 or r[0]) + 0.06]
+        use = inside if inside else rows
+        if not use:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        names = ["active_mask", "hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown",
+                 "sw_power_cap"]
+        reasons = set()
+        for r in use:
+            for n, v in zip(names[1:], r[3][1:]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(r[1] for r in use),
+                "sm_max_mhz": max(r[2] for r in use),
+                "reasons": sorted(reasons), "samples": len(use),
+                "samples_in_timed_region": len(inside)}
+
+
+def smi_gpu_id(local_rank: int) -> str:
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+    if vis:
+        ids = [v.strip() for v in vis.split(",") if v.strip()]
+        if local_rank < len(ids):
+            return ids[local_rank]
+    return str(local_rank)
+
+
+# ----------------------------------------------------------- distributed
+
+class Dist:
+    def __init__(self):
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.rank = int(os.environ.get("RANK", "0"))
+        self.local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+        self.pg = None
+
+    def init(self, backend: str):
+        if self.world > 1:
+            import datetime
+            import torch.distributed as dist
+            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+            self.pg = dist
+
+    def barrier(self):
+        if self.pg is not None:
+            self.pg.barrier()
+
+    def max(self, v: float) -> float:
+        if self.pg is None:
+            return v
+        import torch
+        t = torch.tensor([v], dtype=torch.float64,
+                         device="cuda" if torch.cuda.is_available() else "cpu")
+        self.pg.all_reduce(t, op=self.pg.ReduceOp.MAX)
+        return float(t.item())
+
+    def close(self):
+        if self.pg is not None:
+            self.pg.destroy_process_group()
+
+
+# ------------------------------------------------------------ our arm
+
+def bf16_tensor(bits, device):
+    import torch
+    return torch.from_numpy(bits.view(np.int16).copy()).view(torch.bfloat16).to(device)
+
+
+class DecodeWorkload:
+    """Device-resident inputs of the decode step with ROTATE weight copies."""
+
+    def __init__(self, bl, device):
+        import torch
+        self.bl = bl
+        probs = workloads.decode_gemv_2b(1).problems
+        self.mats = []
+        for p in probs:
+            packed, gamma = bl.bitlinear_pack_weights(p.weights())
+            dev_packed = torch.from_numpy(packed).to(device)
+            copies = [dev_packed] + [dev_packed.clone() for _ in range(ROTATE - 1)]
+            xs = [bf16_tensor(workloads.activations_bf16(1, p.K, p.x_seed + 7919 * i), device)
+                  for i in range(ROTATE)]
+            ys = [torch.empty((1, p.N), dtype=torch.bfloat16, device=device)
+                  for _ in range(ROTATE)]
+            self.mats.append({"p": p, "gamma": gamma, "packed": copies, "x": xs, "y": ys})
+        self.packed_bytes_per_step = sum(m["p"].N * m["p"].K // 4 for m in self.mats)
+        self.io_bytes_per_step = sum(2 * m["p"].K + 2 * m["p"].N for m in self.mats)
+        self.launches_per_step = len(self.mats)
+
+    def step(self, i: int):
+        j = i % ROTATE
+        for m in self.mats:
+            self.bl.bitlinear_forward(m["x"][j], m["packed"][j], m["gamma"], m["p"].N,
+                                      y=m["y"][j])
+
+    def run_steps(self, start: int, count: int):
+        for i in range(start, start + count):
+            self.step(i)
+
+
+def capture_graph(fn):
+    import torch
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        fn()
+    return g
+
+
+def time_graph_steps(dist, wl, steps: int, clocks: ClockSampler | None):
+    """Time exactly `steps` decode steps replayed from CUDA graphs."""
+    import torch
+    full = capture_graph(lambda: wl.run_steps(0, ROTATE))
+    rem = steps % ROTATE
+    tail = capture_graph(lambda: wl.run_steps(0, rem)) if rem else None
+    for _ in range(3):
+        full.replay()
+    torch.cuda.synchronize()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    dist.barrier()
+    torch.cuda.synchronize()
+    if clocks:
+        clocks.mark(True)
+    start.record()
+    for _ in range(steps // ROTATE):
+        full.replay()
+    if tail is not None:
+        tail.replay()
+    end.record()
+    torch.cuda.synchronize()
+    if clocks:
+        clocks.mark(False)
+    dist.barrier()
+    ms = start.elapsed_time(end)
+    del full, tail
+    return dist.max(ms)
+
+
+def time_e2e(dist, wl, steps: int):
+    """Same steps through the public Python API, with each step's tokens copied
+    from pinned host memory and its outputs read back to pinned host memory."""
+    import torch
+    host_x = [[m["x"][j].cpu().pin_memory() for j in range(ROTATE)] for m in wl.mats]
+    host_y = [torch.empty(m["y"][0].shape, dtype=torch.bfloat16).pin_memory() for m in wl.mats]
+    dev_x = [m["x"][0].clone() for m in wl.mats]
+
+    def one(i):
+        j = i % ROTATE
+        for k, m in enumerate(wl.mats):
+            dev_x[k].copy_(host_x[k][j], non_blocking=True)
+            wl.bl.bitlinear_forward(dev_x[k], m["packed"][j], m["gamma"], m["p"].N, y=m["y"][j])
+            host_y[k].copy_(m["y"][j], non_blocking=True)
+
+    for i in range(5):
+        one(i)
+    torch.cuda.synchronize()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    dist.barrier()
+    torch.cuda.synchronize()
+    start.record()
+    for i in range(steps):
+        one(i)
+    end.record()
+    torch.cuda.synchronize()
+    dist.barrier()
+    return dist.max(start.elapsed_time(end))
+
+
+def bench_prefill(bl, device, reps: int = 20):
+    """Prefill step (M = 2048: up and down, quantisation kernel + tcgen05
+    GEMM each), inputs rotating over copies larger than L2. Returns
+    (ms per step, int8 ops per step)."""
+    import torch
+    probs = workloads.prefill_2b(2048).problems
+    mats = []
+    for p in probs:
+        packed, gamma = bl.bitlinear_pack_weights(p.weights())
+        dp = torch.from_numpy(packed).to(device)
+        x = bf16_tensor(p.x_input(), device)
+        ws_bytes = bl.bitlinear_workspace_bytes(p.M, p.N, p.K)
+        mats.append({"p": p, "gamma": gamma,
+                     "packed": [dp] + [dp.clone() for _ in range(PREFILL_COPIES - 1)],
+                     "x": [x] + [x.clone() for _ in range(PREFILL_COPIES - 1)],
+                     "y": torch.empty((p.M, p.N), dtype=torch.bfloat16, device=device),
+                     "ws": torch.empty((ws_bytes,), dtype=torch.uint8, device=device)})
+
+    def step(i):
+        j = i % PREFILL_COPIES
+        for m in mats:
+            bl.bitlinear_forward(m["x"][j], m["packed"][j], m["gamma"], m["p"].N, y=m["y"],
+                                 workspace=m["ws"])
+
+    for i in range(3):
+        step(i)
+    g = capture_graph(lambda: [step(i) for i in range(PREFILL_COPIES)])
+    g.replay()
+    torch.cuda.synchronize()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record()
+    for _ in range(reps):
+        g.replay()
+    end.record()
+    torch.cuda.synchronize()
+    ms = start.elapsed_time(end) / (reps * PREFILL_COPIES)
+    ops = sum(2 * m["p"].M * m["p"].N * m["p"].K for m in mats)
+    return ms, ops
+
+
+def cpu_baseline_oracle(seconds: float = 10.0):
+    """The oracle (single-threaded C) on the decode step: x quantisation,
+    integer product and rescale for the up and down projections, repeated
+    for about `seconds`. Returns (GB/s of packed-weight bytes, steps)."""
+    import oracle
+    orc = oracle.default()
+    mats = []
+    for p in workloads.decode_gemv_2b(1).problems:
+        W = p.weights()
+        g = orc.absmean_gamma(W)
+        mats.append((p, orc.ternarize(W, g), g, orc.bf16_to_f32(p.x_input())))
+    nbytes = sum(p.N * p.K // 4 for p, *_ in mats)
+    t0 = time.perf_counter()
+    steps = 0
+    while True:
+        for p, Wq, g, xf in mats:
+            xq, beta = orc.quant_act(xf)
+            acc = orc.matmul_i32(xq, Wq)
+            orc.rescale_bf16(acc, beta, g)
+        steps += 1
+        el = time.perf_counter() - t0
+        if el >= seconds:
+            break
+    return nbytes * steps / el / 1e9, steps, el
+
+
+def run_ours(args, dist):
+    import torch
+    import ternary_weight_w1_b200 as bl
+    torch.cuda.set_device(dist.local_rank)
+    device = torch.device("cuda", dist.local_rank)
+    bl.lib()
+    peaks = load_peaks()
+    wl = DecodeWorkload(bl, device)
+    for i in range(args.warmup):
+        wl.step(i)
+    torch.cuda.synchronize()
+
+    clocks = ClockSampler(smi_gpu_id(dist.local_rank))
+    clocks.start()
+    ms = time_graph_steps(dist, wl, args.steps, clocks)
+    clk = clocks.stop()
+
+    bytes_all = wl.packed_bytes_per_step * args.steps * dist.world
+    value = bytes_all / (ms * 1e-3) / 1e9
+    launches = wl.launches_per_step * args.steps
+    per_launch_bytes = wl.packed_bytes_per_step / wl.launches_per_step
+    avg_launch_ms = ms / launches
+    achieved = per_launch_bytes / (avg_launch_ms * 1e-3) / 1e9
+    traffic = None
+    t = TRAFFIC.get("gemv")
+    if t is not None and t.get("src") == kernel_source_hash("gemv.cuh"):
+        traffic = t["bytes_per_launch"]
+
+    e2e_steps = min(args.steps, args.e2e_steps)
+    ms_e2e = time_e2e(dist, wl, e2e_steps)
+    e2e_value = wl.packed_bytes_per_step * e2e_steps * dist.world / (ms_e2e * 1e-3) / 1e9
+
+    pre_ms, pre_ops = bench_prefill(bl, device)
+    pre_tops = pre_ops / (pre_ms * 1e-3) / 1e12
+    int8_peak = peaks["bf16_tflops"] * INT8_PER_BF16
+
+    out = {
+        "metric": METRIC,
+        "value": round(value, 2),
+        "unit": UNIT,
+        "n_gpus": dist.world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms / args.steps,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "int8xternary->int32 (bf16 in/out)",
+        "data": "synthetic (seeded N(0,0.02) latents, N(0,1) bf16 tokens with 1% x50 outlier channels)",
+        "config": {"workload": "decode GEMV, 2B shape, M=1: up 2560->6912 then down 6912->2560 "
+                               f"per step, packed weights rotating over {ROTATE} device copies "
+                               f"({ROTATE * wl.packed_bytes_per_step / 1e6:.0f} MB > L2), "
+                               "CUDA-graph replay",
+                   "l2": "inputs larger than L2 (rotating weight copies)",
+                   "parallelism": f"replicas x{dist.world}"},
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 1),
+                     "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": traffic,
+                     "kernel": "gemv_kernel<1,bf16,8>",
+                     "algorithmic_bytes_per_launch": per_launch_bytes,
+                     "peak_source": peaks["source"]},
+        "e2e": {"value": round(e2e_value, 2), "unit": UNIT,
+                "h2d_bytes_per_step": sum(2 * m["p"].K for m in wl.mats),
+                "d2h_bytes_per_step": sum(2 * m["p"].N for m in wl.mats),
+                "steps": e2e_steps},
+        "gpu_launches": launches,
+        "clocks": clk,
+        "prefill_gemm": {"workload": "M=2048 tokens: up 2560->6912 and down 6912->2560, "
+                                     "quantisation kernel + tcgen05 kind::i8 GEMM each",
+                         "value": round(pre_tops, 1), "unit": "TOPS (int8)",
+                         "ms_per_step": pre_ms,
+                         "peak": int8_peak, "peak_note": "measured bf16 burst x 2 (nominal int8/bf16)",
+                         "frac": round(pre_tops / int8_peak, 4)},
+    }
+    if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
+        v, steps, el = cpu_baseline_oracle(args.cpu_seconds)
+        out["cpu_baseline"] = {"value": round(v, 4), "unit": UNIT, "cores": 1, "kind": "oracle",
+                               "sample": f"{steps} full decode steps (up+down, M=1) of the "
+                                         f"single-threaded C oracle in {el:.1f} s"}
+    return out
+
+
+# ------------------------------------------------------ reference arm
+
+def run_reference(args, dist):
+    """The oracle on the host cores: each step a bounded sample of the decode
+    step (1/64 of the output rows of both projections)."""
+    import oracle
+    orc = oracle.default()
+    sample = 64
+    mats = []
+    for p in workloads.decode_gemv_2b(1).problems:
+        W = p.weights()
+        g = orc.absmean_gamma(W)
+        rows = p.N // sample
+        Wq = orc.ternarize(W[:rows], g)
+        mats.append((p, Wq, g, orc.bf16_to_f32(p.x_input())))
+    nbytes = sum(Wq.shape[0] * p.K // 4 for p, Wq, *_ in mats)
+
+    def step():
+        for p, Wq, g, xf in mats:
+            xq, beta = orc.quant_act(xf)
+            acc = orc.matmul_i32(xq, Wq)
+            orc.rescale_bf16(acc, beta, g)
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    el = time.perf_counter() - t0
+    v = nbytes * args.steps / el / 1e9
+    return {"metric": METRIC, "value": round(v, 4), "unit": UNIT, "n_gpus": dist.world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": el * 1e3 / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "int8xternary->int32 (bf16 in/out)", "data": "synthetic",
+            "impl": "reference",
+            "config": {"workload": "decode GEMV, 2B shape, M=1: up 2560->6912 then down "
+                                   "6912->2560 per step (oracle on 1/64 of the output rows)",
+                       "parallelism": "host cores, 1 thread"},
+            "cpu_baseline": {"value": round(v, 4), "unit": UNIT, "cores": 1, "kind": "oracle",
+                             "sample": f"1/{sample} of the output rows of each projection per step"},
+            "e2e": {"value": round(v, 4), "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50000)
+    ap.add_argument("--warmup", type=int, default=64)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--e2e-steps", type=int, default=20000)
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    dist = Dist()
+    if args.impl == "reference":
+        if dist.rank != 0:
+            return 0
+        print(json.dumps(run_reference(args, dist)), flush=True)
+        return 0
+    dist.init("nccl")
+    try:
+        out = run_ours(args, dist)
+        if dist.rank == 0:
+            print(json.dumps(out), flush=True)
+    finally:
+        dist.close()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

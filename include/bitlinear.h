@@ -1,0 +1,202 @@
+/*
+ * bitlinear.h -- C ABI of libbitlinear, the BitNet b1.58 BitLinear W1.58A8
+ * matmul for NVIDIA B200 (sm_100a).
+ *
+ * The operator (page "BitNet b1.58 2B4T Guide: Scaling Native 1-Bit LLMs"):
+ *   - weights W in R^{d_out x d_in} are ternarised once by absmean scaling,
+ *       gamma = max(mean_{i,j} |W_ij|, 1e-5),  W~ = Clip(Round(W / gamma), -1, 1)
+ *     (section "Ternary Weight Quantization: absmean Scaling");
+ *   - each token x in R^{d_in} is quantised to int8 by absmax scaling,
+ *       beta = max(max_j |x_j|, 1e-5),  x~ = Clip(Round(x * (127 / beta)), -128, 127)
+ *     (section "8-Bit Activation Quantization: absmax Scaling");
+ *   - the product is an integer sum, rescaled once:
+ *       y = bf16( float(x~ W~^T) * ((beta * gamma) / 127) )
+ *     (section "Matrix Multiplication as Pure Integer Addition").
+ * Round is round-half-to-even (torch.round in the page's PyTorch listing),
+ * all floating point is IEEE fp32, and the output is rounded once to bf16.
+ *
+ * Notation: M tokens, K = d_in, N = d_out. x is [M][K] row-major, W is [N][K]
+ * row-major, y is [M][N] row-major (y = x W^T).
+ *
+ * Conventions shared by every call:
+ *   - Ownership: the caller allocates and frees every buffer. The library
+ *     never allocates or frees memory; device buffers (x, packed weights, y,
+ *     workspace, debug outputs) are plain device pointers.
+ *   - Streams: cuda_stream is a cudaStream_t (NULL = the legacy default
+ *     stream). All device work is enqueued asynchronously on it; nothing
+ *     synchronises the host except bitlinear_get_fault.
+ *   - Errors: every call returns a bitlinear_status; nothing throws across
+ *     the ABI. Argument errors are detected on the host before any launch.
+ *     BITLINEAR_ERR_CUDA reports a launch error (cudaGetLastError); faults of
+ *     work already enqueued surface at the caller's next synchronisation.
+ *   - Alignment: x, packed weights, y, workspace and int8 outputs must be
+ *     16-byte aligned, fp32/int32 outputs 4-byte aligned.
+ *   - Shapes: K must be a positive multiple of 128 for the device calls;
+ *     M >= 0 (M = 0 is a no-op), N >= 1, K <= 65536 for the forward calls.
+ */
+#ifndef BITLINEAR_H
+#define BITLINEAR_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define BITLINEAR_ABI_VERSION 1
+
+typedef enum {
+    BITLINEAR_OK = 0,
+    BITLINEAR_ERR_ARG = 1,       /* null pointer or negative size */
+    BITLINEAR_ERR_SHAPE = 2,     /* K not a multiple of 128, K or N out of range */
+    BITLINEAR_ERR_ALIGN = 3,     /* a pointer misses its alignment */
+    BITLINEAR_ERR_DTYPE = 4,     /* unknown bitlinear_dtype */
+    BITLINEAR_ERR_CUDA = 5,      /* a CUDA runtime/driver call failed */
+    BITLINEAR_ERR_TIMEOUT = 6,   /* a bounded device-side wait ran out */
+    BITLINEAR_ERR_WORKSPACE = 7  /* workspace missing or smaller than required */
+} bitlinear_status;
+
+typedef enum {
+    BITLINEAR_BF16 = 0,          /* x holds bf16 values (widened exactly to fp32) */
+    BITLINEAR_FP32 = 1           /* x holds fp32 values */
+} bitlinear_dtype;
+
+/* Kernel choice for bitlinear_forward_ex. */
+typedef enum {
+    BITLINEAR_PATH_AUTO = 0,     /* pick by M (what bitlinear_forward does) */
+    BITLINEAR_PATH_GEMV = 1,     /* fused-quant dp4a GEMV, M <= 16 */
+    BITLINEAR_PATH_TC = 2        /* quant kernel + tcgen05 kind::i8 GEMM */
+} bitlinear_path;
+
+/* ---------------------------------------------------------------- packing */
+
+/* Bytes of the packed ternary matrix for N rows of K weights: N * K / 4.
+ * Returns 0 when N < 1, K < 16 or K % 16 != 0.
+ *
+ * Packed layout (this library's own; the "2-bit nibbles" of the bitnet.xin
+ * guide, section "Core Architecture"):
+ *   - N rows of K/4 bytes, row n starting at byte n * K / 4 (row-major, so a
+ *     contiguous range of rows is one contiguous byte range);
+ *   - the 32-bit little-endian word w of a row holds the weights
+ *     k in [16w, 16w + 16);
+ *   - weight k = 16w + 4j + b (j, b in 0..3) sits in bits 8b + 2j and
+ *     8b + 2j + 1 of its word as the code W~ + 1 (0, 1 or 2; 3 is unused).
+ *   So (word >> 2j) & 0x03030303 holds the codes of k = 16w + 4j .. 16w + 4j + 3,
+ *   one per byte, in the order of an int32 word of int8 activations, and a
+ *   16-byte load is 64 consecutive weights of one row. */
+size_t bitlinear_packed_bytes(int64_t N, int64_t K);
+
+/* Offline absmean ternarisation and packing, on the host (no device work).
+ *   W_host      [in]  latent fp32 weights, [N][K] row-major, host memory
+ *   N, K        [in]  d_out, d_in; K must be a positive multiple of 16
+ *   packed_host [out] caller-allocated host buffer of bitlinear_packed_bytes(N, K)
+ *                     bytes (copy it to the device before bitlinear_forward)
+ *   gamma_out   [out] gamma = max(mean |W|, 1e-5), the sum taken in double
+ * Follows section "Ternary Weight Quantization: absmean Scaling" and the
+ * listing's WeightQuantFunction.forward (W / gamma in fp32, ties to even,
+ * clip to [-1, 1]). Returns BITLINEAR_ERR_ARG for null pointers or N < 1,
+ * BITLINEAR_ERR_SHAPE for a bad K. Runs on several host threads; the result
+ * does not depend on their number. */
+int bitlinear_pack_weights(const float *W_host, int64_t N, int64_t K,
+                           void *packed_host, float *gamma_out);
+
+/* ------------------------------------------------- activation quantisation */
+
+/* Per-token absmax int8 quantisation on the device.
+ *   x_dev   [in]  [M][K] activations of type xdt, device memory
+ *   xq_dev  [out] [M][K] int8 x~, device memory (16-byte aligned)
+ *   beta_dev[out] [M] fp32 beta (the clamped absmax of each token)
+ * Section "8-Bit Activation Quantization: absmax Scaling" and the listing's
+ * quantize_activations_int8. One kernel launch on cuda_stream. */
+int bitlinear_quant_act(const void *x_dev, bitlinear_dtype xdt, int64_t M,
+                        int64_t K, int8_t *xq_dev, float *beta_dev,
+                        void *cuda_stream);
+
+/* ---------------------------------------------------------------- forward */
+
+/* Device workspace bytes bitlinear_forward needs for (M, N, K): 0 when the
+ * GEMV path is taken (small M), else room for x~ (M*K bytes), beta and the
+ * per-token sums of x~. Returns SIZE_MAX for invalid shapes. */
+size_t bitlinear_workspace_bytes(int64_t M, int64_t N, int64_t K);
+
+/* y = BitLinear(x) with pre-packed ternary weights, on the device.
+ *   x_dev       [in]  [M][K] activations of type xdt
+ *   packed_dev  [in]  packed weights (layout above), N * K / 4 bytes
+ *   gamma       [in]  the gamma bitlinear_pack_weights returned
+ *   y_dev       [out] [M][N] bf16 (uint16 bit patterns)
+ *   workspace_dev, workspace_bytes
+ *               [in]  scratch of at least bitlinear_workspace_bytes(M, N, K)
+ *                     bytes (may be NULL when that is 0); its contents are
+ *                     overwritten
+ *   acc_dev_or_null  [out, optional] [M][N] int32 x~ W~^T before rescaling
+ *   xq_dev_or_null   [out, optional] [M][K] int8 x~
+ *   beta_dev_or_null [out, optional] [M] fp32 beta
+ * The optional outputs exist so that tests can compare the integer stages
+ * bit for bit; pass NULL in production. Small M runs one fused kernel
+ * (quantisation in the prologue, dp4a over the packed weights); larger M runs
+ * the quantisation kernel and the tcgen05 int8 tensor-core GEMM. */
+int bitlinear_forward(const void *x_dev, bitlinear_dtype xdt, int64_t M,
+                      int64_t K, const void *packed_dev, float gamma,
+                      int64_t N, void *y_dev, void *workspace_dev,
+                      size_t workspace_bytes, void *cuda_stream,
+                      int32_t *acc_dev_or_null, int8_t *xq_dev_or_null,
+                      float *beta_dev_or_null);
+
+/* bitlinear_forward with an explicit kernel choice (bitlinear_path).
+ * BITLINEAR_PATH_GEMV needs M <= 16 and M * K <= 196608; otherwise it
+ * returns BITLINEAR_ERR_SHAPE. The workspace for BITLINEAR_PATH_TC is
+ * bitlinear_workspace_bytes_path(M, N, K, BITLINEAR_PATH_TC). */
+int bitlinear_forward_ex(const void *x_dev, bitlinear_dtype xdt, int64_t M,
+                         int64_t K, const void *packed_dev, float gamma,
+                         int64_t N, void *y_dev, void *workspace_dev,
+                         size_t workspace_bytes, void *cuda_stream,
+                         int32_t *acc_dev_or_null, int8_t *xq_dev_or_null,
+                         float *beta_dev_or_null, int path);
+
+/* Workspace bytes for an explicit path (see bitlinear_forward_ex). */
+size_t bitlinear_workspace_bytes_path(int64_t M, int64_t N, int64_t K,
+                                      int path);
+
+/* ------------------------------------------------------------- diagnostics */
+
+/* Device-side fault word. Every bounded wait in the tensor-core GEMM gives
+ * up after a time limit, records a nonzero code here and lets the kernel
+ * return instead of hanging. This call synchronises cuda_stream, stores the
+ * word in *fault_out (0 = none) and clears it. Returns BITLINEAR_ERR_TIMEOUT
+ * when the word was set, BITLINEAR_ERR_CUDA when the synchronisation failed,
+ * BITLINEAR_OK otherwise. */
+int bitlinear_get_fault(int *fault_out, void *cuda_stream);
+
+/* Human-readable name of a bitlinear_status. Never NULL. */
+const char *bitlinear_status_string(int status);
+
+/* --------------------------------------------------------- measurement aids */
+
+/* Plain int8 x int8 -> int32 GEMM C[M][N] = A[M][K] B[N][K]^T on the same
+ * tcgen05 pipeline as the forward GEMM, with B already int8 (no unpacking).
+ * It has no counterpart on the pages: it measures the int8 tensor-core
+ * roofline the forward GEMM is reported against. A, B: int8 row-major,
+ * 16-byte aligned; C: int32 [M][N]. K % 128 == 0. */
+int bitlinear_int8_gemm(const int8_t *A_dev, const int8_t *B_dev,
+                        int32_t *C_dev, int64_t M, int64_t N, int64_t K,
+                        void *cuda_stream);
+
+/* The forward tensor-core GEMM with one wait made to run out on purpose:
+ * the MMA issuer waits on a barrier nobody arrives at, for timeout_us
+ * microseconds, then the kernel records a fault and every role returns.
+ * Used by the failure-detection test; inputs as for bitlinear_forward_ex
+ * with BITLINEAR_PATH_TC. */
+int bitlinear_forward_inject_timeout(const void *x_dev, bitlinear_dtype xdt,
+                                     int64_t M, int64_t K,
+                                     const void *packed_dev, float gamma,
+                                     int64_t N, void *y_dev,
+                                     void *workspace_dev,
+                                     size_t workspace_bytes,
+                                     void *cuda_stream, int timeout_us);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BITLINEAR_H */

@@ -1,0 +1,232 @@
+"""Python binding of libbitlinear, the BitLinear W1.58A8 matmul for B200.
+
+Argument marshalling only: every step of the path runs in the CUDA library
+(``libbitlinear.so``, built in-tree by ``ternary_weight_w1_b200.build``). The
+functions carry the C ABI's names (see include/bitlinear.h for semantics and
+layouts) and take torch tensors for device buffers; PyTorch supplies device
+memory and streams. There is no CPU fallback: if the library is missing,
+loading it raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libbitlinear.so")
+
+BITLINEAR_OK = 0
+BITLINEAR_ERR_ARG = 1
+BITLINEAR_ERR_SHAPE = 2
+BITLINEAR_ERR_ALIGN = 3
+BITLINEAR_ERR_DTYPE = 4
+BITLINEAR_ERR_CUDA = 5
+BITLINEAR_ERR_TIMEOUT = 6
+BITLINEAR_ERR_WORKSPACE = 7
+
+BITLINEAR_BF16 = 0
+BITLINEAR_FP32 = 1
+
+PATH_AUTO = 0
+PATH_GEMV = 1
+PATH_TC = 2
+
+# Every symbol include/bitlinear.h declares.
+EXPORTS = (
+    "bitlinear_packed_bytes",
+    "bitlinear_pack_weights",
+    "bitlinear_quant_act",
+    "bitlinear_workspace_bytes",
+    "bitlinear_workspace_bytes_path",
+    "bitlinear_forward",
+    "bitlinear_forward_ex",
+    "bitlinear_get_fault",
+    "bitlinear_status_string",
+    "bitlinear_int8_gemm",
+    "bitlinear_forward_inject_timeout",
+)
+
+_lib = None
+
+
+class BitLinearError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {status_string(status)} (status {status})")
+
+
+def lib() -> ctypes.CDLL:
+    """Load libbitlinear.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(
+                f"{LIB_PATH} is missing: build it with "
+                "`python -m ternary_weight_w1_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        i64, p, sz = ctypes.c_int64, ctypes.c_void_p, ctypes.c_size_t
+        L.bitlinear_packed_bytes.restype = sz
+        L.bitlinear_packed_bytes.argtypes = [i64, i64]
+        L.bitlinear_pack_weights.restype = ctypes.c_int
+        L.bitlinear_pack_weights.argtypes = [p, i64, i64, p, p]
+        L.bitlinear_quant_act.restype = ctypes.c_int
+        L.bitlinear_quant_act.argtypes = [p, ctypes.c_int, i64, i64, p, p, p]
+        L.bitlinear_workspace_bytes.restype = sz
+        L.bitlinear_workspace_bytes.argtypes = [i64, i64, i64]
+        L.bitlinear_workspace_bytes_path.restype = sz
+        L.bitlinear_workspace_bytes_path.argtypes = [i64, i64, i64, ctypes.c_int]
+        fwd = [p, ctypes.c_int, i64, i64, p, ctypes.c_float, i64, p, p, sz, p, p, p, p]
+        L.bitlinear_forward.restype = ctypes.c_int
+        L.bitlinear_forward.argtypes = fwd
+        L.bitlinear_forward_ex.restype = ctypes.c_int
+        L.bitlinear_forward_ex.argtypes = fwd + [ctypes.c_int]
+        L.bitlinear_forward_inject_timeout.restype = ctypes.c_int
+        L.bitlinear_forward_inject_timeout.argtypes = fwd[:11] + [ctypes.c_int]
+        L.bitlinear_get_fault.restype = ctypes.c_int
+        L.bitlinear_get_fault.argtypes = [p, p]
+        L.bitlinear_status_string.restype = ctypes.c_char_p
+        L.bitlinear_status_string.argtypes = [ctypes.c_int]
+        L.bitlinear_int8_gemm.restype = ctypes.c_int
+        L.bitlinear_int8_gemm.argtypes = [p, p, p, i64, i64, i64, p]
+        _lib = L
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return lib().bitlinear_status_string(int(status)).decode()
+
+
+def _check(rc: int, where: str) -> None:
+    if rc != BITLINEAR_OK:
+        raise BitLinearError(rc, where)
+
+
+def _ptr(t) -> int | None:
+    return None if t is None else t.data_ptr()
+
+
+def _stream(stream) -> int | None:
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream
+
+
+def _xdt(x) -> int:
+    import torch
+    if x.dtype == torch.bfloat16:
+        return BITLINEAR_BF16
+    if x.dtype == torch.float32:
+        return BITLINEAR_FP32
+    raise TypeError(f"x must be bf16 or fp32, got {x.dtype}")
+
+
+# ---------------------------------------------------------------- packing
+
+def bitlinear_packed_bytes(N: int, K: int) -> int:
+    return int(lib().bitlinear_packed_bytes(N, K))
+
+
+def bitlinear_pack_weights(W) -> tuple[np.ndarray, float]:
+    """Ternarise and pack latent fp32 weights [N][K] on the host.
+    Returns (packed uint8 [N][K/4] numpy array, gamma)."""
+    W = np.ascontiguousarray(np.asarray(W, dtype=np.float32))
+    if W.ndim != 2:
+        raise ValueError("W must be 2-D [N][K]")
+    N, K = W.shape
+    nbytes = bitlinear_packed_bytes(N, K)
+    if nbytes == 0:
+        raise BitLinearError(BITLINEAR_ERR_SHAPE, "bitlinear_pack_weights")
+    out = np.empty((N, K // 4), dtype=np.uint8)
+    gamma = ctypes.c_float(0.0)
+    _check(lib().bitlinear_pack_weights(W.ctypes.data, N, K, out.ctypes.data,
+                                        ctypes.addressof(gamma)),
+           "bitlinear_pack_weights")
+    return out, float(gamma.value)
+
+
+# ------------------------------------------------- activation quantisation
+
+def bitlinear_quant_act(x, xq=None, beta=None, stream=None):
+    """x~ (int8 [M][K]) and beta (fp32 [M]) of device activations x."""
+    import torch
+    M, K = x.shape
+    if xq is None:
+        xq = torch.empty((M, K), dtype=torch.int8, device=x.device)
+    if beta is None:
+        beta = torch.empty((M,), dtype=torch.float32, device=x.device)
+    _check(lib().bitlinear_quant_act(_ptr(x), _xdt(x), M, K, _ptr(xq), _ptr(beta),
+                                     _stream(stream)),
+           "bitlinear_quant_act")
+    return xq, beta
+
+
+# ---------------------------------------------------------------- forward
+
+def bitlinear_workspace_bytes(M: int, N: int, K: int, path: int = PATH_AUTO) -> int:
+    return int(lib().bitlinear_workspace_bytes_path(M, N, K, path))
+
+
+def bitlinear_forward(x, packed, gamma: float, N: int, y=None, workspace=None,
+                      stream=None, acc=None, xq=None, beta=None, path: int = PATH_AUTO):
+    """y (bf16 [M][N]) = BitLinear(x) with device-resident packed weights.
+
+    ``workspace`` is a device uint8 tensor of at least
+    ``bitlinear_workspace_bytes(M, N, K, path)`` bytes (allocated here when
+    omitted); ``acc``/``xq``/``beta`` are optional debug outputs of the
+    integer stages."""
+    import torch
+    M, K = x.shape
+    if y is None:
+        y = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
+    need = bitlinear_workspace_bytes(M, N, K, path)
+    if need == ctypes.c_size_t(-1).value:
+        raise BitLinearError(BITLINEAR_ERR_SHAPE, "bitlinear_workspace_bytes")
+    if workspace is None and need > 0:
+        workspace = torch.empty((need,), dtype=torch.uint8, device=x.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    args = (_ptr(x), _xdt(x), M, K, _ptr(packed), float(gamma), N, _ptr(y),
+            _ptr(workspace), ws_bytes, _stream(stream), _ptr(acc), _ptr(xq), _ptr(beta))
+    if path == PATH_AUTO:
+        rc = lib().bitlinear_forward(*args)
+    else:
+        rc = lib().bitlinear_forward_ex(*args, path)
+    _check(rc, "bitlinear_forward")
+    return y
+
+
+def bitlinear_forward_inject_timeout(x, packed, gamma: float, N: int, timeout_us: int,
+                                     y=None, workspace=None, stream=None) -> int:
+    """Run the tensor-core GEMM with one wait made to run out; returns the
+    status the launch reported (the fault is read by bitlinear_get_fault)."""
+    import torch
+    M, K = x.shape
+    if y is None:
+        y = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
+    need = bitlinear_workspace_bytes(M, N, K, PATH_TC)
+    if workspace is None:
+        workspace = torch.empty((max(need, 1),), dtype=torch.uint8, device=x.device)
+    return int(lib().bitlinear_forward_inject_timeout(
+        _ptr(x), _xdt(x), M, K, _ptr(packed), float(gamma), N, _ptr(y), _ptr(workspace),
+        workspace.numel(), _stream(stream), int(timeout_us)))
+
+
+def bitlinear_get_fault(stream=None) -> tuple[int, int]:
+    """(status, fault word); synchronises the stream and clears the word."""
+    word = ctypes.c_int(0)
+    rc = lib().bitlinear_get_fault(ctypes.addressof(word), _stream(stream))
+    return int(rc), int(word.value)
+
+
+def bitlinear_int8_gemm(A, B, C=None, stream=None):
+    """C (int32 [M][N]) = A (int8 [M][K]) @ B (int8 [N][K])^T on the tensor cores."""
+    import torch
+    M, K = A.shape
+    N = B.shape[0]
+    if C is None:
+        C = torch.empty((M, N), dtype=torch.int32, device=A.device)
+    _check(lib().bitlinear_int8_gemm(_ptr(A), _ptr(B), _ptr(C), M, N, K, _stream(stream)),
+           "bitlinear_int8_gemm")
+    return C

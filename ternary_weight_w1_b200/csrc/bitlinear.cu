@@ -1,0 +1,458 @@
+// C ABI of libbitlinear (declared in include/bitlinear.h): argument checks,
+// kernel choice and launches of the BitLinear W1.58A8 matmul on sm_100a.
+//
+// All kernels live in this translation unit so that they share the device
+// fault word; the offline packer is host code in pack.cpp.
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <atomic>
+#include <climits>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/bitlinear.h"
+#include "common.cuh"
+#include "gemm_tc.cuh"
+#include "gemv.cuh"
+#include "quant_act.cuh"
+
+using namespace bitlinear;
+
+namespace {
+
+constexpr int64_t kMaxK = 65536;
+constexpr int kGemvMaxM = 16;
+constexpr int64_t kGemvMaxXqBytes = 196608;       // M * K bytes of x~ in shared memory
+constexpr int64_t kAutoGemvMaxM = 16;
+constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s: far above any legitimate wait
+constexpr int kMaxDevices = 64;
+
+bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+struct DeviceInfo {
+    int id = 0;
+    int sms = 0;
+    int max_smem_optin = 0;
+};
+
+DeviceInfo g_devices[kMaxDevices];
+std::once_flag g_device_once[kMaxDevices];
+
+int current_device(DeviceInfo **info)
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
+        return BITLINEAR_ERR_CUDA;
+    std::call_once(g_device_once[dev], [dev] {
+        g_devices[dev].id = dev;
+        cudaDeviceGetAttribute(&g_devices[dev].sms, cudaDevAttrMultiProcessorCount, dev);
+        cudaDeviceGetAttribute(&g_devices[dev].max_smem_optin,
+                               cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+    });
+    *info = &g_devices[dev];
+    return g_devices[dev].sms > 0 ? BITLINEAR_OK : BITLINEAR_ERR_CUDA;
+}
+
+// Opt a kernel into more than 48 KiB of dynamic shared memory. The attribute
+// is per function and device; it is set once (and raised when a larger size
+// is needed) so that launches inside a stream capture make no such call.
+template <auto Kernel>
+cudaError_t allow_smem(int dev, int bytes)
+{
+    static std::atomic<int> granted[kMaxDevices];
+    if (bytes <= 48 * 1024 || granted[dev].load(std::memory_order_acquire) >= bytes)
+        return cudaSuccess;
+    cudaError_t e =
+        cudaFuncSetAttribute(Kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess) {
+        int cur = granted[dev].load();
+        while (cur < bytes && !granted[dev].compare_exchange_weak(cur, bytes)) {
+        }
+    }
+    return e;
+}
+
+// ------------------------------------------------------------ tensor maps
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                   const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                   const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn()
+{
+    static EncodeTiledFn fn = [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) !=
+                cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            return static_cast<EncodeTiledFn>(nullptr);
+        return reinterpret_cast<EncodeTiledFn>(p);
+    }();
+    return fn;
+}
+
+// 2-D uint8 tensor [rows][cols] (cols contiguous), box [box_rows][box_cols].
+bool make_map_u8(CUtensorMap *map, const void *ptr, uint64_t rows, uint64_t cols,
+                 uint32_t box_rows, uint32_t box_cols, bool swizzle128)
+{
+    EncodeTiledFn fn = encode_fn();
+    if (fn == nullptr)
+        return false;
+    const cuuint64_t dims[2] = {cols, rows};
+    const cuuint64_t strides[1] = {cols};
+    const cuuint32_t box[2] = {box_cols, box_rows};
+    const cuuint32_t estride[2] = {1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(ptr), dims, strides,
+                    box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                    swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+int launch_status(cudaError_t e)
+{
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return BITLINEAR_ERR_CUDA;
+    }
+    return cudaGetLastError() == cudaSuccess ? BITLINEAR_OK : BITLINEAR_ERR_CUDA;
+}
+
+// ----------------------------------------------------------- quantisation
+
+int launch_quant_act(const void *x, bitlinear_dtype xdt, int M, int K, int8_t *xq, float *beta,
+                     int *rowsum, cudaStream_t st)
+{
+    if (M == 0)
+        return BITLINEAR_OK;
+    if (xdt == BITLINEAR_BF16)
+        qa::quant_act_kernel<true><<<M, qa::THREADS, 0, st>>>(x, K, xq, beta, rowsum);
+    else
+        qa::quant_act_kernel<false><<<M, qa::THREADS, 0, st>>>(x, K, xq, beta, rowsum);
+    return launch_status(cudaSuccess);
+}
+
+// ------------------------------------------------------------------- GEMV
+
+template <int MT, bool BF16, int DEPTH>
+int launch_gemv_t(const gemv::Params &p, int grid, int smem, int dev, cudaStream_t st)
+{
+    cudaError_t e = allow_smem<gemv::gemv_kernel<MT, BF16, DEPTH>>(dev, smem);
+    if (e != cudaSuccess)
+        return launch_status(e);
+    gemv::gemv_kernel<MT, BF16, DEPTH><<<grid, gemv::THREADS, smem, st>>>(p);
+    return launch_status(cudaSuccess);
+}
+
+template <int MT>
+int launch_gemv_mt(const gemv::Params &p, bool bf16, int grid, int smem, bool deep, int dev,
+                   cudaStream_t st)
+{
+    if (bf16)
+        return deep ? launch_gemv_t<MT, true, 16>(p, grid, smem, dev, st)
+                    : launch_gemv_t<MT, true, 8>(p, grid, smem, dev, st);
+    return deep ? launch_gemv_t<MT, false, 16>(p, grid, smem, dev, st)
+                : launch_gemv_t<MT, false, 8>(p, grid, smem, dev, st);
+}
+
+int launch_gemv(const void *x, bitlinear_dtype xdt, int M, int K, const void *packed,
+                float gamma, int N, void *y, int32_t *acc, int8_t *xq, float *beta,
+                const DeviceInfo &dev, cudaStream_t st)
+{
+    const int MT = M <= 1 ? 1 : M <= 2 ? 2 : M <= 4 ? 4 : M <= 8 ? 8 : 16;
+    // Two blocks per SM when the shared memory allows it, else one block with
+    // deeper per-lane prefetch; never more blocks than rows.
+    int per_sm = 2;
+    int grid = 0, smem = 0;
+    for (;; --per_sm) {
+        grid = static_cast<int>(std::min<int64_t>(static_cast<int64_t>(dev.sms) * per_sm, N));
+        const int rows_cap = (N + grid - 1) / grid;
+        smem = gemv::smem_bytes(MT, K, rows_cap);
+        if (per_sm == 1 || smem * per_sm <= 220 * 1024)
+            break;
+    }
+    if (smem > dev.max_smem_optin)
+        return BITLINEAR_ERR_SHAPE;
+    gemv::Params p{x, static_cast<const uint8_t *>(packed), static_cast<uint16_t *>(y), acc, xq,
+                   beta, M, K, N, gamma};
+    const bool bf16 = xdt == BITLINEAR_BF16;
+    const bool deep = per_sm == 1;
+    switch (MT) {
+    case 1: return launch_gemv_mt<1>(p, bf16, grid, smem, deep, dev.id, st);
+    case 2: return launch_gemv_mt<2>(p, bf16, grid, smem, deep, dev.id, st);
+    case 4: return launch_gemv_mt<4>(p, bf16, grid, smem, deep, dev.id, st);
+    case 8: return launch_gemv_mt<8>(p, bf16, grid, smem, deep, dev.id, st);
+    default: return launch_gemv_mt<16>(p, bf16, grid, smem, deep, dev.id, st);
+    }
+}
+
+// ------------------------------------------------------------ tensor cores
+
+struct TcWorkspace {
+    int8_t *xq;
+    float *beta;
+    int *rowsum;
+    size_t bytes;
+};
+
+size_t tc_workspace_bytes(int64_t M, int64_t K)
+{
+    return round_up(static_cast<size_t>(M) * static_cast<size_t>(K), 256) +
+           2 * round_up(static_cast<size_t>(M) * 4, 256);
+}
+
+TcWorkspace tc_workspace(void *ws, int64_t M, int64_t K)
+{
+    char *b = static_cast<char *>(ws);
+    const size_t a = round_up(static_cast<size_t>(M) * static_cast<size_t>(K), 256);
+    const size_t c = round_up(static_cast<size_t>(M) * 4, 256);
+    return {reinterpret_cast<int8_t *>(b), reinterpret_cast<float *>(b + a),
+            reinterpret_cast<int *>(b + a + c), a + 2 * c};
+}
+
+template <bool B_PACKED, bool RESCALE>
+int launch_gemm(const CUtensorMap &ma, const CUtensorMap &mb, const tc::Params &p,
+                const DeviceInfo &dev, cudaStream_t st)
+{
+    cudaError_t e = allow_smem<tc::gemm_kernel<B_PACKED, RESCALE>>(dev.id, tc::SMEM_BYTES);
+    if (e != cudaSuccess)
+        return launch_status(e);
+    const int tiles = ((p.M + tc::BM - 1) / tc::BM) * ((p.N + tc::BN - 1) / tc::BN);
+    const int grid = std::min(tiles, dev.sms);
+    tc::gemm_kernel<B_PACKED, RESCALE><<<grid, tc::THREADS, tc::SMEM_BYTES, st>>>(ma, mb, p);
+    return launch_status(cudaSuccess);
+}
+
+int run_tc_path(const void *x, bitlinear_dtype xdt, int M, int K, const void *packed,
+                float gamma, int N, void *y, void *ws, size_t ws_bytes, int32_t *acc,
+                int8_t *xq_dbg, float *beta_dbg, const DeviceInfo &dev, cudaStream_t st,
+                int inject_timeout_us)
+{
+    const size_t need = tc_workspace_bytes(M, K);
+    if (ws == nullptr || ws_bytes < need)
+        return BITLINEAR_ERR_WORKSPACE;
+    if (!aligned(ws, 256))
+        return BITLINEAR_ERR_ALIGN;
+    TcWorkspace w = tc_workspace(ws, M, K);
+    int rc = launch_quant_act(x, xdt, M, K, w.xq, w.beta, w.rowsum, st);
+    if (rc != BITLINEAR_OK)
+        return rc;
+    CUtensorMap ma, mb;
+    if (!make_map_u8(&ma, w.xq, M, K, tc::BM, tc::BK, true) ||
+        !make_map_u8(&mb, packed, N, K / 4, tc::BN, tc::BK / 4, false))
+        return BITLINEAR_ERR_CUDA;
+    tc::Params p{M, N, K, gamma, w.beta, w.rowsum, static_cast<uint16_t *>(y), acc,
+                 inject_timeout_us > 0 ? static_cast<uint64_t>(inject_timeout_us) * 1000ull
+                                       : kWaitLimitNs,
+                 inject_timeout_us > 0 ? 1 : 0};
+    rc = launch_gemm<true, true>(ma, mb, p, dev, st);
+    if (rc != BITLINEAR_OK)
+        return rc;
+    if (xq_dbg != nullptr &&
+        cudaMemcpyAsync(xq_dbg, w.xq, static_cast<size_t>(M) * K, cudaMemcpyDeviceToDevice, st) !=
+            cudaSuccess)
+        return BITLINEAR_ERR_CUDA;
+    if (beta_dbg != nullptr &&
+        cudaMemcpyAsync(beta_dbg, w.beta, static_cast<size_t>(M) * 4, cudaMemcpyDeviceToDevice,
+                        st) != cudaSuccess)
+        return BITLINEAR_ERR_CUDA;
+    return BITLINEAR_OK;
+}
+
+// --------------------------------------------------------------- checks
+
+int check_forward_args(const void *x, int xdt, int64_t M, int64_t K, const void *packed,
+                       int64_t N, const void *y, const int32_t *acc, const int8_t *xq,
+                       const float *beta)
+{
+    if (M < 0 || N < 1 || K < 1)
+        return BITLINEAR_ERR_ARG;
+    if (M > 0 && (x == nullptr || packed == nullptr || y == nullptr))
+        return BITLINEAR_ERR_ARG;
+    if (xdt != BITLINEAR_BF16 && xdt != BITLINEAR_FP32)
+        return BITLINEAR_ERR_DTYPE;
+    if (K % 128 != 0 || K > kMaxK || N > INT_MAX / 2 || M > INT_MAX / 2 ||
+        M * K > (int64_t(1) << 40))
+        return BITLINEAR_ERR_SHAPE;
+    if (!aligned(x, 16) || !aligned(packed, 16) || !aligned(y, 16) || !aligned(xq, 16) ||
+        !aligned(acc, 4) || !aligned(beta, 4))
+        return BITLINEAR_ERR_ALIGN;
+    return BITLINEAR_OK;
+}
+
+bool gemv_fits(int64_t M, int64_t K) { return M <= kGemvMaxM && M * K <= kGemvMaxXqBytes; }
+
+int choose_path(int64_t M, int64_t K, int path)
+{
+    if (path == BITLINEAR_PATH_GEMV || path == BITLINEAR_PATH_TC)
+        return path;
+    return (M <= kAutoGemvMaxM && gemv_fits(M, K)) ? BITLINEAR_PATH_GEMV : BITLINEAR_PATH_TC;
+}
+
+int forward_impl(const void *x, bitlinear_dtype xdt, int64_t M, int64_t K, const void *packed,
+                 float gamma, int64_t N, void *y, void *ws, size_t ws_bytes, void *stream,
+                 int32_t *acc, int8_t *xq, float *beta, int path, int inject_timeout_us)
+{
+    int rc = check_forward_args(x, xdt, M, K, packed, N, y, acc, xq, beta);
+    if (rc != BITLINEAR_OK)
+        return rc;
+    if (path < BITLINEAR_PATH_AUTO || path > BITLINEAR_PATH_TC)
+        return BITLINEAR_ERR_ARG;
+    if (M == 0)
+        return BITLINEAR_OK;
+    DeviceInfo *dev = nullptr;
+    rc = current_device(&dev);
+    if (rc != BITLINEAR_OK)
+        return rc;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const int chosen = inject_timeout_us > 0 ? BITLINEAR_PATH_TC : choose_path(M, K, path);
+    if (chosen == BITLINEAR_PATH_GEMV) {
+        if (!gemv_fits(M, K))
+            return BITLINEAR_ERR_SHAPE;
+        return launch_gemv(x, xdt, static_cast<int>(M), static_cast<int>(K), packed, gamma,
+                           static_cast<int>(N), y, acc, xq, beta, *dev, st);
+    }
+    return run_tc_path(x, xdt, static_cast<int>(M), static_cast<int>(K), packed, gamma,
+                       static_cast<int>(N), y, ws, ws_bytes, acc, xq, beta, *dev, st,
+                       inject_timeout_us);
+}
+
+}  // namespace
+
+// ================================================================== C ABI
+
+extern "C" const char *bitlinear_status_string(int status)
+{
+    switch (status) {
+    case BITLINEAR_OK: return "ok";
+    case BITLINEAR_ERR_ARG: return "invalid argument";
+    case BITLINEAR_ERR_SHAPE: return "unsupported shape";
+    case BITLINEAR_ERR_ALIGN: return "misaligned pointer";
+    case BITLINEAR_ERR_DTYPE: return "unsupported dtype";
+    case BITLINEAR_ERR_CUDA: return "CUDA error";
+    case BITLINEAR_ERR_TIMEOUT: return "device wait timed out";
+    case BITLINEAR_ERR_WORKSPACE: return "workspace missing or too small";
+    default: return "unknown status";
+    }
+}
+
+extern "C" int bitlinear_quant_act(const void *x_dev, bitlinear_dtype xdt, int64_t M, int64_t K,
+                                   int8_t *xq_dev, float *beta_dev, void *cuda_stream)
+{
+    if (M < 0 || K < 1)
+        return BITLINEAR_ERR_ARG;
+    if (M > 0 && (x_dev == nullptr || xq_dev == nullptr || beta_dev == nullptr))
+        return BITLINEAR_ERR_ARG;
+    if (xdt != BITLINEAR_BF16 && xdt != BITLINEAR_FP32)
+        return BITLINEAR_ERR_DTYPE;
+    if (K % 128 != 0 || K > (int64_t(1) << 30) || M > INT_MAX)
+        return BITLINEAR_ERR_SHAPE;
+    if (!aligned(x_dev, 16) || !aligned(xq_dev, 16) || !aligned(beta_dev, 4))
+        return BITLINEAR_ERR_ALIGN;
+    return launch_quant_act(x_dev, xdt, static_cast<int>(M), static_cast<int>(K), xq_dev,
+                            beta_dev, nullptr, static_cast<cudaStream_t>(cuda_stream));
+}
+
+extern "C" size_t bitlinear_workspace_bytes_path(int64_t M, int64_t N, int64_t K, int path)
+{
+    if (M < 0 || N < 1 || K < 1 || K % 128 != 0 || K > kMaxK)
+        return SIZE_MAX;
+    if (path < BITLINEAR_PATH_AUTO || path > BITLINEAR_PATH_TC)
+        return SIZE_MAX;
+    if (M == 0)
+        return 0;
+    return choose_path(M, K, path) == BITLINEAR_PATH_GEMV ? 0 : tc_workspace_bytes(M, K);
+}
+
+extern "C" size_t bitlinear_workspace_bytes(int64_t M, int64_t N, int64_t K)
+{
+    return bitlinear_workspace_bytes_path(M, N, K, BITLINEAR_PATH_AUTO);
+}
+
+extern "C" int bitlinear_forward(const void *x_dev, bitlinear_dtype xdt, int64_t M, int64_t K,
+                                 const void *packed_dev, float gamma, int64_t N, void *y_dev,
+                                 void *workspace_dev, size_t workspace_bytes, void *cuda_stream,
+                                 int32_t *acc_dev_or_null, int8_t *xq_dev_or_null,
+                                 float *beta_dev_or_null)
+{
+    return forward_impl(x_dev, xdt, M, K, packed_dev, gamma, N, y_dev, workspace_dev,
+                        workspace_bytes, cuda_stream, acc_dev_or_null, xq_dev_or_null,
+                        beta_dev_or_null, BITLINEAR_PATH_AUTO, 0);
+}
+
+extern "C" int bitlinear_forward_ex(const void *x_dev, bitlinear_dtype xdt, int64_t M, int64_t K,
+                                    const void *packed_dev, float gamma, int64_t N, void *y_dev,
+                                    void *workspace_dev, size_t workspace_bytes,
+                                    void *cuda_stream, int32_t *acc_dev_or_null,
+                                    int8_t *xq_dev_or_null, float *beta_dev_or_null, int path)
+{
+    return forward_impl(x_dev, xdt, M, K, packed_dev, gamma, N, y_dev, workspace_dev,
+                        workspace_bytes, cuda_stream, acc_dev_or_null, xq_dev_or_null,
+                        beta_dev_or_null, path, 0);
+}
+
+extern "C" int bitlinear_forward_inject_timeout(const void *x_dev, bitlinear_dtype xdt, int64_t M,
+                                                int64_t K, const void *packed_dev, float gamma,
+                                                int64_t N, void *y_dev, void *workspace_dev,
+                                                size_t workspace_bytes, void *cuda_stream,
+                                                int timeout_us)
+{
+    if (timeout_us < 1 || timeout_us > 10 * 1000 * 1000)
+        return BITLINEAR_ERR_ARG;
+    return forward_impl(x_dev, xdt, M, K, packed_dev, gamma, N, y_dev, workspace_dev,
+                        workspace_bytes, cuda_stream, nullptr, nullptr, nullptr,
+                        BITLINEAR_PATH_TC, timeout_us);
+}
+
+extern "C" int bitlinear_get_fault(int *fault_out, void *cuda_stream)
+{
+    if (fault_out == nullptr)
+        return BITLINEAR_ERR_ARG;
+    if (cudaStreamSynchronize(static_cast<cudaStream_t>(cuda_stream)) != cudaSuccess)
+        return BITLINEAR_ERR_CUDA;
+    unsigned int word = 0;
+    if (cudaMemcpyFromSymbol(&word, g_fault_word, sizeof(word)) != cudaSuccess)
+        return BITLINEAR_ERR_CUDA;
+    *fault_out = static_cast<int>(word);
+    if (word != 0) {
+        const unsigned int zero = 0;
+        if (cudaMemcpyToSymbol(g_fault_word, &zero, sizeof(zero)) != cudaSuccess)
+            return BITLINEAR_ERR_CUDA;
+        return BITLINEAR_ERR_TIMEOUT;
+    }
+    return BITLINEAR_OK;
+}
+
+extern "C" int bitlinear_int8_gemm(const int8_t *A_dev, const int8_t *B_dev, int32_t *C_dev,
+                                   int64_t M, int64_t N, int64_t K, void *cuda_stream)
+{
+    if (M < 0 || N < 1 || K < 1)
+        return BITLINEAR_ERR_ARG;
+    if (M > 0 && (A_dev == nullptr || B_dev == nullptr || C_dev == nullptr))
+        return BITLINEAR_ERR_ARG;
+    if (K % 128 != 0 || M > INT_MAX / 2 || N > INT_MAX / 2 || K > (int64_t(1) << 30))
+        return BITLINEAR_ERR_SHAPE;
+    if (!aligned(A_dev, 16) || !aligned(B_dev, 16) || !aligned(C_dev, 16))
+        return BITLINEAR_ERR_ALIGN;
+    if (M == 0)
+        return BITLINEAR_OK;
+    DeviceInfo *dev = nullptr;
+    int rc = current_device(&dev);
+    if (rc != BITLINEAR_OK)
+        return rc;
+    CUtensorMap ma, mb;
+    if (!make_map_u8(&ma, A_dev, M, K, tc::BM, tc::BK, true) ||
+        !make_map_u8(&mb, B_dev, N, K, tc::BN, tc::BK, true))
+        return BITLINEAR_ERR_CUDA;
+    tc::Params p{static_cast<int>(M), static_cast<int>(N), static_cast<int>(K), 0.0f, nullptr,
+                 nullptr, nullptr, C_dev, kWaitLimitNs, 0};
+    return launch_gemm<false, false>(ma, mb, p, *dev, static_cast<cudaStream_t>(cuda_stream));
+}

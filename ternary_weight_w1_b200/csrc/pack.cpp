@@ -1,0 +1,127 @@
+// Offline absmean ternarisation and 2-bit packing of BitLinear weights (host).
+//
+// Page "BitNet b1.58 2B4T Guide: Scaling Native 1-Bit LLMs", section "Ternary
+// Weight Quantization: absmean Scaling": gamma is the mean of |W| over the
+// whole d_out x d_in matrix and each weight becomes Clip(Round(W / gamma), -1,
+// 1); the page's listing (WeightQuantFunction.forward) clamps gamma at 1e-5,
+// divides in the weight dtype (fp32 here) and rounds half to even. The codes
+// are stored two bits each in the layout documented in include/bitlinear.h.
+//
+// The mean is accumulated in double over fixed 1 Mi-element blocks whose sums
+// are added in block order, so gamma does not depend on the thread count.
+// Must be compiled without fast-math (IEEE division and rounding).
+
+#include <algorithm>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <thread>
+#include <vector>
+
+#include "../../include/bitlinear.h"
+
+namespace {
+
+constexpr float kEps = 1e-5f;
+constexpr int64_t kBlock = int64_t(1) << 20;
+
+unsigned worker_count(int64_t work_items)
+{
+    unsigned hw = std::thread::hardware_concurrency();
+    if (hw == 0)
+        hw = 1;
+    hw = std::min(hw, 32u);
+    int64_t useful = std::max<int64_t>(1, work_items);
+    return static_cast<unsigned>(std::min<int64_t>(hw, useful));
+}
+
+template <class Fn>
+void parallel_for(int64_t count, Fn fn)
+{
+    const unsigned workers = worker_count(count);
+    if (workers <= 1) {
+        for (int64_t i = 0; i < count; ++i)
+            fn(i);
+        return;
+    }
+    std::vector<std::thread> pool;
+    pool.reserve(workers);
+    for (unsigned t = 0; t < workers; ++t) {
+        pool.emplace_back([=, &fn] {
+            for (int64_t i = t; i < count; i += workers)
+                fn(i);
+        });
+    }
+    for (auto &th : pool)
+        th.join();
+}
+
+// Ternary code (W~ + 1) of one latent weight.
+inline uint32_t ternary_code(float w, float gamma)
+{
+    float r = std::nearbyint(w / gamma);  // default rounding mode: ties to even
+    if (r > 1.0f)
+        r = 1.0f;
+    else if (r < -1.0f)
+        r = -1.0f;
+    return static_cast<uint32_t>(static_cast<int>(r) + 1);
+}
+
+}  // namespace
+
+extern "C" size_t bitlinear_packed_bytes(int64_t N, int64_t K)
+{
+    if (N < 1 || K < 16 || K % 16 != 0)
+        return 0;
+    return static_cast<size_t>(N) * static_cast<size_t>(K / 4);
+}
+
+extern "C" int bitlinear_pack_weights(const float *W_host, int64_t N,
+                                      int64_t K, void *packed_host,
+                                      float *gamma_out)
+{
+    if (!W_host || !packed_host || !gamma_out || N < 1 || K < 0)
+        return BITLINEAR_ERR_ARG;
+    if (K < 16 || K % 16 != 0)
+        return BITLINEAR_ERR_SHAPE;
+
+    // gamma = mean |W| (double accumulation in fixed blocks, then one cast).
+    const int64_t total = N * K;
+    const int64_t blocks = (total + kBlock - 1) / kBlock;
+    std::vector<double> partial(static_cast<size_t>(blocks), 0.0);
+    parallel_for(blocks, [&](int64_t b) {
+        const int64_t lo = b * kBlock;
+        const int64_t hi = std::min(total, lo + kBlock);
+        double s = 0.0;
+        for (int64_t i = lo; i < hi; ++i)
+            s += std::fabs(static_cast<double>(W_host[i]));
+        partial[static_cast<size_t>(b)] = s;
+    });
+    double sum = 0.0;
+    for (double s : partial)
+        sum += s;
+    float gamma = static_cast<float>(sum / static_cast<double>(total));
+    if (!(gamma >= kEps))
+        gamma = kEps;
+
+    // Encode row by row: word w of row n collects k = 16w + 4j + b at bit
+    // 8b + 2j.
+    uint8_t *out = static_cast<uint8_t *>(packed_host);
+    const int64_t words = K / 16;
+    parallel_for(N, [&](int64_t n) {
+        const float *row = W_host + n * K;
+        uint8_t *dst = out + n * (K / 4);
+        for (int64_t w = 0; w < words; ++w) {
+            const float *src = row + 16 * w;
+            uint32_t word = 0;
+            for (int k = 0; k < 16; ++k) {
+                const int j = k >> 2;
+                const int b = k & 3;
+                word |= ternary_code(src[k], gamma) << (8 * b + 2 * j);
+            }
+            std::memcpy(dst + 4 * w, &word, 4);  // little-endian host
+        }
+    });
+    *gamma_out = gamma;
+    return BITLINEAR_OK;
+}

@@ -1,0 +1,136 @@
+"""Shared machinery of the GPU parity tests: build one BitLinear problem from
+the seeded generators, run the CUDA library through its C ABI, run the
+oracle on the same inputs, and compare stage by stage.
+
+Bar (see the design notes): x~, beta and acc bit-exact; y within relative
+error 1e-2 elementwise (y_oracle == 0 requires y == 0). The kernels follow
+the oracle's operation order, so y is also expected to be bit-identical and
+the helpers report how many elements are.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+import oracle
+import workloads
+import ternary_weight_w1_b200 as bl
+
+Y_REL_TOL = 1e-2
+
+
+def bf16_bits_to_tensor(bits: np.ndarray, device="cuda"):
+    import torch
+    return torch.from_numpy(bits.view(np.int16).copy()).view(torch.bfloat16).to(device)
+
+
+def tensor_to_bf16_bits(t) -> np.ndarray:
+    import torch
+    return t.contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
+
+
+def bf16_value(bits: np.ndarray) -> np.ndarray:
+    return (bits.astype(np.uint32) << 16).view(np.float32)
+
+
+class Case:
+    """One problem: inputs, the packed weights and the oracle's view of them."""
+
+    def __init__(self, M, K, N, w_seed=1, x_seed=2, x_dtype="bf16", outliers=True,
+                 W=None, x=None):
+        self.M, self.K, self.N = M, K, N
+        self.W = workloads.latent_weights(N, K, w_seed) if W is None else W
+        xf = workloads.activations_f32(M, K, x_seed, outliers) if x is None else x
+        self.x_dtype = x_dtype
+        if x_dtype == "bf16":
+            self.x_bits = workloads.to_bf16_bits(xf)
+            self.orc = oracle.default()
+            self.xf = self.orc.bf16_to_f32(self.x_bits)
+        else:
+            self.orc = oracle.default()
+            self.xf = np.ascontiguousarray(xf, dtype=np.float32)
+        self.packed, self.gamma = bl.bitlinear_pack_weights(self.W)
+        # the oracle ternarises with the packer's gamma (checked separately)
+        self.Wq = self.orc.ternarize(self.W, np.float32(self.gamma))
+        self.xq, self.beta = self.orc.quant_act(self.xf)
+
+    def x_tensor(self):
+        import torch
+        if self.x_dtype == "bf16":
+            return bf16_bits_to_tensor(self.x_bits)
+        return torch.from_numpy(self.xf).cuda()
+
+    def packed_tensor(self):
+        import torch
+        return torch.from_numpy(self.packed).cuda()
+
+    def run(self, path=bl.PATH_AUTO, debug=True):
+        import torch
+        x = self.x_tensor()
+        packed = self.packed_tensor()
+        dev = x.device
+        y = torch.empty((self.M, self.N), dtype=torch.bfloat16, device=dev)
+        acc = torch.full((self.M, self.N), -7, dtype=torch.int32, device=dev) if debug else None
+        xq = torch.full((self.M, self.K), 99, dtype=torch.int8, device=dev) if debug else None
+        beta = torch.full((self.M,), -1.0, dtype=torch.float32, device=dev) if debug else None
+        bl.bitlinear_forward(x, packed, self.gamma, self.N, y=y, acc=acc, xq=xq, beta=beta,
+                             path=path)
+        torch.cuda.synchronize()
+        out = {"y": tensor_to_bf16_bits(y)}
+        if debug:
+            out["acc"] = acc.cpu().numpy()
+            out["xq"] = xq.cpu().numpy()
+            out["beta"] = beta.cpu().numpy()
+        return out
+
+    # ---------------------------------------------------------- checks
+
+    def oracle_full(self):
+        acc = self.orc.matmul_i32(self.xq, self.Wq)
+        y = self.orc.rescale_bf16(acc, self.beta, np.float32(self.gamma))
+        return acc, y
+
+    def check_quant(self, got):
+        np.testing.assert_array_equal(got["beta"], self.beta)
+        np.testing.assert_array_equal(got["xq"], self.xq)
+
+    def check_full(self, got):
+        self.check_quant(got)
+        acc, y = self.oracle_full()
+        np.testing.assert_array_equal(got["acc"], acc)
+        return check_y(got["y"], y)
+
+    def sample_pairs(self, count, seed=0, full_rows=2, full_cols=2):
+        r = np.random.Generator(np.random.PCG64(seed))
+        ms = [r.integers(0, self.M, count)]
+        ns = [r.integers(0, self.N, count)]
+        for m in r.integers(0, self.M, full_rows):
+            ms.append(np.full(self.N, m))
+            ns.append(np.arange(self.N))
+        for n in r.integers(0, self.N, full_cols):
+            ms.append(np.arange(self.M))
+            ns.append(np.full(self.M, n))
+        ms.append(np.array([self.M - 1])); ns.append(np.array([self.N - 1]))
+        return np.concatenate(ms).astype(np.int64), np.concatenate(ns).astype(np.int64)
+
+    def check_sampled(self, got, count=20000, seed=0):
+        self.check_quant(got)
+        ms, ns = self.sample_pairs(count, seed)
+        acc = self.orc.matmul_i32_pairs(self.xq, self.Wq, ms, ns)
+        np.testing.assert_array_equal(got["acc"][ms, ns], acc)
+        # the oracle's rescale, one sampled output per "row"
+        y_ref = self.orc.rescale_bf16(acc.reshape(-1, 1), self.beta[ms],
+                                      np.float32(self.gamma))[:, 0]
+        return check_y(got["y"][ms, ns], y_ref)
+
+
+def check_y(y_bits: np.ndarray, y_ref_bits: np.ndarray) -> float:
+    """Relative-error check of bf16 outputs; returns the fraction of
+    bit-identical elements."""
+    y = bf16_value(y_bits).astype(np.float64)
+    r = bf16_value(y_ref_bits).astype(np.float64)
+    assert np.all(np.isfinite(y))
+    zero = r == 0
+    assert np.all(y[zero] == 0)
+    rel = np.abs(y[~zero] - r[~zero]) / np.abs(r[~zero])
+    assert rel.size == 0 or rel.max() <= Y_REL_TOL, float(rel.max())
+    return float(np.mean(y_bits == y_ref_bits))

@@ -1,0 +1,118 @@
+"""The C ABI library loads, exports every symbol include/bitlinear.h
+declares, and rejects bad arguments on the host (no device work: every check
+here returns before the library touches CUDA)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import ternary_weight_w1_b200 as bl
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))),
+                      "include", "bitlinear.h")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(bitlinear_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_declares_the_binding_exports():
+    assert declared_functions() == sorted(bl.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol():
+    L = bl.lib()
+    for name in declared_functions():
+        assert hasattr(L, name), name
+
+
+def test_status_strings():
+    assert bl.status_string(bl.BITLINEAR_OK) == "ok"
+    assert bl.status_string(bl.BITLINEAR_ERR_TIMEOUT) == "device wait timed out"
+    assert bl.status_string(99) == "unknown status"
+
+
+def test_packed_bytes():
+    assert bl.bitlinear_packed_bytes(6912, 2560) == 6912 * 640
+    assert bl.bitlinear_packed_bytes(1, 16) == 4
+    assert bl.bitlinear_packed_bytes(0, 256) == 0
+    assert bl.bitlinear_packed_bytes(4, 24) == 0
+
+
+def test_workspace_bytes():
+    assert bl.bitlinear_workspace_bytes(1, 6912, 2560) == 0          # GEMV
+    assert bl.bitlinear_workspace_bytes(2048, 6912, 2560) >= 2048 * 2560 + 2 * 2048 * 4
+    assert bl.bitlinear_workspace_bytes(1, 6912, 2560, bl.PATH_TC) >= 2560 + 8
+    assert bl.bitlinear_workspace_bytes(4, 64, 100) == ctypes.c_size_t(-1).value
+    assert bl.bitlinear_workspace_bytes(0, 64, 256) == 0
+
+
+FAKE = 1 << 20          # a 16-byte-aligned non-null address; never dereferenced
+
+
+def fwd(**kw):
+    a = dict(x=FAKE, xdt=0, M=1, K=256, packed=FAKE, gamma=1.0, N=64, y=FAKE, ws=None,
+             wsb=0, stream=None, acc=None, xq=None, beta=None)
+    a.update(kw)
+    return bl.lib().bitlinear_forward(a["x"], a["xdt"], a["M"], a["K"], a["packed"], a["gamma"],
+                                      a["N"], a["y"], a["ws"], a["wsb"], a["stream"], a["acc"],
+                                      a["xq"], a["beta"])
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(x=None), bl.BITLINEAR_ERR_ARG),
+    (dict(packed=None), bl.BITLINEAR_ERR_ARG),
+    (dict(y=None), bl.BITLINEAR_ERR_ARG),
+    (dict(M=-1), bl.BITLINEAR_ERR_ARG),
+    (dict(N=0), bl.BITLINEAR_ERR_ARG),
+    (dict(K=200), bl.BITLINEAR_ERR_SHAPE),
+    (dict(K=64), bl.BITLINEAR_ERR_SHAPE),
+    (dict(K=65536 + 128), bl.BITLINEAR_ERR_SHAPE),
+    (dict(xdt=7), bl.BITLINEAR_ERR_DTYPE),
+    (dict(x=FAKE + 8), bl.BITLINEAR_ERR_ALIGN),
+    (dict(packed=FAKE + 4), bl.BITLINEAR_ERR_ALIGN),
+    (dict(y=FAKE + 2), bl.BITLINEAR_ERR_ALIGN),
+    (dict(xq=FAKE + 1), bl.BITLINEAR_ERR_ALIGN),
+    (dict(acc=FAKE + 2), bl.BITLINEAR_ERR_ALIGN),
+    (dict(M=0), bl.BITLINEAR_OK),                 # empty batch: nothing to do
+    (dict(M=0, x=None, y=None), bl.BITLINEAR_OK),
+])
+def test_forward_rejects_bad_arguments(kw, status):
+    assert fwd(**kw) == status
+
+
+def test_forward_ex_rejects_bad_path():
+    L = bl.lib()
+    rc = L.bitlinear_forward_ex(FAKE, 0, 1, 256, FAKE, 1.0, 64, FAKE, None, 0, None, None,
+                                None, None, 9)
+    assert rc == bl.BITLINEAR_ERR_ARG
+
+
+def test_quant_act_rejects_bad_arguments():
+    L = bl.lib()
+    assert L.bitlinear_quant_act(None, 0, 2, 256, FAKE, FAKE, None) == bl.BITLINEAR_ERR_ARG
+    assert L.bitlinear_quant_act(FAKE, 0, 2, 200, FAKE, FAKE, None) == bl.BITLINEAR_ERR_SHAPE
+    assert L.bitlinear_quant_act(FAKE, 3, 2, 256, FAKE, FAKE, None) == bl.BITLINEAR_ERR_DTYPE
+    assert L.bitlinear_quant_act(FAKE, 0, 2, 256, FAKE + 1, FAKE, None) == bl.BITLINEAR_ERR_ALIGN
+    assert L.bitlinear_quant_act(FAKE, 0, 0, 256, FAKE, FAKE, None) == bl.BITLINEAR_OK
+
+
+def test_int8_gemm_rejects_bad_arguments():
+    L = bl.lib()
+    assert L.bitlinear_int8_gemm(None, FAKE, FAKE, 4, 4, 128, None) == bl.BITLINEAR_ERR_ARG
+    assert L.bitlinear_int8_gemm(FAKE, FAKE, FAKE, 4, 4, 100, None) == bl.BITLINEAR_ERR_SHAPE
+    assert L.bitlinear_int8_gemm(FAKE, FAKE, FAKE + 4, 4, 4, 128, None) == bl.BITLINEAR_ERR_ALIGN
+
+
+def test_inject_timeout_rejects_bad_limit():
+    L = bl.lib()
+    rc = L.bitlinear_forward_inject_timeout(FAKE, 0, 1, 256, FAKE, 1.0, 64, FAKE, FAKE, 4096,
+                                            None, 0)
+    assert rc == bl.BITLINEAR_ERR_ARG
+
+
+def test_get_fault_rejects_null():
+    assert bl.lib().bitlinear_get_fault(None, None) == bl.BITLINEAR_ERR_ARG

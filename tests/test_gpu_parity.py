@@ -1,0 +1,214 @@
+"""Parity of the CUDA library (through its C ABI) with the CPU oracle.
+
+Small and mid sizes that span several tiles and ragged tails are compared
+element by element; the full-size workloads, in the launch configuration the
+benchmark uses (the automatic path), are compared on the full integer
+activation stage and on sampled outputs of the product.
+"""
+import numpy as np
+import pytest
+
+import workloads
+import ternary_weight_w1_b200 as bl
+from tests.gpu_cases import Case, bf16_bits_to_tensor, check_y
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def cuda():
+    import torch
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    bl.lib()
+    return torch
+
+
+# ------------------------------------------------------- quantisation kernel
+
+@pytest.mark.parametrize("M,K,dtype", [(4, 256, "fp32"), (1, 2560, "bf16"), (1, 6912, "bf16"),
+                                       (37, 1280, "bf16"), (300, 2560, "fp32"),
+                                       (2048, 6912, "bf16"), (3, 28672, "bf16"),
+                                       (5, 65536, "fp32")])
+def test_quant_act(cuda, M, K, dtype):
+    xf = workloads.activations_f32(M, K, seed=M * 31 + K)
+    xf[0, :] = 0.0                                           # an all-zero token
+    if M > 2:
+        xf[1, :] = -0.375                                    # a constant token
+    c = Case(M, K, 16, x=xf, x_dtype=dtype)
+    xq, beta = bl.bitlinear_quant_act(c.x_tensor())
+    cuda.cuda.synchronize()
+    np.testing.assert_array_equal(beta.cpu().numpy(), c.beta)
+    np.testing.assert_array_equal(xq.cpu().numpy(), c.xq)
+
+
+# -------------------------------------------------------------- GEMV path
+
+@pytest.mark.parametrize("M", [1, 2, 3, 4, 5, 8, 11, 16])
+@pytest.mark.parametrize("K,N", [(256, 256), (1280, 300), (2560, 640), (6912, 37), (128, 5)])
+def test_gemv_parity(cuda, M, K, N):
+    c = Case(M, K, N, w_seed=K + N, x_seed=M + 7 * K)
+    got = c.run(path=bl.PATH_GEMV)
+    exact = c.check_full(got)
+    assert exact == 1.0
+
+
+def test_gemv_fp32_input(cuda):
+    c = Case(4, 256, 256, w_seed=0, x_seed=0, x_dtype="fp32", outliers=False)
+    assert c.check_full(c.run(path=bl.PATH_GEMV)) == 1.0
+
+
+# ------------------------------------------------------ tensor-core path
+
+@pytest.mark.parametrize("M", [1, 100, 128, 129, 300])
+@pytest.mark.parametrize("K,N", [(256, 256), (1280, 333), (2560, 600), (128, 513)])
+def test_tc_parity(cuda, M, K, N):
+    c = Case(M, K, N, w_seed=3 * K + N, x_seed=M + 5 * K)
+    got = c.run(path=bl.PATH_TC)
+    exact = c.check_full(got)
+    assert exact == 1.0
+
+
+def test_tc_many_tiles_per_cta(cuda):
+    # more tiles than SMs: every CTA loops over several tiles and both TMEM
+    # accumulator buffers are reused
+    c = Case(1024, 512, 8192, w_seed=11, x_seed=12)
+    got = c.run(path=bl.PATH_TC)
+    assert c.check_sampled(got, count=50000) == 1.0
+
+
+def test_tc_fp32_input(cuda):
+    c = Case(200, 256, 256, w_seed=0, x_seed=0, x_dtype="fp32", outliers=False)
+    assert c.check_full(c.run(path=bl.PATH_TC)) == 1.0
+
+
+# ------------------------------------------------------------- edge cases
+
+@pytest.mark.parametrize("path", [bl.PATH_GEMV, bl.PATH_TC])
+def test_zero_activations_and_weights(cuda, path):
+    x = np.zeros((3, 256), dtype=np.float32)
+    c = Case(3, 256, 64, x=x)
+    got = c.run(path=path)
+    c.check_full(got)
+    assert np.all(got["y"] == 0) and np.all(got["beta"] == np.float32(1e-5))
+    W = np.zeros((64, 256), dtype=np.float32)
+    c2 = Case(3, 256, 64, W=W)
+    got2 = c2.run(path=path)
+    c2.check_full(got2)
+    assert np.all(got2["acc"] == 0)
+
+
+@pytest.mark.parametrize("path", [bl.PATH_GEMV, bl.PATH_TC])
+def test_identity_weights(cuda, path):
+    K = 256
+    c = Case(2, K, K, W=np.eye(K, dtype=np.float32))
+    got = c.run(path=path)
+    c.check_full(got)
+    np.testing.assert_array_equal(got["acc"], c.xq.astype(np.int32))
+
+
+def test_empty_batch_is_a_noop(cuda):
+    torch = cuda
+    x = torch.empty((0, 256), dtype=torch.bfloat16, device="cuda")
+    packed = torch.zeros((64, 64), dtype=torch.uint8, device="cuda")
+    y = torch.empty((0, 64), dtype=torch.bfloat16, device="cuda")
+    bl.bitlinear_forward(x, packed, 1.0, 64, y=y)
+    torch.cuda.synchronize()
+
+
+def test_deterministic(cuda):
+    c = Case(300, 1280, 700, w_seed=5, x_seed=6)
+    a = c.run(path=bl.PATH_TC)
+    b = c.run(path=bl.PATH_TC)
+    np.testing.assert_array_equal(a["y"], b["y"])
+    g1 = c.run(path=bl.PATH_AUTO, debug=False)
+    np.testing.assert_array_equal(a["y"], g1["y"])
+
+
+def test_paths_agree_at_m16(cuda):
+    c = Case(16, 2560, 1000, w_seed=8, x_seed=9)
+    a = c.run(path=bl.PATH_GEMV)
+    b = c.run(path=bl.PATH_TC)
+    np.testing.assert_array_equal(a["acc"], b["acc"])
+    np.testing.assert_array_equal(a["y"], b["y"])
+
+
+# ------------------------------------------------- full-size workloads
+
+def _problem_case(p):
+    return Case(p.M, p.K, p.N, w_seed=p.w_seed, x_seed=p.x_seed, x_dtype=p.x_dtype,
+                outliers=p.outliers)
+
+
+def test_tiny_workload(cuda):
+    for p in workloads.tiny().problems:
+        c = _problem_case(p)
+        assert c.check_full(c.run()) == 1.0
+
+
+def test_decode_gemv_2b(cuda):
+    for p in workloads.decode_gemv_2b().problems:
+        c = _problem_case(p)
+        assert c.check_full(c.run()) == 1.0
+
+
+@pytest.mark.parametrize("B", [1, 8, 64])
+def test_layer_set_2b(cuda, B):
+    wl = workloads.layer_set_2b(B)
+    first = wl.problems[:7]           # layer 0: every projection shape
+    last = wl.problems[-7:]           # layer 29
+    for p in first + last:
+        c = _problem_case(p)
+        got = c.run()
+        if B <= 8:
+            assert c.check_full(got) == 1.0
+        else:
+            assert c.check_sampled(got, count=5000) == 1.0
+
+
+def test_prefill_2b(cuda):
+    for p in workloads.prefill_2b().problems:
+        c = _problem_case(p)
+        assert c.check_sampled(c.run(), count=30000) == 1.0
+
+
+@pytest.mark.parametrize("M", [1, 16, 256, 4096])
+def test_large_sweep(cuda, M):
+    for p in workloads.large_sweep(M).problems:
+        c = _problem_case(p)
+        got = c.run()
+        if M == 1:
+            assert c.check_full(got) == 1.0
+        else:
+            assert c.check_sampled(got, count=20000) == 1.0
+
+
+# ------------------------------------------------- int8 GEMM (measurement aid)
+
+@pytest.mark.parametrize("M,N,K", [(300, 600, 512), (128, 256, 128), (1000, 2000, 1280)])
+def test_int8_gemm(cuda, M, N, K):
+    torch = cuda
+    r = np.random.Generator(np.random.PCG64(M + N + K))
+    A = r.integers(-128, 128, (M, K), dtype=np.int8)
+    B = r.integers(-128, 128, (N, K), dtype=np.int8)
+    C = bl.bitlinear_int8_gemm(torch.from_numpy(A).cuda(), torch.from_numpy(B).cuda())
+    torch.cuda.synchronize()
+    ref = A.astype(np.int64) @ B.astype(np.int64).T
+    np.testing.assert_array_equal(C.cpu().numpy().astype(np.int64), ref)
+
+
+# ------------------------------------------------- failure detection
+
+def test_bounded_wait_reports_timeout_and_context_survives(cuda):
+    torch = cuda
+    c = Case(256, 512, 512, w_seed=1, x_seed=1)
+    x = c.x_tensor()
+    packed = c.packed_tensor()
+    assert bl.bitlinear_get_fault() == (bl.BITLINEAR_OK, 0)
+    rc = bl.bitlinear_forward_inject_timeout(x, packed, c.gamma, c.N, timeout_us=2000)
+    assert rc == bl.BITLINEAR_OK
+    status, word = bl.bitlinear_get_fault()
+    assert status == bl.BITLINEAR_ERR_TIMEOUT and word == 1
+    # the word is cleared, and the context still runs correct work
+    assert bl.bitlinear_get_fault() == (bl.BITLINEAR_OK, 0)
+    assert c.check_full(c.run(path=bl.PATH_TC)) == 1.0
+    assert bl.bitlinear_get_fault() == (bl.BITLINEAR_OK, 0)
