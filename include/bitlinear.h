@@ -54,7 +54,8 @@ typedef enum {
     BITLINEAR_ERR_DTYPE = 4,     /* unknown bitlinear_dtype */
     BITLINEAR_ERR_CUDA = 5,      /* a CUDA runtime/driver call failed */
     BITLINEAR_ERR_TIMEOUT = 6,   /* a bounded device-side wait ran out */
-    BITLINEAR_ERR_WORKSPACE = 7  /* workspace missing or smaller than required */
+    BITLINEAR_ERR_WORKSPACE = 7, /* workspace missing or smaller than required */
+    BITLINEAR_ERR_SCRATCH_LIMIT = 8 /* problem too large for the library's static scratch */
 } bitlinear_status;
 
 typedef enum {
@@ -157,6 +158,35 @@ int bitlinear_forward_ex(const void *x_dev, bitlinear_dtype xdt, int64_t M,
 /* Workspace bytes for an explicit path (see bitlinear_forward_ex). */
 size_t bitlinear_workspace_bytes_path(int64_t M, int64_t N, int64_t K,
                                       int path);
+
+/* Bytes of the device array that bitlinear_forward_noalloc uses as scratch. */
+#define BITLINEAR_STATIC_SCRATCH_BYTES (16u << 20)
+
+/* bitlinear_forward on the tensor-core path, for callers that cannot
+ * allocate device memory themselves: for instance a plugin whose host hands
+ * it only the input and output pointers and offers no allocator or workspace,
+ * or a serving loop that forbids allocation once it has started. Nothing is
+ * allocated by anyone. The scratch the path needs (x~, beta and the per-token
+ * sums of x~) lives in one file-scope device array of
+ * BITLINEAR_STATIC_SCRATCH_BYTES (16 MiB) inside the library; every GPU that
+ * loads the library holds that array until the process exits.
+ * The paper has no counterpart of this call; it exists only for such callers.
+ *   x_dev, packed_dev, gamma, y_dev, cuda_stream: as for bitlinear_forward.
+ * Limits: M * K rounded up to 256 bytes, plus 2 * (4 * M rounded up to 256)
+ * bytes, must fit in BITLINEAR_STATIC_SCRATCH_BYTES; larger problems return
+ * BITLINEAR_ERR_SCRATCH_LIMIT before any device work (the largest M is
+ * 6533 for K = 2560, 2424 for K = 6912, 2046 for K = 8192, 584 for K = 28672).
+ * Set-up: the first call on a device (with that device current) looks up the
+ * array's device address once; make that first call before any stream
+ * capture.
+ * Sharing: every call on a device uses the same array and it keeps the last
+ * call's contents. Nothing in it needs to start at zero (each call writes
+ * every scratch byte it reads before reading it), but calls whose work
+ * overlaps on the GPU (different streams, or different host threads) race on
+ * the array: serialise them, e.g. on one stream. */
+int bitlinear_forward_noalloc(const void *x_dev, bitlinear_dtype xdt, int64_t M,
+                              int64_t K, const void *packed_dev, float gamma,
+                              int64_t N, void *y_dev, void *cuda_stream);
 
 /* ------------------------------------------------------------- diagnostics */
 

@@ -25,6 +25,8 @@ BITLINEAR_ERR_DTYPE = 4
 BITLINEAR_ERR_CUDA = 5
 BITLINEAR_ERR_TIMEOUT = 6
 BITLINEAR_ERR_WORKSPACE = 7
+BITLINEAR_ERR_SCRATCH_LIMIT = 8
+BITLINEAR_STATIC_SCRATCH_BYTES = 16 << 20
 
 BITLINEAR_BF16 = 0
 BITLINEAR_FP32 = 1
@@ -46,6 +48,7 @@ EXPORTS = (
     "bitlinear_status_string",
     "bitlinear_int8_gemm",
     "bitlinear_forward_inject_timeout",
+    "bitlinear_forward_noalloc",
 )
 
 _lib = None
@@ -84,6 +87,9 @@ def lib() -> ctypes.CDLL:
         L.bitlinear_forward_ex.argtypes = fwd + [ctypes.c_int]
         L.bitlinear_forward_inject_timeout.restype = ctypes.c_int
         L.bitlinear_forward_inject_timeout.argtypes = fwd[:11] + [ctypes.c_int]
+        L.bitlinear_forward_noalloc.restype = ctypes.c_int
+        L.bitlinear_forward_noalloc.argtypes = [p, ctypes.c_int, i64, i64, p, ctypes.c_float,
+                                                i64, p, p]
         L.bitlinear_get_fault.restype = ctypes.c_int
         L.bitlinear_get_fault.argtypes = [p, p]
         L.bitlinear_status_string.restype = ctypes.c_char_p
@@ -230,3 +236,18 @@ def bitlinear_int8_gemm(A, B, C=None, stream=None):
     _check(lib().bitlinear_int8_gemm(_ptr(A), _ptr(B), _ptr(C), M, N, K, _stream(stream)),
            "bitlinear_int8_gemm")
     return C
+
+
+def bitlinear_forward_noalloc(x, packed, gamma: float, N: int, y=None, stream=None):
+    """y = BitLinear(x) on the tensor-core path with the library's static
+    scratch instead of a workspace, for callers that cannot allocate device
+    memory (see include/bitlinear.h for the size limit and the sharing rules).
+    Pass ``y`` to keep this wrapper from allocating the output."""
+    import torch
+    M, K = x.shape
+    if y is None:
+        y = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
+    _check(lib().bitlinear_forward_noalloc(_ptr(x), _xdt(x), M, K, _ptr(packed), float(gamma),
+                                           N, _ptr(y), _stream(stream)),
+           "bitlinear_forward_noalloc")
+    return y

@@ -340,6 +340,7 @@ extern "C" const char *bitlinear_status_string(int status)
     case BITLINEAR_ERR_CUDA: return "CUDA error";
     case BITLINEAR_ERR_TIMEOUT: return "device wait timed out";
     case BITLINEAR_ERR_WORKSPACE: return "workspace missing or too small";
+    case BITLINEAR_ERR_SCRATCH_LIMIT: return "problem exceeds the static scratch limit";
     default: return "unknown status";
     }
 }
@@ -455,4 +456,63 @@ extern "C" int bitlinear_int8_gemm(const int8_t *A_dev, const int8_t *B_dev, int
     tc::Params p{static_cast<int>(M), static_cast<int>(N), static_cast<int>(K), 0.0f, nullptr,
                  nullptr, nullptr, C_dev, kWaitLimitNs, 0};
     return launch_gemm<false, false>(ma, mb, p, *dev, static_cast<cudaStream_t>(cuda_stream));
+}
+
+// ======================================================== no-allocation path
+//
+// For callers that cannot allocate device memory: the tensor-core path's
+// scratch (x~, beta, row sums of x~) lives in this fixed-size array, which
+// every GPU that loads the library holds until the process exits. Host code
+// must not use the array's name as a device address; its address is looked
+// up once per device with cudaGetSymbolAddress and handed to the kernels.
+
+static __device__ __align__(256) unsigned char g_static_scratch[BITLINEAR_STATIC_SCRATCH_BYTES];
+
+namespace {
+
+std::mutex g_static_scratch_mutex;
+void *g_static_scratch_ptr[kMaxDevices];
+
+// Device address of g_static_scratch on device `dev` (which must be current).
+int static_scratch_address(int dev, void **out)
+{
+    std::lock_guard<std::mutex> lock(g_static_scratch_mutex);
+    if (g_static_scratch_ptr[dev] == nullptr) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || p == nullptr) {
+            cudaGetLastError();
+            return BITLINEAR_ERR_CUDA;
+        }
+        g_static_scratch_ptr[dev] = p;
+    }
+    *out = g_static_scratch_ptr[dev];
+    return BITLINEAR_OK;
+}
+
+}  // namespace
+
+extern "C" int bitlinear_forward_noalloc(const void *x_dev, bitlinear_dtype xdt, int64_t M,
+                                         int64_t K, const void *packed_dev, float gamma,
+                                         int64_t N, void *y_dev, void *cuda_stream)
+{
+    int rc = check_forward_args(x_dev, xdt, M, K, packed_dev, N, y_dev, nullptr, nullptr,
+                                nullptr);
+    if (rc != BITLINEAR_OK)
+        return rc;
+    if (M == 0)
+        return BITLINEAR_OK;
+    if (tc_workspace_bytes(M, K) > BITLINEAR_STATIC_SCRATCH_BYTES)
+        return BITLINEAR_ERR_SCRATCH_LIMIT;
+    DeviceInfo *dev = nullptr;
+    rc = current_device(&dev);
+    if (rc != BITLINEAR_OK)
+        return rc;
+    void *scratch = nullptr;
+    rc = static_scratch_address(dev->id, &scratch);
+    if (rc != BITLINEAR_OK)
+        return rc;
+    return run_tc_path(x_dev, xdt, static_cast<int>(M), static_cast<int>(K), packed_dev, gamma,
+                       static_cast<int>(N), y_dev, scratch, BITLINEAR_STATIC_SCRATCH_BYTES,
+                       nullptr, nullptr, nullptr, *dev, static_cast<cudaStream_t>(cuda_stream),
+                       0);
 }

@@ -1,0 +1,57 @@
+"""bitlinear_forward_noalloc: the tensor-core forward for callers that cannot
+allocate device memory (a plugin handed only its input and output pointers,
+a serving loop that forbids allocation after start-up). Its scratch is a
+fixed 16 MiB array inside the library instead of a caller workspace.
+
+Checked through the C ABI against the existing entry point
+(bitlinear_forward_ex on the tensor-core path with a caller workspace), with
+the tolerance of the other parity tests, on two calls in a row: the second
+call reuses the array the first one left behind. This file is collected
+last so that a run stopping at the first failure has already run every
+other test; it also passes on its own in a fresh process.
+"""
+import ctypes
+
+import numpy as np
+import pytest
+
+import ternary_weight_w1_b200 as bl
+from tests.gpu_cases import Case, check_y, tensor_to_bf16_bits
+
+pytestmark = pytest.mark.gpu
+
+
+def call_noalloc(x, packed, gamma, N, y):
+    import torch
+    M, K = x.shape
+    return bl.lib().bitlinear_forward_noalloc(
+        x.data_ptr(), bl.BITLINEAR_BF16, M, K, packed.data_ptr(), ctypes.c_float(gamma), N,
+        y.data_ptr(), torch.cuda.current_stream().cuda_stream)
+
+
+def test_noalloc_matches_workspace_path_twice():
+    import torch
+    assert torch.cuda.is_available(), "GPU test needs a CUDA device"
+    # two different problems, back to back, sharing the static scratch
+    cases = [Case(300, 1280, 700, w_seed=21, x_seed=22), Case(130, 2560, 513, w_seed=23, x_seed=24)]
+    for c in cases:
+        x, packed = c.x_tensor(), c.packed_tensor()
+        y_ref = torch.empty((c.M, c.N), dtype=torch.bfloat16, device="cuda")
+        bl.bitlinear_forward(x, packed, c.gamma, c.N, y=y_ref, path=bl.PATH_TC)
+        y = torch.full((c.M, c.N), float("nan"), dtype=torch.bfloat16, device="cuda")
+        assert call_noalloc(x, packed, c.gamma, c.N, y) == bl.BITLINEAR_OK
+        torch.cuda.synchronize()
+        got, ref = tensor_to_bf16_bits(y), tensor_to_bf16_bits(y_ref)
+        check_y(got, ref)                        # the parity tolerance (rel 1e-2)
+        np.testing.assert_array_equal(got, ref)  # same kernels: identical bits
+    assert bl.bitlinear_get_fault() == (bl.BITLINEAR_OK, 0)
+
+
+def test_noalloc_rejects_problems_beyond_the_scratch():
+    import torch
+    x = torch.zeros((2425, 6912), dtype=torch.bfloat16, device="cuda")
+    packed = torch.zeros((64, 6912 // 4), dtype=torch.uint8, device="cuda")
+    y = torch.empty((2425, 64), dtype=torch.bfloat16, device="cuda")
+    assert call_noalloc(x, packed, 1.0, 64, y) == bl.BITLINEAR_ERR_SCRATCH_LIMIT
+    assert call_noalloc(x[:2424], packed, 1.0, 64, y[:2424]) == bl.BITLINEAR_OK
+    torch.cuda.synchronize()
