@@ -249,12 +249,14 @@ def time_graph_steps(dist, wl, steps: int, clocks: ClockSampler | None):
     torch.cuda.synchronize()
     if clocks:
         clocks.mark(True)
+    torch.cuda.nvtx.range_push("decode_timed")
     start.record()
     for _ in range(steps // ROTATE):
         full.replay()
     if tail is not None:
         tail.replay()
     end.record()
+    torch.cuda.nvtx.range_pop()
     torch.cuda.synchronize()
     if clocks:
         clocks.mark(False)
@@ -324,10 +326,12 @@ def bench_prefill(bl, device, reps: int = 20):
     g.replay()
     torch.cuda.synchronize()
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.nvtx.range_push("prefill_timed")
     start.record()
     for _ in range(reps):
         g.replay()
     end.record()
+    torch.cuda.nvtx.range_pop()
     torch.cuda.synchronize()
     ms = start.elapsed_time(end) / (reps * PREFILL_COPIES)
     ops = sum(2 * m["p"].M * m["p"].N * m["p"].K for m in mats)

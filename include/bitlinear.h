@@ -72,25 +72,30 @@ typedef enum {
 
 /* ---------------------------------------------------------------- packing */
 
-/* Bytes of the packed ternary matrix for N rows of K weights: N * K / 4.
- * Returns 0 when N < 1, K < 16 or K % 16 != 0.
+/* Bytes of the packed ternary matrix for N rows of K weights:
+ * ceil(N / 16) * 16 * K / 4. Returns 0 when N < 1 or K is not a positive
+ * multiple of 128.
  *
  * Packed layout (this library's own; the "2-bit nibbles" of the bitnet.xin
  * guide, section "Core Architecture"):
- *   - N rows of K/4 bytes, row n starting at byte n * K / 4 (row-major, so a
- *     contiguous range of rows is one contiguous byte range);
- *   - the 32-bit little-endian word w of a row holds the weights
- *     k in [16w, 16w + 16);
- *   - weight k = 16w + 4j + b (j, b in 0..3) sits in bits 8b + 2j and
- *     8b + 2j + 1 of its word as the code W~ + 1 (0, 1 or 2; 3 is unused).
- *   So (word >> 2j) & 0x03030303 holds the codes of k = 16w + 4j .. 16w + 4j + 3,
- *   one per byte, in the order of an int32 word of int8 activations, and a
- *   16-byte load is 64 consecutive weights of one row. */
+ *   - rows are taken in blocks of 16 consecutive rows; block b occupies the
+ *     16 * K / 4 bytes starting at byte b * 16 * K / 4 (when N % 16 != 0 the
+ *     last block is completed with rows of zero weights);
+ *   - inside a block the weights come in k-groups of 128: group g holds the
+ *     weights k in [128g, 128g + 128) of all 16 rows in the 512 bytes at
+ *     offset 512 g, row r of the block in the 32 bytes at offset 32 r;
+ *   - those 32 bytes are 8 little-endian 32-bit words; word w holds the 16
+ *     weights k = 128g + 16w + 4j + b (j, b in 0..3) in bits 8b + 2j and
+ *     8b + 2j + 1 as the code W~ + 1 (0, 1 or 2; 3 is unused).
+ *   So every 512-byte (block, group) piece is contiguous, a block's weights
+ *   are one contiguous byte range, and (word >> 2j) & 0x03030303 holds the
+ *   codes of k = 128g + 16w + 4j .. +3 in the order of an int32 word of int8
+ *   activations. */
 size_t bitlinear_packed_bytes(int64_t N, int64_t K);
 
 /* Offline absmean ternarisation and packing, on the host (no device work).
  *   W_host      [in]  latent fp32 weights, [N][K] row-major, host memory
- *   N, K        [in]  d_out, d_in; K must be a positive multiple of 16
+ *   N, K        [in]  d_out, d_in; K must be a positive multiple of 128
  *   packed_host [out] caller-allocated host buffer of bitlinear_packed_bytes(N, K)
  *                     bytes (copy it to the device before bitlinear_forward)
  *   gamma_out   [out] gamma = max(mean |W|, 1e-5), the sum taken in double
@@ -123,7 +128,8 @@ size_t bitlinear_workspace_bytes(int64_t M, int64_t N, int64_t K);
 
 /* y = BitLinear(x) with pre-packed ternary weights, on the device.
  *   x_dev       [in]  [M][K] activations of type xdt
- *   packed_dev  [in]  packed weights (layout above), N * K / 4 bytes
+ *   packed_dev  [in]  packed weights (layout above), bitlinear_packed_bytes(N, K)
+ *                     bytes
  *   gamma       [in]  the gamma bitlinear_pack_weights returned
  *   y_dev       [out] [M][N] bf16 (uint16 bit patterns)
  *   workspace_dev, workspace_bytes

@@ -18,7 +18,7 @@ Functions:
     matmul_i32_pairs(xq, Wq, ms, ns)   acc at sampled (m, n) pairs
     f32_to_bf16(f)              RNE rounding to bf16 bit patterns (uint16)
     rescale_bf16(acc, beta, gamma)     y bf16 bits [M][N]
-    pack_codes(Wq)              the 2-bit packed layout (uint8 [N][K/4])
+    pack_codes(Wq)              the 2-bit packed layout (flat uint8)
     forward(x, W)               the whole path, returning every stage
 """
 from __future__ import annotations
@@ -169,12 +169,14 @@ class Oracle:
         return y
 
     def pack_codes(self, Wq) -> np.ndarray:
+        """The packed layout as a flat uint8 array of
+        ceil(N/16) * 16 * K/4 bytes."""
         Wq = _c(Wq, np.int8)
         N, K = Wq.shape
-        out = np.empty((N, K // 4), dtype=np.uint8)
+        out = np.empty(((N + 15) // 16) * 16 * (K // 4), dtype=np.uint8)
         rc = self.lib.oracle_pack_codes(_ptr(Wq), N, K, _ptr(out))
         if rc != 0:
-            raise ValueError("oracle_pack_codes: K % 16 != 0 or non-ternary")
+            raise ValueError("oracle_pack_codes: K % 128 != 0 or non-ternary")
         return out
 
     def forward(self, x, W, gamma=None):

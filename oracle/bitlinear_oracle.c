@@ -199,34 +199,45 @@ void oracle_rescale_bf16(const int32_t *acc, const float *beta, float gamma,
 
 /* Packed ternary storage (the "2-bit nibbles" of the bitnet.xin guide, section
  * "Core Architecture"; the layout itself is this library's own):
- *   - the matrix is N rows of K/4 bytes, row n starting at byte n * K / 4;
- *   - the 32-bit little-endian word w of a row holds the 16 weights with
- *     k in [16w, 16w + 16);
- *   - weight k = 16w + 4j + b (j, b in 0..3) sits in bits 8b + 2j and
- *     8b + 2j + 1 of that word, as the code W~ + 1 (0, 1 or 2).
- * Returns 0, or -1 when K is not a multiple of 16 or a weight is not ternary. */
+ *   - rows are taken in blocks of 16 consecutive rows; block b occupies the
+ *     16 * K / 4 bytes starting at byte b * 16 * K / 4, and when N is not a
+ *     multiple of 16 the last block is completed with rows of zero weights;
+ *   - inside a block the weights come in k-groups of 128: group g (the
+ *     weights k in [128g, 128g + 128) of all 16 rows) occupies the 512 bytes at
+ *     offset 512 g, and row r of the block the 32 bytes at offset 32 r in it;
+ *   - those 32 bytes are 8 little-endian 32-bit words; word w holds the 16
+ *     weights k = 128g + 16w + 4j + b (j, b in 0..3) in bits 8b + 2j and
+ *     8b + 2j + 1, as the code W~ + 1 (0, 1 or 2).
+ * The output holds ceil(N / 16) * 16 * K / 4 bytes. Returns 0, or -1 when K
+ * is not a positive multiple of 128 or a weight is not ternary. */
 int oracle_pack_codes(const int8_t *Wq, int64_t N, int64_t K, uint8_t *packed)
 {
-    if (K % 16 != 0)
+    if (K <= 0 || K % 128 != 0)
         return -1;
-    const int64_t words_per_row = K / 16;
-    for (int64_t n = 0; n < N; ++n) {
-        for (int64_t w = 0; w < words_per_row; ++w) {
-            uint32_t word = 0;
-            for (int j = 0; j < 4; ++j) {
-                for (int b = 0; b < 4; ++b) {
-                    const int64_t k = 16 * w + 4 * j + b;
-                    const int v = Wq[n * K + k];
-                    if (v < -1 || v > 1)
-                        return -1;
-                    word |= (uint32_t)(v + 1) << (8 * b + 2 * j);
+    const int64_t blocks = (N + 15) / 16;
+    const int64_t row_bytes = K / 4;
+    for (int64_t blk = 0; blk < blocks; ++blk) {
+        for (int64_t r = 0; r < 16; ++r) {
+            const int64_t n = 16 * blk + r;
+            for (int64_t g = 0; g < K / 128; ++g) {
+                for (int64_t w = 0; w < 8; ++w) {
+                    uint32_t word = 0;
+                    for (int j = 0; j < 4; ++j) {
+                        for (int b = 0; b < 4; ++b) {
+                            const int64_t k = 128 * g + 16 * w + 4 * j + b;
+                            const int v = (n < N) ? Wq[n * K + k] : 0;
+                            if (v < -1 || v > 1)
+                                return -1;
+                            word |= (uint32_t)(v + 1) << (8 * b + 2 * j);
+                        }
+                    }
+                    uint8_t *dst = packed + blk * 16 * row_bytes + 512 * g + 32 * r + 4 * w;
+                    dst[0] = (uint8_t)(word & 0xffu);
+                    dst[1] = (uint8_t)((word >> 8) & 0xffu);
+                    dst[2] = (uint8_t)((word >> 16) & 0xffu);
+                    dst[3] = (uint8_t)((word >> 24) & 0xffu);
                 }
             }
-            uint8_t *dst = packed + n * (K / 4) + 4 * w;
-            dst[0] = (uint8_t)(word & 0xffu);
-            dst[1] = (uint8_t)((word >> 8) & 0xffu);
-            dst[2] = (uint8_t)((word >> 16) & 0xffu);
-            dst[3] = (uint8_t)((word >> 24) & 0xffu);
         }
     }
     return 0;

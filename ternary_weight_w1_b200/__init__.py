@@ -137,7 +137,7 @@ def bitlinear_packed_bytes(N: int, K: int) -> int:
 
 def bitlinear_pack_weights(W) -> tuple[np.ndarray, float]:
     """Ternarise and pack latent fp32 weights [N][K] on the host.
-    Returns (packed uint8 [N][K/4] numpy array, gamma)."""
+    Returns (packed bytes as a flat uint8 numpy array, gamma)."""
     W = np.ascontiguousarray(np.asarray(W, dtype=np.float32))
     if W.ndim != 2:
         raise ValueError("W must be 2-D [N][K]")
@@ -145,7 +145,7 @@ def bitlinear_pack_weights(W) -> tuple[np.ndarray, float]:
     nbytes = bitlinear_packed_bytes(N, K)
     if nbytes == 0:
         raise BitLinearError(BITLINEAR_ERR_SHAPE, "bitlinear_pack_weights")
-    out = np.empty((N, K // 4), dtype=np.uint8)
+    out = np.empty((nbytes,), dtype=np.uint8)
     gamma = ctypes.c_float(0.0)
     _check(lib().bitlinear_pack_weights(W.ctypes.data, N, K, out.ctypes.data,
                                         ctypes.addressof(gamma)),

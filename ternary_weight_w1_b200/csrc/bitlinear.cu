@@ -11,8 +11,10 @@
 #include <atomic>
 #include <climits>
 #include <cstdint>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
+#include <utility>
 
 #include "../../include/bitlinear.h"
 #include "common.cuh"
@@ -117,6 +119,58 @@ bool make_map_u8(CUtensorMap *map, const void *ptr, uint64_t rows, uint64_t cols
     return r == CUDA_SUCCESS;
 }
 
+// Programmatic dependent launch: a kernel launched this way may start while
+// the previous kernel in the stream is still running; it reads nothing the
+// previous work may have written (activations, workspace) before its
+// griddepcontrol.wait, except the packed weights, which the GEMV starts
+// streaming at once. On by default; BITLINEAR_PDL=0 in the environment turns
+// it off (every launch then waits for the previous one as usual).
+bool pdl_enabled()
+{
+    static const bool on = [] {
+        const char *v = std::getenv("BITLINEAR_PDL");
+        return !(v != nullptr && v[0] == '0');
+    }();
+    return on;
+}
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                   cudaStream_t st, Args &&...args)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl_enabled() ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
+// The packed weights as a 4-D uint8 tensor {32 B, 16 rows, K/128 groups,
+// ceil(N/16) row blocks} (strides 32, 512 and 16 * K/4 bytes), boxed as
+// {32, 16, 1, box_rows/16}: one box is box_rows consecutive rows x 128 weights,
+// landing in shared memory as [box_rows][32 B].
+bool make_map_packed(CUtensorMap *map, const void *ptr, int64_t N, int64_t K, uint32_t box_rows)
+{
+    EncodeTiledFn fn = encode_fn();
+    if (fn == nullptr)
+        return false;
+    const cuuint64_t dims[4] = {32, 16, static_cast<cuuint64_t>(K / 128),
+                                static_cast<cuuint64_t>((N + 15) / 16)};
+    const cuuint64_t strides[3] = {32, 512, static_cast<cuuint64_t>(16 * (K / 4))};
+    const cuuint32_t box[4] = {32, 16, 1, box_rows / 16};
+    const cuuint32_t estride[4] = {1, 1, 1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, const_cast<void *>(ptr), dims, strides,
+                    box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 int launch_status(cudaError_t e)
 {
     if (e != cudaSuccess) {
@@ -133,34 +187,35 @@ int launch_quant_act(const void *x, bitlinear_dtype xdt, int M, int K, int8_t *x
 {
     if (M == 0)
         return BITLINEAR_OK;
+    const dim3 grid((M + qa::ROWS_PER_BLOCK - 1) / qa::ROWS_PER_BLOCK);
+    cudaError_t e;
     if (xdt == BITLINEAR_BF16)
-        qa::quant_act_kernel<true><<<M, qa::THREADS, 0, st>>>(x, K, xq, beta, rowsum);
+        e = launch(qa::quant_act_kernel<true, 16>, grid, dim3(qa::THREADS), 0, st, x, M, K, xq,
+                   beta, rowsum);
     else
-        qa::quant_act_kernel<false><<<M, qa::THREADS, 0, st>>>(x, K, xq, beta, rowsum);
-    return launch_status(cudaSuccess);
+        e = launch(qa::quant_act_kernel<false, 8>, grid, dim3(qa::THREADS), 0, st, x, M, K, xq,
+                   beta, rowsum);
+    return launch_status(e);
 }
 
 // ------------------------------------------------------------------- GEMV
 
-template <int MT, bool BF16, int DEPTH>
+template <int MT, bool BF16>
 int launch_gemv_t(const gemv::Params &p, int grid, int smem, int dev, cudaStream_t st)
 {
-    cudaError_t e = allow_smem<gemv::gemv_kernel<MT, BF16, DEPTH>>(dev, smem);
+    cudaError_t e = allow_smem<gemv::gemv_kernel<MT, BF16>>(dev, smem);
     if (e != cudaSuccess)
         return launch_status(e);
-    gemv::gemv_kernel<MT, BF16, DEPTH><<<grid, gemv::THREADS, smem, st>>>(p);
-    return launch_status(cudaSuccess);
+    e = launch(gemv::gemv_kernel<MT, BF16>, dim3(grid), dim3(gemv::THREADS), smem, st, p);
+    return launch_status(e);
 }
 
 template <int MT>
-int launch_gemv_mt(const gemv::Params &p, bool bf16, int grid, int smem, bool deep, int dev,
+int launch_gemv_mt(const gemv::Params &p, bool bf16, int grid, int smem, int dev,
                    cudaStream_t st)
 {
-    if (bf16)
-        return deep ? launch_gemv_t<MT, true, 16>(p, grid, smem, dev, st)
-                    : launch_gemv_t<MT, true, 8>(p, grid, smem, dev, st);
-    return deep ? launch_gemv_t<MT, false, 16>(p, grid, smem, dev, st)
-                : launch_gemv_t<MT, false, 8>(p, grid, smem, dev, st);
+    return bf16 ? launch_gemv_t<MT, true>(p, grid, smem, dev, st)
+                : launch_gemv_t<MT, false>(p, grid, smem, dev, st);
 }
 
 int launch_gemv(const void *x, bitlinear_dtype xdt, int M, int K, const void *packed,
@@ -168,29 +223,32 @@ int launch_gemv(const void *x, bitlinear_dtype xdt, int M, int K, const void *pa
                 const DeviceInfo &dev, cudaStream_t st)
 {
     const int MT = M <= 1 ? 1 : M <= 2 ? 2 : M <= 4 ? 4 : M <= 8 ? 8 : 16;
-    // Two blocks per SM when the shared memory allows it, else one block with
-    // deeper per-lane prefetch; never more blocks than rows.
-    int per_sm = 2;
-    int grid = 0, smem = 0;
-    for (;; --per_sm) {
-        grid = static_cast<int>(std::min<int64_t>(static_cast<int64_t>(dev.sms) * per_sm, N));
-        const int rows_cap = (N + grid - 1) / grid;
-        smem = gemv::smem_bytes(MT, K, rows_cap);
-        if (per_sm == 1 || smem * per_sm <= 220 * 1024)
-            break;
-    }
+    // Whole 16-row blocks per CTA, at most two CTAs per SM, every CTA but the
+    // last with the same number of blocks.
+    const int total_blocks = (N + 15) / 16;
+    const int gmax = 2 * dev.sms;
+    const int q = (total_blocks + gmax - 1) / gmax;
+    const int grid = (total_blocks + q - 1) / q;
+    // Ring depth: the whole share when it is small (room for the next
+    // kernel's blocks on the same SM under programmatic launch), else as deep
+    // as a 110 KiB block allows.
+    const int stages = (q * (K / 128) * gemv::PIECE + gemv::STAGE - 1) / gemv::STAGE;
+    const int fixed = gemv::smem_bytes(MT, K, q, 0);
+    const int budget = stages > 12 ? 110 * 1024 : 56 * 1024;
+    int slots = (budget - fixed) / gemv::STAGE;
+    slots = std::max(2, std::min({slots, stages, gemv::MAX_SLOTS}));
+    const int smem = gemv::smem_bytes(MT, K, q, slots);
     if (smem > dev.max_smem_optin)
         return BITLINEAR_ERR_SHAPE;
-    gemv::Params p{x, static_cast<const uint8_t *>(packed), static_cast<uint16_t *>(y), acc, xq,
-                   beta, M, K, N, gamma};
+    gemv::Params p{x,  static_cast<const uint8_t *>(packed), static_cast<uint16_t *>(y), acc, xq,
+                   beta, M, K, N, gamma, q, slots, kWaitLimitNs};
     const bool bf16 = xdt == BITLINEAR_BF16;
-    const bool deep = per_sm == 1;
     switch (MT) {
-    case 1: return launch_gemv_mt<1>(p, bf16, grid, smem, deep, dev.id, st);
-    case 2: return launch_gemv_mt<2>(p, bf16, grid, smem, deep, dev.id, st);
-    case 4: return launch_gemv_mt<4>(p, bf16, grid, smem, deep, dev.id, st);
-    case 8: return launch_gemv_mt<8>(p, bf16, grid, smem, deep, dev.id, st);
-    default: return launch_gemv_mt<16>(p, bf16, grid, smem, deep, dev.id, st);
+    case 1: return launch_gemv_mt<1>(p, bf16, grid, smem, dev.id, st);
+    case 2: return launch_gemv_mt<2>(p, bf16, grid, smem, dev.id, st);
+    case 4: return launch_gemv_mt<4>(p, bf16, grid, smem, dev.id, st);
+    case 8: return launch_gemv_mt<8>(p, bf16, grid, smem, dev.id, st);
+    default: return launch_gemv_mt<16>(p, bf16, grid, smem, dev.id, st);
     }
 }
 
@@ -227,8 +285,9 @@ int launch_gemm(const CUtensorMap &ma, const CUtensorMap &mb, const tc::Params &
         return launch_status(e);
     const int tiles = ((p.M + tc::BM - 1) / tc::BM) * ((p.N + tc::BN - 1) / tc::BN);
     const int grid = std::min(tiles, dev.sms);
-    tc::gemm_kernel<B_PACKED, RESCALE><<<grid, tc::THREADS, tc::SMEM_BYTES, st>>>(ma, mb, p);
-    return launch_status(cudaSuccess);
+    e = launch(tc::gemm_kernel<B_PACKED, RESCALE>, dim3(grid), dim3(tc::THREADS),
+               static_cast<size_t>(tc::SMEM_BYTES), st, ma, mb, p);
+    return launch_status(e);
 }
 
 int run_tc_path(const void *x, bitlinear_dtype xdt, int M, int K, const void *packed,
@@ -247,7 +306,7 @@ int run_tc_path(const void *x, bitlinear_dtype xdt, int M, int K, const void *pa
         return rc;
     CUtensorMap ma, mb;
     if (!make_map_u8(&ma, w.xq, M, K, tc::BM, tc::BK, true) ||
-        !make_map_u8(&mb, packed, N, K / 4, tc::BN, tc::BK / 4, false))
+        !make_map_packed(&mb, packed, N, K, tc::BN))
         return BITLINEAR_ERR_CUDA;
     tc::Params p{M, N, K, gamma, w.beta, w.rowsum, static_cast<uint16_t *>(y), acc,
                  inject_timeout_us > 0 ? static_cast<uint64_t>(inject_timeout_us) * 1000ull

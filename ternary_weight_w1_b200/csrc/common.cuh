@@ -32,12 +32,10 @@ __device__ __forceinline__ uint64_t global_timer_ns()
     return t;
 }
 
-// dp4a with unsigned bytes in a and signed bytes in b: sum_i a_i * b_i + c.
-__device__ __forceinline__ int dp4a_us(uint32_t a, uint32_t b, int c)
+// dp4a on signed bytes: sum_i a_i * b_i + c.
+__device__ __forceinline__ int dp4a_ss(uint32_t a, uint32_t b, int c)
 {
-    int d;
-    asm("dp4a.u32.s32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
-    return d;
+    return __dp4a(static_cast<int>(a), static_cast<int>(b), c);
 }
 
 // ---------------------------------------------------------------- mbarrier
@@ -103,6 +101,31 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
     }
 }
 
+// Lane 0 waits, the verdict is broadcast, and the warp re-converges.
+__device__ __forceinline__ bool warp_wait_bounded(uint32_t bar, uint32_t parity,
+                                                  volatile int *abort, uint64_t limit_ns)
+{
+    int ok = 0;
+    if ((threadIdx.x & 31) == 0)
+        ok = mbar_wait_bounded(bar, parity, abort, limit_ns) ? 1 : 0;
+    ok = __shfl_sync(0xffffffffu, ok, 0);
+    __syncwarp();
+    return ok != 0;
+}
+
+// Bounded wait that ignores the abort flag: used only to drain this thread's
+// own asynchronous work (copies, MMAs) before the block exits.
+__device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, uint64_t limit_ns)
+{
+    const uint64_t t0 = global_timer_ns();
+    while (!mbar_try_wait(bar, parity)) {
+        if (global_timer_ns() - t0 > limit_ns) {
+            atomicOr(&g_fault_word, FAULT_WAIT_TIMEOUT);
+            return;
+        }
+    }
+}
+
 // -------------------------------------------------------------- bulk / TMA
 
 // Non-tensor bulk copy global -> shared, completion counted on an mbarrier.
@@ -125,6 +148,17 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map
         "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes "
         "[%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
         "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
+        : "memory");
+}
+
+// 4-D tiled tensor copy global -> shared (no multicast).
+__device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap *map, int c0, int c1,
+                                            int c2, int c3, uint32_t bar)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.4d.shared::cluster.global.mbarrier::complete_tx::bytes "
+        "[%0], [%1, {%2, %3, %4, %5}], [%6];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(bar)
         : "memory");
 }
 

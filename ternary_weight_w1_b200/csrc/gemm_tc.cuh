@@ -62,31 +62,6 @@ struct Params {
     int inject_timeout;     // MMA issuer waits on a barrier nobody arrives at
 };
 
-// Lane 0 waits, the verdict is broadcast, and the warp re-converges.
-__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatile int *abort,
-                                          uint64_t limit)
-{
-    int ok = 0;
-    if ((threadIdx.x & 31) == 0)
-        ok = mbar_wait_bounded(bar, parity, abort, limit) ? 1 : 0;
-    ok = __shfl_sync(0xffffffffu, ok, 0);
-    __syncwarp();
-    return ok != 0;
-}
-
-// Bounded wait that ignores the abort flag: used only to drain this thread's
-// own asynchronous work before the block exits.
-__device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, uint64_t limit)
-{
-    const uint64_t t0 = global_timer_ns();
-    while (!mbar_try_wait(bar, parity)) {
-        if (global_timer_ns() - t0 > limit) {
-            atomicOr(&g_fault_word, FAULT_WAIT_TIMEOUT);
-            return;
-        }
-    }
-}
-
 template <bool B_PACKED, bool RESCALE>
 __global__ void __launch_bounds__(THREADS, 1)
 gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
@@ -174,7 +149,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ 
                     armed_load[ls] = static_cast<int>(lph);
                     tma_load_2d(sA + ls * A_BYTES, &tmap_a, kb * BK, m0, full_load(ls));
                     if constexpr (B_PACKED) {
-                        tma_load_2d(sBp + ls * BP_BYTES, &tmap_b, kb * (BK / 4), n0, full_load(ls));
+                        tma_load_4d(sBp + ls * BP_BYTES, &tmap_b, 0, 0, kb, n0 / 16, full_load(ls));
                     } else {
                         if (!mbar_wait_bounded(empty_dec(ds), dph ^ 1u, abort_flag, limit))
                             goto producer_done;
@@ -245,7 +220,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ 
         for (int t = blockIdx.x; t < T; t += gridDim.x, ++lt) {
             const int buf = lt & 1;
             const uint32_t aph = static_cast<uint32_t>(lt >> 1) & 1u;
-            if (!warp_wait(tmem_full(buf), aph, abort_flag, limit))
+            if (!warp_wait_bounded(tmem_full(buf), aph, abort_flag, limit))
                 break;
             tc_fence_after_sync();
             const int m = (t % MB) * BM + q * 32 + lane;
@@ -314,9 +289,9 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ 
         uint32_t lph = 0, dph = 0;
         for (int t = blockIdx.x; t < T; t += gridDim.x) {
             for (int kb = 0; kb < KB; ++kb) {
-                if (!warp_wait(full_load(ls), lph, abort_flag, limit))
+                if (!warp_wait_bounded(full_load(ls), lph, abort_flag, limit))
                     goto decode_done;
-                if (!warp_wait(empty_dec(ds), dph ^ 1u, abort_flag, limit))
+                if (!warp_wait_bounded(empty_dec(ds), dph ^ 1u, abort_flag, limit))
                     goto decode_done;
                 {
                     const uint32_t *src =

@@ -4,32 +4,37 @@
 // Pages: "BitNet b1.58 2B4T Guide: Scaling Native 1-Bit LLMs", sections
 // "8-Bit Activation Quantization: absmax Scaling" (prologue), "Matrix
 // Multiplication as Pure Integer Addition" (contraction and rescale); the
-// memory-wall framing of "BitNet b1.58: The 1-Bit Paradigm Shift" is why this
+// memory-wall framing of "BitNet b1.58: The 1-Bit Paradigm Shift" is why the
 // kernel is organised around the weight bytes.
 //
-// Work split. Block b owns the contiguous rows [b*N/G, (b+1)*N/G) of W, which
-// are one contiguous byte range of the packed matrix. A warp "unit" is 4 rows
-// x 8 lanes: lane (rl, kl) loads 16 bytes (64 weights) of row rl at chunk
-// q*8 + kl, so one warp-wide load touches four fully used 128-byte lines. The
-// units of a block (pass-major, chunk-group-minor) are split evenly across its
-// warps; each warp keeps DEPTH loads in flight per lane, and the first DEPTH
-// are issued before the prologue so the weight stream overlaps it.
+// Work split. The packed layout keeps 16-row blocks contiguous, so block b of
+// the grid owns q whole row blocks = one contiguous byte range. A producer
+// warp streams that range through a ring of 8 KiB shared-memory slots with
+// bulk (TMA) copies, starting before the programmatic-launch wait so the weight
+// stream overlaps the previous kernel and this kernel's prologue. Eight
+// compute warps consume 512-byte pieces (one row block x one k-group of 128
+// weights: 16 rows x 32 B) round-robin; lane (r, t) = (lane / 2, lane % 2)
+// always holds row r of the piece and the k-half t, i.e. 64 weights, so the
+// activations it needs are one 64-byte run of x~ that all 16 rows share (a
+// two-address broadcast read from shared memory).
 //
-// Arithmetic. With codes c = W~ + 1 in {0,1,2}, masking a packed word with
-// 0x03030303 << 2j leaves c * 4^j in each byte for the weights
-// k = 16w + 4j .. 16w + 4j + 3. dp4a (unsigned codes x signed x~) into four
-// plane accumulators, one per j, costs one AND and one dp4a per 4 weights
-// and token; the plane sums are exact multiples of 4^j, so
-//   sum c*x~ = a0 + (a1 >> 2) + (a2 >> 4) + (a3 >> 6)
-// exactly, and acc = sum c*x~ - sum x~ (the row sum of x~ comes from the
-// prologue). Lane partials are reduced over the 8 k-lanes by shuffles and added
-// into per-row int32 shared-memory accumulators (integer, so the order of the
-// atomic adds cannot change the result).
+// Arithmetic. With codes c = W~ + 1 in {0,1,2}, the four 2-bit fields j of
+// each byte of a packed word w hold the weights k = 16w' + 4j .. 16w' + 4j + 3
+// of its 16-weight run. w & 0x03030303 and w & 0x0C0C0C0C leave c and 4c in
+// every byte for j = 0 and 1, and the same two masks on w >> 4 do it for
+// j = 2 and 3: all values fit a signed byte, so one signed dp4a per 4 weights
+// and token multiplies them with the matching x~ word. The two accumulators
+// (scale 1: j = 0, 2; scale 4: j = 1, 3) give
+//   sum c*x~ = s1 + (s4 >> 2)
+// exactly (s4 is a multiple of 4), and acc = sum c*x~ - sum x~ (the token's
+// sum of x~ comes from the prologue). Each piece's partial is folded with the
+// k-half partner lane by one shuffle and added into a per-row int32
+// shared-memory accumulator (integer, so the order of the atomic adds cannot
+// change the result); pieces are therefore independent and a warp works on
+// two at a time.
 //
-// x~ lives in shared memory "piece-major": for token m, chunk c (64 k's) and
-// piece t (16 k's), bytes k = 64c + 16t .. +15 sit at m*K + (t*C + c)*16, so
-// the eight k-lanes of a unit read eight consecutive 16-byte pieces (one
-// conflict-free wavefront, broadcast over the four rows).
+// Every mbarrier wait is bounded; a wait that runs out records the fault word
+// and lets every warp return (the producer first waits for its own copies).
 #pragma once
 
 #include "common.cuh"
@@ -37,10 +42,14 @@
 namespace bitlinear {
 namespace gemv {
 
-constexpr int THREADS = 256;
-constexpr int WARPS = THREADS / 32;
-constexpr int LK = 8;          // lanes across K in a unit
-constexpr int LR = 32 / LK;    // rows in a unit
+constexpr int CWARPS = 8;                          // compute warps
+constexpr int CTHREADS = CWARPS * 32;
+constexpr int THREADS = CTHREADS + 32;             // + the producer warp
+constexpr int PIECE = 512;                         // one (row block, k-group)
+constexpr int STAGE = 16384;                       // bytes per ring slot
+constexpr int PIECES_PER_STAGE = STAGE / PIECE;
+constexpr int MAX_SLOTS = 16;
+constexpr int BAR_BYTES = 2 * MAX_SLOTS * 8 + 16;  // full/empty barriers + abort flag
 
 struct Params {
     const void *x;
@@ -51,93 +60,129 @@ struct Params {
     float *beta_dbg;
     int M, K, N;
     float gamma;
+    int blocks_per_cta;     // row blocks of 16 rows owned by one CTA
+    int slots;              // ring slots (<= MAX_SLOTS)
+    uint64_t wait_limit_ns;
 };
 
-__host__ __device__ constexpr int smem_bytes(int MT, int K, int rows_cap)
+__host__ __device__ constexpr int smem_bytes(int MT, int K, int blocks_per_cta, int slots)
 {
-    return MT * K + rows_cap * MT * 4 + 2 * MT * 4 + 2 * WARPS * 4;
+    return slots * STAGE + BAR_BYTES + MT * K + blocks_per_cta * 16 * MT * 4 + MT * 4 +
+           2 * MT * CWARPS * 4;
 }
 
-__device__ __forceinline__ uint4 ldg_stream(const uint8_t *p)
+__device__ __forceinline__ void compute_sync()
 {
-    uint4 v;
-    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
-                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-                 : "l"(p));
-    return v;
+    asm volatile("bar.sync 1, %0;" ::"r"(CTHREADS) : "memory");
 }
 
-template <int MT, bool BF16, int DEPTH>
-__global__ void __launch_bounds__(THREADS)
+template <int MT, bool BF16>
+__global__ void __launch_bounds__(THREADS, 1)
 gemv_kernel(const Params p)
 {
-    extern __shared__ __align__(16) uint8_t smem[];
+    extern __shared__ __align__(128) uint8_t smem[];
     const int K = p.K, M = p.M, N = p.N;
-    const int C = K >> 6;                 // 16-byte chunks (64 weights) per row
-    const int CG = (C + LK - 1) / LK;     // chunk groups per pass
-    const int r0 = static_cast<int>((static_cast<int64_t>(blockIdx.x) * N) / gridDim.x);
-    const int r1 = static_cast<int>((static_cast<int64_t>(blockIdx.x + 1) * N) / gridDim.x);
-    const int nrows = r1 - r0;
-    const int passes = (nrows + LR - 1) / LR;
-    const int units = passes * CG;
+    const int KG = K >> 7;                              // k-groups per row
+    const int total_blocks = (N + 15) >> 4;
+    const int q = p.blocks_per_cta;
+    const int blk0 = blockIdx.x * q;
+    const int nblk = min(q, total_blocks - blk0);
+    const size_t block_bytes = static_cast<size_t>(K) * 4;   // 16 rows x K/4 bytes
+    const uint8_t *src = p.packed + static_cast<size_t>(blk0) * block_bytes;
+    const int npieces = nblk * KG;
+    const int nstages = (npieces + PIECES_PER_STAGE - 1) / PIECES_PER_STAGE;
+    const int slots = p.slots;
+
+    uint8_t *ring = smem;
+    const uint32_t bars = smem_u32(smem + slots * STAGE);
+    auto full = [&](int s) { return bars + 8u * static_cast<uint32_t>(s); };
+    auto empty = [&](int s) { return bars + 8u * static_cast<uint32_t>(MAX_SLOTS + s); };
+    volatile int *abort_flag =
+        reinterpret_cast<volatile int *>(smem + slots * STAGE + 2 * MAX_SLOTS * 8);
+    uint8_t *xq_sm = smem + slots * STAGE + BAR_BYTES;
+    int *acc_sm = reinterpret_cast<int *>(xq_sm + MT * K);
+    float *beta_sm = reinterpret_cast<float *>(acc_sm + q * 16 * MT);
+    uint32_t *red_u = reinterpret_cast<uint32_t *>(beta_sm + MT);   // [MT][CWARPS] absmax
+    int *red_i = reinterpret_cast<int *>(red_u + MT * CWARPS);      // [MT][CWARPS] sum x~
+
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int rl = lane / LK;
-    const int kl = lane % LK;
-    const int u0 = static_cast<int>(static_cast<int64_t>(warp) * units / WARPS);
-    const int u1 = static_cast<int>(static_cast<int64_t>(warp + 1) * units / WARPS);
+    const uint64_t limit = p.wait_limit_ns;
 
-    uint8_t *xq_sm = smem;
-    int *acc_sm = reinterpret_cast<int *>(smem + MT * K);
-    const int rows_cap = (N + gridDim.x - 1) / gridDim.x;
-    float *beta_sm = reinterpret_cast<float *>(acc_sm + rows_cap * MT);
-    int *rsum_sm = reinterpret_cast<int *>(beta_sm + MT);
-    uint32_t *red_u = reinterpret_cast<uint32_t *>(rsum_sm + MT);
-    int *red_i = reinterpret_cast<int *>(red_u + WARPS);
-
-    const size_t row_bytes = static_cast<size_t>(K) >> 2;
-    const uint8_t *wbase = p.packed + static_cast<size_t>(r0) * row_bytes;
-
-    // ---- 1. start the weight stream (independent of x and of earlier kernels)
-    int ld_p = u0 / CG, ld_q = u0 % CG;   // next unit to load
-    auto load_next = [&]() -> uint4 {
-        const int row = ld_p * LR + rl;
-        const int chunk = ld_q * LK + kl;
-        uint4 v = make_uint4(0u, 0u, 0u, 0u);
-        if (row < nrows && chunk < C)
-            v = ldg_stream(wbase + static_cast<size_t>(row) * row_bytes + chunk * 16);
-        if (++ld_q == CG) {
-            ld_q = 0;
-            ++ld_p;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < slots; ++s) {
+            mbar_init(full(s), 1);
+            mbar_init(empty(s), CWARPS);
         }
-        return v;
-    };
-    uint4 buf[DEPTH];
-#pragma unroll
-    for (int i = 0; i < DEPTH; ++i)
-        buf[i] = (u0 + i < u1) ? load_next() : make_uint4(0u, 0u, 0u, 0u);
+        *abort_flag = 0;
+        fence_barrier_init();
+    }
+    __syncthreads();
 
-    for (int i = threadIdx.x; i < nrows * MT; i += THREADS)
+    if (warp == CWARPS) {
+        // ---------------------------------------------------- weight producer
+        // Reads only the packed weights, so it does not wait for the previous
+        // grid in the stream.
+        if (lane == 0) {
+            int issued = 0;
+            int slot = 0;
+            uint32_t phase = 0;       // parity of this pass over the ring
+            for (int st = 0; st < nstages; ++st) {
+                // from the second pass on, the slot must have been released
+                if (st >= slots && !mbar_wait_bounded(empty(slot), phase ^ 1u, abort_flag, limit))
+                    break;
+                const int off = st * STAGE;
+                const int bytes = min(STAGE, npieces * PIECE - off);
+                mbar_arrive_expect_tx(full(slot), static_cast<uint32_t>(bytes));
+                bulk_g2s(smem_u32(ring + slot * STAGE), src + off, static_cast<uint32_t>(bytes),
+                         full(slot));
+                issued = st + 1;
+                if (++slot == slots) {
+                    slot = 0;
+                    phase ^= 1u;
+                }
+            }
+            // every copy this thread started lands before the block exits
+            for (int st = max(0, issued - slots); st < issued; ++st)
+                drain_wait(full(st % slots), static_cast<uint32_t>(st / slots) & 1u, limit);
+        }
+        return;
+    }
+
+    // ------------------------------------------------------- compute warps
+    const int ctid = threadIdx.x;                       // 0 .. CTHREADS-1
+    for (int i = ctid; i < nblk * 16 * MT; i += CTHREADS)
         acc_sm[i] = 0;
 
-    // ---- 2. prologue: absmax int8 quantisation of the M tokens
+    // x may be the previous kernel's output: read it only after the wait.
     pdl_wait();
-    pdl_launch_dependents();
     for (int m = 0; m < M; ++m) {
         const void *row = static_cast<const char *>(p.x) +
                           static_cast<size_t>(m) * K * (BF16 ? 2 : 4);
         float amax = 0.0f;
-        for (int e = threadIdx.x * 8; e < K; e += THREADS * 8) {
+        for (int e = ctid * 8; e < K; e += CTHREADS * 8) {
             float v[8];
             load8<BF16>(row, e, v);
 #pragma unroll
             for (int i = 0; i < 8; ++i)
                 amax = fmaxf(amax, fabsf(v[i]));
         }
-        const float beta = fmaxf(block_max_nonneg<WARPS>(amax, red_u), 1e-5f);
+        const uint32_t u = __reduce_max_sync(0xffffffffu, __float_as_uint(amax));
+        if (lane == 0)
+            red_u[m * CWARPS + warp] = u;
+    }
+    compute_sync();
+    for (int m = 0; m < M; ++m) {
+        const void *row = static_cast<const char *>(p.x) +
+                          static_cast<size_t>(m) * K * (BF16 ? 2 : 4);
+        uint32_t u = red_u[m * CWARPS];
+#pragma unroll
+        for (int w = 1; w < CWARPS; ++w)
+            u = max(u, red_u[m * CWARPS + w]);
+        const float beta = fmaxf(__uint_as_float(u), 1e-5f);
         const float scale = __fdiv_rn(127.0f, beta);
         int sum = 0;
-        for (int e = threadIdx.x * 8; e < K; e += THREADS * 8) {
+        for (int e = ctid * 8; e < K; e += CTHREADS * 8) {
             float v[8];
             load8<BF16>(row, e, v);
             uint32_t lo = 0, hi = 0;
@@ -149,98 +194,134 @@ gemv_kernel(const Params p)
                 lo |= (static_cast<uint32_t>(q0) & 0xffu) << (8 * i);
                 hi |= (static_cast<uint32_t>(q1) & 0xffu) << (8 * i);
             }
-            const int c = e >> 6, t = (e >> 4) & 3;
-            *reinterpret_cast<uint2 *>(xq_sm + m * K + (t * C + c) * 16 + (e & 15)) =
-                make_uint2(lo, hi);
+            *reinterpret_cast<uint2 *>(xq_sm + m * K + e) = make_uint2(lo, hi);
             if (p.xq_dbg != nullptr && blockIdx.x == 0)
                 *reinterpret_cast<uint2 *>(p.xq_dbg + static_cast<size_t>(m) * K + e) =
                     make_uint2(lo, hi);
         }
-        const int total = block_sum_int<WARPS>(sum, red_i);
-        if (threadIdx.x == 0) {
+        sum = __reduce_add_sync(0xffffffffu, sum);
+        if (lane == 0)
+            red_i[m * CWARPS + warp] = sum;
+        if (ctid == 0) {
             beta_sm[m] = beta;
-            rsum_sm[m] = total;
             if (p.beta_dbg != nullptr && blockIdx.x == 0)
                 p.beta_dbg[m] = beta;
         }
     }
-    __syncthreads();
+    compute_sync();
 
-    // ---- 3. stream the weights: dp4a over 4^j-scaled code planes
-    int acc[MT][4];
+    // ---- stream the pieces: piece i = (row block i / KG, k-group i % KG).
+    // Each piece's partial dot product goes straight into the row
+    // accumulators, so pieces are independent and a warp works on two at a
+    // time (more independent loads and dp4a chains in flight).
+    const int r = lane >> 1;          // row in the block
+    const int t = lane & 1;           // k-half (64 weights) of the group
+    int i = warp;
+    int blk = warp / KG;
+    int g = warp % KG;
+    auto advance = [&](int &b, int &gg) {
+        gg += CWARPS;
+        while (gg >= KG) {
+            gg -= KG;
+            ++b;
+        }
+    };
+    // partial of one piece for token m: sum over its 64 weights of c * x~
+    auto piece_dot = [&](const uint4 &w4, int gg, int m) -> int {
+        const uint8_t *xk = xq_sm + m * K + gg * 128 + t * 64;
+        const uint32_t words[4] = {w4.x, w4.y, w4.z, w4.w};
+        int s1a = 0, s1b = 0, s4a = 0, s4b = 0;
 #pragma unroll
-    for (int m = 0; m < MT; ++m)
-#pragma unroll
-        for (int j = 0; j < 4; ++j)
-            acc[m][j] = 0;
-
-    int cur_p = u0 / CG, cur_q = u0 % CG;
-    for (int base = u0; base < u1; base += DEPTH) {
-#pragma unroll
-        for (int i = 0; i < DEPTH; ++i) {
-            const int u = base + i;
-            if (u < u1) {
-                const uint4 w = buf[i];
-                if (u + DEPTH < u1)
-                    buf[i] = load_next();
-                const int chunk = cur_q * LK + kl;
-                const int cx = chunk < C ? chunk : 0;   // any valid x~ piece; w is 0
-                const uint32_t words[4] = {w.x, w.y, w.z, w.w};
-                uint32_t mw[4][4];
-#pragma unroll
-                for (int t = 0; t < 4; ++t)
-#pragma unroll
-                    for (int j = 0; j < 4; ++j)
-                        mw[t][j] = words[t] & (0x03030303u << (2 * j));
-#pragma unroll
-                for (int m = 0; m < MT; ++m) {
-                    if (m < M) {
-#pragma unroll
-                        for (int t = 0; t < 4; ++t) {
-                            const uint4 xv = *reinterpret_cast<const uint4 *>(
-                                xq_sm + m * K + (t * C + cx) * 16);
-                            acc[m][0] = dp4a_us(mw[t][0], xv.x, acc[m][0]);
-                            acc[m][1] = dp4a_us(mw[t][1], xv.y, acc[m][1]);
-                            acc[m][2] = dp4a_us(mw[t][2], xv.z, acc[m][2]);
-                            acc[m][3] = dp4a_us(mw[t][3], xv.w, acc[m][3]);
-                        }
-                    }
-                }
-                const bool pass_end = (++cur_q == CG);
-                if (pass_end || u + 1 == u1) {
-                    const int row = cur_p * LR + rl;
-#pragma unroll
-                    for (int m = 0; m < MT; ++m) {
-                        int v = acc[m][0] + (acc[m][1] >> 2) + (acc[m][2] >> 4) + (acc[m][3] >> 6);
-                        v += __shfl_xor_sync(0xffffffffu, v, 1);
-                        v += __shfl_xor_sync(0xffffffffu, v, 2);
-                        v += __shfl_xor_sync(0xffffffffu, v, 4);
-                        if (kl == 0 && row < nrows && m < M)
-                            atomicAdd(&acc_sm[row * MT + m], v);
-#pragma unroll
-                        for (int j = 0; j < 4; ++j)
-                            acc[m][j] = 0;
-                    }
-                    if (pass_end) {
-                        cur_q = 0;
-                        ++cur_p;
-                    }
-                }
+        for (int jw = 0; jw < 4; ++jw) {
+            const uint4 xv = *reinterpret_cast<const uint4 *>(xk + 16 * jw);
+            const uint32_t w = words[jw], w_hi = w >> 4;
+            // j = 0, 2 at scale 1; j = 1, 3 at scale 4
+            if (jw & 1) {
+                s1b = dp4a_ss(w & 0x03030303u, xv.x, s1b);
+                s4b = dp4a_ss(w & 0x0C0C0C0Cu, xv.y, s4b);
+                s1b = dp4a_ss(w_hi & 0x03030303u, xv.z, s1b);
+                s4b = dp4a_ss(w_hi & 0x0C0C0C0Cu, xv.w, s4b);
+            } else {
+                s1a = dp4a_ss(w & 0x03030303u, xv.x, s1a);
+                s4a = dp4a_ss(w & 0x0C0C0C0Cu, xv.y, s4a);
+                s1a = dp4a_ss(w_hi & 0x03030303u, xv.z, s1a);
+                s4a = dp4a_ss(w_hi & 0x0C0C0C0Cu, xv.w, s4a);
             }
         }
-    }
-    __syncthreads();
+        return s1a + s1b + ((s4a + s4b) >> 2);
+    };
+    auto commit = [&](int v, int b, int m) {
+        v += __shfl_xor_sync(0xffffffffu, v, 1);
+        if (t == 0)
+            atomicAdd(&acc_sm[(b * 16 + r) * MT + m], v);
+    };
 
-    // ---- 4. epilogue: acc = sum c*x~ - sum x~, rescale, bf16
+    // The next kernel in the stream may start launching now: its weight
+    // stream overlaps this main loop and epilogue.
+    pdl_launch_dependents();
+
+    int slot = 0;
+    uint32_t phase = 0;
+    for (int st = 0; st < nstages; ++st) {
+        if (!warp_wait_bounded(full(slot), phase, abort_flag, limit))
+            break;
+        const uint8_t *stage = ring + slot * STAGE + lane * 16;
+        const int pbase = st * PIECES_PER_STAGE;
+        const int pend = min(npieces, pbase + PIECES_PER_STAGE);
+        for (; i + CWARPS < pend; i += 2 * CWARPS) {
+            int blk2 = blk, g2 = g;
+            advance(blk2, g2);
+            const uint4 wa = *reinterpret_cast<const uint4 *>(stage + (i - pbase) * PIECE);
+            const uint4 wb =
+                *reinterpret_cast<const uint4 *>(stage + (i + CWARPS - pbase) * PIECE);
+#pragma unroll
+            for (int m = 0; m < MT; ++m) {
+                if (m < M) {
+                    const int va = piece_dot(wa, g, m);
+                    const int vb = piece_dot(wb, g2, m);
+                    commit(va, blk, m);
+                    commit(vb, blk2, m);
+                }
+            }
+            blk = blk2;
+            g = g2;
+            advance(blk, g);
+        }
+        if (i < pend) {
+            const uint4 wa = *reinterpret_cast<const uint4 *>(stage + (i - pbase) * PIECE);
+#pragma unroll
+            for (int m = 0; m < MT; ++m)
+                if (m < M)
+                    commit(piece_dot(wa, g, m), blk, m);
+            i += CWARPS;
+            advance(blk, g);
+        }
+        __syncwarp();
+        if (lane == 0)
+            mbar_arrive(empty(slot));
+        if (++slot == slots) {
+            slot = 0;
+            phase ^= 1u;
+        }
+    }
+    compute_sync();
+
+    // ---- epilogue: acc = sum c*x~ - sum x~, rescale, bf16
     for (int m = 0; m < M; ++m) {
         const float s = out_scale(beta_sm[m], p.gamma);
-        const int rs = rsum_sm[m];
-        for (int r = threadIdx.x; r < nrows; r += THREADS) {
-            const int a = acc_sm[r * MT + m] - rs;
-            const size_t o = static_cast<size_t>(m) * N + r0 + r;
-            p.y[o] = rescale_bf16(a, s);
-            if (p.acc_dbg != nullptr)
-                p.acc_dbg[o] = a;
+        int rs = 0;
+#pragma unroll
+        for (int w = 0; w < CWARPS; ++w)
+            rs += red_i[m * CWARPS + w];
+        for (int rl = ctid; rl < nblk * 16; rl += CTHREADS) {
+            const int n = blk0 * 16 + rl;
+            if (n < N) {
+                const int a = acc_sm[rl * MT + m] - rs;
+                const size_t o = static_cast<size_t>(m) * N + n;
+                p.y[o] = rescale_bf16(a, s);
+                if (p.acc_dbg != nullptr)
+                    p.acc_dbg[o] = a;
+            }
         }
     }
 }

@@ -47,8 +47,10 @@ void parallel_for(int64_t count, Fn fn)
     std::vector<std::thread> pool;
     pool.reserve(workers);
     for (unsigned t = 0; t < workers; ++t) {
+        const int64_t lo = count * t / workers;
+        const int64_t hi = count * (t + 1) / workers;
         pool.emplace_back([=, &fn] {
-            for (int64_t i = t; i < count; i += workers)
+            for (int64_t i = lo; i < hi; ++i)
                 fn(i);
         });
     }
@@ -71,18 +73,18 @@ inline uint32_t ternary_code(float w, float gamma)
 
 extern "C" size_t bitlinear_packed_bytes(int64_t N, int64_t K)
 {
-    if (N < 1 || K < 16 || K % 16 != 0)
+    if (N < 1 || K < 128 || K % 128 != 0)
         return 0;
-    return static_cast<size_t>(N) * static_cast<size_t>(K / 4);
+    const int64_t blocks = (N + 15) / 16;
+    return static_cast<size_t>(blocks) * 16 * static_cast<size_t>(K / 4);
 }
 
-extern "C" int bitlinear_pack_weights(const float *W_host, int64_t N,
-                                      int64_t K, void *packed_host,
-                                      float *gamma_out)
+extern "C" int bitlinear_pack_weights(const float *W_host, int64_t N, int64_t K,
+                                      void *packed_host, float *gamma_out)
 {
     if (!W_host || !packed_host || !gamma_out || N < 1 || K < 0)
         return BITLINEAR_ERR_ARG;
-    if (K < 16 || K % 16 != 0)
+    if (K < 128 || K % 128 != 0)
         return BITLINEAR_ERR_SHAPE;
 
     // gamma = mean |W| (double accumulation in fixed blocks, then one cast).
@@ -104,22 +106,29 @@ extern "C" int bitlinear_pack_weights(const float *W_host, int64_t N,
     if (!(gamma >= kEps))
         gamma = kEps;
 
-    // Encode row by row: word w of row n collects k = 16w + 4j + b at bit
-    // 8b + 2j.
+    // Row blocks of 16 rows; inside a block, k-groups of 128 weights laid out
+    // as 16 rows x 32 bytes; word w of a (row, group) holds
+    // k = 128g + 16w + 4j + b at bit 8b + 2j. Rows past N are zero weights.
     uint8_t *out = static_cast<uint8_t *>(packed_host);
-    const int64_t words = K / 16;
-    parallel_for(N, [&](int64_t n) {
-        const float *row = W_host + n * K;
-        uint8_t *dst = out + n * (K / 4);
-        for (int64_t w = 0; w < words; ++w) {
-            const float *src = row + 16 * w;
-            uint32_t word = 0;
-            for (int k = 0; k < 16; ++k) {
-                const int j = k >> 2;
-                const int b = k & 3;
-                word |= ternary_code(src[k], gamma) << (8 * b + 2 * j);
+    const int64_t row_blocks = (N + 15) / 16;
+    const int64_t groups = K / 128;
+    const size_t block_bytes = 16 * static_cast<size_t>(K / 4);
+    parallel_for(row_blocks * 16, [&](int64_t n) {
+        const int64_t blk = n / 16;
+        const int64_t r = n % 16;
+        uint8_t *block = out + static_cast<size_t>(blk) * block_bytes;
+        for (int64_t g = 0; g < groups; ++g) {
+            uint8_t *dst = block + 512 * g + 32 * r;
+            for (int w = 0; w < 8; ++w) {
+                uint32_t word = 0x55555555u;  // zero weights (padding rows)
+                if (n < N) {
+                    const float *src = W_host + n * K + 128 * g + 16 * w;
+                    word = 0;
+                    for (int k = 0; k < 16; ++k)
+                        word |= ternary_code(src[k], gamma) << (8 * (k & 3) + 2 * (k >> 2));
+                }
+                std::memcpy(dst + 4 * w, &word, 4);  // little-endian host
             }
-            std::memcpy(dst + 4 * w, &word, 4);  // little-endian host
         }
     });
     *gamma_out = gamma;

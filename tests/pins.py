@@ -52,6 +52,7 @@ def load_golden(name: str) -> dict:
 
 
 def load_pack_cases() -> list:
+    """(name, N, K, [(row, k, value)], {offset: byte}, size) per golden case."""
     cases = []
     with open(os.path.join(GOLDEN, "pack_words.txt")) as f:
         for line in f:
@@ -59,10 +60,18 @@ def load_pack_cases() -> list:
             if not line.startswith("case"):
                 continue
             head, _, rest = line.partition(":")
-            wq_part, bytes_part = rest.split(";")
-            wq = [int(v) for v in wq_part.split("=")[1].split()]
-            by = [int(v, 16) for v in bytes_part.split("=")[1].split()]
-            cases.append((head.split()[1], wq, by))
+            shape, weights, bytes_part, size = [x.strip() for x in rest.split(";")]
+            N = int(shape.split()[0].split("=")[1])
+            K = int(shape.split()[1].split("=")[1])
+            ws = []
+            for item in weights.split("=")[1].split():
+                r, k, v = item.split(",")
+                ws.append((int(r), int(k), int(v)))
+            by = {}
+            for item in bytes_part.split("=")[1].split():
+                off, val = item.split(":")
+                by[int(off)] = int(val, 16)
+            cases.append((head.split()[1], N, K, ws, by, int(size.split("=")[1])))
     return cases
 
 
@@ -107,36 +116,50 @@ def pin_activation_ties_even(orc):
 
 
 def pin_pack_words(orc):
-    for name, wq, by in load_pack_cases():
-        got = orc.pack_codes(np.array([wq], dtype=np.int8))
-        assert got.tolist() == [by], (name, got.tolist(), by)
+    for name, N, K, ws, by, size in load_pack_cases():
+        Wq = np.zeros((N, K), dtype=np.int8)
+        for r, k, v in ws:
+            Wq[r, k] = v
+        got = orc.pack_codes(Wq)
+        want = np.full(size, 0x55, dtype=np.uint8)
+        for off, val in by.items():
+            want[off] = val
+        assert got.shape == want.shape, (name, got.shape)
+        np.testing.assert_array_equal(got, want, err_msg=name)
 
 
-def decode_packed_spec(packed: np.ndarray, K: int) -> np.ndarray:
+def decode_packed_spec(packed: np.ndarray, N: int, K: int) -> np.ndarray:
     """Independent decoder of the 2-bit layout, bit by bit from its spec:
-    byte 4w + q of a row is bits 8q..8q+7 of word w; weight k = 16w + 4j + b
-    is the 2-bit field at bit 8b + 2j of that word, minus one."""
-    N = packed.shape[0]
-    out = np.zeros((N, K), dtype=np.int8)
-    for n in range(N):
-        for w in range(K // 16):
-            word = 0
-            for q in range(4):
-                word |= int(packed[n, 4 * w + q]) << (8 * q)
-            for j in range(4):
-                for b in range(4):
-                    code = (word >> (8 * b + 2 * j)) & 3
-                    assert code != 3
-                    out[n, 16 * w + 4 * j + b] = code - 1
-    return out
+    row n = 16 blk + r; its weights k = 128 g + 16 w + 4 j + b sit in the
+    32-bit little-endian word at byte blk*16*K/4 + 512 g + 32 r + 4 w, in
+    bits 8b + 2j, as the code W~ + 1. Padding rows must decode to zeros."""
+    packed = np.asarray(packed).reshape(-1)
+    blocks = (N + 15) // 16
+    assert packed.size == blocks * 16 * K // 4
+    out = np.zeros((blocks * 16, K), dtype=np.int8)
+    for blk in range(blocks):
+        for r in range(16):
+            for g in range(K // 128):
+                for w in range(8):
+                    base = blk * 16 * K // 4 + 512 * g + 32 * r + 4 * w
+                    word = 0
+                    for q in range(4):
+                        word |= int(packed[base + q]) << (8 * q)
+                    for j in range(4):
+                        for b in range(4):
+                            code = (word >> (8 * b + 2 * j)) & 3
+                            assert code != 3
+                            out[16 * blk + r, 128 * g + 16 * w + 4 * j + b] = code - 1
+    assert np.all(out[N:] == 0)
+    return out[:N]
 
 
 def pin_pack_roundtrip(orc):
     r = np.random.Generator(np.random.PCG64(7))
-    Wq = r.integers(-1, 2, size=(5, 64), dtype=np.int8)
+    Wq = r.integers(-1, 2, size=(21, 256), dtype=np.int8)
     packed = orc.pack_codes(Wq)
-    assert packed.shape == (5, 16)
-    np.testing.assert_array_equal(decode_packed_spec(packed, 64), Wq)
+    assert packed.size == 32 * 256 // 4
+    np.testing.assert_array_equal(decode_packed_spec(packed, 21, 256), Wq)
 
 
 def pin_constant_token(orc):

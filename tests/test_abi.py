@@ -37,9 +37,11 @@ def test_status_strings():
 
 def test_packed_bytes():
     assert bl.bitlinear_packed_bytes(6912, 2560) == 6912 * 640
-    assert bl.bitlinear_packed_bytes(1, 16) == 4
+    assert bl.bitlinear_packed_bytes(1, 128) == 16 * 32          # one padded row block
+    assert bl.bitlinear_packed_bytes(17, 256) == 32 * 64
     assert bl.bitlinear_packed_bytes(0, 256) == 0
-    assert bl.bitlinear_packed_bytes(4, 24) == 0
+    assert bl.bitlinear_packed_bytes(4, 64) == 0
+    assert bl.bitlinear_packed_bytes(4, 200) == 0
 
 
 def test_workspace_bytes():

@@ -38,6 +38,8 @@ MUTANTS = {
     "pack_swaps_j_b": ("<< (8 * b + 2 * j)", "<< (8 * j + 2 * b)"),
     "pack_code_negated": ("(uint32_t)(v + 1)", "(uint32_t)(1 - v)"),
     "pack_word_index": ("16 * w + 4 * j + b;", "16 * w + 4 * b + j;"),
+    "pack_row_stride": ("512 * g + 32 * r + 4 * w", "512 * g + 32 * w + 4 * r"),
+    "pack_padding_rows": ("(n < N) ? Wq[n * K + k] : 0", "(n < N) ? Wq[n * K + k] : -1"),
 }
 
 

@@ -26,43 +26,48 @@ def check_pack(orc, W):
 
 def test_hand_example(orc):
     g = pins.load_golden("hand_example.txt")
-    W = np.zeros((2, 16), dtype=np.float32)
+    W = np.zeros((2, 128), dtype=np.float32)
     W[:, :4] = np.array(g["W"], dtype=np.float32)
     packed, gamma, Wq = check_pack(orc, W)
-    # 4 weights + 12 zeros: mean over 32 entries is 0.144 / 32
-    assert abs(gamma - 0.144 / 32) < 1e-8
-    np.testing.assert_array_equal(pins.decode_packed_spec(packed, 16), Wq)
+    # 4 weights + 124 zeros per row: the mean over 256 entries is 0.144 / 256
+    assert abs(gamma - 0.144 / 256) < 1e-9
+    np.testing.assert_array_equal(pins.decode_packed_spec(packed, 2, 128), Wq)
 
 
-def test_golden_words(orc):
-    for name, wq, by in pins.load_pack_cases():
-        # a latent whose ternarisation is wq: +-1 map to +-1, 0 to 0 (gamma = mean |W|,
-        # and |W| / gamma >= 1 for the nonzeros, 0 for the zeros)
-        W = np.array([wq], dtype=np.float32)
+def test_golden_bytes(orc):
+    for name, N, K, ws, by, size in pins.load_pack_cases():
+        # latents whose ternarisation is the golden pattern: +-1 entries
+        # among zeros have |W| / mean|W| >= 1 whenever zeros dominate
+        W = np.zeros((N, K), dtype=np.float32)
+        for r, k, v in ws:
+            W[r, k] = v
         packed, gamma = bl.bitlinear_pack_weights(W)
-        assert packed.tolist() == [by], name
+        want = np.full(size, 0x55, dtype=np.uint8)
+        for off, val in by.items():
+            want[off] = val
+        np.testing.assert_array_equal(packed, want, err_msg=name)
 
 
-@pytest.mark.parametrize("N,K,seed", [(256, 256, 0), (7, 16, 1), (33, 1280, 2),
-                                      (640, 2560, 3), (2560, 6912, 2)])
+@pytest.mark.parametrize("N,K,seed", [(256, 256, 0), (7, 128, 1), (33, 1280, 2),
+                                      (640, 2560, 3), (2560, 6912, 2), (1001, 384, 4)])
 def test_random_latents(orc, N, K, seed):
     check_pack(orc, workloads.latent_weights(N, K, seed))
 
 
 def test_zero_and_tiny_matrices(orc):
-    packed, gamma, Wq = check_pack(orc, np.zeros((3, 32), dtype=np.float32))
+    packed, gamma, Wq = check_pack(orc, np.zeros((3, 128), dtype=np.float32))
     assert gamma == np.float32(1e-5) and np.all(Wq == 0)
     assert np.all(packed == 0x55)
-    check_pack(orc, np.full((2, 16), 3e-7, dtype=np.float32))
+    check_pack(orc, np.full((2, 128), 3e-7, dtype=np.float32))
 
 
 def test_rejects_bad_shapes():
     with pytest.raises(bl.BitLinearError):
-        bl.bitlinear_pack_weights(np.zeros((2, 20), dtype=np.float32))
+        bl.bitlinear_pack_weights(np.zeros((2, 64), dtype=np.float32))
     L = bl.lib()
     g = np.zeros(1, dtype=np.float32)
-    out = np.zeros(64, dtype=np.uint8)
-    W = np.zeros((4, 16), dtype=np.float32)
-    assert L.bitlinear_pack_weights(None, 4, 16, out.ctypes.data, g.ctypes.data) == bl.BITLINEAR_ERR_ARG
-    assert L.bitlinear_pack_weights(W.ctypes.data, 0, 16, out.ctypes.data, g.ctypes.data) == bl.BITLINEAR_ERR_ARG
-    assert L.bitlinear_pack_weights(W.ctypes.data, 4, 8, out.ctypes.data, g.ctypes.data) == bl.BITLINEAR_ERR_SHAPE
+    out = np.zeros(16 * 32, dtype=np.uint8)
+    W = np.zeros((4, 128), dtype=np.float32)
+    assert L.bitlinear_pack_weights(None, 4, 128, out.ctypes.data, g.ctypes.data) == bl.BITLINEAR_ERR_ARG
+    assert L.bitlinear_pack_weights(W.ctypes.data, 0, 128, out.ctypes.data, g.ctypes.data) == bl.BITLINEAR_ERR_ARG
+    assert L.bitlinear_pack_weights(W.ctypes.data, 4, 64, out.ctypes.data, g.ctypes.data) == bl.BITLINEAR_ERR_SHAPE
