@@ -240,8 +240,10 @@ int launch_gemv(const void *x, bitlinear_dtype xdt, int M, int K, const void *pa
     const int smem = gemv::smem_bytes(MT, K, q, slots);
     if (smem > dev.max_smem_optin)
         return BITLINEAR_ERR_SHAPE;
+    const uint64_t kg = static_cast<uint64_t>(K / 128);
+    const uint64_t kg_magic = ((uint64_t(1) << 32) + kg - 1) / kg;
     gemv::Params p{x,  static_cast<const uint8_t *>(packed), static_cast<uint16_t *>(y), acc, xq,
-                   beta, M, K, N, gamma, q, slots, kWaitLimitNs};
+                   beta, M, K, N, gamma, q, slots, kWaitLimitNs, kg_magic};
     const bool bf16 = xdt == BITLINEAR_BF16;
     switch (MT) {
     case 1: return launch_gemv_mt<1>(p, bf16, grid, smem, dev.id, st);

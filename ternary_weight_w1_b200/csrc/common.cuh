@@ -350,6 +350,32 @@ __device__ __forceinline__ void load8(const void *row, int e, float (&v)[8])
     }
 }
 
+// Raw 8-activation vectors: four bf16 pairs or eight fp32 words.
+template <bool BF16>
+struct Vec8 {
+    static constexpr int WORDS = BF16 ? 4 : 8;
+    uint32_t w[WORDS];
+
+    __device__ __forceinline__ void load(const void *row, int e)
+    {
+        const uint4 *src = reinterpret_cast<const uint4 *>(static_cast<const char *>(row) +
+                                                           static_cast<size_t>(e) * (BF16 ? 2 : 4));
+#pragma unroll
+        for (int i = 0; i < WORDS / 4; ++i) {
+            const uint4 v = __ldg(src + i);
+            w[4 * i] = v.x; w[4 * i + 1] = v.y; w[4 * i + 2] = v.z; w[4 * i + 3] = v.w;
+        }
+    }
+
+    __device__ __forceinline__ float get(int i) const
+    {
+        if constexpr (BF16)
+            return __uint_as_float((i & 1) ? (w[i >> 1] & 0xffff0000u) : (w[i >> 1] << 16));
+        else
+            return __uint_as_float(w[i]);
+    }
+};
+
 // x~ = clamp(round_half_even(x * scale), -128, 127) as one byte.
 __device__ __forceinline__ int quant1(float x, float scale)
 {

@@ -30,8 +30,8 @@
 // sum of x~ comes from the prologue). Each piece's partial is folded with the
 // k-half partner lane by one shuffle and added into a per-row int32
 // shared-memory accumulator (integer, so the order of the atomic adds cannot
-// change the result); pieces are therefore independent and a warp works on
-// two at a time.
+// change the result); pieces are therefore independent, and each warp works
+// on all of its pieces of a ring slot at once, without branches.
 //
 // Every mbarrier wait is bounded; a wait that runs out records the fault word
 // and lets every warp return (the producer first waits for its own copies).
@@ -48,6 +48,7 @@ constexpr int THREADS = CTHREADS + 32;             // + the producer warp
 constexpr int PIECE = 512;                         // one (row block, k-group)
 constexpr int STAGE = 16384;                       // bytes per ring slot
 constexpr int PIECES_PER_STAGE = STAGE / PIECE;
+constexpr int PIECES_PER_WARP = PIECES_PER_STAGE / CWARPS;   // per stage
 constexpr int MAX_SLOTS = 16;
 constexpr int BAR_BYTES = 2 * MAX_SLOTS * 8 + 16;  // full/empty barriers + abort flag
 
@@ -63,6 +64,7 @@ struct Params {
     int blocks_per_cta;     // row blocks of 16 rows owned by one CTA
     int slots;              // ring slots (<= MAX_SLOTS)
     uint64_t wait_limit_ns;
+    uint64_t kg_magic;      // ceil(2^32 / (K / 128)): i / KG == (i * kg_magic) >> 32
 };
 
 __host__ __device__ constexpr int smem_bytes(int MT, int K, int blocks_per_cta, int slots)
@@ -76,8 +78,10 @@ __device__ __forceinline__ void compute_sync()
     asm volatile("bar.sync 1, %0;" ::"r"(CTHREADS) : "memory");
 }
 
+// Three blocks per SM fit the register file (two of this grid and, under
+// programmatic dependent launch, one of the next).
 template <int MT, bool BF16>
-__global__ void __launch_bounds__(THREADS, 1)
+__global__ void __launch_bounds__(THREADS, 3)
 gemv_kernel(const Params p)
 {
     extern __shared__ __align__(128) uint8_t smem[];
@@ -155,12 +159,29 @@ gemv_kernel(const Params p)
         acc_sm[i] = 0;
 
     // x may be the previous kernel's output: read it only after the wait.
+    // Each thread keeps up to XCACHE vectors of 8 activations in registers
+    // between the absmax pass and the quantisation pass; longer rows are read
+    // again (from L1).
     pdl_wait();
+    constexpr int XCACHE = 4;
+    Vec8<BF16> xc[XCACHE];
+    const int e0 = ctid * 8;
+    const int estride = CTHREADS * 8;
     for (int m = 0; m < M; ++m) {
         const void *row = static_cast<const char *>(p.x) +
                           static_cast<size_t>(m) * K * (BF16 ? 2 : 4);
         float amax = 0.0f;
-        for (int e = ctid * 8; e < K; e += CTHREADS * 8) {
+#pragma unroll
+        for (int c = 0; c < XCACHE; ++c) {
+            const int e = e0 + c * estride;
+            if (m == 0 && e < K) {
+                xc[c].load(row, e);
+#pragma unroll
+                for (int i = 0; i < 8; ++i)
+                    amax = fmaxf(amax, fabsf(xc[c].get(i)));
+            }
+        }
+        for (int e = (m == 0 ? e0 + XCACHE * estride : e0); e < K; e += estride) {
             float v[8];
             load8<BF16>(row, e, v);
 #pragma unroll
@@ -182,14 +203,12 @@ gemv_kernel(const Params p)
         const float beta = fmaxf(__uint_as_float(u), 1e-5f);
         const float scale = __fdiv_rn(127.0f, beta);
         int sum = 0;
-        for (int e = ctid * 8; e < K; e += CTHREADS * 8) {
-            float v[8];
-            load8<BF16>(row, e, v);
+        auto quant_store = [&](const Vec8<BF16> &v, int e) {
             uint32_t lo = 0, hi = 0;
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
-                const int q0 = quant1(v[i], scale);
-                const int q1 = quant1(v[i + 4], scale);
+                const int q0 = quant1(v.get(i), scale);
+                const int q1 = quant1(v.get(i + 4), scale);
                 sum += q0 + q1;
                 lo |= (static_cast<uint32_t>(q0) & 0xffu) << (8 * i);
                 hi |= (static_cast<uint32_t>(q1) & 0xffu) << (8 * i);
@@ -198,6 +217,19 @@ gemv_kernel(const Params p)
             if (p.xq_dbg != nullptr && blockIdx.x == 0)
                 *reinterpret_cast<uint2 *>(p.xq_dbg + static_cast<size_t>(m) * K + e) =
                     make_uint2(lo, hi);
+        };
+        if (m == 0) {
+#pragma unroll
+            for (int c = 0; c < XCACHE; ++c) {
+                const int e = e0 + c * estride;
+                if (e < K)
+                    quant_store(xc[c], e);
+            }
+        }
+        for (int e = (m == 0 ? e0 + XCACHE * estride : e0); e < K; e += estride) {
+            Vec8<BF16> v;
+            v.load(row, e);
+            quant_store(v, e);
         }
         sum = __reduce_add_sync(0xffffffffu, sum);
         if (lane == 0)
@@ -211,21 +243,13 @@ gemv_kernel(const Params p)
     compute_sync();
 
     // ---- stream the pieces: piece i = (row block i / KG, k-group i % KG).
-    // Each piece's partial dot product goes straight into the row
-    // accumulators, so pieces are independent and a warp works on two at a
-    // time (more independent loads and dp4a chains in flight).
+    // Warp w takes pieces w, w + CWARPS, ... of every stage: a fixed number
+    // per stage, fully unrolled, with the (block, group) index of each piece
+    // computed by a multiply-high instead of a division. Each piece's partial
+    // dot product goes straight into the row accumulators, so the pieces of a
+    // stage are independent and their loads and dp4a chains overlap.
     const int r = lane >> 1;          // row in the block
     const int t = lane & 1;           // k-half (64 weights) of the group
-    int i = warp;
-    int blk = warp / KG;
-    int g = warp % KG;
-    auto advance = [&](int &b, int &gg) {
-        gg += CWARPS;
-        while (gg >= KG) {
-            gg -= KG;
-            ++b;
-        }
-    };
     // partial of one piece for token m: sum over its 64 weights of c * x~
     auto piece_dot = [&](const uint4 &w4, int gg, int m) -> int {
         const uint8_t *xk = xq_sm + m * K + gg * 128 + t * 64;
@@ -250,11 +274,6 @@ gemv_kernel(const Params p)
         }
         return s1a + s1b + ((s4a + s4b) >> 2);
     };
-    auto commit = [&](int v, int b, int m) {
-        v += __shfl_xor_sync(0xffffffffu, v, 1);
-        if (t == 0)
-            atomicAdd(&acc_sm[(b * 16 + r) * MT + m], v);
-    };
 
     // The next kernel in the stream may start launching now: its weight
     // stream overlaps this main loop and epilogue.
@@ -267,34 +286,37 @@ gemv_kernel(const Params p)
             break;
         const uint8_t *stage = ring + slot * STAGE + lane * 16;
         const int pbase = st * PIECES_PER_STAGE;
-        const int pend = min(npieces, pbase + PIECES_PER_STAGE);
-        for (; i + CWARPS < pend; i += 2 * CWARPS) {
-            int blk2 = blk, g2 = g;
-            advance(blk2, g2);
-            const uint4 wa = *reinterpret_cast<const uint4 *>(stage + (i - pbase) * PIECE);
-            const uint4 wb =
-                *reinterpret_cast<const uint4 *>(stage + (i + CWARPS - pbase) * PIECE);
+        auto locate = [&](int local, int &b, int &gg) {
+            const int i = pbase + local;
+            b = static_cast<int>((static_cast<uint64_t>(i) * p.kg_magic) >> 32);
+            gg = i - b * KG;
+        };
+        {
+            // all of this warp's pieces of the slot at once, without branches;
+            // the last slot may be short, and its missing pieces are computed
+            // on stale slot bytes but not committed
+            uint4 wv[PIECES_PER_WARP];
+            int bv[PIECES_PER_WARP], gv[PIECES_PER_WARP];
+            bool ok[PIECES_PER_WARP];
+#pragma unroll
+            for (int u = 0; u < PIECES_PER_WARP; ++u) {
+                const int local = warp + CWARPS * u;
+                ok[u] = pbase + local < npieces;
+                wv[u] = *reinterpret_cast<const uint4 *>(stage + local * PIECE);
+                locate(local, bv[u], gv[u]);
+            }
 #pragma unroll
             for (int m = 0; m < MT; ++m) {
                 if (m < M) {
-                    const int va = piece_dot(wa, g, m);
-                    const int vb = piece_dot(wb, g2, m);
-                    commit(va, blk, m);
-                    commit(vb, blk2, m);
+#pragma unroll
+                    for (int u = 0; u < PIECES_PER_WARP; ++u) {
+                        int v = piece_dot(wv[u], gv[u], m);
+                        v += __shfl_xor_sync(0xffffffffu, v, 1);
+                        if (t == 0 && ok[u])
+                            atomicAdd(&acc_sm[(bv[u] * 16 + r) * MT + m], v);
+                    }
                 }
             }
-            blk = blk2;
-            g = g2;
-            advance(blk, g);
-        }
-        if (i < pend) {
-            const uint4 wa = *reinterpret_cast<const uint4 *>(stage + (i - pbase) * PIECE);
-#pragma unroll
-            for (int m = 0; m < MT; ++m)
-                if (m < M)
-                    commit(piece_dot(wa, g, m), blk, m);
-            i += CWARPS;
-            advance(blk, g);
         }
         __syncwarp();
         if (lane == 0)

@@ -19,32 +19,6 @@ namespace qa {
 constexpr int THREADS = 256;
 constexpr int ROWS_PER_BLOCK = THREADS / 32;
 
-// Raw 8-activation vectors: four bf16 pairs or eight fp32 words.
-template <bool BF16>
-struct Vec8 {
-    static constexpr int WORDS = BF16 ? 4 : 8;
-    uint32_t w[WORDS];
-
-    __device__ __forceinline__ void load(const void *row, int e)
-    {
-        const uint4 *src = reinterpret_cast<const uint4 *>(static_cast<const char *>(row) +
-                                                           static_cast<size_t>(e) * (BF16 ? 2 : 4));
-#pragma unroll
-        for (int i = 0; i < WORDS / 4; ++i) {
-            const uint4 v = __ldg(src + i);
-            w[4 * i] = v.x; w[4 * i + 1] = v.y; w[4 * i + 2] = v.z; w[4 * i + 3] = v.w;
-        }
-    }
-
-    __device__ __forceinline__ float get(int i) const
-    {
-        if constexpr (BF16)
-            return __uint_as_float((i & 1) ? (w[i >> 1] & 0xffff0000u) : (w[i >> 1] << 16));
-        else
-            return __uint_as_float(w[i]);
-    }
-};
-
 template <bool BF16, int CACHE>
 __global__ void __launch_bounds__(THREADS)
 quant_act_kernel(const void *__restrict__ x, int M, int K, int8_t *__restrict__ xq,
