@@ -161,6 +161,30 @@ int bitlinear_forward_ex(const void *x_dev, bitlinear_dtype xdt, int64_t M,
                          int32_t *acc_dev_or_null, int8_t *xq_dev_or_null,
                          float *beta_dev_or_null, int path);
 
+/* One problem of bitlinear_forward_grouped. */
+typedef struct {
+    const void *x_dev;       /* [M][K] activations (the group's xdt) */
+    int64_t M, K, N;
+    const void *packed_dev;  /* packed weights, bitlinear_packed_bytes(N, K) bytes */
+    float gamma;             /* gamma from bitlinear_pack_weights */
+    void *y_dev;             /* [M][N] bf16 output */
+} bitlinear_problem;
+
+/* Several independent BitLinear matmuls in one launch of the GEMV kernel,
+ * for example the q/k/v or the gate/up projections of a decoder layer (which
+ * may share x_dev), or any set of small-batch problems that do not depend on
+ * each other's outputs. Each problem is computed exactly as bitlinear_forward
+ * computes it on its own; grouping only shares one launch, and the CTAs of
+ * every problem stream about the same number of weight bytes.
+ *   problems [in] host array of count descriptors (1 <= count <= 8); every
+ *                 problem needs M <= 16 and M * K <= 196608; M = 0 problems
+ *                 are skipped
+ *   xdt      [in] activation dtype of all problems
+ * No workspace is needed. Outputs must not overlap each other or any input.
+ * Argument errors are reported before any launch, as for bitlinear_forward. */
+int bitlinear_forward_grouped(const bitlinear_problem *problems, int count,
+                              bitlinear_dtype xdt, void *cuda_stream);
+
 /* Workspace bytes for an explicit path (see bitlinear_forward_ex). */
 size_t bitlinear_workspace_bytes_path(int64_t M, int64_t N, int64_t K,
                                       int path);

@@ -49,7 +49,14 @@ EXPORTS = (
     "bitlinear_int8_gemm",
     "bitlinear_forward_inject_timeout",
     "bitlinear_forward_noalloc",
+    "bitlinear_forward_grouped",
 )
+
+
+class _Problem(ctypes.Structure):
+    _fields_ = [("x_dev", ctypes.c_void_p), ("M", ctypes.c_int64), ("K", ctypes.c_int64),
+                ("N", ctypes.c_int64), ("packed_dev", ctypes.c_void_p),
+                ("gamma", ctypes.c_float), ("y_dev", ctypes.c_void_p)]
 
 _lib = None
 
@@ -90,6 +97,8 @@ def lib() -> ctypes.CDLL:
         L.bitlinear_forward_noalloc.restype = ctypes.c_int
         L.bitlinear_forward_noalloc.argtypes = [p, ctypes.c_int, i64, i64, p, ctypes.c_float,
                                                 i64, p, p]
+        L.bitlinear_forward_grouped.restype = ctypes.c_int
+        L.bitlinear_forward_grouped.argtypes = [p, ctypes.c_int, ctypes.c_int, p]
         L.bitlinear_get_fault.restype = ctypes.c_int
         L.bitlinear_get_fault.argtypes = [p, p]
         L.bitlinear_status_string.restype = ctypes.c_char_p
@@ -251,3 +260,25 @@ def bitlinear_forward_noalloc(x, packed, gamma: float, N: int, y=None, stream=No
                                            N, _ptr(y), _stream(stream)),
            "bitlinear_forward_noalloc")
     return y
+
+
+def bitlinear_forward_grouped(problems, stream=None):
+    """Several independent BitLinear matmuls in one launch. ``problems`` is a
+    list of (x, packed, gamma, N, y) with device tensors (y may be None to
+    allocate it here); all x share one dtype. Returns the list of outputs."""
+    import torch
+    if not problems:
+        return []
+    arr = (_Problem * len(problems))()
+    outs = []
+    xdt = _xdt(problems[0][0])
+    for i, (x, packed, gamma, N, y) in enumerate(problems):
+        M, K = x.shape
+        if y is None:
+            y = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
+        outs.append(y)
+        arr[i] = _Problem(_ptr(x), M, K, N, _ptr(packed), float(gamma), _ptr(y))
+    _check(lib().bitlinear_forward_grouped(ctypes.addressof(arr), len(problems), xdt,
+                                           _stream(stream)),
+           "bitlinear_forward_grouped")
+    return outs

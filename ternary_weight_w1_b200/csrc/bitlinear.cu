@@ -218,32 +218,94 @@ int launch_gemv_mt(const gemv::Params &p, bool bf16, int grid, int smem, int dev
                 : launch_gemv_t<MT, false>(p, grid, smem, dev, st);
 }
 
-int launch_gemv(const void *x, bitlinear_dtype xdt, int M, int K, const void *packed,
-                float gamma, int N, void *y, int32_t *acc, int8_t *xq, float *beta,
-                const DeviceInfo &dev, cudaStream_t st)
+// One problem of a GEMV launch, as the host sees it.
+struct GemvJob {
+    const void *x;
+    int M, K, N;
+    const void *packed;
+    float gamma;
+    void *y;
+    int32_t *acc;
+    int8_t *xq;
+    float *beta;
+};
+
+// Launches the GEMV kernel over one or more independent problems. Every CTA
+// owns whole 16-row blocks of one problem. A single problem is split over at
+// most two CTAs per SM with the same number of blocks per CTA; a group is
+// split so that the CTAs of every problem stream about the same number of
+// bytes, with at most three CTAs per SM (all resident at once).
+int launch_gemv(const GemvJob *jobs, int count, bitlinear_dtype xdt, const DeviceInfo &dev,
+                cudaStream_t st)
 {
-    const int MT = M <= 1 ? 1 : M <= 2 ? 2 : M <= 4 ? 4 : M <= 8 ? 8 : 16;
-    // Whole 16-row blocks per CTA, at most two CTAs per SM, every CTA but the
-    // last with the same number of blocks.
-    const int total_blocks = (N + 15) / 16;
+    int Mmax = 1, Kmax = 128;
+    double total_bytes = 0.0;
+    for (int i = 0; i < count; ++i) {
+        Mmax = std::max(Mmax, jobs[i].M);
+        Kmax = std::max(Kmax, jobs[i].K);
+        total_bytes += static_cast<double>((jobs[i].N + 15) / 16) * 16.0 * jobs[i].K / 4.0;
+    }
+    const int MT = Mmax <= 1 ? 1 : Mmax <= 2 ? 2 : Mmax <= 4 ? 4 : Mmax <= 8 ? 8 : 16;
     const int gmax = 2 * dev.sms;
-    const int q = (total_blocks + gmax - 1) / gmax;
-    const int grid = (total_blocks + q - 1) / q;
+    const int cap = 3 * dev.sms;
+    int q[gemv::MAX_PROBLEMS], ctas[gemv::MAX_PROBLEMS];
+    int grid = 0;
+    if (count == 1) {
+        const int blocks = (jobs[0].N + 15) / 16;
+        q[0] = (blocks + gmax - 1) / gmax;
+        ctas[0] = (blocks + q[0] - 1) / q[0];
+        grid = ctas[0];
+    } else {
+        double target = total_bytes / gmax;        // bytes per CTA
+        for (int attempt = 0; attempt < 64; ++attempt) {
+            grid = 0;
+            for (int i = 0; i < count; ++i) {
+                const int blocks = (jobs[i].N + 15) / 16;
+                const double block_bytes = 16.0 * jobs[i].K / 4.0;
+                q[i] = std::max(1, static_cast<int>(target / block_bytes + 0.5));
+                q[i] = std::min(q[i], blocks);
+                ctas[i] = (blocks + q[i] - 1) / q[i];
+                grid += ctas[i];
+            }
+            if (grid <= cap)
+                break;
+            target *= 1.25;
+        }
+    }
+    int qmax = 1, stages = 1;
+    for (int i = 0; i < count; ++i) {
+        qmax = std::max(qmax, q[i]);
+        stages = std::max(stages, (q[i] * (jobs[i].K / 128) * gemv::PIECE + gemv::STAGE - 1) /
+                                      gemv::STAGE);
+    }
+    const int xq_cap = MT * Kmax;
+    const int acc_cap = qmax * 16 * MT;
     // Ring depth: the whole share when it is small (room for the next
     // kernel's blocks on the same SM under programmatic launch), else as deep
     // as a 110 KiB block allows.
-    const int stages = (q * (K / 128) * gemv::PIECE + gemv::STAGE - 1) / gemv::STAGE;
-    const int fixed = gemv::smem_bytes(MT, K, q, 0);
+    const int fixed = gemv::smem_bytes(MT, xq_cap, acc_cap, 0);
     const int budget = stages > 12 ? 110 * 1024 : 56 * 1024;
     int slots = (budget - fixed) / gemv::STAGE;
     slots = std::max(2, std::min({slots, stages, gemv::MAX_SLOTS}));
-    const int smem = gemv::smem_bytes(MT, K, q, slots);
+    const int smem = gemv::smem_bytes(MT, xq_cap, acc_cap, slots);
     if (smem > dev.max_smem_optin)
         return BITLINEAR_ERR_SHAPE;
-    const uint64_t kg = static_cast<uint64_t>(K / 128);
-    const uint64_t kg_magic = ((uint64_t(1) << 32) + kg - 1) / kg;
-    gemv::Params p{x,  static_cast<const uint8_t *>(packed), static_cast<uint16_t *>(y), acc, xq,
-                   beta, M, K, N, gamma, q, slots, kWaitLimitNs, kg_magic};
+    gemv::Params p = {};
+    int begin = 0;
+    for (int i = 0; i < count; ++i) {
+        const GemvJob &j = jobs[i];
+        const uint64_t kg = static_cast<uint64_t>(j.K / 128);
+        p.prob[i] = gemv::Problem{j.x, static_cast<const uint8_t *>(j.packed),
+                                  static_cast<uint16_t *>(j.y), j.acc, j.xq, j.beta, j.M, j.K,
+                                  j.N, j.gamma, q[i], begin,
+                                  ((uint64_t(1) << 32) + kg - 1) / kg};
+        begin += ctas[i];
+    }
+    p.count = count;
+    p.slots = slots;
+    p.xq_cap = xq_cap;
+    p.acc_cap = acc_cap;
+    p.wait_limit_ns = kWaitLimitNs;
     const bool bf16 = xdt == BITLINEAR_BF16;
     switch (MT) {
     case 1: return launch_gemv_mt<1>(p, bf16, grid, smem, dev.id, st);
@@ -378,8 +440,9 @@ int forward_impl(const void *x, bitlinear_dtype xdt, int64_t M, int64_t K, const
     if (chosen == BITLINEAR_PATH_GEMV) {
         if (!gemv_fits(M, K))
             return BITLINEAR_ERR_SHAPE;
-        return launch_gemv(x, xdt, static_cast<int>(M), static_cast<int>(K), packed, gamma,
-                           static_cast<int>(N), y, acc, xq, beta, *dev, st);
+        const GemvJob job{x,      static_cast<int>(M), static_cast<int>(K), static_cast<int>(N),
+                          packed, gamma, y, acc, xq, beta};
+        return launch_gemv(&job, 1, xdt, *dev, st);
     }
     return run_tc_path(x, xdt, static_cast<int>(M), static_cast<int>(K), packed, gamma,
                        static_cast<int>(N), y, ws, ws_bytes, acc, xq, beta, *dev, st,
@@ -459,6 +522,36 @@ extern "C" int bitlinear_forward_ex(const void *x_dev, bitlinear_dtype xdt, int6
     return forward_impl(x_dev, xdt, M, K, packed_dev, gamma, N, y_dev, workspace_dev,
                         workspace_bytes, cuda_stream, acc_dev_or_null, xq_dev_or_null,
                         beta_dev_or_null, path, 0);
+}
+
+extern "C" int bitlinear_forward_grouped(const bitlinear_problem *problems, int count,
+                                         bitlinear_dtype xdt, void *cuda_stream)
+{
+    if (problems == nullptr || count < 1 || count > gemv::MAX_PROBLEMS)
+        return BITLINEAR_ERR_ARG;
+    GemvJob jobs[gemv::MAX_PROBLEMS];
+    int n = 0;
+    for (int i = 0; i < count; ++i) {
+        const bitlinear_problem &pr = problems[i];
+        int rc = check_forward_args(pr.x_dev, xdt, pr.M, pr.K, pr.packed_dev, pr.N, pr.y_dev,
+                                    nullptr, nullptr, nullptr);
+        if (rc != BITLINEAR_OK)
+            return rc;
+        if (pr.M == 0)
+            continue;
+        if (!gemv_fits(pr.M, pr.K))
+            return BITLINEAR_ERR_SHAPE;
+        jobs[n++] = GemvJob{pr.x_dev,      static_cast<int>(pr.M), static_cast<int>(pr.K),
+                            static_cast<int>(pr.N), pr.packed_dev, pr.gamma, pr.y_dev,
+                            nullptr, nullptr, nullptr};
+    }
+    if (n == 0)
+        return BITLINEAR_OK;
+    DeviceInfo *dev = nullptr;
+    int rc = current_device(&dev);
+    if (rc != BITLINEAR_OK)
+        return rc;
+    return launch_gemv(jobs, n, xdt, *dev, static_cast<cudaStream_t>(cuda_stream));
 }
 
 extern "C" int bitlinear_forward_inject_timeout(const void *x_dev, bitlinear_dtype xdt, int64_t M,

@@ -52,7 +52,11 @@ constexpr int PIECES_PER_WARP = PIECES_PER_STAGE / CWARPS;   // per stage
 constexpr int MAX_SLOTS = 16;
 constexpr int BAR_BYTES = 2 * MAX_SLOTS * 8 + 16;  // full/empty barriers + abort flag
 
-struct Params {
+constexpr int MAX_PROBLEMS = 8;
+
+// One BitLinear problem of a GEMV launch; a launch may carry several
+// independent problems (a grouped launch), each with its own CTAs.
+struct Problem {
     const void *x;
     const uint8_t *packed;
     uint16_t *y;
@@ -62,15 +66,22 @@ struct Params {
     int M, K, N;
     float gamma;
     int blocks_per_cta;     // row blocks of 16 rows owned by one CTA
-    int slots;              // ring slots (<= MAX_SLOTS)
-    uint64_t wait_limit_ns;
+    int cta_begin;          // this problem's first CTA in the grid
     uint64_t kg_magic;      // ceil(2^32 / (K / 128)): i / KG == (i * kg_magic) >> 32
 };
 
-__host__ __device__ constexpr int smem_bytes(int MT, int K, int blocks_per_cta, int slots)
+struct Params {
+    Problem prob[MAX_PROBLEMS];
+    int count;              // problems in this launch
+    int slots;              // ring slots (<= MAX_SLOTS)
+    int xq_cap;             // shared bytes for x~: max over problems of MT * K
+    int acc_cap;            // row accumulators: max over problems of blocks_per_cta * 16 * MT
+    uint64_t wait_limit_ns;
+};
+
+__host__ __device__ constexpr int smem_bytes(int MT, int xq_cap, int acc_cap, int slots)
 {
-    return slots * STAGE + BAR_BYTES + MT * K + blocks_per_cta * 16 * MT * 4 + MT * 4 +
-           2 * MT * CWARPS * 4;
+    return slots * STAGE + BAR_BYTES + xq_cap + acc_cap * 4 + MT * 4 + 2 * MT * CWARPS * 4;
 }
 
 __device__ __forceinline__ void compute_sync()
@@ -82,17 +93,23 @@ __device__ __forceinline__ void compute_sync()
 // programmatic dependent launch, one of the next).
 template <int MT, bool BF16>
 __global__ void __launch_bounds__(THREADS, 3)
-gemv_kernel(const Params p)
+gemv_kernel(const __grid_constant__ Params p)
 {
     extern __shared__ __align__(128) uint8_t smem[];
-    const int K = p.K, M = p.M, N = p.N;
+    // this CTA's problem (grouped launches give each problem its own CTAs)
+    int pi = 0;
+#pragma unroll 1
+    while (pi + 1 < p.count && static_cast<int>(blockIdx.x) >= p.prob[pi + 1].cta_begin)
+        ++pi;
+    const Problem &P = p.prob[pi];
+    const int K = P.K, M = P.M, N = P.N;
     const int KG = K >> 7;                              // k-groups per row
     const int total_blocks = (N + 15) >> 4;
-    const int q = p.blocks_per_cta;
-    const int blk0 = blockIdx.x * q;
+    const int q = P.blocks_per_cta;
+    const int blk0 = (static_cast<int>(blockIdx.x) - P.cta_begin) * q;
     const int nblk = min(q, total_blocks - blk0);
     const size_t block_bytes = static_cast<size_t>(K) * 4;   // 16 rows x K/4 bytes
-    const uint8_t *src = p.packed + static_cast<size_t>(blk0) * block_bytes;
+    const uint8_t *src = P.packed + static_cast<size_t>(blk0) * block_bytes;
     const int npieces = nblk * KG;
     const int nstages = (npieces + PIECES_PER_STAGE - 1) / PIECES_PER_STAGE;
     const int slots = p.slots;
@@ -104,8 +121,8 @@ gemv_kernel(const Params p)
     volatile int *abort_flag =
         reinterpret_cast<volatile int *>(smem + slots * STAGE + 2 * MAX_SLOTS * 8);
     uint8_t *xq_sm = smem + slots * STAGE + BAR_BYTES;
-    int *acc_sm = reinterpret_cast<int *>(xq_sm + MT * K);
-    float *beta_sm = reinterpret_cast<float *>(acc_sm + q * 16 * MT);
+    int *acc_sm = reinterpret_cast<int *>(xq_sm + p.xq_cap);
+    float *beta_sm = reinterpret_cast<float *>(acc_sm + p.acc_cap);
     uint32_t *red_u = reinterpret_cast<uint32_t *>(beta_sm + MT);   // [MT][CWARPS] absmax
     int *red_i = reinterpret_cast<int *>(red_u + MT * CWARPS);      // [MT][CWARPS] sum x~
 
@@ -168,7 +185,7 @@ gemv_kernel(const Params p)
     const int e0 = ctid * 8;
     const int estride = CTHREADS * 8;
     for (int m = 0; m < M; ++m) {
-        const void *row = static_cast<const char *>(p.x) +
+        const void *row = static_cast<const char *>(P.x) +
                           static_cast<size_t>(m) * K * (BF16 ? 2 : 4);
         float amax = 0.0f;
 #pragma unroll
@@ -194,7 +211,7 @@ gemv_kernel(const Params p)
     }
     compute_sync();
     for (int m = 0; m < M; ++m) {
-        const void *row = static_cast<const char *>(p.x) +
+        const void *row = static_cast<const char *>(P.x) +
                           static_cast<size_t>(m) * K * (BF16 ? 2 : 4);
         uint32_t u = red_u[m * CWARPS];
 #pragma unroll
@@ -214,8 +231,8 @@ gemv_kernel(const Params p)
                 hi |= (static_cast<uint32_t>(q1) & 0xffu) << (8 * i);
             }
             *reinterpret_cast<uint2 *>(xq_sm + m * K + e) = make_uint2(lo, hi);
-            if (p.xq_dbg != nullptr && blockIdx.x == 0)
-                *reinterpret_cast<uint2 *>(p.xq_dbg + static_cast<size_t>(m) * K + e) =
+            if (P.xq_dbg != nullptr && blockIdx.x == 0)
+                *reinterpret_cast<uint2 *>(P.xq_dbg + static_cast<size_t>(m) * K + e) =
                     make_uint2(lo, hi);
         };
         if (m == 0) {
@@ -236,8 +253,8 @@ gemv_kernel(const Params p)
             red_i[m * CWARPS + warp] = sum;
         if (ctid == 0) {
             beta_sm[m] = beta;
-            if (p.beta_dbg != nullptr && blockIdx.x == 0)
-                p.beta_dbg[m] = beta;
+            if (P.beta_dbg != nullptr && blockIdx.x == 0)
+                P.beta_dbg[m] = beta;
         }
     }
     compute_sync();
@@ -288,7 +305,7 @@ gemv_kernel(const Params p)
         const int pbase = st * PIECES_PER_STAGE;
         auto locate = [&](int local, int &b, int &gg) {
             const int i = pbase + local;
-            b = static_cast<int>((static_cast<uint64_t>(i) * p.kg_magic) >> 32);
+            b = static_cast<int>((static_cast<uint64_t>(i) * P.kg_magic) >> 32);
             gg = i - b * KG;
         };
         {
@@ -330,7 +347,7 @@ gemv_kernel(const Params p)
 
     // ---- epilogue: acc = sum c*x~ - sum x~, rescale, bf16
     for (int m = 0; m < M; ++m) {
-        const float s = out_scale(beta_sm[m], p.gamma);
+        const float s = out_scale(beta_sm[m], P.gamma);
         int rs = 0;
 #pragma unroll
         for (int w = 0; w < CWARPS; ++w)
@@ -340,9 +357,9 @@ gemv_kernel(const Params p)
             if (n < N) {
                 const int a = acc_sm[rl * MT + m] - rs;
                 const size_t o = static_cast<size_t>(m) * N + n;
-                p.y[o] = rescale_bf16(a, s);
-                if (p.acc_dbg != nullptr)
-                    p.acc_dbg[o] = a;
+                P.y[o] = rescale_bf16(a, s);
+                if (P.acc_dbg != nullptr)
+                    P.acc_dbg[o] = a;
             }
         }
     }

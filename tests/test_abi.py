@@ -118,3 +118,24 @@ def test_inject_timeout_rejects_bad_limit():
 
 def test_get_fault_rejects_null():
     assert bl.lib().bitlinear_get_fault(None, None) == bl.BITLINEAR_ERR_ARG
+
+
+def grouped(problems, xdt=0):
+    arr = (bl._Problem * max(1, len(problems)))()
+    for i, (x, M, K, N, packed, y) in enumerate(problems):
+        arr[i] = bl._Problem(x, M, K, N, packed, 1.0, y)
+    return bl.lib().bitlinear_forward_grouped(ctypes.addressof(arr), len(problems), xdt, None)
+
+
+def test_grouped_rejects_bad_arguments():
+    good = (FAKE, 1, 256, 64, FAKE, FAKE)
+    assert bl.lib().bitlinear_forward_grouped(None, 1, 0, None) == bl.BITLINEAR_ERR_ARG
+    assert grouped([]) == bl.BITLINEAR_ERR_ARG
+    assert grouped([good] * 9) == bl.BITLINEAR_ERR_ARG
+    assert grouped([good, (FAKE, 1, 200, 64, FAKE, FAKE)]) == bl.BITLINEAR_ERR_SHAPE
+    assert grouped([good, (FAKE, 17, 256, 64, FAKE, FAKE)]) == bl.BITLINEAR_ERR_SHAPE
+    assert grouped([good, (FAKE, 16, 16384, 64, FAKE, FAKE)]) == bl.BITLINEAR_ERR_SHAPE
+    assert grouped([good, (None, 1, 256, 64, FAKE, FAKE)]) == bl.BITLINEAR_ERR_ARG
+    assert grouped([good, (FAKE + 8, 1, 256, 64, FAKE, FAKE)]) == bl.BITLINEAR_ERR_ALIGN
+    assert grouped([good], xdt=5) == bl.BITLINEAR_ERR_DTYPE
+    assert grouped([(None, 0, 256, 64, None, None)]) == bl.BITLINEAR_OK   # only empty problems
