@@ -50,7 +50,11 @@ INT8_PER_BF16 = 2.0        # nominal dense int8 / bf16 tensor ratio (4.5 / 2.25 
 # DRAM traffic per launch of the dominant kernels, from an ncu capture
 # (dram__bytes_read.sum + dram__bytes_write.sum), keyed by the sha256 of the
 # kernel source it was taken on; reported only while that source is unchanged.
-TRAFFIC = {}
+TRAFFIC = {
+    # grouped decode launch (up 2560->6912 + down 6912->2560, M=1): 8,847,360
+    # algorithmic bytes; profiles/gemv_grouped_decode_2b_m1.md
+    "gemv": {"src": "cd95e2f786d16a0e", "bytes_per_launch": 8895232},
+}
 
 
 def kernel_source_hash(name: str) -> str:
