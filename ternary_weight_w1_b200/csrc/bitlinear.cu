@@ -19,6 +19,7 @@
 #include "../../include/bitlinear.h"
 #include "common.cuh"
 #include "gemm_tc.cuh"
+#include "gemm_ws.cuh"
 #include "gemv.cuh"
 #include "quant_act.cuh"
 
@@ -151,21 +152,41 @@ cudaError_t launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
     return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
-// The packed weights as a 4-D uint8 tensor {32 B, 16 rows, K/128 groups,
-// ceil(N/16) row blocks} (strides 32, 512 and 16 * K/4 bytes), boxed as
-// {32, 16, 1, box_rows/16}: one box is box_rows consecutive rows x 128 weights,
-// landing in shared memory as [box_rows][32 B].
-bool make_map_packed(CUtensorMap *map, const void *ptr, int64_t N, int64_t K, uint32_t box_rows)
+// x~ [M][K] int8 as a 3-D tensor {128 B, M rows, K/128 chunks} (strides K
+// and 128 bytes), boxed as {128, box_rows, 2} with the 128-byte swizzle: one
+// box is a 256-k slice of box_rows tokens, landing in shared memory as two
+// swizzled [box_rows][128] sub-tiles.
+bool make_map_xq_k256(CUtensorMap *map, const void *ptr, int64_t M, int64_t K, uint32_t box_rows)
 {
     EncodeTiledFn fn = encode_fn();
     if (fn == nullptr)
         return false;
-    const cuuint64_t dims[4] = {32, 16, static_cast<cuuint64_t>(K / 128),
+    const cuuint64_t dims[3] = {128, static_cast<cuuint64_t>(M), static_cast<cuuint64_t>(K / 128)};
+    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(K), 128};
+    const cuuint32_t box[3] = {128, box_rows, 2};
+    const cuuint32_t estride[3] = {1, 1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void *>(ptr), dims, strides,
+                    box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+// The packed weights as a 3-D tensor of 8-byte elements {64 (= the 512 bytes
+// of one row block and 128-k group), K/128 groups, ceil(N/16) row blocks}
+// (strides 512 and 16 * K/4 bytes), boxed as {64, 2, box_rows/16}: one box
+// is box_rows rows x 256 weights, landing as [box_rows/16][2][16 rows][32 B].
+bool make_map_packed_k256(CUtensorMap *map, const void *ptr, int64_t N, int64_t K,
+                          uint32_t box_rows)
+{
+    EncodeTiledFn fn = encode_fn();
+    if (fn == nullptr)
+        return false;
+    const cuuint64_t dims[3] = {64, static_cast<cuuint64_t>(K / 128),
                                 static_cast<cuuint64_t>((N + 15) / 16)};
-    const cuuint64_t strides[3] = {32, 512, static_cast<cuuint64_t>(16 * (K / 4))};
-    const cuuint32_t box[4] = {32, 16, 1, box_rows / 16};
-    const cuuint32_t estride[4] = {1, 1, 1, 1};
-    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, const_cast<void *>(ptr), dims, strides,
+    const cuuint64_t strides[2] = {512, static_cast<cuuint64_t>(16 * (K / 4))};
+    const cuuint32_t box[3] = {64, 2, box_rows / 16};
+    const cuuint32_t estride[3] = {1, 1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT64, 3, const_cast<void *>(ptr), dims, strides,
                     box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
@@ -182,19 +203,42 @@ int launch_status(cudaError_t e)
 
 // ----------------------------------------------------------- quantisation
 
+template <bool BF16, int CACHE, int WPR>
+cudaError_t launch_qa(const void *x, int M, int K, int8_t *xq, float *beta, int *rowsum,
+                      cudaStream_t st, int *clear, int n_clear)
+{
+    constexpr int rpb = qa::rows_per_block<WPR>();
+    const dim3 grid((M + rpb - 1) / rpb);
+    return launch(qa::quant_act_kernel<BF16, CACHE, WPR>, grid, dim3(qa::THREADS), 0, st, x, M,
+                  K, xq, beta, rowsum, clear, n_clear);
+}
+
+// Register cache per lane and warps per row by row length: one warp per row
+// up to 8192 bf16 (4096 fp32) elements, eight for longer rows.
 int launch_quant_act(const void *x, bitlinear_dtype xdt, int M, int K, int8_t *xq, float *beta,
-                     int *rowsum, cudaStream_t st)
+                     int *rowsum, cudaStream_t st, int *clear = nullptr, int n_clear = 0)
 {
     if (M == 0)
         return BITLINEAR_OK;
-    const dim3 grid((M + qa::ROWS_PER_BLOCK - 1) / qa::ROWS_PER_BLOCK);
+    const int nvec = K / 8;
     cudaError_t e;
-    if (xdt == BITLINEAR_BF16)
-        e = launch(qa::quant_act_kernel<true, 16>, grid, dim3(qa::THREADS), 0, st, x, M, K, xq,
-                   beta, rowsum);
-    else
-        e = launch(qa::quant_act_kernel<false, 8>, grid, dim3(qa::THREADS), 0, st, x, M, K, xq,
-                   beta, rowsum);
+    if (xdt == BITLINEAR_BF16) {
+        if (nvec <= 32 * 4)
+            e = launch_qa<true, 4, 1>(x, M, K, xq, beta, rowsum, st, clear, n_clear);
+        else if (nvec <= 32 * 8)
+            e = launch_qa<true, 8, 1>(x, M, K, xq, beta, rowsum, st, clear, n_clear);
+        else if (nvec <= 32 * 32)
+            e = launch_qa<true, 16, 1>(x, M, K, xq, beta, rowsum, st, clear, n_clear);
+        else
+            e = launch_qa<true, 16, 8>(x, M, K, xq, beta, rowsum, st, clear, n_clear);
+    } else {
+        if (nvec <= 32 * 4)
+            e = launch_qa<false, 4, 1>(x, M, K, xq, beta, rowsum, st, clear, n_clear);
+        else if (nvec <= 32 * 16)
+            e = launch_qa<false, 8, 1>(x, M, K, xq, beta, rowsum, st, clear, n_clear);
+        else
+            e = launch_qa<false, 8, 8>(x, M, K, xq, beta, rowsum, st, clear, n_clear);
+    }
     return launch_status(e);
 }
 
@@ -322,22 +366,54 @@ struct TcWorkspace {
     int8_t *xq;
     float *beta;
     int *rowsum;
-    size_t bytes;
+    int *flags;         // [MAX_GRID][4] (split only)
+    int32_t *partial;   // [MAX_GRID][BW][BT] (split only)
 };
 
-size_t tc_workspace_bytes(int64_t M, int64_t K)
+// Token tile of the weight-stationary GEMM: the candidate that pads M the
+// least (ties go to the larger tile).
+int choose_bt(int64_t M)
+{
+    if (M <= 32)
+        return 32;
+    if (M <= 64)
+        return 64;
+    if (M <= 128)
+        return 128;
+    const int64_t pad128 = (M + 127) / 128 * 128;
+    const int64_t pad192 = (M + 191) / 192 * 192;
+    return pad192 <= pad128 ? 192 : 128;
+}
+
+// x~, beta and the row sums of x~.
+size_t tc_base_bytes(int64_t M, int64_t K)
 {
     return round_up(static_cast<size_t>(M) * static_cast<size_t>(K), 256) +
            2 * round_up(static_cast<size_t>(M) * 4, 256);
 }
 
-TcWorkspace tc_workspace(void *ws, int64_t M, int64_t K)
+// Flags and partial-sum slots for tiles split between CTAs.
+size_t tc_split_bytes(int64_t M)
+{
+    return round_up(static_cast<size_t>(wsg::MAX_GRID) * 4 * 4, 256) +
+           static_cast<size_t>(wsg::MAX_GRID) * wsg::BW * static_cast<size_t>(choose_bt(M)) * 4;
+}
+
+size_t tc_workspace_bytes(int64_t M, int64_t K) { return tc_base_bytes(M, K) + tc_split_bytes(M); }
+
+TcWorkspace tc_workspace(void *ws, int64_t M, int64_t K, bool split)
 {
     char *b = static_cast<char *>(ws);
     const size_t a = round_up(static_cast<size_t>(M) * static_cast<size_t>(K), 256);
     const size_t c = round_up(static_cast<size_t>(M) * 4, 256);
-    return {reinterpret_cast<int8_t *>(b), reinterpret_cast<float *>(b + a),
-            reinterpret_cast<int *>(b + a + c), a + 2 * c};
+    const size_t f = round_up(static_cast<size_t>(wsg::MAX_GRID) * 4 * 4, 256);
+    TcWorkspace w{reinterpret_cast<int8_t *>(b), reinterpret_cast<float *>(b + a),
+                  reinterpret_cast<int *>(b + a + c), nullptr, nullptr};
+    if (split) {
+        w.flags = reinterpret_cast<int *>(b + a + 2 * c);
+        w.partial = reinterpret_cast<int32_t *>(b + a + 2 * c + f);
+    }
+    return w;
 }
 
 template <bool B_PACKED, bool RESCALE>
@@ -354,29 +430,76 @@ int launch_gemm(const CUtensorMap &ma, const CUtensorMap &mb, const tc::Params &
     return launch_status(e);
 }
 
+template <int BT>
+int launch_gemm_ws(const CUtensorMap &mx, const CUtensorMap &mw, const wsg::Params &p, int grid,
+                   const DeviceInfo &dev, cudaStream_t st)
+{
+    constexpr int smem = wsg::Cfg<BT>::SMEM_BYTES;
+    cudaError_t e = allow_smem<wsg::gemm_ws_kernel<BT>>(dev.id, smem);
+    if (e != cudaSuccess)
+        return launch_status(e);
+    e = launch(wsg::gemm_ws_kernel<BT>, dim3(grid), dim3(wsg::THREADS), static_cast<size_t>(smem),
+               st, mx, mw, p);
+    return launch_status(e);
+}
+
+// Quantise x, then run the weight-stationary GEMM with its fused rescale.
+// With `split` the k-blocks of all tiles are shared evenly between the CTAs
+// (stream-K; needs the flag and partial-sum regions of the workspace);
+// without it every CTA takes whole tiles.
 int run_tc_path(const void *x, bitlinear_dtype xdt, int M, int K, const void *packed,
                 float gamma, int N, void *y, void *ws, size_t ws_bytes, int32_t *acc,
                 int8_t *xq_dbg, float *beta_dbg, const DeviceInfo &dev, cudaStream_t st,
-                int inject_timeout_us)
+                int inject_timeout_us, bool split)
 {
-    const size_t need = tc_workspace_bytes(M, K);
+    const size_t need = split ? tc_workspace_bytes(M, K) : tc_base_bytes(M, K);
     if (ws == nullptr || ws_bytes < need)
         return BITLINEAR_ERR_WORKSPACE;
     if (!aligned(ws, 256))
         return BITLINEAR_ERR_ALIGN;
-    TcWorkspace w = tc_workspace(ws, M, K);
-    int rc = launch_quant_act(x, xdt, M, K, w.xq, w.beta, w.rowsum, st);
+    const int BT = choose_bt(M);
+    const int KB = (K + wsg::BK - 1) / wsg::BK;
+    const int MT = (M + BT - 1) / BT;
+    const int T = MT * ((N + wsg::BW - 1) / wsg::BW);
+    const int unit = split ? 1 : KB;
+    const int64_t units = static_cast<int64_t>(T) * KB / unit;
+    const int grid = static_cast<int>(
+        std::min<int64_t>(units, std::min(dev.sms, wsg::MAX_GRID)));
+    TcWorkspace w = tc_workspace(ws, M, K, split);
+    int rc = launch_quant_act(x, xdt, M, K, w.xq, w.beta, w.rowsum, st, w.flags,
+                              split ? 4 * grid : 0);
     if (rc != BITLINEAR_OK)
         return rc;
-    CUtensorMap ma, mb;
-    if (!make_map_u8(&ma, w.xq, M, K, tc::BM, tc::BK, true) ||
-        !make_map_packed(&mb, packed, N, K, tc::BN))
+    CUtensorMap mx, mw;
+    if (!make_map_xq_k256(&mx, w.xq, M, K, static_cast<uint32_t>(BT)) ||
+        !make_map_packed_k256(&mw, packed, N, K, wsg::BW))
         return BITLINEAR_ERR_CUDA;
-    tc::Params p{M, N, K, gamma, w.beta, w.rowsum, static_cast<uint16_t *>(y), acc,
-                 inject_timeout_us > 0 ? static_cast<uint64_t>(inject_timeout_us) * 1000ull
-                                       : kWaitLimitNs,
-                 inject_timeout_us > 0 ? 1 : 0};
-    rc = launch_gemm<true, true>(ma, mb, p, dev, st);
+    wsg::Params p{};
+    p.M = M;
+    p.N = N;
+    p.K = K;
+    p.gamma = gamma;
+    p.beta = w.beta;
+    p.rowsum = w.rowsum;
+    p.y = static_cast<uint16_t *>(y);
+    p.acc_out = acc;
+    p.partial = w.partial;
+    p.flags = w.flags;
+    p.MT = MT;
+    p.T = T;
+    p.KB = KB;
+    p.unit = unit;
+    p.base = static_cast<int>(units / grid);
+    p.extra = static_cast<int>(units % grid);
+    p.wait_limit_ns =
+        inject_timeout_us > 0 ? static_cast<uint64_t>(inject_timeout_us) * 1000ull : kWaitLimitNs;
+    p.inject_timeout = inject_timeout_us > 0 ? 1 : 0;
+    switch (BT) {
+    case 32: rc = launch_gemm_ws<32>(mx, mw, p, grid, dev, st); break;
+    case 64: rc = launch_gemm_ws<64>(mx, mw, p, grid, dev, st); break;
+    case 128: rc = launch_gemm_ws<128>(mx, mw, p, grid, dev, st); break;
+    default: rc = launch_gemm_ws<192>(mx, mw, p, grid, dev, st); break;
+    }
     if (rc != BITLINEAR_OK)
         return rc;
     if (xq_dbg != nullptr &&
@@ -446,7 +569,7 @@ int forward_impl(const void *x, bitlinear_dtype xdt, int64_t M, int64_t K, const
     }
     return run_tc_path(x, xdt, static_cast<int>(M), static_cast<int>(K), packed, gamma,
                        static_cast<int>(N), y, ws, ws_bytes, acc, xq, beta, *dev, st,
-                       inject_timeout_us);
+                       inject_timeout_us, true);
 }
 
 }  // namespace
@@ -655,7 +778,7 @@ extern "C" int bitlinear_forward_noalloc(const void *x_dev, bitlinear_dtype xdt,
         return rc;
     if (M == 0)
         return BITLINEAR_OK;
-    if (tc_workspace_bytes(M, K) > BITLINEAR_STATIC_SCRATCH_BYTES)
+    if (tc_base_bytes(M, K) > BITLINEAR_STATIC_SCRATCH_BYTES)
         return BITLINEAR_ERR_SCRATCH_LIMIT;
     DeviceInfo *dev = nullptr;
     rc = current_device(&dev);
@@ -668,5 +791,5 @@ extern "C" int bitlinear_forward_noalloc(const void *x_dev, bitlinear_dtype xdt,
     return run_tc_path(x_dev, xdt, static_cast<int>(M), static_cast<int>(K), packed_dev, gamma,
                        static_cast<int>(N), y_dev, scratch, BITLINEAR_STATIC_SCRATCH_BYTES,
                        nullptr, nullptr, nullptr, *dev, static_cast<cudaStream_t>(cuda_stream),
-                       0);
+                       0, false);
 }

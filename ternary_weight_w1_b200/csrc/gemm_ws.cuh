@@ -1,0 +1,508 @@
+// Weight-stationary tensor-core GEMM for the BitLinear forward:
+// acc[m][n] = sum_k x~[m][k] * W~[n][k] on tcgen05.mma kind::i8.
+//
+// Pages: "BitNet b1.58 2B4T Guide: Scaling Native 1-Bit LLMs", section
+// "Matrix Multiplication as Pure Integer Addition" (the integer contraction
+// and the rescale by beta * gamma / 127); "Microsoft Releases BitNet b1.58
+// 2B4T", section "The Catch" (GPU kernels must unpack the packed weights).
+//
+// The MMA computes D[128 weight rows][BT tokens] = A * B^T with
+//   A = decoded weight codes c = W~ + 1 in {0, 1, 2}, held in TENSOR MEMORY:
+//       the decode warps unpack the 2-bit codes in registers and write them
+//       with tcgen05.st, so decoded weights never pass through shared memory;
+//   B = x~ tile [BT tokens][k] in shared memory (TMA, 128-byte swizzle).
+// acc = D - sum_k x~[m][k] exactly (the row sums come from the quantiser).
+// Because the weights are the MMA's M side, a tile has 128 weight rows and
+// BT in {32, 64, 128, 192} tokens, so small token counts still use the
+// tensor cores without padding M to 128.
+//
+// Work split (stream-K): the T tiles x KB k-blocks are cut into one
+// contiguous range of k-blocks per CTA (persistent, one CTA per SM). A tile
+// whose k-blocks span two or more CTAs is finished by the CTA holding its
+// first k-block: each other CTA stores its int32 partial accumulator
+// [128][BT] into its own workspace slot and raises per-warp flags; the
+// finishing CTA adds the partials (int32 addition, exact in any order),
+// rescales and stores bf16. A CTA's range is at least one tile long, so the
+// partial of a tile is always written at the start of a range and read at
+// the end of another; flags are cleared by the quantisation kernel that
+// precedes every GEMM launch. With unit = KB the ranges are whole tiles and
+// no partials are used.
+//
+// A k-block is 256 k. One TMA copy brings the x~ tile of a k-block (a 3-D
+// box of two 128-byte-swizzled [BT][128] sub-tiles) and another the packed
+// weights (a 3-D box of 8 row blocks x 2 groups x 512 bytes). A TMA copy
+// costs the issuing thread about the same time whatever its size, so the
+// copies are large and the two streams have a producer warp each. A K that
+// is an odd multiple of 128 leaves the second half of the last k-block
+// outside the tensors, where TMA fills zeros: zero x~ adds nothing.
+//
+// Warp roles (352 threads):
+//   warp 0     TMA producer of the x~ tiles;
+//   warp 1     MMA issuer (one thread) and TMEM owner;
+//   warps 2-5  decode: one thread per weight row (TMEM lane), 256 k per stage;
+//   warps 6-9  epilogue: tcgen05.ld 32 tokens at a time, partial store or
+//              row-sum subtract + rescale to bf16; the [32 tokens][128 rows]
+//              bf16 block is transposed through shared memory (two 8 KiB
+//              buffers) so that y is written with 16-byte stores;
+//   warp 10    TMA producer of the packed weight tiles.
+// TMEM columns: [0, 2 BT) two accumulators, [2 BT, 2 BT + 64 NA) the NA
+// stages of decoded weights (64 columns = 256 k of int8 per lane).
+//
+// Every wait is bounded (mbarriers and inter-CTA flags): on a timeout the
+// kernel records a fault word, raises a block-wide abort flag, each role
+// returns after draining its own copies and MMAs, and TMEM is freed.
+#pragma once
+
+#include "common.cuh"
+
+namespace bitlinear {
+namespace wsg {
+
+constexpr int BW = 128;                    // weight rows per tile (MMA M)
+constexpr int BK = 256;                    // k per stage (k-block)
+constexpr int SUB_K = 128;                 // k per swizzled sub-tile / packed group
+constexpr int UMMA_K = 32;                 // k per tcgen05.mma kind::i8
+constexpr int PK_BYTES = BW * BK / 4;      // packed weights per stage: 8 KiB
+constexpr int DEC_WARPS = 4;
+constexpr int EPI_WARPS = 4;
+constexpr int PK_WARP = 2 + DEC_WARPS + EPI_WARPS;   // second producer
+constexpr int THREADS = (PK_WARP + 1) * 32;
+constexpr uint32_t TMEM_COLS = 512;
+constexpr int SMEM_BUDGET = 200 * 1024;
+constexpr int MAX_GRID = 192;              // upper bound on CTAs (workspace sizing)
+
+template <int BT>
+struct Cfg {
+    static_assert(BT % 32 == 0 && BT >= 32 && BT <= 224, "token tile");
+    static constexpr int X_SUB = BT * SUB_K;                       // one swizzled sub-tile
+    static constexpr int X_BYTES = BT * BK;                        // x~ tile per stage
+    static constexpr int STAGE = X_BYTES + PK_BYTES;
+    static constexpr int NS = (SMEM_BUDGET / STAGE) < 12 ? (SMEM_BUDGET / STAGE) : 12;
+    static constexpr int NA_FIT = (static_cast<int>(TMEM_COLS) - 2 * BT) / 64;
+    static constexpr int NA = NA_FIT < 6 ? NA_FIT : 6;             // TMEM weight stages
+    static constexpr int A_COL0 = 2 * BT;
+    static constexpr int NUM_BARS = 2 * NS + 2 * NA + 4 + 2;
+    static constexpr int EPI_BYTES = 2 * 32 * BW * 2;              // two bf16 [32][128] blocks
+    static constexpr int SMEM_BYTES =
+        1024 + NS * X_BYTES + NS * PK_BYTES + EPI_BYTES + NUM_BARS * 8 + 16;
+    static constexpr uint32_t IDESC = idesc_i8_s32(BW, BT);
+    static_assert(NA >= 2, "TMEM budget");
+    static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
+};
+
+struct Params {
+    int M, N, K;
+    float gamma;
+    const float *beta;      // [M]
+    const int *rowsum;      // [M] sum_k x~
+    uint16_t *y;            // [M][N] bf16
+    int32_t *acc_out;       // [M][N] int32 or null
+    int32_t *partial;       // [grid][BW][BT] int32 (null when unit == KB)
+    int *flags;             // [grid][4] zero at launch (null when unit == KB)
+    int MT;                 // token tiles
+    int T;                  // tiles = MT * ceil(N / BW)
+    int KB;                 // k-blocks (256 k) per tile: ceil(K / 256)
+    int unit;               // k-blocks per partition unit: 1 (stream-K) or KB
+    int base, extra;        // units per CTA: base, plus one for the first `extra`
+    uint64_t wait_limit_ns;
+    int inject_timeout;     // MMA issuer waits on a barrier nobody arrives at
+};
+
+// First k-block (global iteration index) of CTA c's range.
+__device__ __forceinline__ int range_begin(const Params &p, int c)
+{
+    return (c * p.base + min(c, p.extra)) * p.unit;
+}
+
+// The CTA whose range holds global iteration `it`.
+__device__ __forceinline__ int range_owner(const Params &p, int it)
+{
+    const int u = it / p.unit;
+    const int big = p.extra * (p.base + 1);
+    return u < big ? u / (p.base + 1) : p.extra + (u - big) / p.base;
+}
+
+template <int BT>
+__global__ void __launch_bounds__(THREADS, 1)
+gemm_ws_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
+               const Params p)
+{
+    using C = Cfg<BT>;
+    constexpr int NS = C::NS;
+    constexpr int NA = C::NA;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_u32(smem_raw);
+    const uint32_t base = (raw + 1023u) & ~1023u;
+    uint8_t *const base_ptr = smem_raw + (base - raw);
+    const uint32_t sX = base;
+    const uint32_t sP = sX + NS * C::X_BYTES;
+    const uint32_t sEpi = sP + NS * PK_BYTES;
+    const uint32_t sBar = sEpi + C::EPI_BYTES;
+    auto bar = [&](int i) -> uint32_t { return sBar + 8u * static_cast<uint32_t>(i); };
+    auto full_load = [&](int s) { return bar(s); };
+    auto empty_load = [&](int s) { return bar(NS + s); };
+    auto a_full = [&](int a) { return bar(2 * NS + a); };
+    auto a_empty = [&](int a) { return bar(2 * NS + NA + a); };
+    auto acc_full = [&](int b) { return bar(2 * NS + 2 * NA + b); };
+    auto acc_empty = [&](int b) { return bar(2 * NS + 2 * NA + 2 + b); };
+    const uint32_t never_bar = bar(2 * NS + 2 * NA + 4);
+    const uint32_t drain_bar = bar(2 * NS + 2 * NA + 5);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(base_ptr + (sBar - base) + C::NUM_BARS * 8);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const uint64_t limit = p.wait_limit_ns;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < NS; ++s) {
+            mbar_init(full_load(s), 2);
+            mbar_init(empty_load(s), 1 + DEC_WARPS);
+        }
+        for (int a = 0; a < NA; ++a) {
+            mbar_init(a_full(a), DEC_WARPS);
+            mbar_init(a_empty(a), 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(acc_full(b), 1);
+            mbar_init(acc_empty(b), EPI_WARPS);
+        }
+        mbar_init(never_bar, 1);
+        mbar_init(drain_bar, 1);
+        *abort_flag = 0;
+        fence_barrier_init();
+    }
+    if (warp == 0 && lane == 0)
+        prefetch_tensormap(&tmap_x);
+    if (warp == PK_WARP && lane == 0)
+        prefetch_tensormap(&tmap_w);
+    if (warp == 1)
+        tmem_alloc(smem_u32(tmem_slot), TMEM_COLS);
+    tc_fence_before_sync();
+    __syncthreads();
+    tc_fence_after_sync();
+    const uint32_t tmem_base = *tmem_slot;
+    if (warp == 1)
+        tmem_relinquish();
+
+    // x~, beta, the row sums and the flags are written by the preceding
+    // quantisation kernel (programmatic dependent launch).
+    pdl_wait();
+
+    const int it_begin = range_begin(p, blockIdx.x);
+    const int it_end = range_begin(p, blockIdx.x + 1);
+    const int KB = p.KB;
+
+    if (warp == 0 || warp == PK_WARP) {
+        // ----------------------------------------------------- TMA producers
+        // warp 0 copies the x~ tiles, warp PK_WARP the packed weight tiles;
+        // each arms the stage's full barrier with its own byte count.
+        if (lane == 0) {
+            const bool is_x = (warp == 0);
+            int s = 0;
+            uint32_t ph = 0;
+            int armed[NS];
+            for (int i = 0; i < NS; ++i) armed[i] = -1;
+            for (int it = it_begin; it < it_end; ++it) {
+                const int t = it / KB;
+                const int kb = it - t * KB;
+                if (!mbar_wait_bounded(empty_load(s), ph ^ 1u, abort_flag, limit))
+                    break;
+                armed[s] = static_cast<int>(ph);
+                if (is_x) {
+                    const int mt = t % p.MT;
+                    mbar_arrive_expect_tx(full_load(s), C::X_BYTES);
+                    tma_load_3d(sX + s * C::X_BYTES, &tmap_x, 0, mt * BT, 2 * kb, full_load(s));
+                } else {
+                    const int nt = t / p.MT;
+                    mbar_arrive_expect_tx(full_load(s), PK_BYTES);
+                    tma_load_3d(sP + s * PK_BYTES, &tmap_w, 0, 2 * kb, nt * (BW / 16), full_load(s));
+                }
+                if (++s == NS) { s = 0; ph ^= 1u; }
+            }
+            // Wait for every copy this thread started, so no TMA write lands
+            // after the block has exited.
+            for (int i = 0; i < NS; ++i)
+                if (armed[i] >= 0)
+                    drain_wait(full_load(i), static_cast<uint32_t>(armed[i]), limit);
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        // -------------------------------------------------------- MMA issuer
+        if (lane == 0) {
+            int s = 0, a = 0, seg = 0;
+            uint32_t ph = 0, aph = 0;
+            if (p.inject_timeout) {
+                mbar_wait_bounded(never_bar, 0u, abort_flag, limit);
+                goto mma_done;
+            }
+            for (int it = it_begin; it < it_end; ++seg) {
+                const int t = it / KB;
+                const int k0 = it - t * KB;
+                const int k1 = min(KB, k0 + (it_end - it));
+                const int buf = seg & 1;
+                if (!mbar_wait_bounded(acc_empty(buf), ((static_cast<uint32_t>(seg) >> 1) & 1u) ^ 1u,
+                                       abort_flag, limit))
+                    goto mma_done;
+                tc_fence_after_sync();
+                const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * BT);
+                for (int kb = k0; kb < k1; ++kb) {
+                    if (!mbar_wait_bounded(full_load(s), ph, abort_flag, limit))
+                        goto mma_done;
+                    if (!mbar_wait_bounded(a_full(a), aph, abort_flag, limit))
+                        goto mma_done;
+                    tc_fence_after_sync();
+                    const uint32_t a_tmem = tmem_base + static_cast<uint32_t>(C::A_COL0 + 64 * a);
+#pragma unroll
+                    for (int kk = 0; kk < BK / UMMA_K; ++kk) {
+                        const uint64_t bdesc = smem_desc_k128_sw128(
+                            sX + s * C::X_BYTES + (kk / 4) * C::X_SUB + (kk % 4) * UMMA_K);
+                        umma_i8_tmem_a(d_tmem, a_tmem + static_cast<uint32_t>(8 * kk), bdesc,
+                                       C::IDESC, (kb > k0 || kk > 0) ? 1u : 0u);
+                    }
+                    umma_commit(empty_load(s));
+                    umma_commit(a_empty(a));
+                    if (++s == NS) { s = 0; ph ^= 1u; }
+                    if (++a == NA) { a = 0; aph ^= 1u; }
+                }
+                umma_commit(acc_full(buf));
+                it += k1 - k0;
+            }
+        mma_done:
+            // All MMAs issued by this thread complete before TMEM is freed.
+            umma_commit(drain_bar);
+            drain_wait(drain_bar, 0u, limit);
+        }
+        __syncwarp();
+    } else if (warp < 2 + DEC_WARPS) {
+        // ------------------------------------------------------------ decode
+        // Thread = weight row r of the tile = TMEM lane r. The packed stage
+        // is [8 row blocks][2 groups][16 rows][32 B]; in group g, word w of
+        // row r has k = 128 g + 16 w + 4 j + b at bits 8 b + 2 j, so plane j
+        // of word w goes to TMEM column 32 g + 4 w + j (four k per column,
+        // k = 4 c + b in byte b).
+        const int q = warp & 3;
+        const int r = 32 * q + lane;
+        const uint32_t lane_off = static_cast<uint32_t>(32 * q) << 16;
+        const int row_off = (r >> 4) * 1024 + (r & 15) * 32;
+        int s = 0, a = 0;
+        uint32_t ph = 0, aph = 0;
+        for (int it = it_begin; it < it_end; ++it) {
+            if (!warp_wait_bounded(full_load(s), ph, abort_flag, limit))
+                break;
+            if (!warp_wait_bounded(a_empty(a), aph ^ 1u, abort_flag, limit))
+                break;
+            tc_fence_after_sync();
+            const uint8_t *stage = base_ptr + (sP - base) + s * PK_BYTES + row_off;
+#pragma unroll
+            for (int g = 0; g < 2; ++g) {
+                const uint4 w0 = *reinterpret_cast<const uint4 *>(stage + 512 * g);
+                const uint4 w1 = *reinterpret_cast<const uint4 *>(stage + 512 * g + 16);
+                const uint32_t wd[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+                uint32_t v[32];
+#pragma unroll
+                for (int w = 0; w < 8; ++w) {
+                    v[4 * w + 0] = wd[w] & 0x03030303u;
+                    v[4 * w + 1] = (wd[w] >> 2) & 0x03030303u;
+                    v[4 * w + 2] = (wd[w] >> 4) & 0x03030303u;
+                    v[4 * w + 3] = (wd[w] >> 6) & 0x03030303u;
+                }
+                tmem_st_32x32b_x32(
+                    tmem_base + lane_off + static_cast<uint32_t>(C::A_COL0 + 64 * a + 32 * g), v);
+            }
+            tmem_st_wait();
+            tc_fence_before_sync();
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(a_full(a));
+                mbar_arrive(empty_load(s));
+            }
+            if (++s == NS) { s = 0; ph ^= 1u; }
+            if (++a == NA) { a = 0; aph ^= 1u; }
+        }
+    } else {
+        // ---------------------------------------------------------- epilogue
+        const int q = warp & 3;
+        const int row = 32 * q + lane;                      // weight row in the tile
+        const uint32_t lane_off = static_cast<uint32_t>(32 * q) << 16;
+        int seg = 0;
+        int epi_chunk = 0;                 // alternates the two transpose buffers
+        for (int it = it_begin; it < it_end; ++seg) {
+            const int t = it / KB;
+            const int k0 = it - t * KB;
+            const int k1 = min(KB, k0 + (it_end - it));
+            it += k1 - k0;
+            const int buf = seg & 1;
+            const int mt = t % p.MT;
+            const int nt = t / p.MT;
+
+            // Per-token scale and row sum of this tile, fetched before the
+            // accumulator is ready: lane l holds token mt * BT + 32 c + l.
+            float s_pf[BT / 32];
+            int rs_pf[BT / 32];
+            if (k0 == 0) {
+#pragma unroll
+                for (int c = 0; c < BT / 32; ++c) {
+                    const int ml = mt * BT + 32 * c + lane;
+                    s_pf[c] = ml < p.M ? out_scale(__ldg(p.beta + ml), p.gamma) : 0.0f;
+                    rs_pf[c] = ml < p.M ? __ldg(p.rowsum + ml) : 0;
+                }
+            }
+
+            // The four epilogue warps take every wait's verdict together (named
+            // barrier 1), so none can be left behind at the transpose barrier.
+            bool ready = warp_wait_bounded(acc_full(buf), (static_cast<uint32_t>(seg) >> 1) & 1u,
+                                           abort_flag, limit);
+            if (!named_bar_and(1, EPI_WARPS * 32, ready))
+                break;
+            tc_fence_after_sync();
+            const uint32_t d_cols = tmem_base + lane_off + static_cast<uint32_t>(buf * BT);
+
+            if (k0 > 0) {
+                // Not the tile's first k-block: hand the partial sum to the
+                // CTA that finishes the tile.
+                int32_t *slot = p.partial + (static_cast<size_t>(blockIdx.x) * BW + row) * BT;
+#pragma unroll 1
+                for (int c = 0; c < BT / 32; ++c) {
+                    uint32_t r[32];
+                    tmem_ld_32x32b_x32(d_cols + static_cast<uint32_t>(32 * c), r);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int g = 0; g < 8; ++g)
+                        __stcg(reinterpret_cast<int4 *>(slot + 32 * c + 4 * g),
+                               make_int4(static_cast<int>(r[4 * g]), static_cast<int>(r[4 * g + 1]),
+                                         static_cast<int>(r[4 * g + 2]),
+                                         static_cast<int>(r[4 * g + 3])));
+                }
+                __threadfence();
+                tc_fence_before_sync();
+                __syncwarp();
+                if (lane == 0) {
+                    st_release_gpu(p.flags + 4 * blockIdx.x + q, 1);
+                    mbar_arrive(acc_empty(buf));
+                }
+                continue;
+            }
+
+            // First k-block of the tile is here: this CTA finishes the tile.
+            // Other contributors: the CTAs holding the tile's later k-blocks.
+            const int c_last =
+                (k1 < KB) ? range_owner(p, t * KB + KB - 1) : static_cast<int>(blockIdx.x);
+            bool ok = true;
+            if (c_last > static_cast<int>(blockIdx.x)) {
+                if (lane == 0) {
+                    for (int c2 = blockIdx.x + 1; c2 <= c_last && ok; ++c2) {
+                        const int *f = p.flags + 4 * c2 + q;
+                        if (ld_acquire_gpu(f) != 0)
+                            continue;
+                        const uint64_t t0 = global_timer_ns();
+                        for (uint32_t spin = 1;; ++spin) {
+                            if (ld_acquire_gpu(f) != 0)
+                                break;
+                            if ((spin & 15u) == 0u) {
+                                if (*abort_flag) { ok = false; break; }
+                                if (global_timer_ns() - t0 > limit) {
+                                    atomicOr(&g_fault_word, FAULT_WAIT_TIMEOUT);
+                                    *abort_flag = 1;
+                                    ok = false;
+                                    break;
+                                }
+                            }
+                        }
+                    }
+                }
+                ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+                for (int c2 = blockIdx.x + 1; ok && c2 <= c_last; ++c2)
+                    (void)ld_acquire_gpu(p.flags + 4 * c2 + q);
+            }
+            if (!named_bar_and(1, EPI_WARPS * 32, ok))
+                break;
+
+            const int n = nt * BW + row;
+            const bool n_ok = n < p.N;
+            const bool vec_out = (p.N % 8) == 0;
+#pragma unroll
+            for (int c = 0; c < BT / 32; ++c) {
+                const int m0 = mt * BT + 32 * c;
+                if (m0 >= p.M)
+                    break;
+                uint32_t r[32];
+                tmem_ld_32x32b_x32(d_cols + static_cast<uint32_t>(32 * c), r);
+                tmem_ld_wait();
+                for (int c2 = blockIdx.x + 1; c2 <= c_last; ++c2) {
+                    const int32_t *slot =
+                        p.partial + (static_cast<size_t>(c2) * BW + row) * BT + 32 * c;
+#pragma unroll
+                    for (int g = 0; g < 8; ++g) {
+                        const int4 v = __ldcg(reinterpret_cast<const int4 *>(slot + 4 * g));
+                        r[4 * g] += static_cast<uint32_t>(v.x);
+                        r[4 * g + 1] += static_cast<uint32_t>(v.y);
+                        r[4 * g + 2] += static_cast<uint32_t>(v.z);
+                        r[4 * g + 3] += static_cast<uint32_t>(v.w);
+                    }
+                }
+                const int jn = min(32, p.M - m0);
+                if (p.acc_out != nullptr) {
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) {
+                        const int rs = __shfl_sync(0xffffffffu, rs_pf[c], j);
+                        if (j < jn && n_ok)
+                            p.acc_out[static_cast<size_t>(m0 + j) * p.N + n] =
+                                static_cast<int>(r[j]) - rs;
+                    }
+                }
+                if (vec_out) {
+                    // [32 tokens][128 rows] bf16 block in shared memory, then
+                    // 16-byte stores: 16 lanes cover one token's 256 bytes.
+                    uint16_t *blk = reinterpret_cast<uint16_t *>(
+                        base_ptr + (sEpi - base) + (epi_chunk & 1) * (32 * BW * 2));
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) {
+                        const float s = __shfl_sync(0xffffffffu, s_pf[c], j);
+                        const int rs = __shfl_sync(0xffffffffu, rs_pf[c], j);
+                        blk[j * BW + row] = rescale_bf16(static_cast<int>(r[j]) - rs, s);
+                    }
+                    asm volatile("bar.sync 1, %0;" ::"r"(EPI_WARPS * 32) : "memory");
+                    const int et = (warp - 2 - DEC_WARPS) * 32 + lane;   // 0 .. 127
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const int sg = et + 128 * i;                    // 16-byte segment
+                        const int j = sg >> 4;
+                        const int piece = sg & 15;
+                        const int nn = nt * BW + 8 * piece;
+                        if (j < jn && nn < p.N) {
+                            const uint4 v = *reinterpret_cast<const uint4 *>(blk + j * BW + 8 * piece);
+                            *reinterpret_cast<uint4 *>(p.y + static_cast<size_t>(m0 + j) * p.N + nn) = v;
+                        }
+                    }
+                    ++epi_chunk;
+                } else {
+                    uint16_t *yrow = p.y + static_cast<size_t>(m0) * p.N + n;
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) {
+                        const float s = __shfl_sync(0xffffffffu, s_pf[c], j);
+                        const int rs = __shfl_sync(0xffffffffu, rs_pf[c], j);
+                        if (j < jn && n_ok)
+                            yrow[static_cast<size_t>(j) * p.N] =
+                                rescale_bf16(static_cast<int>(r[j]) - rs, s);
+                    }
+                }
+            }
+            tc_fence_before_sync();
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(acc_empty(buf));
+        }
+    }
+
+    // ------------------------------------------------------------ teardown
+    tc_fence_before_sync();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after_sync();
+        tmem_dealloc(tmem_base, TMEM_COLS);
+    }
+}
+
+}  // namespace wsg
+}  // namespace bitlinear

@@ -3,12 +3,14 @@
 // the listing's quantize_activations_int8 fixes the clamp(min=1e-5), the
 // order x * (127 / beta) and ties-to-even rounding).
 //
-// One warp per token row, eight rows per block, no block barriers. Each lane
-// keeps up to CACHE vectors of 8 activations in registers from the absmax
-// pass, so rows of up to 32 * 8 * CACHE elements are read from memory once;
-// longer rows are re-read in the second pass, from L1. The row sum of x~ is
-// written for the tensor-core path, whose GEMM contracts the non-negative
-// weight codes W~ + 1 (acc = sum x~ * code - sum x~).
+// WPR warps per token row (one for rows up to a few thousand elements, eight
+// for long rows), 256 threads per block. Each lane keeps CACHE vectors of 8
+// activations in registers from the absmax pass, so a row is read from
+// memory once when 32 * WPR * 8 * CACHE covers it; anything beyond is
+// re-read in the second pass, four vectors in flight per lane. The row sum
+// of x~ is written for the tensor-core path, whose GEMM contracts the
+// non-negative weight codes W~ + 1 (acc = sum x~ * code - sum x~). Block 0
+// also clears the GEMM's inter-block flag words when asked to.
 #pragma once
 
 #include "common.cuh"
@@ -17,27 +19,46 @@ namespace bitlinear {
 namespace qa {
 
 constexpr int THREADS = 256;
-constexpr int ROWS_PER_BLOCK = THREADS / 32;
+constexpr int WARPS = THREADS / 32;
 
-template <bool BF16, int CACHE>
+template <int WPR>
+__host__ __device__ constexpr int rows_per_block() { return WARPS / WPR; }
+
+template <bool BF16, int CACHE, int WPR>
 __global__ void __launch_bounds__(THREADS)
 quant_act_kernel(const void *__restrict__ x, int M, int K, int8_t *__restrict__ xq,
-                 float *__restrict__ beta_out, int *__restrict__ rowsum_out)
+                 float *__restrict__ beta_out, int *__restrict__ rowsum_out,
+                 int *__restrict__ clear, int n_clear)
 {
+    static_assert(WARPS % WPR == 0, "warps per row");
+    constexpr int STRIDE = 32 * WPR;              // vectors between a lane's vectors
+    __shared__ uint32_t red_max[WARPS];
+    __shared__ int red_sum[WARPS];
+    const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int m = blockIdx.x * ROWS_PER_BLOCK + (threadIdx.x >> 5);
+    const int part = warp % WPR;
+    const int m = blockIdx.x * rows_per_block<WPR>() + warp / WPR;
     pdl_wait();
-    if (m >= M)
+    // The GEMM that follows uses these words as inter-block flags; they are
+    // cleared here, after every earlier grid in the stream has finished.
+    if (clear != nullptr && blockIdx.x == 0)
+        for (int i = threadIdx.x; i < n_clear; i += THREADS)
+            clear[i] = 0;
+    // Rows past M still take part in the block barriers (WPR > 1).
+    const bool active = m < M;
+    if (WPR == 1 && !active)
         return;
     const size_t elem = BF16 ? 2 : 4;
-    const void *row = static_cast<const char *>(x) + static_cast<size_t>(m) * K * elem;
-    const int nvec = K >> 3;
+    const void *row = static_cast<const char *>(x) +
+                      static_cast<size_t>(active ? m : 0) * K * elem;
+    const int nvec = active ? (K >> 3) : 0;
+    const int v0 = part * 32 + lane;
 
     Vec8<BF16> cache[CACHE];
     float amax = 0.0f;
 #pragma unroll
     for (int i = 0; i < CACHE; ++i) {
-        const int v = lane + 32 * i;
+        const int v = v0 + STRIDE * i;
         if (v < nvec) {
             cache[i].load(row, v * 8);
 #pragma unroll
@@ -45,18 +66,34 @@ quant_act_kernel(const void *__restrict__ x, int M, int K, int8_t *__restrict__ 
                 amax = fmaxf(amax, fabsf(cache[i].get(j)));
         }
     }
-    for (int v = lane + 32 * CACHE; v < nvec; v += 32) {
-        Vec8<BF16> t;
-        t.load(row, v * 8);
+    for (int vb = v0 + STRIDE * CACHE; vb < nvec; vb += 4 * STRIDE) {
+        Vec8<BF16> t[4];
 #pragma unroll
-        for (int j = 0; j < 8; ++j)
-            amax = fmaxf(amax, fabsf(t.get(j)));
+        for (int u = 0; u < 4; ++u)
+            if (vb + u * STRIDE < nvec)
+                t[u].load(row, (vb + u * STRIDE) * 8);
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+            if (vb + u * STRIDE < nvec)
+#pragma unroll
+                for (int j = 0; j < 8; ++j)
+                    amax = fmaxf(amax, fabsf(t[u].get(j)));
     }
-    const float beta =
-        fmaxf(__uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(amax))), 1e-5f);
+    uint32_t umax = __reduce_max_sync(0xffffffffu, __float_as_uint(amax));
+    if constexpr (WPR > 1) {
+        if (lane == 0)
+            red_max[warp] = umax;
+        __syncthreads();
+        const int w0 = warp - part;
+        umax = red_max[w0];
+#pragma unroll
+        for (int w = 1; w < WPR; ++w)
+            umax = max(umax, red_max[w0 + w]);
+    }
+    const float beta = fmaxf(__uint_as_float(umax), 1e-5f);
     const float scale = __fdiv_rn(127.0f, beta);
 
-    int8_t *out = xq + static_cast<size_t>(m) * K;
+    int8_t *out = xq + static_cast<size_t>(active ? m : 0) * K;
     int sum = 0;
     auto quant_store = [&](const Vec8<BF16> &t, int v) {
         uint32_t lo = 0, hi = 0;
@@ -72,18 +109,34 @@ quant_act_kernel(const void *__restrict__ x, int M, int K, int8_t *__restrict__ 
     };
 #pragma unroll
     for (int i = 0; i < CACHE; ++i) {
-        const int v = lane + 32 * i;
+        const int v = v0 + STRIDE * i;
         if (v < nvec)
             quant_store(cache[i], v);
     }
-    for (int v = lane + 32 * CACHE; v < nvec; v += 32) {
-        Vec8<BF16> t;
-        t.load(row, v * 8);
-        quant_store(t, v);
+    for (int vb = v0 + STRIDE * CACHE; vb < nvec; vb += 4 * STRIDE) {
+        Vec8<BF16> t[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+            if (vb + u * STRIDE < nvec)
+                t[u].load(row, (vb + u * STRIDE) * 8);
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+            if (vb + u * STRIDE < nvec)
+                quant_store(t[u], vb + u * STRIDE);
     }
     pdl_launch_dependents();
     sum = __reduce_add_sync(0xffffffffu, sum);
-    if (lane == 0) {
+    if constexpr (WPR > 1) {
+        if (lane == 0)
+            red_sum[warp] = sum;
+        __syncthreads();
+        const int w0 = warp - part;
+        sum = 0;
+#pragma unroll
+        for (int w = 0; w < WPR; ++w)
+            sum += red_sum[w0 + w];
+    }
+    if (active && part == 0 && lane == 0) {
         beta_out[m] = beta;
         if (rowsum_out != nullptr)
             rowsum_out[m] = sum;

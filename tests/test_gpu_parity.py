@@ -68,6 +68,21 @@ def test_tc_parity(cuda, M, K, N):
     assert exact == 1.0
 
 
+@pytest.mark.parametrize("M", [20, 50, 200, 300])
+def test_tc_token_tiles_shared_k(cuda, M):
+    # token tiles of 32, 64, 128 and 192 rows; only a few tiles with 54
+    # k-blocks each, so the k-range of every tile is shared by many CTAs
+    # whose int32 partial sums are combined by the tile's first CTA
+    c = Case(M, 6912, 300, w_seed=M, x_seed=M + 1)
+    assert c.check_full(c.run(path=bl.PATH_TC)) == 1.0
+
+
+def test_tc_tiles_split_between_two_ctas(cuda):
+    # 160 tiles of 10 k-blocks over the CTAs: most tiles are split in two
+    c = Case(1000, 1280, 2560, w_seed=21, x_seed=22)
+    assert c.check_full(c.run(path=bl.PATH_TC)) == 1.0
+
+
 def test_tc_many_tiles_per_cta(cuda):
     # more tiles than SMs: every CTA loops over several tiles and both TMEM
     # accumulator buffers are reused
