@@ -231,7 +231,7 @@ gemm_ws_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
         // -------------------------------------------------------- MMA issuer
         if (lane == 0) {
             int s = 0, a = 0, seg = 0;
-            uint32_t ph = 0, aph = 0;
+            uint32_t aph = 0;
             if (p.inject_timeout) {
                 mbar_wait_bounded(never_bar, 0u, abort_flag, limit);
                 goto mma_done;
@@ -247,8 +247,12 @@ gemm_ws_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
                 tc_fence_after_sync();
                 const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * BT);
                 for (int kb = k0; kb < k1; ++kb) {
-                    if (!mbar_wait_bounded(full_load(s), ph, abort_flag, limit))
-                        goto mma_done;
+                    // a_full(a) completes only after the decode warps have
+                    // seen full_load(s) (both TMA copies of the stage, x~
+                    // included, have landed) and written the codes, so one
+                    // wait covers both operands. Waiting on the transaction
+                    // barrier here as well costs the issuing thread more than
+                    // the short MMA queue holds.
                     if (!mbar_wait_bounded(a_full(a), aph, abort_flag, limit))
                         goto mma_done;
                     tc_fence_after_sync();
@@ -262,7 +266,7 @@ gemm_ws_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
                     }
                     umma_commit(empty_load(s));
                     umma_commit(a_empty(a));
-                    if (++s == NS) { s = 0; ph ^= 1u; }
+                    if (++s == NS) s = 0;
                     if (++a == NA) { a = 0; aph ^= 1u; }
                 }
                 umma_commit(acc_full(buf));
