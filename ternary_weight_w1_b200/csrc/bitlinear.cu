@@ -30,7 +30,10 @@ namespace {
 constexpr int64_t kMaxK = 65536;
 constexpr int kGemvMaxM = 16;
 constexpr int64_t kGemvMaxXqBytes = 196608;       // M * K bytes of x~ in shared memory
-constexpr int64_t kAutoGemvMaxM = 16;
+constexpr int64_t kAutoGemvMaxM = 6;                // above: tensor-core path
+// Split the k-range of fewer tiles than CTAs only when a CTA saves more than
+// this many 256-k blocks (each about half a microsecond) by it.
+constexpr double kSplitMinSavedBlocks = 10.0;
 constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s: far above any legitimate wait
 constexpr int kMaxDevices = 64;
 
@@ -461,10 +464,18 @@ int run_tc_path(const void *x, bitlinear_dtype xdt, int M, int K, const void *pa
     const int KB = (K + wsg::BK - 1) / wsg::BK;
     const int MT = (M + BT - 1) / BT;
     const int T = MT * ((N + wsg::BW - 1) / wsg::BW);
+    const int slots = std::min(dev.sms, wsg::MAX_GRID);
+    // Splitting a tile's k-range between CTAs costs a hand-off of a few
+    // microseconds (partial store, flag, partial load). With at least as many
+    // tiles as CTAs it evens out the last wave; with fewer tiles it pays only
+    // when the k-blocks a CTA saves outweigh that hand-off.
+    if (split && T < slots) {
+        const double saved_blocks = KB * (1.0 - static_cast<double>(T) / slots);
+        split = saved_blocks > kSplitMinSavedBlocks;
+    }
     const int unit = split ? 1 : KB;
     const int64_t units = static_cast<int64_t>(T) * KB / unit;
-    const int grid = static_cast<int>(
-        std::min<int64_t>(units, std::min(dev.sms, wsg::MAX_GRID)));
+    const int grid = static_cast<int>(std::min<int64_t>(units, slots));
     TcWorkspace w = tc_workspace(ws, M, K, split);
     int rc = launch_quant_act(x, xdt, M, K, w.xq, w.beta, w.rowsum, st, w.flags,
                               split ? 4 * grid : 0);

@@ -378,7 +378,8 @@ gemm_ws_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
                                          static_cast<int>(r[4 * g + 2]),
                                          static_cast<int>(r[4 * g + 3])));
                 }
-                __threadfence();
+                // The warp barrier orders every lane's stores before lane 0's
+                // release of the flag (a release is cumulative).
                 tc_fence_before_sync();
                 __syncwarp();
                 if (lane == 0) {
@@ -392,32 +393,39 @@ gemm_ws_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
             // Other contributors: the CTAs holding the tile's later k-blocks.
             const int c_last =
                 (k1 < KB) ? range_owner(p, t * KB + KB - 1) : static_cast<int>(blockIdx.x);
+            // Every lane polls some of the contributors' flags (lane l takes
+            // contributors blockIdx.x + 1 + l, + 33, ...), so all of them are
+            // read in one round trip when they are already set.
             bool ok = true;
-            if (c_last > static_cast<int>(blockIdx.x)) {
-                if (lane == 0) {
-                    for (int c2 = blockIdx.x + 1; c2 <= c_last && ok; ++c2) {
-                        const int *f = p.flags + 4 * c2 + q;
-                        if (ld_acquire_gpu(f) != 0)
-                            continue;
-                        const uint64_t t0 = global_timer_ns();
-                        for (uint32_t spin = 1;; ++spin) {
-                            if (ld_acquire_gpu(f) != 0)
-                                break;
-                            if ((spin & 15u) == 0u) {
-                                if (*abort_flag) { ok = false; break; }
-                                if (global_timer_ns() - t0 > limit) {
-                                    atomicOr(&g_fault_word, FAULT_WAIT_TIMEOUT);
-                                    *abort_flag = 1;
-                                    ok = false;
-                                    break;
-                                }
+            const int n_contrib = c_last - static_cast<int>(blockIdx.x);
+            if (n_contrib > 0) {
+                const uint64_t t0 = global_timer_ns();
+                for (uint32_t spin = 0;; ++spin) {
+                    bool mine = true;
+                    for (int c2 = blockIdx.x + 1 + lane; c2 <= c_last; c2 += 32)
+                        mine = mine && (ld_acquire_gpu(p.flags + 4 * c2 + q) != 0);
+                    if (__all_sync(0xffffffffu, mine))
+                        break;
+                    if ((spin & 15u) == 15u) {
+                        int stop = 0;
+                        if (lane == 0) {
+                            if (*abort_flag) {
+                                stop = 1;
+                            } else if (global_timer_ns() - t0 > limit) {
+                                atomicOr(&g_fault_word, FAULT_WAIT_TIMEOUT);
+                                *abort_flag = 1;
+                                stop = 1;
                             }
+                        }
+                        if (__shfl_sync(0xffffffffu, stop, 0)) {
+                            ok = false;
+                            break;
                         }
                     }
                 }
-                ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-                for (int c2 = blockIdx.x + 1; ok && c2 <= c_last; ++c2)
-                    (void)ld_acquire_gpu(p.flags + 4 * c2 + q);
+                // Each flag was read with acquire semantics by some lane; the
+                // warp barrier orders those reads before every lane's loads.
+                __syncwarp();
             }
             if (!named_bar_and(1, EPI_WARPS * 32, ok))
                 break;
@@ -433,16 +441,26 @@ gemm_ws_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
                 uint32_t r[32];
                 tmem_ld_32x32b_x32(d_cols + static_cast<uint32_t>(32 * c), r);
                 tmem_ld_wait();
-                for (int c2 = blockIdx.x + 1; c2 <= c_last; ++c2) {
-                    const int32_t *slot =
-                        p.partial + (static_cast<size_t>(c2) * BW + row) * BT + 32 * c;
+                // Partial sums of the other contributors, two at a time so
+                // that their loads are in flight together.
+                for (int c2 = blockIdx.x + 1; c2 <= c_last; c2 += 2) {
+                    const bool two = (c2 + 1 <= c_last);
+                    const int4 *sa = reinterpret_cast<const int4 *>(
+                        p.partial + (static_cast<size_t>(c2) * BW + row) * BT + 32 * c);
+                    const int4 *sb = reinterpret_cast<const int4 *>(
+                        p.partial + (static_cast<size_t>(two ? c2 + 1 : c2) * BW + row) * BT + 32 * c);
+                    int4 va[8], vb[8];
 #pragma unroll
                     for (int g = 0; g < 8; ++g) {
-                        const int4 v = __ldcg(reinterpret_cast<const int4 *>(slot + 4 * g));
-                        r[4 * g] += static_cast<uint32_t>(v.x);
-                        r[4 * g + 1] += static_cast<uint32_t>(v.y);
-                        r[4 * g + 2] += static_cast<uint32_t>(v.z);
-                        r[4 * g + 3] += static_cast<uint32_t>(v.w);
+                        va[g] = __ldcg(sa + g);
+                        vb[g] = two ? __ldcg(sb + g) : make_int4(0, 0, 0, 0);
+                    }
+#pragma unroll
+                    for (int g = 0; g < 8; ++g) {
+                        r[4 * g] += static_cast<uint32_t>(va[g].x + vb[g].x);
+                        r[4 * g + 1] += static_cast<uint32_t>(va[g].y + vb[g].y);
+                        r[4 * g + 2] += static_cast<uint32_t>(va[g].z + vb[g].z);
+                        r[4 * g + 3] += static_cast<uint32_t>(va[g].w + vb[g].w);
                     }
                 }
                 const int jn = min(32, p.M - m0);
