@@ -9,7 +9,9 @@ N(0, 0.02) latents packed 2 bits per weight. The packed weights rotate over
 32 device copies (283 MB, more than twice the 126 MB L2), so every step
 streams its weights from HBM. The headline is the GEMV's HBM throughput on
 packed-weight bytes. The same line carries the prefill GEMM (M = 2048 tokens,
-int8 tensor cores) in ``prefill_gemm``.
+int8 tensor cores) in ``prefill_gemm``, the 30-layer decoder set at decode
+batches 1, 8 and 64 in ``layer_set`` and the large-model shapes in
+``large_sweep``.
 
 With ``--gpus N`` (launched by torchrun, one process per GPU) every rank runs
 the same independent workload (weak scaling: the path has no data-path
@@ -352,6 +354,102 @@ def bench_prefill(bl, device, reps: int = 20):
     return ms, ops
 
 
+def time_graph(fn, reps: int) -> float:
+    """Mean ms of `fn` (captured once in a CUDA graph) over `reps` replays,
+    after three warm-up replays."""
+    import torch
+    g = capture_graph(fn)
+    for _ in range(3):
+        g.replay()
+    torch.cuda.synchronize()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record()
+    for _ in range(reps):
+        g.replay()
+    end.record()
+    torch.cuda.synchronize()
+    del g
+    return start.elapsed_time(end) / reps
+
+
+def bench_layer_set(bl, device, batches=(1, 8, 64), reps: int = 10):
+    """The seven projections of the 2B decoder layer for 30 layers (521 MB of
+    packed weights, more than four times L2) at decode batch B, through the
+    automatic dispatch: one grouped GEMV launch per layer at B = 1, one
+    bitlinear_forward per projection (quantisation + tensor-core GEMM) at
+    B > 6. The 30 layers hold distinct device copies of one seeded layer's
+    packed weights (the parity tests use independent seeds per layer)."""
+    import torch
+    layer = workloads.layer_set_2b(1, layers=1).problems
+    packed = []
+    for p in layer:
+        pk, gamma = bl.bitlinear_pack_weights(p.weights())
+        packed.append((p, torch.from_numpy(pk).to(device), gamma))
+    layers = workloads.NUM_LAYERS
+    copies = [[(p, dp if li == 0 else dp.clone(), g) for p, dp, g in packed]
+              for li in range(layers)]
+    wbytes = layers * sum(p.N * p.K // 4 for p, _, _ in packed)
+    out = {}
+    for B in batches:
+        xs = [bf16_tensor(workloads.activations_bf16(B, p.K, p.x_seed), device) for p, _, _ in packed]
+        ys = [torch.empty((B, p.N), dtype=torch.bfloat16, device=device) for p, _, _ in packed]
+        ws_bytes = max(bl.bitlinear_workspace_bytes(B, p.N, p.K) for p, _, _ in packed)
+        ws = torch.empty((max(ws_bytes, 1),), dtype=torch.uint8, device=device)
+        if B <= 6:
+            def step():
+                for li in range(layers):
+                    bl.bitlinear_forward_grouped(
+                        [(xs[k], dp, g, p.N, ys[k]) for k, (p, dp, g) in enumerate(copies[li])])
+            launches = layers
+        else:
+            def step():
+                for li in range(layers):
+                    for k, (p, dp, g) in enumerate(copies[li]):
+                        bl.bitlinear_forward(xs[k], dp, g, p.N, y=ys[k], workspace=ws)
+            launches = layers * len(packed) * 2
+        step()
+        torch.cuda.synchronize()
+        ms = time_graph(step, reps)
+        out[f"B={B}"] = {"us_per_layer": round(ms * 1e3 / layers, 2),
+                         "GBps_packed": round(wbytes / (ms * 1e-3) / 1e9, 1),
+                         "TOPS": round(2 * B * wbytes * 4 / (ms * 1e-3) / 1e12, 2),
+                         "launches_per_step": launches}
+    return out
+
+
+def bench_large_sweep(bl, device, ms_list=(1, 16, 256, 4096), reps: int = 5):
+    """K=8192->N=28672 and K=28672->N=8192 (58.7 MB of packed weights each)
+    at M tokens, automatic dispatch, weights rotating over 3 copies per matrix
+    (352 MB in total). Per M: microseconds per matrix pair, GB/s of packed
+    weights and int8 TOPS."""
+    import torch
+    out = {}
+    mats = []
+    for p in workloads.large_sweep(1).problems:
+        pk, gamma = bl.bitlinear_pack_weights(p.weights())
+        dp = torch.from_numpy(pk).to(device)
+        mats.append((p, [dp, dp.clone(), dp.clone()], gamma))
+    wbytes = sum(p.N * p.K // 4 for p, _, _ in mats)
+    for M in ms_list:
+        xs = [bf16_tensor(workloads.activations_bf16(M, p.K, p.x_seed), device) for p, _, _ in mats]
+        ys = [torch.empty((M, p.N), dtype=torch.bfloat16, device=device) for p, _, _ in mats]
+        ws_bytes = max(bl.bitlinear_workspace_bytes(M, p.N, p.K) for p, _, _ in mats)
+        ws = torch.empty((max(ws_bytes, 1),), dtype=torch.uint8, device=device)
+
+        def step():
+            for c in range(3):
+                for k, (p, dps, g) in enumerate(mats):
+                    bl.bitlinear_forward(xs[k], dps[c], g, p.N, y=ys[k], workspace=ws)
+        step()
+        torch.cuda.synchronize()
+        ms = time_graph(step, reps) / 3
+        out[f"M={M}"] = {"us_per_pair": round(ms * 1e3, 2),
+                         "GBps_packed": round(wbytes / (ms * 1e-3) / 1e9, 1),
+                         "TOPS": round(2 * M * wbytes * 4 / (ms * 1e-3) / 1e12, 1)}
+        del xs, ys, ws
+    return out
+
+
 def cpu_baseline_oracle(seconds: float = 10.0):
     """The oracle (single-threaded C) on the decode step: x quantisation,
     integer product and rescale for the up and down projections, repeated
@@ -459,6 +557,14 @@ def run_ours(args, dist):
                          "peak": int8_peak, "peak_note": "measured bf16 burst x 2 (nominal int8/bf16)",
                          "frac": round(pre_tops / int8_peak, 4)},
     }
+    if not args.no_extra:
+        out["layer_set"] = {
+            "workload": "2B decoder layer (q 2560->2560, k/v 2560->640, o 2560->2560, gate/up "
+                        "2560->6912, down 6912->2560) x 30 layers, 521 MB of packed weights",
+            **bench_layer_set(bl, device)}
+        out["large_sweep"] = {
+            "workload": "K=8192->N=28672 and K=28672->N=8192 per step, 117 MB of packed weights",
+            **bench_large_sweep(bl, device)}
     if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
         v, steps, el = cpu_baseline_oracle(args.cpu_seconds)
         out["cpu_baseline"] = {"value": round(v, 4), "unit": UNIT, "cores": 1, "kind": "oracle",
@@ -520,6 +626,8 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=20000)
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extra", action="store_true",
+                    help="skip the layer-set and large-shape measurements")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
