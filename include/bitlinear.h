@@ -122,8 +122,13 @@ int bitlinear_quant_act(const void *x_dev, bitlinear_dtype xdt, int64_t M,
 /* ---------------------------------------------------------------- forward */
 
 /* Device workspace bytes bitlinear_forward needs for (M, N, K): 0 when the
- * GEMV path is taken (small M), else room for x~ (M*K bytes), beta and the
- * per-token sums of x~. Returns SIZE_MAX for invalid shapes. */
+ * GEMV path is taken (M <= 6), else room for x~ (M*K bytes), beta, the
+ * per-token sums of x~, and the tensor-core GEMM's inter-CTA region (flag
+ * words and int32 partial sums of tiles whose k-range is split between
+ * CTAs; at most 192 * 128 * 192 * 4 bytes). The flag words are cleared by
+ * the call itself before its GEMM reads them, so the workspace needs no
+ * initialisation, but two calls that may run at the same time (different
+ * streams) must not share one. Returns SIZE_MAX for invalid shapes. */
 size_t bitlinear_workspace_bytes(int64_t M, int64_t N, int64_t K);
 
 /* y = BitLinear(x) with pre-packed ternary weights, on the device.
@@ -140,9 +145,11 @@ size_t bitlinear_workspace_bytes(int64_t M, int64_t N, int64_t K);
  *   xq_dev_or_null   [out, optional] [M][K] int8 x~
  *   beta_dev_or_null [out, optional] [M] fp32 beta
  * The optional outputs exist so that tests can compare the integer stages
- * bit for bit; pass NULL in production. Small M runs one fused kernel
+ * bit for bit; pass NULL in production. M <= 6 runs one fused kernel
  * (quantisation in the prologue, dp4a over the packed weights); larger M runs
- * the quantisation kernel and the tcgen05 int8 tensor-core GEMM. */
+ * the quantisation kernel and the tcgen05 int8 tensor-core GEMM, whose
+ * results do not depend on how its work is split between CTAs (the int32
+ * partial sums are exact). */
 int bitlinear_forward(const void *x_dev, bitlinear_dtype xdt, int64_t M,
                       int64_t K, const void *packed_dev, float gamma,
                       int64_t N, void *y_dev, void *workspace_dev,
@@ -197,7 +204,8 @@ size_t bitlinear_workspace_bytes_path(int64_t M, int64_t N, int64_t K,
  * it only the input and output pointers and offers no allocator or workspace,
  * or a serving loop that forbids allocation once it has started. Nothing is
  * allocated by anyone. The scratch the path needs (x~, beta and the per-token
- * sums of x~) lives in one file-scope device array of
+ * sums of x~; the GEMM then gives every CTA whole tiles, so it needs no
+ * partial-sum region) lives in one file-scope device array of
  * BITLINEAR_STATIC_SCRATCH_BYTES (16 MiB) inside the library; every GPU that
  * loads the library holds that array until the process exits.
  * The paper has no counterpart of this call; it exists only for such callers.
