@@ -374,11 +374,11 @@ def time_graph(fn, reps: int) -> float:
 
 def bench_layer_set(bl, device, batches=(1, 8, 64), reps: int = 10):
     """The seven projections of the 2B decoder layer for 30 layers (521 MB of
-    packed weights, more than four times L2) at decode batch B, through the
-    automatic dispatch: one grouped GEMV launch per layer at B = 1, one
-    bitlinear_forward per projection (quantisation + tensor-core GEMM) at
-    B > 6. The 30 layers hold distinct device copies of one seeded layer's
-    packed weights (the parity tests use independent seeds per layer)."""
+    packed weights, more than four times L2) at decode batch B, one grouped
+    call per layer: one GEMV launch at B = 1, one quantisation launch and one
+    tensor-core GEMM launch over the seven problems at B > 6. The 30 layers
+    hold distinct device copies of one seeded layer's packed weights (the
+    parity tests use independent seeds per layer)."""
     import torch
     layer = workloads.layer_set_2b(1, layers=1).problems
     packed = []
@@ -393,20 +393,15 @@ def bench_layer_set(bl, device, batches=(1, 8, 64), reps: int = 10):
     for B in batches:
         xs = [bf16_tensor(workloads.activations_bf16(B, p.K, p.x_seed), device) for p, _, _ in packed]
         ys = [torch.empty((B, p.N), dtype=torch.bfloat16, device=device) for p, _, _ in packed]
-        ws_bytes = max(bl.bitlinear_workspace_bytes(B, p.N, p.K) for p, _, _ in packed)
+        groups = [[(xs[k], dp, g, p.N, ys[k]) for k, (p, dp, g) in enumerate(copies[li])]
+                  for li in range(layers)]
+        ws_bytes = bl.bitlinear_workspace_bytes_grouped(groups[0])
         ws = torch.empty((max(ws_bytes, 1),), dtype=torch.uint8, device=device)
-        if B <= 6:
-            def step():
-                for li in range(layers):
-                    bl.bitlinear_forward_grouped(
-                        [(xs[k], dp, g, p.N, ys[k]) for k, (p, dp, g) in enumerate(copies[li])])
-            launches = layers
-        else:
-            def step():
-                for li in range(layers):
-                    for k, (p, dp, g) in enumerate(copies[li]):
-                        bl.bitlinear_forward(xs[k], dp, g, p.N, y=ys[k], workspace=ws)
-            launches = layers * len(packed) * 2
+
+        def step():
+            for li in range(layers):
+                bl.bitlinear_forward_grouped(groups[li], workspace=ws)
+        launches = layers * (1 if ws_bytes == 0 else 2)
         step()
         torch.cuda.synchronize()
         ms = time_graph(step, reps)

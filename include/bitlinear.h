@@ -192,6 +192,34 @@ typedef struct {
 int bitlinear_forward_grouped(const bitlinear_problem *problems, int count,
                               bitlinear_dtype xdt, void *cuda_stream);
 
+/* Device workspace bytes bitlinear_forward_grouped_ws needs for these
+ * problems: 0 when every non-empty problem has M <= 6 (one GEMV launch),
+ * else the sum of each problem's x~, beta and row-sum regions plus one
+ * inter-CTA region (see bitlinear_workspace_bytes). SIZE_MAX for invalid
+ * problems. */
+size_t bitlinear_workspace_bytes_grouped(const bitlinear_problem *problems,
+                                         int count);
+
+/* Several independent BitLinear matmuls, at any batch size, in one pair of
+ * launches. When every non-empty problem has M <= 6 this is
+ * bitlinear_forward_grouped (one GEMV launch, the workspace is not used).
+ * Otherwise all of them go to the tensor-core path: one quantisation launch
+ * for every problem's tokens, then one weight-stationary GEMM launch over
+ * all problems' tiles (stream-K across the problems), so the fixed cost of
+ * the two launches is paid once for the group. Each problem's y is the same
+ * as bitlinear_forward computes for it alone.
+ *   problems, count, xdt [in] as for bitlinear_forward_grouped (no GEMV size
+ *                        limit here)
+ *   workspace_dev, workspace_bytes
+ *               [in]  scratch of at least bitlinear_workspace_bytes_grouped
+ *                     bytes, 256-byte aligned; not shared with a call that
+ *                     may run at the same time
+ * Errors as for bitlinear_forward; argument errors are reported before any
+ * launch. */
+int bitlinear_forward_grouped_ws(const bitlinear_problem *problems, int count,
+                                 bitlinear_dtype xdt, void *workspace_dev,
+                                 size_t workspace_bytes, void *cuda_stream);
+
 /* Workspace bytes for an explicit path (see bitlinear_forward_ex). */
 size_t bitlinear_workspace_bytes_path(int64_t M, int64_t N, int64_t K,
                                       int path);

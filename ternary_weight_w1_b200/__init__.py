@@ -50,6 +50,8 @@ EXPORTS = (
     "bitlinear_forward_inject_timeout",
     "bitlinear_forward_noalloc",
     "bitlinear_forward_grouped",
+    "bitlinear_workspace_bytes_grouped",
+    "bitlinear_forward_grouped_ws",
 )
 
 
@@ -99,6 +101,11 @@ def lib() -> ctypes.CDLL:
                                                 i64, p, p]
         L.bitlinear_forward_grouped.restype = ctypes.c_int
         L.bitlinear_forward_grouped.argtypes = [p, ctypes.c_int, ctypes.c_int, p]
+        L.bitlinear_workspace_bytes_grouped.restype = ctypes.c_size_t
+        L.bitlinear_workspace_bytes_grouped.argtypes = [p, ctypes.c_int]
+        L.bitlinear_forward_grouped_ws.restype = ctypes.c_int
+        L.bitlinear_forward_grouped_ws.argtypes = [p, ctypes.c_int, ctypes.c_int, p,
+                                                   ctypes.c_size_t, p]
         L.bitlinear_get_fault.restype = ctypes.c_int
         L.bitlinear_get_fault.argtypes = [p, p]
         L.bitlinear_status_string.restype = ctypes.c_char_p
@@ -262,23 +269,43 @@ def bitlinear_forward_noalloc(x, packed, gamma: float, N: int, y=None, stream=No
     return y
 
 
-def bitlinear_forward_grouped(problems, stream=None):
-    """Several independent BitLinear matmuls in one launch. ``problems`` is a
-    list of (x, packed, gamma, N, y) with device tensors (y may be None to
-    allocate it here); all x share one dtype. Returns the list of outputs."""
+def _problem_array(problems, alloc_y):
     import torch
-    if not problems:
-        return []
     arr = (_Problem * len(problems))()
     outs = []
-    xdt = _xdt(problems[0][0])
     for i, (x, packed, gamma, N, y) in enumerate(problems):
         M, K = x.shape
-        if y is None:
+        if y is None and alloc_y:
             y = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
         outs.append(y)
         arr[i] = _Problem(_ptr(x), M, K, N, _ptr(packed), float(gamma), _ptr(y))
-    _check(lib().bitlinear_forward_grouped(ctypes.addressof(arr), len(problems), xdt,
-                                           _stream(stream)),
-           "bitlinear_forward_grouped")
+    return arr, outs
+
+
+def bitlinear_workspace_bytes_grouped(problems) -> int:
+    """Workspace bytes of ``bitlinear_forward_grouped(problems, workspace=...)``
+    for a list of (x, packed, gamma, N, y) (only the shapes are read)."""
+    arr, _ = _problem_array(problems, alloc_y=False)
+    return lib().bitlinear_workspace_bytes_grouped(ctypes.addressof(arr), len(problems))
+
+
+def bitlinear_forward_grouped(problems, stream=None, workspace=None):
+    """Several independent BitLinear matmuls in one launch (pair). ``problems``
+    is a list of (x, packed, gamma, N, y) with device tensors (y may be None to
+    allocate it here); all x share one dtype. Without ``workspace`` every
+    problem must fit the GEMV (one launch); with it any batch size is accepted
+    (``bitlinear_forward_grouped_ws``). Returns the list of outputs."""
+    if not problems:
+        return []
+    xdt = _xdt(problems[0][0])
+    arr, outs = _problem_array(problems, alloc_y=True)
+    if workspace is None:
+        _check(lib().bitlinear_forward_grouped(ctypes.addressof(arr), len(problems), xdt,
+                                               _stream(stream)),
+               "bitlinear_forward_grouped")
+    else:
+        _check(lib().bitlinear_forward_grouped_ws(ctypes.addressof(arr), len(problems), xdt,
+                                                  _ptr(workspace), workspace.numel(),
+                                                  _stream(stream)),
+               "bitlinear_forward_grouped_ws")
     return outs

@@ -365,14 +365,6 @@ int launch_gemv(const GemvJob *jobs, int count, bitlinear_dtype xdt, const Devic
 
 // ------------------------------------------------------------ tensor cores
 
-struct TcWorkspace {
-    int8_t *xq;
-    float *beta;
-    int *rowsum;
-    int *flags;         // [MAX_GRID][4] (split only)
-    int32_t *partial;   // [MAX_GRID][BW][BT] (split only)
-};
-
 // Token tile of the weight-stationary GEMM: the candidate that pads M the
 // least (ties go to the larger tile).
 int choose_bt(int64_t M)
@@ -388,7 +380,7 @@ int choose_bt(int64_t M)
     return pad192 <= pad128 ? 192 : 128;
 }
 
-// x~, beta and the row sums of x~.
+// x~, beta and the row sums of x~ of one problem.
 size_t tc_base_bytes(int64_t M, int64_t K)
 {
     return round_up(static_cast<size_t>(M) * static_cast<size_t>(K), 256) +
@@ -396,27 +388,33 @@ size_t tc_base_bytes(int64_t M, int64_t K)
 }
 
 // Flags and partial-sum slots for tiles split between CTAs.
-size_t tc_split_bytes(int64_t M)
+size_t tc_split_bytes(int64_t max_M)
 {
     return round_up(static_cast<size_t>(wsg::MAX_GRID) * 4 * 4, 256) +
-           static_cast<size_t>(wsg::MAX_GRID) * wsg::BW * static_cast<size_t>(choose_bt(M)) * 4;
+           static_cast<size_t>(wsg::MAX_GRID) * wsg::BW * static_cast<size_t>(choose_bt(max_M)) * 4;
 }
 
 size_t tc_workspace_bytes(int64_t M, int64_t K) { return tc_base_bytes(M, K) + tc_split_bytes(M); }
 
-TcWorkspace tc_workspace(void *ws, int64_t M, int64_t K, bool split)
+// One problem of a tensor-core launch, as the host sees it.
+struct TcJob {
+    const void *x;
+    int M, K, N;
+    const void *packed;
+    float gamma;
+    void *y;
+    int32_t *acc;
+};
+
+size_t tc_group_bytes(const TcJob *jobs, int n, bool split)
 {
-    char *b = static_cast<char *>(ws);
-    const size_t a = round_up(static_cast<size_t>(M) * static_cast<size_t>(K), 256);
-    const size_t c = round_up(static_cast<size_t>(M) * 4, 256);
-    const size_t f = round_up(static_cast<size_t>(wsg::MAX_GRID) * 4 * 4, 256);
-    TcWorkspace w{reinterpret_cast<int8_t *>(b), reinterpret_cast<float *>(b + a),
-                  reinterpret_cast<int *>(b + a + c), nullptr, nullptr};
-    if (split) {
-        w.flags = reinterpret_cast<int *>(b + a + 2 * c);
-        w.partial = reinterpret_cast<int32_t *>(b + a + 2 * c + f);
+    size_t b = 0;
+    int max_M = 0;
+    for (int i = 0; i < n; ++i) {
+        b += tc_base_bytes(jobs[i].M, jobs[i].K);
+        max_M = std::max(max_M, jobs[i].M);
     }
-    return w;
+    return b + (split ? tc_split_bytes(max_M) : 0);
 }
 
 template <bool B_PACKED, bool RESCALE>
@@ -434,94 +432,162 @@ int launch_gemm(const CUtensorMap &ma, const CUtensorMap &mb, const tc::Params &
 }
 
 template <int BT>
-int launch_gemm_ws(const CUtensorMap &mx, const CUtensorMap &mw, const wsg::Params &p, int grid,
-                   const DeviceInfo &dev, cudaStream_t st)
+int launch_gemm_ws(const wsg::Maps &maps, const wsg::Params &p, int grid, const DeviceInfo &dev,
+                   cudaStream_t st)
 {
     constexpr int smem = wsg::Cfg<BT>::SMEM_BYTES;
     cudaError_t e = allow_smem<wsg::gemm_ws_kernel<BT>>(dev.id, smem);
     if (e != cudaSuccess)
         return launch_status(e);
     e = launch(wsg::gemm_ws_kernel<BT>, dim3(grid), dim3(wsg::THREADS), static_cast<size_t>(smem),
-               st, mx, mw, p);
+               st, maps, p);
     return launch_status(e);
 }
 
-// Quantise x, then run the weight-stationary GEMM with its fused rescale.
-// With `split` the k-blocks of all tiles are shared evenly between the CTAs
-// (stream-K; needs the flag and partial-sum regions of the workspace);
-// without it every CTA takes whole tiles.
-int run_tc_path(const void *x, bitlinear_dtype xdt, int M, int K, const void *packed,
-                float gamma, int N, void *y, void *ws, size_t ws_bytes, int32_t *acc,
-                int8_t *xq_dbg, float *beta_dbg, const DeviceInfo &dev, cudaStream_t st,
-                int inject_timeout_us, bool split)
+// Quantisation of several problems' rows in one launch (one warp per row).
+int launch_quant_group(const TcJob *jobs, int n, bitlinear_dtype xdt, int8_t *const *xq,
+                       float *const *beta, int *const *rowsum, cudaStream_t st, int *clear,
+                       int n_clear)
 {
-    const size_t need = split ? tc_workspace_bytes(M, K) : tc_base_bytes(M, K);
+    qa::GroupParams g{};
+    int blocks = 0;
+    for (int i = 0; i < n; ++i) {
+        g.prob[i] = qa::GroupRows{jobs[i].x, xq[i], beta[i], rowsum[i], jobs[i].M, jobs[i].K,
+                                  blocks};
+        blocks += (jobs[i].M + qa::WARPS - 1) / qa::WARPS;
+    }
+    g.count = n;
+    g.clear = clear;
+    g.n_clear = n_clear;
+    cudaError_t e;
+    if (xdt == BITLINEAR_BF16)
+        e = launch(qa::quant_act_grouped_kernel<true, 16>, dim3(blocks), dim3(qa::THREADS), 0, st, g);
+    else
+        e = launch(qa::quant_act_grouped_kernel<false, 8>, dim3(blocks), dim3(qa::THREADS), 0, st, g);
+    return launch_status(e);
+}
+
+// Quantise x, then run the weight-stationary GEMM with its fused rescale, for
+// one or several independent problems (at most wsg::MAX_PROBLEMS) in one pair
+// of launches. The workspace holds each problem's x~, beta and row sums, then
+// (with `split`) the flag and partial-sum regions. With `split` the k-blocks
+// of all tiles are shared evenly between the CTAs (stream-K) when that pays;
+// otherwise every CTA takes whole tiles.
+int run_tc_group(const TcJob *jobs, int n, bitlinear_dtype xdt, void *ws, size_t ws_bytes,
+                 int8_t *xq_dbg, float *beta_dbg, const DeviceInfo &dev, cudaStream_t st,
+                 int inject_timeout_us, bool split)
+{
+    const size_t need = tc_group_bytes(jobs, n, split);
     if (ws == nullptr || ws_bytes < need)
         return BITLINEAR_ERR_WORKSPACE;
     if (!aligned(ws, 256))
         return BITLINEAR_ERR_ALIGN;
-    const int BT = choose_bt(M);
-    const int KB = (K + wsg::BK - 1) / wsg::BK;
-    const int MT = (M + BT - 1) / BT;
-    const int T = MT * ((N + wsg::BW - 1) / wsg::BW);
+    int max_M = 0;
+    for (int i = 0; i < n; ++i)
+        max_M = std::max(max_M, jobs[i].M);
+    const int BT = choose_bt(max_M);
+
+    wsg::Params p{};
+    int64_t tiles = 0, iters = 0;
+    for (int i = 0; i < n; ++i) {
+        wsg::Problem &P = p.prob[i];
+        P.M = jobs[i].M;
+        P.N = jobs[i].N;
+        P.MT = (jobs[i].M + BT - 1) / BT;
+        P.KB = (jobs[i].K + wsg::BK - 1) / wsg::BK;
+        P.iter_begin = static_cast<int>(iters);
+        P.tile_begin = static_cast<int>(tiles);
+        P.gamma = jobs[i].gamma;
+        P.y = static_cast<uint16_t *>(jobs[i].y);
+        P.acc_out = jobs[i].acc;
+        const int64_t T = static_cast<int64_t>(P.MT) * ((jobs[i].N + wsg::BW - 1) / wsg::BW);
+        tiles += T;
+        iters += T * P.KB;
+    }
+    if (iters >= (int64_t(1) << 31))
+        return BITLINEAR_ERR_SHAPE;
     const int slots = std::min(dev.sms, wsg::MAX_GRID);
     // Splitting a tile's k-range between CTAs costs a hand-off of a few
     // microseconds (partial store, flag, partial load). With at least as many
     // tiles as CTAs it evens out the last wave; with fewer tiles it pays only
     // when the k-blocks a CTA saves outweigh that hand-off.
-    if (split && T < slots) {
-        const double saved_blocks = KB * (1.0 - static_cast<double>(T) / slots);
+    if (split && tiles < slots) {
+        const double kb_per_tile = static_cast<double>(iters) / static_cast<double>(tiles);
+        const double saved_blocks = kb_per_tile * (1.0 - static_cast<double>(tiles) / slots);
         split = saved_blocks > kSplitMinSavedBlocks;
     }
-    const int unit = split ? 1 : KB;
-    const int64_t units = static_cast<int64_t>(T) * KB / unit;
+    const int64_t units = split ? iters : tiles;
     const int grid = static_cast<int>(std::min<int64_t>(units, slots));
-    TcWorkspace w = tc_workspace(ws, M, K, split);
-    int rc = launch_quant_act(x, xdt, M, K, w.xq, w.beta, w.rowsum, st, w.flags,
-                              split ? 4 * grid : 0);
+
+    // Workspace: per problem x~ | beta | row sums, then flags | partial sums.
+    char *w = static_cast<char *>(ws);
+    int8_t *xq[wsg::MAX_PROBLEMS];
+    float *beta[wsg::MAX_PROBLEMS];
+    int *rowsum[wsg::MAX_PROBLEMS];
+    for (int i = 0; i < n; ++i) {
+        const size_t a = round_up(static_cast<size_t>(jobs[i].M) * jobs[i].K, 256);
+        const size_t c = round_up(static_cast<size_t>(jobs[i].M) * 4, 256);
+        xq[i] = reinterpret_cast<int8_t *>(w);
+        beta[i] = reinterpret_cast<float *>(w + a);
+        rowsum[i] = reinterpret_cast<int *>(w + a + c);
+        p.prob[i].beta = beta[i];
+        p.prob[i].rowsum = rowsum[i];
+        w += a + 2 * c;
+    }
+    int *flags = nullptr;
+    if (split) {
+        flags = reinterpret_cast<int *>(w);
+        p.partial = reinterpret_cast<int32_t *>(
+            w + round_up(static_cast<size_t>(wsg::MAX_GRID) * 4 * 4, 256));
+        p.flags = flags;
+    }
+    int rc = (n == 1) ? launch_quant_act(jobs[0].x, xdt, jobs[0].M, jobs[0].K, xq[0], beta[0],
+                                         rowsum[0], st, flags, split ? 4 * grid : 0)
+                      : launch_quant_group(jobs, n, xdt, xq, beta, rowsum, st, flags,
+                                           split ? 4 * grid : 0);
     if (rc != BITLINEAR_OK)
         return rc;
-    CUtensorMap mx, mw;
-    if (!make_map_xq_k256(&mx, w.xq, M, K, static_cast<uint32_t>(BT)) ||
-        !make_map_packed_k256(&mw, packed, N, K, wsg::BW))
-        return BITLINEAR_ERR_CUDA;
-    wsg::Params p{};
-    p.M = M;
-    p.N = N;
-    p.K = K;
-    p.gamma = gamma;
-    p.beta = w.beta;
-    p.rowsum = w.rowsum;
-    p.y = static_cast<uint16_t *>(y);
-    p.acc_out = acc;
-    p.partial = w.partial;
-    p.flags = w.flags;
-    p.MT = MT;
-    p.T = T;
-    p.KB = KB;
-    p.unit = unit;
+    wsg::Maps maps{};
+    for (int i = 0; i < n; ++i)
+        if (!make_map_xq_k256(&maps.x[i], xq[i], jobs[i].M, jobs[i].K, static_cast<uint32_t>(BT)) ||
+            !make_map_packed_k256(&maps.w[i], jobs[i].packed, jobs[i].N, jobs[i].K, wsg::BW))
+            return BITLINEAR_ERR_CUDA;
+    p.count = n;
+    p.total_iters = static_cast<int>(iters);
+    p.total_tiles = static_cast<int>(tiles);
+    p.split = split ? 1 : 0;
     p.base = static_cast<int>(units / grid);
     p.extra = static_cast<int>(units % grid);
     p.wait_limit_ns =
         inject_timeout_us > 0 ? static_cast<uint64_t>(inject_timeout_us) * 1000ull : kWaitLimitNs;
     p.inject_timeout = inject_timeout_us > 0 ? 1 : 0;
     switch (BT) {
-    case 32: rc = launch_gemm_ws<32>(mx, mw, p, grid, dev, st); break;
-    case 64: rc = launch_gemm_ws<64>(mx, mw, p, grid, dev, st); break;
-    case 128: rc = launch_gemm_ws<128>(mx, mw, p, grid, dev, st); break;
-    default: rc = launch_gemm_ws<192>(mx, mw, p, grid, dev, st); break;
+    case 32: rc = launch_gemm_ws<32>(maps, p, grid, dev, st); break;
+    case 64: rc = launch_gemm_ws<64>(maps, p, grid, dev, st); break;
+    case 128: rc = launch_gemm_ws<128>(maps, p, grid, dev, st); break;
+    default: rc = launch_gemm_ws<192>(maps, p, grid, dev, st); break;
     }
     if (rc != BITLINEAR_OK)
         return rc;
-    if (xq_dbg != nullptr &&
-        cudaMemcpyAsync(xq_dbg, w.xq, static_cast<size_t>(M) * K, cudaMemcpyDeviceToDevice, st) !=
-            cudaSuccess)
+    if (n == 1 && xq_dbg != nullptr &&
+        cudaMemcpyAsync(xq_dbg, xq[0], static_cast<size_t>(jobs[0].M) * jobs[0].K,
+                        cudaMemcpyDeviceToDevice, st) != cudaSuccess)
         return BITLINEAR_ERR_CUDA;
-    if (beta_dbg != nullptr &&
-        cudaMemcpyAsync(beta_dbg, w.beta, static_cast<size_t>(M) * 4, cudaMemcpyDeviceToDevice,
-                        st) != cudaSuccess)
+    if (n == 1 && beta_dbg != nullptr &&
+        cudaMemcpyAsync(beta_dbg, beta[0], static_cast<size_t>(jobs[0].M) * 4,
+                        cudaMemcpyDeviceToDevice, st) != cudaSuccess)
         return BITLINEAR_ERR_CUDA;
     return BITLINEAR_OK;
+}
+
+int run_tc_path(const void *x, bitlinear_dtype xdt, int M, int K, const void *packed,
+                float gamma, int N, void *y, void *ws, size_t ws_bytes, int32_t *acc,
+                int8_t *xq_dbg, float *beta_dbg, const DeviceInfo &dev, cudaStream_t st,
+                int inject_timeout_us, bool split)
+{
+    const TcJob job{x, M, K, N, packed, gamma, y, acc};
+    return run_tc_group(&job, 1, xdt, ws, ws_bytes, xq_dbg, beta_dbg, dev, st, inject_timeout_us,
+                        split);
 }
 
 // --------------------------------------------------------------- checks
@@ -686,6 +752,81 @@ extern "C" int bitlinear_forward_grouped(const bitlinear_problem *problems, int 
     if (rc != BITLINEAR_OK)
         return rc;
     return launch_gemv(jobs, n, xdt, *dev, static_cast<cudaStream_t>(cuda_stream));
+}
+
+namespace {
+
+// Checks a problem list for the grouped calls and collects the non-empty
+// problems. Sets *all_gemv when every one of them fits the GEMV path at the
+// automatic threshold.
+int collect_group(const bitlinear_problem *problems, int count, int xdt, TcJob *jobs, int *n,
+                  bool *all_gemv, bool shapes_only = false)
+{
+    if (problems == nullptr || count < 1 || count > wsg::MAX_PROBLEMS)
+        return BITLINEAR_ERR_ARG;
+    *n = 0;
+    *all_gemv = true;
+    static const uint4 dummy = {};   // stands in for the pointers when sizing
+    for (int i = 0; i < count; ++i) {
+        const bitlinear_problem &pr = problems[i];
+        int rc = shapes_only
+                     ? check_forward_args(&dummy, xdt, pr.M, pr.K, &dummy, pr.N, &dummy, nullptr,
+                                          nullptr, nullptr)
+                     : check_forward_args(pr.x_dev, xdt, pr.M, pr.K, pr.packed_dev, pr.N,
+                                          pr.y_dev, nullptr, nullptr, nullptr);
+        if (rc != BITLINEAR_OK)
+            return rc;
+        if (pr.M == 0)
+            continue;
+        if (!(pr.M <= kAutoGemvMaxM && gemv_fits(pr.M, pr.K)))
+            *all_gemv = false;
+        jobs[(*n)++] = TcJob{pr.x_dev,      static_cast<int>(pr.M), static_cast<int>(pr.K),
+                             static_cast<int>(pr.N), pr.packed_dev, pr.gamma, pr.y_dev, nullptr};
+    }
+    return BITLINEAR_OK;
+}
+
+}  // namespace
+
+extern "C" size_t bitlinear_workspace_bytes_grouped(const bitlinear_problem *problems, int count)
+{
+    TcJob jobs[wsg::MAX_PROBLEMS];
+    int n = 0;
+    bool all_gemv = true;
+    // The dtype does not change the size; BF16 only passes the argument check.
+    if (collect_group(problems, count, BITLINEAR_BF16, jobs, &n, &all_gemv, true) != BITLINEAR_OK)
+        return SIZE_MAX;
+    if (n == 0 || all_gemv)
+        return 0;
+    return tc_group_bytes(jobs, n, true);
+}
+
+extern "C" int bitlinear_forward_grouped_ws(const bitlinear_problem *problems, int count,
+                                            bitlinear_dtype xdt, void *workspace_dev,
+                                            size_t workspace_bytes, void *cuda_stream)
+{
+    TcJob jobs[wsg::MAX_PROBLEMS];
+    int n = 0;
+    bool all_gemv = true;
+    int rc = collect_group(problems, count, xdt, jobs, &n, &all_gemv);
+    if (rc != BITLINEAR_OK)
+        return rc;
+    if (n == 0)
+        return BITLINEAR_OK;
+    DeviceInfo *dev = nullptr;
+    rc = current_device(&dev);
+    if (rc != BITLINEAR_OK)
+        return rc;
+    cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
+    if (all_gemv) {
+        GemvJob g[wsg::MAX_PROBLEMS];
+        for (int i = 0; i < n; ++i)
+            g[i] = GemvJob{jobs[i].x, jobs[i].M, jobs[i].K, jobs[i].N, jobs[i].packed,
+                           jobs[i].gamma, jobs[i].y, nullptr, nullptr, nullptr};
+        return launch_gemv(g, n, xdt, *dev, st);
+    }
+    return run_tc_group(jobs, n, xdt, workspace_dev, workspace_bytes, nullptr, nullptr, *dev, st,
+                        0, true);
 }
 
 extern "C" int bitlinear_forward_inject_timeout(const void *x_dev, bitlinear_dtype xdt, int64_t M,

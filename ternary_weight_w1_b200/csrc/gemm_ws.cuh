@@ -90,42 +90,80 @@ struct Cfg {
     static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
 };
 
-struct Params {
-    int M, N, K;
+constexpr int MAX_PROBLEMS = 8;
+
+// One matmul of a launch. A launch runs one or several independent problems
+// (sharing the token tile BT); their tiles and k-blocks are numbered one
+// after the other.
+struct Problem {
+    int M, N;               // tokens, weight rows
+    int MT, KB;             // token tiles; k-blocks (256 k) per tile: ceil(K / 256)
+    int iter_begin;         // global index of the problem's first k-block
+    int tile_begin;         // global index of the problem's first tile
     float gamma;
     const float *beta;      // [M]
     const int *rowsum;      // [M] sum_k x~
     uint16_t *y;            // [M][N] bf16
     int32_t *acc_out;       // [M][N] int32 or null
-    int32_t *partial;       // [grid][BW][BT] int32 (null when unit == KB)
-    int *flags;             // [grid][4] zero at launch (null when unit == KB)
-    int MT;                 // token tiles
-    int T;                  // tiles = MT * ceil(N / BW)
-    int KB;                 // k-blocks (256 k) per tile: ceil(K / 256)
-    int unit;               // k-blocks per partition unit: 1 (stream-K) or KB
+};
+
+// TMA descriptors of every problem's x~ and packed weights.
+struct Maps {
+    CUtensorMap x[MAX_PROBLEMS];
+    CUtensorMap w[MAX_PROBLEMS];
+};
+
+struct Params {
+    Problem prob[MAX_PROBLEMS];
+    int count;
+    int total_iters, total_tiles;
+    int32_t *partial;       // [grid][BW][BT] int32 (split only)
+    int *flags;             // [grid][4] zero at launch (split only)
+    int split;              // 1: CTA ranges in k-blocks (stream-K); 0: in whole tiles
     int base, extra;        // units per CTA: base, plus one for the first `extra`
     uint64_t wait_limit_ns;
     int inject_timeout;     // MMA issuer waits on a barrier nobody arrives at
 };
 
-// First k-block (global iteration index) of CTA c's range.
-__device__ __forceinline__ int range_begin(const Params &p, int c)
+// The problem holding global k-block `it` / global tile `tile`.
+__device__ __forceinline__ int problem_of_iter(const Params &p, int it)
 {
-    return (c * p.base + min(c, p.extra)) * p.unit;
+    int q = 0;
+    while (q + 1 < p.count && it >= p.prob[q + 1].iter_begin)
+        ++q;
+    return q;
 }
 
-// The CTA whose range holds global iteration `it`.
+__device__ __forceinline__ int problem_of_tile(const Params &p, int tile)
+{
+    int q = 0;
+    while (q + 1 < p.count && tile >= p.prob[q + 1].tile_begin)
+        ++q;
+    return q;
+}
+
+// First global k-block of CTA c's range.
+__device__ __forceinline__ int range_begin(const Params &p, int c)
+{
+    const int u = c * p.base + min(c, p.extra);
+    if (p.split)
+        return u;
+    if (u >= p.total_tiles)
+        return p.total_iters;
+    const int q = problem_of_tile(p, u);
+    return p.prob[q].iter_begin + (u - p.prob[q].tile_begin) * p.prob[q].KB;
+}
+
+// The CTA whose range holds global k-block `it` (stream-K ranges only).
 __device__ __forceinline__ int range_owner(const Params &p, int it)
 {
-    const int u = it / p.unit;
     const int big = p.extra * (p.base + 1);
-    return u < big ? u / (p.base + 1) : p.extra + (u - big) / p.base;
+    return it < big ? it / (p.base + 1) : p.extra + (it - big) / p.base;
 }
 
 template <int BT>
 __global__ void __launch_bounds__(THREADS, 1)
-gemm_ws_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
-               const Params p)
+gemm_ws_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Params p)
 {
     using C = Cfg<BT>;
     constexpr int NS = C::NS;
@@ -172,10 +210,10 @@ gemm_ws_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
         *abort_flag = 0;
         fence_barrier_init();
     }
-    if (warp == 0 && lane == 0)
-        prefetch_tensormap(&tmap_x);
-    if (warp == PK_WARP && lane == 0)
-        prefetch_tensormap(&tmap_w);
+    if (warp == 0 && lane < p.count)
+        prefetch_tensormap(&maps.x[lane]);
+    if (warp == PK_WARP && lane < p.count)
+        prefetch_tensormap(&maps.w[lane]);
     if (warp == 1)
         tmem_alloc(smem_u32(tmem_slot), TMEM_COLS);
     tc_fence_before_sync();
@@ -191,7 +229,6 @@ gemm_ws_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
 
     const int it_begin = range_begin(p, blockIdx.x);
     const int it_end = range_begin(p, blockIdx.x + 1);
-    const int KB = p.KB;
 
     if (warp == 0 || warp == PK_WARP) {
         // ----------------------------------------------------- TMA producers
@@ -203,20 +240,26 @@ gemm_ws_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
             uint32_t ph = 0;
             int armed[NS];
             for (int i = 0; i < NS; ++i) armed[i] = -1;
+            int q = problem_of_iter(p, it_begin);
             for (int it = it_begin; it < it_end; ++it) {
-                const int t = it / KB;
-                const int kb = it - t * KB;
+                while (q + 1 < p.count && it >= p.prob[q + 1].iter_begin)
+                    ++q;
+                const Problem &P = p.prob[q];
+                const int local = it - P.iter_begin;
+                const int t = local / P.KB;
+                const int kb = local - t * P.KB;
                 if (!mbar_wait_bounded(empty_load(s), ph ^ 1u, abort_flag, limit))
                     break;
                 armed[s] = static_cast<int>(ph);
                 if (is_x) {
-                    const int mt = t % p.MT;
+                    const int mt = t % P.MT;
                     mbar_arrive_expect_tx(full_load(s), C::X_BYTES);
-                    tma_load_3d(sX + s * C::X_BYTES, &tmap_x, 0, mt * BT, 2 * kb, full_load(s));
+                    tma_load_3d(sX + s * C::X_BYTES, &maps.x[q], 0, mt * BT, 2 * kb, full_load(s));
                 } else {
-                    const int nt = t / p.MT;
+                    const int nt = t / P.MT;
                     mbar_arrive_expect_tx(full_load(s), PK_BYTES);
-                    tma_load_3d(sP + s * PK_BYTES, &tmap_w, 0, 2 * kb, nt * (BW / 16), full_load(s));
+                    tma_load_3d(sP + s * PK_BYTES, &maps.w[q], 0, 2 * kb, nt * (BW / 16),
+                                full_load(s));
                 }
                 if (++s == NS) { s = 0; ph ^= 1u; }
             }
@@ -237,9 +280,11 @@ gemm_ws_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
                 goto mma_done;
             }
             for (int it = it_begin; it < it_end; ++seg) {
-                const int t = it / KB;
-                const int k0 = it - t * KB;
-                const int k1 = min(KB, k0 + (it_end - it));
+                const Problem &P = p.prob[problem_of_iter(p, it)];
+                const int local = it - P.iter_begin;
+                const int t = local / P.KB;
+                const int k0 = local - t * P.KB;
+                const int k1 = min(P.KB, k0 + (it_end - it));
                 const int buf = seg & 1;
                 if (!mbar_wait_bounded(acc_empty(buf), ((static_cast<uint32_t>(seg) >> 1) & 1u) ^ 1u,
                                        abort_flag, limit))
@@ -332,13 +377,15 @@ gemm_ws_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
         int seg = 0;
         int epi_chunk = 0;                 // alternates the two transpose buffers
         for (int it = it_begin; it < it_end; ++seg) {
-            const int t = it / KB;
-            const int k0 = it - t * KB;
-            const int k1 = min(KB, k0 + (it_end - it));
+            const Problem &P = p.prob[problem_of_iter(p, it)];
+            const int local = it - P.iter_begin;
+            const int t = local / P.KB;
+            const int k0 = local - t * P.KB;
+            const int k1 = min(P.KB, k0 + (it_end - it));
             it += k1 - k0;
             const int buf = seg & 1;
-            const int mt = t % p.MT;
-            const int nt = t / p.MT;
+            const int mt = t % P.MT;
+            const int nt = t / P.MT;
 
             // Per-token scale and row sum of this tile, fetched before the
             // accumulator is ready: lane l holds token mt * BT + 32 c + l.
@@ -348,8 +395,8 @@ gemm_ws_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
 #pragma unroll
                 for (int c = 0; c < BT / 32; ++c) {
                     const int ml = mt * BT + 32 * c + lane;
-                    s_pf[c] = ml < p.M ? out_scale(__ldg(p.beta + ml), p.gamma) : 0.0f;
-                    rs_pf[c] = ml < p.M ? __ldg(p.rowsum + ml) : 0;
+                    s_pf[c] = ml < P.M ? out_scale(__ldg(P.beta + ml), P.gamma) : 0.0f;
+                    rs_pf[c] = ml < P.M ? __ldg(P.rowsum + ml) : 0;
                 }
             }
 
@@ -391,8 +438,8 @@ gemm_ws_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
 
             // First k-block of the tile is here: this CTA finishes the tile.
             // Other contributors: the CTAs holding the tile's later k-blocks.
-            const int c_last =
-                (k1 < KB) ? range_owner(p, t * KB + KB - 1) : static_cast<int>(blockIdx.x);
+            const int c_last = (k1 < P.KB) ? range_owner(p, P.iter_begin + (t + 1) * P.KB - 1)
+                                           : static_cast<int>(blockIdx.x);
             // Every lane polls some of the contributors' flags (lane l takes
             // contributors blockIdx.x + 1 + l, + 33, ...), so all of them are
             // read in one round trip when they are already set.
@@ -431,12 +478,12 @@ gemm_ws_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
                 break;
 
             const int n = nt * BW + row;
-            const bool n_ok = n < p.N;
-            const bool vec_out = (p.N % 8) == 0;
+            const bool n_ok = n < P.N;
+            const bool vec_out = (P.N % 8) == 0;
 #pragma unroll
             for (int c = 0; c < BT / 32; ++c) {
                 const int m0 = mt * BT + 32 * c;
-                if (m0 >= p.M)
+                if (m0 >= P.M)
                     break;
                 uint32_t r[32];
                 tmem_ld_32x32b_x32(d_cols + static_cast<uint32_t>(32 * c), r);
@@ -463,13 +510,13 @@ gemm_ws_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
                         r[4 * g + 3] += static_cast<uint32_t>(va[g].w + vb[g].w);
                     }
                 }
-                const int jn = min(32, p.M - m0);
-                if (p.acc_out != nullptr) {
+                const int jn = min(32, P.M - m0);
+                if (P.acc_out != nullptr) {
 #pragma unroll
                     for (int j = 0; j < 32; ++j) {
                         const int rs = __shfl_sync(0xffffffffu, rs_pf[c], j);
                         if (j < jn && n_ok)
-                            p.acc_out[static_cast<size_t>(m0 + j) * p.N + n] =
+                            P.acc_out[static_cast<size_t>(m0 + j) * P.N + n] =
                                 static_cast<int>(r[j]) - rs;
                     }
                 }
@@ -492,20 +539,20 @@ gemm_ws_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
                         const int j = sg >> 4;
                         const int piece = sg & 15;
                         const int nn = nt * BW + 8 * piece;
-                        if (j < jn && nn < p.N) {
+                        if (j < jn && nn < P.N) {
                             const uint4 v = *reinterpret_cast<const uint4 *>(blk + j * BW + 8 * piece);
-                            *reinterpret_cast<uint4 *>(p.y + static_cast<size_t>(m0 + j) * p.N + nn) = v;
+                            *reinterpret_cast<uint4 *>(P.y + static_cast<size_t>(m0 + j) * P.N + nn) = v;
                         }
                     }
                     ++epi_chunk;
                 } else {
-                    uint16_t *yrow = p.y + static_cast<size_t>(m0) * p.N + n;
+                    uint16_t *yrow = P.y + static_cast<size_t>(m0) * P.N + n;
 #pragma unroll
                     for (int j = 0; j < 32; ++j) {
                         const float s = __shfl_sync(0xffffffffu, s_pf[c], j);
                         const int rs = __shfl_sync(0xffffffffu, rs_pf[c], j);
                         if (j < jn && n_ok)
-                            yrow[static_cast<size_t>(j) * p.N] =
+                            yrow[static_cast<size_t>(j) * P.N] =
                                 rescale_bf16(static_cast<int>(r[j]) - rs, s);
                     }
                 }

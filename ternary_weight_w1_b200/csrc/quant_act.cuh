@@ -7,7 +7,8 @@
 // for long rows), 256 threads per block. Each lane keeps CACHE vectors of 8
 // activations in registers from the absmax pass, so a row is read from
 // memory once when 32 * WPR * 8 * CACHE covers it; anything beyond is
-// re-read in the second pass, four vectors in flight per lane. The row sum
+// re-read in the second pass, four vectors in flight per lane. A grouped
+// variant quantises the rows of several problems in one launch. The row sum
 // of x~ is written for the tensor-core path, whose GEMM contracts the
 // non-negative weight codes W~ + 1 (acc = sum x~ * code - sum x~). Block 0
 // also clears the GEMM's inter-block flag words when asked to.
@@ -24,11 +25,12 @@ constexpr int WARPS = THREADS / 32;
 template <int WPR>
 __host__ __device__ constexpr int rows_per_block() { return WARPS / WPR; }
 
+// Quantises token row m of one problem (warp `part` of the WPR warps that
+// share the row); rows past M take part in the block barriers only.
 template <bool BF16, int CACHE, int WPR>
-__global__ void __launch_bounds__(THREADS)
-quant_act_kernel(const void *__restrict__ x, int M, int K, int8_t *__restrict__ xq,
-                 float *__restrict__ beta_out, int *__restrict__ rowsum_out,
-                 int *__restrict__ clear, int n_clear)
+__device__ __forceinline__ void quant_row(const void *__restrict__ x, int M, int K,
+                                          int8_t *__restrict__ xq, float *__restrict__ beta_out,
+                                          int *__restrict__ rowsum_out, int m, int part)
 {
     static_assert(WARPS % WPR == 0, "warps per row");
     constexpr int STRIDE = 32 * WPR;              // vectors between a lane's vectors
@@ -36,15 +38,6 @@ quant_act_kernel(const void *__restrict__ x, int M, int K, int8_t *__restrict__ 
     __shared__ int red_sum[WARPS];
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int part = warp % WPR;
-    const int m = blockIdx.x * rows_per_block<WPR>() + warp / WPR;
-    pdl_wait();
-    // The GEMM that follows uses these words as inter-block flags; they are
-    // cleared here, after every earlier grid in the stream has finished.
-    if (clear != nullptr && blockIdx.x == 0)
-        for (int i = threadIdx.x; i < n_clear; i += THREADS)
-            clear[i] = 0;
-    // Rows past M still take part in the block barriers (WPR > 1).
     const bool active = m < M;
     if (WPR == 1 && !active)
         return;
@@ -141,6 +134,60 @@ quant_act_kernel(const void *__restrict__ x, int M, int K, int8_t *__restrict__ 
         if (rowsum_out != nullptr)
             rowsum_out[m] = sum;
     }
+}
+
+template <bool BF16, int CACHE, int WPR>
+__global__ void __launch_bounds__(THREADS)
+quant_act_kernel(const void *__restrict__ x, int M, int K, int8_t *__restrict__ xq,
+                 float *__restrict__ beta_out, int *__restrict__ rowsum_out,
+                 int *__restrict__ clear, int n_clear)
+{
+    const int warp = threadIdx.x >> 5;
+    const int m = blockIdx.x * rows_per_block<WPR>() + warp / WPR;
+    pdl_wait();
+    // The GEMM that follows uses these words as inter-block flags; they are
+    // cleared here, after every earlier grid in the stream has finished.
+    if (clear != nullptr && blockIdx.x == 0)
+        for (int i = threadIdx.x; i < n_clear; i += THREADS)
+            clear[i] = 0;
+    quant_row<BF16, CACHE, WPR>(x, M, K, xq, beta_out, rowsum_out, m, warp % WPR);
+}
+
+// Several problems' token rows in one launch (one warp per row): block b
+// belongs to the problem whose block range [first_block, next first_block)
+// holds it.
+constexpr int MAX_PROBLEMS = 8;
+
+struct GroupRows {
+    const void *x;
+    int8_t *xq;
+    float *beta;
+    int *rowsum;
+    int M, K;
+    int first_block;
+};
+
+struct GroupParams {
+    GroupRows prob[MAX_PROBLEMS];
+    int count;
+    int *clear;
+    int n_clear;
+};
+
+template <bool BF16, int CACHE>
+__global__ void __launch_bounds__(THREADS)
+quant_act_grouped_kernel(const __grid_constant__ GroupParams g)
+{
+    int q = 0;
+    while (q + 1 < g.count && static_cast<int>(blockIdx.x) >= g.prob[q + 1].first_block)
+        ++q;
+    const GroupRows &r = g.prob[q];
+    const int m = (static_cast<int>(blockIdx.x) - r.first_block) * WARPS + (threadIdx.x >> 5);
+    pdl_wait();
+    if (g.clear != nullptr && blockIdx.x == 0)
+        for (int i = threadIdx.x; i < g.n_clear; i += THREADS)
+            g.clear[i] = 0;
+    quant_row<BF16, CACHE, 1>(r.x, r.M, r.K, r.xq, r.beta, r.rowsum, m, 0);
 }
 
 }  // namespace qa

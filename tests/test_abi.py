@@ -139,3 +139,42 @@ def test_grouped_rejects_bad_arguments():
     assert grouped([good, (FAKE + 8, 1, 256, 64, FAKE, FAKE)]) == bl.BITLINEAR_ERR_ALIGN
     assert grouped([good], xdt=5) == bl.BITLINEAR_ERR_DTYPE
     assert grouped([(None, 0, 256, 64, None, None)]) == bl.BITLINEAR_OK   # only empty problems
+
+
+def grouped_ws(problems, xdt=0, ws=FAKE, ws_bytes=1 << 30):
+    arr = (bl._Problem * max(1, len(problems)))()
+    for i, (x, M, K, N, packed, y) in enumerate(problems):
+        arr[i] = bl._Problem(x, M, K, N, packed, 1.0, y)
+    return bl.lib().bitlinear_forward_grouped_ws(ctypes.addressof(arr), len(problems), xdt, ws,
+                                                 ws_bytes, None)
+
+
+def grouped_ws_bytes(problems):
+    arr = (bl._Problem * max(1, len(problems)))()
+    for i, (x, M, K, N, packed, y) in enumerate(problems):
+        arr[i] = bl._Problem(x, M, K, N, packed, 1.0, y)
+    return bl.lib().bitlinear_workspace_bytes_grouped(ctypes.addressof(arr), len(problems))
+
+
+def test_grouped_ws_rejects_bad_arguments():
+    good = (FAKE, 8, 256, 64, FAKE, FAKE)
+    assert bl.lib().bitlinear_forward_grouped_ws(None, 1, 0, FAKE, 1, None) == bl.BITLINEAR_ERR_ARG
+    assert grouped_ws([]) == bl.BITLINEAR_ERR_ARG
+    assert grouped_ws([good] * 9) == bl.BITLINEAR_ERR_ARG
+    assert grouped_ws([good, (FAKE, 8, 200, 64, FAKE, FAKE)]) == bl.BITLINEAR_ERR_SHAPE
+    assert grouped_ws([good, (None, 8, 256, 64, FAKE, FAKE)]) == bl.BITLINEAR_ERR_ARG
+    assert grouped_ws([good, (FAKE + 8, 8, 256, 64, FAKE, FAKE)]) == bl.BITLINEAR_ERR_ALIGN
+    assert grouped_ws([good], xdt=5) == bl.BITLINEAR_ERR_DTYPE
+    assert grouped_ws([(None, 0, 256, 64, None, None)]) == bl.BITLINEAR_OK   # only empty problems
+
+
+def test_grouped_ws_bytes():
+    size_max = ctypes.c_size_t(-1).value
+    small = [(None, 1, 2560, 6912, None, None), (None, 6, 6912, 2560, None, None)]
+    assert grouped_ws_bytes(small) == 0                       # one GEMV launch
+    big = [(None, 8, 2560, 6912, None, None), (None, 8, 6912, 2560, None, None)]
+    need = grouped_ws_bytes(big)
+    assert need >= 8 * 2560 + 8 * 6912 + 4 * 8 * 4
+    assert need >= grouped_ws_bytes(big[:1])
+    assert grouped_ws_bytes([(None, 8, 200, 64, None, None)]) == size_max
+    assert grouped_ws_bytes([]) == size_max

@@ -58,3 +58,57 @@ def test_grouped_eight_problems_fp32():
     ys, _ = run_group(cases)
     for c, y in zip(cases, ys):
         assert check_y(y, c.oracle_full()[1]) == 1.0
+
+
+# ---------------------------------------------- grouped tensor-core path
+
+def run_group_ws(cases, xs=None):
+    import torch
+    probs = []
+    for i, c in enumerate(cases):
+        x = c.x_tensor() if xs is None else xs[i]
+        probs.append((x, c.packed_tensor(), c.gamma, c.N, None))
+    need = bl.bitlinear_workspace_bytes_grouped(probs)
+    ws = torch.empty((max(need, 1),), dtype=torch.uint8, device="cuda")
+    outs = bl.bitlinear_forward_grouped(probs, workspace=ws)
+    torch.cuda.synchronize()
+    return [tensor_to_bf16_bits(y) for y in outs]
+
+
+def test_grouped_tc_mixed_shapes_match_single_calls():
+    # batch 8 of four 2B shapes: one quantisation launch and one GEMM launch;
+    # every problem equals the oracle and its own bitlinear_forward call
+    cases = [Case(8, 2560, 2560, w_seed=61, x_seed=71), Case(8, 2560, 640, w_seed=62, x_seed=72),
+             Case(8, 2560, 6912, w_seed=63, x_seed=73), Case(8, 6912, 2560, w_seed=64, x_seed=74)]
+    ys = run_group_ws(cases)
+    for c, y in zip(cases, ys):
+        assert check_y(y, c.oracle_full()[1]) == 1.0
+        single = c.run(path=bl.PATH_TC, debug=False)["y"]
+        np.testing.assert_array_equal(y, single)
+
+
+def test_grouped_tc_layer_b64():
+    # the seven projections of one decoder layer at batch 64 (token tile 64)
+    cases = [Case(p.M, p.K, p.N, w_seed=p.w_seed, x_seed=p.x_seed)
+             for p in workloads.layer_set_2b(64, layers=1).problems]
+    ys = run_group_ws(cases)
+    for c, y in zip(cases, ys):
+        assert check_y(y, c.oracle_full()[1]) == 1.0
+
+
+def test_grouped_tc_mixed_batches_fp32():
+    # one problem above the GEMV threshold sends the whole group to the
+    # tensor-core path, M = 1 and ragged shapes included; largest M sets the tile
+    cases = [Case(1, 256, 300, w_seed=81, x_seed=91, x_dtype="fp32"),
+             Case(40, 1280, 333, w_seed=82, x_seed=92, x_dtype="fp32"),
+             Case(150, 384, 129, w_seed=83, x_seed=93, x_dtype="fp32")]
+    ys = run_group_ws(cases)
+    for c, y in zip(cases, ys):
+        assert check_y(y, c.oracle_full()[1]) == 1.0
+
+
+def test_grouped_ws_small_batches_use_gemv():
+    cases = [Case(1, 2560, 6912, w_seed=1, x_seed=101), Case(4, 6912, 2560, w_seed=2, x_seed=102)]
+    ys = run_group_ws(cases)
+    for c, y in zip(cases, ys):
+        assert check_y(y, c.oracle_full()[1]) == 1.0
