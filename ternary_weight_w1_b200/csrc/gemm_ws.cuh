@@ -16,17 +16,22 @@
 // BT in {32, 64, 128, 192} tokens, so small token counts still use the
 // tensor cores without padding M to 128.
 //
-// Work split (stream-K): the T tiles x KB k-blocks are cut into one
-// contiguous range of k-blocks per CTA (persistent, one CTA per SM). A tile
-// whose k-blocks span two or more CTAs is finished by the CTA holding its
-// first k-block: each other CTA stores its int32 partial accumulator
-// [128][BT] into its own workspace slot and raises per-warp flags; the
-// finishing CTA adds the partials (int32 addition, exact in any order),
-// rescales and stores bf16. A CTA's range is at least one tile long, so the
-// partial of a tile is always written at the start of a range and read at
-// the end of another; flags are cleared by the quantisation kernel that
-// precedes every GEMM launch. With unit = KB the ranges are whole tiles and
-// no partials are used.
+// A launch computes one or several independent problems (a problem table of
+// up to eight, sharing the token tile); their tiles and k-blocks are numbered
+// one problem after the other.
+//
+// Work split (stream-K): the k-blocks of all tiles are cut into one
+// contiguous range per CTA (persistent, one CTA per SM). A tile whose
+// k-blocks span two or more CTAs is finished by the CTA holding its first
+// k-block: each other CTA stores its int32 partial accumulator [128][BT]
+// into its own workspace slot and raises per-warp flags; the finishing CTA
+// adds the partials (int32 addition, exact in any order), rescales and
+// stores bf16. A CTA stores at most one partial (only the first segment of a
+// range can start inside a tile) and finishes tiles only at the end of its
+// range, while its contributors write theirs at the start of their ranges.
+// Flags are cleared by the quantisation kernel that precedes every GEMM
+// launch. Without the split (Params::split = 0) the ranges are whole tiles
+// and no partials are used.
 //
 // A k-block is 256 k. One TMA copy brings the x~ tile of a k-block (a 3-D
 // box of two 128-byte-swizzled [BT][128] sub-tiles) and another the packed
