@@ -417,17 +417,16 @@ size_t tc_group_bytes(const TcJob *jobs, int n, bool split)
     return b + (split ? tc_split_bytes(max_M) : 0);
 }
 
-template <bool B_PACKED, bool RESCALE>
-int launch_gemm(const CUtensorMap &ma, const CUtensorMap &mb, const tc::Params &p,
-                const DeviceInfo &dev, cudaStream_t st)
+int launch_int8_gemm(const CUtensorMap &ma, const CUtensorMap &mb, const tc::Params &p,
+                     const DeviceInfo &dev, cudaStream_t st)
 {
-    cudaError_t e = allow_smem<tc::gemm_kernel<B_PACKED, RESCALE>>(dev.id, tc::SMEM_BYTES);
+    cudaError_t e = allow_smem<tc::gemm_kernel>(dev.id, tc::SMEM_BYTES);
     if (e != cudaSuccess)
         return launch_status(e);
     const int tiles = ((p.M + tc::BM - 1) / tc::BM) * ((p.N + tc::BN - 1) / tc::BN);
     const int grid = std::min(tiles, dev.sms);
-    e = launch(tc::gemm_kernel<B_PACKED, RESCALE>, dim3(grid), dim3(tc::THREADS),
-               static_cast<size_t>(tc::SMEM_BYTES), st, ma, mb, p);
+    e = launch(tc::gemm_kernel, dim3(grid), dim3(tc::THREADS), static_cast<size_t>(tc::SMEM_BYTES),
+               st, ma, mb, p);
     return launch_status(e);
 }
 
@@ -882,9 +881,9 @@ extern "C" int bitlinear_int8_gemm(const int8_t *A_dev, const int8_t *B_dev, int
     if (!make_map_u8(&ma, A_dev, M, K, tc::BM, tc::BK, true) ||
         !make_map_u8(&mb, B_dev, N, K, tc::BN, tc::BK, true))
         return BITLINEAR_ERR_CUDA;
-    tc::Params p{static_cast<int>(M), static_cast<int>(N), static_cast<int>(K), 0.0f, nullptr,
-                 nullptr, nullptr, C_dev, kWaitLimitNs, 0};
-    return launch_gemm<false, false>(ma, mb, p, *dev, static_cast<cudaStream_t>(cuda_stream));
+    tc::Params p{static_cast<int>(M), static_cast<int>(N), static_cast<int>(K), C_dev,
+                 kWaitLimitNs};
+    return launch_int8_gemm(ma, mb, p, *dev, static_cast<cudaStream_t>(cuda_stream));
 }
 
 // ======================================================== no-allocation path
