@@ -281,21 +281,27 @@ def time_graph_steps(dist, wl, steps: int, clocks: ClockSampler | None, separate
 
 def time_e2e(dist, wl, steps: int):
     """Same steps through the public Python API, with each step's tokens copied
-    from pinned host memory and its outputs read back to pinned host memory."""
+    from pinned host memory and its outputs read back to pinned host memory.
+    Both tokens of a step sit in one pinned buffer (one host-to-device copy)
+    and both outputs land in one device buffer (one device-to-host copy)."""
     import torch
-    host_x = [[m["x"][j].cpu().pin_memory() for j in range(ROTATE)] for m in wl.mats]
-    host_y = [torch.empty(m["y"][0].shape, dtype=torch.bfloat16).pin_memory() for m in wl.mats]
-    dev_x = [m["x"][0].clone() for m in wl.mats]
+    xk = [m["p"].K for m in wl.mats]
+    yn = [m["p"].N for m in wl.mats]
+    host_x = [torch.cat([m["x"][j].reshape(-1) for m in wl.mats]).cpu().pin_memory()
+              for j in range(ROTATE)]
+    host_y = torch.empty(sum(yn), dtype=torch.bfloat16).pin_memory()
+    dev_x = torch.empty(sum(xk), dtype=torch.bfloat16, device=wl.mats[0]["x"][0].device)
+    dev_y = torch.empty(sum(yn), dtype=torch.bfloat16, device=dev_x.device)
+    xs = list(torch.split(dev_x, xk))
+    ys = list(torch.split(dev_y, yn))
 
     def one(i):
         j = i % ROTATE
-        for k in range(len(wl.mats)):
-            dev_x[k].copy_(host_x[k][j], non_blocking=True)
+        dev_x.copy_(host_x[j], non_blocking=True)
         wl.bl.bitlinear_forward_grouped(
-            [(dev_x[k], m["packed"][j], m["gamma"], m["p"].N, m["y"][j])
+            [(xs[k].view(1, -1), m["packed"][j], m["gamma"], m["p"].N, ys[k].view(1, -1))
              for k, m in enumerate(wl.mats)])
-        for k, m in enumerate(wl.mats):
-            host_y[k].copy_(m["y"][j], non_blocking=True)
+        host_y.copy_(dev_y, non_blocking=True)
 
     for i in range(5):
         one(i)
@@ -354,19 +360,23 @@ def bench_prefill(bl, device, reps: int = 20):
     return ms, ops
 
 
-def time_graph(fn, reps: int) -> float:
+def time_graph(fn, reps: int, nvtx: str | None = None) -> float:
     """Mean ms of `fn` (captured once in a CUDA graph) over `reps` replays,
-    after three warm-up replays."""
+    after three warm-up replays; the timed replays sit in NVTX range `nvtx`."""
     import torch
     g = capture_graph(fn)
     for _ in range(3):
         g.replay()
     torch.cuda.synchronize()
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if nvtx:
+        torch.cuda.nvtx.range_push(nvtx)
     start.record()
     for _ in range(reps):
         g.replay()
     end.record()
+    if nvtx:
+        torch.cuda.nvtx.range_pop()
     torch.cuda.synchronize()
     del g
     return start.elapsed_time(end) / reps
@@ -404,7 +414,7 @@ def bench_layer_set(bl, device, batches=(1, 8, 64), reps: int = 10):
         launches = layers * (1 if ws_bytes == 0 else 2)
         step()
         torch.cuda.synchronize()
-        ms = time_graph(step, reps)
+        ms = time_graph(step, reps, nvtx=f"layer_set_b{B}_timed")
         out[f"B={B}"] = {"us_per_layer": round(ms * 1e3 / layers, 2),
                          "GBps_packed": round(wbytes / (ms * 1e-3) / 1e9, 1),
                          "TOPS": round(2 * B * wbytes * 4 / (ms * 1e-3) / 1e12, 2),
@@ -504,6 +514,8 @@ def run_ours(args, dist):
     ms_e2e = time_e2e(dist, wl, e2e_steps)
     e2e_value = wl.packed_bytes_per_step * e2e_steps * dist.world / (ms_e2e * 1e-3) / 1e9
 
+    if args.layer_set_only:
+        return {"layer_set": bench_layer_set(bl, device)}
     pre_ms, pre_ops = bench_prefill(bl, device)
     pre_tops = pre_ops / (pre_ms * 1e-3) / 1e12
     int8_peak = peaks["bf16_tflops"] * INT8_PER_BF16
@@ -623,6 +635,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extra", action="store_true",
                     help="skip the layer-set and large-shape measurements")
+    ap.add_argument("--layer-set-only", action="store_true",
+                    help="only the layer-set measurement after the decode step (for profiling)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")

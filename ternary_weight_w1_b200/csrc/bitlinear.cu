@@ -216,8 +216,11 @@ cudaError_t launch_qa(const void *x, int M, int K, int8_t *xq, float *beta, int 
                   K, xq, beta, rowsum, clear, n_clear);
 }
 
-// Register cache per lane and warps per row by row length: one warp per row
-// up to 8192 bf16 (4096 fp32) elements, eight for longer rows.
+// Register cache per lane and warps per row by row length: every lane holds
+// its whole share of a row in registers up to 16384 bf16 (8192 fp32)
+// elements per row, so a row is read from memory once and small batches are
+// not held up by dependent re-reads; longer rows take eight warps and
+// re-read the rest.
 int launch_quant_act(const void *x, bitlinear_dtype xdt, int M, int K, int8_t *xq, float *beta,
                      int *rowsum, cudaStream_t st, int *clear = nullptr, int n_clear = 0)
 {
@@ -230,15 +233,23 @@ int launch_quant_act(const void *x, bitlinear_dtype xdt, int M, int K, int8_t *x
             e = launch_qa<true, 4, 1>(x, M, K, xq, beta, rowsum, st, clear, n_clear);
         else if (nvec <= 32 * 8)
             e = launch_qa<true, 8, 1>(x, M, K, xq, beta, rowsum, st, clear, n_clear);
-        else if (nvec <= 32 * 32)
+        else if (nvec <= 32 * 16)
             e = launch_qa<true, 16, 1>(x, M, K, xq, beta, rowsum, st, clear, n_clear);
+        else if (nvec <= 64 * 16)
+            e = launch_qa<true, 16, 2>(x, M, K, xq, beta, rowsum, st, clear, n_clear);
+        else if (nvec <= 128 * 16)
+            e = launch_qa<true, 16, 4>(x, M, K, xq, beta, rowsum, st, clear, n_clear);
         else
             e = launch_qa<true, 16, 8>(x, M, K, xq, beta, rowsum, st, clear, n_clear);
     } else {
         if (nvec <= 32 * 4)
             e = launch_qa<false, 4, 1>(x, M, K, xq, beta, rowsum, st, clear, n_clear);
-        else if (nvec <= 32 * 16)
+        else if (nvec <= 32 * 8)
             e = launch_qa<false, 8, 1>(x, M, K, xq, beta, rowsum, st, clear, n_clear);
+        else if (nvec <= 64 * 8)
+            e = launch_qa<false, 8, 2>(x, M, K, xq, beta, rowsum, st, clear, n_clear);
+        else if (nvec <= 128 * 8)
+            e = launch_qa<false, 8, 4>(x, M, K, xq, beta, rowsum, st, clear, n_clear);
         else
             e = launch_qa<false, 8, 8>(x, M, K, xq, beta, rowsum, st, clear, n_clear);
     }
@@ -444,25 +455,50 @@ int launch_gemm_ws(const wsg::Maps &maps, const wsg::Params &p, int grid, const 
 }
 
 // Quantisation of several problems' rows in one launch (one warp per row).
-int launch_quant_group(const TcJob *jobs, int n, bitlinear_dtype xdt, int8_t *const *xq,
-                       float *const *beta, int *const *rowsum, cudaStream_t st, int *clear,
-                       int n_clear)
+template <bool BF16, int CACHE, int WPR>
+cudaError_t launch_qa_group(const TcJob *jobs, int n, int8_t *const *xq, float *const *beta,
+                            int *const *rowsum, cudaStream_t st, int *clear, int n_clear)
 {
+    constexpr int rpb = qa::rows_per_block<WPR>();
     qa::GroupParams g{};
     int blocks = 0;
     for (int i = 0; i < n; ++i) {
         g.prob[i] = qa::GroupRows{jobs[i].x, xq[i], beta[i], rowsum[i], jobs[i].M, jobs[i].K,
                                   blocks};
-        blocks += (jobs[i].M + qa::WARPS - 1) / qa::WARPS;
+        blocks += (jobs[i].M + rpb - 1) / rpb;
     }
     g.count = n;
     g.clear = clear;
     g.n_clear = n_clear;
+    return launch(qa::quant_act_grouped_kernel<BF16, CACHE, WPR>, dim3(blocks), dim3(qa::THREADS),
+                  0, st, g);
+}
+
+// Warps per row chosen by the group's longest row, as for one problem.
+int launch_quant_group(const TcJob *jobs, int n, bitlinear_dtype xdt, int8_t *const *xq,
+                       float *const *beta, int *const *rowsum, cudaStream_t st, int *clear,
+                       int n_clear)
+{
+    int max_K = 0;
+    for (int i = 0; i < n; ++i)
+        max_K = std::max(max_K, jobs[i].K);
+    const int nvec = max_K / 8;
     cudaError_t e;
-    if (xdt == BITLINEAR_BF16)
-        e = launch(qa::quant_act_grouped_kernel<true, 16>, dim3(blocks), dim3(qa::THREADS), 0, st, g);
-    else
-        e = launch(qa::quant_act_grouped_kernel<false, 8>, dim3(blocks), dim3(qa::THREADS), 0, st, g);
+    if (xdt == BITLINEAR_BF16) {
+        if (nvec <= 32 * 16)
+            e = launch_qa_group<true, 16, 1>(jobs, n, xq, beta, rowsum, st, clear, n_clear);
+        else if (nvec <= 64 * 16)
+            e = launch_qa_group<true, 16, 2>(jobs, n, xq, beta, rowsum, st, clear, n_clear);
+        else
+            e = launch_qa_group<true, 16, 8>(jobs, n, xq, beta, rowsum, st, clear, n_clear);
+    } else {
+        if (nvec <= 32 * 8)
+            e = launch_qa_group<false, 8, 1>(jobs, n, xq, beta, rowsum, st, clear, n_clear);
+        else if (nvec <= 64 * 8)
+            e = launch_qa_group<false, 8, 2>(jobs, n, xq, beta, rowsum, st, clear, n_clear);
+        else
+            e = launch_qa_group<false, 8, 8>(jobs, n, xq, beta, rowsum, st, clear, n_clear);
+    }
     return launch_status(e);
 }
 

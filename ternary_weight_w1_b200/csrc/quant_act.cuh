@@ -153,7 +153,7 @@ quant_act_kernel(const void *__restrict__ x, int M, int K, int8_t *__restrict__ 
     quant_row<BF16, CACHE, WPR>(x, M, K, xq, beta_out, rowsum_out, m, warp % WPR);
 }
 
-// Several problems' token rows in one launch (one warp per row): block b
+// Several problems' token rows in one launch (WPR warps per row): block b
 // belongs to the problem whose block range [first_block, next first_block)
 // holds it.
 constexpr int MAX_PROBLEMS = 8;
@@ -174,7 +174,7 @@ struct GroupParams {
     int n_clear;
 };
 
-template <bool BF16, int CACHE>
+template <bool BF16, int CACHE, int WPR>
 __global__ void __launch_bounds__(THREADS)
 quant_act_grouped_kernel(const __grid_constant__ GroupParams g)
 {
@@ -182,12 +182,13 @@ quant_act_grouped_kernel(const __grid_constant__ GroupParams g)
     while (q + 1 < g.count && static_cast<int>(blockIdx.x) >= g.prob[q + 1].first_block)
         ++q;
     const GroupRows &r = g.prob[q];
-    const int m = (static_cast<int>(blockIdx.x) - r.first_block) * WARPS + (threadIdx.x >> 5);
+    const int warp = threadIdx.x >> 5;
+    const int m = (static_cast<int>(blockIdx.x) - r.first_block) * rows_per_block<WPR>() + warp / WPR;
     pdl_wait();
     if (g.clear != nullptr && blockIdx.x == 0)
         for (int i = threadIdx.x; i < g.n_clear; i += THREADS)
             g.clear[i] = 0;
-    quant_row<BF16, CACHE, 1>(r.x, r.M, r.K, r.xq, r.beta, r.rowsum, m, 0);
+    quant_row<BF16, CACHE, WPR>(r.x, r.M, r.K, r.xq, r.beta, r.rowsum, m, warp % WPR);
 }
 
 }  // namespace qa
