@@ -162,17 +162,6 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap *map
         : "memory");
 }
 
-// 4-D tiled tensor copy global -> shared (no multicast).
-__device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap *map, int c0, int c1,
-                                            int c2, int c3, uint32_t bar)
-{
-    asm volatile(
-        "cp.async.bulk.tensor.4d.shared::cluster.global.mbarrier::complete_tx::bytes "
-        "[%0], [%1, {%2, %3, %4, %5}], [%6];" ::"r"(dst),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(bar)
-        : "memory");
-}
-
 __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap *map)
 {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map))
@@ -365,41 +354,6 @@ __device__ __forceinline__ void pdl_wait()
 __device__ __forceinline__ void pdl_launch_dependents()
 {
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-}
-
-// ------------------------------------------------------------ block reduce
-
-// Max of non-negative floats over the block (bit patterns compare as uints).
-template <int WARPS>
-__device__ __forceinline__ float block_max_nonneg(float v, uint32_t *red)
-{
-    uint32_t u = __reduce_max_sync(0xffffffffu, __float_as_uint(v));
-    const int warp = threadIdx.x >> 5;
-    if ((threadIdx.x & 31) == 0)
-        red[warp] = u;
-    __syncthreads();
-    uint32_t m = red[0];
-#pragma unroll
-    for (int w = 1; w < WARPS; ++w)
-        m = max(m, red[w]);
-    __syncthreads();
-    return __uint_as_float(m);
-}
-
-template <int WARPS>
-__device__ __forceinline__ int block_sum_int(int v, int *red)
-{
-    int s = __reduce_add_sync(0xffffffffu, v);
-    const int warp = threadIdx.x >> 5;
-    if ((threadIdx.x & 31) == 0)
-        red[warp] = s;
-    __syncthreads();
-    int t = 0;
-#pragma unroll
-    for (int w = 0; w < WARPS; ++w)
-        t += red[w];
-    __syncthreads();
-    return t;
 }
 
 // ------------------------------------------------------ quantisation helpers
