@@ -16,8 +16,8 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libbitlinear.so")
 SOURCES = [os.path.join(CSRC, "bitlinear.cu"), os.path.join(CSRC, "pack.cpp")]
-DEPS = SOURCES + [os.path.join(CSRC, f) for f in
-                  ("common.cuh", "gemv.cuh", "gemm_tc.cuh", "quant_act.cuh")] + [
+# Everything the translation units include: every header in csrc/ and the ABI header.
+DEPS = SOURCES + sorted(os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith(".cuh")) + [
     os.path.join(HERE, "..", "include", "bitlinear.h")]
 
 NVCC_FLAGS = [
