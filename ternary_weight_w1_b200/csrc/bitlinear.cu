@@ -296,11 +296,10 @@ struct GemvJob {
 int launch_gemv(const GemvJob *jobs, int count, bitlinear_dtype xdt, const DeviceInfo &dev,
                 cudaStream_t st)
 {
-    int Mmax = 1, Kmax = 128;
+    int Mmax = 1;
     double total_bytes = 0.0;
     for (int i = 0; i < count; ++i) {
         Mmax = std::max(Mmax, jobs[i].M);
-        Kmax = std::max(Kmax, jobs[i].K);
         total_bytes += static_cast<double>((jobs[i].N + 15) / 16) * 16.0 * jobs[i].K / 4.0;
     }
     const int MT = Mmax <= 1 ? 1 : Mmax <= 2 ? 2 : Mmax <= 4 ? 4 : Mmax <= 8 ? 8 : 16;
@@ -336,7 +335,10 @@ int launch_gemv(const GemvJob *jobs, int count, bitlinear_dtype xdt, const Devic
         stages = std::max(stages, (q[i] * (jobs[i].K / 128) * gemv::PIECE + gemv::STAGE - 1) /
                                       gemv::STAGE);
     }
-    const int xq_cap = MT * Kmax;
+    // Each CTA quantises only its own problem's M rows into shared memory.
+    int xq_cap = 0;
+    for (int i = 0; i < count; ++i)
+        xq_cap = std::max(xq_cap, jobs[i].M * jobs[i].K);
     const int acc_cap = qmax * 16 * MT;
     // Ring depth: the whole share when it is small (room for the next
     // kernel's blocks on the same SM under programmatic launch), else as deep

@@ -74,7 +74,7 @@ struct Params {
     Problem prob[MAX_PROBLEMS];
     int count;              // problems in this launch
     int slots;              // ring slots (<= MAX_SLOTS)
-    int xq_cap;             // shared bytes for x~: max over problems of MT * K
+    int xq_cap;             // shared bytes for x~: max over problems of M * K
     int acc_cap;            // row accumulators: max over problems of blocks_per_cta * 16 * MT
     uint64_t wait_limit_ns;
 };

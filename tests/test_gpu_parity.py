@@ -83,6 +83,18 @@ def test_tc_tiles_split_between_two_ctas(cuda):
     assert c.check_full(c.run(path=bl.PATH_TC)) == 1.0
 
 
+@pytest.mark.parametrize("path,M", [(bl.PATH_GEMV, 1), (bl.PATH_GEMV, 3), (bl.PATH_TC, 3),
+                                    (bl.PATH_TC, 40)])
+def test_maximum_k_and_single_output_row(cuda, path, M):
+    # K = 65536 (the largest K the forward calls accept) and N = 1 (one row
+    # block holding 15 padding rows), on both paths
+    for K, N in [(65536, 130), (2560, 1)]:
+        if path == bl.PATH_GEMV and M * K > 196608:
+            continue
+        c = Case(M, K, N, w_seed=K + N + M, x_seed=M + K)
+        assert c.check_full(c.run(path=path)) == 1.0
+
+
 def test_tc_many_tiles_per_cta(cuda):
     # more tiles than SMs: every CTA loops over several tiles and both TMEM
     # accumulator buffers are reused
