@@ -140,7 +140,7 @@ __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void *src, uint32_t
         : "memory");
 }
 
-// 2-D tiled tensor copy global -> shared (no multicast).
+// 2-D tiled tensor copy global -> this CTA's shared memory.
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, int x,
                                             int y, uint32_t bar)
 {
@@ -151,7 +151,7 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map
         : "memory");
 }
 
-// 3-D tiled tensor copy global -> shared (no multicast).
+// 3-D tiled tensor copy global -> this CTA's shared memory.
 __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap *map, int c0, int c1,
                                             int c2, uint32_t bar)
 {
