@@ -129,6 +129,36 @@ def _ptr(t) -> int | None:
     return None if t is None else t.data_ptr()
 
 
+def _dev(t, name: str, dtype=None, shape=None, min_numel: int = 0) -> int | None:
+    """Device address of tensor ``t`` after checking that the library can use
+    it: a contiguous CUDA tensor on the current device, of ``dtype`` and
+    ``shape`` when given, with at least ``min_numel`` elements. A host tensor
+    handed to a kernel would make it read host addresses, so it is refused
+    here, before any call."""
+    if t is None:
+        return None
+    import torch
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor (got device {t.device})")
+    if t.device.index != torch.cuda.current_device():
+        raise ValueError(f"{name} is on {t.device}, the current device is "
+                         f"cuda:{torch.cuda.current_device()}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    if t.numel() < min_numel:
+        raise ValueError(f"{name} holds {t.numel()} elements, {min_numel} needed")
+    return t.data_ptr()
+
+
+def _packed_ok(packed, N: int, K: int) -> int | None:
+    import torch
+    return _dev(packed, "packed", torch.uint8, min_numel=max(bitlinear_packed_bytes(N, K), 1))
+
+
 def _stream(stream) -> int | None:
     import torch
     if stream is None:
@@ -179,8 +209,9 @@ def bitlinear_quant_act(x, xq=None, beta=None, stream=None):
         xq = torch.empty((M, K), dtype=torch.int8, device=x.device)
     if beta is None:
         beta = torch.empty((M,), dtype=torch.float32, device=x.device)
-    _check(lib().bitlinear_quant_act(_ptr(x), _xdt(x), M, K, _ptr(xq), _ptr(beta),
-                                     _stream(stream)),
+    _check(lib().bitlinear_quant_act(_dev(x, "x"), _xdt(x), M, K,
+                                     _dev(xq, "xq", torch.int8, (M, K)),
+                                     _dev(beta, "beta", torch.float32, (M,)), _stream(stream)),
            "bitlinear_quant_act")
     return xq, beta
 
@@ -209,8 +240,10 @@ def bitlinear_forward(x, packed, gamma: float, N: int, y=None, workspace=None,
     if workspace is None and need > 0:
         workspace = torch.empty((need,), dtype=torch.uint8, device=x.device)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    args = (_ptr(x), _xdt(x), M, K, _ptr(packed), float(gamma), N, _ptr(y),
-            _ptr(workspace), ws_bytes, _stream(stream), _ptr(acc), _ptr(xq), _ptr(beta))
+    args = (_dev(x, "x"), _xdt(x), M, K, _packed_ok(packed, N, K), float(gamma), N,
+            _dev(y, "y", torch.bfloat16, (M, N)), _dev(workspace, "workspace"), ws_bytes,
+            _stream(stream), _dev(acc, "acc", torch.int32, (M, N)),
+            _dev(xq, "xq", torch.int8, (M, K)), _dev(beta, "beta", torch.float32, (M,)))
     if path == PATH_AUTO:
         rc = lib().bitlinear_forward(*args)
     else:
@@ -231,7 +264,8 @@ def bitlinear_forward_inject_timeout(x, packed, gamma: float, N: int, timeout_us
     if workspace is None:
         workspace = torch.empty((max(need, 1),), dtype=torch.uint8, device=x.device)
     return int(lib().bitlinear_forward_inject_timeout(
-        _ptr(x), _xdt(x), M, K, _ptr(packed), float(gamma), N, _ptr(y), _ptr(workspace),
+        _dev(x, "x"), _xdt(x), M, K, _packed_ok(packed, N, K), float(gamma), N,
+        _dev(y, "y", torch.bfloat16, (M, N)), _dev(workspace, "workspace", torch.uint8),
         workspace.numel(), _stream(stream), int(timeout_us)))
 
 
@@ -249,7 +283,8 @@ def bitlinear_int8_gemm(A, B, C=None, stream=None):
     N = B.shape[0]
     if C is None:
         C = torch.empty((M, N), dtype=torch.int32, device=A.device)
-    _check(lib().bitlinear_int8_gemm(_ptr(A), _ptr(B), _ptr(C), M, N, K, _stream(stream)),
+    _check(lib().bitlinear_int8_gemm(_dev(A, "A", torch.int8, (M, K)), _dev(B, "B", torch.int8, (N, K)),
+                                     _dev(C, "C", torch.int32, (M, N)), M, N, K, _stream(stream)),
            "bitlinear_int8_gemm")
     return C
 
@@ -263,8 +298,9 @@ def bitlinear_forward_noalloc(x, packed, gamma: float, N: int, y=None, stream=No
     M, K = x.shape
     if y is None:
         y = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
-    _check(lib().bitlinear_forward_noalloc(_ptr(x), _xdt(x), M, K, _ptr(packed), float(gamma),
-                                           N, _ptr(y), _stream(stream)),
+    _check(lib().bitlinear_forward_noalloc(_dev(x, "x"), _xdt(x), M, K, _packed_ok(packed, N, K),
+                                           float(gamma), N, _dev(y, "y", torch.bfloat16, (M, N)),
+                                           _stream(stream)),
            "bitlinear_forward_noalloc")
     return y
 
@@ -278,7 +314,12 @@ def _problem_array(problems, alloc_y):
         if y is None and alloc_y:
             y = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
         outs.append(y)
-        arr[i] = _Problem(_ptr(x), M, K, N, _ptr(packed), float(gamma), _ptr(y))
+        if alloc_y:
+            arr[i] = _Problem(_dev(x, f"problems[{i}].x"), M, K, N,
+                              _packed_ok(packed, N, K), float(gamma),
+                              _dev(y, f"problems[{i}].y", torch.bfloat16, (M, N)))
+        else:                              # sizing only: shapes, no pointers
+            arr[i] = _Problem(None, M, K, N, None, float(gamma), None)
     return arr, outs
 
 
@@ -295,6 +336,7 @@ def bitlinear_forward_grouped(problems, stream=None, workspace=None):
     allocate it here); all x share one dtype. Without ``workspace`` every
     problem must fit the GEMV (one launch); with it any batch size is accepted
     (``bitlinear_forward_grouped_ws``). Returns the list of outputs."""
+    import torch
     if not problems:
         return []
     xdt = _xdt(problems[0][0])
@@ -305,7 +347,7 @@ def bitlinear_forward_grouped(problems, stream=None, workspace=None):
                "bitlinear_forward_grouped")
     else:
         _check(lib().bitlinear_forward_grouped_ws(ctypes.addressof(arr), len(problems), xdt,
-                                                  _ptr(workspace), workspace.numel(),
-                                                  _stream(stream)),
+                                                  _dev(workspace, "workspace", torch.uint8),
+                                                  workspace.numel(), _stream(stream)),
                "bitlinear_forward_grouped_ws")
     return outs

@@ -178,3 +178,23 @@ def test_grouped_ws_bytes():
     assert need >= grouped_ws_bytes(big[:1])
     assert grouped_ws_bytes([(None, 8, 200, 64, None, None)]) == size_max
     assert grouped_ws_bytes([]) == size_max
+
+
+def test_binding_refuses_host_tensors():
+    # a host tensor handed to a kernel would make it read host addresses:
+    # the binding refuses it before any library call (no GPU needed)
+    import torch
+    x = torch.zeros((4, 256), dtype=torch.bfloat16)
+    packed = torch.zeros((bl.bitlinear_packed_bytes(64, 256),), dtype=torch.uint8)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        bl.bitlinear_quant_act(x, xq=x.to(torch.int8), beta=torch.zeros(4))
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        bl.bitlinear_forward(x, packed, 1.0, 64, y=torch.zeros((4, 64), dtype=torch.bfloat16),
+                             path=bl.PATH_GEMV)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        bl.bitlinear_forward_grouped([(x, packed, 1.0, 64,
+                                       torch.zeros((4, 64), dtype=torch.bfloat16))])
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        bl.bitlinear_int8_gemm(torch.zeros((128, 128), dtype=torch.int8),
+                               torch.zeros((128, 128), dtype=torch.int8),
+                               torch.zeros((128, 128), dtype=torch.int32))
