@@ -129,34 +129,47 @@ def _ptr(t) -> int | None:
     return None if t is None else t.data_ptr()
 
 
-def _dev(t, name: str, dtype=None, shape=None, min_numel: int = 0) -> int | None:
-    """Device address of tensor ``t`` after checking that the library can use
-    it: a contiguous CUDA tensor on the current device, of ``dtype`` and
-    ``shape`` when given, with at least ``min_numel`` elements. A host tensor
-    handed to a kernel would make it read host addresses, so it is refused
-    here, before any call."""
-    if t is None:
-        return None
-    import torch
-    if not t.is_cuda:
-        raise ValueError(f"{name} must be a CUDA tensor (got device {t.device})")
-    if t.device.index != torch.cuda.current_device():
-        raise ValueError(f"{name} is on {t.device}, the current device is "
-                         f"cuda:{torch.cuda.current_device()}")
-    if not t.is_contiguous():
-        raise ValueError(f"{name} must be contiguous")
-    if dtype is not None and t.dtype != dtype:
-        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
-    if shape is not None and tuple(t.shape) != tuple(shape):
-        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
-    if t.numel() < min_numel:
-        raise ValueError(f"{name} holds {t.numel()} elements, {min_numel} needed")
-    return t.data_ptr()
+class _Args:
+    """Device addresses of one call's tensors, after checking that the library
+    can use them: contiguous CUDA tensors on the current device, of the dtype
+    and shape given, with at least ``min_numel`` elements. A host tensor handed
+    to a kernel would make it read host addresses, so it is refused here,
+    before any library call. The current device is looked up once per call."""
+
+    __slots__ = ("cur",)
+
+    def __init__(self):
+        self.cur = None
+
+    def ptr(self, t, name: str, dtype=None, shape=None, min_numel: int = 0) -> int | None:
+        if t is None:
+            return None
+        d = t.get_device()
+        if d < 0:
+            raise ValueError(f"{name} must be a CUDA tensor (got device {t.device})")
+        if self.cur is None:
+            import torch
+            self.cur = torch.cuda.current_device()
+        if d != self.cur:
+            raise ValueError(f"{name} is on cuda:{d}, the current device is cuda:{self.cur}")
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+        if dtype is not None and t.dtype != dtype:
+            raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+        if shape is not None and t.shape != shape:
+            raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+        if min_numel and t.numel() < min_numel:
+            raise ValueError(f"{name} holds {t.numel()} elements, {min_numel} needed")
+        return t.data_ptr()
+
+    def packed(self, packed, N: int, K: int) -> int | None:
+        import torch
+        # bitlinear_packed_bytes(N, K) for valid shapes (the library rejects
+        # the others itself): ceil(N / 16) row blocks of 16 * K / 4 bytes
+        need = (N + 15) // 16 * 16 * (K // 4) if N >= 1 and K >= 128 and K % 128 == 0 else 1
+        return self.ptr(packed, "packed", torch.uint8, min_numel=need)
 
 
-def _packed_ok(packed, N: int, K: int) -> int | None:
-    import torch
-    return _dev(packed, "packed", torch.uint8, min_numel=max(bitlinear_packed_bytes(N, K), 1))
 
 
 def _stream(stream) -> int | None:
@@ -203,15 +216,16 @@ def bitlinear_pack_weights(W) -> tuple[np.ndarray, float]:
 
 def bitlinear_quant_act(x, xq=None, beta=None, stream=None):
     """x~ (int8 [M][K]) and beta (fp32 [M]) of device activations x."""
+    a = _Args()
     import torch
     M, K = x.shape
     if xq is None:
         xq = torch.empty((M, K), dtype=torch.int8, device=x.device)
     if beta is None:
         beta = torch.empty((M,), dtype=torch.float32, device=x.device)
-    _check(lib().bitlinear_quant_act(_dev(x, "x"), _xdt(x), M, K,
-                                     _dev(xq, "xq", torch.int8, (M, K)),
-                                     _dev(beta, "beta", torch.float32, (M,)), _stream(stream)),
+    _check(lib().bitlinear_quant_act(a.ptr(x, "x"), _xdt(x), M, K,
+                                     a.ptr(xq, "xq", torch.int8, (M, K)),
+                                     a.ptr(beta, "beta", torch.float32, (M,)), _stream(stream)),
            "bitlinear_quant_act")
     return xq, beta
 
@@ -230,6 +244,7 @@ def bitlinear_forward(x, packed, gamma: float, N: int, y=None, workspace=None,
     ``bitlinear_workspace_bytes(M, N, K, path)`` bytes (allocated here when
     omitted); ``acc``/``xq``/``beta`` are optional debug outputs of the
     integer stages."""
+    a = _Args()
     import torch
     M, K = x.shape
     if y is None:
@@ -240,10 +255,10 @@ def bitlinear_forward(x, packed, gamma: float, N: int, y=None, workspace=None,
     if workspace is None and need > 0:
         workspace = torch.empty((need,), dtype=torch.uint8, device=x.device)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    args = (_dev(x, "x"), _xdt(x), M, K, _packed_ok(packed, N, K), float(gamma), N,
-            _dev(y, "y", torch.bfloat16, (M, N)), _dev(workspace, "workspace"), ws_bytes,
-            _stream(stream), _dev(acc, "acc", torch.int32, (M, N)),
-            _dev(xq, "xq", torch.int8, (M, K)), _dev(beta, "beta", torch.float32, (M,)))
+    args = (a.ptr(x, "x"), _xdt(x), M, K, a.packed(packed, N, K), float(gamma), N,
+            a.ptr(y, "y", torch.bfloat16, (M, N)), a.ptr(workspace, "workspace"), ws_bytes,
+            _stream(stream), a.ptr(acc, "acc", torch.int32, (M, N)),
+            a.ptr(xq, "xq", torch.int8, (M, K)), a.ptr(beta, "beta", torch.float32, (M,)))
     if path == PATH_AUTO:
         rc = lib().bitlinear_forward(*args)
     else:
@@ -256,6 +271,7 @@ def bitlinear_forward_inject_timeout(x, packed, gamma: float, N: int, timeout_us
                                      y=None, workspace=None, stream=None) -> int:
     """Run the tensor-core GEMM with one wait made to run out; returns the
     status the launch reported (the fault is read by bitlinear_get_fault)."""
+    a = _Args()
     import torch
     M, K = x.shape
     if y is None:
@@ -264,8 +280,8 @@ def bitlinear_forward_inject_timeout(x, packed, gamma: float, N: int, timeout_us
     if workspace is None:
         workspace = torch.empty((max(need, 1),), dtype=torch.uint8, device=x.device)
     return int(lib().bitlinear_forward_inject_timeout(
-        _dev(x, "x"), _xdt(x), M, K, _packed_ok(packed, N, K), float(gamma), N,
-        _dev(y, "y", torch.bfloat16, (M, N)), _dev(workspace, "workspace", torch.uint8),
+        a.ptr(x, "x"), _xdt(x), M, K, a.packed(packed, N, K), float(gamma), N,
+        a.ptr(y, "y", torch.bfloat16, (M, N)), a.ptr(workspace, "workspace", torch.uint8),
         workspace.numel(), _stream(stream), int(timeout_us)))
 
 
@@ -278,13 +294,14 @@ def bitlinear_get_fault(stream=None) -> tuple[int, int]:
 
 def bitlinear_int8_gemm(A, B, C=None, stream=None):
     """C (int32 [M][N]) = A (int8 [M][K]) @ B (int8 [N][K])^T on the tensor cores."""
+    a = _Args()
     import torch
     M, K = A.shape
     N = B.shape[0]
     if C is None:
         C = torch.empty((M, N), dtype=torch.int32, device=A.device)
-    _check(lib().bitlinear_int8_gemm(_dev(A, "A", torch.int8, (M, K)), _dev(B, "B", torch.int8, (N, K)),
-                                     _dev(C, "C", torch.int32, (M, N)), M, N, K, _stream(stream)),
+    _check(lib().bitlinear_int8_gemm(a.ptr(A, "A", torch.int8, (M, K)), a.ptr(B, "B", torch.int8, (N, K)),
+                                     a.ptr(C, "C", torch.int32, (M, N)), M, N, K, _stream(stream)),
            "bitlinear_int8_gemm")
     return C
 
@@ -294,18 +311,19 @@ def bitlinear_forward_noalloc(x, packed, gamma: float, N: int, y=None, stream=No
     scratch instead of a workspace, for callers that cannot allocate device
     memory (see include/bitlinear.h for the size limit and the sharing rules).
     Pass ``y`` to keep this wrapper from allocating the output."""
+    a = _Args()
     import torch
     M, K = x.shape
     if y is None:
         y = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
-    _check(lib().bitlinear_forward_noalloc(_dev(x, "x"), _xdt(x), M, K, _packed_ok(packed, N, K),
-                                           float(gamma), N, _dev(y, "y", torch.bfloat16, (M, N)),
+    _check(lib().bitlinear_forward_noalloc(a.ptr(x, "x"), _xdt(x), M, K, a.packed(packed, N, K),
+                                           float(gamma), N, a.ptr(y, "y", torch.bfloat16, (M, N)),
                                            _stream(stream)),
            "bitlinear_forward_noalloc")
     return y
 
 
-def _problem_array(problems, alloc_y):
+def _problem_array(problems, alloc_y, a=None):
     import torch
     arr = (_Problem * len(problems))()
     outs = []
@@ -315,9 +333,9 @@ def _problem_array(problems, alloc_y):
             y = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
         outs.append(y)
         if alloc_y:
-            arr[i] = _Problem(_dev(x, f"problems[{i}].x"), M, K, N,
-                              _packed_ok(packed, N, K), float(gamma),
-                              _dev(y, f"problems[{i}].y", torch.bfloat16, (M, N)))
+            arr[i] = _Problem(a.ptr(x, f"problems[{i}].x"), M, K, N,
+                              a.packed(packed, N, K), float(gamma),
+                              a.ptr(y, f"problems[{i}].y", torch.bfloat16, (M, N)))
         else:                              # sizing only: shapes, no pointers
             arr[i] = _Problem(None, M, K, N, None, float(gamma), None)
     return arr, outs
@@ -340,14 +358,15 @@ def bitlinear_forward_grouped(problems, stream=None, workspace=None):
     if not problems:
         return []
     xdt = _xdt(problems[0][0])
-    arr, outs = _problem_array(problems, alloc_y=True)
+    a = _Args()
+    arr, outs = _problem_array(problems, alloc_y=True, a=a)
     if workspace is None:
         _check(lib().bitlinear_forward_grouped(ctypes.addressof(arr), len(problems), xdt,
                                                _stream(stream)),
                "bitlinear_forward_grouped")
     else:
         _check(lib().bitlinear_forward_grouped_ws(ctypes.addressof(arr), len(problems), xdt,
-                                                  _dev(workspace, "workspace", torch.uint8),
+                                                  a.ptr(workspace, "workspace", torch.uint8),
                                                   workspace.numel(), _stream(stream)),
                "bitlinear_forward_grouped_ws")
     return outs
