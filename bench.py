@@ -55,9 +55,9 @@ INT8_PER_BF16 = 2.0        # nominal dense int8 / bf16 tensor ratio (4.5 / 2.25 
 TRAFFIC = {
     # grouped decode launch (up 2560->6912 + down 6912->2560, M=1): 8,847,360
     # algorithmic bytes; profiles/gemv_grouped_decode_2b_m1.md. The capture
-    # was taken on this kernel code; the source has changed since only in a
-    # comment of its parameter block.
-    "gemv": {"src": "4c50e519a059e647", "bytes_per_launch": 8895232},
+    # was taken on this kernel code; the source has changed since only in
+    # comments of its parameter block.
+    "gemv": {"src": "ea1ca4c9f8d28831", "bytes_per_launch": 8895232},
 }
 
 

@@ -331,6 +331,10 @@ int launch_gemv(const GemvJob *jobs, int count, bitlinear_dtype xdt, const Devic
     }
     int qmax = 1, stages = 1;
     for (int i = 0; i < count; ++i) {
+        // The kernel divides a piece index by K/128 with a multiply and shift,
+        // exact below 2^23 pieces (4 GiB of packed weights) per CTA.
+        if (static_cast<int64_t>(q[i]) * (jobs[i].K / 128) >= (int64_t(1) << 23))
+            return BITLINEAR_ERR_SHAPE;
         qmax = std::max(qmax, q[i]);
         stages = std::max(stages, (q[i] * (jobs[i].K / 128) * gemv::PIECE + gemv::STAGE - 1) /
                                       gemv::STAGE);

@@ -68,6 +68,8 @@ struct Problem {
     int blocks_per_cta;     // row blocks of 16 rows owned by one CTA
     int cta_begin;          // this problem's first CTA in the grid
     uint64_t kg_magic;      // ceil(2^32 / (K / 128)): i / KG == (i * kg_magic) >> 32
+                            // for every piece index i < 2^23 at any KG <= 512 (the
+                            // host keeps blocks_per_cta * KG below that)
 };
 
 struct Params {
