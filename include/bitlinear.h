@@ -49,7 +49,7 @@ extern "C" {
 typedef enum {
     BITLINEAR_OK = 0,
     BITLINEAR_ERR_ARG = 1,       /* null pointer or negative size */
-    BITLINEAR_ERR_SHAPE = 2,     /* K not a multiple of 128, K or N out of range */
+    BITLINEAR_ERR_SHAPE = 2,     /* K not a multiple of 128, a size out of range */
     BITLINEAR_ERR_ALIGN = 3,     /* a pointer misses its alignment */
     BITLINEAR_ERR_DTYPE = 4,     /* unknown bitlinear_dtype */
     BITLINEAR_ERR_CUDA = 5,      /* a CUDA runtime/driver call failed */
@@ -122,7 +122,8 @@ int bitlinear_quant_act(const void *x_dev, bitlinear_dtype xdt, int64_t M,
 /* ---------------------------------------------------------------- forward */
 
 /* Device workspace bytes bitlinear_forward needs for (M, N, K): 0 when the
- * GEMV path is taken (M <= 6), else room for x~ (M*K bytes), beta, the
+ * GEMV path is taken (M <= 6 and M * K <= 196608), else room for x~ (M*K
+ * bytes), beta, the
  * per-token sums of x~, and the tensor-core GEMM's inter-CTA region (flag
  * words and int32 partial sums of tiles whose k-range is split between
  * CTAs; at most 192 * 128 * 192 * 4 bytes). The flag words are cleared by
@@ -145,9 +146,10 @@ size_t bitlinear_workspace_bytes(int64_t M, int64_t N, int64_t K);
  *   xq_dev_or_null   [out, optional] [M][K] int8 x~
  *   beta_dev_or_null [out, optional] [M] fp32 beta
  * The optional outputs exist so that tests can compare the integer stages
- * bit for bit; pass NULL in production. M <= 6 runs one fused kernel
- * (quantisation in the prologue, dp4a over the packed weights); larger M runs
- * the quantisation kernel and the tcgen05 int8 tensor-core GEMM, whose
+ * bit for bit; pass NULL in production. M <= 6 with M * K <= 196608 runs one
+ * fused kernel (quantisation in the prologue, dp4a over the packed weights);
+ * other shapes run the quantisation kernel and the tcgen05 int8 tensor-core
+ * GEMM, whose
  * results do not depend on how its work is split between CTAs (the int32
  * partial sums are exact). */
 int bitlinear_forward(const void *x_dev, bitlinear_dtype xdt, int64_t M,
@@ -193,7 +195,8 @@ int bitlinear_forward_grouped(const bitlinear_problem *problems, int count,
                               bitlinear_dtype xdt, void *cuda_stream);
 
 /* Device workspace bytes bitlinear_forward_grouped_ws needs for these
- * problems: 0 when every non-empty problem has M <= 6 (one GEMV launch),
+ * problems: 0 when every non-empty problem takes the GEMV path on its own
+ * (M <= 6 and M * K <= 196608; one GEMV launch),
  * else the sum of each problem's x~, beta and row-sum regions plus one
  * inter-CTA region (see bitlinear_workspace_bytes). SIZE_MAX for invalid
  * problems. */
@@ -201,7 +204,8 @@ size_t bitlinear_workspace_bytes_grouped(const bitlinear_problem *problems,
                                          int count);
 
 /* Several independent BitLinear matmuls, at any batch size, in one pair of
- * launches. When every non-empty problem has M <= 6 this is
+ * launches. When every non-empty problem takes the GEMV path on its own
+ * (M <= 6 and M * K <= 196608) this is
  * bitlinear_forward_grouped (one GEMV launch, the workspace is not used).
  * Otherwise all of them go to the tensor-core path: one quantisation launch
  * for every problem's tokens, then one weight-stationary GEMM launch over
@@ -236,7 +240,7 @@ size_t bitlinear_workspace_bytes_path(int64_t M, int64_t N, int64_t K,
  * partial-sum region) lives in one file-scope device array of
  * BITLINEAR_STATIC_SCRATCH_BYTES (16 MiB) inside the library; every GPU that
  * loads the library holds that array until the process exits.
- * The paper has no counterpart of this call; it exists only for such callers.
+ * The method itself has no such call; it exists only for such callers.
  *   x_dev, packed_dev, gamma, y_dev, cuda_stream: as for bitlinear_forward.
  * Limits: M * K rounded up to 256 bytes, plus 2 * (4 * M rounded up to 256)
  * bytes, must fit in BITLINEAR_STATIC_SCRATCH_BYTES; larger problems return

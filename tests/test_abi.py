@@ -50,6 +50,11 @@ def test_workspace_bytes():
     assert bl.bitlinear_workspace_bytes(1, 6912, 2560, bl.PATH_TC) >= 2560 + 8
     assert bl.bitlinear_workspace_bytes(4, 64, 100) == ctypes.c_size_t(-1).value
     assert bl.bitlinear_workspace_bytes(0, 64, 256) == 0
+    # the automatic GEMV path also needs x~ of all tokens in shared memory
+    # (M * K <= 196608): six tokens of K = 32768 fit, of K = 65536 do not
+    assert bl.bitlinear_workspace_bytes(6, 128, 32768) == 0
+    assert bl.bitlinear_workspace_bytes(6, 128, 65536) >= 6 * 65536
+    assert bl.bitlinear_workspace_bytes(7, 128, 256) > 0
 
 
 FAKE = 1 << 20          # a 16-byte-aligned non-null address; never dereferenced
