@@ -13,6 +13,7 @@ Functions:
     absmean_gamma(W)            gamma = max(mean|W|, 1e-5)
     ternarize(W, gamma)         W~ = clip(round(W / gamma), -1, 1)  (int8)
     bf16_to_f32(bits)           exact widening of bf16 bit patterns
+    rmsnorm(x, g, eps)          (x * r) * g per token, r = 1/sqrt(mean x^2 + eps)
     quant_act(x)                (x~ int8 [M][K], beta fp32 [M])
     matmul_i32(xq, Wq)          acc = x~ W~^T in int32
     matmul_i32_pairs(xq, Wq, ms, ns)   acc at sampled (m, n) pairs
@@ -36,6 +37,9 @@ _LIB_PATH = os.path.join(_HERE, "liboracle.so")
 CFLAGS = ["-O2", "-std=c11", "-fPIC", "-shared", "-ffp-contract=off",
           "-fno-fast-math"]
 
+# nn.RMSNorm's default eps for fp32 inputs: the fp32 machine epsilon
+RMSNORM_EPS = float(np.finfo(np.float32).eps)
+
 _lock = threading.Lock()
 _lib = None
 
@@ -56,6 +60,8 @@ def _declare(lib):
     lib.oracle_ternarize.argtypes = [p, c_i64, c_i64, ctypes.c_float, p]
     lib.oracle_bf16_to_f32.restype = None
     lib.oracle_bf16_to_f32.argtypes = [p, c_i64, p]
+    lib.oracle_rmsnorm.restype = None
+    lib.oracle_rmsnorm.argtypes = [p, c_i64, c_i64, p, ctypes.c_float, p]
     lib.oracle_quant_act.restype = None
     lib.oracle_quant_act.argtypes = [p, c_i64, c_i64, p, p]
     lib.oracle_matmul_i32.restype = None
@@ -123,6 +129,18 @@ class Oracle:
         self.lib.oracle_bf16_to_f32(_ptr(bits), bits.size, _ptr(out))
         return out
 
+    def rmsnorm(self, x, g=None, eps=RMSNORM_EPS) -> np.ndarray:
+        """RMS-normalised rows of fp32 x [M][K] with gain g [K] (ones when
+        omitted)."""
+        x = _c(x, np.float32)
+        M, K = x.shape
+        g = np.ones((K,), dtype=np.float32) if g is None else _c(g, np.float32)
+        assert g.shape == (K,)
+        out = np.empty((M, K), dtype=np.float32)
+        self.lib.oracle_rmsnorm(_ptr(x), M, K, _ptr(g), float(np.float32(eps)),
+                                _ptr(out))
+        return out
+
     def quant_act(self, x):
         x = _c(x, np.float32)
         M, K = x.shape
@@ -179,13 +197,17 @@ class Oracle:
             raise ValueError("oracle_pack_codes: K % 128 != 0 or non-ternary")
         return out
 
-    def forward(self, x, W, gamma=None):
+    def forward(self, x, W, gamma=None, norm_gain=None, norm_eps=RMSNORM_EPS):
         """The whole path on the CPU. ``x`` is fp32 [M][K] or bf16 bit
         patterns (uint16); ``W`` is the fp32 latent [N][K]. ``gamma`` may be
-        supplied (e.g. the packer's) instead of recomputed. Returns a dict with
-        gamma, Wq, xq, beta, acc and y (bf16 bit patterns)."""
+        supplied (e.g. the packer's) instead of recomputed. With ``norm_gain``
+        (fp32 [K]) the tokens are RMS-normalised before quantisation (the
+        listing's BitLinear.forward step 1). Returns a dict with gamma, Wq,
+        xq, beta, acc and y (bf16 bit patterns)."""
         x = np.asarray(x)
         xf = self.bf16_to_f32(x) if x.dtype == np.uint16 else _c(x, np.float32)
+        if norm_gain is not None:
+            xf = self.rmsnorm(xf, norm_gain, norm_eps)
         g = self.absmean_gamma(W) if gamma is None else np.float32(gamma)
         Wq = self.ternarize(W, g)
         xq, beta = self.quant_act(xf)

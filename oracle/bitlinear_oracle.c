@@ -17,6 +17,8 @@
  *     beta = max_j |x_j| and x~ = Clip(Round(x * Q_b / beta)), Q_b = 127;
  *   - section "Matrix Multiplication as Pure Integer Addition":
  *     y = (x~ W~^T) * beta * gamma / Q_b, the product being an integer sum;
+ *   - the listing's RMSNorm ahead of the activation quantisation
+ *     (oracle_rmsnorm, for the normalising forms of the path);
  *   - the page's PyTorch listing (WeightQuantFunction.forward,
  *     quantize_activations_int8, BitLinear.forward), which fixes what the
  *     formulas leave open: the epsilon is a clamp(min=1e-5) of gamma and beta,
@@ -88,6 +90,35 @@ void oracle_bf16_to_f32(const uint16_t *in, int64_t n, float *out)
     for (int64_t i = 0; i < n; ++i) {
         uint32_t bits = (uint32_t)in[i] << 16;
         memcpy(&out[i], &bits, sizeof(float));
+    }
+}
+
+/* RMS normalisation of each token row of a row-major [M][K] fp32 matrix,
+ * before its quantisation: the RMSNorm member of the page's BitLinear listing
+ * (step 1 of BitLinear.forward, torch's nn.RMSNorm over in_features), which
+ * the bako.co page's forward flow also puts first ("the input activations
+ * are normalized", section "Architecting the 1-Bit Paradigm").
+ *   out_mk = (x_mk * r_m) * g_k,  r_m = 1 / sqrt(mean_k x_mk^2 + eps)
+ * with g [K] the learned per-channel gain (ones at initialisation).
+ * Readings where the pages are silent: the sum of squares is accumulated in
+ * double (each fp32 square is exact there) and the mean is rounded once to
+ * fp32; sqrt and the division are IEEE fp32, correctly rounded; eps is the
+ * caller's (nn.RMSNorm's default is the machine epsilon of the compute type,
+ * 2^-23 for fp32). */
+void oracle_rmsnorm(const float *x, int64_t M, int64_t K, const float *g,
+                    float eps, float *out)
+{
+    for (int64_t m = 0; m < M; ++m) {
+        const float *row = x + m * K;
+        double ss = 0.0;
+        for (int64_t k = 0; k < K; ++k) {
+            const double v = (double)row[k];
+            ss += v * v;
+        }
+        const float ms = (float)(ss / (double)K);
+        const float r = 1.0f / sqrtf(ms + eps);
+        for (int64_t k = 0; k < K; ++k)
+            out[m * K + k] = (row[k] * r) * g[k];
     }
 }
 

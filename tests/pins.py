@@ -20,7 +20,11 @@ unless stated):
     guide's "Core Architecture" section quotes as about 32% zero entries),
     |x~| <= 127 with the per-token maximum reaching 127, the rounding bound
     |x~ - x*127/beta| <= 1/2, invariance under power-of-two scaling, and the
-    bf16 rounding bound of the output.
+    bf16 rounding bound of the output;
+  * for the RMS normalisation ahead of quantisation (the listing's
+    nn.RMSNorm member of BitLinear): torch's rms_norm in float64 within the
+    fp32 error bound, constant rows in closed form, exact invariance under
+    power-of-two scaling at eps = 0, and the gain applied last.
 """
 from __future__ import annotations
 
@@ -350,6 +354,75 @@ def pin_listing_semantics_torch(orc):
             res["y"], y.view(torch.int16).numpy().view(np.uint16))
 
 
+# ------------------------------------------------------------------- RMSNorm
+#
+# The listing's BitLinear normalises each token with nn.RMSNorm(in_features)
+# before quantising it: out = x / sqrt(mean(x^2) + eps) * g.
+
+def _rms_rows(r):
+    """Four token rows of 384 channels at very different scales (the second
+    so small that eps moves the result), with a few large channels."""
+    x = r.standard_normal((4, 384))
+    x[:, ::97] *= 50.0
+    x *= np.array([1.0, 1e-4, 3e-2, 7.0])[:, None]
+    return x.astype(np.float32)
+
+
+def pin_rmsnorm_vs_torch_f64(orc):
+    """torch.nn.functional.rms_norm in float64 on the same fp32 inputs is
+    within the fp32 error bound of the oracle: six correctly rounded steps
+    (mean, + eps, sqrt, divide, * r, * g), so 8 units of 2^-24 relative."""
+    import torch
+    r = np.random.Generator(np.random.PCG64(81))
+    x = _rms_rows(r)
+    g = r.uniform(0.5, 1.5, size=384).astype(np.float32)
+    for eps in (2.0 ** -23, 1e-6):
+        got = orc.rmsnorm(x, g, eps).astype(np.float64)
+        ref = torch.nn.functional.rms_norm(
+            torch.from_numpy(x.astype(np.float64)), (384,),
+            weight=torch.from_numpy(g.astype(np.float64)), eps=float(np.float32(eps))).numpy()
+        rel = np.abs(got - ref) / np.maximum(np.abs(ref), 1e-30)
+        assert np.all(rel <= 8 * 2.0 ** -24), float(rel.max())
+
+
+def pin_rmsnorm_constant_rows(orc):
+    """A constant row c normalises to c / sqrt(c^2 + eps) (closed form in
+    float64; 1 for |c| >> sqrt(eps), about 0.28 at c = 1e-4 where eps is
+    comparable to c^2), and a zero row stays exactly zero."""
+    eps = 2.0 ** -23
+    cs = np.array([1.0, -3.0, 1e-3, 1e-4, 0.0], dtype=np.float32)
+    x = np.repeat(cs[:, None], 256, axis=1)
+    got = orc.rmsnorm(x, None, eps).astype(np.float64)
+    c = cs.astype(np.float64)
+    ref = c / np.sqrt(c * c + np.float64(np.float32(eps)))
+    for i in range(len(cs)):
+        assert np.all(got[i] == got[i, 0])
+        assert abs(got[i, 0] - ref[i]) <= 4 * 2.0 ** -24 * abs(ref[i]), (cs[i], got[i, 0], ref[i])
+    assert np.all(got[-1] == 0.0)
+    assert abs(got[3, 0] - 0.278) < 1e-3
+
+
+def pin_rmsnorm_pow2_invariance(orc):
+    """With eps = 0 the normalisation is exactly invariant under scaling a
+    row by a power of two: every step scales exactly or cancels."""
+    r = np.random.Generator(np.random.PCG64(82))
+    x = r.standard_normal((3, 256)).astype(np.float32)
+    g = r.uniform(0.5, 1.5, size=256).astype(np.float32)
+    base = orc.rmsnorm(x, g, 0.0)
+    for j in (-20, -3, 5, 30):
+        np.testing.assert_array_equal(orc.rmsnorm(x * np.float32(2.0 ** j), g, 0.0), base)
+
+
+def pin_rmsnorm_gain_applied_last(orc):
+    """The gain multiplies the normalised value, channel by channel:
+    out(x, g)[m, k] is the fp32 product of out(x, 1)[m, k] and g[k]."""
+    r = np.random.Generator(np.random.PCG64(83))
+    x = _rms_rows(r)
+    g = r.uniform(0.25, 4.0, size=384).astype(np.float32)
+    unit = orc.rmsnorm(x, None, 2.0 ** -23)
+    np.testing.assert_array_equal(orc.rmsnorm(x, g, 2.0 ** -23), unit * g[None, :])
+
+
 ALL_PINS = [
     pin_hand_example,
     pin_weight_ties_even,
@@ -371,6 +444,10 @@ ALL_PINS = [
     pin_bf16_rounding_vs_torch,
     pin_rescale_bound,
     pin_listing_semantics_torch,
+    pin_rmsnorm_vs_torch_f64,
+    pin_rmsnorm_constant_rows,
+    pin_rmsnorm_pow2_invariance,
+    pin_rmsnorm_gain_applied_last,
 ]
 
 

@@ -40,6 +40,14 @@ MUTANTS = {
     "pack_word_index": ("16 * w + 4 * j + b;", "16 * w + 4 * b + j;"),
     "pack_row_stride": ("512 * g + 32 * r + 4 * w", "512 * g + 32 * w + 4 * r"),
     "pack_padding_rows": ("(n < N) ? Wq[n * K + k] : 0", "(n < N) ? Wq[n * K + k] : -1"),
+    "rms_drops_eps": ("sqrtf(ms + eps)", "sqrtf(ms)"),
+    "rms_mean_over_k_minus_1": ("ss / (double)K", "ss / (double)(K - 1)"),
+    "rms_forgets_sqrt": ("1.0f / sqrtf(ms + eps)", "1.0f / (ms + eps)"),
+    "rms_multiplies_by_rms": ("1.0f / sqrtf(ms + eps)", "sqrtf(ms + eps)"),
+    "rms_sum_of_abs": ("ss += v * v;", "ss += fabs(v);"),
+    "rms_gain_by_token": ("(row[k] * r) * g[k]", "(row[k] * r) * g[m]"),
+    "rms_gain_first": ("(row[k] * r) * g[k]", "(row[k] * g[k]) * r"),
+    "rms_gain_dropped": ("(row[k] * r) * g[k]", "(row[k] * r)"),
 }
 
 

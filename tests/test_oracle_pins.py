@@ -14,3 +14,24 @@ def orc():
 @pytest.mark.parametrize("pin", pins.ALL_PINS, ids=lambda p: p.__name__)
 def test_pin(orc, pin):
     pin(orc)
+
+
+def test_forward_normalises_before_quantising(orc):
+    """forward(norm_gain=g) quantises the RMS-normalised tokens, both for fp32
+    inputs and for bf16 bit patterns (widened first); without a gain the
+    tokens go to the quantiser as they are."""
+    import numpy as np
+    r = np.random.Generator(np.random.PCG64(84))
+    x = (r.standard_normal((3, 256)) * 4.0).astype(np.float32)
+    W = (r.standard_normal((40, 256)) * 0.02).astype(np.float32)
+    g = r.uniform(0.5, 1.5, size=256).astype(np.float32)
+    res = orc.forward(x, W, norm_gain=g)
+    xq, beta = orc.quant_act(orc.rmsnorm(x, g))
+    np.testing.assert_array_equal(res["xq"], xq)
+    np.testing.assert_array_equal(res["beta"], beta)
+    np.testing.assert_array_equal(res["y"], orc.rescale_bf16(orc.matmul_i32(xq, res["Wq"]),
+                                                            beta, res["gamma"]))
+    bits = (x.view(np.uint32) >> 16).astype(np.uint16)
+    res16 = orc.forward(bits, W, norm_gain=g)
+    np.testing.assert_array_equal(res16["xq"], orc.quant_act(orc.rmsnorm(orc.bf16_to_f32(bits), g))[0])
+    np.testing.assert_array_equal(orc.forward(x, W)["xq"], orc.quant_act(x)[0])
