@@ -320,10 +320,11 @@ def time_e2e(dist, wl, steps: int):
     return dist.max(start.elapsed_time(end))
 
 
-def bench_prefill(bl, device, reps: int = 20):
+def bench_prefill(bl, device, reps: int = 20, norm: bool = False):
     """Prefill step (M = 2048: up and down, quantisation kernel + tcgen05
-    GEMM each), inputs rotating over copies larger than L2. Returns
-    (ms per step, int8 ops per step)."""
+    GEMM each), inputs rotating over copies larger than L2; with `norm` the
+    tokens are RMS-normalised in the quantisation kernel
+    (bitlinear_forward_rmsnorm). Returns (ms per step, int8 ops per step)."""
     import torch
     probs = workloads.prefill_2b(2048).problems
     mats = []
@@ -336,13 +337,18 @@ def bench_prefill(bl, device, reps: int = 20):
                      "packed": [dp] + [dp.clone() for _ in range(PREFILL_COPIES - 1)],
                      "x": [x] + [x.clone() for _ in range(PREFILL_COPIES - 1)],
                      "y": torch.empty((p.M, p.N), dtype=torch.bfloat16, device=device),
-                     "ws": torch.empty((ws_bytes,), dtype=torch.uint8, device=device)})
+                     "ws": torch.empty((ws_bytes,), dtype=torch.uint8, device=device),
+                     "g": torch.from_numpy(workloads.norm_gains(p.K, p.w_seed + 50)).to(device)})
 
     def step(i):
         j = i % PREFILL_COPIES
         for m in mats:
-            bl.bitlinear_forward(m["x"][j], m["packed"][j], m["gamma"], m["p"].N, y=m["y"],
-                                 workspace=m["ws"])
+            if norm:
+                bl.bitlinear_forward_rmsnorm(m["x"][j], m["packed"][j], m["gamma"], m["p"].N,
+                                             m["g"], y=m["y"], workspace=m["ws"])
+            else:
+                bl.bitlinear_forward(m["x"][j], m["packed"][j], m["gamma"], m["p"].N,
+                                     y=m["y"], workspace=m["ws"])
 
     for i in range(3):
         step(i)
@@ -350,7 +356,7 @@ def bench_prefill(bl, device, reps: int = 20):
     g.replay()
     torch.cuda.synchronize()
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    torch.cuda.nvtx.range_push("prefill_timed")
+    torch.cuda.nvtx.range_push("rmsnorm_prefill_timed" if norm else "prefill_timed")
     start.record()
     for _ in range(reps):
         g.replay()
@@ -382,6 +388,25 @@ def time_graph(fn, reps: int, nvtx: str | None = None) -> float:
     torch.cuda.synchronize()
     del g
     return start.elapsed_time(end) / reps
+
+
+def bench_rmsnorm_decode(bl, wl, reps: int = 200) -> float:
+    """The decode step's two projections (M = 1) with the tokens
+    RMS-normalised in the GEMV prologue, one bitlinear_forward_rmsnorm launch
+    per projection, over the same rotating weight copies as the headline
+    step. Returns ms per step."""
+    import torch
+    gains = [torch.from_numpy(workloads.norm_gains(m["p"].K, m["p"].w_seed + 50)).to(
+        m["x"][0].device) for m in wl.mats]
+
+    def steps():
+        for j in range(ROTATE):
+            for m, g in zip(wl.mats, gains):
+                bl.bitlinear_forward_rmsnorm(m["x"][j], m["packed"][j], m["gamma"], m["p"].N,
+                                             g, y=m["y"][j])
+    steps()
+    torch.cuda.synchronize()
+    return time_graph(steps, reps, nvtx="rmsnorm_decode_timed") / ROTATE
 
 
 def bench_layer_set(bl, device, batches=(1, 8, 64), reps: int = 10):
@@ -521,6 +546,9 @@ def run_ours(args, dist):
     pre_ms, pre_ops = bench_prefill(bl, device)
     pre_tops = pre_ops / (pre_ms * 1e-3) / 1e12
     int8_peak = peaks["bf16_tflops"] * INT8_PER_BF16
+    norm_dec_ms = bench_rmsnorm_decode(bl, wl)
+    norm_pre_ms, _ = bench_prefill(bl, device, norm=True)
+    norm_pre_tops = pre_ops / (norm_pre_ms * 1e-3) / 1e12
 
     out = {
         "metric": METRIC,
@@ -565,6 +593,17 @@ def run_ours(args, dist):
                          "ms_per_step": pre_ms,
                          "peak": int8_peak, "peak_note": "measured bf16 burst x 2 (nominal int8/bf16)",
                          "frac": round(pre_tops / int8_peak, 4)},
+        "rmsnorm_forward": {
+            "workload": "the same decode and prefill steps with every token RMS-normalised "
+                        "(gains [K]) inside the quantisation pass (bitlinear_forward_rmsnorm, "
+                        "one launch per projection at decode)",
+            "decode_m1": {"value": round(wl.packed_bytes_per_step * dist.world
+                                         / (norm_dec_ms * 1e-3) / 1e9, 2),
+                          "unit": UNIT, "ms_per_step": norm_dec_ms,
+                          "plain_ms_per_step": ms_sep / args.steps},
+            "prefill_m2048": {"value": round(norm_pre_tops, 1), "unit": "TOPS (int8)",
+                              "ms_per_step": norm_pre_ms, "plain_ms_per_step": pre_ms,
+                              "frac": round(norm_pre_tops / int8_peak, 4)}},
     }
     if not args.no_extra:
         out["layer_set"] = {

@@ -170,6 +170,33 @@ int bitlinear_forward_ex(const void *x_dev, bitlinear_dtype xdt, int64_t M,
                          int32_t *acc_dev_or_null, int8_t *xq_dev_or_null,
                          float *beta_dev_or_null, int path);
 
+/* y = BitLinear(RMSNorm(x)): the tokens are RMS-normalised before their
+ * absmax quantisation, as the page's BitLinear listing does with its
+ * nn.RMSNorm(in_features) member (step 1 of BitLinear.forward), fused into the
+ * quantisation pass of either path (the GEMV prologue or the quantisation
+ * kernel ahead of the tensor-core GEMM). Per token m:
+ *   r_m = 1 / sqrt(mean_k x_mk^2 + norm_eps),  x'_mk = (x_mk * r_m) * g_k
+ * and x' takes the place of x in bitlinear_forward. The sum of squares is
+ * accumulated in double and the mean rounded once to fp32; the square root,
+ * the division and both products are IEEE fp32.
+ *   norm_gain_dev [in] [K] fp32 gains g, device memory, 16-byte aligned
+ *                      (may be NULL only when M = 0)
+ *   norm_eps      [in] finite and > 0 (nn.RMSNorm's default for fp32 is the
+ *                      fp32 machine epsilon, 2^-23)
+ *   path          [in] a bitlinear_path, as for bitlinear_forward_ex
+ * Every other argument, the workspace size and the dispatch are those of
+ * bitlinear_forward_ex; xq_dev_or_null and beta_dev_or_null return the
+ * quantised normalised tokens and their beta. Returns BITLINEAR_ERR_ARG for a
+ * missing gain or a bad eps, BITLINEAR_ERR_ALIGN for a misaligned gain. */
+int bitlinear_forward_rmsnorm(const void *x_dev, bitlinear_dtype xdt, int64_t M,
+                              int64_t K, const float *norm_gain_dev,
+                              float norm_eps, const void *packed_dev,
+                              float gamma, int64_t N, void *y_dev,
+                              void *workspace_dev, size_t workspace_bytes,
+                              void *cuda_stream, int32_t *acc_dev_or_null,
+                              int8_t *xq_dev_or_null, float *beta_dev_or_null,
+                              int path);
+
 /* One problem of bitlinear_forward_grouped. */
 typedef struct {
     const void *x_dev;       /* [M][K] activations (the group's xdt) */

@@ -35,6 +35,10 @@ PATH_AUTO = 0
 PATH_GEMV = 1
 PATH_TC = 2
 
+# default eps of bitlinear_forward_rmsnorm: nn.RMSNorm's default for fp32
+# inputs, the fp32 machine epsilon
+RMSNORM_EPS = 2.0 ** -23
+
 # Every symbol include/bitlinear.h declares.
 EXPORTS = (
     "bitlinear_packed_bytes",
@@ -44,6 +48,7 @@ EXPORTS = (
     "bitlinear_workspace_bytes_path",
     "bitlinear_forward",
     "bitlinear_forward_ex",
+    "bitlinear_forward_rmsnorm",
     "bitlinear_get_fault",
     "bitlinear_status_string",
     "bitlinear_int8_gemm",
@@ -94,6 +99,9 @@ def lib() -> ctypes.CDLL:
         L.bitlinear_forward.argtypes = fwd
         L.bitlinear_forward_ex.restype = ctypes.c_int
         L.bitlinear_forward_ex.argtypes = fwd + [ctypes.c_int]
+        L.bitlinear_forward_rmsnorm.restype = ctypes.c_int
+        L.bitlinear_forward_rmsnorm.argtypes = (fwd[:4] + [p, ctypes.c_float] + fwd[4:] +
+                                                [ctypes.c_int])
         L.bitlinear_forward_inject_timeout.restype = ctypes.c_int
         L.bitlinear_forward_inject_timeout.argtypes = fwd[:11] + [ctypes.c_int]
         L.bitlinear_forward_noalloc.restype = ctypes.c_int
@@ -264,6 +272,35 @@ def bitlinear_forward(x, packed, gamma: float, N: int, y=None, workspace=None,
     else:
         rc = lib().bitlinear_forward_ex(*args, path)
     _check(rc, "bitlinear_forward")
+    return y
+
+
+def bitlinear_forward_rmsnorm(x, packed, gamma: float, N: int, norm_gain,
+                              eps: float = RMSNORM_EPS, y=None, workspace=None, stream=None,
+                              acc=None, xq=None, beta=None, path: int = PATH_AUTO):
+    """y (bf16 [M][N]) = BitLinear(RMSNorm(x)): every token is normalised as
+    (x * r) * g with r = 1 / sqrt(mean(x^2) + eps) and the fp32 gains
+    ``norm_gain`` [K] before its quantisation, in the same launch. Other
+    arguments as for ``bitlinear_forward``; ``xq``/``beta`` return the
+    quantised normalised tokens."""
+    a = _Args()
+    import torch
+    M, K = x.shape
+    if y is None:
+        y = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
+    need = bitlinear_workspace_bytes(M, N, K, path)
+    if need == ctypes.c_size_t(-1).value:
+        raise BitLinearError(BITLINEAR_ERR_SHAPE, "bitlinear_workspace_bytes")
+    if workspace is None and need > 0:
+        workspace = torch.empty((need,), dtype=torch.uint8, device=x.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    rc = lib().bitlinear_forward_rmsnorm(
+        a.ptr(x, "x"), _xdt(x), M, K, a.ptr(norm_gain, "norm_gain", torch.float32, (K,)),
+        float(eps), a.packed(packed, N, K), float(gamma), N,
+        a.ptr(y, "y", torch.bfloat16, (M, N)), a.ptr(workspace, "workspace"), ws_bytes,
+        _stream(stream), a.ptr(acc, "acc", torch.int32, (M, N)),
+        a.ptr(xq, "xq", torch.int8, (M, K)), a.ptr(beta, "beta", torch.float32, (M,)), path)
+    _check(rc, "bitlinear_forward_rmsnorm")
     return y
 
 

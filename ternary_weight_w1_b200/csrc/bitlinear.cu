@@ -9,6 +9,7 @@
 
 #include <algorithm>
 #include <atomic>
+#include <cfloat>
 #include <climits>
 #include <cstdint>
 #include <cstdlib>
@@ -208,21 +209,25 @@ int launch_status(cudaError_t e)
 
 template <bool BF16, int CACHE, int WPR>
 cudaError_t launch_qa(const void *x, int M, int K, int8_t *xq, float *beta, int *rowsum,
-                      cudaStream_t st, int *clear, int n_clear)
+                      cudaStream_t st, int *clear, int n_clear, const float *gain, float eps)
 {
     constexpr int rpb = qa::rows_per_block<WPR>();
     const dim3 grid((M + rpb - 1) / rpb);
-    return launch(qa::quant_act_kernel<BF16, CACHE, WPR>, grid, dim3(qa::THREADS), 0, st, x, M,
-                  K, xq, beta, rowsum, clear, n_clear);
+    if (gain != nullptr)
+        return launch(qa::quant_act_kernel<BF16, CACHE, WPR, true>, grid, dim3(qa::THREADS), 0,
+                      st, x, M, K, xq, beta, rowsum, clear, n_clear, gain, eps);
+    return launch(qa::quant_act_kernel<BF16, CACHE, WPR, false>, grid, dim3(qa::THREADS), 0, st,
+                  x, M, K, xq, beta, rowsum, clear, n_clear, gain, eps);
 }
 
 // Register cache per lane and warps per row by row length: every lane holds
 // its whole share of a row in registers up to 16384 bf16 (8192 fp32)
 // elements per row, so a row is read from memory once and small batches are
 // not held up by dependent re-reads; longer rows take eight warps and
-// re-read the rest.
+// re-read the rest. A non-null gain RMS-normalises each row first.
 int launch_quant_act(const void *x, bitlinear_dtype xdt, int M, int K, int8_t *xq, float *beta,
-                     int *rowsum, cudaStream_t st, int *clear = nullptr, int n_clear = 0)
+                     int *rowsum, cudaStream_t st, int *clear = nullptr, int n_clear = 0,
+                     const float *gain = nullptr, float eps = 0.0f)
 {
     if (M == 0)
         return BITLINEAR_OK;
@@ -230,50 +235,53 @@ int launch_quant_act(const void *x, bitlinear_dtype xdt, int M, int K, int8_t *x
     cudaError_t e;
     if (xdt == BITLINEAR_BF16) {
         if (nvec <= 32 * 4)
-            e = launch_qa<true, 4, 1>(x, M, K, xq, beta, rowsum, st, clear, n_clear);
+            e = launch_qa<true, 4, 1>(x, M, K, xq, beta, rowsum, st, clear, n_clear, gain, eps);
         else if (nvec <= 32 * 8)
-            e = launch_qa<true, 8, 1>(x, M, K, xq, beta, rowsum, st, clear, n_clear);
+            e = launch_qa<true, 8, 1>(x, M, K, xq, beta, rowsum, st, clear, n_clear, gain, eps);
         else if (nvec <= 32 * 16)
-            e = launch_qa<true, 16, 1>(x, M, K, xq, beta, rowsum, st, clear, n_clear);
+            e = launch_qa<true, 16, 1>(x, M, K, xq, beta, rowsum, st, clear, n_clear, gain, eps);
         else if (nvec <= 64 * 16)
-            e = launch_qa<true, 16, 2>(x, M, K, xq, beta, rowsum, st, clear, n_clear);
+            e = launch_qa<true, 16, 2>(x, M, K, xq, beta, rowsum, st, clear, n_clear, gain, eps);
         else if (nvec <= 128 * 16)
-            e = launch_qa<true, 16, 4>(x, M, K, xq, beta, rowsum, st, clear, n_clear);
+            e = launch_qa<true, 16, 4>(x, M, K, xq, beta, rowsum, st, clear, n_clear, gain, eps);
         else
-            e = launch_qa<true, 16, 8>(x, M, K, xq, beta, rowsum, st, clear, n_clear);
+            e = launch_qa<true, 16, 8>(x, M, K, xq, beta, rowsum, st, clear, n_clear, gain, eps);
     } else {
         if (nvec <= 32 * 4)
-            e = launch_qa<false, 4, 1>(x, M, K, xq, beta, rowsum, st, clear, n_clear);
+            e = launch_qa<false, 4, 1>(x, M, K, xq, beta, rowsum, st, clear, n_clear, gain, eps);
         else if (nvec <= 32 * 8)
-            e = launch_qa<false, 8, 1>(x, M, K, xq, beta, rowsum, st, clear, n_clear);
+            e = launch_qa<false, 8, 1>(x, M, K, xq, beta, rowsum, st, clear, n_clear, gain, eps);
         else if (nvec <= 64 * 8)
-            e = launch_qa<false, 8, 2>(x, M, K, xq, beta, rowsum, st, clear, n_clear);
+            e = launch_qa<false, 8, 2>(x, M, K, xq, beta, rowsum, st, clear, n_clear, gain, eps);
         else if (nvec <= 128 * 8)
-            e = launch_qa<false, 8, 4>(x, M, K, xq, beta, rowsum, st, clear, n_clear);
+            e = launch_qa<false, 8, 4>(x, M, K, xq, beta, rowsum, st, clear, n_clear, gain, eps);
         else
-            e = launch_qa<false, 8, 8>(x, M, K, xq, beta, rowsum, st, clear, n_clear);
+            e = launch_qa<false, 8, 8>(x, M, K, xq, beta, rowsum, st, clear, n_clear, gain, eps);
     }
     return launch_status(e);
 }
 
 // ------------------------------------------------------------------- GEMV
 
-template <int MT, bool BF16>
+template <int MT, bool BF16, bool NORM>
 int launch_gemv_t(const gemv::Params &p, int grid, int smem, int dev, cudaStream_t st)
 {
-    cudaError_t e = allow_smem<gemv::gemv_kernel<MT, BF16>>(dev, smem);
+    cudaError_t e = allow_smem<gemv::gemv_kernel<MT, BF16, NORM>>(dev, smem);
     if (e != cudaSuccess)
         return launch_status(e);
-    e = launch(gemv::gemv_kernel<MT, BF16>, dim3(grid), dim3(gemv::THREADS), smem, st, p);
+    e = launch(gemv::gemv_kernel<MT, BF16, NORM>, dim3(grid), dim3(gemv::THREADS), smem, st, p);
     return launch_status(e);
 }
 
 template <int MT>
-int launch_gemv_mt(const gemv::Params &p, bool bf16, int grid, int smem, int dev,
+int launch_gemv_mt(const gemv::Params &p, bool bf16, bool norm, int grid, int smem, int dev,
                    cudaStream_t st)
 {
-    return bf16 ? launch_gemv_t<MT, true>(p, grid, smem, dev, st)
-                : launch_gemv_t<MT, false>(p, grid, smem, dev, st);
+    if (norm)
+        return bf16 ? launch_gemv_t<MT, true, true>(p, grid, smem, dev, st)
+                    : launch_gemv_t<MT, false, true>(p, grid, smem, dev, st);
+    return bf16 ? launch_gemv_t<MT, true, false>(p, grid, smem, dev, st)
+                : launch_gemv_t<MT, false, false>(p, grid, smem, dev, st);
 }
 
 // One problem of a GEMV launch, as the host sees it.
@@ -286,16 +294,23 @@ struct GemvJob {
     int32_t *acc;
     int8_t *xq;
     float *beta;
+    const float *norm_gain;     // non-null: RMS-normalise the tokens first
+    float norm_eps;
 };
 
 // Launches the GEMV kernel over one or more independent problems. Every CTA
 // owns whole 16-row blocks of one problem. A single problem is split over at
 // most two CTAs per SM with the same number of blocks per CTA; a group is
 // split so that the CTAs of every problem stream about the same number of
-// bytes, with at most three CTAs per SM (all resident at once).
+// bytes, with at most three CTAs per SM (all resident at once). Either every
+// problem of the launch is RMS-normalised or none is.
 int launch_gemv(const GemvJob *jobs, int count, bitlinear_dtype xdt, const DeviceInfo &dev,
                 cudaStream_t st)
 {
+    const bool norm = jobs[0].norm_gain != nullptr;
+    for (int i = 1; i < count; ++i)
+        if ((jobs[i].norm_gain != nullptr) != norm)
+            return BITLINEAR_ERR_ARG;
     int Mmax = 1;
     double total_bytes = 0.0;
     for (int i = 0; i < count; ++i) {
@@ -347,11 +362,11 @@ int launch_gemv(const GemvJob *jobs, int count, bitlinear_dtype xdt, const Devic
     // Ring depth: the whole share when it is small (room for the next
     // kernel's blocks on the same SM under programmatic launch), else as deep
     // as a 110 KiB block allows.
-    const int fixed = gemv::smem_bytes(MT, xq_cap, acc_cap, 0);
+    const int fixed = gemv::smem_bytes(MT, xq_cap, acc_cap, 0, norm);
     const int budget = stages > 12 ? 110 * 1024 : 56 * 1024;
     int slots = (budget - fixed) / gemv::STAGE;
     slots = std::max(2, std::min({slots, stages, gemv::MAX_SLOTS}));
-    const int smem = gemv::smem_bytes(MT, xq_cap, acc_cap, slots);
+    const int smem = gemv::smem_bytes(MT, xq_cap, acc_cap, slots, norm);
     if (smem > dev.max_smem_optin)
         return BITLINEAR_ERR_SHAPE;
     gemv::Params p = {};
@@ -361,7 +376,7 @@ int launch_gemv(const GemvJob *jobs, int count, bitlinear_dtype xdt, const Devic
         const uint64_t kg = static_cast<uint64_t>(j.K / 128);
         p.prob[i] = gemv::Problem{j.x, static_cast<const uint8_t *>(j.packed),
                                   static_cast<uint16_t *>(j.y), j.acc, j.xq, j.beta, j.M, j.K,
-                                  j.N, j.gamma, q[i], begin,
+                                  j.N, j.gamma, j.norm_gain, j.norm_eps, q[i], begin,
                                   ((uint64_t(1) << 32) + kg - 1) / kg};
         begin += ctas[i];
     }
@@ -372,11 +387,11 @@ int launch_gemv(const GemvJob *jobs, int count, bitlinear_dtype xdt, const Devic
     p.wait_limit_ns = kWaitLimitNs;
     const bool bf16 = xdt == BITLINEAR_BF16;
     switch (MT) {
-    case 1: return launch_gemv_mt<1>(p, bf16, grid, smem, dev.id, st);
-    case 2: return launch_gemv_mt<2>(p, bf16, grid, smem, dev.id, st);
-    case 4: return launch_gemv_mt<4>(p, bf16, grid, smem, dev.id, st);
-    case 8: return launch_gemv_mt<8>(p, bf16, grid, smem, dev.id, st);
-    default: return launch_gemv_mt<16>(p, bf16, grid, smem, dev.id, st);
+    case 1: return launch_gemv_mt<1>(p, bf16, norm, grid, smem, dev.id, st);
+    case 2: return launch_gemv_mt<2>(p, bf16, norm, grid, smem, dev.id, st);
+    case 4: return launch_gemv_mt<4>(p, bf16, norm, grid, smem, dev.id, st);
+    case 8: return launch_gemv_mt<8>(p, bf16, norm, grid, smem, dev.id, st);
+    default: return launch_gemv_mt<16>(p, bf16, norm, grid, smem, dev.id, st);
     }
 }
 
@@ -421,6 +436,8 @@ struct TcJob {
     float gamma;
     void *y;
     int32_t *acc;
+    const float *norm_gain;     // non-null: RMS-normalise the tokens first (single problem)
+    float norm_eps;
 };
 
 size_t tc_group_bytes(const TcJob *jobs, int n, bool split)
@@ -521,6 +538,10 @@ int run_tc_group(const TcJob *jobs, int n, bitlinear_dtype xdt, void *ws, size_t
     const size_t need = tc_group_bytes(jobs, n, split);
     if (ws == nullptr || ws_bytes < need)
         return BITLINEAR_ERR_WORKSPACE;
+    if (n > 1)
+        for (int i = 0; i < n; ++i)
+            if (jobs[i].norm_gain != nullptr)     // the grouped quantiser does not normalise
+                return BITLINEAR_ERR_ARG;
     if (!aligned(ws, 256))
         return BITLINEAR_ERR_ALIGN;
     int max_M = 0;
@@ -583,7 +604,8 @@ int run_tc_group(const TcJob *jobs, int n, bitlinear_dtype xdt, void *ws, size_t
         p.flags = flags;
     }
     int rc = (n == 1) ? launch_quant_act(jobs[0].x, xdt, jobs[0].M, jobs[0].K, xq[0], beta[0],
-                                         rowsum[0], st, flags, split ? 4 * grid : 0)
+                                         rowsum[0], st, flags, split ? 4 * grid : 0,
+                                         jobs[0].norm_gain, jobs[0].norm_eps)
                       : launch_quant_group(jobs, n, xdt, xq, beta, rowsum, st, flags,
                                            split ? 4 * grid : 0);
     if (rc != BITLINEAR_OK)
@@ -624,9 +646,10 @@ int run_tc_group(const TcJob *jobs, int n, bitlinear_dtype xdt, void *ws, size_t
 int run_tc_path(const void *x, bitlinear_dtype xdt, int M, int K, const void *packed,
                 float gamma, int N, void *y, void *ws, size_t ws_bytes, int32_t *acc,
                 int8_t *xq_dbg, float *beta_dbg, const DeviceInfo &dev, cudaStream_t st,
-                int inject_timeout_us, bool split)
+                int inject_timeout_us, bool split, const float *norm_gain = nullptr,
+                float norm_eps = 0.0f)
 {
-    const TcJob job{x, M, K, N, packed, gamma, y, acc};
+    const TcJob job{x, M, K, N, packed, gamma, y, acc, norm_gain, norm_eps};
     return run_tc_group(&job, 1, xdt, ws, ws_bytes, xq_dbg, beta_dbg, dev, st, inject_timeout_us,
                         split);
 }
@@ -663,7 +686,8 @@ int choose_path(int64_t M, int64_t K, int path)
 
 int forward_impl(const void *x, bitlinear_dtype xdt, int64_t M, int64_t K, const void *packed,
                  float gamma, int64_t N, void *y, void *ws, size_t ws_bytes, void *stream,
-                 int32_t *acc, int8_t *xq, float *beta, int path, int inject_timeout_us)
+                 int32_t *acc, int8_t *xq, float *beta, int path, int inject_timeout_us,
+                 const float *norm_gain = nullptr, float norm_eps = 0.0f)
 {
     int rc = check_forward_args(x, xdt, M, K, packed, N, y, acc, xq, beta);
     if (rc != BITLINEAR_OK)
@@ -682,12 +706,12 @@ int forward_impl(const void *x, bitlinear_dtype xdt, int64_t M, int64_t K, const
         if (!gemv_fits(M, K))
             return BITLINEAR_ERR_SHAPE;
         const GemvJob job{x,      static_cast<int>(M), static_cast<int>(K), static_cast<int>(N),
-                          packed, gamma, y, acc, xq, beta};
+                          packed, gamma, y, acc, xq, beta, norm_gain, norm_eps};
         return launch_gemv(&job, 1, xdt, *dev, st);
     }
     return run_tc_path(x, xdt, static_cast<int>(M), static_cast<int>(K), packed, gamma,
                        static_cast<int>(N), y, ws, ws_bytes, acc, xq, beta, *dev, st,
-                       inject_timeout_us, true);
+                       inject_timeout_us, true, norm_gain, norm_eps);
 }
 
 }  // namespace
@@ -763,6 +787,27 @@ extern "C" int bitlinear_forward_ex(const void *x_dev, bitlinear_dtype xdt, int6
     return forward_impl(x_dev, xdt, M, K, packed_dev, gamma, N, y_dev, workspace_dev,
                         workspace_bytes, cuda_stream, acc_dev_or_null, xq_dev_or_null,
                         beta_dev_or_null, path, 0);
+}
+
+extern "C" int bitlinear_forward_rmsnorm(const void *x_dev, bitlinear_dtype xdt, int64_t M,
+                                         int64_t K, const float *norm_gain_dev, float norm_eps,
+                                         const void *packed_dev, float gamma, int64_t N,
+                                         void *y_dev, void *workspace_dev, size_t workspace_bytes,
+                                         void *cuda_stream, int32_t *acc_dev_or_null,
+                                         int8_t *xq_dev_or_null, float *beta_dev_or_null,
+                                         int path)
+{
+    if (M > 0 && norm_gain_dev == nullptr)
+        return BITLINEAR_ERR_ARG;
+    if (!(norm_eps > 0.0f) || !(norm_eps <= FLT_MAX))
+        return BITLINEAR_ERR_ARG;
+    if (!aligned(norm_gain_dev, 16))
+        return BITLINEAR_ERR_ALIGN;
+    // M = 0 stays a no-op, which needs no gains
+    const float *gain = M > 0 ? norm_gain_dev : nullptr;
+    return forward_impl(x_dev, xdt, M, K, packed_dev, gamma, N, y_dev, workspace_dev,
+                        workspace_bytes, cuda_stream, acc_dev_or_null, xq_dev_or_null,
+                        beta_dev_or_null, path, 0, gain, norm_eps);
 }
 
 extern "C" int bitlinear_forward_grouped(const bitlinear_problem *problems, int count,

@@ -407,6 +407,32 @@ struct Vec8 {
     }
 };
 
+// RMS normalisation of one activation: (x * r) * g, two correctly rounded
+// fp32 products in the order torch's RMSNorm applies them (r = 1 / sqrt(mean
+// x^2 + eps) of the token, g the channel's gain).
+__device__ __forceinline__ float norm1(float x, float r, float g)
+{
+    return __fmul_rn(__fmul_rn(x, r), g);
+}
+
+// r = 1 / sqrt(ss / K + eps) from a token's sum of squares in double: the
+// mean rounded once to fp32, then IEEE fp32 add, square root and division.
+__device__ __forceinline__ float rms_scale(double ss, int K, float eps)
+{
+    const float ms = __double2float_rn(__ddiv_rn(ss, static_cast<double>(K)));
+    return __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(ms, eps)));
+}
+
+// Sum of a double over the warp (xor butterfly: every lane ends with the
+// same bits, as each step adds two commuted copies of the same partial sums).
+__device__ __forceinline__ double warp_sum_f64(double v)
+{
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1)
+        v = __dadd_rn(v, __shfl_xor_sync(0xffffffffu, v, o));
+    return v;
+}
+
 // x~ = clamp(round_half_even(x * scale), -128, 127) as one byte.
 __device__ __forceinline__ int quant1(float x, float scale)
 {

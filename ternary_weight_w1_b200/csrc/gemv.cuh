@@ -33,6 +33,13 @@
 // change the result); pieces are therefore independent, and each warp works
 // on all of its pieces of a ring slot at once, without branches.
 //
+// RMS normalisation (NORM launches). The listing's BitLinear normalises each
+// token with its nn.RMSNorm member before quantising it; here that is one more
+// prologue pass. Each thread sums the squares of its activations in double
+// (exact products), the warps' sums go to shared memory and every thread adds
+// them in the same order, so all CTAs derive the same r = 1 / sqrt(mean +
+// eps); the absmax and quantisation passes then work on (x * r) * g.
+//
 // Every mbarrier wait is bounded; a wait that runs out records the fault word
 // and lets every warp return (the producer first waits for its own copies).
 #pragma once
@@ -65,6 +72,8 @@ struct Problem {
     float *beta_dbg;
     int M, K, N;
     float gamma;
+    const float *norm_gain; // [K] RMS-normalisation gains (NORM launches only)
+    float norm_eps;         // eps of the normalisation (NORM launches only)
     int blocks_per_cta;     // row blocks of 16 rows owned by one CTA
     int cta_begin;          // this problem's first CTA in the grid
     uint64_t kg_magic;      // ceil(2^32 / (K / 128)): i / KG == (i * kg_magic) >> 32
@@ -81,9 +90,21 @@ struct Params {
     uint64_t wait_limit_ns;
 };
 
-__host__ __device__ constexpr int smem_bytes(int MT, int xq_cap, int acc_cap, int slots)
+__host__ __device__ constexpr int smem_bytes(int MT, int xq_cap, int acc_cap, int slots,
+                                             bool norm = false)
 {
-    return slots * STAGE + BAR_BYTES + xq_cap + acc_cap * 4 + MT * 4 + 2 * MT * CWARPS * 4;
+    return slots * STAGE + BAR_BYTES + xq_cap + acc_cap * 4 + (norm ? MT * CWARPS * 8 : 0) +
+           MT * 4 + 2 * MT * CWARPS * 4;
+}
+
+// r of token m from the warps' partial sums of squares, added in warp order.
+__device__ __forceinline__ float row_rms_scale(const double *red_d, int m, int K, float eps)
+{
+    double ss = red_d[m * CWARPS];
+#pragma unroll
+    for (int w = 1; w < CWARPS; ++w)
+        ss = __dadd_rn(ss, red_d[m * CWARPS + w]);
+    return rms_scale(ss, K, eps);
 }
 
 __device__ __forceinline__ void compute_sync()
@@ -93,7 +114,7 @@ __device__ __forceinline__ void compute_sync()
 
 // Three blocks per SM fit the register file (two of this grid and, under
 // programmatic dependent launch, one of the next).
-template <int MT, bool BF16>
+template <int MT, bool BF16, bool NORM>
 __global__ void __launch_bounds__(THREADS, 3)
 gemv_kernel(const __grid_constant__ Params p)
 {
@@ -124,7 +145,10 @@ gemv_kernel(const __grid_constant__ Params p)
         reinterpret_cast<volatile int *>(smem + slots * STAGE + 2 * MAX_SLOTS * 8);
     uint8_t *xq_sm = smem + slots * STAGE + BAR_BYTES;
     int *acc_sm = reinterpret_cast<int *>(xq_sm + p.xq_cap);
-    float *beta_sm = reinterpret_cast<float *>(acc_sm + p.acc_cap);
+    // [MT][CWARPS] partial sums of squares (NORM only; 8-byte aligned: every
+    // region before it is a multiple of 8 bytes)
+    double *red_d = reinterpret_cast<double *>(acc_sm + p.acc_cap);
+    float *beta_sm = reinterpret_cast<float *>(red_d + (NORM ? MT * CWARPS : 0));
     uint32_t *red_u = reinterpret_cast<uint32_t *>(beta_sm + MT);   // [MT][CWARPS] absmax
     int *red_i = reinterpret_cast<int *>(red_u + MT * CWARPS);      // [MT][CWARPS] sum x~
 
@@ -186,26 +210,76 @@ gemv_kernel(const __grid_constant__ Params p)
     Vec8<BF16> xc[XCACHE];
     const int e0 = ctid * 8;
     const int estride = CTHREADS * 8;
+    if constexpr (NORM) {
+        // sums of squares per token (the first token's cache is filled here)
+        for (int m = 0; m < M; ++m) {
+            const void *row = static_cast<const char *>(P.x) +
+                              static_cast<size_t>(m) * K * (BF16 ? 2 : 4);
+            double ss = 0.0;
+#pragma unroll
+            for (int c = 0; c < XCACHE; ++c) {
+                const int e = e0 + c * estride;
+                if (m == 0 && e < K) {
+                    xc[c].load(row, e);
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        const double d = xc[c].get(i);
+                        ss = __fma_rn(d, d, ss);
+                    }
+                }
+            }
+            for (int e = (m == 0 ? e0 + XCACHE * estride : e0); e < K; e += estride) {
+                float v[8];
+                load8<BF16>(row, e, v);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const double d = v[i];
+                    ss = __fma_rn(d, d, ss);
+                }
+            }
+            ss = warp_sum_f64(ss);
+            if (lane == 0)
+                red_d[m * CWARPS + warp] = ss;
+        }
+        compute_sync();
+    }
     for (int m = 0; m < M; ++m) {
         const void *row = static_cast<const char *>(P.x) +
                           static_cast<size_t>(m) * K * (BF16 ? 2 : 4);
+        float r = 1.0f;
+        if constexpr (NORM)
+            r = row_rms_scale(red_d, m, K, P.norm_eps);
         float amax = 0.0f;
 #pragma unroll
         for (int c = 0; c < XCACHE; ++c) {
             const int e = e0 + c * estride;
             if (m == 0 && e < K) {
-                xc[c].load(row, e);
+                float g[8];
+                if constexpr (NORM)
+                    load8<false>(P.norm_gain, e, g);
+                else
+                    xc[c].load(row, e);
 #pragma unroll
-                for (int i = 0; i < 8; ++i)
-                    amax = fmaxf(amax, fabsf(xc[c].get(i)));
+                for (int i = 0; i < 8; ++i) {
+                    float a = xc[c].get(i);
+                    if constexpr (NORM)
+                        a = norm1(a, r, g[i]);
+                    amax = fmaxf(amax, fabsf(a));
+                }
             }
         }
         for (int e = (m == 0 ? e0 + XCACHE * estride : e0); e < K; e += estride) {
-            float v[8];
+            float v[8], g[8];
             load8<BF16>(row, e, v);
+            if constexpr (NORM)
+                load8<false>(P.norm_gain, e, g);
 #pragma unroll
-            for (int i = 0; i < 8; ++i)
-                amax = fmaxf(amax, fabsf(v[i]));
+            for (int i = 0; i < 8; ++i) {
+                float a = v[i];
+                if constexpr (NORM)
+                    a = norm1(a, r, g[i]);
+                amax = fmaxf(amax, fabsf(a));
+            }
         }
         const uint32_t u = __reduce_max_sync(0xffffffffu, __float_as_uint(amax));
         if (lane == 0)
@@ -221,13 +295,24 @@ gemv_kernel(const __grid_constant__ Params p)
             u = max(u, red_u[m * CWARPS + w]);
         const float beta = fmaxf(__uint_as_float(u), 1e-5f);
         const float scale = __fdiv_rn(127.0f, beta);
+        float r = 1.0f;
+        if constexpr (NORM)
+            r = row_rms_scale(red_d, m, K, P.norm_eps);
         int sum = 0;
         auto quant_store = [&](const Vec8<BF16> &v, int e) {
+            float g[8];
+            if constexpr (NORM)
+                load8<false>(P.norm_gain, e, g);
             uint32_t lo = 0, hi = 0;
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
-                const int q0 = quant1(v.get(i), scale);
-                const int q1 = quant1(v.get(i + 4), scale);
+                float a = v.get(i), b = v.get(i + 4);
+                if constexpr (NORM) {
+                    a = norm1(a, r, g[i]);
+                    b = norm1(b, r, g[i + 4]);
+                }
+                const int q0 = quant1(a, scale);
+                const int q1 = quant1(b, scale);
                 sum += q0 + q1;
                 lo |= (static_cast<uint32_t>(q0) & 0xffu) << (8 * i);
                 hi |= (static_cast<uint32_t>(q1) & 0xffu) << (8 * i);

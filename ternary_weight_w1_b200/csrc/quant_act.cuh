@@ -8,7 +8,14 @@
 // activations in registers from the absmax pass, so a row is read from
 // memory once when 32 * WPR * 8 * CACHE covers it; anything beyond is
 // re-read in the second pass, four vectors in flight per lane. A grouped
-// variant quantises the rows of several problems in one launch. The row sum
+// variant quantises the rows of several problems in one launch.
+//
+// With NORM the row is RMS-normalised first, as the listing's BitLinear does
+// with its nn.RMSNorm member before quantising: a first pass sums the squares
+// in double (exact products; the butterfly and the fixed warp order make the
+// sum the same in every block), r = 1 / sqrt(mean + eps) in IEEE fp32, and
+// the absmax and quantisation passes work on (x * r) * g with the channel
+// gains g read as they are needed. The row sum
 // of x~ is written for the tensor-core path, whose GEMM contracts the
 // non-negative weight codes W~ + 1 (acc = sum x~ * code - sum x~). Block 0
 // also clears the GEMM's inter-block flag words when asked to.
@@ -26,11 +33,14 @@ template <int WPR>
 __host__ __device__ constexpr int rows_per_block() { return WARPS / WPR; }
 
 // Quantises token row m of one problem (warp `part` of the WPR warps that
-// share the row); rows past M take part in the block barriers only.
-template <bool BF16, int CACHE, int WPR>
+// share the row); rows past M take part in the block barriers only. With
+// NORM, gain [K] and eps define the RMS normalisation applied first.
+template <bool BF16, int CACHE, int WPR, bool NORM>
 __device__ __forceinline__ void quant_row(const void *__restrict__ x, int M, int K,
                                           int8_t *__restrict__ xq, float *__restrict__ beta_out,
-                                          int *__restrict__ rowsum_out, int m, int part)
+                                          int *__restrict__ rowsum_out,
+                                          const float *__restrict__ gain, float eps, int m,
+                                          int part)
 {
     static_assert(WARPS % WPR == 0, "warps per row");
     constexpr int STRIDE = 32 * WPR;              // vectors between a lane's vectors
@@ -49,28 +59,89 @@ __device__ __forceinline__ void quant_row(const void *__restrict__ x, int M, int
 
     Vec8<BF16> cache[CACHE];
     float amax = 0.0f;
+    float r = 1.0f;                               // NORM: 1 / rms of the row
+    if constexpr (!NORM) {
 #pragma unroll
-    for (int i = 0; i < CACHE; ++i) {
-        const int v = v0 + STRIDE * i;
-        if (v < nvec) {
-            cache[i].load(row, v * 8);
-#pragma unroll
-            for (int j = 0; j < 8; ++j)
-                amax = fmaxf(amax, fabsf(cache[i].get(j)));
-        }
-    }
-    for (int vb = v0 + STRIDE * CACHE; vb < nvec; vb += 4 * STRIDE) {
-        Vec8<BF16> t[4];
-#pragma unroll
-        for (int u = 0; u < 4; ++u)
-            if (vb + u * STRIDE < nvec)
-                t[u].load(row, (vb + u * STRIDE) * 8);
-#pragma unroll
-        for (int u = 0; u < 4; ++u)
-            if (vb + u * STRIDE < nvec)
+        for (int i = 0; i < CACHE; ++i) {
+            const int v = v0 + STRIDE * i;
+            if (v < nvec) {
+                cache[i].load(row, v * 8);
 #pragma unroll
                 for (int j = 0; j < 8; ++j)
-                    amax = fmaxf(amax, fabsf(t[u].get(j)));
+                    amax = fmaxf(amax, fabsf(cache[i].get(j)));
+            }
+        }
+        for (int vb = v0 + STRIDE * CACHE; vb < nvec; vb += 4 * STRIDE) {
+            Vec8<BF16> t[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+                if (vb + u * STRIDE < nvec)
+                    t[u].load(row, (vb + u * STRIDE) * 8);
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+                if (vb + u * STRIDE < nvec)
+#pragma unroll
+                    for (int j = 0; j < 8; ++j)
+                        amax = fmaxf(amax, fabsf(t[u].get(j)));
+        }
+    } else {
+        // sum of squares (each product exact in double)
+        double ss = 0.0;
+#pragma unroll
+        for (int i = 0; i < CACHE; ++i) {
+            const int v = v0 + STRIDE * i;
+            if (v < nvec) {
+                cache[i].load(row, v * 8);
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const double d = cache[i].get(j);
+                    ss = __fma_rn(d, d, ss);
+                }
+            }
+        }
+        for (int vb = v0 + STRIDE * CACHE; vb < nvec; vb += STRIDE) {
+            Vec8<BF16> t;
+            t.load(row, vb * 8);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const double d = t.get(j);
+                ss = __fma_rn(d, d, ss);
+            }
+        }
+        ss = warp_sum_f64(ss);
+        if constexpr (WPR > 1) {
+            __shared__ double red_ss[WARPS];
+            if (lane == 0)
+                red_ss[warp] = ss;
+            __syncthreads();
+            const int w0 = warp - part;
+            ss = red_ss[w0];
+#pragma unroll
+            for (int w = 1; w < WPR; ++w)
+                ss = __dadd_rn(ss, red_ss[w0 + w]);
+        }
+        r = rms_scale(ss, K, eps);
+        // absmax of the normalised row
+#pragma unroll
+        for (int i = 0; i < CACHE; ++i) {
+            const int v = v0 + STRIDE * i;
+            if (v < nvec) {
+                float g[8];
+                load8<false>(gain, v * 8, g);
+#pragma unroll
+                for (int j = 0; j < 8; ++j)
+                    amax = fmaxf(amax, fabsf(norm1(cache[i].get(j), r, g[j])));
+            }
+        }
+        for (int vb = v0 + STRIDE * CACHE; vb < nvec; vb += STRIDE) {
+            Vec8<BF16> t;
+            float g[8];
+            t.load(row, vb * 8);
+            load8<false>(gain, vb * 8, g);
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+                amax = fmaxf(amax, fabsf(norm1(t.get(j), r, g[j])));
+        }
     }
     uint32_t umax = __reduce_max_sync(0xffffffffu, __float_as_uint(amax));
     if constexpr (WPR > 1) {
@@ -89,11 +160,19 @@ __device__ __forceinline__ void quant_row(const void *__restrict__ x, int M, int
     int8_t *out = xq + static_cast<size_t>(active ? m : 0) * K;
     int sum = 0;
     auto quant_store = [&](const Vec8<BF16> &t, int v) {
+        float g[8];
+        if constexpr (NORM)
+            load8<false>(gain, v * 8, g);
         uint32_t lo = 0, hi = 0;
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-            const int q0 = quant1(t.get(i), scale);
-            const int q1 = quant1(t.get(i + 4), scale);
+            float a = t.get(i), b = t.get(i + 4);
+            if constexpr (NORM) {
+                a = norm1(a, r, g[i]);
+                b = norm1(b, r, g[i + 4]);
+            }
+            const int q0 = quant1(a, scale);
+            const int q1 = quant1(b, scale);
             sum += q0 + q1;
             lo |= (static_cast<uint32_t>(q0) & 0xffu) << (8 * i);
             hi |= (static_cast<uint32_t>(q1) & 0xffu) << (8 * i);
@@ -136,11 +215,11 @@ __device__ __forceinline__ void quant_row(const void *__restrict__ x, int M, int
     }
 }
 
-template <bool BF16, int CACHE, int WPR>
+template <bool BF16, int CACHE, int WPR, bool NORM>
 __global__ void __launch_bounds__(THREADS)
 quant_act_kernel(const void *__restrict__ x, int M, int K, int8_t *__restrict__ xq,
                  float *__restrict__ beta_out, int *__restrict__ rowsum_out,
-                 int *__restrict__ clear, int n_clear)
+                 int *__restrict__ clear, int n_clear, const float *__restrict__ gain, float eps)
 {
     const int warp = threadIdx.x >> 5;
     const int m = blockIdx.x * rows_per_block<WPR>() + warp / WPR;
@@ -150,7 +229,8 @@ quant_act_kernel(const void *__restrict__ x, int M, int K, int8_t *__restrict__ 
     if (clear != nullptr && blockIdx.x == 0)
         for (int i = threadIdx.x; i < n_clear; i += THREADS)
             clear[i] = 0;
-    quant_row<BF16, CACHE, WPR>(x, M, K, xq, beta_out, rowsum_out, m, warp % WPR);
+    quant_row<BF16, CACHE, WPR, NORM>(x, M, K, xq, beta_out, rowsum_out, gain, eps, m,
+                                      warp % WPR);
 }
 
 // Several problems' token rows in one launch (WPR warps per row): block b
@@ -188,7 +268,8 @@ quant_act_grouped_kernel(const __grid_constant__ GroupParams g)
     if (g.clear != nullptr && blockIdx.x == 0)
         for (int i = threadIdx.x; i < g.n_clear; i += THREADS)
             g.clear[i] = 0;
-    quant_row<BF16, CACHE, WPR>(r.x, r.M, r.K, r.xq, r.beta, r.rowsum, m, warp % WPR);
+    quant_row<BF16, CACHE, WPR, false>(r.x, r.M, r.K, r.xq, r.beta, r.rowsum, nullptr, 0.0f, m,
+                                       warp % WPR);
 }
 
 }  // namespace qa

@@ -123,6 +123,76 @@ class Case:
         return check_y(got["y"][ms, ns], y_ref)
 
 
+# Half-integer band of the normalised forms: an x~ whose oracle value
+# n * 127 / beta lies this close to a tie may round to either neighbour.
+TIE_BAND = 1e-4
+
+
+class NormCase(Case):
+    """A Case whose tokens go through the RMS normalisation first
+    (bitlinear_forward_rmsnorm against the oracle's rmsnorm + forward).
+
+    The device adds a token's squares in another order than the oracle (both
+    in double), so its fp32 mean can differ in the last bit when the two sums
+    straddle an fp32 rounding boundary; every normalised value then moves by
+    at most an ulp. Hence beta is compared within 2 ulps and x~ exactly
+    except within TIE_BAND of a half-integer, and acc and y exactly against
+    the oracle applied to the kernel's own x~ and beta."""
+
+    def __init__(self, M, K, N, g_seed=7, eps=bl.RMSNORM_EPS, gain=None, **kw):
+        super().__init__(M, K, N, **kw)
+        self.eps = eps
+        self.gain = workloads.norm_gains(K, g_seed) if gain is None else gain
+        self.xn = self.orc.rmsnorm(self.xf, self.gain, eps)
+        self.xq, self.beta = self.orc.quant_act(self.xn)
+
+    def run(self, path=bl.PATH_AUTO, debug=True):
+        import torch
+        x = self.x_tensor()
+        dev = x.device
+        g = torch.from_numpy(self.gain).to(dev)
+        y = torch.empty((self.M, self.N), dtype=torch.bfloat16, device=dev)
+        acc = torch.full((self.M, self.N), -7, dtype=torch.int32, device=dev)
+        xq = torch.full((self.M, self.K), 99, dtype=torch.int8, device=dev)
+        beta = torch.full((self.M,), -1.0, dtype=torch.float32, device=dev)
+        bl.bitlinear_forward_rmsnorm(x, self.packed_tensor(), self.gamma, self.N, g,
+                                     eps=self.eps, y=y, acc=acc, xq=xq, beta=beta, path=path)
+        torch.cuda.synchronize()
+        return {"y": tensor_to_bf16_bits(y), "acc": acc.cpu().numpy(),
+                "xq": xq.cpu().numpy(), "beta": beta.cpu().numpy()}
+
+    def check_norm_quant(self, got) -> int:
+        """x~ and beta of the normalised tokens (see the class docstring);
+        returns how many x~ differ from the oracle's."""
+        b_or = self.beta.astype(np.float64)
+        assert np.all(np.abs(got["beta"].astype(np.float64) - b_or) <=
+                      2 * np.spacing(self.beta).astype(np.float64))
+        v = self.xn.astype(np.float64) * 127.0 / b_or[:, None]
+        near_tie = np.abs(np.abs(v - np.floor(v)) - 0.5) < TIE_BAND
+        diff = got["xq"].astype(np.int32) - self.xq.astype(np.int32)
+        assert np.all(np.abs(diff) <= 1)
+        assert np.all(near_tie[diff != 0])
+        return int(np.count_nonzero(diff))
+
+    def check_norm_full(self, got) -> int:
+        ndiff = self.check_norm_quant(got)
+        acc = self.orc.matmul_i32(got["xq"], self.Wq)
+        np.testing.assert_array_equal(got["acc"], acc)
+        np.testing.assert_array_equal(
+            got["y"], self.orc.rescale_bf16(acc, got["beta"], np.float32(self.gamma)))
+        return ndiff
+
+    def check_norm_sampled(self, got, count=20000, seed=0) -> int:
+        ndiff = self.check_norm_quant(got)
+        ms, ns = self.sample_pairs(count, seed)
+        acc = self.orc.matmul_i32_pairs(got["xq"], self.Wq, ms, ns)
+        np.testing.assert_array_equal(got["acc"][ms, ns], acc)
+        y_ref = self.orc.rescale_bf16(acc.reshape(-1, 1), got["beta"][ms],
+                                      np.float32(self.gamma))[:, 0]
+        np.testing.assert_array_equal(got["y"][ms, ns], y_ref)
+        return ndiff
+
+
 def check_y(y_bits: np.ndarray, y_ref_bits: np.ndarray) -> float:
     """Relative-error check of bf16 outputs; returns the fraction of
     bit-identical elements."""

@@ -98,6 +98,33 @@ def test_forward_ex_rejects_bad_path():
     assert rc == bl.BITLINEAR_ERR_ARG
 
 
+def fwd_norm(**kw):
+    a = dict(x=FAKE, xdt=0, M=1, K=256, g=FAKE, eps=2.0 ** -23, packed=FAKE, gamma=1.0, N=64,
+             y=FAKE, ws=None, wsb=0, stream=None, acc=None, xq=None, beta=None, path=0)
+    a.update(kw)
+    return bl.lib().bitlinear_forward_rmsnorm(a["x"], a["xdt"], a["M"], a["K"], a["g"], a["eps"],
+                                              a["packed"], a["gamma"], a["N"], a["y"], a["ws"],
+                                              a["wsb"], a["stream"], a["acc"], a["xq"], a["beta"],
+                                              a["path"])
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(g=None), bl.BITLINEAR_ERR_ARG),             # gains required for a non-empty batch
+    (dict(g=FAKE + 4), bl.BITLINEAR_ERR_ALIGN),
+    (dict(eps=0.0), bl.BITLINEAR_ERR_ARG),
+    (dict(eps=-1e-6), bl.BITLINEAR_ERR_ARG),
+    (dict(eps=float("nan")), bl.BITLINEAR_ERR_ARG),
+    (dict(eps=float("inf")), bl.BITLINEAR_ERR_ARG),
+    (dict(K=200), bl.BITLINEAR_ERR_SHAPE),            # the forward's own checks follow
+    (dict(x=None), bl.BITLINEAR_ERR_ARG),
+    (dict(y=FAKE + 2), bl.BITLINEAR_ERR_ALIGN),
+    (dict(path=9), bl.BITLINEAR_ERR_ARG),
+    (dict(M=0, g=None), bl.BITLINEAR_OK),             # empty batch: nothing to do
+])
+def test_forward_rmsnorm_rejects_bad_arguments(kw, status):
+    assert fwd_norm(**kw) == status
+
+
 def test_quant_act_rejects_bad_arguments():
     L = bl.lib()
     assert L.bitlinear_quant_act(None, 0, 2, 256, FAKE, FAKE, None) == bl.BITLINEAR_ERR_ARG
@@ -199,6 +226,10 @@ def test_binding_refuses_host_tensors():
     with pytest.raises(ValueError, match="CUDA tensor"):
         bl.bitlinear_forward_grouped([(x, packed, 1.0, 64,
                                        torch.zeros((4, 64), dtype=torch.bfloat16))])
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        bl.bitlinear_forward_rmsnorm(x, packed, 1.0, 64, torch.ones(256),
+                                     y=torch.zeros((4, 64), dtype=torch.bfloat16),
+                                     path=bl.PATH_GEMV)
     with pytest.raises(ValueError, match="CUDA tensor"):
         bl.bitlinear_int8_gemm(torch.zeros((128, 128), dtype=torch.int8),
                                torch.zeros((128, 128), dtype=torch.int8),

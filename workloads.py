@@ -12,6 +12,8 @@ Recipe (no trained weights or datasets are used):
     choice, the same channels for every token) multiplied by 50 as outlier
     channels, then rounded to bf16 (the tiny case keeps fp32 and has no
     outliers);
+  * RMS-normalisation gains g [K] (the normalising forms of the path) are
+    drawn uniformly from [0.5, 1.5);
   * every draw uses numpy's PCG64 generator seeded per (workload, matrix).
 """
 from __future__ import annotations
@@ -62,6 +64,12 @@ def activations_f32(M: int, K: int, seed: int, outliers: bool = True,
     if outliers and K > 0:
         x[:, outlier_channels(K, seed, fraction)] *= np.float32(scale)
     return x
+
+
+def norm_gains(K: int, seed: int, low: float = 0.5, high: float = 1.5) -> np.ndarray:
+    """fp32 [K] RMS-normalisation gains drawn uniformly from [low, high): a
+    stand-in for learned per-channel gains, which start at one."""
+    return rng(seed ^ 0x6A15).uniform(low, high, size=K).astype(np.float32)
 
 
 def to_bf16_bits(x: np.ndarray) -> np.ndarray:
