@@ -20,7 +20,9 @@ Functions:
     f32_to_bf16(f)              RNE rounding to bf16 bit patterns (uint16)
     rescale_bf16(acc, beta, gamma)     y bf16 bits [M][N]
     pack_codes(Wq)              the 2-bit packed layout (flat uint8)
+    relu2_glu(gate, up)         h = max(gate, 0)^2 * up (fp32, elementwise)
     forward(x, W)               the whole path, returning every stage
+    ffn(x, W_gate, W_up, W_down)   gate/up -> gated ReLU^2 -> down, every stage
 """
 from __future__ import annotations
 
@@ -74,6 +76,8 @@ def _declare(lib):
     lib.oracle_f32_to_bf16_array.argtypes = [p, c_i64, p]
     lib.oracle_rescale_bf16.restype = None
     lib.oracle_rescale_bf16.argtypes = [p, p, ctypes.c_float, c_i64, c_i64, p]
+    lib.oracle_relu2_glu.restype = None
+    lib.oracle_relu2_glu.argtypes = [p, p, c_i64, p]
     lib.oracle_pack_codes.restype = ctypes.c_int
     lib.oracle_pack_codes.argtypes = [p, c_i64, c_i64, p]
     return lib
@@ -197,6 +201,15 @@ class Oracle:
             raise ValueError("oracle_pack_codes: K % 128 != 0 or non-ternary")
         return out
 
+    def relu2_glu(self, gate, up) -> np.ndarray:
+        """h = max(gate, 0)^2 * up elementwise on fp32 arrays of one shape."""
+        gate = _c(gate, np.float32)
+        up = _c(up, np.float32)
+        assert gate.shape == up.shape
+        h = np.empty(gate.shape, dtype=np.float32)
+        self.lib.oracle_relu2_glu(_ptr(gate), _ptr(up), gate.size, _ptr(h))
+        return h
+
     def forward(self, x, W, gamma=None, norm_gain=None, norm_eps=RMSNORM_EPS):
         """The whole path on the CPU. ``x`` is fp32 [M][K] or bf16 bit
         patterns (uint16); ``W`` is the fp32 latent [N][K]. ``gamma`` may be
@@ -215,6 +228,20 @@ class Oracle:
         y = self.rescale_bf16(acc, beta, g)
         return {"gamma": g, "Wq": Wq, "xq": xq, "beta": beta, "acc": acc,
                 "y": y}
+
+    def ffn(self, x, W_gate, W_up, W_down, gammas=(None, None, None),
+            gains=(None, None, None), norm_eps=RMSNORM_EPS):
+        """The feed-forward chain on the CPU: the gate and up BitLinears of
+        the tokens x, the gated ReLU^2 of their bf16 outputs in fp32, and the
+        down BitLinear of that fp32 h. ``gammas`` may supply each matrix's
+        gamma (e.g. the packer's); ``gains`` gives each BitLinear's RMSNorm
+        gains (None: no normalisation), the down projection's being the one
+        ahead of its quantisation. Returns the three forward dicts and h."""
+        rg = self.forward(x, W_gate, gammas[0], gains[0], norm_eps)
+        ru = self.forward(x, W_up, gammas[1], gains[1], norm_eps)
+        h = self.relu2_glu(self.bf16_to_f32(rg["y"]), self.bf16_to_f32(ru["y"]))
+        rd = self.forward(h, W_down, gammas[2], gains[2], norm_eps)
+        return {"gate": rg, "up": ru, "h": h, "down": rd}
 
 
 _default = None

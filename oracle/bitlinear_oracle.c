@@ -19,6 +19,8 @@
  *     y = (x~ W~^T) * beta * gamma / Q_b, the product being an integer sum;
  *   - the listing's RMSNorm ahead of the activation quantisation
  *     (oracle_rmsnorm, for the normalising forms of the path);
+ *   - the gated ReLU^2 between the gate/up and down projections of the
+ *     feed-forward block (oracle_relu2_glu, for the FFN chain);
  *   - the page's PyTorch listing (WeightQuantFunction.forward,
  *     quantize_activations_int8, BitLinear.forward), which fixes what the
  *     formulas leave open: the epsilon is a clamp(min=1e-5) of gamma and beta,
@@ -223,6 +225,26 @@ void oracle_rescale_bf16(const int32_t *acc, const float *beta, float gamma,
         const float s = (beta[m] * gamma) / ORACLE_QB;
         for (int64_t n = 0; n < N; ++n)
             y[m * N + n] = oracle_f32_to_bf16((float)acc[m * N + n] * s);
+    }
+}
+
+/* -------------------------------------------------------------- FFN chain */
+
+/* Gated squared-ReLU of the feed-forward block, elementwise over n values:
+ *   h_i = (r_i * r_i) * up_i,  r_i = max(gate_i, 0)
+ * The winbuzzer.com release article (section "Under the Hood") says ReLU^2
+ * replaces SwiGLU in the model's feed-forward networks, and the bako.co page
+ * names ReLU^2 as the FFN activation; replacing the Swish of SwiGLU keeps its
+ * gate, so ReLU^2 applies to the gate projection's output and multiplies the
+ * up projection's output elementwise. fp32 arithmetic in that order; when
+ * gate and up hold bf16 values (the BitLinear outputs) every product is exact
+ * in fp32 (at most 8 + 8 + 8 significant bits). A non-positive gate gives a
+ * zero (of the sign of up). */
+void oracle_relu2_glu(const float *gate, const float *up, int64_t n, float *h)
+{
+    for (int64_t i = 0; i < n; ++i) {
+        const float r = gate[i] > 0.0f ? gate[i] : 0.0f;
+        h[i] = (r * r) * up[i];
     }
 }
 

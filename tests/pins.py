@@ -24,7 +24,10 @@ unless stated):
   * for the RMS normalisation ahead of quantisation (the listing's
     nn.RMSNorm member of BitLinear): torch's rms_norm in float64 within the
     fp32 error bound, constant rows in closed form, exact invariance under
-    power-of-two scaling at eps = 0, and the gain applied last.
+    power-of-two scaling at eps = 0, and the gain applied last;
+  * for the gated ReLU^2 of the feed-forward chain: exact products on bf16
+    operands (float64 reference), closed forms, and the roles of the gate and
+    up projections in the whole chain.
 """
 from __future__ import annotations
 
@@ -423,6 +426,54 @@ def pin_rmsnorm_gain_applied_last(orc):
     np.testing.assert_array_equal(orc.rmsnorm(x, g, 2.0 ** -23), unit * g[None, :])
 
 
+# ---------------------------------------------------------------- FFN chain
+#
+# ReLU^2 replaces SwiGLU in the feed-forward block (winbuzzer.com release
+# article, "Under the Hood"): h = max(gate, 0)^2 * up on the BitLinear outputs.
+
+def _bf16_round(x):
+    import torch
+    return torch.from_numpy(np.ascontiguousarray(x, dtype=np.float32)).to(
+        torch.bfloat16).float().numpy()
+
+
+def pin_relu2_glu_exact_on_bf16(orc):
+    """On bf16 operands every product has at most 24 significant bits, so
+    the fp32 result equals the exact product (computed in float64)."""
+    r = np.random.Generator(np.random.PCG64(91))
+    scale = 10.0 ** r.uniform(-6, 4, size=4096)
+    g = _bf16_round(r.standard_normal(4096) * scale)
+    u = _bf16_round(r.standard_normal(4096) * scale[::-1])
+    h = orc.relu2_glu(g, u).astype(np.float64)
+    exact = np.maximum(g.astype(np.float64), 0.0) ** 2 * u.astype(np.float64)
+    assert np.all(h == exact)
+    assert np.count_nonzero(h) > 1500          # about half the gates are positive
+
+
+def pin_relu2_glu_closed_forms(orc):
+    g = np.array([2.0, -1.0, 0.0, 0.5, 1.0, 3.0, -1e-3], dtype=np.float32)
+    u = np.array([-3.0, 5.0, 7.0, 2.0, -0.75, 1.0, 4.0], dtype=np.float32)
+    h = orc.relu2_glu(g, u)
+    np.testing.assert_array_equal(h, np.array([-12.0, 0.0, 0.0, 0.5, -0.75, 9.0, 0.0],
+                                              dtype=np.float32))
+
+
+def pin_ffn_gate_and_up_roles(orc):
+    """With every gate output negative the block's output is exactly zero
+    (h = 0, so the down projection quantises a zero token); swapping the
+    gate and up weights then gives a non-zero output."""
+    K, F, N = 256, 64, 48
+    x = np.ones((2, K), dtype=np.float32)
+    neg = np.full((F, K), -0.02, dtype=np.float32)       # ternarises to all -1
+    pos = np.full((F, K), 0.02, dtype=np.float32)        # all +1
+    Wd = (np.random.Generator(np.random.PCG64(92)).standard_normal((N, F)) * 0.02).astype(
+        np.float32)
+    off = orc.ffn(x, neg, pos, Wd)
+    assert np.all(off["h"] == 0.0) and np.all(off["down"]["y"] == 0)
+    on = orc.ffn(x, pos, neg, Wd)
+    assert np.all(on["h"] < 0.0) and np.count_nonzero(on["down"]["y"]) > N
+
+
 ALL_PINS = [
     pin_hand_example,
     pin_weight_ties_even,
@@ -448,6 +499,9 @@ ALL_PINS = [
     pin_rmsnorm_constant_rows,
     pin_rmsnorm_pow2_invariance,
     pin_rmsnorm_gain_applied_last,
+    pin_relu2_glu_exact_on_bf16,
+    pin_relu2_glu_closed_forms,
+    pin_ffn_gate_and_up_roles,
 ]
 
 

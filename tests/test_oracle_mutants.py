@@ -48,6 +48,11 @@ MUTANTS = {
     "rms_gain_by_token": ("(row[k] * r) * g[k]", "(row[k] * r) * g[m]"),
     "rms_gain_first": ("(row[k] * r) * g[k]", "(row[k] * g[k]) * r"),
     "rms_gain_dropped": ("(row[k] * r) * g[k]", "(row[k] * r)"),
+    "glu_no_relu": ("gate[i] > 0.0f ? gate[i] : 0.0f", "gate[i]"),
+    "glu_relu_inverted": ("gate[i] > 0.0f ? gate[i] : 0.0f", "gate[i] < 0.0f ? gate[i] : 0.0f"),
+    "glu_no_square": ("(r * r) * up[i]", "r * up[i]"),
+    "glu_ignores_up": ("(r * r) * up[i]", "(r * r)"),
+    "glu_adds_up": ("(r * r) * up[i]", "(r * r) + up[i]"),
 }
 
 
