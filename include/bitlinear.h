@@ -55,7 +55,8 @@ typedef enum {
     BITLINEAR_ERR_CUDA = 5,      /* a CUDA runtime/driver call failed */
     BITLINEAR_ERR_TIMEOUT = 6,   /* a bounded device-side wait ran out */
     BITLINEAR_ERR_WORKSPACE = 7, /* workspace missing or smaller than required */
-    BITLINEAR_ERR_SCRATCH_LIMIT = 8 /* problem too large for the library's static scratch */
+    BITLINEAR_ERR_SCRATCH_LIMIT = 8, /* problem too large for the library's static scratch */
+    BITLINEAR_ERR_HOST = 9       /* a host allocation failed */
 } bitlinear_status;
 
 typedef enum {
@@ -102,8 +103,9 @@ size_t bitlinear_packed_bytes(int64_t N, int64_t K);
  * Follows section "Ternary Weight Quantization: absmean Scaling" and the
  * listing's WeightQuantFunction.forward (W / gamma in fp32, ties to even,
  * clip to [-1, 1]). Returns BITLINEAR_ERR_ARG for null pointers or N < 1,
- * BITLINEAR_ERR_SHAPE for a bad K. Runs on several host threads; the result
- * does not depend on their number. */
+ * BITLINEAR_ERR_SHAPE for a bad K, BITLINEAR_ERR_HOST if a host allocation
+ * fails. Runs on several host threads (on the calling thread alone when no
+ * thread can be created); the result does not depend on their number. */
 int bitlinear_pack_weights(const float *W_host, int64_t N, int64_t K,
                            void *packed_host, float *gamma_out);
 

@@ -26,6 +26,7 @@ BITLINEAR_ERR_CUDA = 5
 BITLINEAR_ERR_TIMEOUT = 6
 BITLINEAR_ERR_WORKSPACE = 7
 BITLINEAR_ERR_SCRATCH_LIMIT = 8
+BITLINEAR_ERR_HOST = 9
 BITLINEAR_STATIC_SCRATCH_BYTES = 16 << 20
 
 BITLINEAR_BF16 = 0

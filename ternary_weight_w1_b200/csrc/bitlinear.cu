@@ -730,6 +730,7 @@ extern "C" const char *bitlinear_status_string(int status)
     case BITLINEAR_ERR_TIMEOUT: return "device wait timed out";
     case BITLINEAR_ERR_WORKSPACE: return "workspace missing or too small";
     case BITLINEAR_ERR_SCRATCH_LIMIT: return "problem exceeds the static scratch limit";
+    case BITLINEAR_ERR_HOST: return "host allocation failed";
     default: return "unknown status";
     }
 }

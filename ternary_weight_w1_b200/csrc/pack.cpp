@@ -35,25 +35,32 @@ unsigned worker_count(int64_t work_items)
     return static_cast<unsigned>(std::min<int64_t>(hw, useful));
 }
 
+// Runs fn(0 .. count-1) over worker threads (fn must be safe to call
+// concurrently for different i). If a thread cannot be created, the items not
+// yet handed out run on the calling thread instead.
 template <class Fn>
 void parallel_for(int64_t count, Fn fn)
 {
     const unsigned workers = worker_count(count);
-    if (workers <= 1) {
-        for (int64_t i = 0; i < count; ++i)
-            fn(i);
-        return;
-    }
     std::vector<std::thread> pool;
-    pool.reserve(workers);
-    for (unsigned t = 0; t < workers; ++t) {
-        const int64_t lo = count * t / workers;
-        const int64_t hi = count * (t + 1) / workers;
-        pool.emplace_back([=, &fn] {
-            for (int64_t i = lo; i < hi; ++i)
-                fn(i);
-        });
+    int64_t handed_out = 0;
+    if (workers > 1) {
+        try {
+            pool.reserve(workers);
+            for (unsigned t = 0; t < workers; ++t) {
+                const int64_t lo = count * t / workers;
+                const int64_t hi = count * (t + 1) / workers;
+                pool.emplace_back([=, &fn] {
+                    for (int64_t i = lo; i < hi; ++i)
+                        fn(i);
+                });
+                handed_out = hi;
+            }
+        } catch (...) {
+        }
     }
+    for (int64_t i = handed_out; i < count; ++i)
+        fn(i);
     for (auto &th : pool)
         th.join();
 }
@@ -79,14 +86,10 @@ extern "C" size_t bitlinear_packed_bytes(int64_t N, int64_t K)
     return static_cast<size_t>(blocks) * 16 * static_cast<size_t>(K / 4);
 }
 
-extern "C" int bitlinear_pack_weights(const float *W_host, int64_t N, int64_t K,
-                                      void *packed_host, float *gamma_out)
-{
-    if (!W_host || !packed_host || !gamma_out || N < 1 || K < 0)
-        return BITLINEAR_ERR_ARG;
-    if (K < 128 || K % 128 != 0)
-        return BITLINEAR_ERR_SHAPE;
+namespace {
 
+int pack_weights(const float *W_host, int64_t N, int64_t K, void *packed_host, float *gamma_out)
+{
     // gamma = mean |W| (double accumulation in fixed blocks, then one cast).
     const int64_t total = N * K;
     const int64_t blocks = (total + kBlock - 1) / kBlock;
@@ -133,4 +136,21 @@ extern "C" int bitlinear_pack_weights(const float *W_host, int64_t N, int64_t K,
     });
     *gamma_out = gamma;
     return BITLINEAR_OK;
+}
+
+}  // namespace
+
+extern "C" int bitlinear_pack_weights(const float *W_host, int64_t N, int64_t K,
+                                      void *packed_host, float *gamma_out)
+{
+    if (!W_host || !packed_host || !gamma_out || N < 1 || K < 0)
+        return BITLINEAR_ERR_ARG;
+    if (K < 128 || K % 128 != 0)
+        return BITLINEAR_ERR_SHAPE;
+    try {
+        return pack_weights(W_host, N, K, packed_host, gamma_out);
+    } catch (...) {
+        // nothing crosses the C ABI; only host allocation can fail here
+        return BITLINEAR_ERR_HOST;
+    }
 }

@@ -32,7 +32,18 @@ def test_library_exports_every_declared_symbol():
 def test_status_strings():
     assert bl.status_string(bl.BITLINEAR_OK) == "ok"
     assert bl.status_string(bl.BITLINEAR_ERR_TIMEOUT) == "device wait timed out"
+    assert bl.status_string(bl.BITLINEAR_ERR_HOST) == "host allocation failed"
     assert bl.status_string(99) == "unknown status"
+
+
+def test_binding_status_codes_match_the_header():
+    text = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
+    enum = re.search(r"typedef enum \{(.*?)\} bitlinear_status;", text, flags=re.S).group(1)
+    codes = dict((k, int(v)) for k, v in re.findall(r"(BITLINEAR_\w+)\s*=\s*(\d+)", enum))
+    assert len(codes) >= 10
+    for name, value in codes.items():
+        assert getattr(bl, name) == value, name
+        assert bl.status_string(value) != "unknown status", name
 
 
 def test_packed_bytes():
