@@ -56,7 +56,9 @@ typedef enum {
     BITLINEAR_ERR_TIMEOUT = 6,   /* a bounded device-side wait ran out */
     BITLINEAR_ERR_WORKSPACE = 7, /* workspace missing or smaller than required */
     BITLINEAR_ERR_SCRATCH_LIMIT = 8, /* problem too large for the library's static scratch */
-    BITLINEAR_ERR_HOST = 9       /* a host allocation failed */
+    BITLINEAR_ERR_HOST = 9,      /* a host allocation failed */
+    BITLINEAR_ERR_IO = 10,       /* a file could not be opened, written or renamed */
+    BITLINEAR_ERR_FORMAT = 11    /* not a valid packed-weight file (header, size or checksum) */
 } bitlinear_status;
 
 typedef enum {
@@ -74,8 +76,8 @@ typedef enum {
 /* ---------------------------------------------------------------- packing */
 
 /* Bytes of the packed ternary matrix for N rows of K weights:
- * ceil(N / 16) * 16 * K / 4. Returns 0 when N < 1 or K is not a positive
- * multiple of 128.
+ * ceil(N / 16) * 16 * K / 4. Returns 0 when N < 1, K is not a positive
+ * multiple of 128, or the size does not fit in 64 bits.
  *
  * Packed layout (this library's own; the "2-bit nibbles" of the bitnet.xin
  * guide, section "Core Architecture"):
@@ -108,6 +110,43 @@ size_t bitlinear_packed_bytes(int64_t N, int64_t K);
  * thread can be created); the result does not depend on their number. */
 int bitlinear_pack_weights(const float *W_host, int64_t N, int64_t K,
                            void *packed_host, float *gamma_out);
+
+/* ------------------------------------------------------ packed-weight files */
+
+/* The packer's output stored once and loaded at serving time (the ternary
+ * weights are exported once after training: "BitNet b1.58 2B4T Guide",
+ * section "High-Precision Master Weights"). A file is a 64-byte little-endian
+ * header followed by the payload:
+ *   0  "BITLIN58"   8  u32 version (1)   12 u32 layout (1 = the layout above)
+ *   16 i64 N        24 i64 K             32 f32 gamma       36 u32 0
+ *   40 u64 payload bytes (= bitlinear_packed_bytes(N, K))
+ *   48 u64 FNV-1a 64-bit hash of the payload                56 u64 0
+ *   64 payload (the packed bytes, as bitlinear_pack_weights wrote them)
+ * All three calls are host-only and thread-safe for different paths. */
+
+/* Writes a packed matrix and its gamma to `path` (through "<path>.tmp" and a
+ * rename, so the final name never holds a partial file). Returns
+ * BITLINEAR_ERR_ARG for null pointers or a gamma that is not finite and > 0,
+ * BITLINEAR_ERR_SHAPE for a bad (N, K), BITLINEAR_ERR_IO when the file
+ * cannot be written. */
+int bitlinear_save_packed(const char *path, const void *packed_host, int64_t N,
+                          int64_t K, float gamma);
+
+/* Reads only the header of `path`: N, K and gamma, so the caller can size
+ * the payload buffer (bitlinear_packed_bytes(N, K)). BITLINEAR_ERR_IO when
+ * the file cannot be opened, BITLINEAR_ERR_FORMAT for a bad header. */
+int bitlinear_read_packed_header(const char *path, int64_t *N_out,
+                                 int64_t *K_out, float *gamma_out);
+
+/* Reads `path` into the caller's host buffer of packed_bytes bytes (at least
+ * the payload) and returns N, K and gamma. The payload hash is checked:
+ * BITLINEAR_ERR_FORMAT for a bad header, a truncated or over-long file or a
+ * hash mismatch; BITLINEAR_ERR_ARG when the buffer is too small;
+ * BITLINEAR_ERR_IO when the file cannot be opened. The outputs are written
+ * only on success. */
+int bitlinear_load_packed(const char *path, void *packed_host,
+                          size_t packed_bytes, int64_t *N_out, int64_t *K_out,
+                          float *gamma_out);
 
 /* ------------------------------------------------- activation quantisation */
 

@@ -27,6 +27,8 @@ BITLINEAR_ERR_TIMEOUT = 6
 BITLINEAR_ERR_WORKSPACE = 7
 BITLINEAR_ERR_SCRATCH_LIMIT = 8
 BITLINEAR_ERR_HOST = 9
+BITLINEAR_ERR_IO = 10
+BITLINEAR_ERR_FORMAT = 11
 BITLINEAR_STATIC_SCRATCH_BYTES = 16 << 20
 
 BITLINEAR_BF16 = 0
@@ -44,6 +46,9 @@ RMSNORM_EPS = 2.0 ** -23
 EXPORTS = (
     "bitlinear_packed_bytes",
     "bitlinear_pack_weights",
+    "bitlinear_save_packed",
+    "bitlinear_read_packed_header",
+    "bitlinear_load_packed",
     "bitlinear_quant_act",
     "bitlinear_workspace_bytes",
     "bitlinear_workspace_bytes_path",
@@ -89,6 +94,12 @@ def lib() -> ctypes.CDLL:
         L.bitlinear_packed_bytes.argtypes = [i64, i64]
         L.bitlinear_pack_weights.restype = ctypes.c_int
         L.bitlinear_pack_weights.argtypes = [p, i64, i64, p, p]
+        L.bitlinear_save_packed.restype = ctypes.c_int
+        L.bitlinear_save_packed.argtypes = [ctypes.c_char_p, p, i64, i64, ctypes.c_float]
+        L.bitlinear_read_packed_header.restype = ctypes.c_int
+        L.bitlinear_read_packed_header.argtypes = [ctypes.c_char_p, p, p, p]
+        L.bitlinear_load_packed.restype = ctypes.c_int
+        L.bitlinear_load_packed.argtypes = [ctypes.c_char_p, p, sz, p, p, p]
         L.bitlinear_quant_act.restype = ctypes.c_int
         L.bitlinear_quant_act.argtypes = [p, ctypes.c_int, i64, i64, p, p, p]
         L.bitlinear_workspace_bytes.restype = sz
@@ -219,6 +230,40 @@ def bitlinear_pack_weights(W) -> tuple[np.ndarray, float]:
                                         ctypes.addressof(gamma)),
            "bitlinear_pack_weights")
     return out, float(gamma.value)
+
+
+def bitlinear_save_packed(path, packed, N: int, K: int, gamma: float) -> None:
+    """Write packed weights (host uint8 array of bitlinear_packed_bytes(N, K)
+    bytes, as bitlinear_pack_weights returns it) and gamma to a file."""
+    packed = np.ascontiguousarray(packed, dtype=np.uint8)
+    need = bitlinear_packed_bytes(N, K)
+    if need and packed.size < need:
+        raise ValueError(f"packed must hold {need} bytes, got {packed.size}")
+    _check(lib().bitlinear_save_packed(os.fsencode(path), packed.ctypes.data, N, K,
+                                       float(gamma)),
+           "bitlinear_save_packed")
+
+
+def bitlinear_read_packed_header(path) -> tuple[int, int, float]:
+    """(N, K, gamma) from a packed-weight file's header."""
+    n, k, g = ctypes.c_int64(0), ctypes.c_int64(0), ctypes.c_float(0.0)
+    _check(lib().bitlinear_read_packed_header(os.fsencode(path), ctypes.addressof(n),
+                                              ctypes.addressof(k), ctypes.addressof(g)),
+           "bitlinear_read_packed_header")
+    return n.value, k.value, float(g.value)
+
+
+def bitlinear_load_packed(path) -> tuple[np.ndarray, int, int, float]:
+    """(packed uint8 array, N, K, gamma) from a packed-weight file; the
+    payload's hash is checked."""
+    N, K, _ = bitlinear_read_packed_header(path)
+    out = np.empty((bitlinear_packed_bytes(N, K),), dtype=np.uint8)
+    n, k, g = ctypes.c_int64(0), ctypes.c_int64(0), ctypes.c_float(0.0)
+    _check(lib().bitlinear_load_packed(os.fsencode(path), out.ctypes.data, out.size,
+                                       ctypes.addressof(n), ctypes.addressof(k),
+                                       ctypes.addressof(g)),
+           "bitlinear_load_packed")
+    return out, n.value, k.value, float(g.value)
 
 
 # ------------------------------------------------- activation quantisation

@@ -3,8 +3,9 @@
     python -m ternary_weight_w1_b200.build        # or build() from Python
 
 The library is one CUDA translation unit (the kernels and the C ABI) plus
-the host packer. cudart is linked statically so the library does not depend
-on which CUDA runtime the host process loaded first.
+the host packer and the packed-weight file reader and writer. cudart is
+linked statically so the library does not depend on which CUDA runtime the
+host process loaded first.
 """
 from __future__ import annotations
 
@@ -15,7 +16,8 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libbitlinear.so")
-SOURCES = [os.path.join(CSRC, "bitlinear.cu"), os.path.join(CSRC, "pack.cpp")]
+SOURCES = [os.path.join(CSRC, "bitlinear.cu"), os.path.join(CSRC, "pack.cpp"),
+           os.path.join(CSRC, "packfile.cpp")]
 # Everything the translation units include: every header in csrc/ and the ABI header.
 DEPS = SOURCES + sorted(os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith(".cuh")) + [
     os.path.join(HERE, "..", "include", "bitlinear.h")]

@@ -731,6 +731,8 @@ extern "C" const char *bitlinear_status_string(int status)
     case BITLINEAR_ERR_WORKSPACE: return "workspace missing or too small";
     case BITLINEAR_ERR_SCRATCH_LIMIT: return "problem exceeds the static scratch limit";
     case BITLINEAR_ERR_HOST: return "host allocation failed";
+    case BITLINEAR_ERR_IO: return "file could not be read or written";
+    case BITLINEAR_ERR_FORMAT: return "not a valid packed-weight file";
     default: return "unknown status";
     }
 }

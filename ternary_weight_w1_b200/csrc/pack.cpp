@@ -12,6 +12,7 @@
 // Must be compiled without fast-math (IEEE division and rounding).
 
 #include <algorithm>
+#include <climits>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -82,7 +83,9 @@ extern "C" size_t bitlinear_packed_bytes(int64_t N, int64_t K)
 {
     if (N < 1 || K < 128 || K % 128 != 0)
         return 0;
-    const int64_t blocks = (N + 15) / 16;
+    const int64_t blocks = N / 16 + (N % 16 != 0 ? 1 : 0);
+    if (K / 4 > INT64_MAX / 16 / blocks)          // the size would not fit in 64 bits
+        return 0;
     return static_cast<size_t>(blocks) * 16 * static_cast<size_t>(K / 4);
 }
 
