@@ -32,6 +32,65 @@ def bf16_value(bits: np.ndarray) -> np.ndarray:
     return (bits.astype(np.uint32) << 16).view(np.float32)
 
 
+class Guarded:
+    """An output tensor inside a larger buffer whose PAD_BYTES before and
+    after it, and the output itself, start filled with a canary bit pattern
+    no correct result holds. After a launch, check() fails if a kernel wrote
+    past either end of the output (the interior is compared with the oracle,
+    so an element left unwritten shows there)."""
+
+    PAD_BYTES = 256
+    RAW = {1: "int8", 2: "int16", 4: "int32"}
+
+    def __init__(self, shape, dtype, device, canary: int):
+        import torch
+        esz = torch.empty((), dtype=dtype).element_size()
+        self.pad = self.PAD_BYTES // esz
+        self.n = int(np.prod(shape))
+        self.canary = canary
+        self.raw = torch.full((2 * self.pad + self.n,), canary,
+                              dtype=getattr(torch, self.RAW[esz]), device=device)
+        self.t = self.raw[self.pad:self.pad + self.n].view(dtype).view(*shape)
+
+    def check(self, name: str = "output"):
+        import torch
+        head = self.raw[:self.pad]
+        tail = self.raw[self.pad + self.n:]
+        assert bool(torch.all(head == self.canary)), f"write before the start of {name}"
+        assert bool(torch.all(tail == self.canary)), f"write past the end of {name}"
+
+
+# canaries: a bf16 NaN, an accumulator far beyond 127 * 65536, an x~ of -128
+# (|x~| <= 127) and an fp32 NaN
+CANARY_Y = 0x7FA5
+CANARY_ACC = 0x5A5A5A5A
+CANARY_XQ = -128
+CANARY_BETA = 0x7FC0A5A5
+
+
+def guarded_outputs(M, N, K, device, debug=True):
+    """Guarded y (bf16 [M][N]) and, with `debug`, acc, xq and beta."""
+    import torch
+    out = {"y": Guarded((M, N), torch.bfloat16, device, CANARY_Y)}
+    if debug:
+        out["acc"] = Guarded((M, N), torch.int32, device, CANARY_ACC)
+        out["xq"] = Guarded((M, K), torch.int8, device, CANARY_XQ)
+        out["beta"] = Guarded((M,), torch.float32, device, CANARY_BETA)
+    return out
+
+
+def read_guarded(g) -> dict:
+    """Checks every canary and returns the outputs as numpy arrays (y as
+    bf16 bit patterns)."""
+    for name, v in g.items():
+        v.check(name)
+    out = {"y": tensor_to_bf16_bits(g["y"].t)}
+    for name in ("acc", "xq", "beta"):
+        if name in g:
+            out[name] = g[name].t.cpu().numpy()
+    return out
+
+
 class Case:
     """One problem: inputs, the packed weights and the oracle's view of them."""
 
@@ -67,20 +126,11 @@ class Case:
         import torch
         x = self.x_tensor()
         packed = self.packed_tensor()
-        dev = x.device
-        y = torch.empty((self.M, self.N), dtype=torch.bfloat16, device=dev)
-        acc = torch.full((self.M, self.N), -7, dtype=torch.int32, device=dev) if debug else None
-        xq = torch.full((self.M, self.K), 99, dtype=torch.int8, device=dev) if debug else None
-        beta = torch.full((self.M,), -1.0, dtype=torch.float32, device=dev) if debug else None
-        bl.bitlinear_forward(x, packed, self.gamma, self.N, y=y, acc=acc, xq=xq, beta=beta,
-                             path=path)
+        g = guarded_outputs(self.M, self.N, self.K, x.device, debug)
+        dbg = {k: g[k].t for k in ("acc", "xq", "beta")} if debug else {}
+        bl.bitlinear_forward(x, packed, self.gamma, self.N, y=g["y"].t, path=path, **dbg)
         torch.cuda.synchronize()
-        out = {"y": tensor_to_bf16_bits(y)}
-        if debug:
-            out["acc"] = acc.cpu().numpy()
-            out["xq"] = xq.cpu().numpy()
-            out["beta"] = beta.cpu().numpy()
-        return out
+        return read_guarded(g)
 
     # ---------------------------------------------------------- checks
 
@@ -149,17 +199,13 @@ class NormCase(Case):
     def run(self, path=bl.PATH_AUTO, debug=True):
         import torch
         x = self.x_tensor()
-        dev = x.device
-        g = torch.from_numpy(self.gain).to(dev)
-        y = torch.empty((self.M, self.N), dtype=torch.bfloat16, device=dev)
-        acc = torch.full((self.M, self.N), -7, dtype=torch.int32, device=dev)
-        xq = torch.full((self.M, self.K), 99, dtype=torch.int8, device=dev)
-        beta = torch.full((self.M,), -1.0, dtype=torch.float32, device=dev)
-        bl.bitlinear_forward_rmsnorm(x, self.packed_tensor(), self.gamma, self.N, g,
-                                     eps=self.eps, y=y, acc=acc, xq=xq, beta=beta, path=path)
+        gain = torch.from_numpy(self.gain).to(x.device)
+        g = guarded_outputs(self.M, self.N, self.K, x.device, True)
+        bl.bitlinear_forward_rmsnorm(x, self.packed_tensor(), self.gamma, self.N, gain,
+                                     eps=self.eps, y=g["y"].t, acc=g["acc"].t, xq=g["xq"].t,
+                                     beta=g["beta"].t, path=path)
         torch.cuda.synchronize()
-        return {"y": tensor_to_bf16_bits(y), "acc": acc.cpu().numpy(),
-                "xq": xq.cpu().numpy(), "beta": beta.cpu().numpy()}
+        return read_guarded(g)
 
     def check_norm_quant(self, got) -> int:
         """x~ and beta of the normalised tokens (see the class docstring);
