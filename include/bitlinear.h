@@ -201,8 +201,12 @@ int bitlinear_forward(const void *x_dev, bitlinear_dtype xdt, int64_t M,
                       float *beta_dev_or_null);
 
 /* bitlinear_forward with an explicit kernel choice (bitlinear_path).
- * BITLINEAR_PATH_GEMV needs M <= 16 and M * K <= 196608; otherwise it
- * returns BITLINEAR_ERR_SHAPE. The workspace for BITLINEAR_PATH_TC is
+ * BITLINEAR_PATH_GEMV needs M <= 16 and the tokens' x~ (M * K bytes) within
+ * the GEMV's shared-memory limit: 196608 bytes for M <= 8, 196272 for
+ * M = 9..16; otherwise it returns BITLINEAR_ERR_SHAPE, before any device
+ * work. For matrices so tall that their per-CTA row accumulators would not
+ * fit beside a large x~, the GEMV gives each CTA fewer row blocks and runs
+ * in more than one wave. The workspace for BITLINEAR_PATH_TC is
  * bitlinear_workspace_bytes_path(M, N, K, BITLINEAR_PATH_TC). */
 int bitlinear_forward_ex(const void *x_dev, bitlinear_dtype xdt, int64_t M,
                          int64_t K, const void *packed_dev, float gamma,
@@ -254,8 +258,10 @@ typedef struct {
  * computes it on its own; grouping only shares one launch, and the CTAs of
  * every problem stream about the same number of weight bytes.
  *   problems [in] host array of count descriptors (1 <= count <= 8); every
- *                 problem needs M <= 16 and M * K <= 196608; M = 0 problems
- *                 are skipped
+ *                 problem needs the GEMV limits of bitlinear_forward_ex, and
+ *                 the group's largest M * K must be within the limit of its
+ *                 largest M (one launch holds both); M = 0 problems are
+ *                 skipped
  *   xdt      [in] activation dtype of all problems
  * No workspace is needed. Outputs must not overlap each other or any input.
  * Argument errors are reported before any launch, as for bitlinear_forward. */

@@ -30,7 +30,8 @@ namespace {
 
 constexpr int64_t kMaxK = 65536;
 constexpr int kGemvMaxM = 16;
-constexpr int64_t kGemvMaxXqBytes = 196608;       // M * K bytes of x~ in shared memory
+constexpr int64_t kGemvMaxXqBytes = 196608;       // at most M * K bytes of x~ in shared memory
+constexpr int kSmemOptinSm100 = 227 * 1024;        // opt-in shared memory per block on sm_100
 constexpr int64_t kAutoGemvMaxM = 6;                // above: tensor-core path
 // Split the k-range of fewer tiles than CTAs only when a CTA saves more than
 // this many 256-k blocks (each about half a microsecond) by it.
@@ -39,6 +40,22 @@ constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s: far above any legitima
 constexpr int kMaxDevices = 64;
 
 bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// Token tile of a GEMV launch for up to M tokens.
+int gemv_tile(int64_t M) { return M <= 1 ? 1 : M <= 2 ? 2 : M <= 4 ? 4 : M <= 8 ? 8 : 16; }
+
+// Largest x~ (M * K bytes; for a group, the largest problem's) a GEMV launch
+// for up to M tokens admits: it must fit in sm_100's opt-in shared memory
+// beside two ring slots, one row block's accumulators per CTA and the
+// normalising form's reduction arrays, and is at most kGemvMaxXqBytes.
+int64_t gemv_max_xq(int64_t M)
+{
+    const int MT = gemv_tile(M);
+    return std::min<int64_t>(kGemvMaxXqBytes,
+                             kSmemOptinSm100 - gemv::smem_bytes(MT, 0, 16 * MT, 2, true));
+}
+
+bool gemv_fits(int64_t M, int64_t K) { return M <= kGemvMaxM && M * K <= gemv_max_xq(M); }
 
 size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
@@ -302,8 +319,11 @@ struct GemvJob {
 // owns whole 16-row blocks of one problem. A single problem is split over at
 // most two CTAs per SM with the same number of blocks per CTA; a group is
 // split so that the CTAs of every problem stream about the same number of
-// bytes, with at most three CTAs per SM (all resident at once). Either every
-// problem of the launch is RMS-normalised or none is.
+// bytes, with at most three CTAs per SM (all resident at once). The one
+// exception is a matrix so tall, next to so large an x~, that a CTA's row
+// accumulators would not fit: its CTAs then take fewer row blocks and the
+// grid runs in more than one wave. Either every problem of the launch is
+// RMS-normalised or none is.
 int launch_gemv(const GemvJob *jobs, int count, bitlinear_dtype xdt, const DeviceInfo &dev,
                 cudaStream_t st)
 {
@@ -317,14 +337,25 @@ int launch_gemv(const GemvJob *jobs, int count, bitlinear_dtype xdt, const Devic
         Mmax = std::max(Mmax, jobs[i].M);
         total_bytes += static_cast<double>((jobs[i].N + 15) / 16) * 16.0 * jobs[i].K / 4.0;
     }
-    const int MT = Mmax <= 1 ? 1 : Mmax <= 2 ? 2 : Mmax <= 4 ? 4 : Mmax <= 8 ? 8 : 16;
+    const int MT = gemv_tile(Mmax);
+    // Each CTA quantises only its own problem's M rows into shared memory.
+    int xq_cap = 0;
+    for (int i = 0; i < count; ++i)
+        xq_cap = std::max(xq_cap, jobs[i].M * jobs[i].K);
+    // Row blocks per CTA that fit: their int32 row accumulators share the
+    // block's shared memory with x~, so a very tall matrix next to a large x~
+    // takes more, smaller CTAs (and then more than one wave).
+    const int q_fit =
+        (dev.max_smem_optin - gemv::smem_bytes(MT, xq_cap, 0, 2, norm)) / (16 * MT * 4);
+    if (q_fit < 1)
+        return BITLINEAR_ERR_SHAPE;
     const int gmax = 2 * dev.sms;
     const int cap = 3 * dev.sms;
     int q[gemv::MAX_PROBLEMS], ctas[gemv::MAX_PROBLEMS];
     int grid = 0;
     if (count == 1) {
         const int blocks = (jobs[0].N + 15) / 16;
-        q[0] = (blocks + gmax - 1) / gmax;
+        q[0] = std::min((blocks + gmax - 1) / gmax, q_fit);
         ctas[0] = (blocks + q[0] - 1) / q[0];
         grid = ctas[0];
     } else {
@@ -335,7 +366,7 @@ int launch_gemv(const GemvJob *jobs, int count, bitlinear_dtype xdt, const Devic
                 const int blocks = (jobs[i].N + 15) / 16;
                 const double block_bytes = 16.0 * jobs[i].K / 4.0;
                 q[i] = std::max(1, static_cast<int>(target / block_bytes + 0.5));
-                q[i] = std::min(q[i], blocks);
+                q[i] = std::min({q[i], blocks, q_fit});
                 ctas[i] = (blocks + q[i] - 1) / q[i];
                 grid += ctas[i];
             }
@@ -354,10 +385,6 @@ int launch_gemv(const GemvJob *jobs, int count, bitlinear_dtype xdt, const Devic
         stages = std::max(stages, (q[i] * (jobs[i].K / 128) * gemv::PIECE + gemv::STAGE - 1) /
                                       gemv::STAGE);
     }
-    // Each CTA quantises only its own problem's M rows into shared memory.
-    int xq_cap = 0;
-    for (int i = 0; i < count; ++i)
-        xq_cap = std::max(xq_cap, jobs[i].M * jobs[i].K);
     const int acc_cap = qmax * 16 * MT;
     // Ring depth: the whole share when it is small (room for the next
     // kernel's blocks on the same SM under programmatic launch), else as deep
@@ -675,7 +702,6 @@ int check_forward_args(const void *x, int xdt, int64_t M, int64_t K, const void 
     return BITLINEAR_OK;
 }
 
-bool gemv_fits(int64_t M, int64_t K) { return M <= kGemvMaxM && M * K <= kGemvMaxXqBytes; }
 
 int choose_path(int64_t M, int64_t K, int path)
 {
@@ -696,15 +722,15 @@ int forward_impl(const void *x, bitlinear_dtype xdt, int64_t M, int64_t K, const
         return BITLINEAR_ERR_ARG;
     if (M == 0)
         return BITLINEAR_OK;
+    const int chosen = inject_timeout_us > 0 ? BITLINEAR_PATH_TC : choose_path(M, K, path);
+    if (chosen == BITLINEAR_PATH_GEMV && !gemv_fits(M, K))
+        return BITLINEAR_ERR_SHAPE;
     DeviceInfo *dev = nullptr;
     rc = current_device(&dev);
     if (rc != BITLINEAR_OK)
         return rc;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    const int chosen = inject_timeout_us > 0 ? BITLINEAR_PATH_TC : choose_path(M, K, path);
     if (chosen == BITLINEAR_PATH_GEMV) {
-        if (!gemv_fits(M, K))
-            return BITLINEAR_ERR_SHAPE;
         const GemvJob job{x,      static_cast<int>(M), static_cast<int>(K), static_cast<int>(N),
                           packed, gamma, y, acc, xq, beta, norm_gain, norm_eps};
         return launch_gemv(&job, 1, xdt, *dev, st);
@@ -820,6 +846,7 @@ extern "C" int bitlinear_forward_grouped(const bitlinear_problem *problems, int 
         return BITLINEAR_ERR_ARG;
     GemvJob jobs[gemv::MAX_PROBLEMS];
     int n = 0;
+    int64_t max_M = 0, max_xq = 0;
     for (int i = 0; i < count; ++i) {
         const bitlinear_problem &pr = problems[i];
         int rc = check_forward_args(pr.x_dev, xdt, pr.M, pr.K, pr.packed_dev, pr.N, pr.y_dev,
@@ -830,12 +857,17 @@ extern "C" int bitlinear_forward_grouped(const bitlinear_problem *problems, int 
             continue;
         if (!gemv_fits(pr.M, pr.K))
             return BITLINEAR_ERR_SHAPE;
+        max_M = std::max(max_M, pr.M);
+        max_xq = std::max(max_xq, pr.M * pr.K);
         jobs[n++] = GemvJob{pr.x_dev,      static_cast<int>(pr.M), static_cast<int>(pr.K),
                             static_cast<int>(pr.N), pr.packed_dev, pr.gamma, pr.y_dev,
                             nullptr, nullptr, nullptr};
     }
     if (n == 0)
         return BITLINEAR_OK;
+    // one launch holds the largest x~ next to the largest problem's token tile
+    if (max_xq > gemv_max_xq(max_M))
+        return BITLINEAR_ERR_SHAPE;
     DeviceInfo *dev = nullptr;
     int rc = current_device(&dev);
     if (rc != BITLINEAR_OK)
@@ -855,6 +887,7 @@ int collect_group(const bitlinear_problem *problems, int count, int xdt, TcJob *
         return BITLINEAR_ERR_ARG;
     *n = 0;
     *all_gemv = true;
+    int64_t max_M = 0, max_xq = 0;
     static const uint4 dummy = {};   // stands in for the pointers when sizing
     for (int i = 0; i < count; ++i) {
         const bitlinear_problem &pr = problems[i];
@@ -869,9 +902,14 @@ int collect_group(const bitlinear_problem *problems, int count, int xdt, TcJob *
             continue;
         if (!(pr.M <= kAutoGemvMaxM && gemv_fits(pr.M, pr.K)))
             *all_gemv = false;
+        max_M = std::max(max_M, pr.M);
+        max_xq = std::max(max_xq, pr.M * pr.K);
         jobs[(*n)++] = TcJob{pr.x_dev,      static_cast<int>(pr.M), static_cast<int>(pr.K),
                              static_cast<int>(pr.N), pr.packed_dev, pr.gamma, pr.y_dev, nullptr};
     }
+    // one GEMV launch holds the largest x~ next to the largest problem's token tile
+    if (*n > 0 && max_xq > gemv_max_xq(max_M))
+        *all_gemv = false;
     return BITLINEAR_OK;
 }
 

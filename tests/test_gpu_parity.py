@@ -95,6 +95,14 @@ def test_maximum_k_and_single_output_row(cuda, path, M):
         assert c.check_full(c.run(path=path)) == 1.0
 
 
+def test_gemv_tall_matrix_next_to_large_x(cuda):
+    # x~ of 16 x 12160 bytes leaves shared memory for the row accumulators of
+    # only three row blocks per CTA, so the 1499 row blocks (the last one
+    # ragged) take 500 CTAs: more than one wave, the last CTA short
+    c = Case(16, 12160, 23970, w_seed=61, x_seed=62)
+    assert c.check_sampled(c.run(path=bl.PATH_GEMV), count=20000) == 1.0
+
+
 def test_tc_many_tiles_per_cta(cuda):
     # more tiles than SMs: every CTA loops over several tiles and both TMEM
     # accumulator buffers are reused
