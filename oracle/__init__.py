@@ -37,7 +37,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "bitlinear_oracle.c")
 _LIB_PATH = os.path.join(_HERE, "liboracle.so")
 CFLAGS = ["-O2", "-std=c11", "-fPIC", "-shared", "-ffp-contract=off",
-          "-fno-fast-math"]
+          "-fno-fast-math", "-Wall", "-Wextra"]
 
 # nn.RMSNorm's default eps for fp32 inputs: the fp32 machine epsilon
 RMSNORM_EPS = float(np.finfo(np.float32).eps)

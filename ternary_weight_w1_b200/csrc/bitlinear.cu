@@ -861,7 +861,7 @@ extern "C" int bitlinear_forward_grouped(const bitlinear_problem *problems, int 
         max_xq = std::max(max_xq, pr.M * pr.K);
         jobs[n++] = GemvJob{pr.x_dev,      static_cast<int>(pr.M), static_cast<int>(pr.K),
                             static_cast<int>(pr.N), pr.packed_dev, pr.gamma, pr.y_dev,
-                            nullptr, nullptr, nullptr};
+                            nullptr, nullptr, nullptr, nullptr, 0.0f};
     }
     if (n == 0)
         return BITLINEAR_OK;
@@ -905,7 +905,8 @@ int collect_group(const bitlinear_problem *problems, int count, int xdt, TcJob *
         max_M = std::max(max_M, pr.M);
         max_xq = std::max(max_xq, pr.M * pr.K);
         jobs[(*n)++] = TcJob{pr.x_dev,      static_cast<int>(pr.M), static_cast<int>(pr.K),
-                             static_cast<int>(pr.N), pr.packed_dev, pr.gamma, pr.y_dev, nullptr};
+                             static_cast<int>(pr.N), pr.packed_dev, pr.gamma, pr.y_dev, nullptr,
+                             nullptr, 0.0f};
     }
     // one GEMV launch holds the largest x~ next to the largest problem's token tile
     if (*n > 0 && max_xq > gemv_max_xq(max_M))
@@ -948,8 +949,9 @@ extern "C" int bitlinear_forward_grouped_ws(const bitlinear_problem *problems, i
     if (all_gemv) {
         GemvJob g[wsg::MAX_PROBLEMS];
         for (int i = 0; i < n; ++i)
-            g[i] = GemvJob{jobs[i].x, jobs[i].M, jobs[i].K, jobs[i].N, jobs[i].packed,
-                           jobs[i].gamma, jobs[i].y, nullptr, nullptr, nullptr};
+            g[i] = GemvJob{jobs[i].x,     jobs[i].M, jobs[i].K, jobs[i].N, jobs[i].packed,
+                           jobs[i].gamma, jobs[i].y, nullptr,   nullptr,   nullptr,
+                           nullptr,       0.0f};
         return launch_gemv(g, n, xdt, *dev, st);
     }
     return run_tc_group(jobs, n, xdt, workspace_dev, workspace_bytes, nullptr, nullptr, *dev, st,
