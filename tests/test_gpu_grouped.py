@@ -6,20 +6,35 @@ import pytest
 
 import workloads
 import ternary_weight_w1_b200 as bl
-from tests.gpu_cases import Case, check_y, tensor_to_bf16_bits
+from tests.gpu_cases import CANARY_Y, Case, Guarded, check_y, tensor_to_bf16_bits
 
 pytestmark = pytest.mark.gpu
 
 
-def run_group(cases, xs=None):
+def _guarded_problems(cases, xs):
+    """(problems with canary-guarded outputs, the guards)."""
     import torch
-    probs = []
+    probs, guards = [], []
     for i, c in enumerate(cases):
         x = c.x_tensor() if xs is None else xs[i]
-        probs.append((x, c.packed_tensor(), c.gamma, c.N, None))
-    outs = bl.bitlinear_forward_grouped(probs)
+        g = Guarded((c.M, c.N), torch.bfloat16, x.device, CANARY_Y)
+        guards.append(g)
+        probs.append((x, c.packed_tensor(), c.gamma, c.N, g.t))
+    return probs, guards
+
+
+def _read(guards):
+    for i, g in enumerate(guards):
+        g.check(f"problem {i}'s y")
+    return [tensor_to_bf16_bits(g.t) for g in guards]
+
+
+def run_group(cases, xs=None):
+    import torch
+    probs, guards = _guarded_problems(cases, xs)
+    bl.bitlinear_forward_grouped(probs)
     torch.cuda.synchronize()
-    return [tensor_to_bf16_bits(y) for y in outs], probs
+    return _read(guards), probs
 
 
 def test_grouped_mixed_shapes():
@@ -64,15 +79,12 @@ def test_grouped_eight_problems_fp32():
 
 def run_group_ws(cases, xs=None):
     import torch
-    probs = []
-    for i, c in enumerate(cases):
-        x = c.x_tensor() if xs is None else xs[i]
-        probs.append((x, c.packed_tensor(), c.gamma, c.N, None))
+    probs, guards = _guarded_problems(cases, xs)
     need = bl.bitlinear_workspace_bytes_grouped(probs)
     ws = torch.empty((max(need, 1),), dtype=torch.uint8, device="cuda")
-    outs = bl.bitlinear_forward_grouped(probs, workspace=ws)
+    bl.bitlinear_forward_grouped(probs, workspace=ws)
     torch.cuda.synchronize()
-    return [tensor_to_bf16_bits(y) for y in outs]
+    return _read(guards)
 
 
 def test_grouped_tc_mixed_shapes_match_single_calls():
