@@ -298,7 +298,8 @@ int bitlinear_forward_grouped_ws(const bitlinear_problem *problems, int count,
                                  bitlinear_dtype xdt, void *workspace_dev,
                                  size_t workspace_bytes, void *cuda_stream);
 
-/* Workspace bytes for an explicit path (see bitlinear_forward_ex). */
+/* Workspace bytes for an explicit path (see bitlinear_forward_ex); SIZE_MAX
+ * for invalid shapes, including those BITLINEAR_PATH_GEMV cannot take. */
 size_t bitlinear_workspace_bytes_path(int64_t M, int64_t N, int64_t K,
                                       int path);
 

@@ -788,6 +788,8 @@ extern "C" size_t bitlinear_workspace_bytes_path(int64_t M, int64_t N, int64_t K
         return SIZE_MAX;
     if (M == 0)
         return 0;
+    if (path == BITLINEAR_PATH_GEMV && !gemv_fits(M, K))
+        return SIZE_MAX;                          // the GEMV cannot take this shape
     return choose_path(M, K, path) == BITLINEAR_PATH_GEMV ? 0 : tc_workspace_bytes(M, K);
 }
 
