@@ -21,6 +21,7 @@ unless stated):
     |x~| <= 127 with the per-token maximum reaching 127, the rounding bound
     |x~ - x*127/beta| <= 1/2, invariance under power-of-two scaling, and the
     bf16 rounding bound of the output;
+  * the exact widening of every bf16 bit pattern against torch's conversion;
   * for the RMS normalisation ahead of quantisation (the listing's
     nn.RMSNorm member of BitLinear): torch's rms_norm in float64 within the
     fp32 error bound, constant rows in closed form, exact invariance under
@@ -317,6 +318,24 @@ def pin_bf16_rounding_vs_torch(orc):
     assert np.isnan(_bf16_value(nan_bits))[0]
 
 
+def pin_bf16_widening_vs_torch(orc):
+    """Every one of the 65,536 bf16 bit patterns widens to the fp32 value
+    torch's bf16 -> fp32 conversion gives, bit for bit (NaNs by class: any
+    NaN for a NaN). The listing's quantiser takes the activations in their
+    input dtype, so this widening is where every bf16 token enters the path."""
+    import torch
+    bits = np.arange(1 << 16, dtype=np.uint32).astype(np.uint16)
+    got = orc.bf16_to_f32(bits)
+    ref = torch.from_numpy(bits.view(np.int16).copy()).view(torch.bfloat16).float().numpy()
+    nan = np.isnan(ref)
+    assert np.array_equal(np.isnan(got), nan)
+    np.testing.assert_array_equal(got[~nan].view(np.uint32), ref[~nan].view(np.uint32))
+    # a few values by hand: 1.0, -2.0, the smallest subnormal, -0, +inf
+    hand = np.array([0x3F80, 0xC000, 0x0001, 0x8000, 0x7F80], dtype=np.uint16)
+    want = np.array([1.0, -2.0, 2.0 ** -133, -0.0, np.inf], dtype=np.float32)
+    np.testing.assert_array_equal(orc.bf16_to_f32(hand).view(np.uint32), want.view(np.uint32))
+
+
 def pin_rescale_bound(orc):
     r = np.random.Generator(np.random.PCG64(61))
     acc = r.integers(-3_000_000, 3_000_000, size=(5, 70)).astype(np.int32)
@@ -493,6 +512,7 @@ ALL_PINS = [
     pin_quant_act_invariants,
     pin_quant_act_pow2_invariance,
     pin_bf16_rounding_vs_torch,
+    pin_bf16_widening_vs_torch,
     pin_rescale_bound,
     pin_listing_semantics_torch,
     pin_rmsnorm_vs_torch_f64,

@@ -35,6 +35,12 @@ MUTANTS = {
     "rescale_divides_acc": ("(float)acc[m * N + n] * s", "(float)acc[m * N + n] / s"),
     "bf16_ties_away": ("(dropped == 0x8000u && (kept & 1u))", "(dropped == 0x8000u)"),
     "bf16_truncates": ("kept += 1u;", "kept += 0u;"),
+    "bf16_widen_stray_low_bit": ("uint32_t bits = (uint32_t)in[i] << 16;",
+                                 "uint32_t bits = ((uint32_t)in[i] << 16) | 0x8000u;"),
+    "bf16_widen_shift_15": ("uint32_t bits = (uint32_t)in[i] << 16;",
+                            "uint32_t bits = (uint32_t)in[i] << 15;"),
+    "bf16_widen_drops_sign": ("uint32_t bits = (uint32_t)in[i] << 16;",
+                              "uint32_t bits = ((uint32_t)in[i] & 0x7fffu) << 16;"),
     "pack_swaps_j_b": ("<< (8 * b + 2 * j)", "<< (8 * j + 2 * b)"),
     "pack_code_negated": ("(uint32_t)(v + 1)", "(uint32_t)(1 - v)"),
     "pack_word_index": ("16 * w + 4 * j + b;", "16 * w + 4 * b + j;"),
