@@ -521,18 +521,27 @@ def bench_large_sweep(bl, device, ms_list=(1, 16, 256, 4096), reps: int = 5):
     return out
 
 
-def cpu_baseline_oracle(seconds: float = 10.0):
-    """The oracle (single-threaded C) on the decode step: x quantisation,
-    integer product and rescale for the up and down projections, repeated
-    for about `seconds`. Returns (GB/s of packed-weight bytes, steps)."""
-    import oracle
-    orc = oracle.default()
-    mats = []
-    for p in workloads.decode_gemv_2b(1).problems:
-        W = p.weights()
-        g = orc.absmean_gamma(W)
-        mats.append((p, orc.ternarize(W, g), g, orc.bf16_to_f32(p.x_input())))
-    nbytes = sum(p.N * p.K // 4 for p, *_ in mats)
+def cpu_info():
+    """(CPU model name, logical cores available to this process)."""
+    model = "unknown"
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    try:
+        cores = len(os.sched_getaffinity(0))
+    except (AttributeError, OSError):
+        cores = os.cpu_count() or 1
+    return model, cores
+
+
+def _oracle_decode_rate(orc, mats, seconds):
+    """Full decode steps (quantise, integer product, rescale of both
+    projections) of one oracle build for about `seconds`: (steps, seconds)."""
     t0 = time.perf_counter()
     steps = 0
     while True:
@@ -543,8 +552,77 @@ def cpu_baseline_oracle(seconds: float = 10.0):
         steps += 1
         el = time.perf_counter() - t0
         if el >= seconds:
-            break
-    return nbytes * steps / el / 1e9, steps, el
+            return steps, el
+
+
+def _oracle_forward_us(orc, problems):
+    """Microseconds of one oracle forward over each prepared problem, summed.
+    A problem prepared on a sample of its tokens or weight rows is scaled to
+    its full M and N (an extrapolation; the time is linear in both)."""
+    total = 0.0
+    for p, Wq, g, xf in problems:
+        t0 = time.perf_counter()
+        xq, beta = orc.quant_act(xf)
+        acc = orc.matmul_i32(xq, Wq)
+        orc.rescale_bf16(acc, beta, g)
+        el = time.perf_counter() - t0
+        total += el * (p.M / xf.shape[0]) * (p.N / Wq.shape[0])
+    return total * 1e6
+
+
+def cpu_baseline_oracle(seconds: float = 10.0):
+    """The oracle (plain C) on the host cores: the headline is the
+    single-threaded build on full decode steps (both projections, M = 1) for
+    about `seconds`; the same steps run on the OpenMP build over all cores
+    for half as long; and one forward per workload with each build (the
+    prefill and M = 4096 times extrapolated from a token sample, as labelled).
+    Returns the cpu_baseline dict."""
+    import oracle
+    one = oracle.default()
+    omp = oracle.Oracle(oracle.load_omp())
+    model, cores = cpu_info()
+
+    def prep(problems, tokens=None, row_div=1):
+        """Oracle inputs of each problem: every weight row, or the first
+        N / row_div of them (seeded latents of that many rows), and every
+        token or the first `tokens`."""
+        out = []
+        for p in problems:
+            W = workloads.latent_weights(p.N // row_div, p.K, p.w_seed)
+            g = one.absmean_gamma(W)
+            xf = one.bf16_to_f32(workloads.to_bf16_bits(
+                workloads.activations_f32(tokens or p.M, p.K, p.x_seed)))
+            out.append((p, one.ternarize(W, g), g, xf))
+        return out
+
+    dec = prep(workloads.decode_gemv_2b(1).problems)
+    nbytes = sum(p.N * p.K // 4 for p, *_ in dec)
+    steps1, el1 = _oracle_decode_rate(one, dec, seconds)
+    stepsn, eln = _oracle_decode_rate(omp, dec, seconds / 2)
+    layer = prep(workloads.layer_set_2b(1, layers=1).problems)
+    pre = prep(workloads.prefill_2b(2048).problems, tokens=16)
+    big1 = prep(workloads.large_sweep(1).problems, row_div=8)
+    per_config = {}
+    for name, probs, label in (
+            ("decode_2b_m1_us_per_step", dec, "measured"),
+            ("layer_2b_b1_us_per_layer", layer, "measured"),
+            ("prefill_2b_m2048_us_per_step", pre, "extrapolated from 16 of the 2048 tokens"),
+            ("large_m1_us_per_pair", big1, "extrapolated from 1/8 of the weight rows")):
+        per_config[name] = {"one_thread": round(_oracle_forward_us(one, probs), 1),
+                            "all_cores": round(_oracle_forward_us(omp, probs), 1),
+                            "how": label}
+    v1 = nbytes * steps1 / el1 / 1e9
+    vn = nbytes * stepsn / eln / 1e9
+    return {"value": round(v1, 4), "unit": UNIT, "cores": 1, "kind": "oracle",
+            "sample": f"{steps1} full decode steps (up+down, M=1) of the single-threaded "
+                      f"C oracle in {el1:.1f} s",
+            "cpu_model": model, "nproc": cores,
+            "all_cores": {"value": round(vn, 4), "unit": UNIT, "cores": cores,
+                          "kind": "oracle-omp",
+                          "sample": f"{stepsn} full decode steps of the same oracle built with "
+                                    f"-fopenmp (integer products over all {cores} cores) in "
+                                    f"{eln:.1f} s"},
+            "per_config": per_config}
 
 
 def run_ours(args, dist):
@@ -660,10 +738,7 @@ def run_ours(args, dist):
             "workload": "K=8192->N=28672 and K=28672->N=8192 per step, 117 MB of packed weights",
             **bench_large_sweep(bl, device)}
     if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
-        v, steps, el = cpu_baseline_oracle(args.cpu_seconds)
-        out["cpu_baseline"] = {"value": round(v, 4), "unit": UNIT, "cores": 1, "kind": "oracle",
-                               "sample": f"{steps} full decode steps (up+down, M=1) of the "
-                                         f"single-threaded C oracle in {el:.1f} s"}
+        out["cpu_baseline"] = cpu_baseline_oracle(args.cpu_seconds)
     return out
 
 

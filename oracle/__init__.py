@@ -36,6 +36,8 @@ import numpy as np
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "bitlinear_oracle.c")
 _LIB_PATH = os.path.join(_HERE, "liboracle.so")
+# the same source built with -fopenmp: the benchmark's all-core CPU baseline
+_OMP_LIB_PATH = os.path.join(_HERE, "liboracle_omp.so")
 CFLAGS = ["-O2", "-std=c11", "-fPIC", "-shared", "-ffp-contract=off",
           "-fno-fast-math", "-Wall", "-Wextra"]
 
@@ -81,6 +83,28 @@ def _declare(lib):
     lib.oracle_pack_codes.restype = ctypes.c_int
     lib.oracle_pack_codes.argtypes = [p, c_i64, c_i64, p]
     return lib
+
+
+def build_omp() -> str:
+    """The same C source compiled with -fopenmp (integer products over all
+    cores). Only the benchmark's CPU baseline uses it; the tests check that it
+    gives the single-threaded build's results."""
+    return build(_SRC, _OMP_LIB_PATH, extra_flags=("-fopenmp",))
+
+
+_omp_lib = None
+
+
+def load_omp():
+    """Load (building first if needed) the OpenMP build of the oracle."""
+    global _omp_lib
+    with _lock:
+        if _omp_lib is None:
+            if (not os.path.exists(_OMP_LIB_PATH) or
+                    os.path.getmtime(_OMP_LIB_PATH) < os.path.getmtime(_SRC)):
+                build_omp()
+            _omp_lib = _declare(ctypes.CDLL(_OMP_LIB_PATH))
+    return _omp_lib
 
 
 def load(path: str | None = None):

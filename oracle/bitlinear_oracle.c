@@ -38,6 +38,8 @@
  * (see the layout comment above oracle_pack_codes), not from the library.
  *
  * Build: gcc -O2 -std=c11 -fPIC -shared -ffp-contract=off -fno-fast-math
+ * (plus -fopenmp for the all-core copy that only the benchmark's CPU baseline
+ * times: the integer products' independent outputs then run on all cores)
  */
 #include <math.h>
 #include <stdint.h>
@@ -162,6 +164,11 @@ void oracle_quant_act(const float *x, int64_t M, int64_t K, int8_t *xq,
 void oracle_matmul_i32(const int8_t *xq, const int8_t *Wq, int64_t M,
                        int64_t N, int64_t K, int32_t *acc)
 {
+    /* Built with -fopenmp (the all-core CPU baseline only), the independent
+     * outputs are shared between threads; each is still the same plain sum. */
+#ifdef _OPENMP
+#pragma omp parallel for collapse(2) schedule(static)
+#endif
     for (int64_t m = 0; m < M; ++m) {
         for (int64_t n = 0; n < N; ++n) {
             int64_t s = 0;
@@ -178,6 +185,9 @@ void oracle_matmul_i32_pairs(const int8_t *xq, const int8_t *Wq, int64_t K,
                              const int64_t *ms, const int64_t *ns,
                              int64_t count, int32_t *acc)
 {
+#ifdef _OPENMP
+#pragma omp parallel for schedule(static)
+#endif
     for (int64_t i = 0; i < count; ++i) {
         const int8_t *a = xq + ms[i] * K;
         const int8_t *w = Wq + ns[i] * K;

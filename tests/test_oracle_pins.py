@@ -35,3 +35,20 @@ def test_forward_normalises_before_quantising(orc):
     res16 = orc.forward(bits, W, norm_gain=g)
     np.testing.assert_array_equal(res16["xq"], orc.quant_act(orc.rmsnorm(orc.bf16_to_f32(bits), g))[0])
     np.testing.assert_array_equal(orc.forward(x, W)["xq"], orc.quant_act(x)[0])
+
+
+def test_openmp_build_gives_the_same_products(orc):
+    """The all-core copy of the oracle (the same source built with -fopenmp,
+    timed only by the benchmark's CPU baseline) computes the same integer
+    products as the single-threaded build: each output is the same plain sum,
+    only the outputs are shared between threads."""
+    import numpy as np
+    omp = oracle.Oracle(oracle.load_omp())
+    r = np.random.Generator(np.random.PCG64(85))
+    xq = r.integers(-127, 128, size=(5, 1280)).astype(np.int8)
+    Wq = r.integers(-1, 2, size=(333, 1280)).astype(np.int8)
+    np.testing.assert_array_equal(omp.matmul_i32(xq, Wq), orc.matmul_i32(xq, Wq))
+    ms = r.integers(0, 5, 999)
+    ns = r.integers(0, 333, 999)
+    np.testing.assert_array_equal(omp.matmul_i32_pairs(xq, Wq, ms, ns),
+                                  orc.matmul_i32_pairs(xq, Wq, ms, ns))
