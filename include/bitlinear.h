@@ -346,16 +346,7 @@ int bitlinear_get_fault(int *fault_out, void *cuda_stream);
 /* Human-readable name of a bitlinear_status. Never NULL. */
 const char *bitlinear_status_string(int status);
 
-/* --------------------------------------------------------- measurement aids */
-
-/* Plain int8 x int8 -> int32 GEMM C[M][N] = A[M][K] B[N][K]^T on the same
- * tcgen05 pipeline as the forward GEMM, with B already int8 (no unpacking).
- * It has no counterpart on the pages: it measures the int8 tensor-core
- * roofline the forward GEMM is reported against. A, B: int8 row-major,
- * 16-byte aligned; C: int32 [M][N]. K % 128 == 0. */
-int bitlinear_int8_gemm(const int8_t *A_dev, const int8_t *B_dev,
-                        int32_t *C_dev, int64_t M, int64_t N, int64_t K,
-                        void *cuda_stream);
+/* ------------------------------------------------- failure-detection aids */
 
 /* The forward tensor-core GEMM with one wait made to run out on purpose:
  * the MMA issuer waits on a barrier nobody arrives at, for timeout_us

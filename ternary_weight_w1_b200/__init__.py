@@ -57,7 +57,6 @@ EXPORTS = (
     "bitlinear_forward_rmsnorm",
     "bitlinear_get_fault",
     "bitlinear_status_string",
-    "bitlinear_int8_gemm",
     "bitlinear_forward_inject_timeout",
     "bitlinear_forward_noalloc",
     "bitlinear_forward_grouped",
@@ -130,8 +129,6 @@ def lib() -> ctypes.CDLL:
         L.bitlinear_get_fault.argtypes = [p, p]
         L.bitlinear_status_string.restype = ctypes.c_char_p
         L.bitlinear_status_string.argtypes = [ctypes.c_int]
-        L.bitlinear_int8_gemm.restype = ctypes.c_int
-        L.bitlinear_int8_gemm.argtypes = [p, p, p, i64, i64, i64, p]
         _lib = L
     return _lib
 
@@ -373,20 +370,6 @@ def bitlinear_get_fault(stream=None) -> tuple[int, int]:
     word = ctypes.c_int(0)
     rc = lib().bitlinear_get_fault(ctypes.addressof(word), _stream(stream))
     return int(rc), int(word.value)
-
-
-def bitlinear_int8_gemm(A, B, C=None, stream=None):
-    """C (int32 [M][N]) = A (int8 [M][K]) @ B (int8 [N][K])^T on the tensor cores."""
-    a = _Args()
-    import torch
-    M, K = A.shape
-    N = B.shape[0]
-    if C is None:
-        C = torch.empty((M, N), dtype=torch.int32, device=A.device)
-    _check(lib().bitlinear_int8_gemm(a.ptr(A, "A", torch.int8, (M, K)), a.ptr(B, "B", torch.int8, (N, K)),
-                                     a.ptr(C, "C", torch.int32, (M, N)), M, N, K, _stream(stream)),
-           "bitlinear_int8_gemm")
-    return C
 
 
 def bitlinear_forward_noalloc(x, packed, gamma: float, N: int, y=None, stream=None):

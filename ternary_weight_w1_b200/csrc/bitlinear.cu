@@ -19,7 +19,6 @@
 
 #include "../../include/bitlinear.h"
 #include "common.cuh"
-#include "gemm_tc.cuh"
 #include "gemm_ws.cuh"
 #include "gemv.cuh"
 #include "quant_act.cuh"
@@ -121,24 +120,6 @@ EncodeTiledFn encode_fn()
         return reinterpret_cast<EncodeTiledFn>(p);
     }();
     return fn;
-}
-
-// 2-D uint8 tensor [rows][cols] (cols contiguous), box [box_rows][box_cols].
-bool make_map_u8(CUtensorMap *map, const void *ptr, uint64_t rows, uint64_t cols,
-                 uint32_t box_rows, uint32_t box_cols, bool swizzle128)
-{
-    EncodeTiledFn fn = encode_fn();
-    if (fn == nullptr)
-        return false;
-    const cuuint64_t dims[2] = {cols, rows};
-    const cuuint64_t strides[1] = {cols};
-    const cuuint32_t box[2] = {box_cols, box_rows};
-    const cuuint32_t estride[2] = {1, 1};
-    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(ptr), dims, strides,
-                    box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                    swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
-                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS;
 }
 
 // Programmatic dependent launch: a kernel launched this way may start while
@@ -476,19 +457,6 @@ size_t tc_group_bytes(const TcJob *jobs, int n, bool split)
         max_M = std::max(max_M, jobs[i].M);
     }
     return b + (split ? tc_split_bytes(max_M) : 0);
-}
-
-int launch_int8_gemm(const CUtensorMap &ma, const CUtensorMap &mb, const tc::Params &p,
-                     const DeviceInfo &dev, cudaStream_t st)
-{
-    cudaError_t e = allow_smem<tc::gemm_kernel>(dev.id, tc::SMEM_BYTES);
-    if (e != cudaSuccess)
-        return launch_status(e);
-    const int tiles = ((p.M + tc::BM - 1) / tc::BM) * ((p.N + tc::BN - 1) / tc::BN);
-    const int grid = std::min(tiles, dev.sms);
-    e = launch(tc::gemm_kernel, dim3(grid), dim3(tc::THREADS), static_cast<size_t>(tc::SMEM_BYTES),
-               st, ma, mb, p);
-    return launch_status(e);
 }
 
 template <int BT>
@@ -990,32 +958,6 @@ extern "C" int bitlinear_get_fault(int *fault_out, void *cuda_stream)
         return BITLINEAR_ERR_TIMEOUT;
     }
     return BITLINEAR_OK;
-}
-
-extern "C" int bitlinear_int8_gemm(const int8_t *A_dev, const int8_t *B_dev, int32_t *C_dev,
-                                   int64_t M, int64_t N, int64_t K, void *cuda_stream)
-{
-    if (M < 0 || N < 1 || K < 1)
-        return BITLINEAR_ERR_ARG;
-    if (M > 0 && (A_dev == nullptr || B_dev == nullptr || C_dev == nullptr))
-        return BITLINEAR_ERR_ARG;
-    if (K % 128 != 0 || M > INT_MAX / 2 || N > INT_MAX / 2 || K > (int64_t(1) << 30))
-        return BITLINEAR_ERR_SHAPE;
-    if (!aligned(A_dev, 16) || !aligned(B_dev, 16) || !aligned(C_dev, 16))
-        return BITLINEAR_ERR_ALIGN;
-    if (M == 0)
-        return BITLINEAR_OK;
-    DeviceInfo *dev = nullptr;
-    int rc = current_device(&dev);
-    if (rc != BITLINEAR_OK)
-        return rc;
-    CUtensorMap ma, mb;
-    if (!make_map_u8(&ma, A_dev, M, K, tc::BM, tc::BK, true) ||
-        !make_map_u8(&mb, B_dev, N, K, tc::BN, tc::BK, true))
-        return BITLINEAR_ERR_CUDA;
-    tc::Params p{static_cast<int>(M), static_cast<int>(N), static_cast<int>(K), C_dev,
-                 kWaitLimitNs};
-    return launch_int8_gemm(ma, mb, p, *dev, static_cast<cudaStream_t>(cuda_stream));
 }
 
 // ======================================================== no-allocation path

@@ -169,13 +169,6 @@ def test_quant_act_rejects_bad_arguments():
     assert L.bitlinear_quant_act(FAKE, 0, 0, 256, FAKE, FAKE, None) == bl.BITLINEAR_OK
 
 
-def test_int8_gemm_rejects_bad_arguments():
-    L = bl.lib()
-    assert L.bitlinear_int8_gemm(None, FAKE, FAKE, 4, 4, 128, None) == bl.BITLINEAR_ERR_ARG
-    assert L.bitlinear_int8_gemm(FAKE, FAKE, FAKE, 4, 4, 100, None) == bl.BITLINEAR_ERR_SHAPE
-    assert L.bitlinear_int8_gemm(FAKE, FAKE, FAKE + 4, 4, 4, 128, None) == bl.BITLINEAR_ERR_ALIGN
-
-
 def test_inject_timeout_rejects_bad_limit():
     L = bl.lib()
     rc = L.bitlinear_forward_inject_timeout(FAKE, 0, 1, 256, FAKE, 1.0, 64, FAKE, FAKE, 4096,
@@ -265,7 +258,3 @@ def test_binding_refuses_host_tensors():
         bl.bitlinear_forward_rmsnorm(x, packed, 1.0, 64, torch.ones(256),
                                      y=torch.zeros((4, 64), dtype=torch.bfloat16),
                                      path=bl.PATH_GEMV)
-    with pytest.raises(ValueError, match="CUDA tensor"):
-        bl.bitlinear_int8_gemm(torch.zeros((128, 128), dtype=torch.int8),
-                               torch.zeros((128, 128), dtype=torch.int8),
-                               torch.zeros((128, 128), dtype=torch.int32))

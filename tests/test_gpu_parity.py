@@ -217,20 +217,6 @@ def test_large_sweep(cuda, M):
             assert c.check_sampled(got, count=20000) == 1.0
 
 
-# ------------------------------------------------- int8 GEMM (measurement aid)
-
-@pytest.mark.parametrize("M,N,K", [(300, 600, 512), (128, 256, 128), (1000, 2000, 1280)])
-def test_int8_gemm(cuda, M, N, K):
-    torch = cuda
-    r = np.random.Generator(np.random.PCG64(M + N + K))
-    A = r.integers(-128, 128, (M, K), dtype=np.int8)
-    B = r.integers(-128, 128, (N, K), dtype=np.int8)
-    C = bl.bitlinear_int8_gemm(torch.from_numpy(A).cuda(), torch.from_numpy(B).cuda())
-    torch.cuda.synchronize()
-    ref = A.astype(np.int64) @ B.astype(np.int64).T
-    np.testing.assert_array_equal(C.cpu().numpy().astype(np.int64), ref)
-
-
 # ------------------------------------------------- failure detection
 
 def test_bounded_wait_reports_timeout_and_context_survives(cuda):

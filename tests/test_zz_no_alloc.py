@@ -47,11 +47,24 @@ def test_noalloc_matches_workspace_path_twice():
     assert bl.bitlinear_get_fault() == (bl.BITLINEAR_OK, 0)
 
 
-def test_noalloc_rejects_problems_beyond_the_scratch():
+def test_noalloc_fills_the_scratch_exactly_and_rejects_beyond_it():
+    """M = 2424 tokens of K = 6912 fill the 16 MiB array to its last bytes
+    (x~, beta and the row sums of x~); on seeded nonzero data the result must
+    equal the workspace path's bit for bit. One more token is refused before
+    any device work."""
     import torch
-    x = torch.zeros((2425, 6912), dtype=torch.bfloat16, device="cuda")
-    packed = torch.zeros((64, 6912 // 4), dtype=torch.uint8, device="cuda")
-    y = torch.empty((2425, 64), dtype=torch.bfloat16, device="cuda")
-    assert call_noalloc(x, packed, 1.0, 64, y) == bl.BITLINEAR_ERR_SCRATCH_LIMIT
-    assert call_noalloc(x[:2424], packed, 1.0, 64, y[:2424]) == bl.BITLINEAR_OK
+    c = Case(2424, 6912, 80, w_seed=25, x_seed=26)
+    x, packed = c.x_tensor(), c.packed_tensor()
+    y_ref = torch.empty((c.M, c.N), dtype=torch.bfloat16, device="cuda")
+    bl.bitlinear_forward(x, packed, c.gamma, c.N, y=y_ref, path=bl.PATH_TC)
+    y = torch.full((c.M, c.N), float("nan"), dtype=torch.bfloat16, device="cuda")
+    assert call_noalloc(x, packed, c.gamma, c.N, y) == bl.BITLINEAR_OK
     torch.cuda.synchronize()
+    got, ref = tensor_to_bf16_bits(y), tensor_to_bf16_bits(y_ref)
+    check_y(got, ref)
+    np.testing.assert_array_equal(got, ref)
+    assert bl.bitlinear_get_fault() == (bl.BITLINEAR_OK, 0)
+
+    x1 = torch.zeros((2425, 6912), dtype=torch.bfloat16, device="cuda")
+    y1 = torch.empty((2425, 80), dtype=torch.bfloat16, device="cuda")
+    assert call_noalloc(x1, packed, c.gamma, 80, y1) == bl.BITLINEAR_ERR_SCRATCH_LIMIT
