@@ -448,6 +448,42 @@ def bench_rmsnorm_decode(bl, wl, reps: int = 200) -> float:
     return time_graph(steps, reps, nvtx="rmsnorm_decode_timed") / ROTATE
 
 
+def bench_ffn(bl, device, batches=(1, 8), copies: int = 16, reps: int = 20):
+    """The 2B decoder's feed-forward block (gate and up 2560 -> 6912, the
+    gated ReLU^2, down 6912 -> 2560) for B decode tokens through
+    bitlinear_ffn_forward: one GEMV launch for gate and up with h written
+    from its epilogue, one launch (pair) for down. The three matrices (13.3 MB
+    packed) rotate over `copies` device copies (212 MB > L2). Per B:
+    microseconds per block and GB/s of packed weights."""
+    import torch
+    K, F = 2560, 6912
+    mats = []
+    for seed, (n, k) in zip((7001, 7002, 7003), ((F, K), (F, K), (K, F))):
+        pk, gamma = bl.bitlinear_pack_weights(workloads.latent_weights(n, k, seed))
+        dp = torch.from_numpy(pk).to(device)
+        mats.append(([dp] + [dp.clone() for _ in range(copies - 1)], gamma))
+    wbytes = 3 * F * K // 4
+    out = {}
+    for B in batches:
+        x = bf16_tensor(workloads.activations_bf16(B, K, 7004), device)
+        h = torch.empty((B, F), dtype=torch.float32, device=device)
+        y = torch.empty((B, K), dtype=torch.bfloat16, device=device)
+        need = bl.bitlinear_workspace_bytes_ffn(B, K, F)
+        ws = torch.empty((max(need, 1),), dtype=torch.uint8, device=device)
+
+        def steps():
+            for c in range(copies):
+                bl.bitlinear_ffn_forward(x, *[(m[0][c], m[1]) for m in mats], h=h, y=y,
+                                         workspace=ws)
+        steps()
+        torch.cuda.synchronize()
+        ms = time_graph(steps, reps, nvtx=f"ffn_b{B}_timed") / copies
+        out[f"B={B}"] = {"us_per_block": round(ms * 1e3, 2),
+                         "GBps_packed": round(wbytes / (ms * 1e-3) / 1e9, 1),
+                         "launches_per_block": 2 if need == 0 else 3}
+    return out
+
+
 def bench_layer_set(bl, device, batches=(1, 8, 64), reps: int = 10):
     """The seven projections of the 2B decoder layer for 30 layers (521 MB of
     packed weights, more than four times L2) at decode batch B, one grouped
@@ -513,7 +549,7 @@ def bench_large_sweep(bl, device, ms_list=(1, 16, 256, 4096), reps: int = 5):
                     bl.bitlinear_forward(xs[k], dps[c], g, p.N, y=ys[k], workspace=ws)
         step()
         torch.cuda.synchronize()
-        ms = time_graph(step, reps) / 3
+        ms = time_graph(step, reps, nvtx=f"large_m{M}_timed") / 3
         out[f"M={M}"] = {"us_per_pair": round(ms * 1e3, 2),
                          "GBps_packed": round(wbytes / (ms * 1e-3) / 1e9, 1),
                          "TOPS": round(2 * M * wbytes * 4 / (ms * 1e-3) / 1e12, 1)}
@@ -661,6 +697,8 @@ def run_ours(args, dist):
 
     if args.layer_set_only:
         return {"layer_set": bench_layer_set(bl, device)}
+    if args.large_only:
+        return {"large_sweep": bench_large_sweep(bl, device, ms_list=(1,))}
     if args.decode_only:
         return {"decode_only": {"value": round(value, 2), "unit": UNIT,
                                 "ms_per_step": ms / args.steps, "steps": args.steps,
@@ -730,6 +768,11 @@ def run_ours(args, dist):
                               "frac": round(norm_pre_tops / int8_peak, 4)}},
     }
     if not args.no_extra:
+        out["ffn_chain"] = {
+            "workload": "2B feed-forward block: gate and up 2560->6912 (one GEMV launch, h = "
+                        "max(gate,0)^2 * up written from its epilogue), down 6912->2560 on h; "
+                        "13.3 MB of packed weights per block",
+            **bench_ffn(bl, device)}
         out["layer_set"] = {
             "workload": "2B decoder layer (q 2560->2560, k/v 2560->640, o 2560->2560, gate/up "
                         "2560->6912, down 6912->2560) x 30 layers, 521 MB of packed weights",
@@ -797,6 +840,9 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extra", action="store_true",
                     help="skip the layer-set and large-shape measurements")
+    ap.add_argument("--large-only", action="store_true",
+                    help="only the large-shape M = 1 measurement after the decode step "
+                         "(for profiling)")
     ap.add_argument("--decode-only", action="store_true",
                     help="only the decode step (headline) measurements (for profiling)")
     ap.add_argument("--layer-set-only", action="store_true",

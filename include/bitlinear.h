@@ -202,11 +202,9 @@ int bitlinear_forward(const void *x_dev, bitlinear_dtype xdt, int64_t M,
 
 /* bitlinear_forward with an explicit kernel choice (bitlinear_path).
  * BITLINEAR_PATH_GEMV needs M <= 16 and the tokens' x~ (M * K bytes) within
- * the GEMV's shared-memory limit: 196608 bytes for M <= 8, 196272 for
- * M = 9..16; otherwise it returns BITLINEAR_ERR_SHAPE, before any device
- * work. For matrices so tall that their per-CTA row accumulators would not
- * fit beside a large x~, the GEMV gives each CTA fewer row blocks and runs
- * in more than one wave. The workspace for BITLINEAR_PATH_TC is
+ * the GEMV's shared-memory limit of 196608 bytes; otherwise it returns
+ * BITLINEAR_ERR_SHAPE, before any device work. Beside a large x~ the GEMV
+ * streams its weights in smaller stages. The workspace for BITLINEAR_PATH_TC is
  * bitlinear_workspace_bytes_path(M, N, K, BITLINEAR_PATH_TC). */
 int bitlinear_forward_ex(const void *x_dev, bitlinear_dtype xdt, int64_t M,
                          int64_t K, const void *packed_dev, float gamma,
@@ -241,6 +239,65 @@ int bitlinear_forward_rmsnorm(const void *x_dev, bitlinear_dtype xdt, int64_t M,
                               void *cuda_stream, int32_t *acc_dev_or_null,
                               int8_t *xq_dev_or_null, float *beta_dev_or_null,
                               int path);
+
+/* ----------------------------------------------------- feed-forward chain */
+
+/* Device workspace bytes bitlinear_ffn_forward needs: that of its down
+ * projection (M tokens of F features to K), i.e.
+ * bitlinear_workspace_bytes(M, K, F); 0 when that projection takes the GEMV
+ * path. SIZE_MAX for shapes bitlinear_ffn_forward refuses. */
+size_t bitlinear_workspace_bytes_ffn(int64_t M, int64_t K, int64_t F);
+
+/* The feed-forward block of a BitNet b1.58 decoder layer for M decode tokens:
+ *   gate = BitLinear_gate(x), up = BitLinear_up(x)        ([M][F], bf16)
+ *   h    = (r * r) * up,  r = max(gate, 0)                 ([M][F], fp32)
+ *   y    = BitLinear_down(h)                               ([M][K], bf16)
+ * ReLU^2 replaces SwiGLU in the model's feed-forward networks ("Microsoft
+ * Releases BitNet b1.58 2B4T", section "Under the Hood"; "BitNet b1.58: The
+ * 1-Bit Paradigm Shift"), read here as gated: the squared ReLU of the gate
+ * projection multiplies the up projection elementwise. h is computed in
+ * fp32 from the two bf16 outputs (exact: every product of bf16 values fits
+ * fp32). Each BitLinear is the one of bitlinear_forward (its own gamma); with
+ * gains, each RMS-normalises its input first as bitlinear_forward_rmsnorm
+ * does (the listing's per-BitLinear nn.RMSNorm).
+ * Two launches on cuda_stream: one GEMV launch streams the gate and up
+ * weights together (a CTA holds the same rows of both), applies the
+ * quantised tokens to both and writes h from its epilogue; then the down
+ * projection runs on h as bitlinear_forward_rmsnorm (or bitlinear_forward
+ * without a down gain) does, GEMV or tensor cores by M.
+ *   x_dev           [in]  [M][K] activations of type xdt
+ *   M, K, F         [in]  tokens, d_model, d_ff; K and F positive multiples
+ *                         of 128, at most 65536; M <= 16 and M * K (2 M K
+ *                         with gate/up gains) <= 196608 (the gate/up
+ *                         launch is the GEMV), else BITLINEAR_ERR_SHAPE
+ *   gate_packed_dev, gate_gamma, up_packed_dev, up_gamma
+ *                   [in]  F x K packed weights and their gammas
+ *   down_packed_dev, down_gamma
+ *                   [in]  K x F packed weights and gamma
+ *   gate_gain_dev, up_gain_dev
+ *                   [in]  [K] fp32 RMSNorm gains, both or neither (NULL:
+ *                         no normalisation), 16-byte aligned
+ *   down_gain_dev   [in]  [F] fp32 gains of the down projection, or NULL
+ *   norm_eps        [in]  eps of the normalisations (finite, > 0) when any
+ *                         gain is given; ignored otherwise
+ *   h_dev           [out] [M][F] fp32, 16-byte aligned (the down input)
+ *   y_dev           [out] [M][K] bf16
+ *   workspace_dev, workspace_bytes
+ *                   [in]  scratch of bitlinear_workspace_bytes_ffn(M, K, F)
+ *                         bytes (may be NULL when that is 0)
+ *   gate_y_dev_or_null, up_y_dev_or_null
+ *                   [out, optional] [M][F] bf16 gate and up outputs
+ * Errors as for bitlinear_forward, all reported before any launch. */
+int bitlinear_ffn_forward(const void *x_dev, bitlinear_dtype xdt, int64_t M,
+                          int64_t K, int64_t F, const void *gate_packed_dev,
+                          float gate_gamma, const void *up_packed_dev,
+                          float up_gamma, const void *down_packed_dev,
+                          float down_gamma, const float *gate_gain_dev,
+                          const float *up_gain_dev, const float *down_gain_dev,
+                          float norm_eps, float *h_dev, void *y_dev,
+                          void *workspace_dev, size_t workspace_bytes,
+                          void *cuda_stream, void *gate_y_dev_or_null,
+                          void *up_y_dev_or_null);
 
 /* One problem of bitlinear_forward_grouped. */
 typedef struct {
@@ -348,18 +405,24 @@ const char *bitlinear_status_string(int status);
 
 /* ------------------------------------------------- failure-detection aids */
 
-/* The forward tensor-core GEMM with one wait made to run out on purpose:
- * the MMA issuer waits on a barrier nobody arrives at, for timeout_us
- * microseconds, then the kernel records a fault and every role returns.
- * Used by the failure-detection test; inputs as for bitlinear_forward_ex
- * with BITLINEAR_PATH_TC. */
+/* A forward with one wait made to run out on purpose, for the
+ * failure-detection test. path selects the kernel (BITLINEAR_PATH_GEMV or
+ * BITLINEAR_PATH_TC; anything else is BITLINEAR_ERR_ARG):
+ *   - GEMV: the weight producer leaves the first stage unloaded, so the
+ *     compute warps' first wait gives up after timeout_us microseconds;
+ *   - TC: the MMA issuer waits on a barrier nobody arrives at, for
+ *     timeout_us microseconds.
+ * The kernel then records a fault (read by bitlinear_get_fault), every role
+ * returns, and y is not written. Other inputs as for bitlinear_forward_ex
+ * with that path; timeout_us in [1, 10^7]. */
 int bitlinear_forward_inject_timeout(const void *x_dev, bitlinear_dtype xdt,
                                      int64_t M, int64_t K,
                                      const void *packed_dev, float gamma,
                                      int64_t N, void *y_dev,
                                      void *workspace_dev,
                                      size_t workspace_bytes,
-                                     void *cuda_stream, int timeout_us);
+                                     void *cuda_stream, int path,
+                                     int timeout_us);
 
 #ifdef __cplusplus
 }

@@ -62,6 +62,8 @@ EXPORTS = (
     "bitlinear_forward_grouped",
     "bitlinear_workspace_bytes_grouped",
     "bitlinear_forward_grouped_ws",
+    "bitlinear_workspace_bytes_ffn",
+    "bitlinear_ffn_forward",
 )
 
 
@@ -114,7 +116,7 @@ def lib() -> ctypes.CDLL:
         L.bitlinear_forward_rmsnorm.argtypes = (fwd[:4] + [p, ctypes.c_float] + fwd[4:] +
                                                 [ctypes.c_int])
         L.bitlinear_forward_inject_timeout.restype = ctypes.c_int
-        L.bitlinear_forward_inject_timeout.argtypes = fwd[:11] + [ctypes.c_int]
+        L.bitlinear_forward_inject_timeout.argtypes = fwd[:11] + [ctypes.c_int, ctypes.c_int]
         L.bitlinear_forward_noalloc.restype = ctypes.c_int
         L.bitlinear_forward_noalloc.argtypes = [p, ctypes.c_int, i64, i64, p, ctypes.c_float,
                                                 i64, p, p]
@@ -125,6 +127,12 @@ def lib() -> ctypes.CDLL:
         L.bitlinear_forward_grouped_ws.restype = ctypes.c_int
         L.bitlinear_forward_grouped_ws.argtypes = [p, ctypes.c_int, ctypes.c_int, p,
                                                    ctypes.c_size_t, p]
+        L.bitlinear_workspace_bytes_ffn.restype = sz
+        L.bitlinear_workspace_bytes_ffn.argtypes = [i64, i64, i64]
+        f32 = ctypes.c_float
+        L.bitlinear_ffn_forward.restype = ctypes.c_int
+        L.bitlinear_ffn_forward.argtypes = [p, ctypes.c_int, i64, i64, i64, p, f32, p, f32, p,
+                                            f32, p, p, p, f32, p, p, p, sz, p, p, p]
         L.bitlinear_get_fault.restype = ctypes.c_int
         L.bitlinear_get_fault.argtypes = [p, p]
         L.bitlinear_status_string.restype = ctypes.c_char_p
@@ -348,21 +356,71 @@ def bitlinear_forward_rmsnorm(x, packed, gamma: float, N: int, norm_gain,
 
 
 def bitlinear_forward_inject_timeout(x, packed, gamma: float, N: int, timeout_us: int,
-                                     y=None, workspace=None, stream=None) -> int:
-    """Run the tensor-core GEMM with one wait made to run out; returns the
-    status the launch reported (the fault is read by bitlinear_get_fault)."""
+                                     y=None, workspace=None, stream=None,
+                                     path: int = PATH_TC) -> int:
+    """Run the GEMV (path=PATH_GEMV) or the tensor-core GEMM (PATH_TC) with
+    one wait made to run out; returns the status the launch reported (the
+    fault is read by bitlinear_get_fault)."""
     a = _Args()
     import torch
     M, K = x.shape
     if y is None:
         y = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
-    need = bitlinear_workspace_bytes(M, N, K, PATH_TC)
+    need = bitlinear_workspace_bytes(M, N, K, path)
     if workspace is None:
         workspace = torch.empty((max(need, 1),), dtype=torch.uint8, device=x.device)
     return int(lib().bitlinear_forward_inject_timeout(
         a.ptr(x, "x"), _xdt(x), M, K, a.packed(packed, N, K), float(gamma), N,
         a.ptr(y, "y", torch.bfloat16, (M, N)), a.ptr(workspace, "workspace", torch.uint8),
-        workspace.numel(), _stream(stream), int(timeout_us)))
+        workspace.numel(), _stream(stream), int(path), int(timeout_us)))
+
+
+def bitlinear_workspace_bytes_ffn(M: int, K: int, F: int) -> int:
+    return int(lib().bitlinear_workspace_bytes_ffn(M, K, F))
+
+
+def bitlinear_ffn_forward(x, gate, up, down, gains=(None, None, None),
+                          eps: float = RMSNORM_EPS, h=None, y=None, workspace=None,
+                          stream=None, gate_y=None, up_y=None):
+    """The feed-forward block: y = down(h), h = max(gate(x), 0)^2 * up(x) in
+    fp32, for M decode tokens x [M][K]. ``gate``, ``up`` and ``down`` are
+    (packed, gamma) pairs (gate/up F x K, down K x F); ``gains`` gives each
+    BitLinear's RMSNorm gains (fp32 device tensors or None; gate and up
+    together). Returns (y bf16 [M][K], h fp32 [M][F]); ``gate_y``/``up_y``
+    optionally receive the bf16 gate and up outputs."""
+    a = _Args()
+    import torch
+    M, K = x.shape
+    (gp, gg), (upk, ug), (dp, dg) = gate, up, down
+    F = _ffn_width(upk, K)
+    if h is None:
+        h = torch.empty((M, F), dtype=torch.float32, device=x.device)
+    if y is None:
+        y = torch.empty((M, K), dtype=torch.bfloat16, device=x.device)
+    need = bitlinear_workspace_bytes_ffn(M, K, F)
+    if need == ctypes.c_size_t(-1).value:
+        raise BitLinearError(BITLINEAR_ERR_SHAPE, "bitlinear_workspace_bytes_ffn")
+    if workspace is None and need > 0:
+        workspace = torch.empty((need,), dtype=torch.uint8, device=x.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    g0, g1, g2 = gains
+    rc = lib().bitlinear_ffn_forward(
+        a.ptr(x, "x"), _xdt(x), M, K, F, a.packed(gp, F, K), float(gg), a.packed(upk, F, K),
+        float(ug), a.packed(dp, K, F), float(dg),
+        a.ptr(g0, "gate gain", torch.float32, (K,)), a.ptr(g1, "up gain", torch.float32, (K,)),
+        a.ptr(g2, "down gain", torch.float32, (F,)), float(eps),
+        a.ptr(h, "h", torch.float32, (M, F)), a.ptr(y, "y", torch.bfloat16, (M, K)),
+        a.ptr(workspace, "workspace"), ws_bytes, _stream(stream),
+        a.ptr(gate_y, "gate_y", torch.bfloat16, (M, F)),
+        a.ptr(up_y, "up_y", torch.bfloat16, (M, F)))
+    _check(rc, "bitlinear_ffn_forward")
+    return y, h
+
+
+def _ffn_width(packed, K: int) -> int:
+    """F of an F x K packed matrix whose F is a multiple of 16 (as every d_ff
+    the feed-forward call accepts, a multiple of 128, is)."""
+    return packed.numel() // (K // 4)
 
 
 def bitlinear_get_fault(stream=None) -> tuple[int, int]:

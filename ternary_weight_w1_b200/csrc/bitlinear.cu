@@ -44,14 +44,16 @@ bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p
 int gemv_tile(int64_t M) { return M <= 1 ? 1 : M <= 2 ? 2 : M <= 4 ? 4 : M <= 8 ? 8 : 16; }
 
 // Largest x~ (M * K bytes; for a group, the largest problem's) a GEMV launch
-// for up to M tokens admits: it must fit in sm_100's opt-in shared memory
-// beside two ring slots, one row block's accumulators per CTA and the
-// normalising form's reduction arrays, and is at most kGemvMaxXqBytes.
+// for up to M tokens admits. With the smallest stage geometry (one row block
+// of 8 k-groups per slot, two slots) the launch then still fits in sm_100's
+// opt-in shared memory beside the reduction area and the normalising form's
+// arrays, for every token tile.
 int64_t gemv_max_xq(int64_t M)
 {
     const int MT = gemv_tile(M);
-    return std::min<int64_t>(kGemvMaxXqBytes,
-                             kSmemOptinSm100 - gemv::smem_bytes(MT, 0, 16 * MT, 2, true));
+    return std::min<int64_t>(
+        kGemvMaxXqBytes,
+        kSmemOptinSm100 - gemv::smem_bytes(MT, 0, 2, 8 * gemv::PIECE, 1, true));
 }
 
 bool gemv_fits(int64_t M, int64_t K) { return M <= kGemvMaxM && M * K <= gemv_max_xq(M); }
@@ -261,25 +263,33 @@ int launch_quant_act(const void *x, bitlinear_dtype xdt, int M, int K, int8_t *x
 
 // ------------------------------------------------------------------- GEMV
 
-template <int MT, bool BF16, bool NORM>
+template <int MT, bool BF16, bool NORM, bool FFN>
 int launch_gemv_t(const gemv::Params &p, int grid, int smem, int dev, cudaStream_t st)
 {
-    cudaError_t e = allow_smem<gemv::gemv_kernel<MT, BF16, NORM>>(dev, smem);
+    cudaError_t e = allow_smem<gemv::gemv_kernel<MT, BF16, NORM, FFN>>(dev, smem);
     if (e != cudaSuccess)
         return launch_status(e);
-    e = launch(gemv::gemv_kernel<MT, BF16, NORM>, dim3(grid), dim3(gemv::THREADS), smem, st, p);
+    e = launch(gemv::gemv_kernel<MT, BF16, NORM, FFN>, dim3(grid), dim3(gemv::THREADS), smem, st,
+               p);
     return launch_status(e);
 }
 
 template <int MT>
-int launch_gemv_mt(const gemv::Params &p, bool bf16, bool norm, int grid, int smem, int dev,
-                   cudaStream_t st)
+int launch_gemv_mt(const gemv::Params &p, bool bf16, bool norm, bool ffn, int grid, int smem,
+                   int dev, cudaStream_t st)
 {
+    if (ffn) {
+        if (norm)
+            return bf16 ? launch_gemv_t<MT, true, true, true>(p, grid, smem, dev, st)
+                        : launch_gemv_t<MT, false, true, true>(p, grid, smem, dev, st);
+        return bf16 ? launch_gemv_t<MT, true, false, true>(p, grid, smem, dev, st)
+                    : launch_gemv_t<MT, false, false, true>(p, grid, smem, dev, st);
+    }
     if (norm)
-        return bf16 ? launch_gemv_t<MT, true, true>(p, grid, smem, dev, st)
-                    : launch_gemv_t<MT, false, true>(p, grid, smem, dev, st);
-    return bf16 ? launch_gemv_t<MT, true, false>(p, grid, smem, dev, st)
-                : launch_gemv_t<MT, false, false>(p, grid, smem, dev, st);
+        return bf16 ? launch_gemv_t<MT, true, true, false>(p, grid, smem, dev, st)
+                    : launch_gemv_t<MT, false, true, false>(p, grid, smem, dev, st);
+    return bf16 ? launch_gemv_t<MT, true, false, false>(p, grid, smem, dev, st)
+                : launch_gemv_t<MT, false, false, false>(p, grid, smem, dev, st);
 }
 
 // One problem of a GEMV launch, as the host sees it.
@@ -294,112 +304,134 @@ struct GemvJob {
     float *beta;
     const float *norm_gain;     // non-null: RMS-normalise the tokens first
     float norm_eps;
+    // the feed-forward form (one job per launch): the up projection, whose
+    // rows pair with the gate rows above, and the output h
+    const void *packed2 = nullptr;
+    float gamma2 = 0.0f;
+    const float *norm_gain2 = nullptr;
+    void *y2 = nullptr;
+    float *h = nullptr;
 };
 
 // Launches the GEMV kernel over one or more independent problems. Every CTA
-// owns whole 16-row blocks of one problem. A single problem is split over at
-// most two CTAs per SM with the same number of blocks per CTA; a group is
-// split so that the CTAs of every problem stream about the same number of
-// bytes, with at most three CTAs per SM (all resident at once). The one
-// exception is a matrix so tall, next to so large an x~, that a CTA's row
-// accumulators would not fit: its CTAs then take fewer row blocks and the
-// grid runs in more than one wave. Either every problem of the launch is
-// RMS-normalised or none is.
+// owns whole 16-row blocks of one problem, about the same number of weight
+// bytes in every CTA of the launch: the launch's bytes spread over two CTAs
+// per SM, kept between 16 and 64 KiB per CTA, so large matrices run in
+// several waves of small CTAs that the hardware balances over the SMs. Each
+// CTA streams its blocks in chunks of up to QB blocks, a stage holding G
+// k-groups of every block of the chunk (about 16 KiB). Either every problem
+// of the launch is RMS-normalised or none is. With inject_timeout_us > 0 the
+// producer leaves the first stage unloaded and every wait gives up after that
+// many microseconds (the failure-detection test). A job with a non-null h is
+// the feed-forward form (gate and up streamed together, h written); it is the
+// launch's only job.
 int launch_gemv(const GemvJob *jobs, int count, bitlinear_dtype xdt, const DeviceInfo &dev,
-                cudaStream_t st)
+                cudaStream_t st, int inject_timeout_us = 0)
 {
     const bool norm = jobs[0].norm_gain != nullptr;
+    const bool ffn = jobs[0].h != nullptr;
+    if (ffn && count != 1)
+        return BITLINEAR_ERR_ARG;
     for (int i = 1; i < count; ++i)
         if ((jobs[i].norm_gain != nullptr) != norm)
             return BITLINEAR_ERR_ARG;
     int Mmax = 1;
     double total_bytes = 0.0;
+    int xq_cap = 0;
     for (int i = 0; i < count; ++i) {
         Mmax = std::max(Mmax, jobs[i].M);
         total_bytes += static_cast<double>((jobs[i].N + 15) / 16) * 16.0 * jobs[i].K / 4.0;
+        xq_cap = std::max(xq_cap, jobs[i].M * jobs[i].K);
     }
     const int MT = gemv_tile(Mmax);
-    // Each CTA quantises only its own problem's M rows into shared memory.
-    int xq_cap = 0;
-    for (int i = 0; i < count; ++i)
-        xq_cap = std::max(xq_cap, jobs[i].M * jobs[i].K);
-    // Row blocks per CTA that fit: their int32 row accumulators share the
-    // block's shared memory with x~, so a very tall matrix next to a large x~
-    // takes more, smaller CTAs (and then more than one wave).
-    const int q_fit =
-        (dev.max_smem_optin - gemv::smem_bytes(MT, xq_cap, 0, 2, norm)) / (16 * MT * 4);
-    if (q_fit < 1)
-        return BITLINEAR_ERR_SHAPE;
-    const int gmax = 2 * dev.sms;
-    const int cap = 3 * dev.sms;
-    int q[gemv::MAX_PROBLEMS], ctas[gemv::MAX_PROBLEMS];
-    int grid = 0;
-    if (count == 1) {
-        const int blocks = (jobs[0].N + 15) / 16;
-        q[0] = std::min((blocks + gmax - 1) / gmax, q_fit);
-        ctas[0] = (blocks + q[0] - 1) / q[0];
-        grid = ctas[0];
-    } else {
-        double target = total_bytes / gmax;        // bytes per CTA
-        for (int attempt = 0; attempt < 64; ++attempt) {
-            grid = 0;
-            for (int i = 0; i < count; ++i) {
-                const int blocks = (jobs[i].N + 15) / 16;
-                const double block_bytes = 16.0 * jobs[i].K / 4.0;
-                q[i] = std::max(1, static_cast<int>(target / block_bytes + 0.5));
-                q[i] = std::min({q[i], blocks, q_fit});
-                ctas[i] = (blocks + q[i] - 1) / q[i];
-                grid += ctas[i];
-            }
-            if (grid <= cap)
-                break;
-            target *= 1.25;
+    const int QB = gemv::chunk_blocks(MT, ffn);
+    const int nmat = ffn ? 2 : 1;
+    double target = std::min(64.0 * 1024, std::max(16.0 * 1024, total_bytes / (2.0 * dev.sms)));
+    int gcap = 1 << 30;               // upper bound on k-groups per stage
+    int q[gemv::MAX_PROBLEMS], ctas[gemv::MAX_PROBLEMS], G[gemv::MAX_PROBLEMS];
+    int grid = 0, slot_bytes = 0, slots = 0, red_blocks = 1, smem = 0;
+    for (int attempt = 0;; ++attempt) {
+        grid = 0;
+        slot_bytes = 0;
+        red_blocks = 1;
+        int stages = 1;
+        for (int i = 0; i < count; ++i) {
+            const int blocks = (jobs[i].N + 15) / 16;
+            const int KG = jobs[i].K / 128;
+            const double block_bytes = nmat * 16.0 * jobs[i].K / 4.0;
+            q[i] = std::max(1, std::min(blocks, static_cast<int>(target / block_bytes + 0.5)));
+            ctas[i] = (blocks + q[i] - 1) / q[i];
+            grid += ctas[i];
+            const int qb = std::min(q[i], QB);
+            // about 16 KiB per stage: G a multiple of 8 (each warp owns the
+            // groups of one residue mod 8), or the whole row when that is less
+            int g = std::max(8, (16384 / (nmat * qb * gemv::PIECE)) & ~7);
+            g = std::min(g, std::max(8, gcap));
+            G[i] = g >= KG ? KG : g;
+            slot_bytes = std::max(slot_bytes, nmat * qb * G[i] * gemv::PIECE);
+            red_blocks = std::max(red_blocks, qb);
+            stages = std::max(stages, ((q[i] + QB - 1) / QB) * ((KG + G[i] - 1) / G[i]));
         }
-    }
-    int qmax = 1, stages = 1;
-    for (int i = 0; i < count; ++i) {
-        // The kernel divides a piece index by K/128 with a multiply and shift,
-        // exact below 2^23 pieces (4 GiB of packed weights) per CTA.
-        if (static_cast<int64_t>(q[i]) * (jobs[i].K / 128) >= (int64_t(1) << 23))
+        // Ring depth: the whole share when it is small, else as deep as a
+        // 72 KiB block allows (three blocks per SM fit beside each other).
+        const int fixed = gemv::smem_bytes(MT, xq_cap, 0, 0, red_blocks, norm, ffn);
+        slots = (72 * 1024 - fixed) / slot_bytes;
+        slots = std::max(2, std::min({slots, stages, gemv::MAX_SLOTS}));
+        smem = gemv::smem_bytes(MT, xq_cap, slots, slot_bytes, red_blocks, norm, ffn);
+        if (smem <= dev.max_smem_optin)
+            break;
+        // too large beside a large x~: smaller stages first, then fewer
+        // blocks per CTA
+        if (gcap > 8)
+            gcap = (gcap > 64 ? 64 : gcap) / 2;
+        else if (target > 1024.0)
+            target /= 2.0;
+        else
             return BITLINEAR_ERR_SHAPE;
-        qmax = std::max(qmax, q[i]);
-        stages = std::max(stages, (q[i] * (jobs[i].K / 128) * gemv::PIECE + gemv::STAGE - 1) /
-                                      gemv::STAGE);
+        if (attempt > 64)
+            return BITLINEAR_ERR_SHAPE;
     }
-    const int acc_cap = qmax * 16 * MT;
-    // Ring depth: the whole share when it is small (room for the next
-    // kernel's blocks on the same SM under programmatic launch), else as deep
-    // as a 110 KiB block allows.
-    const int fixed = gemv::smem_bytes(MT, xq_cap, acc_cap, 0, norm);
-    const int budget = stages > 12 ? 110 * 1024 : 56 * 1024;
-    int slots = (budget - fixed) / gemv::STAGE;
-    slots = std::max(2, std::min({slots, stages, gemv::MAX_SLOTS}));
-    const int smem = gemv::smem_bytes(MT, xq_cap, acc_cap, slots, norm);
-    if (smem > dev.max_smem_optin)
-        return BITLINEAR_ERR_SHAPE;
     gemv::Params p = {};
     int begin = 0;
     for (int i = 0; i < count; ++i) {
         const GemvJob &j = jobs[i];
-        const uint64_t kg = static_cast<uint64_t>(j.K / 128);
-        p.prob[i] = gemv::Problem{j.x, static_cast<const uint8_t *>(j.packed),
-                                  static_cast<uint16_t *>(j.y), j.acc, j.xq, j.beta, j.M, j.K,
-                                  j.N, j.gamma, j.norm_gain, j.norm_eps, q[i], begin,
-                                  ((uint64_t(1) << 32) + kg - 1) / kg};
+        p.prob[i] = gemv::Problem{j.x,
+                                  static_cast<const uint8_t *>(j.packed),
+                                  static_cast<uint16_t *>(j.y),
+                                  j.acc,
+                                  j.xq,
+                                  j.beta,
+                                  j.M,
+                                  j.K,
+                                  j.N,
+                                  j.gamma,
+                                  j.norm_gain,
+                                  j.norm_eps,
+                                  q[i],
+                                  begin,
+                                  G[i],
+                                  static_cast<const uint8_t *>(j.packed2),
+                                  j.gamma2,
+                                  j.norm_gain2,
+                                  static_cast<uint16_t *>(j.y2),
+                                  j.h};
         begin += ctas[i];
     }
     p.count = count;
     p.slots = slots;
+    p.slot_bytes = slot_bytes;
     p.xq_cap = xq_cap;
-    p.acc_cap = acc_cap;
-    p.wait_limit_ns = kWaitLimitNs;
+    p.red_blocks = red_blocks;
+    p.wait_limit_ns = inject_timeout_us > 0 ? static_cast<uint64_t>(inject_timeout_us) * 1000ull
+                                            : kWaitLimitNs;
+    p.inject_timeout = inject_timeout_us > 0 ? 1 : 0;
     const bool bf16 = xdt == BITLINEAR_BF16;
     switch (MT) {
-    case 1: return launch_gemv_mt<1>(p, bf16, norm, grid, smem, dev.id, st);
-    case 2: return launch_gemv_mt<2>(p, bf16, norm, grid, smem, dev.id, st);
-    case 4: return launch_gemv_mt<4>(p, bf16, norm, grid, smem, dev.id, st);
-    case 8: return launch_gemv_mt<8>(p, bf16, norm, grid, smem, dev.id, st);
-    default: return launch_gemv_mt<16>(p, bf16, norm, grid, smem, dev.id, st);
+    case 1: return launch_gemv_mt<1>(p, bf16, norm, ffn, grid, smem, dev.id, st);
+    case 2: return launch_gemv_mt<2>(p, bf16, norm, ffn, grid, smem, dev.id, st);
+    case 4: return launch_gemv_mt<4>(p, bf16, norm, ffn, grid, smem, dev.id, st);
+    case 8: return launch_gemv_mt<8>(p, bf16, norm, ffn, grid, smem, dev.id, st);
+    default: return launch_gemv_mt<16>(p, bf16, norm, ffn, grid, smem, dev.id, st);
     }
 }
 
@@ -690,7 +722,7 @@ int forward_impl(const void *x, bitlinear_dtype xdt, int64_t M, int64_t K, const
         return BITLINEAR_ERR_ARG;
     if (M == 0)
         return BITLINEAR_OK;
-    const int chosen = inject_timeout_us > 0 ? BITLINEAR_PATH_TC : choose_path(M, K, path);
+    const int chosen = choose_path(M, K, path);
     if (chosen == BITLINEAR_PATH_GEMV && !gemv_fits(M, K))
         return BITLINEAR_ERR_SHAPE;
     DeviceInfo *dev = nullptr;
@@ -701,7 +733,7 @@ int forward_impl(const void *x, bitlinear_dtype xdt, int64_t M, int64_t K, const
     if (chosen == BITLINEAR_PATH_GEMV) {
         const GemvJob job{x,      static_cast<int>(M), static_cast<int>(K), static_cast<int>(N),
                           packed, gamma, y, acc, xq, beta, norm_gain, norm_eps};
-        return launch_gemv(&job, 1, xdt, *dev, st);
+        return launch_gemv(&job, 1, xdt, *dev, st, inject_timeout_us);
     }
     return run_tc_path(x, xdt, static_cast<int>(M), static_cast<int>(K), packed, gamma,
                        static_cast<int>(N), y, ws, ws_bytes, acc, xq, beta, *dev, st,
@@ -807,6 +839,97 @@ extern "C" int bitlinear_forward_rmsnorm(const void *x_dev, bitlinear_dtype xdt,
     return forward_impl(x_dev, xdt, M, K, packed_dev, gamma, N, y_dev, workspace_dev,
                         workspace_bytes, cuda_stream, acc_dev_or_null, xq_dev_or_null,
                         beta_dev_or_null, path, 0, gain, norm_eps);
+}
+
+namespace {
+
+// Argument checks of the feed-forward calls that do not depend on pointers:
+// returns BITLINEAR_OK when (M, K, F) and the gains' presence are acceptable.
+int check_ffn_shape(int64_t M, int64_t K, int64_t F, bool gate_up_norm)
+{
+    if (M < 0 || K < 1 || F < 1)
+        return BITLINEAR_ERR_ARG;
+    if (K % 128 != 0 || F % 128 != 0 || K > kMaxK || F > kMaxK)
+        return BITLINEAR_ERR_SHAPE;
+    // the gate/up launch is the GEMV (with two quantised copies of the
+    // tokens when both projections normalise them with their own gains)
+    if (M > kGemvMaxM || (gate_up_norm ? 2 : 1) * M * K > gemv_max_xq(M))
+        return BITLINEAR_ERR_SHAPE;
+    return BITLINEAR_OK;
+}
+
+}  // namespace
+
+extern "C" size_t bitlinear_workspace_bytes_ffn(int64_t M, int64_t K, int64_t F)
+{
+    if (check_ffn_shape(M, K, F, false) != BITLINEAR_OK)
+        return SIZE_MAX;
+    return bitlinear_workspace_bytes_path(M, K, F, BITLINEAR_PATH_AUTO);
+}
+
+extern "C" int bitlinear_ffn_forward(const void *x_dev, bitlinear_dtype xdt, int64_t M, int64_t K,
+                                     int64_t F, const void *gate_packed_dev, float gate_gamma,
+                                     const void *up_packed_dev, float up_gamma,
+                                     const void *down_packed_dev, float down_gamma,
+                                     const float *gate_gain_dev, const float *up_gain_dev,
+                                     const float *down_gain_dev, float norm_eps, float *h_dev,
+                                     void *y_dev, void *workspace_dev, size_t workspace_bytes,
+                                     void *cuda_stream, void *gate_y_dev_or_null,
+                                     void *up_y_dev_or_null)
+{
+    if ((gate_gain_dev == nullptr) != (up_gain_dev == nullptr))
+        return BITLINEAR_ERR_ARG;
+    const bool gu_norm = gate_gain_dev != nullptr;
+    int rc = check_ffn_shape(M, K, F, gu_norm);
+    if (rc != BITLINEAR_OK)
+        return rc;
+    if (xdt != BITLINEAR_BF16 && xdt != BITLINEAR_FP32)
+        return BITLINEAR_ERR_DTYPE;
+    if ((gu_norm || down_gain_dev != nullptr) && (!(norm_eps > 0.0f) || !(norm_eps <= FLT_MAX)))
+        return BITLINEAR_ERR_ARG;
+    if (M == 0)
+        return BITLINEAR_OK;
+    if (x_dev == nullptr || gate_packed_dev == nullptr || up_packed_dev == nullptr ||
+        down_packed_dev == nullptr || h_dev == nullptr || y_dev == nullptr)
+        return BITLINEAR_ERR_ARG;
+    if (!aligned(x_dev, 16) || !aligned(gate_packed_dev, 16) || !aligned(up_packed_dev, 16) ||
+        !aligned(down_packed_dev, 16) || !aligned(h_dev, 16) || !aligned(y_dev, 16) ||
+        !aligned(gate_gain_dev, 16) || !aligned(up_gain_dev, 16) || !aligned(down_gain_dev, 16) ||
+        !aligned(gate_y_dev_or_null, 16) || !aligned(up_y_dev_or_null, 16))
+        return BITLINEAR_ERR_ALIGN;
+    // the down projection's own checks (workspace included) before any launch
+    const int down_path = choose_path(M, F, BITLINEAR_PATH_AUTO);
+    if (down_path == BITLINEAR_PATH_TC &&
+        (workspace_dev == nullptr || workspace_bytes < tc_workspace_bytes(M, F)))
+        return BITLINEAR_ERR_WORKSPACE;
+    DeviceInfo *dev = nullptr;
+    rc = current_device(&dev);
+    if (rc != BITLINEAR_OK)
+        return rc;
+    cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
+    GemvJob job{x_dev,
+                static_cast<int>(M),
+                static_cast<int>(K),
+                static_cast<int>(F),
+                gate_packed_dev,
+                gate_gamma,
+                gate_y_dev_or_null,
+                nullptr,
+                nullptr,
+                nullptr,
+                gate_gain_dev,
+                norm_eps};
+    job.packed2 = up_packed_dev;
+    job.gamma2 = up_gamma;
+    job.norm_gain2 = up_gain_dev;
+    job.y2 = up_y_dev_or_null;
+    job.h = h_dev;
+    rc = launch_gemv(&job, 1, xdt, *dev, st);
+    if (rc != BITLINEAR_OK)
+        return rc;
+    return forward_impl(h_dev, BITLINEAR_FP32, M, F, down_packed_dev, down_gamma, K, y_dev,
+                        workspace_dev, workspace_bytes, cuda_stream, nullptr, nullptr, nullptr,
+                        BITLINEAR_PATH_AUTO, 0, down_gain_dev, norm_eps);
 }
 
 extern "C" int bitlinear_forward_grouped(const bitlinear_problem *problems, int count,
@@ -932,13 +1055,15 @@ extern "C" int bitlinear_forward_inject_timeout(const void *x_dev, bitlinear_dty
                                                 int64_t K, const void *packed_dev, float gamma,
                                                 int64_t N, void *y_dev, void *workspace_dev,
                                                 size_t workspace_bytes, void *cuda_stream,
-                                                int timeout_us)
+                                                int path, int timeout_us)
 {
     if (timeout_us < 1 || timeout_us > 10 * 1000 * 1000)
         return BITLINEAR_ERR_ARG;
+    if (path != BITLINEAR_PATH_GEMV && path != BITLINEAR_PATH_TC)
+        return BITLINEAR_ERR_ARG;
     return forward_impl(x_dev, xdt, M, K, packed_dev, gamma, N, y_dev, workspace_dev,
-                        workspace_bytes, cuda_stream, nullptr, nullptr, nullptr,
-                        BITLINEAR_PATH_TC, timeout_us);
+                        workspace_bytes, cuda_stream, nullptr, nullptr, nullptr, path,
+                        timeout_us);
 }
 
 extern "C" int bitlinear_get_fault(int *fault_out, void *cuda_stream)

@@ -7,41 +7,59 @@
 // memory-wall framing of "BitNet b1.58: The 1-Bit Paradigm Shift" is why the
 // kernel is organised around the weight bytes.
 //
-// Work split. The packed layout keeps 16-row blocks contiguous, so block b of
-// the grid owns q whole row blocks = one contiguous byte range. A producer
-// warp streams that range through a ring of 8 KiB shared-memory slots with
-// bulk (TMA) copies, starting before the programmatic-launch wait so the weight
-// stream overlaps the previous kernel and this kernel's prologue. Eight
-// compute warps consume 512-byte pieces (one row block x one k-group of 128
-// weights: 16 rows x 32 B) round-robin; lane (r, t) = (lane / 2, lane % 2)
-// always holds row r of the piece and the k-half t, i.e. 64 weights, so the
-// activations it needs are one 64-byte run of x~ that all 16 rows share (a
-// two-address broadcast read from shared memory).
+// Work split. The packed layout keeps 16-row blocks contiguous, each block a
+// run of K/128 512-byte pieces (one 128-k group of its 16 rows). CTA c owns
+// q consecutive row blocks of one problem and takes them in chunks of up to
+// QB blocks. A chunk is streamed k-group-major: stage s holds groups
+// [G s, G s + G) of every block of the chunk, one bulk copy per block issued
+// by its own producer lane, all landing on the stage's mbarrier. The producer
+// starts before the programmatic-launch wait (the weights are never written
+// by an earlier kernel), so the stream overlaps the previous kernel and this
+// kernel's prologue.
 //
-// Arithmetic. With codes c = W~ + 1 in {0,1,2}, the four 2-bit fields j of
-// each byte of a packed word w hold the weights k = 16w' + 4j .. 16w' + 4j + 3
-// of its 16-weight run. w & 0x03030303 and w & 0x0C0C0C0C leave c and 4c in
-// every byte for j = 0 and 1, and the same two masks on w >> 4 do it for
-// j = 2 and 3: all values fit a signed byte, so one signed dp4a per 4 weights
-// and token multiplies them with the matching x~ word. The two accumulators
-// (scale 1: j = 0, 2; scale 4: j = 1, 3) give
-//   sum c*x~ = s1 + (s4 >> 2)
-// exactly (s4 is a multiple of 4), and acc = sum c*x~ - sum x~ (the token's
-// sum of x~ comes from the prologue). Each piece's partial is folded with the
-// k-half partner lane by one shuffle and added into a per-row int32
-// shared-memory accumulator (integer, so the order of the atomic adds cannot
-// change the result); pieces are therefore independent, and each warp works
-// on all of its pieces of a ring slot at once, without branches.
+// Compute warp w owns the k-groups g = w (mod 8). In a stage it loads, for
+// each of its groups, the 64 bytes of x~ its lane needs into registers once
+// and applies them to that group's piece of every block of the chunk: lane
+// (r, t) = (lane / 2, lane % 2) holds row r of the block and the k-half t of
+// the group (64 weights, 16 bytes). The row partial sums stay in registers
+// for the whole chunk; one shuffle (the two k-halves) and one pass through
+// shared memory (the eight warps) per chunk give the rows' sums.
 //
-// RMS normalisation (NORM launches). The listing's BitLinear normalises each
-// token with its nn.RMSNorm member before quantising it; here that is one more
-// prologue pass. Each thread sums the squares of its activations in double
-// (exact products), the warps' sums go to shared memory and every thread adds
-// them in the same order, so all CTAs derive the same r = 1 / sqrt(mean +
-// eps); the absmax and quantisation passes then work on (x * r) * g.
+// Arithmetic. With codes c = W~ + 1 in {0, 1, 2} at bits 2j of every byte of
+// a packed word, w & (3 << 2j) leaves c * 4^j in each byte (at most 128,
+// which fits an unsigned byte), so one dp4a of unsigned weight bytes by
+// signed x~ bytes per plane and token multiplies four weights by the matching
+// x~ word. The plane sums a_j are exact multiples of 4^j, so
+//   sum c * x~ = a_0 + (a_1 >> 2) + (a_2 >> 4) + (a_3 >> 6)
+// exactly, and acc = sum c * x~ - sum x~. Integer sums: the order of the
+// partial sums cannot change the result.
 //
-// Every mbarrier wait is bounded; a wait that runs out records the fault word
-// and lets every warp return (the producer first waits for its own copies).
+// Prologue. Each thread reads the activations of its own warp's groups (lane
+// l: elements 128 g + 4 l .. + 3), the warps combine their absmax through
+// shared memory (one barrier), and every warp quantises its own groups into
+// shared memory, where only its own lanes read them. The sum of x~ of each
+// warp's groups goes to shared memory for the epilogue. With RMS
+// normalisation (NORM launches; the listing's BitLinear normalises each token
+// with its nn.RMSNorm member before quantising it) a first pass sums each
+// token's squares in double (exact products), the warps' sums go to shared
+// memory and every thread adds them in warp order, so all CTAs derive the
+// same r = 1 / sqrt(mean + eps); the absmax and quantisation passes then work
+// on (x * r) * g.
+//
+// Feed-forward form (FFN launches). The gate and up projections of a
+// feed-forward block read the same tokens: a CTA streams block b of both
+// matrices in the same stage (gate blocks in the first half of the slot, up
+// blocks in the second), applies the same x~ registers to both (or, when
+// each projection RMS-normalises the tokens with its own gains, its own x~),
+// and its epilogue rounds both outputs to bf16 and writes the gated squared
+// ReLU h = (r * r) * up, r = max(gate, 0), in fp32: the feed-forward
+// activation of "Microsoft Releases BitNet b1.58 2B4T" ("Under the Hood":
+// ReLU^2 in place of SwiGLU), read as gated. h is the down projection's input.
+//
+// Every mbarrier wait is bounded; a wait that runs out records the fault
+// word, raises the block's abort flag so that every warp stops waiting, and
+// the epilogue then writes nothing (no partial y). The producer waits for its
+// own copies before it returns.
 #pragma once
 
 #include "common.cuh"
@@ -53,13 +71,30 @@ constexpr int CWARPS = 8;                          // compute warps
 constexpr int CTHREADS = CWARPS * 32;
 constexpr int THREADS = CTHREADS + 32;             // + the producer warp
 constexpr int PIECE = 512;                         // one (row block, k-group)
-constexpr int STAGE = 16384;                       // bytes per ring slot
-constexpr int PIECES_PER_STAGE = STAGE / PIECE;
-constexpr int PIECES_PER_WARP = PIECES_PER_STAGE / CWARPS;   // per stage
-constexpr int MAX_SLOTS = 16;
+constexpr int MAX_SLOTS = 8;
 constexpr int BAR_BYTES = 2 * MAX_SLOTS * 8 + 16;  // full/empty barriers + abort flag
-
 constexpr int MAX_PROBLEMS = 8;
+constexpr int XCACHE = 4;                          // groups of token 0 kept through the prologue
+
+// Row blocks per chunk and tokens whose x~ a lane holds in registers at once,
+// by token tile MT. Only MT = 1 keeps the four plane sums apart for a whole
+// chunk; larger tiles fold them into one sum per piece.
+template <int MT, bool FFN = false>
+struct Shape {
+    // an FFN chunk carries each block twice (gate and up)
+    static constexpr int QB = (MT == 1 ? 8 : MT == 2 ? 4 : 2) / (FFN ? 2 : 1);
+    static constexpr int TQ = MT == 4 ? 4 : MT == 1 ? 1 : 2;
+    static constexpr bool PERSIST = MT == 1;
+    // blocks per SM the register budget is set for: three for the small
+    // tiles (two of this launch and, under programmatic dependent launch, one
+    // of the next), two for the larger ones
+    static constexpr int MIN_BLOCKS = (MT <= 2 && !FFN) ? 3 : 2;
+};
+
+__host__ __device__ constexpr int chunk_blocks(int MT, bool ffn = false)
+{
+    return (MT == 1 ? 8 : MT == 2 ? 4 : 2) / (ffn ? 2 : 1);
+}
 
 // One BitLinear problem of a GEMV launch; a launch may carry several
 // independent problems (a grouped launch), each with its own CTAs.
@@ -76,25 +111,37 @@ struct Problem {
     float norm_eps;         // eps of the normalisation (NORM launches only)
     int blocks_per_cta;     // row blocks of 16 rows owned by one CTA
     int cta_begin;          // this problem's first CTA in the grid
-    uint64_t kg_magic;      // ceil(2^32 / (K / 128)): i / KG == (i * kg_magic) >> 32
-                            // for every piece index i < 2^23 at any KG <= 512 (the
-                            // host keeps blocks_per_cta * KG below that)
+    int G;                  // k-groups per stage (a multiple of 8, or all K/128)
+    // FFN launches only: `packed`, `gamma`, `norm_gain` and `y` (optional)
+    // are the gate projection's; these are the up projection's and h
+    const uint8_t *packed2;
+    float gamma2;
+    const float *norm_gain2;
+    uint16_t *y2;           // [M][N] bf16 up output, or null
+    float *h;               // [M][N] fp32 (r * r) * up, r = max(gate, 0)
 };
 
 struct Params {
     Problem prob[MAX_PROBLEMS];
     int count;              // problems in this launch
     int slots;              // ring slots (<= MAX_SLOTS)
+    int slot_bytes;         // bytes per ring slot (a multiple of 512)
     int xq_cap;             // shared bytes for x~: max over problems of M * K
-    int acc_cap;            // row accumulators: max over problems of blocks_per_cta * 16 * MT
+    int red_blocks;         // row blocks per chunk the reduction area holds
     uint64_t wait_limit_ns;
+    int inject_timeout;     // the producer leaves the first stage unloaded
 };
 
-__host__ __device__ constexpr int smem_bytes(int MT, int xq_cap, int acc_cap, int slots,
-                                             bool norm = false)
+// Shared-memory bytes of a launch (the regions in the order the kernel
+// carves them out; every region size is a multiple of 16 bytes). An FFN
+// launch keeps two reduction areas (gate and up) and, when it normalises,
+// two quantised copies of the tokens with their own beta and sums.
+__host__ __device__ constexpr int smem_bytes(int MT, int xq_cap, int slots, int slot_bytes,
+                                             int red_blocks, bool norm, bool ffn = false)
 {
-    return slots * STAGE + BAR_BYTES + xq_cap + acc_cap * 4 + (norm ? MT * CWARPS * 8 : 0) +
-           MT * 4 + 2 * MT * CWARPS * 4;
+    return slots * slot_bytes + BAR_BYTES + (ffn && norm ? 2 : 1) * xq_cap +
+           (ffn ? 2 : 1) * CWARPS * red_blocks * 16 * MT * 4 + (norm ? MT * CWARPS * 8 : 0) +
+           (ffn && norm ? 2 : 1) * (16 * ((MT * 4 + 15) / 16) + 2 * MT * CWARPS * 4);
 }
 
 // r of token m from the warps' partial sums of squares, added in warp order.
@@ -112,12 +159,44 @@ __device__ __forceinline__ void compute_sync()
     asm volatile("bar.sync 1, %0;" ::"r"(CTHREADS) : "memory");
 }
 
-// Three blocks per SM fit the register file (two of this grid and, under
-// programmatic dependent launch, one of the next).
-template <int MT, bool BF16, bool NORM>
-__global__ void __launch_bounds__(THREADS, 3)
+// dp4a of four unsigned bytes (weight codes times a power of 4, at most 128)
+// by four signed bytes (x~), accumulated in int32.
+__device__ __forceinline__ int dp4a_us(uint32_t a, uint32_t b, int c)
+{
+    int d;
+    asm("dp4a.u32.s32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+    return d;
+}
+
+// Four consecutive activations (element e, a multiple of 4) of a row as fp32
+// (bf16 widening is exact).
+template <bool BF16>
+__device__ __forceinline__ void load4(const void *row, int e, float (&v)[4])
+{
+    if constexpr (BF16) {
+        const uint2 raw =
+            __ldg(reinterpret_cast<const uint2 *>(static_cast<const __nv_bfloat16 *>(row) + e));
+        v[0] = __uint_as_float(raw.x << 16);
+        v[1] = __uint_as_float(raw.x & 0xffff0000u);
+        v[2] = __uint_as_float(raw.y << 16);
+        v[3] = __uint_as_float(raw.y & 0xffff0000u);
+    } else {
+        const float4 a = __ldg(reinterpret_cast<const float4 *>(static_cast<const float *>(row) + e));
+        v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+    }
+}
+
+template <int MT, bool BF16, bool NORM, bool FFN>
+__global__ void __launch_bounds__(THREADS, (Shape<MT, FFN>::MIN_BLOCKS))
 gemv_kernel(const __grid_constant__ Params p)
 {
+    using S = Shape<MT, FFN>;
+    constexpr int QB = S::QB;
+    constexpr int NMAT = FFN ? 2 : 1;          // matrices streamed (gate, up)
+    constexpr int NX = (FFN && NORM) ? 2 : 1;   // quantised copies of the tokens
+    // with two copies of x~ in registers, fewer tokens at a time
+    constexpr int TQ = NX == 1 ? S::TQ : MT >= 8 ? 1 : (S::TQ < 2 ? S::TQ : 2);
+    constexpr int NACC = S::PERSIST ? 4 : MT;   // accumulators per block and matrix
     extern __shared__ __align__(128) uint8_t smem[];
     // this CTA's problem (grouped launches give each problem its own CTAs)
     int pi = 0;
@@ -127,30 +206,37 @@ gemv_kernel(const __grid_constant__ Params p)
     const Problem &P = p.prob[pi];
     const int K = P.K, M = P.M, N = P.N;
     const int KG = K >> 7;                              // k-groups per row
+    const int G = P.G;
     const int total_blocks = (N + 15) >> 4;
-    const int q = P.blocks_per_cta;
-    const int blk0 = (static_cast<int>(blockIdx.x) - P.cta_begin) * q;
-    const int nblk = min(q, total_blocks - blk0);
-    const size_t block_bytes = static_cast<size_t>(K) * 4;   // 16 rows x K/4 bytes
-    const uint8_t *src = P.packed + static_cast<size_t>(blk0) * block_bytes;
-    const int npieces = nblk * KG;
-    const int nstages = (npieces + PIECES_PER_STAGE - 1) / PIECES_PER_STAGE;
+    const int blk0 = (static_cast<int>(blockIdx.x) - P.cta_begin) * P.blocks_per_cta;
+    const int nblk = min(P.blocks_per_cta, total_blocks - blk0);
+    const int nchunks = (nblk + QB - 1) / QB;
+    const int kstages = (KG + G - 1) / G;
+    const int nstages = nchunks * kstages;
     const int slots = p.slots;
+    const int slot_bytes = p.slot_bytes;
+    const int red_stride = CWARPS * p.red_blocks * 16 * MT;     // ints per reduction area
+    const bool first_cta = static_cast<int>(blockIdx.x) == P.cta_begin;
 
     uint8_t *ring = smem;
-    const uint32_t bars = smem_u32(smem + slots * STAGE);
+    const uint32_t ring_u32 = smem_u32(ring);
+    const uint32_t bars = smem_u32(smem + slots * slot_bytes);
     auto full = [&](int s) { return bars + 8u * static_cast<uint32_t>(s); };
     auto empty = [&](int s) { return bars + 8u * static_cast<uint32_t>(MAX_SLOTS + s); };
     volatile int *abort_flag =
-        reinterpret_cast<volatile int *>(smem + slots * STAGE + 2 * MAX_SLOTS * 8);
-    uint8_t *xq_sm = smem + slots * STAGE + BAR_BYTES;
-    int *acc_sm = reinterpret_cast<int *>(xq_sm + p.xq_cap);
+        reinterpret_cast<volatile int *>(smem + slots * slot_bytes + 2 * MAX_SLOTS * 8);
+    uint8_t *xq_sm = smem + slots * slot_bytes + BAR_BYTES;        // [NX][xq_cap]
+    int *red = reinterpret_cast<int *>(xq_sm + NX * p.xq_cap);      // [NMAT][CWARPS][blocks*16][MT]
     // [MT][CWARPS] partial sums of squares (NORM only; 8-byte aligned: every
-    // region before it is a multiple of 8 bytes)
-    double *red_d = reinterpret_cast<double *>(acc_sm + p.acc_cap);
-    float *beta_sm = reinterpret_cast<float *>(red_d + (NORM ? MT * CWARPS : 0));
-    uint32_t *red_u = reinterpret_cast<uint32_t *>(beta_sm + MT);   // [MT][CWARPS] absmax
-    int *red_i = reinterpret_cast<int *>(red_u + MT * CWARPS);      // [MT][CWARPS] sum x~
+    // region before it is a multiple of 16 bytes)
+    double *red_d = reinterpret_cast<double *>(red + NMAT * red_stride);
+    // per quantised copy: beta [MT (rounded up to 4)], absmax and sum of x~
+    // partials [MT][CWARPS]
+    constexpr int QSET = 4 * ((MT + 3) / 4) + 2 * MT * CWARPS;
+    float *qset = reinterpret_cast<float *>(red_d + (NORM ? MT * CWARPS : 0));
+    auto beta_sm = [&](int x) { return qset + x * QSET; };
+    auto red_u = [&](int x) { return reinterpret_cast<uint32_t *>(qset + x * QSET + 4 * ((MT + 3) / 4)); };
+    auto red_s = [&](int x) { return reinterpret_cast<int *>(red_u(x) + MT * CWARPS); };
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -169,286 +255,397 @@ gemv_kernel(const __grid_constant__ Params p)
     if (warp == CWARPS) {
         // ---------------------------------------------------- weight producer
         // Reads only the packed weights, so it does not wait for the previous
-        // grid in the stream.
-        if (lane == 0) {
-            int issued = 0;
-            int slot = 0;
-            uint32_t phase = 0;       // parity of this pass over the ring
-            for (int st = 0; st < nstages; ++st) {
-                // from the second pass on, the slot must have been released
-                if (st >= slots && !mbar_wait_bounded(empty(slot), phase ^ 1u, abort_flag, limit))
-                    break;
-                const int off = st * STAGE;
-                const int bytes = min(STAGE, npieces * PIECE - off);
-                mbar_arrive_expect_tx(full(slot), static_cast<uint32_t>(bytes));
-                bulk_g2s(smem_u32(ring + slot * STAGE), src + off, static_cast<uint32_t>(bytes),
-                         full(slot));
-                issued = st + 1;
-                if (++slot == slots) {
-                    slot = 0;
-                    phase ^= 1u;
+        // grid in the stream. Lane l copies block l of the chunk (FFN: lanes
+        // qb .. 2 qb - 1 copy the up projection's blocks); lane 0 arms the
+        // stage's barrier with the whole stage's bytes first.
+        int slot = 0;
+        uint32_t phase = 0;        // parity of this pass over the ring
+        uint32_t in_flight = 0;    // slots holding a copy this warp issued
+        uint32_t parity = 0;       // the phase of that copy, per slot
+        for (int st = 0; st < nstages; ++st) {
+            // from the second pass on, the slot must have been released
+            if (st >= slots && !warp_wait_bounded(empty(slot), phase ^ 1u, abort_flag, limit))
+                break;
+            const int c = st / kstages;
+            const int ks = st - c * kstages;
+            const int b0 = c * QB;
+            const int qb = min(QB, nblk - b0);
+            const int g0 = ks * G;
+            const int gs = min(G, KG - g0);
+            const uint32_t bytes = static_cast<uint32_t>(gs * PIECE);
+            // the failure-detection test leaves the first stage unloaded, so
+            // the compute warps' first wait runs out
+            if (!(p.inject_timeout && st == 0)) {
+                if (lane == 0)
+                    mbar_arrive_expect_tx(full(slot), bytes * static_cast<uint32_t>(NMAT * qb));
+                __syncwarp();
+                if (lane < NMAT * qb) {
+                    const int mat = lane >= qb ? 1 : 0;
+                    const int bl = lane - mat * qb;
+                    const uint8_t *src = (FFN && mat) ? P.packed2 : P.packed;
+                    bulk_g2s(ring_u32 + static_cast<uint32_t>(slot * slot_bytes) + lane * bytes,
+                             src + (static_cast<size_t>(blk0 + b0 + bl) * KG + g0) * PIECE, bytes,
+                             full(slot));
                 }
+                in_flight |= 1u << slot;
+                parity = (parity & ~(1u << slot)) | (phase << slot);
             }
-            // every copy this thread started lands before the block exits
-            for (int st = max(0, issued - slots); st < issued; ++st)
-                drain_wait(full(st % slots), static_cast<uint32_t>(st / slots) & 1u, limit);
+            if (++slot == slots) {
+                slot = 0;
+                phase ^= 1u;
+            }
         }
+        // every copy this warp started lands before the block exits
+        if (lane == 0)
+            for (int s = 0; s < slots; ++s)
+                if (in_flight & (1u << s))
+                    drain_wait(full(s), (parity >> s) & 1u, limit);
+        __syncwarp();
         return;
     }
 
     // ------------------------------------------------------- compute warps
     const int ctid = threadIdx.x;                       // 0 .. CTHREADS-1
-    for (int i = ctid; i < nblk * 16 * MT; i += CTHREADS)
-        acc_sm[i] = 0;
+    const size_t row_bytes = static_cast<size_t>(K) * (BF16 ? 2 : 4);
+    const int ngw = (KG - warp + CWARPS - 1) / CWARPS;  // this warp's groups: warp + 8 i
 
     // x may be the previous kernel's output: read it only after the wait.
-    // Each thread keeps up to XCACHE vectors of 8 activations in registers
-    // between the absmax pass and the quantisation pass; longer rows are read
-    // again (from L1).
     pdl_wait();
-    constexpr int XCACHE = 4;
-    Vec8<BF16> xc[XCACHE];
-    const int e0 = ctid * 8;
-    const int estride = CTHREADS * 8;
-    if constexpr (NORM) {
-        // sums of squares per token (the first token's cache is filled here)
-        for (int m = 0; m < M; ++m) {
-            const void *row = static_cast<const char *>(P.x) +
-                              static_cast<size_t>(m) * K * (BF16 ? 2 : 4);
-            double ss = 0.0;
+    // Element e of token m is at (warp + 8 i) * 128 + 4 * lane for this
+    // thread's i-th group. Token 0's first XCACHE groups stay in registers
+    // between the passes; the rest are read again (from L1 or L2).
+    auto elem = [&](int i) { return (warp + CWARPS * i) * 128 + 4 * lane; };
+    // gains of quantised copy x (FFN: 0 = gate, 1 = up)
+    auto gain_of = [&](int x) { return (FFN && x == 1) ? P.norm_gain2 : P.norm_gain; };
+    float xc[XCACHE][4];
+    // groups whose loads are issued together (their latencies overlap)
+    constexpr int XB = NORM ? 2 : 4;
+    // Visits this thread's groups of token m: f(i, v, g) with v the four raw
+    // activations and, when `gains` is set (NORM launches), g the four gains
+    // of each quantised copy. Token 0's first XCACHE groups come from the
+    // registers once `fill` has stored them there.
+    auto for_groups = [&](int m, bool fill, bool gains, auto &&f) {
+        const void *row = static_cast<const char *>(P.x) + m * row_bytes;
+        int i0 = 0;
+        if (m == 0) {
+            float g[XCACHE][NX][4];
 #pragma unroll
-            for (int c = 0; c < XCACHE; ++c) {
-                const int e = e0 + c * estride;
-                if (m == 0 && e < K) {
-                    xc[c].load(row, e);
+            for (int i = 0; i < XCACHE; ++i) {
+                if (i < ngw) {
+                    if (fill)
+                        load4<BF16>(row, elem(i), xc[i]);
+                    if constexpr (NORM) {
+                        if (gains) {
 #pragma unroll
-                    for (int i = 0; i < 8; ++i) {
-                        const double d = xc[c].get(i);
-                        ss = __fma_rn(d, d, ss);
+                            for (int x = 0; x < NX; ++x)
+                                load4<false>(gain_of(x), elem(i), g[i][x]);
+                        }
                     }
                 }
             }
-            for (int e = (m == 0 ? e0 + XCACHE * estride : e0); e < K; e += estride) {
-                float v[8];
-                load8<BF16>(row, e, v);
 #pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    const double d = v[i];
-                    ss = __fma_rn(d, d, ss);
+            for (int i = 0; i < XCACHE; ++i)
+                if (i < ngw)
+                    f(i, xc[i], g[i]);
+            i0 = XCACHE;
+        }
+        for (int ib = i0; ib < ngw; ib += XB) {
+            float v[XB][4];
+            float g[XB][NX][4];
+#pragma unroll
+            for (int u = 0; u < XB; ++u) {
+                if (ib + u < ngw) {
+                    load4<BF16>(row, elem(ib + u), v[u]);
+                    if constexpr (NORM) {
+                        if (gains) {
+#pragma unroll
+                            for (int x = 0; x < NX; ++x)
+                                load4<false>(gain_of(x), elem(ib + u), g[u][x]);
+                        }
+                    }
                 }
             }
+#pragma unroll
+            for (int u = 0; u < XB; ++u)
+                if (ib + u < ngw)
+                    f(ib + u, v[u], g[u]);
+        }
+    };
+    using Gains = float[NX][4];
+
+    if constexpr (NORM) {
+        // sums of squares per token
+        for (int m = 0; m < M; ++m) {
+            double ss = 0.0;
+            for_groups(m, true, false, [&](int, const float (&v)[4], const Gains &) {
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const double d = v[u];
+                    ss = __fma_rn(d, d, ss);
+                }
+            });
             ss = warp_sum_f64(ss);
             if (lane == 0)
                 red_d[m * CWARPS + warp] = ss;
         }
         compute_sync();
     }
+    // absmax per token over this thread's elements (per quantised copy)
     for (int m = 0; m < M; ++m) {
-        const void *row = static_cast<const char *>(P.x) +
-                          static_cast<size_t>(m) * K * (BF16 ? 2 : 4);
         float r = 1.0f;
         if constexpr (NORM)
             r = row_rms_scale(red_d, m, K, P.norm_eps);
-        float amax = 0.0f;
+        float amax[NX];
 #pragma unroll
-        for (int c = 0; c < XCACHE; ++c) {
-            const int e = e0 + c * estride;
-            if (m == 0 && e < K) {
-                float g[8];
-                if constexpr (NORM)
-                    load8<false>(P.norm_gain, e, g);
-                else
-                    xc[c].load(row, e);
+        for (int x = 0; x < NX; ++x)
+            amax[x] = 0.0f;
+        for_groups(m, !NORM, true, [&](int, const float (&v)[4], const Gains &g) {
 #pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    float a = xc[c].get(i);
+            for (int x = 0; x < NX; ++x) {
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    float a = v[u];
                     if constexpr (NORM)
-                        a = norm1(a, r, g[i]);
-                    amax = fmaxf(amax, fabsf(a));
+                        a = norm1(a, r, g[x][u]);
+                    amax[x] = fmaxf(amax[x], fabsf(a));
                 }
             }
-        }
-        for (int e = (m == 0 ? e0 + XCACHE * estride : e0); e < K; e += estride) {
-            float v[8], g[8];
-            load8<BF16>(row, e, v);
-            if constexpr (NORM)
-                load8<false>(P.norm_gain, e, g);
+        });
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                float a = v[i];
-                if constexpr (NORM)
-                    a = norm1(a, r, g[i]);
-                amax = fmaxf(amax, fabsf(a));
-            }
+        for (int x = 0; x < NX; ++x) {
+            const uint32_t u = __reduce_max_sync(0xffffffffu, __float_as_uint(amax[x]));
+            if (lane == 0)
+                red_u(x)[m * CWARPS + warp] = u;
         }
-        const uint32_t u = __reduce_max_sync(0xffffffffu, __float_as_uint(amax));
-        if (lane == 0)
-            red_u[m * CWARPS + warp] = u;
     }
     compute_sync();
+    // quantise this warp's own groups into shared memory (only this warp
+    // reads them), with their sums of x~
     for (int m = 0; m < M; ++m) {
-        const void *row = static_cast<const char *>(P.x) +
-                          static_cast<size_t>(m) * K * (BF16 ? 2 : 4);
-        uint32_t u = red_u[m * CWARPS];
-#pragma unroll
-        for (int w = 1; w < CWARPS; ++w)
-            u = max(u, red_u[m * CWARPS + w]);
-        const float beta = fmaxf(__uint_as_float(u), 1e-5f);
-        const float scale = __fdiv_rn(127.0f, beta);
         float r = 1.0f;
         if constexpr (NORM)
             r = row_rms_scale(red_d, m, K, P.norm_eps);
-        int sum = 0;
-        auto quant_store = [&](const Vec8<BF16> &v, int e) {
-            float g[8];
-            if constexpr (NORM)
-                load8<false>(P.norm_gain, e, g);
-            uint32_t lo = 0, hi = 0;
+        float scale[NX];
+        int sum[NX];
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                float a = v.get(i), b = v.get(i + 4);
-                if constexpr (NORM) {
-                    a = norm1(a, r, g[i]);
-                    b = norm1(b, r, g[i + 4]);
+        for (int x = 0; x < NX; ++x) {
+            uint32_t ub = red_u(x)[m * CWARPS];
+#pragma unroll
+            for (int w = 1; w < CWARPS; ++w)
+                ub = max(ub, red_u(x)[m * CWARPS + w]);
+            const float beta = fmaxf(__uint_as_float(ub), 1e-5f);
+            scale[x] = __fdiv_rn(127.0f, beta);
+            sum[x] = 0;
+            if (ctid == 0) {
+                beta_sm(x)[m] = beta;
+                if (x == 0 && P.beta_dbg != nullptr && first_cta)
+                    P.beta_dbg[m] = beta;
+            }
+        }
+        for_groups(m, false, true, [&](int i, const float (&v)[4], const Gains &g) {
+            const int e = elem(i);
+#pragma unroll
+            for (int x = 0; x < NX; ++x) {
+                uint32_t word = 0;
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    float a = v[u];
+                    if constexpr (NORM)
+                        a = norm1(a, r, g[x][u]);
+                    const int q = quant1(a, scale[x]);
+                    sum[x] += q;
+                    word |= (static_cast<uint32_t>(q) & 0xffu) << (8 * u);
                 }
-                const int q0 = quant1(a, scale);
-                const int q1 = quant1(b, scale);
-                sum += q0 + q1;
-                lo |= (static_cast<uint32_t>(q0) & 0xffu) << (8 * i);
-                hi |= (static_cast<uint32_t>(q1) & 0xffu) << (8 * i);
+                *reinterpret_cast<uint32_t *>(xq_sm + x * p.xq_cap + m * K + e) = word;
+                if (x == 0 && P.xq_dbg != nullptr && first_cta)
+                    *reinterpret_cast<uint32_t *>(P.xq_dbg + static_cast<size_t>(m) * K + e) = word;
             }
-            *reinterpret_cast<uint2 *>(xq_sm + m * K + e) = make_uint2(lo, hi);
-            if (P.xq_dbg != nullptr && blockIdx.x == 0)
-                *reinterpret_cast<uint2 *>(P.xq_dbg + static_cast<size_t>(m) * K + e) =
-                    make_uint2(lo, hi);
-        };
-        if (m == 0) {
+        });
 #pragma unroll
-            for (int c = 0; c < XCACHE; ++c) {
-                const int e = e0 + c * estride;
-                if (e < K)
-                    quant_store(xc[c], e);
-            }
-        }
-        for (int e = (m == 0 ? e0 + XCACHE * estride : e0); e < K; e += estride) {
-            Vec8<BF16> v;
-            v.load(row, e);
-            quant_store(v, e);
-        }
-        sum = __reduce_add_sync(0xffffffffu, sum);
-        if (lane == 0)
-            red_i[m * CWARPS + warp] = sum;
-        if (ctid == 0) {
-            beta_sm[m] = beta;
-            if (P.beta_dbg != nullptr && blockIdx.x == 0)
-                P.beta_dbg[m] = beta;
+        for (int x = 0; x < NX; ++x) {
+            const int s = __reduce_add_sync(0xffffffffu, sum[x]);
+            if (lane == 0)
+                red_s(x)[m * CWARPS + warp] = s;
         }
     }
-    compute_sync();
-
-    // ---- stream the pieces: piece i = (row block i / KG, k-group i % KG).
-    // Warp w takes pieces w, w + CWARPS, ... of every stage: a fixed number
-    // per stage, fully unrolled, with the (block, group) index of each piece
-    // computed by a multiply-high instead of a division. Each piece's partial
-    // dot product goes straight into the row accumulators, so the pieces of a
-    // stage are independent and their loads and dp4a chains overlap.
-    const int r = lane >> 1;          // row in the block
-    const int t = lane & 1;           // k-half (64 weights) of the group
-    // partial of one piece for token m: sum over its 64 weights of c * x~
-    auto piece_dot = [&](const uint4 &w4, int gg, int m) -> int {
-        const uint8_t *xk = xq_sm + m * K + gg * 128 + t * 64;
-        const uint32_t words[4] = {w4.x, w4.y, w4.z, w4.w};
-        int s1a = 0, s1b = 0, s4a = 0, s4b = 0;
-#pragma unroll
-        for (int jw = 0; jw < 4; ++jw) {
-            const uint4 xv = *reinterpret_cast<const uint4 *>(xk + 16 * jw);
-            const uint32_t w = words[jw], w_hi = w >> 4;
-            // j = 0, 2 at scale 1; j = 1, 3 at scale 4
-            if (jw & 1) {
-                s1b = dp4a_ss(w & 0x03030303u, xv.x, s1b);
-                s4b = dp4a_ss(w & 0x0C0C0C0Cu, xv.y, s4b);
-                s1b = dp4a_ss(w_hi & 0x03030303u, xv.z, s1b);
-                s4b = dp4a_ss(w_hi & 0x0C0C0C0Cu, xv.w, s4b);
-            } else {
-                s1a = dp4a_ss(w & 0x03030303u, xv.x, s1a);
-                s4a = dp4a_ss(w & 0x0C0C0C0Cu, xv.y, s4a);
-                s1a = dp4a_ss(w_hi & 0x03030303u, xv.z, s1a);
-                s4a = dp4a_ss(w_hi & 0x0C0C0C0Cu, xv.w, s4a);
-            }
-        }
-        return s1a + s1b + ((s4a + s4b) >> 2);
-    };
+    // this warp's lanes read the groups its lanes just wrote
+    __syncwarp();
 
     // The next kernel in the stream may start launching now: its weight
     // stream overlaps this main loop and epilogue.
     pdl_launch_dependents();
 
+    const int r = lane >> 1;          // row in the block
+    const int t = lane & 1;           // k-half (64 weights) of the group
     int slot = 0;
     uint32_t phase = 0;
-    for (int st = 0; st < nstages; ++st) {
-        if (!warp_wait_bounded(full(slot), phase, abort_flag, limit))
-            break;
-        const uint8_t *stage = ring + slot * STAGE + lane * 16;
-        const int pbase = st * PIECES_PER_STAGE;
-        auto locate = [&](int local, int &b, int &gg) {
-            const int i = pbase + local;
-            b = static_cast<int>((static_cast<uint64_t>(i) * P.kg_magic) >> 32);
-            gg = i - b * KG;
-        };
-        {
-            // all of this warp's pieces of the slot at once, without branches;
-            // the last slot may be short, and its missing pieces are computed
-            // on stale slot bytes but not committed
-            uint4 wv[PIECES_PER_WARP];
-            int bv[PIECES_PER_WARP], gv[PIECES_PER_WARP];
-            bool ok[PIECES_PER_WARP];
+    bool ok = true;
+    for (int c = 0; c < nchunks; ++c) {
+        const int b0 = c * QB;
+        const int qb = min(QB, nblk - b0);
+        // acc[mat][bi][.]: row sums of this lane's weights (PERSIST: the four
+        // plane sums of token 0 kept apart, combined at the end of the chunk)
+        int acc[NMAT][QB][NACC];
 #pragma unroll
-            for (int u = 0; u < PIECES_PER_WARP; ++u) {
-                const int local = warp + CWARPS * u;
-                ok[u] = pbase + local < npieces;
-                wv[u] = *reinterpret_cast<const uint4 *>(stage + local * PIECE);
-                locate(local, bv[u], gv[u]);
-            }
+        for (int mat = 0; mat < NMAT; ++mat)
 #pragma unroll
-            for (int m = 0; m < MT; ++m) {
-                if (m < M) {
+            for (int bi = 0; bi < QB; ++bi)
 #pragma unroll
-                    for (int u = 0; u < PIECES_PER_WARP; ++u) {
-                        int v = piece_dot(wv[u], gv[u], m);
-                        v += __shfl_xor_sync(0xffffffffu, v, 1);
-                        if (t == 0 && ok[u])
-                            atomicAdd(&acc_sm[(bv[u] * 16 + r) * MT + m], v);
+                for (int j = 0; j < NACC; ++j)
+                    acc[mat][bi][j] = 0;
+
+        for (int ks = 0; ks < kstages; ++ks) {
+            if (ok)
+                ok = warp_wait_bounded(full(slot), phase, abort_flag, limit);
+            if (ok) {
+                const int g0 = ks * G;
+                const int gs = min(G, KG - g0);
+                const uint8_t *stage = ring + slot * slot_bytes + lane * 16;
+                for (int gi = warp; gi < gs; gi += CWARPS) {
+#pragma unroll
+                    for (int m0 = 0; m0 < MT; m0 += TQ) {
+                        if (m0 < M) {
+                            // x~ of this lane's 64 weights for tokens m0 .. m0+TQ-1
+                            uint32_t X[NX][TQ][16];
+#pragma unroll
+                            for (int x = 0; x < NX; ++x) {
+                                const uint8_t *xg = xq_sm + x * p.xq_cap + (g0 + gi) * 128 + t * 64;
+#pragma unroll
+                                for (int mq = 0; mq < TQ; ++mq) {
+#pragma unroll
+                                    for (int v = 0; v < 4; ++v) {
+                                        // tokens past M (a smaller problem of a
+                                        // grouped launch) read nothing
+                                        const uint4 xv = (m0 + mq < M)
+                                                             ? *reinterpret_cast<const uint4 *>(
+                                                                   xg + (m0 + mq) * K + 16 * v)
+                                                             : make_uint4(0, 0, 0, 0);
+                                        X[x][mq][4 * v] = xv.x; X[x][mq][4 * v + 1] = xv.y;
+                                        X[x][mq][4 * v + 2] = xv.z; X[x][mq][4 * v + 3] = xv.w;
+                                    }
+                                }
+                            }
+#pragma unroll
+                            for (int mat = 0; mat < NMAT; ++mat) {
+                                constexpr int XL = NX - 1;
+                                const int xs = mat < NX ? mat : XL;   // the copy this matrix reads
+#pragma unroll
+                                for (int bi = 0; bi < QB; ++bi) {
+                                    if (bi < qb) {
+                                        const uint4 w4 = *reinterpret_cast<const uint4 *>(
+                                            stage + ((mat * qb + bi) * gs + gi) * PIECE);
+                                        const uint32_t wd[4] = {w4.x, w4.y, w4.z, w4.w};
+                                        if constexpr (S::PERSIST) {
+#pragma unroll
+                                            for (int jw = 0; jw < 4; ++jw) {
+                                                acc[mat][bi][0] = dp4a_us(wd[jw] & 0x03030303u, X[xs][0][4 * jw], acc[mat][bi][0]);
+                                                acc[mat][bi][1] = dp4a_us(wd[jw] & 0x0C0C0C0Cu, X[xs][0][4 * jw + 1], acc[mat][bi][1]);
+                                                acc[mat][bi][2] = dp4a_us(wd[jw] & 0x30303030u, X[xs][0][4 * jw + 2], acc[mat][bi][2]);
+                                                acc[mat][bi][3] = dp4a_us(wd[jw] & 0xC0C0C0C0u, X[xs][0][4 * jw + 3], acc[mat][bi][3]);
+                                            }
+                                        } else {
+                                            uint32_t pl[16];
+#pragma unroll
+                                            for (int jw = 0; jw < 4; ++jw) {
+                                                pl[4 * jw] = wd[jw] & 0x03030303u;
+                                                pl[4 * jw + 1] = wd[jw] & 0x0C0C0C0Cu;
+                                                pl[4 * jw + 2] = wd[jw] & 0x30303030u;
+                                                pl[4 * jw + 3] = wd[jw] & 0xC0C0C0C0u;
+                                            }
+#pragma unroll
+                                            for (int mq = 0; mq < TQ; ++mq) {
+                                                int a0 = 0, a1 = 0, a2 = 0, a3 = 0;
+#pragma unroll
+                                                for (int jw = 0; jw < 4; ++jw) {
+                                                    a0 = dp4a_us(pl[4 * jw], X[xs][mq][4 * jw], a0);
+                                                    a1 = dp4a_us(pl[4 * jw + 1], X[xs][mq][4 * jw + 1], a1);
+                                                    a2 = dp4a_us(pl[4 * jw + 2], X[xs][mq][4 * jw + 2], a2);
+                                                    a3 = dp4a_us(pl[4 * jw + 3], X[xs][mq][4 * jw + 3], a3);
+                                                }
+                                                acc[mat][bi][m0 + mq] += a0 + (a1 >> 2) + (a2 >> 4) + (a3 >> 6);
+                                            }
+                                        }
+                                    }
+                                }
+                            }
+                        }
                     }
+                }
+                __syncwarp();
+                if (lane == 0)
+                    mbar_arrive(empty(slot));
+            }
+            if (++slot == slots) {
+                slot = 0;
+                phase ^= 1u;
+            }
+        }
+
+        // ---- chunk epilogue: fold the k-halves, then the warps (in shared
+        // memory); acc = sum c*x~ - sum x~, rescale, bf16
+#pragma unroll
+        for (int mat = 0; mat < NMAT; ++mat) {
+#pragma unroll
+            for (int bi = 0; bi < QB; ++bi) {
+#pragma unroll
+                for (int m = 0; m < MT; ++m) {
+                    int v;
+                    if constexpr (S::PERSIST)
+                        v = acc[mat][bi][0] + (acc[mat][bi][1] >> 2) + (acc[mat][bi][2] >> 4) +
+                            (acc[mat][bi][3] >> 6);
+                    else
+                        v = acc[mat][bi][m];
+                    v += __shfl_xor_sync(0xffffffffu, v, 1);
+                    if (t == 0 && bi < qb)
+                        red[mat * red_stride + (warp * p.red_blocks * 16 + bi * 16 + r) * MT + m] = v;
                 }
             }
         }
-        __syncwarp();
-        if (lane == 0)
-            mbar_arrive(empty(slot));
-        if (++slot == slots) {
-            slot = 0;
-            phase ^= 1u;
-        }
-    }
-    compute_sync();
-
-    // ---- epilogue: acc = sum c*x~ - sum x~, rescale, bf16
-    for (int m = 0; m < M; ++m) {
-        const float s = out_scale(beta_sm[m], P.gamma);
-        int rs = 0;
+        compute_sync();
+        if (!*abort_flag) {
+            const int rows = qb * 16;
+            for (int o = ctid; o < rows * M; o += CTHREADS) {
+                const int m = o / rows;
+                const int rl = o - m * rows;
+                const int n = (blk0 + b0) * 16 + rl;
+                if (n < N) {
+                    // row sum of matrix `mat` minus the sum of the x~ it read
+                    auto row_acc = [&](int mat) {
+                        const int xs = mat < NX ? mat : NX - 1;
+                        int a = 0, s = 0;
 #pragma unroll
-        for (int w = 0; w < CWARPS; ++w)
-            rs += red_i[m * CWARPS + w];
-        for (int rl = ctid; rl < nblk * 16; rl += CTHREADS) {
-            const int n = blk0 * 16 + rl;
-            if (n < N) {
-                const int a = acc_sm[rl * MT + m] - rs;
-                const size_t o = static_cast<size_t>(m) * N + n;
-                P.y[o] = rescale_bf16(a, s);
-                if (P.acc_dbg != nullptr)
-                    P.acc_dbg[o] = a;
+                        for (int w = 0; w < CWARPS; ++w) {
+                            a += red[mat * red_stride + (w * p.red_blocks * 16 + rl) * MT + m];
+                            s += red_s(xs)[m * CWARPS + w];
+                        }
+                        return a - s;
+                    };
+                    const size_t oi = static_cast<size_t>(m) * N + n;
+                    const int a = row_acc(0);
+                    const uint16_t y0 = rescale_bf16(a, out_scale(beta_sm(0)[m], P.gamma));
+                    if constexpr (FFN) {
+                        const uint16_t y1 =
+                            rescale_bf16(row_acc(1), out_scale(beta_sm(NX - 1)[m], P.gamma2));
+                        if (P.y != nullptr)
+                            P.y[oi] = y0;
+                        if (P.y2 != nullptr)
+                            P.y2[oi] = y1;
+                        // h = (r * r) * up with r = max(gate, 0), fp32 (exact
+                        // for bf16 operands)
+                        const float gv = __uint_as_float(static_cast<uint32_t>(y0) << 16);
+                        const float uv = __uint_as_float(static_cast<uint32_t>(y1) << 16);
+                        const float rg = gv > 0.0f ? gv : 0.0f;
+                        P.h[oi] = __fmul_rn(__fmul_rn(rg, rg), uv);
+                    } else {
+                        P.y[oi] = y0;
+                    }
+                    if (P.acc_dbg != nullptr)
+                        P.acc_dbg[oi] = a;
+                }
             }
         }
+        // the reduction area is reused by the next chunk
+        compute_sync();
     }
 }
 

@@ -138,27 +138,27 @@ def test_forward_rmsnorm_rejects_bad_arguments(kw, status):
 
 def test_gemv_admits_what_its_shared_memory_holds():
     # x~ (M * K bytes) must fit beside the GEMV's other shared memory: at
-    # most 196608 bytes, and 196272 for the 16-token tile (M = 9..16). Only
-    # host-side calls here: the sizing function, and forward calls whose
-    # shape is refused before any device work.
+    # most 196608 bytes for every token tile. Only host-side calls here: the
+    # sizing function, and forward calls whose shape is refused before any
+    # device work.
     size_max = ctypes.c_size_t(-1).value
 
     def gemv_ok(M, K):
         return bl.bitlinear_workspace_bytes(M, 64, K, bl.PATH_GEMV) != size_max
-    assert not gemv_ok(16, 12288)                 # 196608 > 196272
-    assert gemv_ok(16, 12160)
-    assert not gemv_ok(12, 16384)
-    assert gemv_ok(8, 24576)                      # 196608, 8-token tile
+    assert gemv_ok(16, 12288)                     # 196608
+    assert not gemv_ok(16, 12416)                 # 198656
+    assert gemv_ok(12, 16384)
+    assert not gemv_ok(12, 16512)
+    assert gemv_ok(8, 24576)
     assert gemv_ok(3, 65536)
     assert not gemv_ok(17, 128)
     L = bl.lib()
-    rc = L.bitlinear_forward_ex(FAKE, 0, 16, 12288, FAKE, 1.0, 64, FAKE, None, 0, None, None,
+    rc = L.bitlinear_forward_ex(FAKE, 0, 16, 12416, FAKE, 1.0, 64, FAKE, None, 0, None, None,
                                 None, None, bl.PATH_GEMV)
     assert rc == bl.BITLINEAR_ERR_SHAPE
-    # a group is one launch: its largest x~ next to its largest token tile
-    big4, small16 = (FAKE, 4, 49152, 64, FAKE, FAKE), (FAKE, 16, 128, 64, FAKE, FAKE)
+    # a group is one launch: its largest x~ must fit
+    big4, small16 = (FAKE, 4, 49280, 64, FAKE, FAKE), (FAKE, 16, 128, 64, FAKE, FAKE)
     assert grouped([big4, small16]) == bl.BITLINEAR_ERR_SHAPE
-
 
 def test_quant_act_rejects_bad_arguments():
     L = bl.lib()
@@ -172,8 +172,13 @@ def test_quant_act_rejects_bad_arguments():
 def test_inject_timeout_rejects_bad_limit():
     L = bl.lib()
     rc = L.bitlinear_forward_inject_timeout(FAKE, 0, 1, 256, FAKE, 1.0, 64, FAKE, FAKE, 4096,
-                                            None, 0)
+                                            None, bl.PATH_TC, 0)
     assert rc == bl.BITLINEAR_ERR_ARG
+    # only an explicit kernel choice is accepted
+    for path in (bl.PATH_AUTO, 3, -1):
+        rc = L.bitlinear_forward_inject_timeout(FAKE, 0, 1, 256, FAKE, 1.0, 64, FAKE, FAKE, 4096,
+                                                None, path, 1000)
+        assert rc == bl.BITLINEAR_ERR_ARG
 
 
 def test_get_fault_rejects_null():
@@ -258,3 +263,42 @@ def test_binding_refuses_host_tensors():
         bl.bitlinear_forward_rmsnorm(x, packed, 1.0, 64, torch.ones(256),
                                      y=torch.zeros((4, 64), dtype=torch.bfloat16),
                                      path=bl.PATH_GEMV)
+
+
+def ffn(M=1, K=256, F=512, x=FAKE, gp=FAKE, up=FAKE, dp=FAKE, gg=None, ug=None, dg=None,
+        eps=2.0 ** -23, h=FAKE, y=FAKE, ws=None, ws_bytes=0, xdt=0):
+    return bl.lib().bitlinear_ffn_forward(x, xdt, M, K, F, gp, 1.0, up, 1.0, dp, 1.0, gg, ug, dg,
+                                          eps, h, y, ws, ws_bytes, None, None, None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(gg=FAKE), bl.BITLINEAR_ERR_ARG),             # gate gains without up gains
+    (dict(ug=FAKE), bl.BITLINEAR_ERR_ARG),
+    (dict(K=200), bl.BITLINEAR_ERR_SHAPE),
+    (dict(F=1000), bl.BITLINEAR_ERR_SHAPE),
+    (dict(M=17), bl.BITLINEAR_ERR_SHAPE),               # the gate/up launch is the GEMV
+    (dict(M=16, K=16384), bl.BITLINEAR_ERR_SHAPE),      # x~ beyond the GEMV's limit
+    (dict(M=8, K=16384, gg=FAKE, ug=FAKE), bl.BITLINEAR_ERR_SHAPE),  # two copies of x~
+    (dict(M=-1), bl.BITLINEAR_ERR_ARG),
+    (dict(xdt=7), bl.BITLINEAR_ERR_DTYPE),
+    (dict(dg=FAKE, eps=0.0), bl.BITLINEAR_ERR_ARG),
+    (dict(gg=FAKE, ug=FAKE, eps=float("nan")), bl.BITLINEAR_ERR_ARG),
+    (dict(h=None), bl.BITLINEAR_ERR_ARG),
+    (dict(dp=None), bl.BITLINEAR_ERR_ARG),
+    (dict(h=FAKE + 4), bl.BITLINEAR_ERR_ALIGN),
+    (dict(y=FAKE + 2), bl.BITLINEAR_ERR_ALIGN),
+    (dict(dg=FAKE + 4), bl.BITLINEAR_ERR_ALIGN),
+    (dict(M=12, K=2560, F=6912), bl.BITLINEAR_ERR_WORKSPACE),   # down projection on tensor cores
+    (dict(M=0, x=None, h=None, y=None), bl.BITLINEAR_OK),       # empty batch: nothing to do
+])
+def test_ffn_forward_rejects_bad_arguments(kw, status):
+    assert ffn(**kw) == status
+
+
+def test_ffn_workspace_is_the_down_projections():
+    size_max = ctypes.c_size_t(-1).value
+    assert bl.bitlinear_workspace_bytes_ffn(1, 2560, 6912) == 0
+    assert (bl.bitlinear_workspace_bytes_ffn(12, 2560, 6912) ==
+            bl.bitlinear_workspace_bytes(12, 2560, 6912))
+    assert bl.bitlinear_workspace_bytes_ffn(17, 2560, 6912) == size_max
+    assert bl.bitlinear_workspace_bytes_ffn(1, 2560, 1000) == size_max

@@ -18,7 +18,7 @@ REACHES_DEVICE = "device"
 
 
 def gemv_fits(M, K):
-    return M <= 16 and M * K <= (196608 if M <= 8 else 196272)
+    return M <= 16 and M * K <= 196608
 
 
 def model(M, K, N, xdt, path, x, packed, y, acc, xq, beta):

@@ -10,7 +10,7 @@ import pytest
 
 import workloads
 import ternary_weight_w1_b200 as bl
-from tests.gpu_cases import Case, bf16_bits_to_tensor, check_y
+from tests.gpu_cases import Case, bf16_bits_to_tensor, check_y, tensor_to_bf16_bits
 
 pytestmark = pytest.mark.gpu
 
@@ -219,17 +219,29 @@ def test_large_sweep(cuda, M):
 
 # ------------------------------------------------- failure detection
 
-def test_bounded_wait_reports_timeout_and_context_survives(cuda):
+@pytest.mark.parametrize("path,M,K,N", [(bl.PATH_TC, 256, 512, 512),
+                                         (bl.PATH_GEMV, 1, 2560, 700),
+                                         (bl.PATH_GEMV, 3, 6912, 300)])
+def test_bounded_wait_reports_timeout_and_context_survives(cuda, path, M, K, N):
+    """One wait made to run out (GEMV: the first weight stage is never loaded;
+    tensor cores: the MMA issuer waits on a barrier nobody arrives at): the
+    fault word reports it, y is left untouched (no partial results), the word
+    is cleared by reading it, and the context still computes correct
+    results."""
     torch = cuda
-    c = Case(256, 512, 512, w_seed=1, x_seed=1)
+    c = Case(M, K, N, w_seed=1, x_seed=1)
     x = c.x_tensor()
     packed = c.packed_tensor()
+    y = torch.full((M, N), float("nan"), dtype=torch.bfloat16, device="cuda")
+    canary = tensor_to_bf16_bits(y)
     assert bl.bitlinear_get_fault() == (bl.BITLINEAR_OK, 0)
-    rc = bl.bitlinear_forward_inject_timeout(x, packed, c.gamma, c.N, timeout_us=2000)
+    rc = bl.bitlinear_forward_inject_timeout(x, packed, c.gamma, c.N, timeout_us=2000, y=y,
+                                             path=path)
     assert rc == bl.BITLINEAR_OK
     status, word = bl.bitlinear_get_fault()
     assert status == bl.BITLINEAR_ERR_TIMEOUT and word == 1
+    np.testing.assert_array_equal(tensor_to_bf16_bits(y), canary)
     # the word is cleared, and the context still runs correct work
     assert bl.bitlinear_get_fault() == (bl.BITLINEAR_OK, 0)
-    assert c.check_full(c.run(path=bl.PATH_TC)) == 1.0
+    assert c.check_full(c.run(path=path)) == 1.0
     assert bl.bitlinear_get_fault() == (bl.BITLINEAR_OK, 0)
