@@ -355,6 +355,26 @@ int bitlinear_forward_grouped_ws(const bitlinear_problem *problems, int count,
                                  bitlinear_dtype xdt, void *workspace_dev,
                                  size_t workspace_bytes, void *cuda_stream);
 
+/* bitlinear_forward_grouped_ws with every problem's tokens RMS-normalised
+ * first (bitlinear_forward_rmsnorm's normalisation), each problem with its
+ * own gains: for example the seven projections of a decoder layer, each
+ * BitLinear with its own nn.RMSNorm as in the page's listing.
+ *   problems, count, xdt, workspace_dev, workspace_bytes, cuda_stream
+ *                  as for bitlinear_forward_grouped_ws (the same workspace
+ *                  size, bitlinear_workspace_bytes_grouped)
+ *   norm_gains_dev [in] host array of count device pointers, the [K] fp32
+ *                  gains of each problem (16-byte aligned; NULL only for a
+ *                  problem with M = 0)
+ *   norm_eps       [in] finite and > 0
+ * One GEMV launch when every problem takes the GEMV path on its own, else
+ * one grouped quantisation launch (which normalises) and one GEMM launch.
+ * Argument errors are reported before any launch. */
+int bitlinear_forward_grouped_rmsnorm(const bitlinear_problem *problems,
+                                      const float *const *norm_gains_dev,
+                                      int count, float norm_eps,
+                                      bitlinear_dtype xdt, void *workspace_dev,
+                                      size_t workspace_bytes, void *cuda_stream);
+
 /* Workspace bytes for an explicit path (see bitlinear_forward_ex); SIZE_MAX
  * for invalid shapes, including those BITLINEAR_PATH_GEMV cannot take. */
 size_t bitlinear_workspace_bytes_path(int64_t M, int64_t N, int64_t K,

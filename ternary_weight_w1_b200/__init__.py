@@ -62,6 +62,7 @@ EXPORTS = (
     "bitlinear_forward_grouped",
     "bitlinear_workspace_bytes_grouped",
     "bitlinear_forward_grouped_ws",
+    "bitlinear_forward_grouped_rmsnorm",
     "bitlinear_workspace_bytes_ffn",
     "bitlinear_ffn_forward",
 )
@@ -127,6 +128,9 @@ def lib() -> ctypes.CDLL:
         L.bitlinear_forward_grouped_ws.restype = ctypes.c_int
         L.bitlinear_forward_grouped_ws.argtypes = [p, ctypes.c_int, ctypes.c_int, p,
                                                    ctypes.c_size_t, p]
+        L.bitlinear_forward_grouped_rmsnorm.restype = ctypes.c_int
+        L.bitlinear_forward_grouped_rmsnorm.argtypes = [p, p, ctypes.c_int, ctypes.c_float,
+                                                        ctypes.c_int, p, sz, p]
         L.bitlinear_workspace_bytes_ffn.restype = sz
         L.bitlinear_workspace_bytes_ffn.argtypes = [i64, i64, i64]
         f32 = ctypes.c_float
@@ -373,6 +377,32 @@ def bitlinear_forward_inject_timeout(x, packed, gamma: float, N: int, timeout_us
         a.ptr(x, "x"), _xdt(x), M, K, a.packed(packed, N, K), float(gamma), N,
         a.ptr(y, "y", torch.bfloat16, (M, N)), a.ptr(workspace, "workspace", torch.uint8),
         workspace.numel(), _stream(stream), int(path), int(timeout_us)))
+
+
+def bitlinear_forward_grouped_rmsnorm(problems, gains, eps: float = RMSNORM_EPS,
+                                      stream=None, workspace=None):
+    """bitlinear_forward_grouped with each problem's tokens RMS-normalised by
+    its own fp32 gains (``gains``: one [K] device tensor per problem).
+    ``workspace`` (bitlinear_workspace_bytes_grouped bytes) is needed when
+    any problem takes the tensor-core path. Returns the list of outputs."""
+    import torch
+    if not problems:
+        return []
+    if len(gains) != len(problems):
+        raise ValueError("one gain tensor per problem")
+    xdt = _xdt(problems[0][0])
+    a = _Args()
+    arr, outs = _problem_array(problems, alloc_y=True, a=a)
+    gp = (ctypes.c_void_p * len(problems))(
+        *[a.ptr(g, f"gains[{i}]", torch.float32, (problems[i][0].shape[1],))
+          for i, g in enumerate(gains)])
+    ws = None if workspace is None else a.ptr(workspace, "workspace", torch.uint8)
+    ws_bytes = 0 if workspace is None else workspace.numel()
+    _check(lib().bitlinear_forward_grouped_rmsnorm(ctypes.addressof(arr), ctypes.addressof(gp),
+                                                   len(problems), float(eps), xdt, ws, ws_bytes,
+                                                   _stream(stream)),
+           "bitlinear_forward_grouped_rmsnorm")
+    return outs
 
 
 def bitlinear_workspace_bytes_ffn(M: int, K: int, F: int) -> int:

@@ -346,23 +346,50 @@ int launch_gemv(const GemvJob *jobs, int count, bitlinear_dtype xdt, const Devic
     const int MT = gemv_tile(Mmax);
     const int QB = gemv::chunk_blocks(MT, ffn);
     const int nmat = ffn ? 2 : 1;
-    double target = std::min(64.0 * 1024, std::max(16.0 * 1024, total_bytes / (2.0 * dev.sms)));
+    int blocks[gemv::MAX_PROBLEMS], ctas[gemv::MAX_PROBLEMS], G[gemv::MAX_PROBLEMS];
+    double bbytes[gemv::MAX_PROBLEMS];
+    double max_block = 0.0;
+    for (int i = 0; i < count; ++i) {
+        blocks[i] = (jobs[i].N + 15) / 16;
+        bbytes[i] = nmat * 16.0 * jobs[i].K / 4.0;
+        max_block = std::max(max_block, bbytes[i]);
+    }
+    // CTAs: one wave of two per SM (a third fits beside them, for the next
+    // kernel under programmatic dependent launch). One problem spreads its
+    // blocks over min(blocks, 2 * SMs) CTAs, as evenly as whole blocks allow.
+    // A group gives every CTA about the same bytes: each problem's CTAs hold at
+    // most `target` bytes, the launch's bytes spread over two CTAs per SM (10%
+    // slack, and at least one block), raised while the grid exceeds three CTAs
+    // per SM.
+    if (count == 1) {
+        ctas[0] = std::min(blocks[0], 2 * dev.sms);
+    } else {
+        double target = std::max(max_block, 1.1 * total_bytes / (2.0 * dev.sms));
+        for (int attempt = 0;; ++attempt) {
+            int grid = 0;
+            for (int i = 0; i < count; ++i) {
+                const int q = std::max(1, static_cast<int>(target / bbytes[i]));
+                ctas[i] = (blocks[i] + q - 1) / q;
+                grid += ctas[i];
+            }
+            if (grid <= 3 * dev.sms || attempt > 64)
+                break;
+            target *= 1.25;
+        }
+    }
+    int grid = 0;
+    for (int i = 0; i < count; ++i)
+        grid += ctas[i];
     int gcap = 1 << 30;               // upper bound on k-groups per stage
-    int q[gemv::MAX_PROBLEMS], ctas[gemv::MAX_PROBLEMS], G[gemv::MAX_PROBLEMS];
-    int grid = 0, slot_bytes = 0, slots = 0, red_blocks = 1, smem = 0;
+    int slot_bytes = 0, slots = 0, red_blocks = 1, smem = 0;
     for (int attempt = 0;; ++attempt) {
-        grid = 0;
         slot_bytes = 0;
         red_blocks = 1;
         int stages = 1;
         for (int i = 0; i < count; ++i) {
-            const int blocks = (jobs[i].N + 15) / 16;
             const int KG = jobs[i].K / 128;
-            const double block_bytes = nmat * 16.0 * jobs[i].K / 4.0;
-            q[i] = std::max(1, std::min(blocks, static_cast<int>(target / block_bytes + 0.5)));
-            ctas[i] = (blocks + q[i] - 1) / q[i];
-            grid += ctas[i];
-            const int qb = std::min(q[i], QB);
+            const int q = (blocks[i] + ctas[i] - 1) / ctas[i];
+            const int qb = std::min(q, QB);
             // about 16 KiB per stage: G a multiple of 8 (each warp owns the
             // groups of one residue mod 8), or the whole row when that is less
             int g = std::max(8, (16384 / (nmat * qb * gemv::PIECE)) & ~7);
@@ -370,7 +397,7 @@ int launch_gemv(const GemvJob *jobs, int count, bitlinear_dtype xdt, const Devic
             G[i] = g >= KG ? KG : g;
             slot_bytes = std::max(slot_bytes, nmat * qb * G[i] * gemv::PIECE);
             red_blocks = std::max(red_blocks, qb);
-            stages = std::max(stages, ((q[i] + QB - 1) / QB) * ((KG + G[i] - 1) / G[i]));
+            stages = std::max(stages, ((q + QB - 1) / QB) * ((KG + G[i] - 1) / G[i]));
         }
         // Ring depth: the whole share when it is small, else as deep as a
         // 72 KiB block allows (three blocks per SM fit beside each other).
@@ -380,15 +407,10 @@ int launch_gemv(const GemvJob *jobs, int count, bitlinear_dtype xdt, const Devic
         smem = gemv::smem_bytes(MT, xq_cap, slots, slot_bytes, red_blocks, norm, ffn);
         if (smem <= dev.max_smem_optin)
             break;
-        // too large beside a large x~: smaller stages first, then fewer
-        // blocks per CTA
-        if (gcap > 8)
+        // too large beside a large x~: smaller stages
+        if (gcap > 8 && attempt < 8)
             gcap = (gcap > 64 ? 64 : gcap) / 2;
-        else if (target > 1024.0)
-            target /= 2.0;
         else
-            return BITLINEAR_ERR_SHAPE;
-        if (attempt > 64)
             return BITLINEAR_ERR_SHAPE;
     }
     gemv::Params p = {};
@@ -407,7 +429,8 @@ int launch_gemv(const GemvJob *jobs, int count, bitlinear_dtype xdt, const Devic
                                   j.gamma,
                                   j.norm_gain,
                                   j.norm_eps,
-                                  q[i],
+                                  blocks[i] / ctas[i],
+                                  blocks[i] % ctas[i],
                                   begin,
                                   G[i],
                                   static_cast<const uint8_t *>(j.packed2),
@@ -504,7 +527,9 @@ int launch_gemm_ws(const wsg::Maps &maps, const wsg::Params &p, int grid, const 
     return launch_status(e);
 }
 
-// Quantisation of several problems' rows in one launch (one warp per row).
+// Quantisation of several problems' rows in one launch (WPR warps per row),
+// RMS-normalising each problem's rows with its own gains when they are given
+// (all problems or none).
 template <bool BF16, int CACHE, int WPR>
 cudaError_t launch_qa_group(const TcJob *jobs, int n, int8_t *const *xq, float *const *beta,
                             int *const *rowsum, cudaStream_t st, int *clear, int n_clear)
@@ -513,15 +538,19 @@ cudaError_t launch_qa_group(const TcJob *jobs, int n, int8_t *const *xq, float *
     qa::GroupParams g{};
     int blocks = 0;
     for (int i = 0; i < n; ++i) {
-        g.prob[i] = qa::GroupRows{jobs[i].x, xq[i], beta[i], rowsum[i], jobs[i].M, jobs[i].K,
-                                  blocks};
+        g.prob[i] = qa::GroupRows{jobs[i].x,        xq[i],    beta[i], rowsum[i],
+                                  jobs[i].M,        jobs[i].K, blocks, jobs[i].norm_gain,
+                                  jobs[i].norm_eps};
         blocks += (jobs[i].M + rpb - 1) / rpb;
     }
     g.count = n;
     g.clear = clear;
     g.n_clear = n_clear;
-    return launch(qa::quant_act_grouped_kernel<BF16, CACHE, WPR>, dim3(blocks), dim3(qa::THREADS),
-                  0, st, g);
+    if (jobs[0].norm_gain != nullptr)
+        return launch(qa::quant_act_grouped_kernel<BF16, CACHE, WPR, true>, dim3(blocks),
+                      dim3(qa::THREADS), 0, st, g);
+    return launch(qa::quant_act_grouped_kernel<BF16, CACHE, WPR, false>, dim3(blocks),
+                  dim3(qa::THREADS), 0, st, g);
 }
 
 // Warps per row chosen by the group's longest row, as for one problem.
@@ -565,10 +594,9 @@ int run_tc_group(const TcJob *jobs, int n, bitlinear_dtype xdt, void *ws, size_t
     const size_t need = tc_group_bytes(jobs, n, split);
     if (ws == nullptr || ws_bytes < need)
         return BITLINEAR_ERR_WORKSPACE;
-    if (n > 1)
-        for (int i = 0; i < n; ++i)
-            if (jobs[i].norm_gain != nullptr)     // the grouped quantiser does not normalise
-                return BITLINEAR_ERR_ARG;
+    for (int i = 1; i < n; ++i)                   // normalise every problem or none
+        if ((jobs[i].norm_gain != nullptr) != (jobs[0].norm_gain != nullptr))
+            return BITLINEAR_ERR_ARG;
     if (!aligned(ws, 256))
         return BITLINEAR_ERR_ALIGN;
     int max_M = 0;
@@ -974,7 +1002,8 @@ namespace {
 // problems. Sets *all_gemv when every one of them fits the GEMV path at the
 // automatic threshold.
 int collect_group(const bitlinear_problem *problems, int count, int xdt, TcJob *jobs, int *n,
-                  bool *all_gemv, bool shapes_only = false)
+                  bool *all_gemv, bool shapes_only = false,
+                  const float *const *gains = nullptr, float eps = 0.0f)
 {
     if (problems == nullptr || count < 1 || count > wsg::MAX_PROBLEMS)
         return BITLINEAR_ERR_ARG;
@@ -997,9 +1026,16 @@ int collect_group(const bitlinear_problem *problems, int count, int xdt, TcJob *
             *all_gemv = false;
         max_M = std::max(max_M, pr.M);
         max_xq = std::max(max_xq, pr.M * pr.K);
-        jobs[(*n)++] = TcJob{pr.x_dev,      static_cast<int>(pr.M), static_cast<int>(pr.K),
-                             static_cast<int>(pr.N), pr.packed_dev, pr.gamma, pr.y_dev, nullptr,
-                             nullptr, 0.0f};
+        jobs[(*n)++] = TcJob{pr.x_dev,
+                             static_cast<int>(pr.M),
+                             static_cast<int>(pr.K),
+                             static_cast<int>(pr.N),
+                             pr.packed_dev,
+                             pr.gamma,
+                             pr.y_dev,
+                             nullptr,
+                             gains != nullptr ? gains[i] : nullptr,
+                             eps};
     }
     // one GEMV launch holds the largest x~ next to the largest problem's token tile
     if (*n > 0 && max_xq > gemv_max_xq(max_M))
@@ -1045,6 +1081,49 @@ extern "C" int bitlinear_forward_grouped_ws(const bitlinear_problem *problems, i
             g[i] = GemvJob{jobs[i].x,     jobs[i].M, jobs[i].K, jobs[i].N, jobs[i].packed,
                            jobs[i].gamma, jobs[i].y, nullptr,   nullptr,   nullptr,
                            nullptr,       0.0f};
+        return launch_gemv(g, n, xdt, *dev, st);
+    }
+    return run_tc_group(jobs, n, xdt, workspace_dev, workspace_bytes, nullptr, nullptr, *dev, st,
+                        0, true);
+}
+
+extern "C" int bitlinear_forward_grouped_rmsnorm(const bitlinear_problem *problems,
+                                                 const float *const *norm_gains_dev, int count,
+                                                 float norm_eps, bitlinear_dtype xdt,
+                                                 void *workspace_dev, size_t workspace_bytes,
+                                                 void *cuda_stream)
+{
+    if (problems == nullptr || norm_gains_dev == nullptr || count < 1 ||
+        count > wsg::MAX_PROBLEMS)
+        return BITLINEAR_ERR_ARG;
+    if (!(norm_eps > 0.0f) || !(norm_eps <= FLT_MAX))
+        return BITLINEAR_ERR_ARG;
+    for (int i = 0; i < count; ++i) {
+        if (problems[i].M > 0 && norm_gains_dev[i] == nullptr)
+            return BITLINEAR_ERR_ARG;
+        if (!aligned(norm_gains_dev[i], 16))
+            return BITLINEAR_ERR_ALIGN;
+    }
+    TcJob jobs[wsg::MAX_PROBLEMS];
+    int n = 0;
+    bool all_gemv = true;
+    int rc = collect_group(problems, count, xdt, jobs, &n, &all_gemv, false, norm_gains_dev,
+                           norm_eps);
+    if (rc != BITLINEAR_OK)
+        return rc;
+    if (n == 0)
+        return BITLINEAR_OK;
+    DeviceInfo *dev = nullptr;
+    rc = current_device(&dev);
+    if (rc != BITLINEAR_OK)
+        return rc;
+    cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
+    if (all_gemv) {
+        GemvJob g[wsg::MAX_PROBLEMS];
+        for (int i = 0; i < n; ++i)
+            g[i] = GemvJob{jobs[i].x,     jobs[i].M, jobs[i].K, jobs[i].N, jobs[i].packed,
+                           jobs[i].gamma, jobs[i].y, nullptr,   nullptr,   nullptr,
+                           jobs[i].norm_gain, jobs[i].norm_eps};
         return launch_gemv(g, n, xdt, *dev, st);
     }
     return run_tc_group(jobs, n, xdt, workspace_dev, workspace_bytes, nullptr, nullptr, *dev, st,

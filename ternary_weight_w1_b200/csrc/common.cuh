@@ -101,6 +101,57 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
     }
 }
 
+// mbarrier.try_wait with a suspend-time hint: a thread whose phase has not
+// completed sleeps until it does or about hint_ns nanoseconds pass, instead of
+// spinning (the waiting warps then take no issue slots from working ones).
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parity,
+                                                    uint32_t hint_ns)
+{
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done)
+        : "r"(bar), "r"(parity), "r"(hint_ns)
+        : "memory");
+    return done != 0;
+}
+
+// mbar_wait_bounded for long waits (data from HBM): each try sleeps up to
+// 20 us, and the limit and the abort flag are checked after every try.
+__device__ __forceinline__ bool mbar_wait_sleep_bounded(uint32_t bar, uint32_t parity,
+                                                        volatile int *abort, uint64_t limit_ns)
+{
+    if (mbar_try_wait_sleep(bar, parity, 20000u))
+        return true;
+    const uint64_t t0 = global_timer_ns();
+    for (;;) {
+        if (mbar_try_wait_sleep(bar, parity, 20000u))
+            return true;
+        if (*abort)
+            return false;
+        if (global_timer_ns() - t0 > limit_ns) {
+            atomicOr(&g_fault_word, FAULT_WAIT_TIMEOUT);
+            *abort = 1;
+            return false;
+        }
+    }
+}
+
+// Lane 0 waits (sleeping between tries), the verdict is broadcast, and the
+// warp re-converges.
+__device__ __forceinline__ bool warp_wait_sleep_bounded(uint32_t bar, uint32_t parity,
+                                                        volatile int *abort, uint64_t limit_ns)
+{
+    int ok = 0;
+    if ((threadIdx.x & 31) == 0)
+        ok = mbar_wait_sleep_bounded(bar, parity, abort, limit_ns) ? 1 : 0;
+    ok = __shfl_sync(0xffffffffu, ok, 0);
+    __syncwarp();
+    return ok != 0;
+}
+
 // Lane 0 waits, the verdict is broadcast, and the warp re-converges.
 __device__ __forceinline__ bool warp_wait_bounded(uint32_t bar, uint32_t parity,
                                                   volatile int *abort, uint64_t limit_ns)

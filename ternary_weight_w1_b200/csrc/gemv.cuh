@@ -74,7 +74,7 @@ constexpr int PIECE = 512;                         // one (row block, k-group)
 constexpr int MAX_SLOTS = 8;
 constexpr int BAR_BYTES = 2 * MAX_SLOTS * 8 + 16;  // full/empty barriers + abort flag
 constexpr int MAX_PROBLEMS = 8;
-constexpr int XCACHE = 4;                          // groups of token 0 kept through the prologue
+constexpr int XCACHE = 4;                          // 16-byte slots of token 0 kept through the prologue
 
 // Row blocks per chunk and tokens whose x~ a lane holds in registers at once,
 // by token tile MT. Only MT = 1 keeps the four plane sums apart for a whole
@@ -87,7 +87,7 @@ struct Shape {
     static constexpr bool PERSIST = MT == 1;
     // blocks per SM the register budget is set for: three for the small
     // tiles (two of this launch and, under programmatic dependent launch, one
-    // of the next), two for the larger ones
+    // of the next), two for the larger ones and the normalising forms
     static constexpr int MIN_BLOCKS = (MT <= 2 && !FFN) ? 3 : 2;
 };
 
@@ -109,7 +109,8 @@ struct Problem {
     float gamma;
     const float *norm_gain; // [K] RMS-normalisation gains (NORM launches only)
     float norm_eps;         // eps of the normalisation (NORM launches only)
-    int blocks_per_cta;     // row blocks of 16 rows owned by one CTA
+    int base, extra;        // row blocks of 16 rows per CTA: base, one more for the
+                            // problem's first `extra` CTAs
     int cta_begin;          // this problem's first CTA in the grid
     int G;                  // k-groups per stage (a multiple of 8, or all K/128)
     // FFN launches only: `packed`, `gamma`, `norm_gain` and `y` (optional)
@@ -187,7 +188,7 @@ __device__ __forceinline__ void load4(const void *row, int e, float (&v)[4])
 }
 
 template <int MT, bool BF16, bool NORM, bool FFN>
-__global__ void __launch_bounds__(THREADS, (Shape<MT, FFN>::MIN_BLOCKS))
+__global__ void __launch_bounds__(THREADS, (NORM ? 2 : Shape<MT, FFN>::MIN_BLOCKS))
 gemv_kernel(const __grid_constant__ Params p)
 {
     using S = Shape<MT, FFN>;
@@ -208,8 +209,9 @@ gemv_kernel(const __grid_constant__ Params p)
     const int KG = K >> 7;                              // k-groups per row
     const int G = P.G;
     const int total_blocks = (N + 15) >> 4;
-    const int blk0 = (static_cast<int>(blockIdx.x) - P.cta_begin) * P.blocks_per_cta;
-    const int nblk = min(P.blocks_per_cta, total_blocks - blk0);
+    const int cta = static_cast<int>(blockIdx.x) - P.cta_begin;
+    const int blk0 = cta * P.base + min(cta, P.extra);
+    const int nblk = min(P.base + (cta < P.extra ? 1 : 0), total_blocks - blk0);
     const int nchunks = (nblk + QB - 1) / QB;
     const int kstages = (KG + G - 1) / G;
     const int nstages = nchunks * kstages;
@@ -264,7 +266,8 @@ gemv_kernel(const __grid_constant__ Params p)
         uint32_t parity = 0;       // the phase of that copy, per slot
         for (int st = 0; st < nstages; ++st) {
             // from the second pass on, the slot must have been released
-            if (st >= slots && !warp_wait_bounded(empty(slot), phase ^ 1u, abort_flag, limit))
+            if (st >= slots &&
+                !warp_wait_sleep_bounded(empty(slot), phase ^ 1u, abort_flag, limit))
                 break;
             const int c = st / kstages;
             const int ks = st - c * kstages;
@@ -311,76 +314,84 @@ gemv_kernel(const __grid_constant__ Params p)
 
     // x may be the previous kernel's output: read it only after the wait.
     pdl_wait();
-    // Element e of token m is at (warp + 8 i) * 128 + 4 * lane for this
-    // thread's i-th group. Token 0's first XCACHE groups stay in registers
-    // between the passes; the rest are read again (from L1 or L2).
-    auto elem = [&](int i) { return (warp + CWARPS * i) * 128 + 4 * lane; };
+    // Slot i of this thread: group g = warp + 8 (2 i + h), h = lane / 16 (two
+    // of this warp's groups per slot), elements 128 g + 8 (lane % 16) .. + 7,
+    // one 16-byte load of bf16 (two of fp32). Token 0's first XCACHE slots
+    // stay in registers between the passes; the rest are read again, XB
+    // slots at a time so that their loads are in flight together.
+    const int h = lane >> 4;
+    auto slot_group = [&](int i) { return warp + CWARPS * (2 * i + h); };
+    auto slot_elem = [&](int i) { return slot_group(i) * 128 + 8 * (lane & 15); };
+    const int nsl = (ngw + 1) / 2;                    // slots of this warp
     // gains of quantised copy x (FFN: 0 = gate, 1 = up)
     auto gain_of = [&](int x) { return (FFN && x == 1) ? P.norm_gain2 : P.norm_gain; };
-    float xc[XCACHE][4];
-    // groups whose loads are issued together (their latencies overlap)
-    constexpr int XB = NORM ? 2 : 4;
-    // Visits this thread's groups of token m: f(i, v, g) with v the four raw
-    // activations and, when `gains` is set (NORM launches), g the four gains
-    // of each quantised copy. Token 0's first XCACHE groups come from the
-    // registers once `fill` has stored them there.
-    auto for_groups = [&](int m, bool fill, bool gains, auto &&f) {
+    Vec8<BF16> xc[XCACHE];
+    // slots whose loads are issued together, and gain loads of cached slots
+    constexpr int XB = NORM ? 2 : (BF16 ? 4 : 2);
+    constexpr int XG = NORM ? 2 : XCACHE;
+    using Gains = float[NX][8];
+    // Visits this thread's valid slots of token m: f(i, v, g) with v the eight
+    // raw activations and, when `gains` is set (NORM launches), g the eight
+    // gains of each quantised copy.
+    auto for_slots = [&](int m, bool fill, bool gains, auto &&f) {
         const void *row = static_cast<const char *>(P.x) + m * row_bytes;
-        int i0 = 0;
-        if (m == 0) {
-            float g[XCACHE][NX][4];
+        auto valid = [&](int i) { return i < nsl && slot_group(i) < KG; };
+        auto load_gains = [&](int i, Gains &g) {
+            if constexpr (NORM) {
+                if (gains) {
 #pragma unroll
-            for (int i = 0; i < XCACHE; ++i) {
-                if (i < ngw) {
-                    if (fill)
-                        load4<BF16>(row, elem(i), xc[i]);
-                    if constexpr (NORM) {
-                        if (gains) {
-#pragma unroll
-                            for (int x = 0; x < NX; ++x)
-                                load4<false>(gain_of(x), elem(i), g[i][x]);
-                        }
-                    }
+                    for (int x = 0; x < NX; ++x)
+                        load8<false>(gain_of(x), slot_elem(i), g[x]);
                 }
             }
+        };
+        int i0 = 0;
+        if (m == 0) {
+            if (fill) {
 #pragma unroll
-            for (int i = 0; i < XCACHE; ++i)
-                if (i < ngw)
-                    f(i, xc[i], g[i]);
+                for (int i = 0; i < XCACHE; ++i)
+                    if (valid(i))
+                        xc[i].load(row, slot_elem(i));
+            }
+#pragma unroll
+            for (int ic = 0; ic < XCACHE; ic += XG) {
+                float g[XG][NX][8];
+#pragma unroll
+                for (int u = 0; u < XG; ++u)
+                    if (valid(ic + u))
+                        load_gains(ic + u, g[u]);
+#pragma unroll
+                for (int u = 0; u < XG; ++u)
+                    if (valid(ic + u))
+                        f(ic + u, xc[ic + u], g[u]);
+            }
             i0 = XCACHE;
         }
-        for (int ib = i0; ib < ngw; ib += XB) {
-            float v[XB][4];
-            float g[XB][NX][4];
+        for (int ib = i0; ib < nsl; ib += XB) {
+            Vec8<BF16> v[XB];
+            float g[XB][NX][8];
 #pragma unroll
             for (int u = 0; u < XB; ++u) {
-                if (ib + u < ngw) {
-                    load4<BF16>(row, elem(ib + u), v[u]);
-                    if constexpr (NORM) {
-                        if (gains) {
-#pragma unroll
-                            for (int x = 0; x < NX; ++x)
-                                load4<false>(gain_of(x), elem(ib + u), g[u][x]);
-                        }
-                    }
+                if (valid(ib + u)) {
+                    v[u].load(row, slot_elem(ib + u));
+                    load_gains(ib + u, g[u]);
                 }
             }
 #pragma unroll
             for (int u = 0; u < XB; ++u)
-                if (ib + u < ngw)
+                if (valid(ib + u))
                     f(ib + u, v[u], g[u]);
         }
     };
-    using Gains = float[NX][4];
 
     if constexpr (NORM) {
         // sums of squares per token
         for (int m = 0; m < M; ++m) {
             double ss = 0.0;
-            for_groups(m, true, false, [&](int, const float (&v)[4], const Gains &) {
+            for_slots(m, true, false, [&](int, const Vec8<BF16> &v, const Gains &) {
 #pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const double d = v[u];
+                for (int u = 0; u < 8; ++u) {
+                    const double d = v.get(u);
                     ss = __fma_rn(d, d, ss);
                 }
             });
@@ -399,12 +410,12 @@ gemv_kernel(const __grid_constant__ Params p)
 #pragma unroll
         for (int x = 0; x < NX; ++x)
             amax[x] = 0.0f;
-        for_groups(m, !NORM, true, [&](int, const float (&v)[4], const Gains &g) {
+        for_slots(m, !NORM, true, [&](int, const Vec8<BF16> &v, const Gains &g) {
 #pragma unroll
             for (int x = 0; x < NX; ++x) {
 #pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    float a = v[u];
+                for (int u = 0; u < 8; ++u) {
+                    float a = v.get(u);
                     if constexpr (NORM)
                         a = norm1(a, r, g[x][u]);
                     amax[x] = fmaxf(amax[x], fabsf(a));
@@ -442,30 +453,35 @@ gemv_kernel(const __grid_constant__ Params p)
                     P.beta_dbg[m] = beta;
             }
         }
-        for_groups(m, false, true, [&](int i, const float (&v)[4], const Gains &g) {
-            const int e = elem(i);
+        for_slots(m, false, true, [&](int i, const Vec8<BF16> &v, const Gains &g) {
+            const int e = slot_elem(i);
 #pragma unroll
             for (int x = 0; x < NX; ++x) {
-                uint32_t word = 0;
+                uint32_t lo = 0, hi = 0;
 #pragma unroll
                 for (int u = 0; u < 4; ++u) {
-                    float a = v[u];
-                    if constexpr (NORM)
+                    float a = v.get(u), b = v.get(u + 4);
+                    if constexpr (NORM) {
                         a = norm1(a, r, g[x][u]);
-                    const int q = quant1(a, scale[x]);
-                    sum[x] += q;
-                    word |= (static_cast<uint32_t>(q) & 0xffu) << (8 * u);
+                        b = norm1(b, r, g[x][u + 4]);
+                    }
+                    const int qa = quant1(a, scale[x]);
+                    const int qb = quant1(b, scale[x]);
+                    sum[x] += qa + qb;
+                    lo |= (static_cast<uint32_t>(qa) & 0xffu) << (8 * u);
+                    hi |= (static_cast<uint32_t>(qb) & 0xffu) << (8 * u);
                 }
-                *reinterpret_cast<uint32_t *>(xq_sm + x * p.xq_cap + m * K + e) = word;
+                *reinterpret_cast<uint2 *>(xq_sm + x * p.xq_cap + m * K + e) = make_uint2(lo, hi);
                 if (x == 0 && P.xq_dbg != nullptr && first_cta)
-                    *reinterpret_cast<uint32_t *>(P.xq_dbg + static_cast<size_t>(m) * K + e) = word;
+                    *reinterpret_cast<uint2 *>(P.xq_dbg + static_cast<size_t>(m) * K + e) =
+                        make_uint2(lo, hi);
             }
         });
 #pragma unroll
         for (int x = 0; x < NX; ++x) {
-            const int s = __reduce_add_sync(0xffffffffu, sum[x]);
+            const int sm = __reduce_add_sync(0xffffffffu, sum[x]);
             if (lane == 0)
-                red_s(x)[m * CWARPS + warp] = s;
+                red_s(x)[m * CWARPS + warp] = sm;
         }
     }
     // this warp's lanes read the groups its lanes just wrote
@@ -496,7 +512,7 @@ gemv_kernel(const __grid_constant__ Params p)
 
         for (int ks = 0; ks < kstages; ++ks) {
             if (ok)
-                ok = warp_wait_bounded(full(slot), phase, abort_flag, limit);
+                ok = warp_wait_sleep_bounded(full(slot), phase, abort_flag, limit);
             if (ok) {
                 const int g0 = ks * G;
                 const int gs = min(G, KG - g0);
@@ -531,7 +547,9 @@ gemv_kernel(const __grid_constant__ Params p)
                                 const int xs = mat < NX ? mat : XL;   // the copy this matrix reads
 #pragma unroll
                                 for (int bi = 0; bi < QB; ++bi) {
-                                    if (bi < qb) {
+                                    if (bi >= qb)
+                                        break;
+                                    {
                                         const uint4 w4 = *reinterpret_cast<const uint4 *>(
                                             stage + ((mat * qb + bi) * gs + gi) * PIECE);
                                         const uint32_t wd[4] = {w4.x, w4.y, w4.z, w4.w};
@@ -587,6 +605,8 @@ gemv_kernel(const __grid_constant__ Params p)
         for (int mat = 0; mat < NMAT; ++mat) {
 #pragma unroll
             for (int bi = 0; bi < QB; ++bi) {
+                if (bi >= qb)
+                    break;
 #pragma unroll
                 for (int m = 0; m < MT; ++m) {
                     int v;
@@ -596,7 +616,7 @@ gemv_kernel(const __grid_constant__ Params p)
                     else
                         v = acc[mat][bi][m];
                     v += __shfl_xor_sync(0xffffffffu, v, 1);
-                    if (t == 0 && bi < qb)
+                    if (t == 0)
                         red[mat * red_stride + (warp * p.red_blocks * 16 + bi * 16 + r) * MT + m] = v;
                 }
             }

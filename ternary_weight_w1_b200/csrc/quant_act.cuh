@@ -8,7 +8,8 @@
 // activations in registers from the absmax pass, so a row is read from
 // memory once when 32 * WPR * 8 * CACHE covers it; anything beyond is
 // re-read in the second pass, four vectors in flight per lane. A grouped
-// variant quantises the rows of several problems in one launch.
+// variant quantises the rows of several problems in one launch (each with
+// its own gains when it normalises).
 //
 // With NORM the row is RMS-normalised first, as the listing's BitLinear does
 // with its nn.RMSNorm member before quantising: a first pass sums the squares
@@ -245,6 +246,8 @@ struct GroupRows {
     int *rowsum;
     int M, K;
     int first_block;
+    const float *gain;      // [K] RMS-normalisation gains (NORM launches only)
+    float eps;
 };
 
 struct GroupParams {
@@ -254,7 +257,7 @@ struct GroupParams {
     int n_clear;
 };
 
-template <bool BF16, int CACHE, int WPR>
+template <bool BF16, int CACHE, int WPR, bool NORM>
 __global__ void __launch_bounds__(THREADS)
 quant_act_grouped_kernel(const __grid_constant__ GroupParams g)
 {
@@ -268,8 +271,8 @@ quant_act_grouped_kernel(const __grid_constant__ GroupParams g)
     if (g.clear != nullptr && blockIdx.x == 0)
         for (int i = threadIdx.x; i < g.n_clear; i += THREADS)
             g.clear[i] = 0;
-    quant_row<BF16, CACHE, WPR, false>(r.x, r.M, r.K, r.xq, r.beta, r.rowsum, nullptr, 0.0f, m,
-                                       warp % WPR);
+    quant_row<BF16, CACHE, WPR, NORM>(r.x, r.M, r.K, r.xq, r.beta, r.rowsum, r.gain, r.eps, m,
+                                      warp % WPR);
 }
 
 }  // namespace qa

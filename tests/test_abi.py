@@ -302,3 +302,28 @@ def test_ffn_workspace_is_the_down_projections():
             bl.bitlinear_workspace_bytes(12, 2560, 6912))
     assert bl.bitlinear_workspace_bytes_ffn(17, 2560, 6912) == size_max
     assert bl.bitlinear_workspace_bytes_ffn(1, 2560, 1000) == size_max
+
+
+def test_grouped_rmsnorm_rejects_bad_arguments():
+    L = bl.lib()
+    good = (FAKE, 1, 256, 64, FAKE, FAKE)
+
+    def call(problems, gains, eps=2.0 ** -23, count=None):
+        arr = (bl._Problem * max(1, len(problems)))()
+        for i, (x, M, K, N, packed, y) in enumerate(problems):
+            arr[i] = bl._Problem(x, M, K, N, packed, 1.0, y)
+        g = None if gains is None else (ctypes.c_void_p * max(1, len(gains)))(*gains)
+        n = len(problems) if count is None else count
+        return L.bitlinear_forward_grouped_rmsnorm(ctypes.addressof(arr),
+                                                   None if g is None else ctypes.addressof(g),
+                                                   n, eps, 0, None, 0, None)
+    assert call([good], None) == bl.BITLINEAR_ERR_ARG              # no gains array
+    assert call([good], [None]) == bl.BITLINEAR_ERR_ARG            # a missing gain
+    assert call([good], [FAKE + 4]) == bl.BITLINEAR_ERR_ALIGN
+    assert call([good], [FAKE], eps=0.0) == bl.BITLINEAR_ERR_ARG
+    assert call([good], [FAKE], eps=float("inf")) == bl.BITLINEAR_ERR_ARG
+    assert call([good], [FAKE], count=0) == bl.BITLINEAR_ERR_ARG
+    assert call([good] * 9, [FAKE] * 9) == bl.BITLINEAR_ERR_ARG
+    assert call([(FAKE, 1, 200, 64, FAKE, FAKE)], [FAKE]) == bl.BITLINEAR_ERR_SHAPE
+    # an empty batch needs no gain and does nothing
+    assert call([(FAKE, 0, 256, 64, FAKE, FAKE)], [None]) == bl.BITLINEAR_OK

@@ -124,3 +124,41 @@ def test_grouped_ws_small_batches_use_gemv():
     ys = run_group_ws(cases)
     for c, y in zip(cases, ys):
         assert check_y(y, c.oracle_full()[1]) == 1.0
+
+
+# ------------------------------------------- grouped, RMS-normalised tokens
+
+def run_group_norm(cases, gains, eps=bl.RMSNORM_EPS):
+    import torch
+    probs, guards = _guarded_problems(cases, None)
+    need = bl.bitlinear_workspace_bytes_grouped(probs)
+    ws = torch.empty((max(need, 1),), dtype=torch.uint8, device="cuda")
+    g_dev = [torch.from_numpy(g).cuda() for g in gains]
+    bl.bitlinear_forward_grouped_rmsnorm(probs, g_dev, eps=eps, workspace=ws)
+    torch.cuda.synchronize()
+    return _read(guards)
+
+
+@pytest.mark.parametrize("B", [1, 8, 64])
+def test_grouped_rmsnorm_layer_matches_oracle(B):
+    """The seven projections of a decoder layer, each normalising its tokens
+    with its own gains (GEMV launch at B = 1, grouped quantisation and GEMM
+    at B = 8 and 64), against the oracle's RMSNorm + forward. The device adds
+    each token's squares in another order, so an x~ on a rounding tie may go
+    either way (the bar of the other normalised forms): y within the parity
+    tolerance and bit-identical almost everywhere, and the same against the
+    single-problem normalising call (whose quantiser may combine a long row's
+    partial sums in another order)."""
+    probs = workloads.layer_set_2b(B, layers=1).problems
+    cases = [Case(p.M, p.K, p.N, w_seed=p.w_seed, x_seed=p.x_seed) for p in probs]
+    gains = [workloads.norm_gains(p.K, p.w_seed + 7) for p in probs]
+    ys = run_group_norm(cases, gains)
+    import torch
+    for c, g, y in zip(cases, gains, ys):
+        ref = c.orc.forward(c.x_bits, c.W, gamma=c.gamma, norm_gain=g)
+        assert check_y(y, ref["y"]) >= 0.99
+        single = torch.empty((c.M, c.N), dtype=torch.bfloat16, device="cuda")
+        bl.bitlinear_forward_rmsnorm(c.x_tensor(), c.packed_tensor(), c.gamma, c.N,
+                                     torch.from_numpy(g).cuda(), y=single)
+        torch.cuda.synchronize()
+        assert check_y(y, tensor_to_bf16_bits(single)) >= 0.99
