@@ -263,14 +263,14 @@ int launch_quant_act(const void *x, bitlinear_dtype xdt, int M, int K, int8_t *x
 
 // ------------------------------------------------------------------- GEMV
 
-template <int MT, bool BF16, bool NORM, bool FFN>
+template <int MT, bool BF16, bool NORM, bool FFN, bool WIDE = false>
 int launch_gemv_t(const gemv::Params &p, int grid, int smem, int dev, cudaStream_t st)
 {
-    cudaError_t e = allow_smem<gemv::gemv_kernel<MT, BF16, NORM, FFN>>(dev, smem);
+    cudaError_t e = allow_smem<gemv::gemv_kernel<MT, BF16, NORM, FFN, WIDE>>(dev, smem);
     if (e != cudaSuccess)
         return launch_status(e);
-    e = launch(gemv::gemv_kernel<MT, BF16, NORM, FFN>, dim3(grid), dim3(gemv::THREADS), smem, st,
-               p);
+    e = launch(gemv::gemv_kernel<MT, BF16, NORM, FFN, WIDE>, dim3(grid), dim3(gemv::THREADS), smem,
+               st, p);
     return launch_status(e);
 }
 
@@ -290,6 +290,13 @@ int launch_gemv_mt(const gemv::Params &p, bool bf16, bool norm, bool ffn, int gr
                     : launch_gemv_t<MT, false, true, false>(p, grid, smem, dev, st);
     return bf16 ? launch_gemv_t<MT, true, false, false>(p, grid, smem, dev, st)
                 : launch_gemv_t<MT, false, false, false>(p, grid, smem, dev, st);
+}
+
+// The single-token bf16 kernel that stages a long row (8192 < K <= 32768) in
+// shared memory for its prologue.
+int launch_gemv_wide(const gemv::Params &p, int grid, int smem, int dev, cudaStream_t st)
+{
+    return launch_gemv_t<1, true, false, false, true>(p, grid, smem, dev, st);
 }
 
 // One problem of a GEMV launch, as the host sees it.
@@ -346,6 +353,16 @@ int launch_gemv(const GemvJob *jobs, int count, bitlinear_dtype xdt, const Devic
     const int MT = gemv_tile(Mmax);
     const int QB = gemv::chunk_blocks(MT, ffn);
     const int nmat = ffn ? 2 : 1;
+    int max_K = 0;
+    for (int i = 0; i < count; ++i)
+        max_K = std::max(max_K, jobs[i].K);
+    // one bf16 token of a long row: the wide kernel, whose x~ region first
+    // holds the staged bf16 row (2 K bytes), two blocks per SM
+    const bool wide = MT == 1 && !norm && !ffn && xdt == BITLINEAR_BF16 && max_K > 8192 &&
+                      max_K <= 32768;
+    if (wide)
+        xq_cap *= 2;
+    const int ring_budget = wide ? 110 * 1024 : 72 * 1024;
     int blocks[gemv::MAX_PROBLEMS], ctas[gemv::MAX_PROBLEMS], G[gemv::MAX_PROBLEMS];
     double bbytes[gemv::MAX_PROBLEMS];
     double max_block = 0.0;
@@ -380,7 +397,14 @@ int launch_gemv(const GemvJob *jobs, int count, bitlinear_dtype xdt, const Devic
     int grid = 0;
     for (int i = 0; i < count; ++i)
         grid += ctas[i];
-    int gcap = 1 << 30;               // upper bound on k-groups per stage
+    // Stage geometry. When the whole rows of two or more blocks (or of a
+    // CTA's only block) fit in a slot target (32 KiB), a chunk of cb blocks
+    // streams as one contiguous copy per matrix (G = all K/128 groups);
+    // otherwise a stage is a k-range of G groups (a multiple of 8, so that
+    // each warp keeps its groups) of every block of the chunk, about 16 KiB,
+    // one copy per block. Beside a large x~ the targets shrink.
+    int cb[gemv::MAX_PROBLEMS];
+    int target_rows = 32 * 1024, target_split = 16 * 1024;
     int slot_bytes = 0, slots = 0, red_blocks = 1, smem = 0;
     for (int attempt = 0;; ++attempt) {
         slot_bytes = 0;
@@ -389,29 +413,35 @@ int launch_gemv(const GemvJob *jobs, int count, bitlinear_dtype xdt, const Devic
         for (int i = 0; i < count; ++i) {
             const int KG = jobs[i].K / 128;
             const int q = (blocks[i] + ctas[i] - 1) / ctas[i];
-            const int qb = std::min(q, QB);
-            // about 16 KiB per stage: G a multiple of 8 (each warp owns the
-            // groups of one residue mod 8), or the whole row when that is less
-            int g = std::max(8, (16384 / (nmat * qb * gemv::PIECE)) & ~7);
-            g = std::min(g, std::max(8, gcap));
-            G[i] = g >= KG ? KG : g;
-            slot_bytes = std::max(slot_bytes, nmat * qb * G[i] * gemv::PIECE);
-            red_blocks = std::max(red_blocks, qb);
-            stages = std::max(stages, ((q + QB - 1) / QB) * ((KG + G[i] - 1) / G[i]));
+            const int row_block = nmat * KG * gemv::PIECE;     // one block, all matrices
+            if (2 * row_block <= target_rows || (q == 1 && row_block <= target_rows)) {
+                cb[i] = std::max(1, std::min({QB, q, target_rows / row_block}));
+                G[i] = KG;
+            } else {
+                cb[i] = std::min(q, QB);
+                int g = std::max(8, (target_split / (nmat * cb[i] * gemv::PIECE)) & ~7);
+                G[i] = g >= KG ? KG : g;
+            }
+            slot_bytes = std::max(slot_bytes, nmat * cb[i] * G[i] * gemv::PIECE);
+            red_blocks = std::max(red_blocks, cb[i]);
+            stages = std::max(stages, ((q + cb[i] - 1) / cb[i]) * ((KG + G[i] - 1) / G[i]));
         }
         // Ring depth: the whole share when it is small, else as deep as a
-        // 72 KiB block allows (three blocks per SM fit beside each other).
+        // 72 KiB block allows (three blocks per SM fit beside each other;
+        // 110 KiB for the wide kernel's two).
         const int fixed = gemv::smem_bytes(MT, xq_cap, 0, 0, red_blocks, norm, ffn);
-        slots = (72 * 1024 - fixed) / slot_bytes;
-        slots = std::max(2, std::min({slots, stages, gemv::MAX_SLOTS}));
+        slots = (ring_budget - fixed) / slot_bytes;
+        slots = std::max(1, std::min({slots, stages, gemv::MAX_SLOTS}));
+        if (stages > 1)
+            slots = std::max(slots, 2);
         smem = gemv::smem_bytes(MT, xq_cap, slots, slot_bytes, red_blocks, norm, ffn);
         if (smem <= dev.max_smem_optin)
             break;
         // too large beside a large x~: smaller stages
-        if (gcap > 8 && attempt < 8)
-            gcap = (gcap > 64 ? 64 : gcap) / 2;
-        else
+        if (attempt >= 8 || (target_rows <= 4096 && target_split <= 4096))
             return BITLINEAR_ERR_SHAPE;
+        target_rows = std::max(4096, target_rows / 2);
+        target_split = std::max(4096, target_split / 2);
     }
     gemv::Params p = {};
     int begin = 0;
@@ -432,6 +462,7 @@ int launch_gemv(const GemvJob *jobs, int count, bitlinear_dtype xdt, const Devic
                                   blocks[i] / ctas[i],
                                   blocks[i] % ctas[i],
                                   begin,
+                                  cb[i],
                                   G[i],
                                   static_cast<const uint8_t *>(j.packed2),
                                   j.gamma2,
@@ -449,6 +480,8 @@ int launch_gemv(const GemvJob *jobs, int count, bitlinear_dtype xdt, const Devic
                                             : kWaitLimitNs;
     p.inject_timeout = inject_timeout_us > 0 ? 1 : 0;
     const bool bf16 = xdt == BITLINEAR_BF16;
+    if (wide)
+        return launch_gemv_wide(p, grid, smem, dev.id, st);
     switch (MT) {
     case 1: return launch_gemv_mt<1>(p, bf16, norm, ffn, grid, smem, dev.id, st);
     case 2: return launch_gemv_mt<2>(p, bf16, norm, ffn, grid, smem, dev.id, st);

@@ -191,6 +191,18 @@ __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void *src, uint32_t
         : "memory");
 }
 
+// 16-byte asynchronous copy global -> shared (L2 only); dst and src 16-byte
+// aligned. Complete for the issuing thread after cp_async_wait_all.
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src)
+{
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+
+__device__ __forceinline__ void cp_async_wait_all()
+{
+    asm volatile("cp.async.wait_all;" ::: "memory");
+}
+
 // 2-D tiled tensor copy global -> this CTA's shared memory.
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, int x,
                                             int y, uint32_t bar)

@@ -74,7 +74,9 @@ constexpr int PIECE = 512;                         // one (row block, k-group)
 constexpr int MAX_SLOTS = 8;
 constexpr int BAR_BYTES = 2 * MAX_SLOTS * 8 + 16;  // full/empty barriers + abort flag
 constexpr int MAX_PROBLEMS = 8;
-constexpr int XCACHE = 4;                          // 16-byte slots of token 0 kept through the prologue
+// 16-byte slots of token 0 kept in registers through the prologue (a warp's
+// share of K <= 8192)
+constexpr int XCACHE = 4;
 
 // Row blocks per chunk and tokens whose x~ a lane holds in registers at once,
 // by token tile MT. Only MT = 1 keeps the four plane sums apart for a whole
@@ -112,7 +114,9 @@ struct Problem {
     int base, extra;        // row blocks of 16 rows per CTA: base, one more for the
                             // problem's first `extra` CTAs
     int cta_begin;          // this problem's first CTA in the grid
-    int G;                  // k-groups per stage (a multiple of 8, or all K/128)
+    int cb;                 // row blocks per chunk (<= QB)
+    int G;                  // k-groups per stage (a multiple of 8, or all K/128: then a
+                            // stage is whole rows, one contiguous copy per matrix)
     // FFN launches only: `packed`, `gamma`, `norm_gain` and `y` (optional)
     // are the gate projection's; these are the up projection's and h
     const uint8_t *packed2;
@@ -187,8 +191,10 @@ __device__ __forceinline__ void load4(const void *row, int e, float (&v)[4])
     }
 }
 
-template <int MT, bool BF16, bool NORM, bool FFN>
-__global__ void __launch_bounds__(THREADS, (NORM ? 2 : Shape<MT, FFN>::MIN_BLOCKS))
+// WIDE (one bf16 token of 8192 < K <= 32768, no normalisation, not FFN)
+// stages the token row in shared memory for the prologue (two blocks per SM).
+template <int MT, bool BF16, bool NORM, bool FFN, bool WIDE>
+__global__ void __launch_bounds__(THREADS, ((NORM || WIDE) ? 2 : Shape<MT, FFN>::MIN_BLOCKS))
 gemv_kernel(const __grid_constant__ Params p)
 {
     using S = Shape<MT, FFN>;
@@ -212,7 +218,8 @@ gemv_kernel(const __grid_constant__ Params p)
     const int cta = static_cast<int>(blockIdx.x) - P.cta_begin;
     const int blk0 = cta * P.base + min(cta, P.extra);
     const int nblk = min(P.base + (cta < P.extra ? 1 : 0), total_blocks - blk0);
-    const int nchunks = (nblk + QB - 1) / QB;
+    const int cb = P.cb;
+    const int nchunks = (nblk + cb - 1) / cb;
     const int kstages = (KG + G - 1) / G;
     const int nstages = nchunks * kstages;
     const int slots = p.slots;
@@ -257,9 +264,11 @@ gemv_kernel(const __grid_constant__ Params p)
     if (warp == CWARPS) {
         // ---------------------------------------------------- weight producer
         // Reads only the packed weights, so it does not wait for the previous
-        // grid in the stream. Lane l copies block l of the chunk (FFN: lanes
-        // qb .. 2 qb - 1 copy the up projection's blocks); lane 0 arms the
-        // stage's barrier with the whole stage's bytes first.
+        // grid in the stream. A stage of whole rows is one copy per matrix
+        // (lane 1: the up projection's rows of an FFN launch); a stage of a
+        // k-range takes lane l for block l of the chunk (FFN: lanes qb ..
+        // 2 qb - 1 for the up projection). Lane 0 arms the stage's barrier with
+        // the whole stage's bytes first.
         int slot = 0;
         uint32_t phase = 0;        // parity of this pass over the ring
         uint32_t in_flight = 0;    // slots holding a copy this warp issued
@@ -271,8 +280,8 @@ gemv_kernel(const __grid_constant__ Params p)
                 break;
             const int c = st / kstages;
             const int ks = st - c * kstages;
-            const int b0 = c * QB;
-            const int qb = min(QB, nblk - b0);
+            const int b0 = c * cb;
+            const int qb = min(cb, nblk - b0);
             const int g0 = ks * G;
             const int gs = min(G, KG - g0);
             const uint32_t bytes = static_cast<uint32_t>(gs * PIECE);
@@ -282,7 +291,18 @@ gemv_kernel(const __grid_constant__ Params p)
                 if (lane == 0)
                     mbar_arrive_expect_tx(full(slot), bytes * static_cast<uint32_t>(NMAT * qb));
                 __syncwarp();
-                if (lane < NMAT * qb) {
+                if (gs == KG) {
+                    // whole rows: the chunk's blocks are one contiguous range
+                    // per matrix
+                    if (lane < NMAT) {
+                        const uint8_t *src = (FFN && lane == 1) ? P.packed2 : P.packed;
+                        bulk_g2s(ring_u32 + static_cast<uint32_t>(slot * slot_bytes) +
+                                     lane * qb * bytes,
+                                 src + static_cast<size_t>(blk0 + b0) * KG * PIECE,
+                                 bytes * static_cast<uint32_t>(qb), full(slot));
+                    }
+                } else if (lane < NMAT * qb) {
+                    // a k-range of every block: one copy per block
                     const int mat = lane >= qb ? 1 : 0;
                     const int bl = lane - mat * qb;
                     const uint8_t *src = (FFN && mat) ? P.packed2 : P.packed;
@@ -325,163 +345,246 @@ gemv_kernel(const __grid_constant__ Params p)
     const int nsl = (ngw + 1) / 2;                    // slots of this warp
     // gains of quantised copy x (FFN: 0 = gate, 1 = up)
     auto gain_of = [&](int x) { return (FFN && x == 1) ? P.norm_gain2 : P.norm_gain; };
-    Vec8<BF16> xc[XCACHE];
-    // slots whose loads are issued together, and gain loads of cached slots
-    constexpr int XB = NORM ? 2 : (BF16 ? 4 : 2);
-    constexpr int XG = NORM ? 2 : XCACHE;
-    using Gains = float[NX][8];
-    // Visits this thread's valid slots of token m: f(i, v, g) with v the eight
-    // raw activations and, when `gains` is set (NORM launches), g the eight
-    // gains of each quantised copy.
-    auto for_slots = [&](int m, bool fill, bool gains, auto &&f) {
-        const void *row = static_cast<const char *>(P.x) + m * row_bytes;
+    if constexpr (WIDE) {
+        // One bf16 token of up to 32768 activations. Its row is staged in
+        // shared memory (the 2 K bytes of the x~ region, which x~ overwrites
+        // at the end) with 16-byte asynchronous copies of every slot of this
+        // thread, all in flight at once; both passes then read shared memory,
+        // and the quantised words wait in registers until every thread has
+        // read its slots.
+        static_assert(BF16 && !NORM && !FFN && MT == 1, "wide kernel");
+        constexpr int WSL = 16;                       // slots per thread at K = 32768
+        const char *row = static_cast<const char *>(P.x);
         auto valid = [&](int i) { return i < nsl && slot_group(i) < KG; };
-        auto load_gains = [&](int i, Gains &g) {
-            if constexpr (NORM) {
-                if (gains) {
 #pragma unroll
-                    for (int x = 0; x < NX; ++x)
-                        load8<false>(gain_of(x), slot_elem(i), g[x]);
+        for (int i = 0; i < WSL; ++i)
+            if (valid(i))
+                cp_async16(smem_u32(xq_sm + 2 * slot_elem(i)), row + 2 * slot_elem(i));
+        cp_async_wait_all();
+        auto staged = [&](int i) {
+            Vec8<true> v;
+            const uint4 raw = *reinterpret_cast<const uint4 *>(xq_sm + 2 * slot_elem(i));
+            v.w[0] = raw.x; v.w[1] = raw.y; v.w[2] = raw.z; v.w[3] = raw.w;
+            return v;
+        };
+        float amax = 0.0f;
+#pragma unroll
+        for (int i = 0; i < WSL; ++i) {
+            if (valid(i)) {
+                const Vec8<true> v = staged(i);
+#pragma unroll
+                for (int u = 0; u < 8; ++u)
+                    amax = fmaxf(amax, fabsf(v.get(u)));
+            }
+        }
+        const uint32_t um = __reduce_max_sync(0xffffffffu, __float_as_uint(amax));
+        if (lane == 0)
+            red_u(0)[warp] = um;
+        compute_sync();
+        uint32_t ub = red_u(0)[0];
+#pragma unroll
+        for (int w = 1; w < CWARPS; ++w)
+            ub = max(ub, red_u(0)[w]);
+        const float beta = fmaxf(__uint_as_float(ub), 1e-5f);
+        const float scale = __fdiv_rn(127.0f, beta);
+        uint32_t qw[WSL][2];
+        int sum = 0;
+#pragma unroll
+        for (int i = 0; i < WSL; ++i) {
+            if (valid(i)) {
+                const Vec8<true> v = staged(i);
+                // |x * (127 / beta)| <= 127: the listing's clamp cannot bind
+                int q[8];
+#pragma unroll
+                for (int u = 0; u < 8; ++u)
+                    q[u] = __float2int_rn(__fmul_rn(v.get(u), scale));
+                qw[i][0] = __byte_perm(__byte_perm(q[0], q[1], 0x0040),
+                                       __byte_perm(q[2], q[3], 0x0040), 0x5410);
+                qw[i][1] = __byte_perm(__byte_perm(q[4], q[5], 0x0040),
+                                       __byte_perm(q[6], q[7], 0x0040), 0x5410);
+                sum = dp4a_ss(qw[i][1], 0x01010101u, dp4a_ss(qw[i][0], 0x01010101u, sum));
+            }
+        }
+        // every thread has read its staged slots before x~ overwrites them
+        compute_sync();
+#pragma unroll
+        for (int i = 0; i < WSL; ++i) {
+            if (valid(i)) {
+                const int e = slot_elem(i);
+                *reinterpret_cast<uint2 *>(xq_sm + e) = make_uint2(qw[i][0], qw[i][1]);
+                if (P.xq_dbg != nullptr && first_cta)
+                    *reinterpret_cast<uint2 *>(P.xq_dbg + e) = make_uint2(qw[i][0], qw[i][1]);
+            }
+        }
+        sum = __reduce_add_sync(0xffffffffu, sum);
+        if (lane == 0)
+            red_s(0)[warp] = sum;
+        if (ctid == 0) {
+            beta_sm(0)[0] = beta;
+            if (P.beta_dbg != nullptr && first_cta)
+                P.beta_dbg[0] = beta;
+        }
+    } else {
+        Vec8<BF16> xc[XCACHE];
+        // slots whose loads are issued together, and gain loads of cached slots
+        constexpr int XB = NORM ? 2 : (BF16 ? 4 : 2);
+        constexpr int XG = NORM ? 2 : XCACHE;
+        using Gains = float[NX][8];
+        // Visits this thread's valid slots of token m: f(i, v, g) with v the eight
+        // raw activations and, when `gains` is set (NORM launches), g the eight
+        // gains of each quantised copy.
+        auto for_slots = [&](int m, bool fill, bool gains, auto &&f) {
+            const void *row = static_cast<const char *>(P.x) + m * row_bytes;
+            auto valid = [&](int i) { return i < nsl && slot_group(i) < KG; };
+            auto load_gains = [&](int i, Gains &g) {
+                if constexpr (NORM) {
+                    if (gains) {
+    #pragma unroll
+                        for (int x = 0; x < NX; ++x)
+                            load8<false>(gain_of(x), slot_elem(i), g[x]);
+                    }
                 }
+            };
+            int i0 = 0;
+            if (m == 0) {
+                if (fill) {
+    #pragma unroll
+                    for (int i = 0; i < XCACHE; ++i)
+                        if (valid(i))
+                            xc[i].load(row, slot_elem(i));
+                }
+    #pragma unroll
+                for (int ic = 0; ic < XCACHE; ic += XG) {
+                    float g[XG][NX][8];
+    #pragma unroll
+                    for (int u = 0; u < XG; ++u)
+                        if (valid(ic + u))
+                            load_gains(ic + u, g[u]);
+    #pragma unroll
+                    for (int u = 0; u < XG; ++u)
+                        if (valid(ic + u))
+                            f(ic + u, xc[ic + u], g[u]);
+                }
+                i0 = XCACHE;
+            }
+            for (int ib = i0; ib < nsl; ib += XB) {
+                Vec8<BF16> v[XB];
+                float g[XB][NX][8];
+    #pragma unroll
+                for (int u = 0; u < XB; ++u) {
+                    if (valid(ib + u)) {
+                        v[u].load(row, slot_elem(ib + u));
+                        load_gains(ib + u, g[u]);
+                    }
+                }
+    #pragma unroll
+                for (int u = 0; u < XB; ++u)
+                    if (valid(ib + u))
+                        f(ib + u, v[u], g[u]);
             }
         };
-        int i0 = 0;
-        if (m == 0) {
-            if (fill) {
-#pragma unroll
-                for (int i = 0; i < XCACHE; ++i)
-                    if (valid(i))
-                        xc[i].load(row, slot_elem(i));
-            }
-#pragma unroll
-            for (int ic = 0; ic < XCACHE; ic += XG) {
-                float g[XG][NX][8];
-#pragma unroll
-                for (int u = 0; u < XG; ++u)
-                    if (valid(ic + u))
-                        load_gains(ic + u, g[u]);
-#pragma unroll
-                for (int u = 0; u < XG; ++u)
-                    if (valid(ic + u))
-                        f(ic + u, xc[ic + u], g[u]);
-            }
-            i0 = XCACHE;
-        }
-        for (int ib = i0; ib < nsl; ib += XB) {
-            Vec8<BF16> v[XB];
-            float g[XB][NX][8];
-#pragma unroll
-            for (int u = 0; u < XB; ++u) {
-                if (valid(ib + u)) {
-                    v[u].load(row, slot_elem(ib + u));
-                    load_gains(ib + u, g[u]);
-                }
-            }
-#pragma unroll
-            for (int u = 0; u < XB; ++u)
-                if (valid(ib + u))
-                    f(ib + u, v[u], g[u]);
-        }
-    };
 
-    if constexpr (NORM) {
-        // sums of squares per token
+        if constexpr (NORM) {
+            // sums of squares per token
+            for (int m = 0; m < M; ++m) {
+                double ss = 0.0;
+                for_slots(m, true, false, [&](int, const Vec8<BF16> &v, const Gains &) {
+    #pragma unroll
+                    for (int u = 0; u < 8; ++u) {
+                        const double d = v.get(u);
+                        ss = __fma_rn(d, d, ss);
+                    }
+                });
+                ss = warp_sum_f64(ss);
+                if (lane == 0)
+                    red_d[m * CWARPS + warp] = ss;
+            }
+            compute_sync();
+        }
+        // absmax per token over this thread's elements (per quantised copy)
         for (int m = 0; m < M; ++m) {
-            double ss = 0.0;
-            for_slots(m, true, false, [&](int, const Vec8<BF16> &v, const Gains &) {
-#pragma unroll
-                for (int u = 0; u < 8; ++u) {
-                    const double d = v.get(u);
-                    ss = __fma_rn(d, d, ss);
+            float r = 1.0f;
+            if constexpr (NORM)
+                r = row_rms_scale(red_d, m, K, P.norm_eps);
+            float amax[NX];
+    #pragma unroll
+            for (int x = 0; x < NX; ++x)
+                amax[x] = 0.0f;
+            for_slots(m, !NORM, true, [&](int, const Vec8<BF16> &v, const Gains &g) {
+    #pragma unroll
+                for (int x = 0; x < NX; ++x) {
+    #pragma unroll
+                    for (int u = 0; u < 8; ++u) {
+                        float a = v.get(u);
+                        if constexpr (NORM)
+                            a = norm1(a, r, g[x][u]);
+                        amax[x] = fmaxf(amax[x], fabsf(a));
+                    }
                 }
             });
-            ss = warp_sum_f64(ss);
-            if (lane == 0)
-                red_d[m * CWARPS + warp] = ss;
+    #pragma unroll
+            for (int x = 0; x < NX; ++x) {
+                const uint32_t u = __reduce_max_sync(0xffffffffu, __float_as_uint(amax[x]));
+                if (lane == 0)
+                    red_u(x)[m * CWARPS + warp] = u;
+            }
         }
         compute_sync();
-    }
-    // absmax per token over this thread's elements (per quantised copy)
-    for (int m = 0; m < M; ++m) {
-        float r = 1.0f;
-        if constexpr (NORM)
-            r = row_rms_scale(red_d, m, K, P.norm_eps);
-        float amax[NX];
-#pragma unroll
-        for (int x = 0; x < NX; ++x)
-            amax[x] = 0.0f;
-        for_slots(m, !NORM, true, [&](int, const Vec8<BF16> &v, const Gains &g) {
-#pragma unroll
+        // quantise this warp's own groups into shared memory (only this warp
+        // reads them), with their sums of x~
+        for (int m = 0; m < M; ++m) {
+            float r = 1.0f;
+            if constexpr (NORM)
+                r = row_rms_scale(red_d, m, K, P.norm_eps);
+            float scale[NX];
+            int sum[NX];
+    #pragma unroll
             for (int x = 0; x < NX; ++x) {
-#pragma unroll
-                for (int u = 0; u < 8; ++u) {
-                    float a = v.get(u);
-                    if constexpr (NORM)
-                        a = norm1(a, r, g[x][u]);
-                    amax[x] = fmaxf(amax[x], fabsf(a));
+                uint32_t ub = red_u(x)[m * CWARPS];
+    #pragma unroll
+                for (int w = 1; w < CWARPS; ++w)
+                    ub = max(ub, red_u(x)[m * CWARPS + w]);
+                const float beta = fmaxf(__uint_as_float(ub), 1e-5f);
+                scale[x] = __fdiv_rn(127.0f, beta);
+                sum[x] = 0;
+                if (ctid == 0) {
+                    beta_sm(x)[m] = beta;
+                    if (x == 0 && P.beta_dbg != nullptr && first_cta)
+                        P.beta_dbg[m] = beta;
                 }
             }
-        });
-#pragma unroll
-        for (int x = 0; x < NX; ++x) {
-            const uint32_t u = __reduce_max_sync(0xffffffffu, __float_as_uint(amax[x]));
-            if (lane == 0)
-                red_u(x)[m * CWARPS + warp] = u;
-        }
-    }
-    compute_sync();
-    // quantise this warp's own groups into shared memory (only this warp
-    // reads them), with their sums of x~
-    for (int m = 0; m < M; ++m) {
-        float r = 1.0f;
-        if constexpr (NORM)
-            r = row_rms_scale(red_d, m, K, P.norm_eps);
-        float scale[NX];
-        int sum[NX];
-#pragma unroll
-        for (int x = 0; x < NX; ++x) {
-            uint32_t ub = red_u(x)[m * CWARPS];
-#pragma unroll
-            for (int w = 1; w < CWARPS; ++w)
-                ub = max(ub, red_u(x)[m * CWARPS + w]);
-            const float beta = fmaxf(__uint_as_float(ub), 1e-5f);
-            scale[x] = __fdiv_rn(127.0f, beta);
-            sum[x] = 0;
-            if (ctid == 0) {
-                beta_sm(x)[m] = beta;
-                if (x == 0 && P.beta_dbg != nullptr && first_cta)
-                    P.beta_dbg[m] = beta;
-            }
-        }
-        for_slots(m, false, true, [&](int i, const Vec8<BF16> &v, const Gains &g) {
-            const int e = slot_elem(i);
-#pragma unroll
-            for (int x = 0; x < NX; ++x) {
-                uint32_t lo = 0, hi = 0;
-#pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    float a = v.get(u), b = v.get(u + 4);
-                    if constexpr (NORM) {
-                        a = norm1(a, r, g[x][u]);
-                        b = norm1(b, r, g[x][u + 4]);
+            for_slots(m, false, true, [&](int i, const Vec8<BF16> &v, const Gains &g) {
+                const int e = slot_elem(i);
+    #pragma unroll
+                for (int x = 0; x < NX; ++x) {
+                    // |a * (127 / beta)| <= 127 (beta is the row's absmax, or
+                    // 1e-5 above every |a|), so rint never leaves [-127, 127]
+                    // and the listing's clamp to [-128, 127] cannot bind
+                    int q[8];
+    #pragma unroll
+                    for (int u = 0; u < 8; ++u) {
+                        float a = v.get(u);
+                        if constexpr (NORM)
+                            a = norm1(a, r, g[x][u]);
+                        q[u] = __float2int_rn(__fmul_rn(a, scale[x]));
                     }
-                    const int qa = quant1(a, scale[x]);
-                    const int qb = quant1(b, scale[x]);
-                    sum[x] += qa + qb;
-                    lo |= (static_cast<uint32_t>(qa) & 0xffu) << (8 * u);
-                    hi |= (static_cast<uint32_t>(qb) & 0xffu) << (8 * u);
+                    const uint32_t lo = __byte_perm(__byte_perm(q[0], q[1], 0x0040),
+                                                    __byte_perm(q[2], q[3], 0x0040), 0x5410);
+                    const uint32_t hi = __byte_perm(__byte_perm(q[4], q[5], 0x0040),
+                                                    __byte_perm(q[6], q[7], 0x0040), 0x5410);
+                    sum[x] = dp4a_ss(hi, 0x01010101u, dp4a_ss(lo, 0x01010101u, sum[x]));
+                    *reinterpret_cast<uint2 *>(xq_sm + x * p.xq_cap + m * K + e) = make_uint2(lo, hi);
+                    if (x == 0 && P.xq_dbg != nullptr && first_cta)
+                        *reinterpret_cast<uint2 *>(P.xq_dbg + static_cast<size_t>(m) * K + e) =
+                            make_uint2(lo, hi);
                 }
-                *reinterpret_cast<uint2 *>(xq_sm + x * p.xq_cap + m * K + e) = make_uint2(lo, hi);
-                if (x == 0 && P.xq_dbg != nullptr && first_cta)
-                    *reinterpret_cast<uint2 *>(P.xq_dbg + static_cast<size_t>(m) * K + e) =
-                        make_uint2(lo, hi);
+            });
+    #pragma unroll
+            for (int x = 0; x < NX; ++x) {
+                const int sm = __reduce_add_sync(0xffffffffu, sum[x]);
+                if (lane == 0)
+                    red_s(x)[m * CWARPS + warp] = sm;
             }
-        });
-#pragma unroll
-        for (int x = 0; x < NX; ++x) {
-            const int sm = __reduce_add_sync(0xffffffffu, sum[x]);
-            if (lane == 0)
-                red_s(x)[m * CWARPS + warp] = sm;
         }
     }
     // this warp's lanes read the groups its lanes just wrote
@@ -497,8 +600,8 @@ gemv_kernel(const __grid_constant__ Params p)
     uint32_t phase = 0;
     bool ok = true;
     for (int c = 0; c < nchunks; ++c) {
-        const int b0 = c * QB;
-        const int qb = min(QB, nblk - b0);
+        const int b0 = c * cb;
+        const int qb = min(cb, nblk - b0);
         // acc[mat][bi][.]: row sums of this lane's weights (PERSIST: the four
         // plane sums of token 0 kept apart, combined at the end of the chunk)
         int acc[NMAT][QB][NACC];

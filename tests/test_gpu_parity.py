@@ -96,11 +96,23 @@ def test_maximum_k_and_single_output_row(cuda, path, M):
 
 
 def test_gemv_tall_matrix_next_to_large_x(cuda):
-    # x~ of 16 x 12160 bytes leaves shared memory for the row accumulators of
-    # only three row blocks per CTA, so the 1499 row blocks (the last one
-    # ragged) take 500 CTAs: more than one wave, the last CTA short
+    # x~ of 16 x 12160 bytes leaves little shared memory beside it, so the
+    # weights stream in small stages; 1499 row blocks (the last one ragged)
+    # spread over the CTAs, some holding one block more than others
     c = Case(16, 12160, 23970, w_seed=61, x_seed=62)
     assert c.check_sampled(c.run(path=bl.PATH_GEMV), count=20000) == 1.0
+
+
+@pytest.mark.parametrize("K,N,dtype", [(8320, 700, "bf16"), (16384, 333, "bf16"),
+                                       (28672, 1000, "bf16"), (32768, 130, "bf16"),
+                                       (16384, 300, "fp32"), (33024, 77, "bf16")])
+def test_gemv_long_rows_single_token(cuda, K, N, dtype):
+    # one bf16 token of 8192 < K <= 32768 takes the kernel that stages the
+    # row in shared memory for its prologue (x~ then overwrites the staged
+    # row); fp32 tokens and K = 33024 take the register-cached prologue with
+    # reloads
+    c = Case(1, K, N, w_seed=K + N, x_seed=K - N, x_dtype=dtype)
+    assert c.check_full(c.run(path=bl.PATH_GEMV)) == 1.0
 
 
 def test_tc_many_tiles_per_cta(cuda):
