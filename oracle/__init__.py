@@ -20,6 +20,7 @@ Functions:
     f32_to_bf16(f)              RNE rounding to bf16 bit patterns (uint16)
     rescale_bf16(acc, beta, gamma)     y bf16 bits [M][N]
     pack_codes(Wq)              the 2-bit packed layout (flat uint8)
+    pack_codes_b3(Wq)           the base-3 layout, 5 codes per byte (flat uint8)
     relu2_glu(gate, up)         h = max(gate, 0)^2 * up (fp32, elementwise)
     forward(x, W)               the whole path, returning every stage
     ffn(x, W_gate, W_up, W_down)   gate/up -> gated ReLU^2 -> down, every stage
@@ -82,6 +83,8 @@ def _declare(lib):
     lib.oracle_relu2_glu.argtypes = [p, p, c_i64, p]
     lib.oracle_pack_codes.restype = ctypes.c_int
     lib.oracle_pack_codes.argtypes = [p, c_i64, c_i64, p]
+    lib.oracle_pack_codes_b3.restype = ctypes.c_int
+    lib.oracle_pack_codes_b3.argtypes = [p, c_i64, c_i64, p]
     return lib
 
 
@@ -223,6 +226,18 @@ class Oracle:
         rc = self.lib.oracle_pack_codes(_ptr(Wq), N, K, _ptr(out))
         if rc != 0:
             raise ValueError("oracle_pack_codes: K % 128 != 0 or non-ternary")
+        return out
+
+    def pack_codes_b3(self, Wq) -> np.ndarray:
+        """The base-3 layout (5 codes per byte, K padded to a multiple of
+        160) of int8 ternary weights [N][K]."""
+        Wq = _c(Wq, np.int8)
+        N, K = Wq.shape
+        Kp = (K + 159) // 160 * 160
+        out = np.empty(((N + 15) // 16 * 16 * Kp // 5,), dtype=np.uint8)
+        rc = self.lib.oracle_pack_codes_b3(_ptr(Wq), N, K, _ptr(out))
+        if rc != 0:
+            raise ValueError("oracle_pack_codes_b3: K % 128 != 0 or non-ternary")
         return out
 
     def relu2_glu(self, gate, up) -> np.ndarray:

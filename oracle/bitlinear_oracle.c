@@ -305,3 +305,56 @@ int oracle_pack_codes(const int8_t *Wq, int64_t N, int64_t K, uint8_t *packed)
     }
     return 0;
 }
+
+/* ------------------------------------------------- base-3 layout (5 per byte) */
+
+/* Denser storage of the same codes, 5 per byte (3^5 = 243 <= 256, 1.6 bits
+ * per weight): the log2(3) = 1.58-bit density behind the 0.4 GB footprint
+ * of the 2B model ("Microsoft Releases BitNet b1.58 2B4T", opening section;
+ * "BitNet b1.58 2B4T Guide", section "Mathematical Architecture"). The layout
+ * is this library's own:
+ *   - K is padded with zero weights to Kp, a multiple of 160; rows come in
+ *     blocks of 16 (the last block completed with zero rows); block b
+ *     occupies the 16 * Kp / 5 bytes starting at byte b * 16 * Kp / 5;
+ *   - inside a block the weights come in k-groups of 160: group g holds the
+ *     weights k in [160 g, 160 g + 160) of all 16 rows in the 512 bytes at
+ *     offset 512 g, row r of the block in the 32 bytes at offset 32 r;
+ *   - those 32 bytes hold the 160 codes c = W~ + 1 of the row in "stream
+ *     order": stream position p = 16 w + 4 b + j is the weight
+ *     k = 160 g + 16 w + 4 j + b (w in 0..9, j, b in 0..3) -- the order of the
+ *     2-bit fields of the 2-bit layout's words, read from bit 0 up;
+ *   - byte B (0..31) holds the codes of stream positions 5 B .. 5 B + 4 as
+ *     the number sum_i c(5 B + i) * 3^i (0..242).
+ * The output holds ceil(N / 16) * 16 * Kp / 5 bytes. Returns 0, or -1 when K
+ * is not a positive multiple of 128 or a weight is not ternary. */
+int oracle_pack_codes_b3(const int8_t *Wq, int64_t N, int64_t K, uint8_t *packed)
+{
+    if (K <= 0 || K % 128 != 0)
+        return -1;
+    const int64_t Kp = (K + 159) / 160 * 160;
+    const int64_t blocks = (N + 15) / 16;
+    const int64_t row_bytes = Kp / 5;
+    for (int64_t blk = 0; blk < blocks; ++blk) {
+        for (int64_t r = 0; r < 16; ++r) {
+            const int64_t n = 16 * blk + r;
+            for (int64_t g = 0; g < Kp / 160; ++g) {
+                for (int64_t B = 0; B < 32; ++B) {
+                    int value = 0;
+                    int power = 1;
+                    for (int i = 0; i < 5; ++i) {
+                        const int64_t p = 5 * B + i;          /* stream position */
+                        const int64_t w = p / 16, b = (p % 16) / 4, j = p % 4;
+                        const int64_t k = 160 * g + 16 * w + 4 * j + b;
+                        const int v = (n < N && k < K) ? Wq[n * K + k] : 0;
+                        if (v < -1 || v > 1)
+                            return -1;
+                        value += (v + 1) * power;
+                        power *= 3;
+                    }
+                    packed[blk * 16 * row_bytes + 512 * g + 32 * r + B] = (uint8_t)value;
+                }
+            }
+        }
+    }
+    return 0;
+}

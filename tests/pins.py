@@ -59,10 +59,10 @@ def load_golden(name: str) -> dict:
     return out
 
 
-def load_pack_cases() -> list:
+def load_pack_cases(name: str = "pack_words.txt") -> list:
     """(name, N, K, [(row, k, value)], {offset: byte}, size) per golden case."""
     cases = []
-    with open(os.path.join(GOLDEN, "pack_words.txt")) as f:
+    with open(os.path.join(GOLDEN, name)) as f:
         for line in f:
             line = line.strip()
             if not line.startswith("case"):
@@ -168,6 +168,58 @@ def pin_pack_roundtrip(orc):
     packed = orc.pack_codes(Wq)
     assert packed.size == 32 * 256 // 4
     np.testing.assert_array_equal(decode_packed_spec(packed, 21, 256), Wq)
+
+
+def pin_pack_b3_bytes(orc):
+    for name, N, K, ws, by, size in load_pack_cases("pack_b3_bytes.txt"):
+        Wq = np.zeros((N, K), dtype=np.int8)
+        for r, k, v in ws:
+            Wq[r, k] = v
+        got = orc.pack_codes_b3(Wq)
+        want = np.full(size, 121, dtype=np.uint8)
+        for off, val in by.items():
+            want[off] = val
+        assert got.shape == want.shape, (name, got.shape)
+        np.testing.assert_array_equal(got, want, err_msg=name)
+
+
+def decode_packed_b3_spec(packed: np.ndarray, N: int, K: int) -> np.ndarray:
+    """Independent decoder of the base-3 layout from its spec: byte B of row
+    n = 16 blk + r, group g sits at blk*16*Kp/5 + 512 g + 32 r + B and holds
+    the base-3 digits of stream positions p = 5B + i (digit i is worth 3^i);
+    position p = 16 w + 4 b + j is the weight k = 160 g + 16 w + 4 j + b.
+    Padding rows and padding columns (k >= K) must decode to zeros."""
+    packed = np.asarray(packed).reshape(-1)
+    Kp = (K + 159) // 160 * 160
+    blocks = (N + 15) // 16
+    assert packed.size == blocks * 16 * Kp // 5
+    out = np.zeros((blocks * 16, Kp), dtype=np.int8)
+    for blk in range(blocks):
+        for r in range(16):
+            for g in range(Kp // 160):
+                for B in range(32):
+                    v = int(packed[blk * 16 * Kp // 5 + 512 * g + 32 * r + B])
+                    assert v < 243
+                    for i in range(5):
+                        code = v % 3
+                        v //= 3
+                        p = 5 * B + i
+                        w, b, j = p // 16, (p % 16) // 4, p % 4
+                        out[16 * blk + r, 160 * g + 16 * w + 4 * j + b] = code - 1
+    assert np.all(out[N:] == 0) and np.all(out[:, K:] == 0)
+    return out[:N, :K]
+
+
+def pin_pack_b3_roundtrip(orc):
+    """Random ternary weights, ragged rows and a K that is not a multiple of
+    160, decode back to themselves; both layouts decode to the same weights."""
+    r = np.random.Generator(np.random.PCG64(8))
+    for N, K in [(21, 384), (5, 128), (16, 640)]:
+        Wq = r.integers(-1, 2, size=(N, K), dtype=np.int8)
+        packed = orc.pack_codes_b3(Wq)
+        assert packed.size == (N + 15) // 16 * 16 * ((K + 159) // 160 * 160) // 5
+        np.testing.assert_array_equal(decode_packed_b3_spec(packed, N, K), Wq)
+        np.testing.assert_array_equal(decode_packed_spec(orc.pack_codes(Wq), N, K), Wq)
 
 
 def pin_constant_token(orc):
@@ -499,6 +551,8 @@ ALL_PINS = [
     pin_activation_ties_even,
     pin_pack_words,
     pin_pack_roundtrip,
+    pin_pack_b3_bytes,
+    pin_pack_b3_roundtrip,
     pin_constant_token,
     pin_zero_inputs,
     pin_tiny_scale_epsilon,

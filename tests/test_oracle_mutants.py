@@ -46,6 +46,13 @@ MUTANTS = {
     "pack_word_index": ("16 * w + 4 * j + b;", "16 * w + 4 * b + j;"),
     "pack_row_stride": ("512 * g + 32 * r + 4 * w", "512 * g + 32 * w + 4 * r"),
     "pack_padding_rows": ("(n < N) ? Wq[n * K + k] : 0", "(n < N) ? Wq[n * K + k] : -1"),
+    "b3_digit_order": ("value += (v + 1) * power;", "value = value * 3 + (v + 1);"),
+    "b3_stream_transposed": ("const int64_t k = 160 * g + 16 * w + 4 * j + b;",
+                             "const int64_t k = 160 * g + 16 * w + 4 * b + j;"),
+    "b3_padding_code": ("const int v = (n < N && k < K) ? Wq[n * K + k] : 0;",
+                        "const int v = (n < N && k < K) ? Wq[n * K + k] : -1;"),
+    "b3_byte_order": ("packed[blk * 16 * row_bytes + 512 * g + 32 * r + B]",
+                      "packed[blk * 16 * row_bytes + 512 * g + 32 * r + (31 - B)]"),
     "rms_drops_eps": ("sqrtf(ms + eps)", "sqrtf(ms)"),
     "rms_mean_over_k_minus_1": ("ss / (double)K", "ss / (double)(K - 1)"),
     "rms_forgets_sqrt": ("1.0f / sqrtf(ms + eps)", "1.0f / (ms + eps)"),
