@@ -448,6 +448,34 @@ def bench_rmsnorm_decode(bl, wl, reps: int = 200) -> float:
     return time_graph(steps, reps, nvtx="rmsnorm_decode_timed") / ROTATE
 
 
+def bench_b3_decode(bl, wl, reps: int = 200):
+    """The decode step's two projections (M = 1) on base-3 packed weights
+    (bitlinear_forward_b3, one launch per projection) over ROTATE copies, the
+    footprint option: µs per step, GB/s of base-3 bytes, and the bytes per
+    step against the 2-bit layout's."""
+    import torch
+    mats = []
+    for m in wl.mats:
+        p = m["p"]
+        pk, gamma = bl.bitlinear_pack_weights_b3(p.weights())
+        dp = torch.from_numpy(pk).to(m["x"][0].device)
+        mats.append((m, [dp] + [dp.clone() for _ in range(ROTATE - 1)], gamma))
+    b3_bytes = sum(d[0].numel() for _, d, _ in mats)
+
+    def steps():
+        for j in range(ROTATE):
+            for m, d, g in mats:
+                bl.bitlinear_forward_b3(m["x"][j], d[j], g, m["p"].N, y=m["y"][j])
+    steps()
+    torch.cuda.synchronize()
+    ms = time_graph(steps, reps, nvtx="b3_decode_timed") / ROTATE
+    return {"us_per_step": round(ms * 1e3, 3),
+            "GBps_b3_bytes": round(b3_bytes / (ms * 1e-3) / 1e9, 1),
+            "b3_bytes_per_step": b3_bytes,
+            "two_bit_bytes_per_step": wl.packed_bytes_per_step,
+            "launches_per_step": 2}
+
+
 def bench_ffn(bl, device, batches=(1, 8), copies: int = 16, reps: int = 20):
     """The 2B decoder's feed-forward block (gate and up 2560 -> 6912, the
     gated ReLU^2, down 6912 -> 2560) for B decode tokens through
@@ -768,6 +796,11 @@ def run_ours(args, dist):
                               "frac": round(norm_pre_tops / int8_peak, 4)}},
     }
     if not args.no_extra:
+        out["b3_decode"] = {
+            "workload": "the decode step (up 2560->6912, down 6912->2560, M=1) on base-3 packed "
+                        "weights (5 codes per byte, K padded to a multiple of 160), one launch "
+                        "per projection; compare decode_separate_launches",
+            **bench_b3_decode(bl, wl)}
         out["ffn_chain"] = {
             "workload": "2B feed-forward block: gate and up 2560->6912 (one GEMV launch, h = "
                         "max(gate,0)^2 * up written from its epilogue), down 6912->2560 on h; "

@@ -111,6 +111,45 @@ size_t bitlinear_packed_bytes(int64_t N, int64_t K);
 int bitlinear_pack_weights(const float *W_host, int64_t N, int64_t K,
                            void *packed_host, float *gamma_out);
 
+/* ------------------------------------------------------- base-3 packing */
+
+/* Bytes of the base-3 packed matrix: ceil(N / 16) * 16 * Kp / 5 with Kp = K
+ * rounded up to a multiple of 160 (1.6 bits per weight, 20% less than the
+ * 2-bit layout). 0 for the shapes bitlinear_packed_bytes refuses.
+ *
+ * Base-3 layout (this library's own; log2(3) = 1.58 bits per weight is what
+ * puts the 2B model's non-embedding weights near 0.4 GB: "Microsoft Releases
+ * BitNet b1.58 2B4T", opening section):
+ *   - K is padded with zero weights to Kp; rows come in blocks of 16 (the last
+ *     completed with zero rows); block b occupies the 16 * Kp / 5 bytes
+ *     starting at byte b * 16 * Kp / 5;
+ *   - inside a block the weights come in k-groups of 160: group g holds the
+ *     weights k in [160g, 160g + 160) of all 16 rows in the 512 bytes at
+ *     offset 512 g, row r of the block in the 32 bytes at offset 32 r;
+ *   - those 32 bytes hold the 160 codes W~ + 1 of the row in stream order:
+ *     stream position p = 16w + 4b + j is the weight k = 160g + 16w + 4j + b
+ *     (the 2-bit fields of the 2-bit layout's words, read from bit 0 up);
+ *   - byte B holds stream positions 5B .. 5B + 4 as sum_i code(5B + i) * 3^i. */
+size_t bitlinear_packed_bytes_b3(int64_t N, int64_t K);
+
+/* bitlinear_pack_weights into the base-3 layout: the same gamma and codes,
+ * five per byte. packed_host holds bitlinear_packed_bytes_b3(N, K) bytes.
+ * Errors as for bitlinear_pack_weights. */
+int bitlinear_pack_weights_b3(const float *W_host, int64_t N, int64_t K,
+                              void *packed_host, float *gamma_out);
+
+/* bitlinear_forward on base-3 packed weights (a footprint option: 20% fewer
+ * weight bytes in HBM, decoded in the GEMV through a 256-entry table in
+ * shared memory). The GEMV path only: M <= 16 and M * Kp <= 196608, else
+ * BITLINEAR_ERR_SHAPE before any device work. Arguments and results as for
+ * bitlinear_forward, with packed_b3_dev holding
+ * bitlinear_packed_bytes_b3(N, K) bytes; no workspace. */
+int bitlinear_forward_b3(const void *x_dev, bitlinear_dtype xdt, int64_t M,
+                         int64_t K, const void *packed_b3_dev, float gamma,
+                         int64_t N, void *y_dev, void *cuda_stream,
+                         int32_t *acc_dev_or_null, int8_t *xq_dev_or_null,
+                         float *beta_dev_or_null);
+
 /* ------------------------------------------------------ packed-weight files */
 
 /* The packer's output stored once and loaded at serving time (the ternary

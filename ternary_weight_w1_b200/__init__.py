@@ -46,6 +46,9 @@ RMSNORM_EPS = 2.0 ** -23
 EXPORTS = (
     "bitlinear_packed_bytes",
     "bitlinear_pack_weights",
+    "bitlinear_packed_bytes_b3",
+    "bitlinear_pack_weights_b3",
+    "bitlinear_forward_b3",
     "bitlinear_save_packed",
     "bitlinear_read_packed_header",
     "bitlinear_load_packed",
@@ -96,6 +99,13 @@ def lib() -> ctypes.CDLL:
         L.bitlinear_packed_bytes.argtypes = [i64, i64]
         L.bitlinear_pack_weights.restype = ctypes.c_int
         L.bitlinear_pack_weights.argtypes = [p, i64, i64, p, p]
+        L.bitlinear_packed_bytes_b3.restype = sz
+        L.bitlinear_packed_bytes_b3.argtypes = [i64, i64]
+        L.bitlinear_pack_weights_b3.restype = ctypes.c_int
+        L.bitlinear_pack_weights_b3.argtypes = [p, i64, i64, p, p]
+        L.bitlinear_forward_b3.restype = ctypes.c_int
+        L.bitlinear_forward_b3.argtypes = [p, ctypes.c_int, i64, i64, p, ctypes.c_float, i64, p,
+                                           p, p, p, p]
         L.bitlinear_save_packed.restype = ctypes.c_int
         L.bitlinear_save_packed.argtypes = [ctypes.c_char_p, p, i64, i64, ctypes.c_float]
         L.bitlinear_read_packed_header.restype = ctypes.c_int
@@ -241,6 +251,28 @@ def bitlinear_pack_weights(W) -> tuple[np.ndarray, float]:
     return out, float(gamma.value)
 
 
+def bitlinear_packed_bytes_b3(N: int, K: int) -> int:
+    return int(lib().bitlinear_packed_bytes_b3(N, K))
+
+
+def bitlinear_pack_weights_b3(W) -> tuple[np.ndarray, float]:
+    """Ternarise and pack latent fp32 weights [N][K] into the base-3 layout
+    (five codes per byte) on the host. Returns (packed bytes, gamma)."""
+    W = np.ascontiguousarray(np.asarray(W, dtype=np.float32))
+    if W.ndim != 2:
+        raise ValueError("W must be 2-D [N][K]")
+    N, K = W.shape
+    nbytes = bitlinear_packed_bytes_b3(N, K)
+    if nbytes == 0:
+        raise BitLinearError(BITLINEAR_ERR_SHAPE, "bitlinear_pack_weights_b3")
+    out = np.empty((nbytes,), dtype=np.uint8)
+    gamma = ctypes.c_float(0.0)
+    _check(lib().bitlinear_pack_weights_b3(W.ctypes.data, N, K, out.ctypes.data,
+                                           ctypes.addressof(gamma)),
+           "bitlinear_pack_weights_b3")
+    return out, float(gamma.value)
+
+
 def bitlinear_save_packed(path, packed, N: int, K: int, gamma: float) -> None:
     """Write packed weights (host uint8 array of bitlinear_packed_bytes(N, K)
     bytes, as bitlinear_pack_weights returns it) and gamma to a file."""
@@ -327,6 +359,25 @@ def bitlinear_forward(x, packed, gamma: float, N: int, y=None, workspace=None,
     else:
         rc = lib().bitlinear_forward_ex(*args, path)
     _check(rc, "bitlinear_forward")
+    return y
+
+
+def bitlinear_forward_b3(x, packed_b3, gamma: float, N: int, y=None, stream=None, acc=None,
+                         xq=None, beta=None):
+    """y (bf16 [M][N]) = BitLinear(x) with base-3 packed weights (the GEMV
+    path: M <= 16); ``acc``/``xq``/``beta`` are optional debug outputs."""
+    a = _Args()
+    import torch
+    M, K = x.shape
+    if y is None:
+        y = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
+    need = bitlinear_packed_bytes_b3(N, K) if N >= 1 and K >= 128 and K % 128 == 0 else 1
+    rc = lib().bitlinear_forward_b3(
+        a.ptr(x, "x"), _xdt(x), M, K, a.ptr(packed_b3, "packed_b3", torch.uint8, min_numel=need),
+        float(gamma), N, a.ptr(y, "y", torch.bfloat16, (M, N)), _stream(stream),
+        a.ptr(acc, "acc", torch.int32, (M, N)), a.ptr(xq, "xq", torch.int8, (M, K)),
+        a.ptr(beta, "beta", torch.float32, (M,)))
+    _check(rc, "bitlinear_forward_b3")
     return y
 
 

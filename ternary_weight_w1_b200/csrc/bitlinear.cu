@@ -263,15 +263,23 @@ int launch_quant_act(const void *x, bitlinear_dtype xdt, int M, int K, int8_t *x
 
 // ------------------------------------------------------------------- GEMV
 
-template <int MT, bool BF16, bool NORM, bool FFN, bool WIDE = false>
+template <int MT, bool BF16, bool NORM, bool FFN, bool WIDE = false, bool B3 = false>
 int launch_gemv_t(const gemv::Params &p, int grid, int smem, int dev, cudaStream_t st)
 {
-    cudaError_t e = allow_smem<gemv::gemv_kernel<MT, BF16, NORM, FFN, WIDE>>(dev, smem);
+    cudaError_t e = allow_smem<gemv::gemv_kernel<MT, BF16, NORM, FFN, WIDE, B3>>(dev, smem);
     if (e != cudaSuccess)
         return launch_status(e);
-    e = launch(gemv::gemv_kernel<MT, BF16, NORM, FFN, WIDE>, dim3(grid), dim3(gemv::THREADS), smem,
-               st, p);
+    e = launch(gemv::gemv_kernel<MT, BF16, NORM, FFN, WIDE, B3>, dim3(grid), dim3(gemv::THREADS),
+               smem, st, p);
     return launch_status(e);
+}
+
+// The kernels that read the base-3 layout.
+template <int MT>
+int launch_gemv_b3(const gemv::Params &p, bool bf16, int grid, int smem, int dev, cudaStream_t st)
+{
+    return bf16 ? launch_gemv_t<MT, true, false, false, false, true>(p, grid, smem, dev, st)
+                : launch_gemv_t<MT, false, false, false, false, true>(p, grid, smem, dev, st);
 }
 
 template <int MT>
@@ -318,6 +326,7 @@ struct GemvJob {
     const float *norm_gain2 = nullptr;
     void *y2 = nullptr;
     float *h = nullptr;
+    bool b3 = false;            // `packed` is in the base-3 layout
 };
 
 // Launches the GEMV kernel over one or more independent problems. Every CTA
@@ -337,8 +346,18 @@ int launch_gemv(const GemvJob *jobs, int count, bitlinear_dtype xdt, const Devic
 {
     const bool norm = jobs[0].norm_gain != nullptr;
     const bool ffn = jobs[0].h != nullptr;
+    const bool b3 = jobs[0].b3;
     if (ffn && count != 1)
         return BITLINEAR_ERR_ARG;
+    for (int i = 1; i < count; ++i)
+        if (jobs[i].b3 != b3)
+            return BITLINEAR_ERR_ARG;
+    if (b3 && (norm || ffn))
+        return BITLINEAR_ERR_ARG;
+    // k-groups per row: of 128 weights, or of 160 in the base-3 layout, whose
+    // rows (and the x~ rows) are padded to 160 per group
+    auto groups_of = [b3](int K) { return b3 ? (K + 159) / 160 : K / 128; };
+    auto xrow_of = [b3, &groups_of](int K) { return b3 ? groups_of(K) * 160 : K; };
     for (int i = 1; i < count; ++i)
         if ((jobs[i].norm_gain != nullptr) != norm)
             return BITLINEAR_ERR_ARG;
@@ -347,8 +366,8 @@ int launch_gemv(const GemvJob *jobs, int count, bitlinear_dtype xdt, const Devic
     int xq_cap = 0;
     for (int i = 0; i < count; ++i) {
         Mmax = std::max(Mmax, jobs[i].M);
-        total_bytes += static_cast<double>((jobs[i].N + 15) / 16) * 16.0 * jobs[i].K / 4.0;
-        xq_cap = std::max(xq_cap, jobs[i].M * jobs[i].K);
+        total_bytes += static_cast<double>((jobs[i].N + 15) / 16) * groups_of(jobs[i].K) * 512.0;
+        xq_cap = std::max(xq_cap, jobs[i].M * xrow_of(jobs[i].K));
     }
     const int MT = gemv_tile(Mmax);
     const int QB = gemv::chunk_blocks(MT, ffn);
@@ -358,7 +377,7 @@ int launch_gemv(const GemvJob *jobs, int count, bitlinear_dtype xdt, const Devic
         max_K = std::max(max_K, jobs[i].K);
     // one bf16 token of a long row: the wide kernel, whose x~ region first
     // holds the staged bf16 row (2 K bytes), two blocks per SM
-    const bool wide = MT == 1 && !norm && !ffn && xdt == BITLINEAR_BF16 && max_K > 8192 &&
+    const bool wide = MT == 1 && !norm && !ffn && !b3 && xdt == BITLINEAR_BF16 && max_K > 8192 &&
                       max_K <= 32768;
     if (wide)
         xq_cap *= 2;
@@ -368,7 +387,7 @@ int launch_gemv(const GemvJob *jobs, int count, bitlinear_dtype xdt, const Devic
     double max_block = 0.0;
     for (int i = 0; i < count; ++i) {
         blocks[i] = (jobs[i].N + 15) / 16;
-        bbytes[i] = nmat * 16.0 * jobs[i].K / 4.0;
+        bbytes[i] = nmat * 512.0 * groups_of(jobs[i].K);
         max_block = std::max(max_block, bbytes[i]);
     }
     // CTAs: one wave of two per SM (a third fits beside them, for the next
@@ -411,7 +430,7 @@ int launch_gemv(const GemvJob *jobs, int count, bitlinear_dtype xdt, const Devic
         red_blocks = 1;
         int stages = 1;
         for (int i = 0; i < count; ++i) {
-            const int KG = jobs[i].K / 128;
+            const int KG = groups_of(jobs[i].K);
             const int q = (blocks[i] + ctas[i] - 1) / ctas[i];
             const int row_block = nmat * KG * gemv::PIECE;     // one block, all matrices
             if (2 * row_block <= target_rows || (q == 1 && row_block <= target_rows)) {
@@ -429,12 +448,12 @@ int launch_gemv(const GemvJob *jobs, int count, bitlinear_dtype xdt, const Devic
         // Ring depth: the whole share when it is small, else as deep as a
         // 72 KiB block allows (three blocks per SM fit beside each other;
         // 110 KiB for the wide kernel's two).
-        const int fixed = gemv::smem_bytes(MT, xq_cap, 0, 0, red_blocks, norm, ffn);
+        const int fixed = gemv::smem_bytes(MT, xq_cap, 0, 0, red_blocks, norm, ffn, b3);
         slots = (ring_budget - fixed) / slot_bytes;
         slots = std::max(1, std::min({slots, stages, gemv::MAX_SLOTS}));
         if (stages > 1)
             slots = std::max(slots, 2);
-        smem = gemv::smem_bytes(MT, xq_cap, slots, slot_bytes, red_blocks, norm, ffn);
+        smem = gemv::smem_bytes(MT, xq_cap, slots, slot_bytes, red_blocks, norm, ffn, b3);
         if (smem <= dev.max_smem_optin)
             break;
         // too large beside a large x~: smaller stages
@@ -482,6 +501,15 @@ int launch_gemv(const GemvJob *jobs, int count, bitlinear_dtype xdt, const Devic
     const bool bf16 = xdt == BITLINEAR_BF16;
     if (wide)
         return launch_gemv_wide(p, grid, smem, dev.id, st);
+    if (b3) {
+        switch (MT) {
+        case 1: return launch_gemv_b3<1>(p, bf16, grid, smem, dev.id, st);
+        case 2: return launch_gemv_b3<2>(p, bf16, grid, smem, dev.id, st);
+        case 4: return launch_gemv_b3<4>(p, bf16, grid, smem, dev.id, st);
+        case 8: return launch_gemv_b3<8>(p, bf16, grid, smem, dev.id, st);
+        default: return launch_gemv_b3<16>(p, bf16, grid, smem, dev.id, st);
+        }
+    }
     switch (MT) {
     case 1: return launch_gemv_mt<1>(p, bf16, norm, ffn, grid, smem, dev.id, st);
     case 2: return launch_gemv_mt<2>(p, bf16, norm, ffn, grid, smem, dev.id, st);
@@ -991,6 +1019,41 @@ extern "C" int bitlinear_ffn_forward(const void *x_dev, bitlinear_dtype xdt, int
     return forward_impl(h_dev, BITLINEAR_FP32, M, F, down_packed_dev, down_gamma, K, y_dev,
                         workspace_dev, workspace_bytes, cuda_stream, nullptr, nullptr, nullptr,
                         BITLINEAR_PATH_AUTO, 0, down_gain_dev, norm_eps);
+}
+
+extern "C" int bitlinear_forward_b3(const void *x_dev, bitlinear_dtype xdt, int64_t M, int64_t K,
+                                    const void *packed_b3_dev, float gamma, int64_t N,
+                                    void *y_dev, void *cuda_stream, int32_t *acc_dev_or_null,
+                                    int8_t *xq_dev_or_null, float *beta_dev_or_null)
+{
+    int rc = check_forward_args(x_dev, xdt, M, K, packed_b3_dev, N, y_dev, acc_dev_or_null,
+                                xq_dev_or_null, beta_dev_or_null);
+    if (rc != BITLINEAR_OK)
+        return rc;
+    if (M == 0)
+        return BITLINEAR_OK;
+    // the GEMV holds the tokens' x~ rows, padded to 160-weight groups
+    const int64_t Kp = (K + 159) / 160 * 160;
+    if (M > kGemvMaxM || M * Kp > gemv_max_xq(M))
+        return BITLINEAR_ERR_SHAPE;
+    DeviceInfo *dev = nullptr;
+    rc = current_device(&dev);
+    if (rc != BITLINEAR_OK)
+        return rc;
+    GemvJob job{x_dev,
+                static_cast<int>(M),
+                static_cast<int>(K),
+                static_cast<int>(N),
+                packed_b3_dev,
+                gamma,
+                y_dev,
+                acc_dev_or_null,
+                xq_dev_or_null,
+                beta_dev_or_null,
+                nullptr,
+                0.0f};
+    job.b3 = true;
+    return launch_gemv(&job, 1, xdt, *dev, static_cast<cudaStream_t>(cuda_stream));
 }
 
 extern "C" int bitlinear_forward_grouped(const bitlinear_problem *problems, int count,

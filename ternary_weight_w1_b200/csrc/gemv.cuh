@@ -141,12 +141,15 @@ struct Params {
 // carves them out; every region size is a multiple of 16 bytes). An FFN
 // launch keeps two reduction areas (gate and up) and, when it normalises,
 // two quantised copies of the tokens with their own beta and sums.
+// A base-3 launch adds its 256-entry decoding table.
 __host__ __device__ constexpr int smem_bytes(int MT, int xq_cap, int slots, int slot_bytes,
-                                             int red_blocks, bool norm, bool ffn = false)
+                                             int red_blocks, bool norm, bool ffn = false,
+                                             bool b3 = false)
 {
     return slots * slot_bytes + BAR_BYTES + (ffn && norm ? 2 : 1) * xq_cap +
            (ffn ? 2 : 1) * CWARPS * red_blocks * 16 * MT * 4 + (norm ? MT * CWARPS * 8 : 0) +
-           (ffn && norm ? 2 : 1) * (16 * ((MT * 4 + 15) / 16) + 2 * MT * CWARPS * 4);
+           (ffn && norm ? 2 : 1) * (16 * ((MT * 4 + 15) / 16) + 2 * MT * CWARPS * 4) +
+           (b3 ? 256 * 4 : 0);
 }
 
 // r of token m from the warps' partial sums of squares, added in warp order.
@@ -193,8 +196,12 @@ __device__ __forceinline__ void load4(const void *row, int e, float (&v)[4])
 
 // WIDE (one bf16 token of 8192 < K <= 32768, no normalisation, not FFN)
 // stages the token row in shared memory for the prologue (two blocks per SM).
-template <int MT, bool BF16, bool NORM, bool FFN, bool WIDE>
-__global__ void __launch_bounds__(THREADS, ((NORM || WIDE) ? 2 : Shape<MT, FFN>::MIN_BLOCKS))
+// B3 reads the base-3 layout (five codes per byte; no normalisation, not FFN,
+// not WIDE): a 256-entry table in shared memory turns each byte back into ten
+// bits of 2-bit codes, rebuilding the 2-bit layout's words in registers.
+template <int MT, bool BF16, bool NORM, bool FFN, bool WIDE, bool B3 = false>
+__global__ void __launch_bounds__(THREADS,
+                                  ((NORM || WIDE || B3) ? 2 : Shape<MT, FFN>::MIN_BLOCKS))
 gemv_kernel(const __grid_constant__ Params p)
 {
     using S = Shape<MT, FFN>;
@@ -202,7 +209,8 @@ gemv_kernel(const __grid_constant__ Params p)
     constexpr int NMAT = FFN ? 2 : 1;          // matrices streamed (gate, up)
     constexpr int NX = (FFN && NORM) ? 2 : 1;   // quantised copies of the tokens
     // with two copies of x~ in registers, fewer tokens at a time
-    constexpr int TQ = NX == 1 ? S::TQ : MT >= 8 ? 1 : (S::TQ < 2 ? S::TQ : 2);
+    // (and with the base-3 layout's five-word x~ runs)
+    constexpr int TQ = (NX == 1 && !B3) ? S::TQ : MT >= 8 ? 1 : (S::TQ < 2 ? S::TQ : 2);
     constexpr int NACC = S::PERSIST ? 4 : MT;   // accumulators per block and matrix
     extern __shared__ __align__(128) uint8_t smem[];
     // this CTA's problem (grouped launches give each problem its own CTAs)
@@ -212,7 +220,12 @@ gemv_kernel(const __grid_constant__ Params p)
         ++pi;
     const Problem &P = p.prob[pi];
     const int K = P.K, M = P.M, N = P.N;
-    const int KG = K >> 7;                              // k-groups per row
+    // k-groups per row: of 128 weights, or of 160 in the base-3 layout, whose
+    // rows (and x~ rows) are padded to XS = 160 KG
+    constexpr int GW = B3 ? 160 : 128;                  // weights per k-group
+    constexpr int NW = GW / 32;                         // code words per lane and piece
+    const int KG = B3 ? (K + 159) / 160 : K >> 7;
+    const int XS = B3 ? KG * 160 : K;
     const int G = P.G;
     const int total_blocks = (N + 15) >> 4;
     const int cta = static_cast<int>(blockIdx.x) - P.cta_begin;
@@ -246,6 +259,8 @@ gemv_kernel(const __grid_constant__ Params p)
     auto beta_sm = [&](int x) { return qset + x * QSET; };
     auto red_u = [&](int x) { return reinterpret_cast<uint32_t *>(qset + x * QSET + 4 * ((MT + 3) / 4)); };
     auto red_s = [&](int x) { return reinterpret_cast<int *>(red_u(x) + MT * CWARPS); };
+    // base-3 decoding table: byte value -> its five codes as 2-bit fields
+    uint32_t *lut = reinterpret_cast<uint32_t *>(qset + NX * QSET);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -258,6 +273,22 @@ gemv_kernel(const __grid_constant__ Params p)
         }
         *abort_flag = 0;
         fence_barrier_init();
+    }
+    if constexpr (B3) {
+        // entry v: the base-3 digits of v (0 .. 242) as 2-bit codes at bits
+        // 2i; bytes above 242 do not occur and decode to zero weights
+        for (int v = threadIdx.x; v < 256; v += THREADS) {
+            uint32_t f = 0x155u;
+            if (v < 243) {
+                f = 0;
+                int t = v;
+                for (int i = 0; i < 5; ++i) {
+                    f |= static_cast<uint32_t>(t % 3) << (2 * i);
+                    t /= 3;
+                }
+            }
+            lut[v] = f;
+        }
     }
     __syncthreads();
 
@@ -345,7 +376,68 @@ gemv_kernel(const __grid_constant__ Params p)
     const int nsl = (ngw + 1) / 2;                    // slots of this warp
     // gains of quantised copy x (FFN: 0 = gate, 1 = up)
     auto gain_of = [&](int x) { return (FFN && x == 1) ? P.norm_gain2 : P.norm_gain; };
-    if constexpr (WIDE) {
+    if constexpr (B3) {
+        // The base-3 layout pads each row to XS = 160 KG weights: the tokens
+        // are quantised by all compute threads together into x~ rows of XS
+        // bytes whose padding is zero, and a block barrier makes them visible
+        // to every warp.
+        static_assert(!NORM && !FFN && !WIDE, "base-3 kernel");
+        for (int m = 0; m < M; ++m) {
+            const void *row = static_cast<const char *>(P.x) + m * row_bytes;
+            float amax = 0.0f;
+            for (int e = ctid * 8; e < K; e += CTHREADS * 8) {
+                Vec8<BF16> v;
+                v.load(row, e);
+#pragma unroll
+                for (int u = 0; u < 8; ++u)
+                    amax = fmaxf(amax, fabsf(v.get(u)));
+            }
+            const uint32_t um = __reduce_max_sync(0xffffffffu, __float_as_uint(amax));
+            if (lane == 0)
+                red_u(0)[m * CWARPS + warp] = um;
+        }
+        compute_sync();
+        for (int m = 0; m < M; ++m) {
+            const void *row = static_cast<const char *>(P.x) + m * row_bytes;
+            uint32_t ub = red_u(0)[m * CWARPS];
+#pragma unroll
+            for (int w = 1; w < CWARPS; ++w)
+                ub = max(ub, red_u(0)[m * CWARPS + w]);
+            const float beta = fmaxf(__uint_as_float(ub), 1e-5f);
+            const float scale = __fdiv_rn(127.0f, beta);
+            int sum = 0;
+            for (int e = ctid * 8; e < XS; e += CTHREADS * 8) {
+                uint32_t lo = 0, hi = 0;
+                if (e < K) {
+                    Vec8<BF16> v;
+                    v.load(row, e);
+                    // |x * (127 / beta)| <= 127: the listing's clamp cannot bind
+                    int q[8];
+#pragma unroll
+                    for (int u = 0; u < 8; ++u)
+                        q[u] = __float2int_rn(__fmul_rn(v.get(u), scale));
+                    lo = __byte_perm(__byte_perm(q[0], q[1], 0x0040),
+                                     __byte_perm(q[2], q[3], 0x0040), 0x5410);
+                    hi = __byte_perm(__byte_perm(q[4], q[5], 0x0040),
+                                     __byte_perm(q[6], q[7], 0x0040), 0x5410);
+                    sum = dp4a_ss(hi, 0x01010101u, dp4a_ss(lo, 0x01010101u, sum));
+                    if (P.xq_dbg != nullptr && first_cta)
+                        *reinterpret_cast<uint2 *>(P.xq_dbg + static_cast<size_t>(m) * K + e) =
+                            make_uint2(lo, hi);
+                }
+                *reinterpret_cast<uint2 *>(xq_sm + m * XS + e) = make_uint2(lo, hi);
+            }
+            sum = __reduce_add_sync(0xffffffffu, sum);
+            if (lane == 0)
+                red_s(0)[m * CWARPS + warp] = sum;
+            if (ctid == 0) {
+                beta_sm(0)[m] = beta;
+                if (P.beta_dbg != nullptr && first_cta)
+                    P.beta_dbg[m] = beta;
+            }
+        }
+        compute_sync();
+    } else if constexpr (WIDE) {
         // One bf16 token of up to 32768 activations. Its row is staged in
         // shared memory (the 2 K bytes of the x~ region, which x~ overwrites
         // at the end) with 16-byte asynchronous copies of every slot of this
@@ -624,20 +716,21 @@ gemv_kernel(const __grid_constant__ Params p)
 #pragma unroll
                     for (int m0 = 0; m0 < MT; m0 += TQ) {
                         if (m0 < M) {
-                            // x~ of this lane's 64 weights for tokens m0 .. m0+TQ-1
-                            uint32_t X[NX][TQ][16];
+                            // x~ of this lane's GW / 2 weights for tokens m0 .. m0+TQ-1
+                            uint32_t X[NX][TQ][4 * NW];
 #pragma unroll
                             for (int x = 0; x < NX; ++x) {
-                                const uint8_t *xg = xq_sm + x * p.xq_cap + (g0 + gi) * 128 + t * 64;
+                                const uint8_t *xg =
+                                    xq_sm + x * p.xq_cap + (g0 + gi) * GW + t * (GW / 2);
 #pragma unroll
                                 for (int mq = 0; mq < TQ; ++mq) {
 #pragma unroll
-                                    for (int v = 0; v < 4; ++v) {
+                                    for (int v = 0; v < NW; ++v) {
                                         // tokens past M (a smaller problem of a
                                         // grouped launch) read nothing
                                         const uint4 xv = (m0 + mq < M)
                                                              ? *reinterpret_cast<const uint4 *>(
-                                                                   xg + (m0 + mq) * K + 16 * v)
+                                                                   xg + (m0 + mq) * XS + 16 * v)
                                                              : make_uint4(0, 0, 0, 0);
                                         X[x][mq][4 * v] = xv.x; X[x][mq][4 * v + 1] = xv.y;
                                         X[x][mq][4 * v + 2] = xv.z; X[x][mq][4 * v + 3] = xv.w;
@@ -655,19 +748,39 @@ gemv_kernel(const __grid_constant__ Params p)
                                     {
                                         const uint4 w4 = *reinterpret_cast<const uint4 *>(
                                             stage + ((mat * qb + bi) * gs + gi) * PIECE);
-                                        const uint32_t wd[4] = {w4.x, w4.y, w4.z, w4.w};
+                                        uint32_t wd[NW];
+                                        if constexpr (B3) {
+                                            // byte B of the lane's 16 holds the
+                                            // 2-bit fields 5B .. 5B+4 of its
+                                            // five-word code stream
+                                            const uint32_t by[4] = {w4.x, w4.y, w4.z, w4.w};
+#pragma unroll
+                                            for (int q = 0; q < NW; ++q)
+                                                wd[q] = 0;
+#pragma unroll
+                                            for (int B = 0; B < 16; ++B) {
+                                                const uint32_t f =
+                                                    lut[(by[B >> 2] >> (8 * (B & 3))) & 0xffu];
+                                                const int pos = 10 * B;
+                                                wd[pos >> 5] |= f << (pos & 31);
+                                                if ((pos & 31) > 22)
+                                                    wd[(pos >> 5) + 1] |= f >> (32 - (pos & 31));
+                                            }
+                                        } else {
+                                            wd[0] = w4.x; wd[1] = w4.y; wd[2] = w4.z; wd[3] = w4.w;
+                                        }
                                         if constexpr (S::PERSIST) {
 #pragma unroll
-                                            for (int jw = 0; jw < 4; ++jw) {
+                                            for (int jw = 0; jw < NW; ++jw) {
                                                 acc[mat][bi][0] = dp4a_us(wd[jw] & 0x03030303u, X[xs][0][4 * jw], acc[mat][bi][0]);
                                                 acc[mat][bi][1] = dp4a_us(wd[jw] & 0x0C0C0C0Cu, X[xs][0][4 * jw + 1], acc[mat][bi][1]);
                                                 acc[mat][bi][2] = dp4a_us(wd[jw] & 0x30303030u, X[xs][0][4 * jw + 2], acc[mat][bi][2]);
                                                 acc[mat][bi][3] = dp4a_us(wd[jw] & 0xC0C0C0C0u, X[xs][0][4 * jw + 3], acc[mat][bi][3]);
                                             }
                                         } else {
-                                            uint32_t pl[16];
+                                            uint32_t pl[4 * NW];
 #pragma unroll
-                                            for (int jw = 0; jw < 4; ++jw) {
+                                            for (int jw = 0; jw < NW; ++jw) {
                                                 pl[4 * jw] = wd[jw] & 0x03030303u;
                                                 pl[4 * jw + 1] = wd[jw] & 0x0C0C0C0Cu;
                                                 pl[4 * jw + 2] = wd[jw] & 0x30303030u;
@@ -677,7 +790,7 @@ gemv_kernel(const __grid_constant__ Params p)
                                             for (int mq = 0; mq < TQ; ++mq) {
                                                 int a0 = 0, a1 = 0, a2 = 0, a3 = 0;
 #pragma unroll
-                                                for (int jw = 0; jw < 4; ++jw) {
+                                                for (int jw = 0; jw < NW; ++jw) {
                                                     a0 = dp4a_us(pl[4 * jw], X[xs][mq][4 * jw], a0);
                                                     a1 = dp4a_us(pl[4 * jw + 1], X[xs][mq][4 * jw + 1], a1);
                                                     a2 = dp4a_us(pl[4 * jw + 2], X[xs][mq][4 * jw + 2], a2);

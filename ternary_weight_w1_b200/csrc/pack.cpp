@@ -1,4 +1,5 @@
-// Offline absmean ternarisation and 2-bit packing of BitLinear weights (host).
+// Offline absmean ternarisation and packing of BitLinear weights (host): the
+// 2-bit layout, and the denser base-3 layout (five codes per byte).
 //
 // Page "BitNet b1.58 2B4T Guide: Scaling Native 1-Bit LLMs", section "Ternary
 // Weight Quantization: absmean Scaling": gamma is the mean of |W| over the
@@ -91,9 +92,10 @@ extern "C" size_t bitlinear_packed_bytes(int64_t N, int64_t K)
 
 namespace {
 
-int pack_weights(const float *W_host, int64_t N, int64_t K, void *packed_host, float *gamma_out)
+// gamma = max(mean |W|, 1e-5): double accumulation in fixed blocks, added in
+// block order, then one cast.
+float absmean_gamma(const float *W_host, int64_t N, int64_t K)
 {
-    // gamma = mean |W| (double accumulation in fixed blocks, then one cast).
     const int64_t total = N * K;
     const int64_t blocks = (total + kBlock - 1) / kBlock;
     std::vector<double> partial(static_cast<size_t>(blocks), 0.0);
@@ -111,7 +113,27 @@ int pack_weights(const float *W_host, int64_t N, int64_t K, void *packed_host, f
     float gamma = static_cast<float>(sum / static_cast<double>(total));
     if (!(gamma >= kEps))
         gamma = kEps;
+    return gamma;
+}
 
+// One 2-bit-layout word: the 16 weights k0 .. k0 + 15 of row n, weight
+// k0 + 4j + b at bits 8b + 2j as the code W~ + 1; weights past the row (or
+// rows past N) are zeros (code 1).
+inline uint32_t code_word(const float *W_host, int64_t N, int64_t K, int64_t n, int64_t k0,
+                          float gamma)
+{
+    uint32_t word = 0;
+    for (int k = 0; k < 16; ++k) {
+        const uint32_t code = (n < N && k0 + k < K) ? ternary_code(W_host[n * K + k0 + k], gamma)
+                                                    : 1u;
+        word |= code << (8 * (k & 3) + 2 * (k >> 2));
+    }
+    return word;
+}
+
+int pack_weights(const float *W_host, int64_t N, int64_t K, void *packed_host, float *gamma_out)
+{
+    const float gamma = absmean_gamma(W_host, N, K);
     // Row blocks of 16 rows; inside a block, k-groups of 128 weights laid out
     // as 16 rows x 32 bytes; word w of a (row, group) holds
     // k = 128g + 16w + 4j + b at bit 8b + 2j. Rows past N are zero weights.
@@ -126,14 +148,44 @@ int pack_weights(const float *W_host, int64_t N, int64_t K, void *packed_host, f
         for (int64_t g = 0; g < groups; ++g) {
             uint8_t *dst = block + 512 * g + 32 * r;
             for (int w = 0; w < 8; ++w) {
-                uint32_t word = 0x55555555u;  // zero weights (padding rows)
-                if (n < N) {
-                    const float *src = W_host + n * K + 128 * g + 16 * w;
-                    word = 0;
-                    for (int k = 0; k < 16; ++k)
-                        word |= ternary_code(src[k], gamma) << (8 * (k & 3) + 2 * (k >> 2));
-                }
+                const uint32_t word = code_word(W_host, N, K, n, 128 * g + 16 * w, gamma);
                 std::memcpy(dst + 4 * w, &word, 4);  // little-endian host
+            }
+        }
+    });
+    *gamma_out = gamma;
+    return BITLINEAR_OK;
+}
+
+// The base-3 layout: K padded to Kp (a multiple of 160), k-groups of 160
+// weights as 16 rows x 32 bytes. A (row, group)'s codes are the ten 2-bit
+// layout words of its 160 weights read as one stream of 2-bit fields from bit
+// 0 up; byte B holds stream fields 5B .. 5B + 4 as base-3 digits 0 .. 4.
+int pack_weights_b3(const float *W_host, int64_t N, int64_t K, void *packed_host,
+                    float *gamma_out)
+{
+    const float gamma = absmean_gamma(W_host, N, K);
+    uint8_t *out = static_cast<uint8_t *>(packed_host);
+    const int64_t Kp = (K + 159) / 160 * 160;
+    const int64_t row_blocks = (N + 15) / 16;
+    const int64_t groups = Kp / 160;
+    const size_t block_bytes = 16 * static_cast<size_t>(Kp / 5);
+    parallel_for(row_blocks * 16, [&](int64_t n) {
+        const int64_t blk = n / 16;
+        const int64_t r = n % 16;
+        uint8_t *block = out + static_cast<size_t>(blk) * block_bytes;
+        for (int64_t g = 0; g < groups; ++g) {
+            uint32_t words[10];
+            for (int w = 0; w < 10; ++w)
+                words[w] = code_word(W_host, N, K, n, 160 * g + 16 * w, gamma);
+            uint8_t *dst = block + 512 * g + 32 * r;
+            for (int B = 0; B < 32; ++B) {
+                uint32_t value = 0;
+                for (int i = 4; i >= 0; --i) {            // Horner: digit 4 first
+                    const int f = 5 * B + i;
+                    value = 3 * value + ((words[f >> 4] >> (2 * (f & 15))) & 3u);
+                }
+                dst[B] = static_cast<uint8_t>(value);
             }
         }
     });
@@ -154,6 +206,31 @@ extern "C" int bitlinear_pack_weights(const float *W_host, int64_t N, int64_t K,
         return pack_weights(W_host, N, K, packed_host, gamma_out);
     } catch (...) {
         // nothing crosses the C ABI; only host allocation can fail here
+        return BITLINEAR_ERR_HOST;
+    }
+}
+
+extern "C" size_t bitlinear_packed_bytes_b3(int64_t N, int64_t K)
+{
+    if (N < 1 || K < 128 || K % 128 != 0 || K > (int64_t(1) << 40))
+        return 0;
+    const int64_t blocks = N / 16 + (N % 16 != 0 ? 1 : 0);
+    const int64_t row = (K + 159) / 160 * 32;      // bytes of one row: Kp / 5
+    if (row > INT64_MAX / 16 / blocks)             // the size would not fit in 64 bits
+        return 0;
+    return static_cast<size_t>(blocks) * 16 * static_cast<size_t>(row);
+}
+
+extern "C" int bitlinear_pack_weights_b3(const float *W_host, int64_t N, int64_t K,
+                                         void *packed_host, float *gamma_out)
+{
+    if (!W_host || !packed_host || !gamma_out || N < 1 || K < 0)
+        return BITLINEAR_ERR_ARG;
+    if (K < 128 || K % 128 != 0)
+        return BITLINEAR_ERR_SHAPE;
+    try {
+        return pack_weights_b3(W_host, N, K, packed_host, gamma_out);
+    } catch (...) {
         return BITLINEAR_ERR_HOST;
     }
 }

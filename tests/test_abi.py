@@ -327,3 +327,17 @@ def test_grouped_rmsnorm_rejects_bad_arguments():
     assert call([(FAKE, 1, 200, 64, FAKE, FAKE)], [FAKE]) == bl.BITLINEAR_ERR_SHAPE
     # an empty batch needs no gain and does nothing
     assert call([(FAKE, 0, 256, 64, FAKE, FAKE)], [None]) == bl.BITLINEAR_OK
+
+
+def test_forward_b3_rejects_bad_arguments():
+    L = bl.lib()
+
+    def call(M=1, K=256, N=64, x=FAKE, packed=FAKE, y=FAKE, xdt=0):
+        return L.bitlinear_forward_b3(x, xdt, M, K, packed, 1.0, N, y, None, None, None, None)
+    assert call(x=None) == bl.BITLINEAR_ERR_ARG
+    assert call(K=200) == bl.BITLINEAR_ERR_SHAPE
+    assert call(M=17) == bl.BITLINEAR_ERR_SHAPE                 # the GEMV path only
+    assert call(M=16, K=12288) == bl.BITLINEAR_ERR_SHAPE        # padded x~ 16 * 12320 bytes
+    assert call(xdt=3) == bl.BITLINEAR_ERR_DTYPE
+    assert call(y=FAKE + 2) == bl.BITLINEAR_ERR_ALIGN
+    assert call(M=0, x=None, y=None) == bl.BITLINEAR_OK

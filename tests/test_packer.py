@@ -71,3 +71,55 @@ def test_rejects_bad_shapes():
     assert L.bitlinear_pack_weights(None, 4, 128, out.ctypes.data, g.ctypes.data) == bl.BITLINEAR_ERR_ARG
     assert L.bitlinear_pack_weights(W.ctypes.data, 0, 128, out.ctypes.data, g.ctypes.data) == bl.BITLINEAR_ERR_ARG
     assert L.bitlinear_pack_weights(W.ctypes.data, 4, 64, out.ctypes.data, g.ctypes.data) == bl.BITLINEAR_ERR_SHAPE
+
+
+# ------------------------------------------------------------- base-3 layout
+
+def check_pack_b3(orc, W):
+    """The base-3 packer: the same gamma as the 2-bit packer, and bytes equal
+    to the oracle's base-3 layout of the oracle's ternary weights."""
+    packed, gamma = bl.bitlinear_pack_weights_b3(W)
+    _, gamma2 = bl.bitlinear_pack_weights(W)
+    assert gamma == gamma2
+    Wq = orc.ternarize(W, np.float32(gamma))
+    np.testing.assert_array_equal(packed, orc.pack_codes_b3(Wq))
+    N, K = W.shape
+    assert packed.size == bl.bitlinear_packed_bytes_b3(N, K)
+    assert packed.size == (N + 15) // 16 * 16 * ((K + 159) // 160 * 160) // 5
+    return packed, Wq
+
+
+def test_b3_golden_bytes():
+    for name, N, K, ws, by, size in pins.load_pack_cases("pack_b3_bytes.txt"):
+        W = np.zeros((N, K), dtype=np.float32)
+        for r, k, v in ws:
+            W[r, k] = v
+        packed, _ = bl.bitlinear_pack_weights_b3(W)
+        want = np.full(size, 121, dtype=np.uint8)
+        for off, val in by.items():
+            want[off] = val
+        np.testing.assert_array_equal(packed, want, err_msg=name)
+
+
+@pytest.mark.parametrize("N,K,seed", [(256, 256, 0), (7, 128, 1), (33, 1280, 2),
+                                      (640, 2560, 3), (2560, 6912, 2), (1001, 384, 4)])
+def test_b3_random_latents(orc, N, K, seed):
+    packed, Wq = check_pack_b3(orc, workloads.latent_weights(N, K, seed))
+    if N * K <= 64 * 1024:
+        np.testing.assert_array_equal(pins.decode_packed_b3_spec(packed, N, K), Wq)
+
+
+def test_b3_sizes_and_bad_shapes():
+    # 1.6 bits per weight once K is a multiple of 160
+    assert bl.bitlinear_packed_bytes_b3(16, 2560) * 5 == 16 * 2560
+    assert bl.bitlinear_packed_bytes_b3(16, 6912) == 16 * 7040 // 5
+    assert bl.bitlinear_packed_bytes_b3(0, 128) == 0
+    assert bl.bitlinear_packed_bytes_b3(4, 100) == 0
+    with pytest.raises(bl.BitLinearError):
+        bl.bitlinear_pack_weights_b3(np.zeros((2, 64), dtype=np.float32))
+    L = bl.lib()
+    g = np.zeros(1, dtype=np.float32)
+    out = np.zeros(16 * 32, dtype=np.uint8)
+    W = np.zeros((4, 128), dtype=np.float32)
+    assert L.bitlinear_pack_weights_b3(None, 4, 128, out.ctypes.data, g.ctypes.data) == bl.BITLINEAR_ERR_ARG
+    assert L.bitlinear_pack_weights_b3(W.ctypes.data, 4, 64, out.ctypes.data, g.ctypes.data) == bl.BITLINEAR_ERR_SHAPE
