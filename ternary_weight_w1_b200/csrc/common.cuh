@@ -496,10 +496,24 @@ __device__ __forceinline__ double warp_sum_f64(double v)
     return v;
 }
 
-// x~ = clamp(round_half_even(x * scale), -128, 127) as one byte.
+// rint(v) for |v| < 2^22, as the bit pattern of an fp32 sum: adding 1.5 * 2^23
+// puts v + c in [2^23, 2^24), where the spacing is 1, so the IEEE addition
+// rounds v to an integer (ties to even, as rint) and the result's bits are
+// 0x4B400000 + rint(v). Its low byte is rint(v) as a two's-complement byte. A
+// full-rate addition in place of a float-to-integer conversion.
+__device__ __forceinline__ uint32_t rint_bits(float v)
+{
+    return __float_as_uint(__fadd_rn(v, 12582912.0f));
+}
+
+// x~ = clamp(round_half_even(x * scale), -128, 127): the product rounded to
+// fp32 first, as the listing computes it, then to an integer. With scale =
+// 127 / beta and beta the absmax of the row (or 1e-5 above every |x|),
+// |x * scale| <= 127, so the clamp never binds; it is kept here for callers
+// whose scale is not that.
 __device__ __forceinline__ int quant1(float x, float scale)
 {
-    int q = __float2int_rn(__fmul_rn(x, scale));
+    const int q = static_cast<int>(rint_bits(__fmul_rn(x, scale)) - 0x4B400000u);
     return min(127, max(-128, q));
 }
 

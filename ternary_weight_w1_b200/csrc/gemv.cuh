@@ -412,10 +412,10 @@ gemv_kernel(const __grid_constant__ Params p)
                     Vec8<BF16> v;
                     v.load(row, e);
                     // |x * (127 / beta)| <= 127: the listing's clamp cannot bind
-                    int q[8];
+                    uint32_t q[8];   // rint(x * scale) in the low byte (rint_bits)
 #pragma unroll
                     for (int u = 0; u < 8; ++u)
-                        q[u] = __float2int_rn(__fmul_rn(v.get(u), scale));
+                        q[u] = rint_bits(__fmul_rn(v.get(u), scale));
                     lo = __byte_perm(__byte_perm(q[0], q[1], 0x0040),
                                      __byte_perm(q[2], q[3], 0x0040), 0x5410);
                     hi = __byte_perm(__byte_perm(q[4], q[5], 0x0040),
@@ -486,10 +486,10 @@ gemv_kernel(const __grid_constant__ Params p)
             if (valid(i)) {
                 const Vec8<true> v = staged(i);
                 // |x * (127 / beta)| <= 127: the listing's clamp cannot bind
-                int q[8];
+                uint32_t q[8];   // rint(x * scale) in the low byte (rint_bits)
 #pragma unroll
                 for (int u = 0; u < 8; ++u)
-                    q[u] = __float2int_rn(__fmul_rn(v.get(u), scale));
+                    q[u] = rint_bits(__fmul_rn(v.get(u), scale));
                 qw[i][0] = __byte_perm(__byte_perm(q[0], q[1], 0x0040),
                                        __byte_perm(q[2], q[3], 0x0040), 0x5410);
                 qw[i][1] = __byte_perm(__byte_perm(q[4], q[5], 0x0040),
@@ -652,13 +652,13 @@ gemv_kernel(const __grid_constant__ Params p)
                     // |a * (127 / beta)| <= 127 (beta is the row's absmax, or
                     // 1e-5 above every |a|), so rint never leaves [-127, 127]
                     // and the listing's clamp to [-128, 127] cannot bind
-                    int q[8];
+                    uint32_t q[8];   // rint(x * scale) in the low byte (rint_bits)
     #pragma unroll
                     for (int u = 0; u < 8; ++u) {
                         float a = v.get(u);
                         if constexpr (NORM)
                             a = norm1(a, r, g[x][u]);
-                        q[u] = __float2int_rn(__fmul_rn(a, scale[x]));
+                        q[u] = rint_bits(__fmul_rn(a, scale[x]));
                     }
                     const uint32_t lo = __byte_perm(__byte_perm(q[0], q[1], 0x0040),
                                                     __byte_perm(q[2], q[3], 0x0040), 0x5410);
