@@ -55,17 +55,23 @@ INT8_PER_BF16 = 2.0        # nominal dense int8 / bf16 tensor ratio (4.5 / 2.25 
 # kernel source it was taken on; reported only while that source is unchanged.
 TRAFFIC = {
     # grouped decode launch (up 2560->6912 + down 6912->2560, M=1): 8,847,360
-    # algorithmic bytes; profiles/gemv_grouped_decode_2b_m1.md. The capture
-    # was taken on this kernel code; the source has changed since only in
-    # comments of its parameter block.
-    "gemv": {"src": "ea1ca4c9f8d28831", "bytes_per_launch": 8895232},
+    # algorithmic bytes; dram__bytes_read.sum + dram__bytes_write.sum of one
+    # ncu capture (profiles/gemv_grouped_decode_2b_m1.md), keyed by the hash
+    # of the kernel sources it was taken on.
+    "gemv": {"src": "01571e9c5bc6abfd", "bytes_per_launch": 8902400},
 }
 
 
-def kernel_source_hash(name: str) -> str:
-    path = os.path.join(ROOT, "ternary_weight_w1_b200", "csrc", name)
-    with open(path, "rb") as f:
-        return hashlib.sha256(f.read()).hexdigest()[:16]
+GEMV_SOURCES = ("gemv.cuh", "common.cuh")
+
+
+def kernel_source_hash(*names: str) -> str:
+    """First 16 hex digits of the SHA-256 of the named csrc files, in order."""
+    h = hashlib.sha256()
+    for name in names:
+        with open(os.path.join(ROOT, "ternary_weight_w1_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
 
 
 def load_peaks():
@@ -321,10 +327,13 @@ def time_graph_steps(dist, wl, steps: int, clocks: ClockSampler | None, separate
 
 
 def time_e2e(dist, wl, steps: int):
-    """Same steps through the public Python API, with each step's tokens copied
-    from pinned host memory and its outputs read back to pinned host memory.
-    Both tokens of a step sit in one pinned buffer (one host-to-device copy)
-    and both outputs land in one device buffer (one device-to-host copy)."""
+    """Same steps through the library's host-buffer call
+    (bitlinear_forward_grouped_host): each step's tokens are copied from
+    pinned host memory, the grouped launch runs, and its outputs are copied
+    back to pinned host memory, all inside one library call per step. Both
+    tokens of a step sit in one pinned buffer and one device staging buffer
+    (one host-to-device copy); both outputs land in one device buffer and one
+    pinned buffer (one device-to-host copy)."""
     import torch
     xk = [m["p"].K for m in wl.mats]
     yn = [m["p"].N for m in wl.mats]
@@ -335,14 +344,14 @@ def time_e2e(dist, wl, steps: int):
     dev_y = torch.empty(sum(yn), dtype=torch.bfloat16, device=dev_x.device)
     xs = list(torch.split(dev_x, xk))
     ys = list(torch.split(dev_y, yn))
+    calls = [wl.bl.GroupedHostCall(
+                 [(xs[k].view(1, -1), m["packed"][j], m["gamma"], m["p"].N, ys[k].view(1, -1))
+                  for k, m in enumerate(wl.mats)])
+             for j in range(ROTATE)]
 
     def one(i):
         j = i % ROTATE
-        dev_x.copy_(host_x[j], non_blocking=True)
-        wl.bl.bitlinear_forward_grouped(
-            [(xs[k].view(1, -1), m["packed"][j], m["gamma"], m["p"].N, ys[k].view(1, -1))
-             for k, m in enumerate(wl.mats)])
-        host_y.copy_(dev_y, non_blocking=True)
+        calls[j](host_x[j], host_y)
 
     for i in range(5):
         one(i)
@@ -716,7 +725,7 @@ def run_ours(args, dist):
     achieved = per_launch_bytes / (avg_launch_ms * 1e-3) / 1e9
     traffic = None
     t = TRAFFIC.get("gemv")
-    if t is not None and t.get("src") == kernel_source_hash("gemv.cuh"):
+    if t is not None and t.get("src") == kernel_source_hash(*GEMV_SOURCES):
         traffic = t["bytes_per_launch"]
 
     e2e_steps = min(args.steps, args.e2e_steps)

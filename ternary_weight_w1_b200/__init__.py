@@ -63,6 +63,7 @@ EXPORTS = (
     "bitlinear_forward_inject_timeout",
     "bitlinear_forward_noalloc",
     "bitlinear_forward_grouped",
+    "bitlinear_forward_grouped_host",
     "bitlinear_workspace_bytes_grouped",
     "bitlinear_forward_grouped_ws",
     "bitlinear_forward_grouped_rmsnorm",
@@ -133,6 +134,8 @@ def lib() -> ctypes.CDLL:
                                                 i64, p, p]
         L.bitlinear_forward_grouped.restype = ctypes.c_int
         L.bitlinear_forward_grouped.argtypes = [p, ctypes.c_int, ctypes.c_int, p]
+        L.bitlinear_forward_grouped_host.restype = ctypes.c_int
+        L.bitlinear_forward_grouped_host.argtypes = [p, ctypes.c_int, ctypes.c_int, p, p, p]
         L.bitlinear_workspace_bytes_grouped.restype = ctypes.c_size_t
         L.bitlinear_workspace_bytes_grouped.argtypes = [p, ctypes.c_int]
         L.bitlinear_forward_grouped_ws.restype = ctypes.c_int
@@ -575,3 +578,59 @@ def bitlinear_forward_grouped(problems, stream=None, workspace=None):
                                                   workspace.numel(), _stream(stream)),
                "bitlinear_forward_grouped_ws")
     return outs
+
+
+def _host_buffer(t, name: str, dtype, numel: int) -> int:
+    if t.device.type != "cpu":
+        raise ValueError(f"{name} must be a host tensor (got device {t.device})")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if t.numel() != numel:
+        raise ValueError(f"{name} holds {t.numel()} elements, {numel} expected")
+    return t.data_ptr()
+
+
+class GroupedHostCall:
+    """bitlinear_forward_grouped_host with its problem list checked and
+    marshalled once. ``problems`` is a list of (x_dev, packed, gamma, N,
+    y_dev): the device staging buffers for the tokens and outputs (allocated
+    back to back, one copy serves all of them), the packed weights and gamma.
+    Each call takes a host tensor of every problem's tokens in problem order
+    (sum of M*K elements of x's dtype) and a host bf16 tensor for every
+    problem's outputs (sum of M*N elements), and makes one library call:
+    copy in, grouped launch, copy out, enqueued on ``stream`` (the current
+    stream when None). Pinned host tensors keep the copies asynchronous;
+    ``y_host`` holds the results once the stream has synchronised."""
+
+    __slots__ = ("_arr", "_count", "_xdt", "_x_dtype", "_x_numel", "_y_numel", "_stream")
+
+    def __init__(self, problems, stream=None):
+        if not problems:
+            raise ValueError("at least one problem")
+        if any(pr[4] is None for pr in problems):
+            raise ValueError("every problem needs its device output buffer y_dev")
+        self._xdt = _xdt(problems[0][0])
+        self._x_dtype = problems[0][0].dtype
+        self._arr, _ = _problem_array(problems, alloc_y=True, a=_Args())
+        self._count = len(problems)
+        self._x_numel = sum(pr[0].numel() for pr in problems)
+        self._y_numel = sum(pr[0].shape[0] * pr[3] for pr in problems)
+        self._stream = _stream(stream)
+
+    def __call__(self, x_host, y_host):
+        import torch
+        _check(lib().bitlinear_forward_grouped_host(
+                   ctypes.addressof(self._arr), self._count, self._xdt,
+                   _host_buffer(x_host, "x_host", self._x_dtype, self._x_numel),
+                   _host_buffer(y_host, "y_host", torch.bfloat16, self._y_numel), self._stream),
+               "bitlinear_forward_grouped_host")
+        return y_host
+
+
+def bitlinear_forward_grouped_host(problems, x_host, y_host, stream=None):
+    """One grouped decode call with host tokens and outputs (see
+    GroupedHostCall, which prepares the problem list once for repeated
+    calls). Returns ``y_host``, valid after the stream synchronises."""
+    return GroupedHostCall(problems, stream)(x_host, y_host)

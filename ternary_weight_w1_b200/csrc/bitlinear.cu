@@ -1056,13 +1056,16 @@ extern "C" int bitlinear_forward_b3(const void *x_dev, bitlinear_dtype xdt, int6
     return launch_gemv(&job, 1, xdt, *dev, static_cast<cudaStream_t>(cuda_stream));
 }
 
-extern "C" int bitlinear_forward_grouped(const bitlinear_problem *problems, int count,
-                                         bitlinear_dtype xdt, void *cuda_stream)
+namespace {
+
+// Checks a problem list for the one-launch grouped GEMV and collects its
+// non-empty problems into jobs[0 .. *n).
+int collect_gemv_group(const bitlinear_problem *problems, int count, bitlinear_dtype xdt,
+                       GemvJob *jobs, int *n)
 {
     if (problems == nullptr || count < 1 || count > gemv::MAX_PROBLEMS)
         return BITLINEAR_ERR_ARG;
-    GemvJob jobs[gemv::MAX_PROBLEMS];
-    int n = 0;
+    *n = 0;
     int64_t max_M = 0, max_xq = 0;
     for (int i = 0; i < count; ++i) {
         const bitlinear_problem &pr = problems[i];
@@ -1076,20 +1079,97 @@ extern "C" int bitlinear_forward_grouped(const bitlinear_problem *problems, int 
             return BITLINEAR_ERR_SHAPE;
         max_M = std::max(max_M, pr.M);
         max_xq = std::max(max_xq, pr.M * pr.K);
-        jobs[n++] = GemvJob{pr.x_dev,      static_cast<int>(pr.M), static_cast<int>(pr.K),
-                            static_cast<int>(pr.N), pr.packed_dev, pr.gamma, pr.y_dev,
-                            nullptr, nullptr, nullptr, nullptr, 0.0f};
+        jobs[(*n)++] = GemvJob{pr.x_dev,      static_cast<int>(pr.M), static_cast<int>(pr.K),
+                               static_cast<int>(pr.N), pr.packed_dev, pr.gamma, pr.y_dev,
+                               nullptr, nullptr, nullptr, nullptr, 0.0f};
     }
-    if (n == 0)
-        return BITLINEAR_OK;
     // one launch holds the largest x~ next to the largest problem's token tile
-    if (max_xq > gemv_max_xq(max_M))
+    if (*n > 0 && max_xq > gemv_max_xq(max_M))
         return BITLINEAR_ERR_SHAPE;
+    return BITLINEAR_OK;
+}
+
+// Copies `count` pieces of sizes[i] bytes between one packed host buffer and
+// the device pointers dev[i], merging pieces that lie back to back on the
+// device into one copy.
+int copy_pieces(const void *const *dev, const size_t *sizes, int count, char *host,
+                cudaMemcpyKind kind, cudaStream_t st)
+{
+    int i = 0;
+    while (i < count) {
+        char *start = static_cast<char *>(const_cast<void *>(dev[i]));
+        size_t bytes = sizes[i];
+        int j = i + 1;
+        while (j < count && static_cast<const char *>(dev[j]) == start + bytes) {
+            bytes += sizes[j];
+            ++j;
+        }
+        if (bytes > 0) {
+            cudaError_t e = kind == cudaMemcpyHostToDevice
+                                ? cudaMemcpyAsync(start, host, bytes, kind, st)
+                                : cudaMemcpyAsync(host, start, bytes, kind, st);
+            if (e != cudaSuccess)
+                return BITLINEAR_ERR_CUDA;
+        }
+        host += bytes;
+        i = j;
+    }
+    return BITLINEAR_OK;
+}
+
+}  // namespace
+
+extern "C" int bitlinear_forward_grouped(const bitlinear_problem *problems, int count,
+                                         bitlinear_dtype xdt, void *cuda_stream)
+{
+    GemvJob jobs[gemv::MAX_PROBLEMS];
+    int n = 0;
+    int rc = collect_gemv_group(problems, count, xdt, jobs, &n);
+    if (rc != BITLINEAR_OK || n == 0)
+        return rc;
     DeviceInfo *dev = nullptr;
-    int rc = current_device(&dev);
+    rc = current_device(&dev);
     if (rc != BITLINEAR_OK)
         return rc;
     return launch_gemv(jobs, n, xdt, *dev, static_cast<cudaStream_t>(cuda_stream));
+}
+
+extern "C" int bitlinear_forward_grouped_host(const bitlinear_problem *problems, int count,
+                                              bitlinear_dtype xdt, const void *x_host,
+                                              void *y_host, void *cuda_stream)
+{
+    GemvJob jobs[gemv::MAX_PROBLEMS];
+    int n = 0;
+    int rc = collect_gemv_group(problems, count, xdt, jobs, &n);
+    if (rc != BITLINEAR_OK)
+        return rc;
+    if (x_host == nullptr || y_host == nullptr)
+        return BITLINEAR_ERR_ARG;
+    if (n == 0)
+        return BITLINEAR_OK;
+    DeviceInfo *dev = nullptr;
+    rc = current_device(&dev);
+    if (rc != BITLINEAR_OK)
+        return rc;
+    const size_t xsize = xdt == BITLINEAR_BF16 ? 2 : 4;
+    const void *xd[gemv::MAX_PROBLEMS];
+    const void *yd[gemv::MAX_PROBLEMS];
+    size_t xb[gemv::MAX_PROBLEMS], yb[gemv::MAX_PROBLEMS];
+    for (int i = 0; i < n; ++i) {
+        xd[i] = jobs[i].x;
+        xb[i] = size_t(jobs[i].M) * jobs[i].K * xsize;
+        yd[i] = jobs[i].y;
+        yb[i] = size_t(jobs[i].M) * jobs[i].N * 2;
+    }
+    cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
+    rc = copy_pieces(xd, xb, n, static_cast<char *>(const_cast<void *>(x_host)),
+                     cudaMemcpyHostToDevice, st);
+    if (rc != BITLINEAR_OK)
+        return rc;
+    rc = launch_gemv(jobs, n, xdt, *dev, st);
+    if (rc != BITLINEAR_OK)
+        return rc;
+    return copy_pieces(yd, yb, n, static_cast<char *>(y_host), cudaMemcpyDeviceToHost, st);
 }
 
 namespace {

@@ -206,6 +206,50 @@ def test_grouped_rejects_bad_arguments():
     assert grouped([(None, 0, 256, 64, None, None)]) == bl.BITLINEAR_OK   # only empty problems
 
 
+def grouped_host(problems, xdt=0, x_host=FAKE, y_host=FAKE):
+    arr = (bl._Problem * max(1, len(problems)))()
+    for i, (x, M, K, N, packed, y) in enumerate(problems):
+        arr[i] = bl._Problem(x, M, K, N, packed, 1.0, y)
+    return bl.lib().bitlinear_forward_grouped_host(ctypes.addressof(arr), len(problems), xdt,
+                                                   x_host, y_host, None)
+
+
+def test_grouped_host_rejects_bad_arguments():
+    """The host-buffer call checks what bitlinear_forward_grouped checks, and
+    its host buffers, before any copy or launch."""
+    good = (FAKE, 1, 256, 64, FAKE, FAKE)
+    assert bl.lib().bitlinear_forward_grouped_host(None, 1, 0, FAKE, FAKE, None) == \
+        bl.BITLINEAR_ERR_ARG
+    assert grouped_host([]) == bl.BITLINEAR_ERR_ARG
+    assert grouped_host([good] * 9) == bl.BITLINEAR_ERR_ARG
+    assert grouped_host([good, (FAKE, 17, 256, 64, FAKE, FAKE)]) == bl.BITLINEAR_ERR_SHAPE
+    assert grouped_host([good, (FAKE + 8, 1, 256, 64, FAKE, FAKE)]) == bl.BITLINEAR_ERR_ALIGN
+    assert grouped_host([good], xdt=5) == bl.BITLINEAR_ERR_DTYPE
+    assert grouped_host([good], x_host=None) == bl.BITLINEAR_ERR_ARG
+    assert grouped_host([good], y_host=None) == bl.BITLINEAR_ERR_ARG
+    assert grouped_host([(None, 0, 256, 64, None, None)]) == bl.BITLINEAR_OK   # nothing to do
+
+
+def test_grouped_host_call_refuses_device_or_wrong_host_buffers():
+    """The prepared binding checks the host tensors' place, dtype and size
+    before its library call (no GPU needed: the problem list is built from
+    shapes alone and never reaches the library here)."""
+    import torch
+    x = torch.zeros(256, dtype=torch.bfloat16)
+    y = torch.zeros(64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="elements"):
+        bl._host_buffer(torch.zeros(255, dtype=torch.bfloat16), "x_host", torch.bfloat16, 256)
+    with pytest.raises(TypeError, match="must be"):
+        bl._host_buffer(torch.zeros(256, dtype=torch.float32), "x_host", torch.bfloat16, 256)
+    with pytest.raises(ValueError, match="contiguous"):
+        bl._host_buffer(torch.zeros(512, dtype=torch.bfloat16)[::2], "x_host", torch.bfloat16,
+                        256)
+    assert bl._host_buffer(x, "x_host", torch.bfloat16, 256) == x.data_ptr()
+    assert bl._host_buffer(y, "y_host", torch.bfloat16, 64) == y.data_ptr()
+    with pytest.raises(ValueError, match="y_dev"):
+        bl.GroupedHostCall([(x.view(1, -1), None, 1.0, 64, None)])
+
+
 def grouped_ws(problems, xdt=0, ws=FAKE, ws_bytes=1 << 30):
     arr = (bl._Problem * max(1, len(problems)))()
     for i, (x, M, K, N, packed, y) in enumerate(problems):

@@ -162,3 +162,53 @@ def test_grouped_rmsnorm_layer_matches_oracle(B):
                                      torch.from_numpy(g).cuda(), y=single)
         torch.cuda.synchronize()
         assert check_y(y, tensor_to_bf16_bits(single)) >= 0.99
+
+
+# ------------------------------------------- host buffers in and out
+
+def _host_call_check(cases, contiguous, pinned, rounds=1):
+    """Runs bitlinear_forward_grouped_host on the cases' tokens (host memory,
+    problem after problem) and compares the host outputs with the oracle bit
+    for bit; the device staging buffers lie back to back (one copy each way)
+    or in separate allocations (one copy per problem)."""
+    import torch
+    dt = torch.bfloat16 if cases[0].x_dtype == "bf16" else torch.float32
+    xk = [c.M * c.K for c in cases]
+    yn = [c.M * c.N for c in cases]
+    if contiguous:
+        xs = [t.view(c.M, c.K) for t, c in zip(torch.split(torch.empty(sum(xk), dtype=dt,
+                                                                      device="cuda"), xk), cases)]
+        ys = [t.view(c.M, c.N) for t, c in
+              zip(torch.split(torch.empty(sum(yn), dtype=torch.bfloat16, device="cuda"), yn),
+                  cases)]
+    else:
+        xs = [torch.empty((c.M, c.K), dtype=dt, device="cuda") for c in cases]
+        ys = [torch.empty((c.M, c.N), dtype=torch.bfloat16, device="cuda") for c in cases]
+    call = bl.GroupedHostCall([(x, c.packed_tensor(), c.gamma, c.N, y)
+                               for x, c, y in zip(xs, cases, ys)])
+    host_x = torch.cat([c.x_tensor().reshape(-1).cpu() for c in cases])
+    host_y = torch.full((sum(yn),), CANARY_Y, dtype=torch.int16).view(torch.bfloat16)
+    if pinned:
+        host_x, host_y = host_x.pin_memory(), host_y.pin_memory()
+    for _ in range(rounds):
+        call(host_x, host_y)
+        torch.cuda.synchronize()
+    got = host_y.view(torch.int16).numpy().view(np.uint16)
+    assert not np.any(got == CANARY_Y), "an output element was not written"
+    off = 0
+    for c, n in zip(cases, yn):
+        assert check_y(got[off:off + n].reshape(c.M, c.N), c.oracle_full()[1]) == 1.0
+        off += n
+    assert bl.bitlinear_get_fault() == (bl.BITLINEAR_OK, 0)
+
+
+def test_grouped_host_decode_step_2b_pinned():
+    cases = [Case(p.M, p.K, p.N, w_seed=p.w_seed, x_seed=p.x_seed)
+             for p in workloads.decode_gemv_2b(1).problems]
+    _host_call_check(cases, contiguous=True, pinned=True, rounds=3)
+
+
+def test_grouped_host_mixed_fp32_separate_buffers_pageable():
+    cases = [Case(1 + i % 3, 256 * (1 + i % 3), 80 + 48 * i, w_seed=60 + i, x_seed=70 + i,
+                  x_dtype="fp32") for i in range(5)]
+    _host_call_check(cases, contiguous=False, pinned=False)
