@@ -90,8 +90,9 @@ def _declare(lib):
 
 def build_omp() -> str:
     """The same C source compiled with -fopenmp (integer products over all
-    cores). Only the benchmark's CPU baseline uses it; the tests check that it
-    gives the single-threaded build's results."""
+    cores). The benchmark's all-core CPU baseline and the full-size parity
+    tests use it; the CPU tests check that it gives the single-threaded
+    build's results."""
     return build(_SRC, _OMP_LIB_PATH, extra_flags=("-fopenmp",))
 
 

@@ -602,9 +602,12 @@ class GroupedHostCall:
     problem's outputs (sum of M*N elements), and makes one library call:
     copy in, grouped launch, copy out, enqueued on ``stream`` (the current
     stream when None). Pinned host tensors keep the copies asynchronous;
-    ``y_host`` holds the results once the stream has synchronised."""
+    ``y_host`` holds the results once the stream has synchronised. The
+    object holds references to the problems' tensors, so their memory stays
+    theirs for as long as the prepared call exists."""
 
-    __slots__ = ("_arr", "_count", "_xdt", "_x_dtype", "_x_numel", "_y_numel", "_stream")
+    __slots__ = ("_arr", "_count", "_xdt", "_x_dtype", "_x_numel", "_y_numel", "_stream",
+                 "_tensors")
 
     def __init__(self, problems, stream=None):
         if not problems:
@@ -614,6 +617,7 @@ class GroupedHostCall:
         self._xdt = _xdt(problems[0][0])
         self._x_dtype = problems[0][0].dtype
         self._arr, _ = _problem_array(problems, alloc_y=True, a=_Args())
+        self._tensors = [(pr[0], pr[1], pr[4]) for pr in problems]
         self._count = len(problems)
         self._x_numel = sum(pr[0].numel() for pr in problems)
         self._y_numel = sum(pr[0].shape[0] * pr[3] for pr in problems)

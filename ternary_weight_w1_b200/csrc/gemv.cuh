@@ -291,6 +291,10 @@ gemv_kernel(const __grid_constant__ Params p)
         }
     }
     __syncthreads();
+    // The next kernel in the stream may start launching at once: its CTAs
+    // take the SMs' free slots and start their weight streams while this
+    // launch runs (they wait for it to complete before reading its outputs).
+    pdl_launch_dependents();
 
     if (warp == CWARPS) {
         // ---------------------------------------------------- weight producer
@@ -681,10 +685,6 @@ gemv_kernel(const __grid_constant__ Params p)
     }
     // this warp's lanes read the groups its lanes just wrote
     __syncwarp();
-
-    // The next kernel in the stream may start launching now: its weight
-    // stream overlaps this main loop and epilogue.
-    pdl_launch_dependents();
 
     const int r = lane >> 1;          // row in the block
     const int t = lane & 1;           // k-half (64 weights) of the group

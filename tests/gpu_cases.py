@@ -134,8 +134,11 @@ class Case:
 
     # ---------------------------------------------------------- checks
 
-    def oracle_full(self):
-        acc = self.orc.matmul_i32(self.xq, self.Wq)
+    def oracle_full(self, orc=None):
+        """acc and y of the whole problem; ``orc`` may name another copy of
+        the oracle for the integer products (the OpenMP build, whose results
+        equal the single-threaded build's, for the full-size cases)."""
+        acc = (orc or self.orc).matmul_i32(self.xq, self.Wq)
         y = self.orc.rescale_bf16(acc, self.beta, np.float32(self.gamma))
         return acc, y
 
@@ -143,9 +146,9 @@ class Case:
         np.testing.assert_array_equal(got["beta"], self.beta)
         np.testing.assert_array_equal(got["xq"], self.xq)
 
-    def check_full(self, got):
+    def check_full(self, got, orc=None):
         self.check_quant(got)
-        acc, y = self.oracle_full()
+        acc, y = self.oracle_full(orc)
         np.testing.assert_array_equal(got["acc"], acc)
         return check_y(got["y"], y)
 
