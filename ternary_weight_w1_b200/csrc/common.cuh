@@ -297,6 +297,22 @@ __device__ __forceinline__ void umma_i8_tmem_a(uint32_t d_tmem, uint32_t a_tmem,
         : "memory");
 }
 
+// umma_i8_tmem_a with the B descriptor given as its two 32-bit words, so that
+// an issuing loop can step the start address (the low word's bits 0-13, in
+// 16-byte units) with one 32-bit add per MMA.
+__device__ __forceinline__ void umma_i8_tmem_a_w(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_lo,
+                                                 uint32_t b_hi, uint32_t idesc,
+                                                 uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t.reg .b64 bd;\n\t"
+        "setp.ne.b32 p, %5, 0;\n\t"
+        "mov.b64 bd, {%2, %3};\n\t"
+        "tcgen05.mma.cta_group::1.kind::i8 [%0], [%1], bd, %4, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "r"(b_lo), "r"(b_hi), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
 // Arrive (once) on an mbarrier when all previously issued tcgen05.mma of
 // this thread have completed.
 __device__ __forceinline__ void umma_commit(uint32_t bar)

@@ -280,6 +280,15 @@ gemm_ws_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Params
         if (lane == 0) {
             int s = 0, a = 0, seg = 0;
             uint32_t aph = 0;
+            // The x~ descriptors of every stage and k-step differ from stage
+            // 0's first one only in the start address (low word, 16-byte
+            // units, no carry: shared addresses stay below 2^18), so the
+            // issuing loop adds constants instead of rebuilding 64-bit
+            // descriptors: a lone thread has no other work to hide the
+            // latency of that arithmetic behind.
+            const uint64_t bdesc0 = smem_desc_k128_sw128(sX);
+            const uint32_t b_lo0 = static_cast<uint32_t>(bdesc0);
+            const uint32_t b_hi = static_cast<uint32_t>(bdesc0 >> 32);
             if (p.inject_timeout) {
                 mbar_wait_bounded(never_bar, 0u, abort_flag, limit);
                 goto mma_done;
@@ -307,12 +316,15 @@ gemm_ws_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Params
                         goto mma_done;
                     tc_fence_after_sync();
                     const uint32_t a_tmem = tmem_base + static_cast<uint32_t>(C::A_COL0 + 64 * a);
+                    const uint32_t b_lo = b_lo0 + static_cast<uint32_t>(s * (C::X_BYTES >> 4));
+                    const uint32_t first = kb > k0 ? 1u : 0u;
 #pragma unroll
                     for (int kk = 0; kk < BK / UMMA_K; ++kk) {
-                        const uint64_t bdesc = smem_desc_k128_sw128(
-                            sX + s * C::X_BYTES + (kk / 4) * C::X_SUB + (kk % 4) * UMMA_K);
-                        umma_i8_tmem_a(d_tmem, a_tmem + static_cast<uint32_t>(8 * kk), bdesc,
-                                       C::IDESC, (kb > k0 || kk > 0) ? 1u : 0u);
+                        constexpr int X_SUB16 = C::X_SUB >> 4;
+                        umma_i8_tmem_a_w(d_tmem, a_tmem + static_cast<uint32_t>(8 * kk),
+                                         b_lo + static_cast<uint32_t>((kk / 4) * X_SUB16 +
+                                                                      (kk % 4) * (UMMA_K >> 4)),
+                                         b_hi, C::IDESC, kk > 0 ? 1u : first);
                     }
                     umma_commit(empty_load(s));
                     umma_commit(a_empty(a));
