@@ -365,19 +365,25 @@ int bitlinear_forward_grouped(const bitlinear_problem *problems, int count,
                               bitlinear_dtype xdt, void *cuda_stream);
 
 /* bitlinear_forward_grouped with the tokens taken from, and the outputs
- * returned to, host memory: on cuda_stream it copies every problem's tokens
- * from x_host into the problem's x_dev, makes the grouped launch, and copies
- * every problem's y_dev back into y_host. This is the one call a decode step
- * makes when its tokens arrive from the host and its outputs leave for it.
+ * returned to, host memory, all on cuda_stream. This is the one call a
+ * decode step makes when its tokens arrive from the host and its outputs
+ * leave for it.
  *   problems, count, xdt [in] as for bitlinear_forward_grouped; x_dev and
  *                  y_dev are the device staging buffers (caller-owned)
  *   x_host [in]  problem 0's M*K tokens (xdt elements, row-major), then
  *                problem 1's, and so on: sum of M*K elements
  *   y_host [out] problem 0's M*N bf16 outputs, then problem 1's, and so on
- * Problems whose x_dev (y_dev) buffers lie back to back in problem order
- * share one copy. The call returns once the work is enqueued; y_host holds
- * the results after the stream synchronises. With pinned host buffers the
- * copies are asynchronous; with pageable ones CUDA makes them synchronous.
+ * Tokens: when x_host is pinned memory mapped into the device's address
+ * space (as cudaHostAlloc / cudaMallocHost memory is under unified
+ * addressing), a small kernel reads it and writes every problem's x_dev;
+ * otherwise cudaMemcpyAsync copies them (one copy for problems whose x_dev
+ * buffers lie back to back). Outputs: when y_host is such memory and every
+ * problem's part of it is 16-byte aligned, the GEMV writes the outputs
+ * straight into y_host and y_dev is not written; otherwise the outputs go
+ * to y_dev and cudaMemcpyAsync copies them back. The call returns once the
+ * work is enqueued; y_host holds the results after the stream synchronises,
+ * and x_host must keep this call's tokens until then. With pageable host
+ * buffers CUDA makes the copies synchronous.
  * Errors: those of bitlinear_forward_grouped, reported before any copy or
  * launch; BITLINEAR_ERR_ARG for a NULL host buffer; BITLINEAR_ERR_CUDA when
  * a copy or the launch cannot be enqueued (earlier parts may be enqueued). */

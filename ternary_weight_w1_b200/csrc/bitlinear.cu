@@ -22,6 +22,7 @@
 #include "gemm_ws.cuh"
 #include "gemv.cuh"
 #include "quant_act.cuh"
+#include "stage_io.cuh"
 
 using namespace bitlinear;
 
@@ -1134,6 +1135,18 @@ extern "C" int bitlinear_forward_grouped(const bitlinear_problem *problems, int 
     return launch_gemv(jobs, n, xdt, *dev, static_cast<cudaStream_t>(cuda_stream));
 }
 
+// The device address of host memory the device can read and write (pinned
+// and mapped into its address space), or null for any other pointer.
+void *mapped_device_ptr(const void *host)
+{
+    cudaPointerAttributes a = {};
+    if (cudaPointerGetAttributes(&a, host) != cudaSuccess) {
+        cudaGetLastError();                       // not a pointer CUDA knows: clear it
+        return nullptr;
+    }
+    return a.type == cudaMemoryTypeHost ? a.devicePointer : nullptr;
+}
+
 extern "C" int bitlinear_forward_grouped_host(const bitlinear_problem *problems, int count,
                                               bitlinear_dtype xdt, const void *x_host,
                                               void *y_host, void *cuda_stream)
@@ -1155,19 +1168,58 @@ extern "C" int bitlinear_forward_grouped_host(const bitlinear_problem *problems,
     const void *xd[gemv::MAX_PROBLEMS];
     const void *yd[gemv::MAX_PROBLEMS];
     size_t xb[gemv::MAX_PROBLEMS], yb[gemv::MAX_PROBLEMS];
+    size_t x_total = 0;
     for (int i = 0; i < n; ++i) {
         xd[i] = jobs[i].x;
-        xb[i] = size_t(jobs[i].M) * jobs[i].K * xsize;
+        xb[i] = size_t(jobs[i].M) * jobs[i].K * xsize;     // a multiple of 256 (K % 128 == 0)
         yd[i] = jobs[i].y;
         yb[i] = size_t(jobs[i].M) * jobs[i].N * 2;
+        x_total += xb[i];
     }
     cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
-    rc = copy_pieces(xd, xb, n, static_cast<char *>(const_cast<void *>(x_host)),
-                     cudaMemcpyHostToDevice, st);
-    if (rc != BITLINEAR_OK)
-        return rc;
+
+    // Tokens: host memory the device can read is staged by a kernel (no
+    // copy-engine transfer); any other host memory by cudaMemcpyAsync.
+    const void *x_map = mapped_device_ptr(x_host);
+    if (x_map != nullptr && aligned(x_map, 16) && x_total / 16 <= INT_MAX) {
+        stage::Pieces pc = {};
+        pc.src = static_cast<const uint4 *>(x_map);
+        pc.count = n;
+        size_t end = 0;
+        for (int i = 0; i < n; ++i) {
+            pc.dst[i] = static_cast<uint4 *>(const_cast<void *>(xd[i]));
+            end += xb[i] / 16;
+            pc.end[i] = static_cast<int>(end);
+        }
+        const int vecs = static_cast<int>(end);
+        const int per_cta = stage::THREADS * stage::PER_THREAD;
+        const int grid = std::max(1, std::min((vecs + per_cta - 1) / per_cta, dev->sms));
+        if (launch(stage::stage_tokens_kernel, dim3(grid), dim3(stage::THREADS), 0, st, pc) !=
+            cudaSuccess)
+            return BITLINEAR_ERR_CUDA;
+    } else {
+        rc = copy_pieces(xd, xb, n, static_cast<char *>(const_cast<void *>(x_host)),
+                         cudaMemcpyHostToDevice, st);
+        if (rc != BITLINEAR_OK)
+            return rc;
+    }
+
+    // Outputs: into host memory the device can write, straight from the GEMV's
+    // epilogue when every problem's part of it is 16-byte aligned (y_dev is
+    // then not written); otherwise into y_dev and back by cudaMemcpyAsync.
+    char *y_map = static_cast<char *>(mapped_device_ptr(y_host));
+    bool direct = y_map != nullptr;
+    for (size_t off = 0, i = 0; direct && i < static_cast<size_t>(n); off += yb[i], ++i)
+        direct = aligned(y_map + off, 16);
+    if (direct) {
+        size_t off = 0;
+        for (int i = 0; i < n; ++i) {
+            jobs[i].y = y_map + off;
+            off += yb[i];
+        }
+    }
     rc = launch_gemv(jobs, n, xdt, *dev, st);
-    if (rc != BITLINEAR_OK)
+    if (rc != BITLINEAR_OK || direct)
         return rc;
     return copy_pieces(yd, yb, n, static_cast<char *>(y_host), cudaMemcpyDeviceToHost, st);
 }

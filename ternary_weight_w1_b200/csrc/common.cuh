@@ -164,6 +164,54 @@ __device__ __forceinline__ bool warp_wait_bounded(uint32_t bar, uint32_t parity,
     return ok != 0;
 }
 
+__device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity)
+{
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return done != 0;
+}
+
+// Waits for the given phases of two barriers at once: every lane of the warp
+// polls both (non-blocking tests), and the warp leaves together when all
+// lanes have seen both complete, so the two waits overlap instead of running
+// one after the other. Bounded like mbar_wait_bounded (lane 0 keeps the time
+// and the abort flag; the verdict is shared).
+__device__ __forceinline__ bool warp_wait2_bounded(uint32_t bar1, uint32_t parity1, uint32_t bar2,
+                                                   uint32_t parity2, volatile int *abort,
+                                                   uint64_t limit_ns)
+{
+    bool d1 = false, d2 = false;
+    uint64_t t0 = 0;
+    for (uint32_t spin = 0;; ++spin) {
+        d1 = d1 || mbar_test_wait(bar1, parity1);
+        d2 = d2 || mbar_test_wait(bar2, parity2);
+        if (__all_sync(0xffffffffu, d1 && d2))
+            return true;
+        if ((spin & 63u) == 0u) {
+            int stop = 0;
+            if ((threadIdx.x & 31) == 0) {
+                if (spin == 0) {
+                    t0 = global_timer_ns();
+                } else if (*abort) {
+                    stop = 1;
+                } else if (global_timer_ns() - t0 > limit_ns) {
+                    atomicOr(&g_fault_word, FAULT_WAIT_TIMEOUT);
+                    *abort = 1;
+                    stop = 1;
+                }
+            }
+            if (__shfl_sync(0xffffffffu, stop, 0))
+                return false;
+        }
+    }
+}
+
 // Bounded wait that ignores the abort flag: used only to drain this thread's
 // own asynchronous work (copies, MMAs) before the block exits.
 __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, uint64_t limit_ns)

@@ -354,9 +354,8 @@ gemm_ws_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Params
         int s = 0, a = 0;
         uint32_t ph = 0, aph = 0;
         for (int it = it_begin; it < it_end; ++it) {
-            if (!warp_wait_bounded(full_load(s), ph, abort_flag, limit))
-                break;
-            if (!warp_wait_bounded(a_empty(a), aph ^ 1u, abort_flag, limit))
+            // the stage's copies have landed and its TMEM slot is free
+            if (!warp_wait2_bounded(full_load(s), ph, a_empty(a), aph ^ 1u, abort_flag, limit))
                 break;
             tc_fence_after_sync();
             const uint8_t *stage = base_ptr + (sP - base) + s * PK_BYTES + row_off;

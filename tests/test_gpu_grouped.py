@@ -166,11 +166,15 @@ def test_grouped_rmsnorm_layer_matches_oracle(B):
 
 # ------------------------------------------- host buffers in and out
 
-def _host_call_check(cases, contiguous, pinned, rounds=1):
+def _host_call_check(cases, contiguous, pinned, rounds=1, pinned_y=None):
     """Runs bitlinear_forward_grouped_host on the cases' tokens (host memory,
     problem after problem) and compares the host outputs with the oracle bit
     for bit; the device staging buffers lie back to back (one copy each way)
-    or in separate allocations (one copy per problem)."""
+    or in separate allocations (one copy per problem). Pinned host memory
+    takes the kernel-staged tokens and the direct output path (when every
+    problem's output part is 16-byte aligned), pageable memory the copies."""
+    if pinned_y is None:
+        pinned_y = pinned
     import torch
     dt = torch.bfloat16 if cases[0].x_dtype == "bf16" else torch.float32
     xk = [c.M * c.K for c in cases]
@@ -189,7 +193,9 @@ def _host_call_check(cases, contiguous, pinned, rounds=1):
     host_x = torch.cat([c.x_tensor().reshape(-1).cpu() for c in cases])
     host_y = torch.full((sum(yn),), CANARY_Y, dtype=torch.int16).view(torch.bfloat16)
     if pinned:
-        host_x, host_y = host_x.pin_memory(), host_y.pin_memory()
+        host_x = host_x.pin_memory()
+    if pinned_y:
+        host_y = host_y.pin_memory()
     for _ in range(rounds):
         call(host_x, host_y)
         torch.cuda.synchronize()
@@ -212,3 +218,16 @@ def test_grouped_host_mixed_fp32_separate_buffers_pageable():
     cases = [Case(1 + i % 3, 256 * (1 + i % 3), 80 + 48 * i, w_seed=60 + i, x_seed=70 + i,
                   x_dtype="fp32") for i in range(5)]
     _host_call_check(cases, contiguous=False, pinned=False)
+
+
+def test_grouped_host_pinned_tokens_pageable_outputs():
+    cases = [Case(p.M, p.K, p.N, w_seed=p.w_seed, x_seed=p.x_seed)
+             for p in workloads.decode_gemv_2b(1).problems]
+    _host_call_check(cases, contiguous=True, pinned=True, pinned_y=False, rounds=2)
+
+
+def test_grouped_host_pinned_unaligned_output_parts():
+    """N = 17 and 40: the second problem's outputs start 34 bytes into y_host,
+    so the outputs go through the device buffers and a copy back."""
+    cases = [Case(1, 512, 17, w_seed=81, x_seed=91), Case(2, 384, 40, w_seed=82, x_seed=92)]
+    _host_call_check(cases, contiguous=False, pinned=True, rounds=2)
