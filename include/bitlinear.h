@@ -33,6 +33,8 @@
  *     16-byte aligned, fp32/int32 outputs 4-byte aligned.
  *   - Shapes: K must be a positive multiple of 128 for the device calls;
  *     M >= 0 (M = 0 is a no-op), N >= 1, K <= 65536 for the forward calls.
+ *   - Values: activations are finite; a token holding a NaN has unspecified
+ *     outputs (an infinity makes beta infinite, as in the page's listing).
  */
 #ifndef BITLINEAR_H
 #define BITLINEAR_H

@@ -575,6 +575,14 @@ __device__ __forceinline__ uint32_t rint_bits(float v)
 // 127 / beta and beta the absmax of the row (or 1e-5 above every |x|),
 // |x * scale| <= 127, so the clamp never binds; it is kept here for callers
 // whose scale is not that.
+// Lane-wise unsigned maximum of two pairs of 16-bit fields.
+__device__ __forceinline__ uint32_t max_u16x2(uint32_t a, uint32_t b)
+{
+    uint32_t d;
+    asm("max.u16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+
 __device__ __forceinline__ int quant1(float x, float scale)
 {
     const int q = static_cast<int>(rint_bits(__fmul_rn(x, scale)) - 0x4B400000u);

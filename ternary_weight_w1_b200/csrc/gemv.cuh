@@ -606,18 +606,31 @@ gemv_kernel(const __grid_constant__ Params p)
     #pragma unroll
             for (int x = 0; x < NX; ++x)
                 amax[x] = 0.0f;
-            for_slots(m, !NORM, true, [&](int, const Vec8<BF16> &v, const Gains &g) {
+            if constexpr (BF16 && !NORM) {
+                // |x| of a finite bf16 orders like its bit pattern with the
+                // sign cleared: the maximum of those 15-bit fields, two per
+                // word, is the absmax (widened exactly at the end)
+                uint32_t mb = 0;
+                for_slots(m, true, false, [&](int, const Vec8<BF16> &v, const Gains &) {
     #pragma unroll
-                for (int x = 0; x < NX; ++x) {
+                    for (int j = 0; j < 4; ++j)
+                        mb = max_u16x2(mb, v.w[j] & 0x7fff7fffu);
+                });
+                amax[0] = __uint_as_float(max(mb & 0xffffu, mb >> 16) << 16);
+            } else {
+                for_slots(m, !NORM, true, [&](int, const Vec8<BF16> &v, const Gains &g) {
     #pragma unroll
-                    for (int u = 0; u < 8; ++u) {
-                        float a = v.get(u);
-                        if constexpr (NORM)
-                            a = norm1(a, r, g[x][u]);
-                        amax[x] = fmaxf(amax[x], fabsf(a));
+                    for (int x = 0; x < NX; ++x) {
+    #pragma unroll
+                        for (int u = 0; u < 8; ++u) {
+                            float a = v.get(u);
+                            if constexpr (NORM)
+                                a = norm1(a, r, g[x][u]);
+                            amax[x] = fmaxf(amax[x], fabsf(a));
+                        }
                     }
-                }
-            });
+                });
+            }
     #pragma unroll
             for (int x = 0; x < NX; ++x) {
                 const uint32_t u = __reduce_max_sync(0xffffffffu, __float_as_uint(amax[x]));
