@@ -36,6 +36,8 @@ constexpr int64_t kAutoGemvMaxM = 6;                // above: tensor-core path
 // Split the k-range of fewer tiles than CTAs only when a CTA saves more than
 // this many 256-k blocks (each about half a microsecond) by it.
 constexpr double kSplitMinSavedBlocks = 10.0;
+// k-blocks of 256 per CTA from which the small token tiles take 512-k stages
+constexpr int64_t kDeepStageMinBlocks = 8;
 constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s: far above any legitimate wait
 constexpr int kMaxDevices = 64;
 
@@ -158,17 +160,18 @@ cudaError_t launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
 }
 
 // x~ [M][K] int8 as a 3-D tensor {128 B, M rows, K/128 chunks} (strides K
-// and 128 bytes), boxed as {128, box_rows, 2} with the 128-byte swizzle: one
-// box is a 256-k slice of box_rows tokens, landing in shared memory as two
-// swizzled [box_rows][128] sub-tiles.
-bool make_map_xq_k256(CUtensorMap *map, const void *ptr, int64_t M, int64_t K, uint32_t box_rows)
+// and 128 bytes), boxed as {128, box_rows, groups} with the 128-byte swizzle:
+// one box is a (128 groups)-k slice of box_rows tokens, landing in shared
+// memory as `groups` swizzled [box_rows][128] sub-tiles.
+bool make_map_xq(CUtensorMap *map, const void *ptr, int64_t M, int64_t K, uint32_t box_rows,
+                 uint32_t groups)
 {
     EncodeTiledFn fn = encode_fn();
     if (fn == nullptr)
         return false;
     const cuuint64_t dims[3] = {128, static_cast<cuuint64_t>(M), static_cast<cuuint64_t>(K / 128)};
     const cuuint64_t strides[2] = {static_cast<cuuint64_t>(K), 128};
-    const cuuint32_t box[3] = {128, box_rows, 2};
+    const cuuint32_t box[3] = {128, box_rows, groups};
     const cuuint32_t estride[3] = {1, 1, 1};
     CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void *>(ptr), dims, strides,
                     box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -178,10 +181,11 @@ bool make_map_xq_k256(CUtensorMap *map, const void *ptr, int64_t M, int64_t K, u
 
 // The packed weights as a 3-D tensor of 8-byte elements {64 (= the 512 bytes
 // of one row block and 128-k group), K/128 groups, ceil(N/16) row blocks}
-// (strides 512 and 16 * K/4 bytes), boxed as {64, 2, box_rows/16}: one box
-// is box_rows rows x 256 weights, landing as [box_rows/16][2][16 rows][32 B].
-bool make_map_packed_k256(CUtensorMap *map, const void *ptr, int64_t N, int64_t K,
-                          uint32_t box_rows)
+// (strides 512 and 16 * K/4 bytes), boxed as {64, groups, box_rows/16}: one
+// box is box_rows rows x (128 groups) weights, landing as
+// [box_rows/16][groups][16 rows][32 B].
+bool make_map_packed(CUtensorMap *map, const void *ptr, int64_t N, int64_t K, uint32_t box_rows,
+                     uint32_t groups)
 {
     EncodeTiledFn fn = encode_fn();
     if (fn == nullptr)
@@ -189,7 +193,7 @@ bool make_map_packed_k256(CUtensorMap *map, const void *ptr, int64_t N, int64_t 
     const cuuint64_t dims[3] = {64, static_cast<cuuint64_t>(K / 128),
                                 static_cast<cuuint64_t>((N + 15) / 16)};
     const cuuint64_t strides[2] = {512, static_cast<cuuint64_t>(16 * (K / 4))};
-    const cuuint32_t box[3] = {64, 2, box_rows / 16};
+    const cuuint32_t box[3] = {64, groups, box_rows / 16};
     const cuuint32_t estride[3] = {1, 1, 1};
     CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT64, 3, const_cast<void *>(ptr), dims, strides,
                     box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
@@ -576,16 +580,16 @@ size_t tc_group_bytes(const TcJob *jobs, int n, bool split)
     return b + (split ? tc_split_bytes(max_M) : 0);
 }
 
-template <int BT>
+template <int BT, int BK = 256>
 int launch_gemm_ws(const wsg::Maps &maps, const wsg::Params &p, int grid, const DeviceInfo &dev,
                    cudaStream_t st)
 {
-    constexpr int smem = wsg::Cfg<BT>::SMEM_BYTES;
-    cudaError_t e = allow_smem<wsg::gemm_ws_kernel<BT>>(dev.id, smem);
+    constexpr int smem = wsg::Cfg<BT, BK>::SMEM_BYTES;
+    cudaError_t e = allow_smem<wsg::gemm_ws_kernel<BT, BK>>(dev.id, smem);
     if (e != cudaSuccess)
         return launch_status(e);
-    e = launch(wsg::gemm_ws_kernel<BT>, dim3(grid), dim3(wsg::THREADS), static_cast<size_t>(smem),
-               st, maps, p);
+    e = launch(wsg::gemm_ws_kernel<BT, BK>, dim3(grid), dim3(wsg::THREADS),
+               static_cast<size_t>(smem), st, maps, p);
     return launch_status(e);
 }
 
@@ -665,6 +669,15 @@ int run_tc_group(const TcJob *jobs, int n, bitlinear_dtype xdt, void *ws, size_t
     for (int i = 0; i < n; ++i)
         max_M = std::max(max_M, jobs[i].M);
     const int BT = choose_bt(max_M);
+    const int slots = std::min(dev.sms, wsg::MAX_GRID);
+    // Stage depth: 512 k for the small token tiles when every CTA has at
+    // least kDeepStageMinBlocks k-blocks of 256 to stream (deep_stages_fit).
+    int64_t iters256 = 0;
+    for (int i = 0; i < n; ++i)
+        iters256 += static_cast<int64_t>((jobs[i].M + BT - 1) / BT) *
+                    ((jobs[i].N + wsg::BW - 1) / wsg::BW) * ((jobs[i].K + 255) / 256);
+    const int BK =
+        (wsg::deep_stages_fit(BT) && iters256 >= kDeepStageMinBlocks * slots) ? 512 : 256;
 
     wsg::Params p{};
     int64_t tiles = 0, iters = 0;
@@ -673,7 +686,7 @@ int run_tc_group(const TcJob *jobs, int n, bitlinear_dtype xdt, void *ws, size_t
         P.M = jobs[i].M;
         P.N = jobs[i].N;
         P.MT = (jobs[i].M + BT - 1) / BT;
-        P.KB = (jobs[i].K + wsg::BK - 1) / wsg::BK;
+        P.KB = (jobs[i].K + BK - 1) / BK;
         P.iter_begin = static_cast<int>(iters);
         P.tile_begin = static_cast<int>(tiles);
         P.gamma = jobs[i].gamma;
@@ -685,7 +698,6 @@ int run_tc_group(const TcJob *jobs, int n, bitlinear_dtype xdt, void *ws, size_t
     }
     if (iters >= (int64_t(1) << 31))
         return BITLINEAR_ERR_SHAPE;
-    const int slots = std::min(dev.sms, wsg::MAX_GRID);
     // Splitting a tile's k-range between CTAs costs a hand-off of a few
     // microseconds (partial store, flag, partial load). With at least as many
     // tiles as CTAs it evens out the last wave; with fewer tiles it pays only
@@ -693,7 +705,8 @@ int run_tc_group(const TcJob *jobs, int n, bitlinear_dtype xdt, void *ws, size_t
     if (split && tiles < slots) {
         const double kb_per_tile = static_cast<double>(iters) / static_cast<double>(tiles);
         const double saved_blocks = kb_per_tile * (1.0 - static_cast<double>(tiles) / slots);
-        split = saved_blocks > kSplitMinSavedBlocks;
+        // in 256-k blocks, whatever the launch's stage depth
+        split = saved_blocks * (BK / 256) > kSplitMinSavedBlocks;
     }
     const int64_t units = split ? iters : tiles;
     const int grid = static_cast<int>(std::min<int64_t>(units, slots));
@@ -729,8 +742,10 @@ int run_tc_group(const TcJob *jobs, int n, bitlinear_dtype xdt, void *ws, size_t
         return rc;
     wsg::Maps maps{};
     for (int i = 0; i < n; ++i)
-        if (!make_map_xq_k256(&maps.x[i], xq[i], jobs[i].M, jobs[i].K, static_cast<uint32_t>(BT)) ||
-            !make_map_packed_k256(&maps.w[i], jobs[i].packed, jobs[i].N, jobs[i].K, wsg::BW))
+        if (!make_map_xq(&maps.x[i], xq[i], jobs[i].M, jobs[i].K, static_cast<uint32_t>(BT),
+                         static_cast<uint32_t>(BK / wsg::SUB_K)) ||
+            !make_map_packed(&maps.w[i], jobs[i].packed, jobs[i].N, jobs[i].K, wsg::BW,
+                             static_cast<uint32_t>(BK / wsg::SUB_K)))
             return BITLINEAR_ERR_CUDA;
     p.count = n;
     p.total_iters = static_cast<int>(iters);
@@ -742,8 +757,14 @@ int run_tc_group(const TcJob *jobs, int n, bitlinear_dtype xdt, void *ws, size_t
         inject_timeout_us > 0 ? static_cast<uint64_t>(inject_timeout_us) * 1000ull : kWaitLimitNs;
     p.inject_timeout = inject_timeout_us > 0 ? 1 : 0;
     switch (BT) {
-    case 32: rc = launch_gemm_ws<32>(maps, p, grid, dev, st); break;
-    case 64: rc = launch_gemm_ws<64>(maps, p, grid, dev, st); break;
+    case 32:
+        rc = BK == 512 ? launch_gemm_ws<32, 512>(maps, p, grid, dev, st)
+                       : launch_gemm_ws<32>(maps, p, grid, dev, st);
+        break;
+    case 64:
+        rc = BK == 512 ? launch_gemm_ws<64, 512>(maps, p, grid, dev, st)
+                       : launch_gemm_ws<64>(maps, p, grid, dev, st);
+        break;
     case 128: rc = launch_gemm_ws<128>(maps, p, grid, dev, st); break;
     default: rc = launch_gemm_ws<192>(maps, p, grid, dev, st); break;
     }

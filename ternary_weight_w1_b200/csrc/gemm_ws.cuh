@@ -33,25 +33,27 @@
 // launch. Without the split (Params::split = 0) the ranges are whole tiles
 // and no partials are used.
 //
-// A k-block is 256 k. One TMA copy brings the x~ tile of a k-block (a 3-D
-// box of two 128-byte-swizzled [BT][128] sub-tiles) and another the packed
-// weights (a 3-D box of 8 row blocks x 2 groups x 512 bytes). A TMA copy
-// costs the issuing thread about the same time whatever its size, so the
-// copies are large and the two streams have a producer warp each. A K that
-// is an odd multiple of 128 leaves the second half of the last k-block
-// outside the tensors, where TMA fills zeros: zero x~ adds nothing.
+// A k-block (one pipeline stage) is 256 k, or 512 k for token tiles of 32
+// and 64 with enough k-blocks per CTA (deep_stages_fit; the host decides). One TMA copy brings the x~ tile of a
+// k-block (a 3-D box of 2 or 4 128-byte-swizzled [BT][128] sub-tiles) and
+// another the packed weights (a 3-D box of 8 row blocks x 2 or 4 groups x
+// 512 bytes). A TMA copy costs the issuing thread about the same time
+// whatever its size, so the copies are large and the two streams have a
+// producer warp each. A K that is not a multiple of the k-block leaves the
+// end of the last k-block outside the tensors, where TMA fills zeros: zero
+// x~ and zero codes add nothing.
 //
 // Warp roles (352 threads):
 //   warp 0     TMA producer of the x~ tiles;
 //   warp 1     MMA issuer (one thread) and TMEM owner;
-//   warps 2-5  decode: one thread per weight row (TMEM lane), 256 k per stage;
+//   warps 2-5  decode: one thread per weight row (TMEM lane), one k-block per stage;
 //   warps 6-9  epilogue: tcgen05.ld 32 tokens at a time, partial store or
 //              row-sum subtract + rescale to bf16; the [32 tokens][128 rows]
 //              bf16 block is transposed through shared memory (two 8 KiB
 //              buffers) so that y is written with 16-byte stores;
 //   warp 10    TMA producer of the packed weight tiles.
-// TMEM columns: [0, 2 BT) two accumulators, [2 BT, 2 BT + 64 NA) the NA
-// stages of decoded weights (64 columns = 256 k of int8 per lane).
+// TMEM columns: [0, 2 BT) two accumulators, then the NA stages of decoded
+// weights (BK / 4 columns each: four int8 codes per column and lane).
 //
 // Every wait is bounded (mbarriers and inter-CTA flags): on a timeout the
 // kernel records a fault word, raises a block-wide abort flag, each role
@@ -64,10 +66,17 @@ namespace bitlinear {
 namespace wsg {
 
 constexpr int BW = 128;                    // weight rows per tile (MMA M)
-constexpr int BK = 256;                    // k per stage (k-block)
 constexpr int SUB_K = 128;                 // k per swizzled sub-tile / packed group
 constexpr int UMMA_K = 32;                 // k per tcgen05.mma kind::i8
-constexpr int PK_BYTES = BW * BK / 4;      // packed weights per stage: 8 KiB
+
+// k per stage (k-block): 256, or 512 for the small token tiles (32 and 64)
+// when every CTA has enough k-blocks to fill the deeper stages. A 256-k
+// stage of a 32-token tile holds only 364 cycles of MMA (8 MMAs), so there
+// a stage's fixed hand-off cost is better paid once per 16 MMAs; the large
+// tiles' stages already hold 512 or more cycles and need the shared memory
+// for depth, and a launch with few k-blocks per CTA needs its first stage
+// early more than it needs fewer stages.
+__host__ __device__ constexpr bool deep_stages_fit(int BT) { return BT <= 64; }
 constexpr int DEC_WARPS = 4;
 constexpr int EPI_WARPS = 4;
 constexpr int PK_WARP = 2 + DEC_WARPS + EPI_WARPS;   // second producer
@@ -76,14 +85,19 @@ constexpr uint32_t TMEM_COLS = 512;
 constexpr int SMEM_BUDGET = 200 * 1024;
 constexpr int MAX_GRID = 192;              // upper bound on CTAs (workspace sizing)
 
-template <int BT>
+template <int BT, int BK_ = 256>
 struct Cfg {
     static_assert(BT % 32 == 0 && BT >= 32 && BT <= 224, "token tile");
+    static_assert(BK_ == 256 || (BK_ == 512 && deep_stages_fit(BT)), "stage depth");
+    static constexpr int BK = BK_;                                 // k per stage
+    static constexpr int GROUPS = BK / SUB_K;                      // 128-k groups per stage
+    static constexpr int PK_BYTES = BW * BK / 4;                   // packed weights per stage
+    static constexpr int A_COLS = BK / 4;                          // TMEM columns per weight stage
     static constexpr int X_SUB = BT * SUB_K;                       // one swizzled sub-tile
     static constexpr int X_BYTES = BT * BK;                        // x~ tile per stage
     static constexpr int STAGE = X_BYTES + PK_BYTES;
     static constexpr int NS = (SMEM_BUDGET / STAGE) < 12 ? (SMEM_BUDGET / STAGE) : 12;
-    static constexpr int NA_FIT = (static_cast<int>(TMEM_COLS) - 2 * BT) / 64;
+    static constexpr int NA_FIT = (static_cast<int>(TMEM_COLS) - 2 * BT) / A_COLS;
     static constexpr int NA = NA_FIT < 6 ? NA_FIT : 6;             // TMEM weight stages
     static constexpr int A_COL0 = 2 * BT;
     static constexpr int NUM_BARS = 2 * NS + 2 * NA + 4 + 2;
@@ -166,11 +180,11 @@ __device__ __forceinline__ int range_owner(const Params &p, int it)
     return it < big ? it / (p.base + 1) : p.extra + (it - big) / p.base;
 }
 
-template <int BT>
+template <int BT, int BK = 256>
 __global__ void __launch_bounds__(THREADS, 1)
 gemm_ws_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Params p)
 {
-    using C = Cfg<BT>;
+    using C = Cfg<BT, BK>;
     constexpr int NS = C::NS;
     constexpr int NA = C::NA;
     extern __shared__ uint8_t smem_raw[];
@@ -179,6 +193,7 @@ gemm_ws_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Params
     uint8_t *const base_ptr = smem_raw + (base - raw);
     const uint32_t sX = base;
     const uint32_t sP = sX + NS * C::X_BYTES;
+    constexpr int PK_BYTES = C::PK_BYTES;
     const uint32_t sEpi = sP + NS * PK_BYTES;
     const uint32_t sBar = sEpi + C::EPI_BYTES;
     auto bar = [&](int i) -> uint32_t { return sBar + 8u * static_cast<uint32_t>(i); };
@@ -259,11 +274,12 @@ gemm_ws_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Params
                 if (is_x) {
                     const int mt = t % P.MT;
                     mbar_arrive_expect_tx(full_load(s), C::X_BYTES);
-                    tma_load_3d(sX + s * C::X_BYTES, &maps.x[q], 0, mt * BT, 2 * kb, full_load(s));
+                    tma_load_3d(sX + s * C::X_BYTES, &maps.x[q], 0, mt * BT, C::GROUPS * kb,
+                                full_load(s));
                 } else {
                     const int nt = t / P.MT;
                     mbar_arrive_expect_tx(full_load(s), PK_BYTES);
-                    tma_load_3d(sP + s * PK_BYTES, &maps.w[q], 0, 2 * kb, nt * (BW / 16),
+                    tma_load_3d(sP + s * PK_BYTES, &maps.w[q], 0, C::GROUPS * kb, nt * (BW / 16),
                                 full_load(s));
                 }
                 if (++s == NS) { s = 0; ph ^= 1u; }
@@ -315,11 +331,12 @@ gemm_ws_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Params
                     if (!mbar_wait_bounded(a_full(a), aph, abort_flag, limit))
                         goto mma_done;
                     tc_fence_after_sync();
-                    const uint32_t a_tmem = tmem_base + static_cast<uint32_t>(C::A_COL0 + 64 * a);
+                    const uint32_t a_tmem =
+                        tmem_base + static_cast<uint32_t>(C::A_COL0 + C::A_COLS * a);
                     const uint32_t b_lo = b_lo0 + static_cast<uint32_t>(s * (C::X_BYTES >> 4));
                     const uint32_t first = kb > k0 ? 1u : 0u;
 #pragma unroll
-                    for (int kk = 0; kk < BK / UMMA_K; ++kk) {
+                    for (int kk = 0; kk < C::BK / UMMA_K; ++kk) {
                         constexpr int X_SUB16 = C::X_SUB >> 4;
                         umma_i8_tmem_a_w(d_tmem, a_tmem + static_cast<uint32_t>(8 * kk),
                                          b_lo + static_cast<uint32_t>((kk / 4) * X_SUB16 +
@@ -350,7 +367,7 @@ gemm_ws_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Params
         const int q = warp & 3;
         const int r = 32 * q + lane;
         const uint32_t lane_off = static_cast<uint32_t>(32 * q) << 16;
-        const int row_off = (r >> 4) * 1024 + (r & 15) * 32;
+        const int row_off = (r >> 4) * (C::GROUPS * 512) + (r & 15) * 32;
         int s = 0, a = 0;
         uint32_t ph = 0, aph = 0;
         for (int it = it_begin; it < it_end; ++it) {
@@ -360,7 +377,7 @@ gemm_ws_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Params
             tc_fence_after_sync();
             const uint8_t *stage = base_ptr + (sP - base) + s * PK_BYTES + row_off;
 #pragma unroll
-            for (int g = 0; g < 2; ++g) {
+            for (int g = 0; g < C::GROUPS; ++g) {
                 const uint4 w0 = *reinterpret_cast<const uint4 *>(stage + 512 * g);
                 const uint4 w1 = *reinterpret_cast<const uint4 *>(stage + 512 * g + 16);
                 const uint32_t wd[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
@@ -373,7 +390,8 @@ gemm_ws_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Params
                     v[4 * w + 3] = (wd[w] >> 6) & 0x03030303u;
                 }
                 tmem_st_32x32b_x32(
-                    tmem_base + lane_off + static_cast<uint32_t>(C::A_COL0 + 64 * a + 32 * g), v);
+                    tmem_base + lane_off +
+                        static_cast<uint32_t>(C::A_COL0 + C::A_COLS * a + 32 * g), v);
             }
             tmem_st_wait();
             tc_fence_before_sync();
