@@ -488,10 +488,12 @@ def bench_b3_decode(bl, wl, reps: int = 200):
 def bench_ffn(bl, device, batches=(1, 8), copies: int = 16, reps: int = 20):
     """The 2B decoder's feed-forward block (gate and up 2560 -> 6912, the
     gated ReLU^2, down 6912 -> 2560) for B decode tokens through
-    bitlinear_ffn_forward: one GEMV launch for gate and up with h written
-    from its epilogue, one launch (pair) for down. The three matrices (13.3 MB
-    packed) rotate over `copies` device copies (212 MB > L2). Per B:
-    microseconds per block and GB/s of packed weights."""
+    bitlinear_ffn_forward: at B <= 6 one GEMV launch for gate and up with h
+    written from its epilogue and one launch for down; at larger B a grouped
+    quantisation + GEMM pair for gate and up, the h kernel, and a
+    quantisation + GEMM pair for down. The three matrices (13.3 MB packed)
+    rotate over `copies` device copies (212 MB > L2). Per B: microseconds per
+    block and GB/s of packed weights."""
     import torch
     K, F = 2560, 6912
     mats = []
@@ -517,7 +519,7 @@ def bench_ffn(bl, device, batches=(1, 8), copies: int = 16, reps: int = 20):
         ms = time_graph(steps, reps, nvtx=f"ffn_b{B}_timed") / copies
         out[f"B={B}"] = {"us_per_block": round(ms * 1e3, 2),
                          "GBps_packed": round(wbytes / (ms * 1e-3) / 1e9, 1),
-                         "launches_per_block": 2 if need == 0 else 3}
+                         "launches_per_block": 2 if need == 0 else (3 if B <= 6 else 5)}
     return out
 
 
@@ -811,8 +813,9 @@ def run_ours(args, dist):
                         "per projection; compare decode_separate_launches",
             **bench_b3_decode(bl, wl)}
         out["ffn_chain"] = {
-            "workload": "2B feed-forward block: gate and up 2560->6912 (one GEMV launch, h = "
-                        "max(gate,0)^2 * up written from its epilogue), down 6912->2560 on h; "
+            "workload": "2B feed-forward block: gate and up 2560->6912 (B<=6: one GEMV "
+                        "launch, h = max(gate,0)^2 * up written from its epilogue; larger B: "
+                        "grouped tensor-core launches and an h kernel), down 6912->2560 on h; "
                         "13.3 MB of packed weights per block",
             **bench_ffn(bl, device)}
         out["layer_set"] = {

@@ -283,10 +283,13 @@ int bitlinear_forward_rmsnorm(const void *x_dev, bitlinear_dtype xdt, int64_t M,
 
 /* ----------------------------------------------------- feed-forward chain */
 
-/* Device workspace bytes bitlinear_ffn_forward needs: that of its down
- * projection (M tokens of F features to K), i.e.
- * bitlinear_workspace_bytes(M, K, F); 0 when that projection takes the GEMV
- * path. SIZE_MAX for shapes bitlinear_ffn_forward refuses. */
+/* Device workspace bytes bitlinear_ffn_forward needs for M tokens, whatever
+ * gains it is given. For decode batches (M <= 6 and 2 M K <= 196608) it is
+ * that of the down projection (M tokens of F features to K), i.e.
+ * bitlinear_workspace_bytes(M, K, F), 0 when that projection takes the
+ * GEMV path. Otherwise the gate/up launches' scratch and their two bf16
+ * outputs, or the down projection's scratch if larger. SIZE_MAX for shapes
+ * bitlinear_ffn_forward refuses. */
 size_t bitlinear_workspace_bytes_ffn(int64_t M, int64_t K, int64_t F);
 
 /* The feed-forward block of a BitNet b1.58 decoder layer for M decode tokens:
@@ -301,16 +304,17 @@ size_t bitlinear_workspace_bytes_ffn(int64_t M, int64_t K, int64_t F);
  * fp32). Each BitLinear is the one of bitlinear_forward (its own gamma); with
  * gains, each RMS-normalises its input first as bitlinear_forward_rmsnorm
  * does (the listing's per-BitLinear nn.RMSNorm).
- * Two launches on cuda_stream: one GEMV launch streams the gate and up
- * weights together (a CTA holds the same rows of both), applies the
- * quantised tokens to both and writes h from its epilogue; then the down
- * projection runs on h as bitlinear_forward_rmsnorm (or bitlinear_forward
- * without a down gain) does, GEMV or tensor cores by M.
+ * Decode batches (M <= 6, and M K <= 196608, 2 M K with gate/up gains):
+ * one GEMV launch streams the gate and up weights together (a CTA holds the
+ * same rows of both), applies the quantised tokens to both and writes h from
+ * its epilogue. Larger batches: gate and up as one grouped quantisation +
+ * tensor-core launch pair (bitlinear_forward_grouped_ws, each with its own
+ * gains), then a small kernel computes h from their bf16 outputs (the same
+ * values). Then the down projection runs on h as bitlinear_forward_rmsnorm
+ * (or bitlinear_forward without a down gain) does, GEMV or tensor cores by M.
  *   x_dev           [in]  [M][K] activations of type xdt
  *   M, K, F         [in]  tokens, d_model, d_ff; K and F positive multiples
- *                         of 128, at most 65536; M <= 16 and M * K (2 M K
- *                         with gate/up gains) <= 196608 (the gate/up
- *                         launch is the GEMV), else BITLINEAR_ERR_SHAPE
+ *                         of 128, at most 65536, else BITLINEAR_ERR_SHAPE
  *   gate_packed_dev, gate_gamma, up_packed_dev, up_gamma
  *                   [in]  F x K packed weights and their gammas
  *   down_packed_dev, down_gamma
@@ -325,7 +329,8 @@ size_t bitlinear_workspace_bytes_ffn(int64_t M, int64_t K, int64_t F);
  *   y_dev           [out] [M][K] bf16
  *   workspace_dev, workspace_bytes
  *                   [in]  scratch of bitlinear_workspace_bytes_ffn(M, K, F)
- *                         bytes (may be NULL when that is 0)
+ *                         bytes, 256-byte aligned (may be NULL when that
+ *                         is 0)
  *   gate_y_dev_or_null, up_y_dev_or_null
  *                   [out, optional] [M][F] bf16 gate and up outputs
  * Errors as for bitlinear_forward, all reported before any launch. */

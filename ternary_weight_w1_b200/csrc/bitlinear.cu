@@ -23,6 +23,7 @@
 #include "gemv.cuh"
 #include "quant_act.cuh"
 #include "stage_io.cuh"
+#include "ffn_act.cuh"
 
 using namespace bitlinear;
 
@@ -956,26 +957,57 @@ namespace {
 
 // Argument checks of the feed-forward calls that do not depend on pointers:
 // returns BITLINEAR_OK when (M, K, F) and the gains' presence are acceptable.
-int check_ffn_shape(int64_t M, int64_t K, int64_t F, bool gate_up_norm)
+int check_ffn_shape(int64_t M, int64_t K, int64_t F)
 {
     if (M < 0 || K < 1 || F < 1)
         return BITLINEAR_ERR_ARG;
-    if (K % 128 != 0 || F % 128 != 0 || K > kMaxK || F > kMaxK)
-        return BITLINEAR_ERR_SHAPE;
-    // the gate/up launch is the GEMV (with two quantised copies of the
-    // tokens when both projections normalise them with their own gains)
-    if (M > kGemvMaxM || (gate_up_norm ? 2 : 1) * M * K > gemv_max_xq(M))
+    if (K % 128 != 0 || F % 128 != 0 || K > kMaxK || F > kMaxK || M > INT_MAX / 2 ||
+        M * K > (int64_t(1) << 40) || M * F > (int64_t(1) << 40))
         return BITLINEAR_ERR_SHAPE;
     return BITLINEAR_OK;
+}
+
+// The fused GEMV launch takes the gate and up projections for decode batches
+// (the automatic GEMV threshold) whose quantised tokens fit beside it (two
+// copies when both projections normalise with their own gains); other
+// batches take the tensor-core route.
+bool ffn_fused(int64_t M, int64_t K, bool gate_up_norm)
+{
+    return M <= kAutoGemvMaxM && (gate_up_norm ? 2 : 1) * M * K <= gemv_max_xq(M);
+}
+
+// Workspace of the tensor-core route: the grouped gate/up launch's scratch
+// (*group_bytes) and its two bf16 outputs (*out_bytes each), then, reusing
+// all of it once they are consumed (stream order), the down projection's.
+size_t ffn_tc_bytes(int64_t M, int64_t K, int64_t F, size_t *group_bytes = nullptr,
+                    size_t *out_bytes = nullptr)
+{
+    TcJob jobs[2] = {};
+    for (TcJob &j : jobs) {
+        j.M = static_cast<int>(M);
+        j.K = static_cast<int>(K);
+        j.N = static_cast<int>(F);
+    }
+    const size_t g = tc_group_bytes(jobs, 2, true);
+    const size_t o = round_up(static_cast<size_t>(M) * static_cast<size_t>(F) * 2, 256);
+    if (group_bytes != nullptr)
+        *group_bytes = g;
+    if (out_bytes != nullptr)
+        *out_bytes = o;
+    return std::max(g + 2 * o, bitlinear_workspace_bytes_path(M, K, F, BITLINEAR_PATH_AUTO));
 }
 
 }  // namespace
 
 extern "C" size_t bitlinear_workspace_bytes_ffn(int64_t M, int64_t K, int64_t F)
 {
-    if (check_ffn_shape(M, K, F, false) != BITLINEAR_OK)
+    if (check_ffn_shape(M, K, F) != BITLINEAR_OK)
         return SIZE_MAX;
-    return bitlinear_workspace_bytes_path(M, K, F, BITLINEAR_PATH_AUTO);
+    // without knowing the gains: the route that normalised gate/up inputs
+    // would take sets the size
+    if (ffn_fused(M, K, true))
+        return bitlinear_workspace_bytes_path(M, K, F, BITLINEAR_PATH_AUTO);
+    return ffn_tc_bytes(M, K, F);
 }
 
 extern "C" int bitlinear_ffn_forward(const void *x_dev, bitlinear_dtype xdt, int64_t M, int64_t K,
@@ -991,7 +1023,7 @@ extern "C" int bitlinear_ffn_forward(const void *x_dev, bitlinear_dtype xdt, int
     if ((gate_gain_dev == nullptr) != (up_gain_dev == nullptr))
         return BITLINEAR_ERR_ARG;
     const bool gu_norm = gate_gain_dev != nullptr;
-    int rc = check_ffn_shape(M, K, F, gu_norm);
+    int rc = check_ffn_shape(M, K, F);
     if (rc != BITLINEAR_OK)
         return rc;
     if (xdt != BITLINEAR_BF16 && xdt != BITLINEAR_FP32)
@@ -1008,16 +1040,55 @@ extern "C" int bitlinear_ffn_forward(const void *x_dev, bitlinear_dtype xdt, int
         !aligned(gate_gain_dev, 16) || !aligned(up_gain_dev, 16) || !aligned(down_gain_dev, 16) ||
         !aligned(gate_y_dev_or_null, 16) || !aligned(up_y_dev_or_null, 16))
         return BITLINEAR_ERR_ALIGN;
+    const bool fused = ffn_fused(M, K, gu_norm);
     // the down projection's own checks (workspace included) before any launch
     const int down_path = choose_path(M, F, BITLINEAR_PATH_AUTO);
     if (down_path == BITLINEAR_PATH_TC &&
         (workspace_dev == nullptr || workspace_bytes < tc_workspace_bytes(M, F)))
         return BITLINEAR_ERR_WORKSPACE;
+    if (!fused && (workspace_dev == nullptr || workspace_bytes < ffn_tc_bytes(M, K, F)))
+        return BITLINEAR_ERR_WORKSPACE;
+    if (!fused && !aligned(workspace_dev, 256))
+        return BITLINEAR_ERR_ALIGN;
     DeviceInfo *dev = nullptr;
     rc = current_device(&dev);
     if (rc != BITLINEAR_OK)
         return rc;
     cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
+    if (!fused) {
+        // Tensor-core route: gate and up as one grouped launch pair (each
+        // with its own gains), h from their bf16 outputs, then the down
+        // projection, which reuses the whole workspace.
+        size_t group_bytes = 0, out_bytes = 0;
+        ffn_tc_bytes(M, K, F, &group_bytes, &out_bytes);
+        char *w = static_cast<char *>(workspace_dev);
+        void *gy = gate_y_dev_or_null != nullptr ? gate_y_dev_or_null : w + group_bytes;
+        void *uy = up_y_dev_or_null != nullptr ? up_y_dev_or_null : w + group_bytes + out_bytes;
+        TcJob jobs[2] = {};
+        const void *packs[2] = {gate_packed_dev, up_packed_dev};
+        const float gammas[2] = {gate_gamma, up_gamma};
+        const float *gains[2] = {gate_gain_dev, up_gain_dev};
+        void *outs[2] = {gy, uy};
+        for (int i = 0; i < 2; ++i)
+            jobs[i] = TcJob{x_dev, static_cast<int>(M), static_cast<int>(K), static_cast<int>(F),
+                            packs[i], gammas[i], outs[i], nullptr, gains[i], norm_eps};
+        rc = run_tc_group(jobs, 2, xdt, workspace_dev, group_bytes, nullptr, nullptr, *dev, st, 0,
+                          true);
+        if (rc != BITLINEAR_OK)
+            return rc;
+        const int64_t n8 = M * F / 8;
+        const int grid = static_cast<int>(
+            std::max<int64_t>(1, std::min<int64_t>((n8 + ffn::THREADS - 1) / ffn::THREADS,
+                                                   2 * dev->sms)));
+        rc = launch_status(launch(ffn::relu2_glu_kernel, dim3(grid), dim3(ffn::THREADS), 0, st,
+                                  static_cast<const uint16_t *>(gy),
+                                  static_cast<const uint16_t *>(uy), h_dev, n8));
+        if (rc != BITLINEAR_OK)
+            return rc;
+        return forward_impl(h_dev, BITLINEAR_FP32, M, F, down_packed_dev, down_gamma, K, y_dev,
+                            workspace_dev, workspace_bytes, cuda_stream, nullptr, nullptr,
+                            nullptr, BITLINEAR_PATH_AUTO, 0, down_gain_dev, norm_eps);
+    }
     GemvJob job{x_dev,
                 static_cast<int>(M),
                 static_cast<int>(K),

@@ -320,9 +320,10 @@ def ffn(M=1, K=256, F=512, x=FAKE, gp=FAKE, up=FAKE, dp=FAKE, gg=None, ug=None, 
     (dict(ug=FAKE), bl.BITLINEAR_ERR_ARG),
     (dict(K=200), bl.BITLINEAR_ERR_SHAPE),
     (dict(F=1000), bl.BITLINEAR_ERR_SHAPE),
-    (dict(M=17), bl.BITLINEAR_ERR_SHAPE),               # the gate/up launch is the GEMV
-    (dict(M=16, K=16384), bl.BITLINEAR_ERR_SHAPE),      # x~ beyond the GEMV's limit
-    (dict(M=8, K=16384, gg=FAKE, ug=FAKE), bl.BITLINEAR_ERR_SHAPE),  # two copies of x~
+    (dict(M=17), bl.BITLINEAR_ERR_WORKSPACE),           # gate/up on the tensor cores
+    (dict(M=4, K=65536, F=128), bl.BITLINEAR_ERR_WORKSPACE),   # x~ beyond the GEMV's limit
+    (dict(M=6, K=32768, gg=FAKE, ug=FAKE), bl.BITLINEAR_ERR_WORKSPACE),  # two copies of x~
+    (dict(M=1, K=65664), bl.BITLINEAR_ERR_SHAPE),       # K beyond 65536
     (dict(M=-1), bl.BITLINEAR_ERR_ARG),
     (dict(xdt=7), bl.BITLINEAR_ERR_DTYPE),
     (dict(dg=FAKE, eps=0.0), bl.BITLINEAR_ERR_ARG),
@@ -339,13 +340,20 @@ def test_ffn_forward_rejects_bad_arguments(kw, status):
     assert ffn(**kw) == status
 
 
-def test_ffn_workspace_is_the_down_projections():
+def test_ffn_workspace():
+    """Decode batches: the down projection's workspace (0 on the GEMV).
+    Larger batches: at least the gate/up group's scratch plus its two bf16
+    outputs, and at least the down projection's."""
     size_max = ctypes.c_size_t(-1).value
     assert bl.bitlinear_workspace_bytes_ffn(1, 2560, 6912) == 0
-    assert (bl.bitlinear_workspace_bytes_ffn(12, 2560, 6912) ==
-            bl.bitlinear_workspace_bytes(12, 2560, 6912))
-    assert bl.bitlinear_workspace_bytes_ffn(17, 2560, 6912) == size_max
+    assert (bl.bitlinear_workspace_bytes_ffn(6, 2560, 6912) ==
+            bl.bitlinear_workspace_bytes(6, 2560, 6912))
+    for M in (7, 12, 17, 300):
+        need = bl.bitlinear_workspace_bytes_ffn(M, 2560, 6912)
+        assert need >= bl.bitlinear_workspace_bytes(M, 2560, 6912)
+        assert need >= 2 * M * 6912 * 2 + M * 2560
     assert bl.bitlinear_workspace_bytes_ffn(1, 2560, 1000) == size_max
+    assert bl.bitlinear_workspace_bytes_ffn(-1, 2560, 6912) == size_max
 
 
 def test_grouped_rmsnorm_rejects_bad_arguments():

@@ -84,8 +84,10 @@ class FfnCase:
                 "up": tensor_to_bf16_bits(out["up"].t)}
 
 
+# M <= 6 takes the fused GEMV launch; larger batches the tensor-core route
+# (grouped gate/up GEMM, the h kernel, then the down projection)
 PLAIN = [(1, 2560, 6912), (3, 2560, 6912), (6, 512, 1024), (12, 2560, 6912), (16, 384, 896),
-         (2, 128, 128)]
+         (2, 128, 128), (7, 1280, 2560), (40, 2560, 6912), (300, 512, 1024)]
 
 
 @pytest.mark.parametrize("M,K,F", PLAIN)
@@ -105,7 +107,8 @@ def test_ffn_fp32_tokens():
     np.testing.assert_array_equal(got["y"], c.ref["down"]["y"])
 
 
-@pytest.mark.parametrize("M,K,F", [(1, 2560, 6912), (5, 1024, 2048), (16, 2560, 6912)])
+@pytest.mark.parametrize("M,K,F", [(1, 2560, 6912), (5, 1024, 2048), (16, 2560, 6912),
+                                   (24, 1024, 2048)])
 def test_ffn_normalised_matches_oracle(M, K, F):
     c = FfnCase(M, K, F, seed=M * 11 + K + F, norm=True)
     got = c.run()

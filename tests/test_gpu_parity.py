@@ -71,6 +71,16 @@ def test_tc_parity(cuda, M, K, N):
     assert exact == 1.0
 
 
+@pytest.mark.parametrize("M,K,N", [(40, 6912, 8192), (17, 2560, 19000), (64, 8320, 4600)])
+def test_tc_deep_stages(cuda, M, K, N):
+    """Token tiles of 32 and 64 with at least 8 k-blocks of 256 per CTA take
+    512-k stages; K = 6912 and 8320 leave part of the last stage outside the
+    tensors (zero-filled), N a ragged last weight tile. Full comparison."""
+    c = Case(M, K, N, w_seed=7 * K + N, x_seed=M + 3 * K)
+    got = c.run(path=bl.PATH_TC)
+    assert c.check_full(got, _omp_oracle()) == 1.0
+
+
 @pytest.mark.parametrize("M", [20, 50, 200, 300])
 def test_tc_token_tiles_shared_k(cuda, M):
     # token tiles of 32, 64, 128 and 192 rows; only a few tiles with 54
