@@ -244,8 +244,10 @@ gemm_ws_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Params
         tmem_relinquish();
 
     // x~, beta, the row sums and the flags are written by the preceding
-    // quantisation kernel (programmatic dependent launch).
-    pdl_wait();
+    // quantisation kernel (programmatic dependent launch). The packed
+    // weights are not: their producer starts streaming at once.
+    if (warp != PK_WARP)
+        pdl_wait();
 
     const int it_begin = range_begin(p, blockIdx.x);
     const int it_end = range_begin(p, blockIdx.x + 1);

@@ -267,6 +267,10 @@ quant_act_grouped_kernel(const __grid_constant__ GroupParams g)
     const GroupRows &r = g.prob[q];
     const int warp = threadIdx.x >> 5;
     const int m = (static_cast<int>(blockIdx.x) - r.first_block) * rows_per_block<WPR>() + warp / WPR;
+    // The GEMM that follows may launch at once: a grouped call's grid is
+    // small (decode batches), and the GEMM's weight stream needs nothing
+    // from this kernel.
+    pdl_launch_dependents();
     pdl_wait();
     if (g.clear != nullptr && blockIdx.x == 0)
         for (int i = threadIdx.x; i < g.n_clear; i += THREADS)
