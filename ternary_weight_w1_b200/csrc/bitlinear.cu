@@ -387,7 +387,6 @@ int launch_gemv(const GemvJob *jobs, int count, bitlinear_dtype xdt, const Devic
                       max_K <= 32768;
     if (wide)
         xq_cap *= 2;
-    const int ring_budget = wide ? 110 * 1024 : 72 * 1024;
     int blocks[gemv::MAX_PROBLEMS], ctas[gemv::MAX_PROBLEMS], G[gemv::MAX_PROBLEMS];
     double bbytes[gemv::MAX_PROBLEMS];
     double max_block = 0.0;
@@ -452,9 +451,14 @@ int launch_gemv(const GemvJob *jobs, int count, bitlinear_dtype xdt, const Devic
             stages = std::max(stages, ((q + cb[i] - 1) / cb[i]) * ((KG + G[i] - 1) / G[i]));
         }
         // Ring depth: the whole share when it is small, else as deep as a
-        // 72 KiB block allows (three blocks per SM fit beside each other;
-        // 110 KiB for the wide kernel's two).
+        // 72 KiB block allows (three blocks per SM fit beside each other, the
+        // third for the next launch under programmatic dependent launch). A
+        // stream of four or more stages per CTA (long rows, many blocks) and
+        // the wide kernel get 110 KiB: two blocks per SM then keep more bytes
+        // in flight, which a long stream needs more than the overlap with the
+        // next launch (measured: 2B layer at B = 1 7.0 -> 6.4 us).
         const int fixed = gemv::smem_bytes(MT, xq_cap, 0, 0, red_blocks, norm, ffn, b3);
+        const int ring_budget = (wide || stages >= 4) ? 110 * 1024 : 72 * 1024;
         slots = (ring_budget - fixed) / slot_bytes;
         slots = std::max(1, std::min({slots, stages, gemv::MAX_SLOTS}));
         if (stages > 1)
