@@ -251,17 +251,6 @@ __device__ __forceinline__ void cp_async_wait_all()
     asm volatile("cp.async.wait_all;" ::: "memory");
 }
 
-// 2-D tiled tensor copy global -> this CTA's shared memory.
-__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, int x,
-                                            int y, uint32_t bar)
-{
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes "
-        "[%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
-        : "memory");
-}
-
 // 3-D tiled tensor copy global -> this CTA's shared memory.
 __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap *map, int c0, int c1,
                                             int c2, uint32_t bar)
@@ -277,13 +266,6 @@ __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap *map)
 {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map))
                  : "memory");
-}
-
-// Make this thread's generic-proxy shared-memory writes visible to the async
-// proxy (TMA, tensor cores) before signalling their consumer.
-__device__ __forceinline__ void fence_proxy_async_smem()
-{
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
 // ----------------------------------------------------------------- tcgen05
@@ -318,36 +300,12 @@ __device__ __forceinline__ void tc_fence_after_sync()
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
 
-// D[tmem] (+)= A[smem] * B[smem]^T, int8 inputs, int32 accumulator.
-__device__ __forceinline__ void umma_i8(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
-                                        uint32_t idesc, uint32_t accumulate)
-{
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
-        : "memory");
-}
-
 // D[tmem] (+)= A[tmem] * B[smem]^T, int8 inputs, int32 accumulator. For
 // M = 128 the A tile occupies TMEM lanes 0..127 (lane = row) and k runs along
 // the columns, four int8 values per 32-bit column (k = 4c .. 4c+3 in bytes
-// 0..3), eight columns per k-step of 32.
-__device__ __forceinline__ void umma_i8_tmem_a(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
-                                               uint32_t idesc, uint32_t accumulate)
-{
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::i8 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
-        : "memory");
-}
-
-// umma_i8_tmem_a with the B descriptor given as its two 32-bit words, so that
-// an issuing loop can step the start address (the low word's bits 0-13, in
-// 16-byte units) with one 32-bit add per MMA.
+// 0..3), eight columns per k-step of 32. The B descriptor comes as its two
+// 32-bit words, so that an issuing loop can step the start address (the low
+// word's bits 0-13, in 16-byte units) with one 32-bit add per MMA.
 __device__ __forceinline__ void umma_i8_tmem_a_w(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_lo,
                                                  uint32_t b_hi, uint32_t idesc,
                                                  uint32_t accumulate)

@@ -62,14 +62,26 @@ __device__ __forceinline__ void quant_row(const void *__restrict__ x, int M, int
     float amax = 0.0f;
     float r = 1.0f;                               // NORM: 1 / rms of the row
     if constexpr (!NORM) {
+        // bf16: the largest 15-bit magnitude field, two per word (for finite
+        // values that order is the order of |x|), widened at the end
+        uint32_t mb = 0;
+        auto take = [&](const Vec8<BF16> &t) {
+            if constexpr (BF16) {
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                    mb = max_u16x2(mb, t.w[j] & 0x7fff7fffu);
+            } else {
+#pragma unroll
+                for (int j = 0; j < 8; ++j)
+                    amax = fmaxf(amax, fabsf(t.get(j)));
+            }
+        };
 #pragma unroll
         for (int i = 0; i < CACHE; ++i) {
             const int v = v0 + STRIDE * i;
             if (v < nvec) {
                 cache[i].load(row, v * 8);
-#pragma unroll
-                for (int j = 0; j < 8; ++j)
-                    amax = fmaxf(amax, fabsf(cache[i].get(j)));
+                take(cache[i]);
             }
         }
         for (int vb = v0 + STRIDE * CACHE; vb < nvec; vb += 4 * STRIDE) {
@@ -81,10 +93,10 @@ __device__ __forceinline__ void quant_row(const void *__restrict__ x, int M, int
 #pragma unroll
             for (int u = 0; u < 4; ++u)
                 if (vb + u * STRIDE < nvec)
-#pragma unroll
-                    for (int j = 0; j < 8; ++j)
-                        amax = fmaxf(amax, fabsf(t[u].get(j)));
+                    take(t[u]);
         }
+        if constexpr (BF16)
+            amax = __uint_as_float(max(mb & 0xffffu, mb >> 16) << 16);
     } else {
         // sum of squares (each product exact in double)
         double ss = 0.0;
