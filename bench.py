@@ -459,9 +459,9 @@ def bench_rmsnorm_decode(bl, wl, reps: int = 200) -> float:
 
 def bench_b3_decode(bl, wl, reps: int = 200):
     """The decode step's two projections (M = 1) on base-3 packed weights
-    (bitlinear_forward_b3, one launch per projection) over ROTATE copies, the
-    footprint option: µs per step, GB/s of base-3 bytes, and the bytes per
-    step against the 2-bit layout's."""
+    (bitlinear_forward_grouped_b3, one launch per step, as the 2-bit step)
+    over ROTATE copies, the footprint option: µs per step, GB/s of base-3
+    bytes, and the bytes per step against the 2-bit layout's."""
     import torch
     mats = []
     for m in wl.mats:
@@ -473,8 +473,8 @@ def bench_b3_decode(bl, wl, reps: int = 200):
 
     def steps():
         for j in range(ROTATE):
-            for m, d, g in mats:
-                bl.bitlinear_forward_b3(m["x"][j], d[j], g, m["p"].N, y=m["y"][j])
+            bl.bitlinear_forward_grouped_b3(
+                [(m["x"][j], d[j], g, m["p"].N, m["y"][j]) for m, d, g in mats])
     steps()
     torch.cuda.synchronize()
     ms = time_graph(steps, reps, nvtx="b3_decode_timed") / ROTATE
@@ -482,7 +482,7 @@ def bench_b3_decode(bl, wl, reps: int = 200):
             "GBps_b3_bytes": round(b3_bytes / (ms * 1e-3) / 1e9, 1),
             "b3_bytes_per_step": b3_bytes,
             "two_bit_bytes_per_step": wl.packed_bytes_per_step,
-            "launches_per_step": 2}
+            "launches_per_step": 1}
 
 
 def bench_ffn(bl, device, batches=(1, 8), copies: int = 16, reps: int = 20):
@@ -809,8 +809,8 @@ def run_ours(args, dist):
     if not args.no_extra:
         out["b3_decode"] = {
             "workload": "the decode step (up 2560->6912, down 6912->2560, M=1) on base-3 packed "
-                        "weights (5 codes per byte, K padded to a multiple of 160), one launch "
-                        "per projection; compare decode_separate_launches",
+                        "weights (5 codes per byte, K padded to a multiple of 160), one grouped "
+                        "launch per step; compare the headline value",
             **bench_b3_decode(bl, wl)}
         out["ffn_chain"] = {
             "workload": "2B feed-forward block: gate and up 2560->6912 (B<=6: one GEMV "

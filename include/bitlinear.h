@@ -371,6 +371,19 @@ typedef struct {
 int bitlinear_forward_grouped(const bitlinear_problem *problems, int count,
                               bitlinear_dtype xdt, void *cuda_stream);
 
+/* bitlinear_forward_grouped with base-3 packed weights
+ * (bitlinear_pack_weights_b3) for every problem: one GEMV launch, each
+ * problem computed exactly as bitlinear_forward_b3 computes it alone.
+ *   problems [in] as for bitlinear_forward_grouped, packed_dev holding
+ *                 bitlinear_packed_bytes_b3(N, K) bytes; M <= 16 and M * Kp
+ *                 <= 196608 per problem (Kp = K rounded up to a multiple of
+ *                 160), and the group's largest M * Kp within the limit of
+ *                 its largest M
+ *   xdt      [in] activation dtype of all problems
+ * Errors as for bitlinear_forward_grouped, all reported before any launch. */
+int bitlinear_forward_grouped_b3(const bitlinear_problem *problems, int count,
+                                 bitlinear_dtype xdt, void *cuda_stream);
+
 /* bitlinear_forward_grouped with the tokens taken from, and the outputs
  * returned to, host memory, all on cuda_stream. This is the one call a
  * decode step makes when its tokens arrive from the host and its outputs

@@ -64,6 +64,7 @@ EXPORTS = (
     "bitlinear_forward_noalloc",
     "bitlinear_forward_grouped",
     "bitlinear_forward_grouped_host",
+    "bitlinear_forward_grouped_b3",
     "bitlinear_workspace_bytes_grouped",
     "bitlinear_forward_grouped_ws",
     "bitlinear_forward_grouped_rmsnorm",
@@ -134,6 +135,8 @@ def lib() -> ctypes.CDLL:
                                                 i64, p, p]
         L.bitlinear_forward_grouped.restype = ctypes.c_int
         L.bitlinear_forward_grouped.argtypes = [p, ctypes.c_int, ctypes.c_int, p]
+        L.bitlinear_forward_grouped_b3.restype = ctypes.c_int
+        L.bitlinear_forward_grouped_b3.argtypes = [p, ctypes.c_int, ctypes.c_int, p]
         L.bitlinear_forward_grouped_host.restype = ctypes.c_int
         L.bitlinear_forward_grouped_host.argtypes = [p, ctypes.c_int, ctypes.c_int, p, p, p]
         L.bitlinear_workspace_bytes_grouped.restype = ctypes.c_size_t
@@ -531,7 +534,7 @@ def bitlinear_forward_noalloc(x, packed, gamma: float, N: int, y=None, stream=No
     return y
 
 
-def _problem_array(problems, alloc_y, a=None):
+def _problem_array(problems, alloc_y, a=None, b3=False):
     import torch
     arr = (_Problem * len(problems))()
     outs = []
@@ -541,8 +544,13 @@ def _problem_array(problems, alloc_y, a=None):
             y = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
         outs.append(y)
         if alloc_y:
-            arr[i] = _Problem(a.ptr(x, f"problems[{i}].x"), M, K, N,
-                              a.packed(packed, N, K), float(gamma),
+            if b3:
+                need = (bitlinear_packed_bytes_b3(N, K)
+                        if N >= 1 and K >= 128 and K % 128 == 0 else 1)
+                pk = a.ptr(packed, f"problems[{i}].packed_b3", torch.uint8, min_numel=need)
+            else:
+                pk = a.packed(packed, N, K)
+            arr[i] = _Problem(a.ptr(x, f"problems[{i}].x"), M, K, N, pk, float(gamma),
                               a.ptr(y, f"problems[{i}].y", torch.bfloat16, (M, N)))
         else:                              # sizing only: shapes, no pointers
             arr[i] = _Problem(None, M, K, N, None, float(gamma), None)
@@ -577,6 +585,21 @@ def bitlinear_forward_grouped(problems, stream=None, workspace=None):
                                                   a.ptr(workspace, "workspace", torch.uint8),
                                                   workspace.numel(), _stream(stream)),
                "bitlinear_forward_grouped_ws")
+    return outs
+
+
+def bitlinear_forward_grouped_b3(problems, stream=None):
+    """bitlinear_forward_grouped with base-3 packed weights (one GEMV
+    launch). ``problems`` is a list of (x, packed_b3, gamma, N, y) with device
+    tensors (y may be None). Returns the list of outputs."""
+    if not problems:
+        return []
+    xdt = _xdt(problems[0][0])
+    a = _Args()
+    arr, outs = _problem_array(problems, alloc_y=True, a=a, b3=True)
+    _check(lib().bitlinear_forward_grouped_b3(ctypes.addressof(arr), len(problems), xdt,
+                                              _stream(stream)),
+           "bitlinear_forward_grouped_b3")
     return outs
 
 

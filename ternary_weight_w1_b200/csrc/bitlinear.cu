@@ -1156,9 +1156,10 @@ extern "C" int bitlinear_forward_b3(const void *x_dev, bitlinear_dtype xdt, int6
 namespace {
 
 // Checks a problem list for the one-launch grouped GEMV and collects its
-// non-empty problems into jobs[0 .. *n).
+// non-empty problems into jobs[0 .. *n). With b3 the weights are in the
+// base-3 layout, whose x~ rows the GEMV pads to 160-weight groups.
 int collect_gemv_group(const bitlinear_problem *problems, int count, bitlinear_dtype xdt,
-                       GemvJob *jobs, int *n)
+                       GemvJob *jobs, int *n, bool b3 = false)
 {
     if (problems == nullptr || count < 1 || count > gemv::MAX_PROBLEMS)
         return BITLINEAR_ERR_ARG;
@@ -1172,13 +1173,15 @@ int collect_gemv_group(const bitlinear_problem *problems, int count, bitlinear_d
             return rc;
         if (pr.M == 0)
             continue;
-        if (!gemv_fits(pr.M, pr.K))
+        const int64_t xrow = b3 ? (pr.K + 159) / 160 * 160 : pr.K;
+        if (!gemv_fits(pr.M, xrow))
             return BITLINEAR_ERR_SHAPE;
         max_M = std::max(max_M, pr.M);
-        max_xq = std::max(max_xq, pr.M * pr.K);
-        jobs[(*n)++] = GemvJob{pr.x_dev,      static_cast<int>(pr.M), static_cast<int>(pr.K),
-                               static_cast<int>(pr.N), pr.packed_dev, pr.gamma, pr.y_dev,
-                               nullptr, nullptr, nullptr, nullptr, 0.0f};
+        max_xq = std::max(max_xq, pr.M * xrow);
+        jobs[*n] = GemvJob{pr.x_dev,      static_cast<int>(pr.M), static_cast<int>(pr.K),
+                           static_cast<int>(pr.N), pr.packed_dev, pr.gamma, pr.y_dev,
+                           nullptr, nullptr, nullptr, nullptr, 0.0f};
+        jobs[(*n)++].b3 = b3;
     }
     // one launch holds the largest x~ next to the largest problem's token tile
     if (*n > 0 && max_xq > gemv_max_xq(max_M))
@@ -1241,6 +1244,21 @@ void *mapped_device_ptr(const void *host)
         return nullptr;
     }
     return a.type == cudaMemoryTypeHost ? a.devicePointer : nullptr;
+}
+
+extern "C" int bitlinear_forward_grouped_b3(const bitlinear_problem *problems, int count,
+                                            bitlinear_dtype xdt, void *cuda_stream)
+{
+    GemvJob jobs[gemv::MAX_PROBLEMS];
+    int n = 0;
+    int rc = collect_gemv_group(problems, count, xdt, jobs, &n, true);
+    if (rc != BITLINEAR_OK || n == 0)
+        return rc;
+    DeviceInfo *dev = nullptr;
+    rc = current_device(&dev);
+    if (rc != BITLINEAR_OK)
+        return rc;
+    return launch_gemv(jobs, n, xdt, *dev, static_cast<cudaStream_t>(cuda_stream));
 }
 
 extern "C" int bitlinear_forward_grouped_host(const bitlinear_problem *problems, int count,

@@ -214,6 +214,26 @@ def grouped_host(problems, xdt=0, x_host=FAKE, y_host=FAKE):
                                                    x_host, y_host, None)
 
 
+def test_grouped_b3_rejects_bad_arguments():
+    def call(problems, xdt=0):
+        arr = (bl._Problem * max(1, len(problems)))()
+        for i, (x, M, K, N, packed, y) in enumerate(problems):
+            arr[i] = bl._Problem(x, M, K, N, packed, 1.0, y)
+        return bl.lib().bitlinear_forward_grouped_b3(ctypes.addressof(arr), len(problems), xdt,
+                                                     None)
+    good = (FAKE, 1, 256, 64, FAKE, FAKE)
+    assert bl.lib().bitlinear_forward_grouped_b3(None, 1, 0, None) == bl.BITLINEAR_ERR_ARG
+    assert call([]) == bl.BITLINEAR_ERR_ARG
+    assert call([good] * 9) == bl.BITLINEAR_ERR_ARG
+    assert call([good, (FAKE, 17, 256, 64, FAKE, FAKE)]) == bl.BITLINEAR_ERR_SHAPE
+    # 16 x 12288 is within the 2-bit GEMV's limit (196608), but the base-3
+    # rows pad to 12320
+    assert call([(FAKE, 16, 12288, 64, FAKE, FAKE)]) == bl.BITLINEAR_ERR_SHAPE
+    assert call([good, (FAKE + 8, 1, 256, 64, FAKE, FAKE)]) == bl.BITLINEAR_ERR_ALIGN
+    assert call([good], xdt=5) == bl.BITLINEAR_ERR_DTYPE
+    assert call([(None, 0, 256, 64, None, None)]) == bl.BITLINEAR_OK   # nothing to do
+
+
 def test_grouped_host_rejects_bad_arguments():
     """The host-buffer call checks what bitlinear_forward_grouped checks, and
     its host buffers, before any copy or launch."""

@@ -56,3 +56,26 @@ def test_b3_equals_2bit_path():
     np.testing.assert_array_equal(got["y"], ref["y"])
     np.testing.assert_array_equal(got["acc"], ref["acc"])
     assert bl.bitlinear_get_fault() == (bl.BITLINEAR_OK, 0)
+
+
+def test_b3_grouped_decode_pair_and_mixed():
+    """bitlinear_forward_grouped_b3: the decode step's two projections and a
+    mixed group in one launch each, every problem bit-exact against the
+    oracle and equal to its single base-3 call."""
+    import torch
+    groups = [[Case(1, 2560, 6912, w_seed=21, x_seed=22), Case(1, 6912, 2560, w_seed=23, x_seed=24)],
+              [Case(3, 384, 500, w_seed=25, x_seed=26), Case(1, 8192, 96, w_seed=27, x_seed=28),
+               Case(6, 640, 33, w_seed=29, x_seed=30)]]
+    for cases in groups:
+        probs = []
+        for c in cases:
+            packed, gamma = bl.bitlinear_pack_weights_b3(c.W)
+            probs.append((c.x_tensor(), torch.from_numpy(packed).cuda(), gamma, c.N, None))
+        ys = bl.bitlinear_forward_grouped_b3(probs)
+        torch.cuda.synchronize()
+        for c, y, pr in zip(cases, ys, probs):
+            got = y.view(torch.int16).cpu().numpy().view(np.uint16)
+            np.testing.assert_array_equal(got, c.oracle_full()[1])
+            single = run_b3(c)["y"]
+            np.testing.assert_array_equal(got, single)
+    assert bl.bitlinear_get_fault() == (bl.BITLINEAR_OK, 0)
