@@ -34,7 +34,8 @@
 // and no partials are used.
 //
 // A k-block (one pipeline stage) is 256 k, or 512 k for token tiles of 32
-// and 64 with enough k-blocks per CTA (deep_stages_fit; the host decides). One TMA copy brings the x~ tile of a
+// and 64 with enough k-blocks per CTA (deep_stages_fit; the host decides).
+// One TMA copy brings the x~ tile of a
 // k-block (a 3-D box of 2 or 4 128-byte-swizzled [BT][128] sub-tiles) and
 // another the packed weights (a 3-D box of 8 row blocks x 2 or 4 groups x
 // 512 bytes). A TMA copy costs the issuing thread about the same time
@@ -51,7 +52,11 @@
 //              row-sum subtract + rescale to bf16; the [32 tokens][128 rows]
 //              bf16 block is transposed through shared memory (two 8 KiB
 //              buffers) so that y is written with 16-byte stores;
-//   warp 10    TMA producer of the packed weight tiles.
+//   warp 10    TMA producer of the packed weight tiles; it starts before
+//              griddepcontrol.wait (no earlier kernel writes the weights).
+// The decode warps wait on a stage's two barriers (copies landed, TMEM slot
+// free) at once; the MMA issuer waits only on the decoded-weights barrier,
+// since every synchronising wait of that thread idles the tensor pipe.
 // TMEM columns: [0, 2 BT) two accumulators, then the NA stages of decoded
 // weights (BK / 4 columns each: four int8 codes per column and lane).
 //

@@ -34,10 +34,14 @@
 // exactly, and acc = sum c * x~ - sum x~. Integer sums: the order of the
 // partial sums cannot change the result.
 //
-// Prologue. Each thread reads the activations of its own warp's groups (lane
-// l: elements 128 g + 4 l .. + 3), the warps combine their absmax through
-// shared memory (one barrier), and every warp quantises its own groups into
-// shared memory, where only its own lanes read them. The sum of x~ of each
+// Prologue. Each thread reads the activations of its own warp's groups in
+// 16-byte slots (half-warp h: group w + 8 (2 i + h), lane l: elements
+// 128 g + 8 (l % 16) .. + 7), keeping the first slots of token 0 in
+// registers between the passes; the warps combine their absmax through
+// shared memory (one barrier; for bf16 the maximum of the 15-bit magnitude
+// fields, two per word, which orders finite values as |x| does), and every
+// warp quantises its own groups into shared memory, where only its own lanes
+// read them. The sum of x~ of each
 // warp's groups goes to shared memory for the epilogue. With RMS
 // normalisation (NORM launches; the listing's BitLinear normalises each token
 // with its nn.RMSNorm member before quantising it) a first pass sums each
