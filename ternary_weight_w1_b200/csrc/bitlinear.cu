@@ -593,7 +593,7 @@ int launch_gemm_ws(const wsg::Maps &maps, const wsg::Params &p, int grid, const 
     cudaError_t e = allow_smem<wsg::gemm_ws_kernel<BT, BK>>(dev.id, smem);
     if (e != cudaSuccess)
         return launch_status(e);
-    e = launch(wsg::gemm_ws_kernel<BT, BK>, dim3(grid), dim3(wsg::THREADS),
+    e = launch(wsg::gemm_ws_kernel<BT, BK>, dim3(grid), dim3(wsg::Cfg<BT, BK>::THREADS),
                static_cast<size_t>(smem), st, maps, p);
     return launch_status(e);
 }

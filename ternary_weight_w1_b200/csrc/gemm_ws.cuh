@@ -85,7 +85,7 @@ __host__ __device__ constexpr bool deep_stages_fit(int BT) { return BT <= 64; }
 constexpr int DEC_WARPS = 4;
 constexpr int EPI_WARPS = 4;
 constexpr int PK_WARP = 2 + DEC_WARPS + EPI_WARPS;   // second producer
-constexpr int THREADS = (PK_WARP + 1) * 32;
+constexpr int MMA2_WARP = PK_WARP + 1;          // second MMA issuer (DUAL launches)
 constexpr uint32_t TMEM_COLS = 512;
 constexpr int SMEM_BUDGET = 200 * 1024;
 constexpr int MAX_GRID = 192;              // upper bound on CTAs (workspace sizing)
@@ -93,6 +93,16 @@ constexpr int MAX_GRID = 192;              // upper bound on CTAs (workspace siz
 template <int BT, int BK_ = 256>
 struct Cfg {
     static_assert(BT % 32 == 0 && BT >= 32 && BT <= 224, "token tile");
+    // Two MMA-issuing threads (warps 1 and MMA2_WARP) taking alternate
+    // stages, each into its own accumulators, for the smallest token tile: a
+    // lone issuing thread idles the tensor pipe at every synchronising wait,
+    // and short MMAs leave it no time to catch up. At BT = 32 the second pair
+    // of accumulators costs no weight stage in TMEM; at BT = 64 it would cost
+    // two of six (one of three at BK = 512), which loses more than the
+    // second issuer gains.
+    static constexpr bool DUAL = BT <= 32;
+    static constexpr int ISSUERS = DUAL ? 2 : 1;
+    static constexpr int THREADS = (PK_WARP + 1 + (DUAL ? 1 : 0)) * 32;
     static_assert(BK_ == 256 || (BK_ == 512 && deep_stages_fit(BT)), "stage depth");
     static constexpr int BK = BK_;                                 // k per stage
     static constexpr int GROUPS = BK / SUB_K;                      // 128-k groups per stage
@@ -102,10 +112,11 @@ struct Cfg {
     static constexpr int X_BYTES = BT * BK;                        // x~ tile per stage
     static constexpr int STAGE = X_BYTES + PK_BYTES;
     static constexpr int NS = (SMEM_BUDGET / STAGE) < 12 ? (SMEM_BUDGET / STAGE) : 12;
-    static constexpr int NA_FIT = (static_cast<int>(TMEM_COLS) - 2 * BT) / A_COLS;
+    static constexpr int ACC_COLS = 2 * ISSUERS * BT;              // [issuer][buffer] accumulators
+    static constexpr int NA_FIT = (static_cast<int>(TMEM_COLS) - ACC_COLS) / A_COLS;
     static constexpr int NA = NA_FIT < 6 ? NA_FIT : 6;             // TMEM weight stages
-    static constexpr int A_COL0 = 2 * BT;
-    static constexpr int NUM_BARS = 2 * NS + 2 * NA + 4 + 2;
+    static constexpr int A_COL0 = ACC_COLS;
+    static constexpr int NUM_BARS = 2 * NS + 2 * NA + 4 * ISSUERS + 1 + ISSUERS;
     static constexpr int EPI_BYTES = 2 * 32 * BW * 2;              // two bf16 [32][128] blocks
     static constexpr int SMEM_BYTES =
         1024 + NS * X_BYTES + NS * PK_BYTES + EPI_BYTES + NUM_BARS * 8 + 16;
@@ -186,7 +197,7 @@ __device__ __forceinline__ int range_owner(const Params &p, int it)
 }
 
 template <int BT, int BK = 256>
-__global__ void __launch_bounds__(THREADS, 1)
+__global__ void __launch_bounds__((Cfg<BT, BK>::THREADS), 1)
 gemm_ws_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Params p)
 {
     using C = Cfg<BT, BK>;
@@ -206,10 +217,12 @@ gemm_ws_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Params
     auto empty_load = [&](int s) { return bar(NS + s); };
     auto a_full = [&](int a) { return bar(2 * NS + a); };
     auto a_empty = [&](int a) { return bar(2 * NS + NA + a); };
-    auto acc_full = [&](int b) { return bar(2 * NS + 2 * NA + b); };
-    auto acc_empty = [&](int b) { return bar(2 * NS + 2 * NA + 2 + b); };
-    const uint32_t never_bar = bar(2 * NS + 2 * NA + 4);
-    const uint32_t drain_bar = bar(2 * NS + 2 * NA + 5);
+    constexpr int ISSUERS = C::ISSUERS;
+    // accumulator barriers per issuer i and buffer b
+    auto acc_full = [&](int i, int b) { return bar(2 * NS + 2 * NA + 2 * i + b); };
+    auto acc_empty = [&](int i, int b) { return bar(2 * NS + 2 * NA + 2 * ISSUERS + 2 * i + b); };
+    const uint32_t never_bar = bar(2 * NS + 2 * NA + 4 * ISSUERS);
+    auto drain_bar = [&](int i) { return bar(2 * NS + 2 * NA + 4 * ISSUERS + 1 + i); };
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(base_ptr + (sBar - base) + C::NUM_BARS * 8);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
@@ -226,12 +239,14 @@ gemm_ws_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Params
             mbar_init(a_full(a), DEC_WARPS);
             mbar_init(a_empty(a), 1);
         }
-        for (int b = 0; b < 2; ++b) {
-            mbar_init(acc_full(b), 1);
-            mbar_init(acc_empty(b), EPI_WARPS);
+        for (int i = 0; i < ISSUERS; ++i) {
+            for (int b = 0; b < 2; ++b) {
+                mbar_init(acc_full(i, b), 1);
+                mbar_init(acc_empty(i, b), EPI_WARPS);
+            }
+            mbar_init(drain_bar(i), 1);
         }
         mbar_init(never_bar, 1);
-        mbar_init(drain_bar, 1);
         *abort_flag = 0;
         fence_barrier_init();
     }
@@ -298,11 +313,13 @@ gemm_ws_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Params
                     drain_wait(full_load(i), static_cast<uint32_t>(armed[i]), limit);
         }
         __syncwarp();
-    } else if (warp == 1) {
+    } else if (warp == 1 || (C::DUAL && warp == MMA2_WARP)) {
         // -------------------------------------------------------- MMA issuer
+        // Issuer me takes this CTA's stages c with c % ISSUERS == me, into
+        // its own accumulator pair; the epilogue adds the issuers' sums.
         if (lane == 0) {
-            int s = 0, a = 0, seg = 0;
-            uint32_t aph = 0;
+            const int me = (warp == 1) ? 0 : 1;
+            int seg = 0;
             // The x~ descriptors of every stage and k-step differ from stage
             // 0's first one only in the start address (low word, 16-byte
             // units, no carry: shared addresses stay below 2^18), so the
@@ -323,12 +340,21 @@ gemm_ws_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Params
                 const int k0 = local - t * P.KB;
                 const int k1 = min(P.KB, k0 + (it_end - it));
                 const int buf = seg & 1;
-                if (!mbar_wait_bounded(acc_empty(buf), ((static_cast<uint32_t>(seg) >> 1) & 1u) ^ 1u,
-                                       abort_flag, limit))
+                if (!mbar_wait_bounded(acc_empty(me, buf),
+                                       ((static_cast<uint32_t>(seg) >> 1) & 1u) ^ 1u, abort_flag,
+                                       limit))
                     goto mma_done;
                 tc_fence_after_sync();
-                const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * BT);
+                const uint32_t d_tmem =
+                    tmem_base + static_cast<uint32_t>((2 * me + buf) * BT);
+                bool first = true;
                 for (int kb = k0; kb < k1; ++kb) {
+                    const int c = it - it_begin + (kb - k0);   // this CTA's stage number
+                    if (ISSUERS > 1 && (c % ISSUERS) != me)
+                        continue;
+                    const int s = c % NS;
+                    const int a = c % NA;
+                    const uint32_t aph = static_cast<uint32_t>(c / NA) & 1u;
                     // a_full(a) completes only after the decode warps have
                     // seen full_load(s) (both TMA copies of the stage, x~
                     // included, have landed) and written the codes, so one
@@ -341,27 +367,28 @@ gemm_ws_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Params
                     const uint32_t a_tmem =
                         tmem_base + static_cast<uint32_t>(C::A_COL0 + C::A_COLS * a);
                     const uint32_t b_lo = b_lo0 + static_cast<uint32_t>(s * (C::X_BYTES >> 4));
-                    const uint32_t first = kb > k0 ? 1u : 0u;
+                    const uint32_t acc_in = first ? 0u : 1u;
 #pragma unroll
                     for (int kk = 0; kk < C::BK / UMMA_K; ++kk) {
                         constexpr int X_SUB16 = C::X_SUB >> 4;
                         umma_i8_tmem_a_w(d_tmem, a_tmem + static_cast<uint32_t>(8 * kk),
                                          b_lo + static_cast<uint32_t>((kk / 4) * X_SUB16 +
                                                                       (kk % 4) * (UMMA_K >> 4)),
-                                         b_hi, C::IDESC, kk > 0 ? 1u : first);
+                                         b_hi, C::IDESC, kk > 0 ? 1u : acc_in);
                     }
+                    first = false;
                     umma_commit(empty_load(s));
                     umma_commit(a_empty(a));
-                    if (++s == NS) s = 0;
-                    if (++a == NA) { a = 0; aph ^= 1u; }
                 }
-                umma_commit(acc_full(buf));
+                // arrives once this issuer's MMAs of the segment are done (at
+                // once when it had none: the epilogue then skips its sum)
+                umma_commit(acc_full(me, buf));
                 it += k1 - k0;
             }
         mma_done:
             // All MMAs issued by this thread complete before TMEM is freed.
-            umma_commit(drain_bar);
-            drain_wait(drain_bar, 0u, limit);
+            umma_commit(drain_bar(me));
+            drain_wait(drain_bar(me), 0u, limit);
         }
         __syncwarp();
     } else if (warp < 2 + DEC_WARPS) {
@@ -423,6 +450,11 @@ gemm_ws_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Params
             const int t = local / P.KB;
             const int k0 = local - t * P.KB;
             const int k1 = min(P.KB, k0 + (it_end - it));
+            // which issuers have stages in this segment (with two, a segment
+            // of one stage belongs to the issuer of its parity)
+            const int c0 = it - it_begin;
+            const bool has0 = ISSUERS == 1 || k1 - k0 >= 2 || (c0 & 1) == 0;
+            const bool has1 = ISSUERS == 2 && (k1 - k0 >= 2 || (c0 & 1) == 1);
             it += k1 - k0;
             const int buf = seg & 1;
             const int mt = t % P.MT;
@@ -443,12 +475,39 @@ gemm_ws_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Params
 
             // The four epilogue warps take every wait's verdict together (named
             // barrier 1), so none can be left behind at the transpose barrier.
-            bool ready = warp_wait_bounded(acc_full(buf), (static_cast<uint32_t>(seg) >> 1) & 1u,
-                                           abort_flag, limit);
+            const uint32_t acc_par = (static_cast<uint32_t>(seg) >> 1) & 1u;
+            bool ready = ISSUERS == 1
+                             ? warp_wait_bounded(acc_full(0, buf), acc_par, abort_flag, limit)
+                             : warp_wait2_bounded(acc_full(0, buf), acc_par,
+                                                  acc_full(ISSUERS - 1, buf), acc_par, abort_flag,
+                                                  limit);
             if (!named_bar_and(1, EPI_WARPS * 32, ready))
                 break;
             tc_fence_after_sync();
-            const uint32_t d_cols = tmem_base + lane_off + static_cast<uint32_t>(buf * BT);
+            // chunk c of the segment's sum: issuer 0's accumulator plus, with
+            // two issuers, issuer 1's (only the issuers that had stages)
+            auto load_acc = [&](int c, uint32_t (&r)[32]) {
+                const uint32_t col = lane_off + static_cast<uint32_t>(32 * c);
+                if (has0)
+                    tmem_ld_32x32b_x32(tmem_base + col + static_cast<uint32_t>(buf * BT), r);
+                if constexpr (ISSUERS == 2) {
+                    if (has1) {
+                        uint32_t r1[32];
+                        tmem_ld_32x32b_x32(
+                            tmem_base + col + static_cast<uint32_t>((2 + buf) * BT), r1);
+                        tmem_ld_wait();
+#pragma unroll
+                        for (int j = 0; j < 32; ++j)
+                            r[j] = has0 ? r[j] + r1[j] : r1[j];
+                    }
+                }
+                tmem_ld_wait();
+            };
+            auto release_acc = [&]() {
+                if (lane == 0)
+                    for (int i = 0; i < ISSUERS; ++i)
+                        mbar_arrive(acc_empty(i, buf));
+            };
 
             if (k0 > 0) {
                 // Not the tile's first k-block: hand the partial sum to the
@@ -457,8 +516,7 @@ gemm_ws_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Params
 #pragma unroll 1
                 for (int c = 0; c < BT / 32; ++c) {
                     uint32_t r[32];
-                    tmem_ld_32x32b_x32(d_cols + static_cast<uint32_t>(32 * c), r);
-                    tmem_ld_wait();
+                    load_acc(c, r);
 #pragma unroll
                     for (int g = 0; g < 8; ++g)
                         __stcg(reinterpret_cast<int4 *>(slot + 32 * c + 4 * g),
@@ -470,10 +528,9 @@ gemm_ws_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Params
                 // release of the flag (a release is cumulative).
                 tc_fence_before_sync();
                 __syncwarp();
-                if (lane == 0) {
+                if (lane == 0)
                     st_release_gpu(p.flags + 4 * blockIdx.x + q, 1);
-                    mbar_arrive(acc_empty(buf));
-                }
+                release_acc();
                 continue;
             }
 
@@ -527,8 +584,7 @@ gemm_ws_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Params
                 if (m0 >= P.M)
                     break;
                 uint32_t r[32];
-                tmem_ld_32x32b_x32(d_cols + static_cast<uint32_t>(32 * c), r);
-                tmem_ld_wait();
+                load_acc(c, r);
                 // Partial sums of the other contributors, two at a time so
                 // that their loads are in flight together.
                 for (int c2 = blockIdx.x + 1; c2 <= c_last; c2 += 2) {
@@ -600,8 +656,7 @@ gemm_ws_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Params
             }
             tc_fence_before_sync();
             __syncwarp();
-            if (lane == 0)
-                mbar_arrive(acc_empty(buf));
+            release_acc();
         }
     }
 
