@@ -44,7 +44,7 @@
 // end of the last k-block outside the tensors, where TMA fills zeros: zero
 // x~ and zero codes add nothing.
 //
-// Warp roles (352 threads):
+// Warp roles (352 threads; 384 with a second MMA issuer):
 //   warp 0     TMA producer of the x~ tiles;
 //   warp 1     MMA issuer (one thread) and TMEM owner;
 //   warps 2-5  decode: one thread per weight row (TMEM lane), one k-block per stage;
@@ -53,12 +53,14 @@
 //              bf16 block is transposed through shared memory (two 8 KiB
 //              buffers) so that y is written with 16-byte stores;
 //   warp 10    TMA producer of the packed weight tiles; it starts before
-//              griddepcontrol.wait (no earlier kernel writes the weights).
+//              griddepcontrol.wait (no earlier kernel writes the weights);
+//   warp 11    second MMA issuer for the 32-token tile (Cfg::DUAL).
 // The decode warps wait on a stage's two barriers (copies landed, TMEM slot
 // free) at once; the MMA issuer waits only on the decoded-weights barrier,
 // since every synchronising wait of that thread idles the tensor pipe.
-// TMEM columns: [0, 2 BT) two accumulators, then the NA stages of decoded
-// weights (BK / 4 columns each: four int8 codes per column and lane).
+// TMEM columns: [0, 2 BT) two accumulators (four with two issuers), then the
+// NA stages of decoded weights (BK / 4 columns each: four int8 codes per
+// column and lane).
 //
 // Every wait is bounded (mbarriers and inter-CTA flags): on a timeout the
 // kernel records a fault word, raises a block-wide abort flag, each role
