@@ -124,6 +124,7 @@ struct Cfg {
         1024 + NS * X_BYTES + NS * PK_BYTES + EPI_BYTES + NUM_BARS * 8 + 16;
     static constexpr uint32_t IDESC = idesc_i8_s32(BW, BT);
     static_assert(NA >= 2, "TMEM budget");
+    static_assert(NS <= 32, "slot masks");
     static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
 };
 
@@ -282,37 +283,61 @@ gemm_ws_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Params
             const bool is_x = (warp == 0);
             int s = 0;
             uint32_t ph = 0;
-            int armed[NS];
-            for (int i = 0; i < NS; ++i) armed[i] = -1;
+            uint32_t armed = 0, armed_ph = 0;   // slots armed (bit i) and their phase
+            // The stage's coordinates are stepped, not recomputed: problem q,
+            // its k-block kb and tile t = nt * MT + mt (the token tile varies
+            // fastest). A lone thread issues the copies, and the loop's own
+            // latency (parameter reads, divisions) would otherwise pace it.
             int q = problem_of_iter(p, it_begin);
-            for (int it = it_begin; it < it_end; ++it) {
-                while (q + 1 < p.count && it >= p.prob[q + 1].iter_begin)
-                    ++q;
+            int kb = 0, mt = 0, nt = 0, KB = 1, MT = 1;
+            const CUtensorMap *map = nullptr;
+            auto enter = [&](int it) {
                 const Problem &P = p.prob[q];
+                KB = P.KB;
+                MT = P.MT;
                 const int local = it - P.iter_begin;
-                const int t = local / P.KB;
-                const int kb = local - t * P.KB;
+                const int t = local / KB;
+                kb = local - t * KB;
+                mt = t % MT;
+                nt = t / MT;
+                map = is_x ? &maps.x[q] : &maps.w[q];
+            };
+            if (it_begin < it_end)
+                enter(it_begin);
+            int next_begin = q + 1 < p.count ? p.prob[q + 1].iter_begin : it_end;
+            for (int it = it_begin; it < it_end; ++it) {
+                if (it >= next_begin) {
+                    // first k-block of a later problem (skipping empty ones)
+                    do {
+                        ++q;
+                    } while (q + 1 < p.count && it >= p.prob[q + 1].iter_begin);
+                    enter(it);
+                    next_begin = q + 1 < p.count ? p.prob[q + 1].iter_begin : it_end;
+                }
                 if (!mbar_wait_bounded(empty_load(s), ph ^ 1u, abort_flag, limit))
                     break;
-                armed[s] = static_cast<int>(ph);
+                armed |= 1u << s;
+                armed_ph = (armed_ph & ~(1u << s)) | (ph << s);
                 if (is_x) {
-                    const int mt = t % P.MT;
                     mbar_arrive_expect_tx(full_load(s), C::X_BYTES);
-                    tma_load_3d(sX + s * C::X_BYTES, &maps.x[q], 0, mt * BT, C::GROUPS * kb,
+                    tma_load_3d(sX + s * C::X_BYTES, map, 0, mt * BT, C::GROUPS * kb,
                                 full_load(s));
                 } else {
-                    const int nt = t / P.MT;
                     mbar_arrive_expect_tx(full_load(s), PK_BYTES);
-                    tma_load_3d(sP + s * PK_BYTES, &maps.w[q], 0, C::GROUPS * kb, nt * (BW / 16),
+                    tma_load_3d(sP + s * PK_BYTES, map, 0, C::GROUPS * kb, nt * (BW / 16),
                                 full_load(s));
+                }
+                if (++kb == KB) {
+                    kb = 0;
+                    if (++mt == MT) { mt = 0; ++nt; }
                 }
                 if (++s == NS) { s = 0; ph ^= 1u; }
             }
             // Wait for every copy this thread started, so no TMA write lands
             // after the block has exited.
             for (int i = 0; i < NS; ++i)
-                if (armed[i] >= 0)
-                    drain_wait(full_load(i), static_cast<uint32_t>(armed[i]), limit);
+                if (armed & (1u << i))
+                    drain_wait(full_load(i), (armed_ph >> i) & 1u, limit);
         }
         __syncwarp();
     } else if (warp == 1 || (C::DUAL && warp == MMA2_WARP)) {
@@ -412,10 +437,20 @@ gemm_ws_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Params
                 break;
             tc_fence_after_sync();
             const uint8_t *stage = base_ptr + (sP - base) + s * PK_BYTES + row_off;
+            // All of the stage's packed words are loaded before the first
+            // TMEM store: the stores are asm statements the compiler does not
+            // move loads across, so loads interleaved with them would wait out
+            // one shared-memory latency per group.
+            uint4 wv[2 * C::GROUPS];
 #pragma unroll
             for (int g = 0; g < C::GROUPS; ++g) {
-                const uint4 w0 = *reinterpret_cast<const uint4 *>(stage + 512 * g);
-                const uint4 w1 = *reinterpret_cast<const uint4 *>(stage + 512 * g + 16);
+                wv[2 * g] = *reinterpret_cast<const uint4 *>(stage + 512 * g);
+                wv[2 * g + 1] = *reinterpret_cast<const uint4 *>(stage + 512 * g + 16);
+            }
+#pragma unroll
+            for (int g = 0; g < C::GROUPS; ++g) {
+                const uint4 w0 = wv[2 * g];
+                const uint4 w1 = wv[2 * g + 1];
                 const uint32_t wd[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
                 uint32_t v[32];
 #pragma unroll
