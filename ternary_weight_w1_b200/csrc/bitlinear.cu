@@ -226,6 +226,25 @@ cudaError_t launch_qa(const void *x, int M, int K, int8_t *xq, float *beta, int 
                   x, M, K, xq, beta, rowsum, clear, n_clear, gain, eps);
 }
 
+// Prefill batches (at least kStagedQuantMinRows tokens, no normalisation,
+// four or more rows in kStagedQuantSmem bytes) take the staged kernel: R rows
+// per block in shared memory, one wave for the batch.
+constexpr int kStagedQuantMinRows = 1024;
+constexpr int kStagedQuantSmem = 112 * 1024;
+
+template <bool BF16>
+int launch_qa_staged(const void *x, int M, int K, int rpb, int8_t *xq, float *beta, int *rowsum,
+                     cudaStream_t st, int *clear, int n_clear, int dev)
+{
+    const int smem = rpb * K * (BF16 ? 2 : 4);
+    cudaError_t e = allow_smem<qa::quant_act_staged_kernel<BF16>>(dev, smem);
+    if (e == cudaSuccess)
+        e = launch(qa::quant_act_staged_kernel<BF16>, dim3((M + rpb - 1) / rpb),
+                   dim3(qa::THREADS), smem, st, x, M, K, rpb, xq, beta, rowsum, clear, n_clear,
+                   kWaitLimitNs);
+    return launch_status(e);
+}
+
 // Register cache per lane and warps per row by row length: every lane holds
 // its whole share of a row in registers up to 16384 bf16 (8192 fp32)
 // elements per row, so a row is read from memory once and small batches are
@@ -237,6 +256,19 @@ int launch_quant_act(const void *x, bitlinear_dtype xdt, int M, int K, int8_t *x
 {
     if (M == 0)
         return BITLINEAR_OK;
+    const int row_bytes = K * (xdt == BITLINEAR_BF16 ? 2 : 4);
+    const int rpb = std::min(qa::WARPS, kStagedQuantSmem / row_bytes);
+    if (gain == nullptr && M >= kStagedQuantMinRows && rpb >= 4) {
+        DeviceInfo *dev = nullptr;
+        const int rc = current_device(&dev);
+        if (rc != BITLINEAR_OK)
+            return rc;
+        return xdt == BITLINEAR_BF16
+                   ? launch_qa_staged<true>(x, M, K, rpb, xq, beta, rowsum, st, clear, n_clear,
+                                            dev->id)
+                   : launch_qa_staged<false>(x, M, K, rpb, xq, beta, rowsum, st, clear, n_clear,
+                                             dev->id);
+    }
     const int nvec = K / 8;
     cudaError_t e;
     if (xdt == BITLINEAR_BF16) {

@@ -19,7 +19,9 @@
 // gains g read as they are needed. The row sum
 // of x~ is written for the tensor-core path, whose GEMM contracts the
 // non-negative weight codes W~ + 1 (acc = sum x~ * code - sum x~). Block 0
-// also clears the GEMM's inter-block flag words when asked to.
+// also clears the GEMM's inter-block flag words when asked to. Prefill
+// batches take a variant that stages whole rows in shared memory with bulk
+// copies (quant_act_staged_kernel), so that one wave of blocks covers them.
 #pragma once
 
 #include "common.cuh"
@@ -244,6 +246,118 @@ quant_act_kernel(const void *__restrict__ x, int M, int K, int8_t *__restrict__ 
             clear[i] = 0;
     quant_row<BF16, CACHE, WPR, NORM>(x, M, K, xq, beta_out, rowsum_out, gain, eps, m,
                                       warp % WPR);
+}
+
+// Rows staged in shared memory, for prefill batches: thread 0 brings the
+// block's R whole rows into shared memory with one bulk copy per row, all
+// completing on one mbarrier, so a block keeps R rows in flight without
+// holding them in registers and one wave of blocks covers the batch. Warp w
+// then quantises rows w, w + WARPS, ... from shared memory in two passes
+// (absmax, then quantise and store) with the arithmetic of quant_row's plain
+// path, so x~, beta and the row sums are the same bits. A wait that gives up
+// records the fault and the block writes nothing.
+template <bool BF16>
+__global__ void __launch_bounds__(THREADS)
+quant_act_staged_kernel(const void *__restrict__ x, int M, int K, int rpb,
+                        int8_t *__restrict__ xq, float *__restrict__ beta_out,
+                        int *__restrict__ rowsum_out, int *__restrict__ clear, int n_clear,
+                        uint64_t limit_ns)
+{
+    extern __shared__ __align__(128) uint8_t rows_sm[];
+    __shared__ __align__(8) uint64_t bar_sm;
+    __shared__ int abort_sm;
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const uint32_t bar = smem_u32(&bar_sm);
+    const int m0 = blockIdx.x * rpb;
+    const int rows = min(rpb, M - m0);
+    const uint32_t row_bytes = static_cast<uint32_t>(K) * (BF16 ? 2u : 4u);
+    if (threadIdx.x == 0) {
+        mbar_init(bar, 1);
+        abort_sm = 0;
+        fence_barrier_init();
+    }
+    __syncthreads();
+    pdl_wait();
+    // The GEMM that follows uses these words as inter-block flags.
+    if (clear != nullptr && blockIdx.x == 0)
+        for (int i = threadIdx.x; i < n_clear; i += THREADS)
+            clear[i] = 0;
+    if (threadIdx.x == 0) {
+        mbar_arrive_expect_tx(bar, row_bytes * static_cast<uint32_t>(rows));
+        for (int r = 0; r < rows; ++r)
+            bulk_g2s(smem_u32(rows_sm) + static_cast<uint32_t>(r) * row_bytes,
+                     static_cast<const char *>(x) + static_cast<size_t>(m0 + r) * row_bytes,
+                     row_bytes, bar);
+    }
+    // every lane of a warp takes the same verdict, so the warp's reductions
+    // below run with all its lanes or with none
+    const bool ok =
+        __all_sync(0xffffffffu, mbar_wait_bounded(bar, 0u, &abort_sm, limit_ns)) != 0;
+    pdl_launch_dependents();
+    if (ok) {
+        const int nvec = K >> 3;
+        constexpr int VB = BF16 ? 16 : 32;              // bytes per vector of 8
+        for (int r = warp; r < rows; r += WARPS) {
+            const uint8_t *row = rows_sm + static_cast<size_t>(r) * row_bytes;
+            auto vec = [&](int v) {
+                Vec8<BF16> t;
+                const uint4 *src = reinterpret_cast<const uint4 *>(row + static_cast<size_t>(v) * VB);
+#pragma unroll
+                for (int i = 0; i < Vec8<BF16>::WORDS / 4; ++i) {
+                    const uint4 a = src[i];
+                    t.w[4 * i] = a.x; t.w[4 * i + 1] = a.y; t.w[4 * i + 2] = a.z; t.w[4 * i + 3] = a.w;
+                }
+                return t;
+            };
+            float amax = 0.0f;
+            if constexpr (BF16) {
+                uint32_t mb = 0;
+                for (int v = lane; v < nvec; v += 32) {
+                    const Vec8<BF16> t = vec(v);
+#pragma unroll
+                    for (int j = 0; j < 4; ++j)
+                        mb = max_u16x2(mb, t.w[j] & 0x7fff7fffu);
+                }
+                amax = __uint_as_float(max(mb & 0xffffu, mb >> 16) << 16);
+            } else {
+                for (int v = lane; v < nvec; v += 32) {
+                    const Vec8<BF16> t = vec(v);
+#pragma unroll
+                    for (int j = 0; j < 8; ++j)
+                        amax = fmaxf(amax, fabsf(t.get(j)));
+                }
+            }
+            const uint32_t umax = __reduce_max_sync(0xffffffffu, __float_as_uint(amax));
+            const float beta = fmaxf(__uint_as_float(umax), 1e-5f);
+            const float scale = __fdiv_rn(127.0f, beta);
+            const int m = m0 + r;
+            int8_t *out = xq + static_cast<size_t>(m) * K;
+            int sum = 0;
+            for (int v = lane; v < nvec; v += 32) {
+                const Vec8<BF16> t = vec(v);
+                uint32_t lo = 0, hi = 0;
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const int q0 = quant1(t.get(i), scale);
+                    const int q1 = quant1(t.get(i + 4), scale);
+                    sum += q0 + q1;
+                    lo |= (static_cast<uint32_t>(q0) & 0xffu) << (8 * i);
+                    hi |= (static_cast<uint32_t>(q1) & 0xffu) << (8 * i);
+                }
+                *reinterpret_cast<uint2 *>(out + v * 8) = make_uint2(lo, hi);
+            }
+            sum = __reduce_add_sync(0xffffffffu, sum);
+            if (lane == 0) {
+                beta_out[m] = beta;
+                if (rowsum_out != nullptr)
+                    rowsum_out[m] = sum;
+            }
+        }
+    } else if (threadIdx.x == 0) {
+        // no copy may land after the block has exited
+        drain_wait(bar, 0u, limit_ns);
+    }
 }
 
 // Several problems' token rows in one launch (WPR warps per row): block b
