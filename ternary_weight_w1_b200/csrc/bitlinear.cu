@@ -226,22 +226,41 @@ cudaError_t launch_qa(const void *x, int M, int K, int8_t *xq, float *beta, int 
                   x, M, K, xq, beta, rowsum, clear, n_clear, gain, eps);
 }
 
-// Prefill batches (at least kStagedQuantMinRows tokens, no normalisation,
-// four or more rows in kStagedQuantSmem bytes) take the staged kernel: R rows
-// per block in shared memory, one wave for the batch.
+// Prefill batches (at least kStagedQuantMinRows tokens, four or more rows in
+// kStagedQuantSmem bytes) take the staged kernel: R rows per block in shared
+// memory, one wave for the batch.
 constexpr int kStagedQuantMinRows = 1024;
 constexpr int kStagedQuantSmem = 112 * 1024;
 
-template <bool BF16>
-int launch_qa_staged(const void *x, int M, int K, int rpb, int8_t *xq, float *beta, int *rowsum,
-                     cudaStream_t st, int *clear, int n_clear, int dev)
+template <bool BF16, bool NORM>
+cudaError_t launch_qa_staged_t(const void *x, int M, int K, int rpb, int8_t *xq, float *beta,
+                               int *rowsum, cudaStream_t st, int *clear, int n_clear,
+                               const float *gain, float eps, int dev)
 {
     const int smem = rpb * K * (BF16 ? 2 : 4);
-    cudaError_t e = allow_smem<qa::quant_act_staged_kernel<BF16>>(dev, smem);
+    cudaError_t e = allow_smem<qa::quant_act_staged_kernel<BF16, NORM>>(dev, smem);
     if (e == cudaSuccess)
-        e = launch(qa::quant_act_staged_kernel<BF16>, dim3((M + rpb - 1) / rpb),
+        e = launch(qa::quant_act_staged_kernel<BF16, NORM>, dim3((M + rpb - 1) / rpb),
                    dim3(qa::THREADS), smem, st, x, M, K, rpb, xq, beta, rowsum, clear, n_clear,
-                   kWaitLimitNs);
+                   gain, eps, kWaitLimitNs);
+    return e;
+}
+
+int launch_qa_staged(const void *x, bool bf16, int M, int K, int rpb, int8_t *xq, float *beta,
+                     int *rowsum, cudaStream_t st, int *clear, int n_clear, const float *gain,
+                     float eps, int dev)
+{
+    cudaError_t e;
+    if (gain != nullptr)
+        e = bf16 ? launch_qa_staged_t<true, true>(x, M, K, rpb, xq, beta, rowsum, st, clear,
+                                                  n_clear, gain, eps, dev)
+                 : launch_qa_staged_t<false, true>(x, M, K, rpb, xq, beta, rowsum, st, clear,
+                                                   n_clear, gain, eps, dev);
+    else
+        e = bf16 ? launch_qa_staged_t<true, false>(x, M, K, rpb, xq, beta, rowsum, st, clear,
+                                                   n_clear, gain, eps, dev)
+                 : launch_qa_staged_t<false, false>(x, M, K, rpb, xq, beta, rowsum, st, clear,
+                                                    n_clear, gain, eps, dev);
     return launch_status(e);
 }
 
@@ -258,16 +277,13 @@ int launch_quant_act(const void *x, bitlinear_dtype xdt, int M, int K, int8_t *x
         return BITLINEAR_OK;
     const int row_bytes = K * (xdt == BITLINEAR_BF16 ? 2 : 4);
     const int rpb = std::min(qa::WARPS, kStagedQuantSmem / row_bytes);
-    if (gain == nullptr && M >= kStagedQuantMinRows && rpb >= 4) {
+    if (M >= kStagedQuantMinRows && rpb >= 4) {
         DeviceInfo *dev = nullptr;
         const int rc = current_device(&dev);
         if (rc != BITLINEAR_OK)
             return rc;
-        return xdt == BITLINEAR_BF16
-                   ? launch_qa_staged<true>(x, M, K, rpb, xq, beta, rowsum, st, clear, n_clear,
-                                            dev->id)
-                   : launch_qa_staged<false>(x, M, K, rpb, xq, beta, rowsum, st, clear, n_clear,
-                                             dev->id);
+        return launch_qa_staged(x, xdt == BITLINEAR_BF16, M, K, rpb, xq, beta, rowsum, st, clear,
+                                n_clear, gain, eps, dev->id);
     }
     const int nvec = K / 8;
     cudaError_t e;

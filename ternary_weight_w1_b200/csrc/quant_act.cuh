@@ -253,15 +253,16 @@ quant_act_kernel(const void *__restrict__ x, int M, int K, int8_t *__restrict__ 
 // completing on one mbarrier, so a block keeps R rows in flight without
 // holding them in registers and one wave of blocks covers the batch. Warp w
 // then quantises rows w, w + WARPS, ... from shared memory in two passes
-// (absmax, then quantise and store) with the arithmetic of quant_row's plain
-// path, so x~, beta and the row sums are the same bits. A wait that gives up
-// records the fault and the block writes nothing.
-template <bool BF16>
+// (absmax, then quantise and store; with NORM a sum-of-squares pass first)
+// with quant_row's arithmetic for one warp per row, so x~, beta and the row
+// sums are the same bits as quant_row with one warp per row gives. A wait
+// that gives up records the fault and the block writes nothing.
+template <bool BF16, bool NORM>
 __global__ void __launch_bounds__(THREADS)
 quant_act_staged_kernel(const void *__restrict__ x, int M, int K, int rpb,
                         int8_t *__restrict__ xq, float *__restrict__ beta_out,
                         int *__restrict__ rowsum_out, int *__restrict__ clear, int n_clear,
-                        uint64_t limit_ns)
+                        const float *__restrict__ gain, float eps, uint64_t limit_ns)
 {
     extern __shared__ __align__(128) uint8_t rows_sm[];
     __shared__ __align__(8) uint64_t bar_sm;
@@ -311,7 +312,27 @@ quant_act_staged_kernel(const void *__restrict__ x, int M, int K, int rpb,
                 return t;
             };
             float amax = 0.0f;
-            if constexpr (BF16) {
+            float rn = 1.0f;                            // NORM: 1 / rms of the row
+            if constexpr (NORM) {
+                double ss = 0.0;
+                for (int v = lane; v < nvec; v += 32) {
+                    const Vec8<BF16> t = vec(v);
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        const double d = t.get(j);
+                        ss = __fma_rn(d, d, ss);
+                    }
+                }
+                rn = rms_scale(warp_sum_f64(ss), K, eps);
+                for (int v = lane; v < nvec; v += 32) {
+                    const Vec8<BF16> t = vec(v);
+                    float g[8];
+                    load8<false>(gain, v * 8, g);
+#pragma unroll
+                    for (int j = 0; j < 8; ++j)
+                        amax = fmaxf(amax, fabsf(norm1(t.get(j), rn, g[j])));
+                }
+            } else if constexpr (BF16) {
                 uint32_t mb = 0;
                 for (int v = lane; v < nvec; v += 32) {
                     const Vec8<BF16> t = vec(v);
@@ -336,11 +357,19 @@ quant_act_staged_kernel(const void *__restrict__ x, int M, int K, int rpb,
             int sum = 0;
             for (int v = lane; v < nvec; v += 32) {
                 const Vec8<BF16> t = vec(v);
+                float g[8];
+                if constexpr (NORM)
+                    load8<false>(gain, v * 8, g);
                 uint32_t lo = 0, hi = 0;
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
-                    const int q0 = quant1(t.get(i), scale);
-                    const int q1 = quant1(t.get(i + 4), scale);
+                    float a = t.get(i), b = t.get(i + 4);
+                    if constexpr (NORM) {
+                        a = norm1(a, rn, g[i]);
+                        b = norm1(b, rn, g[i + 4]);
+                    }
+                    const int q0 = quant1(a, scale);
+                    const int q1 = quant1(b, scale);
                     sum += q0 + q1;
                     lo |= (static_cast<uint32_t>(q0) & 0xffu) << (8 * i);
                     hi |= (static_cast<uint32_t>(q1) & 0xffu) << (8 * i);

@@ -71,6 +71,14 @@ def test_tc_rmsnorm_long_rows(cuda, dtype):
     c.check_norm_full(c.run(path=bl.PATH_TC))
 
 
+@pytest.mark.parametrize("M,K,dtype", [(1030, 2560, "bf16"), (1027, 1280, "fp32")])
+def test_tc_rmsnorm_staged_rows(cuda, M, K, dtype):
+    # from 1024 tokens the quantiser stages whole rows in shared memory (eight
+    # per block, a ragged last block)
+    c = NormCase(M, K, 48, g_seed=M, w_seed=K + 1, x_seed=M + K, x_dtype=dtype)
+    c.check_norm_full(c.run(path=bl.PATH_TC))
+
+
 # ------------------------------------------------------------- edge cases
 
 @pytest.mark.parametrize("path", [bl.PATH_GEMV, bl.PATH_TC])
