@@ -15,6 +15,7 @@ import ctypes
 import numpy as np
 import pytest
 
+import oracle
 import ternary_weight_w1_b200 as bl
 from tests.gpu_cases import Case, check_y, tensor_to_bf16_bits
 
@@ -44,14 +45,15 @@ def test_noalloc_matches_workspace_path_twice():
         got, ref = tensor_to_bf16_bits(y), tensor_to_bf16_bits(y_ref)
         check_y(got, ref)                        # the parity tolerance (rel 1e-2)
         np.testing.assert_array_equal(got, ref)  # same kernels: identical bits
+        assert check_y(got, c.oracle_full()[1]) == 1.0   # and the oracle's bits
     assert bl.bitlinear_get_fault() == (bl.BITLINEAR_OK, 0)
 
 
 def test_noalloc_fills_the_scratch_exactly_and_rejects_beyond_it():
     """M = 2424 tokens of K = 6912 fill the 16 MiB array to its last bytes
     (x~, beta and the row sums of x~); on seeded nonzero data the result must
-    equal the workspace path's bit for bit. One more token is refused before
-    any device work."""
+    equal the workspace path's and the oracle's bit for bit. One more token
+    is refused before any device work."""
     import torch
     c = Case(2424, 6912, 80, w_seed=25, x_seed=26)
     x, packed = c.x_tensor(), c.packed_tensor()
@@ -63,6 +65,8 @@ def test_noalloc_fills_the_scratch_exactly_and_rejects_beyond_it():
     got, ref = tensor_to_bf16_bits(y), tensor_to_bf16_bits(y_ref)
     check_y(got, ref)
     np.testing.assert_array_equal(got, ref)
+    # the oracle's bits for the whole problem (integer products on all host cores)
+    assert check_y(got, c.oracle_full(oracle.Oracle(oracle.load_omp()))[1]) == 1.0
     assert bl.bitlinear_get_fault() == (bl.BITLINEAR_OK, 0)
 
     x1 = torch.zeros((2425, 6912), dtype=torch.bfloat16, device="cuda")
