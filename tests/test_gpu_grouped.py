@@ -166,7 +166,7 @@ def test_grouped_rmsnorm_layer_matches_oracle(B):
 
 # ------------------------------------------- host buffers in and out
 
-def _host_call_check(cases, contiguous, pinned, rounds=1, pinned_y=None):
+def _host_call_check(cases, contiguous, pinned, repeats=1, pinned_y=None):
     """Runs bitlinear_forward_grouped_host on the cases' tokens (host memory,
     problem after problem) and compares the host outputs with the oracle bit
     for bit; the device staging buffers lie back to back (one copy each way)
@@ -196,7 +196,7 @@ def _host_call_check(cases, contiguous, pinned, rounds=1, pinned_y=None):
         host_x = host_x.pin_memory()
     if pinned_y:
         host_y = host_y.pin_memory()
-    for _ in range(rounds):
+    for _ in range(repeats):
         call(host_x, host_y)
         torch.cuda.synchronize()
     got = host_y.view(torch.int16).numpy().view(np.uint16)
@@ -211,7 +211,7 @@ def _host_call_check(cases, contiguous, pinned, rounds=1, pinned_y=None):
 def test_grouped_host_decode_step_2b_pinned():
     cases = [Case(p.M, p.K, p.N, w_seed=p.w_seed, x_seed=p.x_seed)
              for p in workloads.decode_gemv_2b(1).problems]
-    _host_call_check(cases, contiguous=True, pinned=True, rounds=3)
+    _host_call_check(cases, contiguous=True, pinned=True, repeats=3)
 
 
 def test_grouped_host_mixed_fp32_separate_buffers_pageable():
@@ -223,11 +223,11 @@ def test_grouped_host_mixed_fp32_separate_buffers_pageable():
 def test_grouped_host_pinned_tokens_pageable_outputs():
     cases = [Case(p.M, p.K, p.N, w_seed=p.w_seed, x_seed=p.x_seed)
              for p in workloads.decode_gemv_2b(1).problems]
-    _host_call_check(cases, contiguous=True, pinned=True, pinned_y=False, rounds=2)
+    _host_call_check(cases, contiguous=True, pinned=True, pinned_y=False, repeats=2)
 
 
 def test_grouped_host_pinned_unaligned_output_parts():
     """N = 17 and 40: the second problem's outputs start 34 bytes into y_host,
     so the outputs go through the device buffers and a copy back."""
     cases = [Case(1, 512, 17, w_seed=81, x_seed=91), Case(2, 384, 40, w_seed=82, x_seed=92)]
-    _host_call_check(cases, contiguous=False, pinned=True, rounds=2)
+    _host_call_check(cases, contiguous=False, pinned=True, repeats=2)
