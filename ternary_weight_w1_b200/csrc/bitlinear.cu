@@ -37,6 +37,10 @@ constexpr int64_t kAutoGemvMaxM = 6;                // above: tensor-core path
 // Split the k-range of fewer tiles than CTAs only when a CTA saves more than
 // this many 256-k blocks (each about half a microsecond) by it.
 constexpr double kSplitMinSavedBlocks = 10.0;
+// A split launch with fewer tiles than CTAs gives each CTA at least this many
+// k-blocks of 256: a tile shared by many CTAs pays one partial-sum hand-off
+// per contributor.
+constexpr int64_t kSplitMinCtaBlocks = 8;
 // k-blocks of 256 per CTA from which the small token tiles take 512-k stages
 constexpr int64_t kDeepStageMinBlocks = 8;
 constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s: far above any legitimate wait
@@ -762,7 +766,11 @@ int run_tc_group(const TcJob *jobs, int n, bitlinear_dtype xdt, void *ws, size_t
         split = saved_blocks * (BK / 256) > kSplitMinSavedBlocks;
     }
     const int64_t units = split ? iters : tiles;
-    const int grid = static_cast<int>(std::min<int64_t>(units, slots));
+    int64_t grid64 = std::min<int64_t>(units, slots);
+    if (split && tiles < slots)
+        grid64 = std::max<int64_t>(
+            tiles, std::min<int64_t>(grid64, iters * (BK / 256) / kSplitMinCtaBlocks));
+    const int grid = static_cast<int>(grid64);
 
     // Workspace: per problem x~ | beta | row sums, then flags | partial sums.
     char *w = static_cast<char *>(ws);
